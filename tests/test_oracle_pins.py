@@ -1,0 +1,399 @@
+"""Pins of the fp64 oracle against things other than itself (CPU only).
+
+Each test gets its expected values from a library routine (numpy/torch
+matmul, torch's bf16 and e4m3 conversions), brute force over all subsets,
+closed forms, hand-derived fixtures under tests/golden/, or central finite
+differences of the pure fp64 forward -- never from the oracle function under
+test.
+"""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _f32_to_bf16_bits_torch(v):
+    return torch.from_numpy(np.asarray(v, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _bits_to_f64(b):
+    return (np.asarray(b, np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# ------------------------------------------------------------------ scalars
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(1)
+    v = np.concatenate([rng.standard_normal(4000).astype(np.float32) * 10.0 ** rng.integers(-30, 30, 4000),
+                        np.float32([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 2 ** -130, 3e38])])
+    v = v.astype(np.float32)
+    want = _bits_to_f64(_f32_to_bf16_bits_torch(v))
+    got = np.array([oracle.round_bf16(float(a)) for a in v])
+    assert np.array_equal(got, want)
+
+
+def test_e4m3_codes_match_torch_and_golden():
+    codes = np.arange(256, dtype=np.uint8)
+    tv = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    for c in range(256):
+        ov = oracle.e4m3_value(c)
+        if math.isnan(tv[c]):
+            assert math.isnan(ov)
+            continue
+        assert ov == tv[c], c
+        assert math.copysign(1, ov) == math.copysign(1, tv[c])
+        assert oracle.e4m3_bits(ov) == c, c      # round trip
+        assert oracle.round_e4m3(ov) == ov
+    for line in open(os.path.join(GOLDEN, "e4m3_fn_values.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        code, val = line.split()
+        assert oracle.e4m3_value(int(code, 16)) == float(val)
+        assert oracle.e4m3_bits(float(val)) == int(code, 16)
+
+
+def test_e4m3_rounding_matches_torch():
+    rng = np.random.default_rng(2)
+    v = rng.uniform(-448, 448, 20000) * 2.0 ** rng.integers(-14, 1, 20000)
+    v = v.astype(np.float32).astype(np.float64)
+    # add exact ties between neighbours (even / odd mantissa) and the subnormal range
+    ties = [1.0625, 1.1875, 0.001953125 * 1.5, 0.001953125 * 2.5, 240.0 + 8.0, 416 + 16]
+    v = np.concatenate([v, ties, [-t for t in ties]])
+    want = torch.from_numpy(v.astype(np.float32)).to(torch.float8_e4m3fn).float().numpy()
+    got = np.array([oracle.round_e4m3(a) for a in v])
+    assert np.array_equal(got, want.astype(np.float64))
+    # saturation to the largest finite value
+    for a in (449.0, 463.9, 464.0, 500.0, 1e9):
+        assert oracle.round_e4m3(a) == 448.0 and oracle.round_e4m3(-a) == -448.0
+
+
+def test_mx_scale_golden():
+    for line in open(os.path.join(GOLDEN, "mx_scale_cases.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        a, e = line.split()
+        assert oracle.mx_scale_exp(float(a)) == int(e), a
+
+
+def test_mx_quantize_blocks():
+    # block 0: all zeros; block 1: amax exactly 448 * 2^-3; block 2: amax just above
+    rows = np.zeros((1, 96), np.float32)
+    rows[0, 32:64] = np.linspace(-56, 56, 32)
+    rows[0, 64:96] = np.linspace(-1, 1, 32) * 57.0
+    bits = _f32_to_bf16_bits_torch(rows)
+    q, s = oracle.mx_quantize(bits)
+    assert s[0, 0] == 0 and not q[0, :32].any()
+    assert s[0, 1] == 127 - 3 and s[0, 2] == 127 - 2
+    vals = _bits_to_f64(bits)[0]
+    for b in range(3):
+        e = int(s[0, b]) - 127
+        deq = np.array([oracle.e4m3_value(c) for c in q[0, 32 * b:32 * b + 32]]) * 2.0 ** e
+        ref = torch.from_numpy((vals[32 * b:32 * b + 32] / 2.0 ** e).astype(np.float32)).to(
+            torch.float8_e4m3fn).float().numpy() * 2.0 ** e
+        assert np.array_equal(deq, ref)
+    fq = bits.copy()
+    oracle.mx_fakequant_bf16(fq)
+    assert np.array_equal(_bits_to_f64(fq)[0, 32:96],
+                          np.concatenate([np.array([oracle.e4m3_value(c) for c in q[0, 32 * b:32 * b + 32]]) * 2.0 ** (int(s[0, b]) - 127) for b in (1, 2)]))
+
+
+# ------------------------------------------------------------------ routing
+def _tiny_router(T, H, E, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    x = _f32_to_bf16_bits_torch(rng.standard_normal((T, H)).astype(np.float32))
+    Wr = (rng.standard_normal((E, H)) * scale).astype(np.float32)
+    return x, Wr
+
+
+def _logits_np(x, Wr, lbias=None):
+    lg = _bits_to_f64(x) @ Wr.astype(np.float64).T
+    return lg if lbias is None else lg + lbias.astype(np.float64)
+
+
+@pytest.mark.parametrize("k", [1, 2, 3])
+def test_softmax_topk_bruteforce(k):
+    T, H, E = 40, 16, 8
+    x, Wr = _tiny_router(T, H, E, seed=10 + k)
+    L = oracle.Layer(T, H, E, k, 8, routed_scale=1.0).set(x=x, Wr=Wr)
+    idx, w, gap = L.route()
+    lg = _logits_np(x, Wr)
+    for t in range(T):
+        # the top-k set is the unique k-subset with the largest sum of logits
+        best = max(itertools.combinations(range(E), k), key=lambda s: sum(lg[t, list(s)]))
+        assert set(idx[t]) == set(best)
+        # slots in descending score order
+        assert list(idx[t]) == sorted(best, key=lambda e: -lg[t, e])
+        sel = lg[t, idx[t]]
+        ref = np.exp(sel - sel.max()) / np.exp(sel - sel.max()).sum()
+        np.testing.assert_allclose(w[t], ref, rtol=1e-12, atol=0)
+
+
+def test_sigmoid_group_limited_bruteforce():
+    T, H, E, G, TG, k = 40, 16, 8, 4, 2, 3
+    x, Wr = _tiny_router(T, H, E, seed=5)
+    bias = (0.3 * np.random.default_rng(6).standard_normal(E)).astype(np.float32)
+    lb = np.float32([0, -0.5, 0.2, 0, 0, 0.1, -1, 0])
+    rs = 2.5
+    L = oracle.Layer(T, H, E, k, 8, score_fn=1, n_group=G, topk_group=TG, routed_scale=rs)
+    L.set(x=x, Wr=Wr, bias=bias, lbias=lb)
+    idx, w, gap = L.route()
+    lg = _logits_np(x, Wr, lb)
+    s = 1 / (1 + np.exp(-lg))
+    sc = s + bias
+    gs = E // G
+    for t in range(T):
+        gscore = [max(sc[t, g * gs + a] + sc[t, g * gs + b] for a, b in itertools.combinations(range(gs), 2))
+                  for g in range(G)]
+        groups = max(itertools.combinations(range(G), TG), key=lambda c: sum(gscore[g] for g in c))
+        cand = [g * gs + i for g in groups for i in range(gs)]
+        best = max(itertools.combinations(cand, k), key=lambda c: sum(sc[t, list(c)]))
+        assert set(idx[t]) == set(best), t
+        assert list(idx[t]) == sorted(best, key=lambda e: -sc[t, e])
+        ref = rs * s[t, idx[t]] / s[t, idx[t]].sum()      # unbiased scores, renormalised
+        np.testing.assert_allclose(w[t], ref, rtol=1e-12, atol=0)
+
+
+def test_ties_go_to_lower_index():
+    T, H, E, k = 6, 16, 8, 3
+    x, Wr = _tiny_router(T, H, E, seed=7)
+    Wr[5] = Wr[2]          # experts 2 and 5 always tie
+    Wr[6] = Wr[2]
+    L = oracle.Layer(T, H, E, k, 8).set(x=x, Wr=Wr)
+    idx, w, gap = L.route()
+    lg = _logits_np(x, Wr)
+    for t in range(T):
+        order = sorted(range(E), key=lambda e: (-lg[t, e], e))
+        assert list(idx[t]) == order[:k]
+    # group ties: two identical groups, the lower group id wins
+    Wr2 = Wr.copy()
+    Wr2[4:6] = Wr2[0:2]
+    L2 = oracle.Layer(T, H, E, 2, 8, score_fn=1, n_group=4, topk_group=1).set(x=x, Wr=Wr2)
+    idx2, _, _ = L2.route()
+    lg2 = _logits_np(x, Wr2)
+    sc2 = 1 / (1 + np.exp(-lg2))
+    for t in range(T):
+        gsc = [sc2[t, 2 * g] + sc2[t, 2 * g + 1] for g in range(4)]
+        gbest = sorted(range(4), key=lambda g: (-gsc[g], g))[0]
+        assert set(idx2[t]) == {2 * gbest, 2 * gbest + 1}
+
+
+def test_dispatch_invariants():
+    T, H, E, k = 300, 16, 8, 3
+    x, Wr = _tiny_router(T, H, E, seed=8)
+    L = oracle.Layer(T, H, E, k, 8).set(x=x, Wr=Wr)
+    idx, w, _ = L.route()
+    counts, offsets, perm, inv = L.dispatch(idx)
+    assert counts.sum() == T * k
+    assert np.array_equal(np.bincount(idx.ravel(), minlength=E), counts)
+    assert np.array_equal(perm[inv], np.arange(T * k))      # dispatch then inverse = identity
+    assert np.array_equal(inv[perm], np.arange(T * k))
+    for e in range(E):
+        rows = perm[offsets[e]:offsets[e + 1]]
+        assert np.all(idx.ravel()[rows] == e)
+        toks = rows // k
+        assert np.all(np.diff(toks) > 0)                     # ascending in token
+
+
+# ------------------------------------------------------------------ expert math
+def _mlp_np(xd, Wg, Wu, Wd):
+    g = xd @ Wg.T
+    u = xd @ Wu.T
+    h = g / (1 + np.exp(-g)) * u
+    return h @ Wd.T
+
+
+def _rand_bf16(rng, shape, std):
+    return _f32_to_bf16_bits_torch((rng.standard_normal(shape) * std).astype(np.float32))
+
+
+@pytest.mark.parametrize("shared", [0, 1])
+def test_single_expert_equals_dense_swiglu(shared):
+    """E=1, top-1, weight 1 (softmax over one expert) is a dense SwiGLU MLP."""
+    rng = np.random.default_rng(20 + shared)
+    T, H, I, Is = 12, 64, 96, 32
+    x = _rand_bf16(rng, (T, H), 1.0)
+    Wr = rng.standard_normal((1, H)).astype(np.float32)
+    Wgu = _rand_bf16(rng, (1, 2 * I, H), 0.1)
+    Wdn = _rand_bf16(rng, (1, H, I), 0.1)
+    Wgu_s = _rand_bf16(rng, (1, 2 * Is, H), 0.1) if shared else None
+    Wdn_s = _rand_bf16(rng, (1, H, Is), 0.1) if shared else None
+    L = oracle.Layer(T, H, 1, 1, I, S=shared, Is=Is if shared else 0, pure=True)
+    L.set(x=x, Wr=Wr, Wgu=Wgu, Wdn=Wdn, Wgu_s=Wgu_s, Wdn_s=Wdn_s)
+    idx, w, _ = L.route()
+    assert np.all(idx == 0) and np.all(w == 1.0)
+    y = L.fwd(idx, w)
+    xd = _bits_to_f64(x)
+    ref = _mlp_np(xd, _bits_to_f64(Wgu[0, :I]), _bits_to_f64(Wgu[0, I:]), _bits_to_f64(Wdn[0]))
+    if shared:
+        ref = ref + _mlp_np(xd, _bits_to_f64(Wgu_s[0, :Is]), _bits_to_f64(Wgu_s[0, Is:]), _bits_to_f64(Wdn_s[0]))
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def _bf16_round_via_torch(a):
+    # double -> float32 -> bf16 may round twice; agreement is checked to 1 ulp
+    return torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def test_mirrors_sit_at_stored_tensors():
+    """With mirrors on, the two-expert forward equals the weighted sum of per-expert
+    MLPs with bf16 rounding of h, o and y (computed here with torch's rounding)."""
+    rng = np.random.default_rng(30)
+    T, H, E, k, I = 16, 64, 4, 2, 64
+    x = _rand_bf16(rng, (T, H), 1.0)
+    Wr = rng.standard_normal((E, H)).astype(np.float32) / 8
+    Wgu = _rand_bf16(rng, (E, 2 * I, H), 0.1)
+    Wdn = _rand_bf16(rng, (E, H, I), 0.1)
+    L = oracle.Layer(T, H, E, k, I).set(x=x, Wr=Wr, Wgu=Wgu, Wdn=Wdn)
+    idx, w, _ = L.route()
+    y, O, h = L.fwd(idx, w, want_slots=True)
+    xd = _bits_to_f64(x)
+    for t in range(T):
+        acc = np.zeros(H)
+        for j in range(k):
+            e = idx[t, j]
+            g = xd[t] @ _bits_to_f64(Wgu[e, :I]).T
+            u = xd[t] @ _bits_to_f64(Wgu[e, I:]).T
+            hh = _bf16_round_via_torch(g / (1 + np.exp(-g)) * u)
+            np.testing.assert_allclose(h[t, j], hh, rtol=2 ** -8, atol=0)
+            o = _bf16_round_via_torch(h[t, j] @ _bits_to_f64(Wdn[e]).T)
+            np.testing.assert_allclose(O[t, j], o, rtol=2 ** -8, atol=0)
+            acc += w[t, j] * O[t, j]
+        np.testing.assert_allclose(y[t], _bf16_round_via_torch(acc), rtol=2 ** -8, atol=0)
+
+
+def test_mxfp8_single_expert_matches_fakequant_mlp():
+    """MXFP8 mode: x and h quantised per 1x32 block (scale rule from the golden
+    definition, e4m3 rounding by torch), weights fake-quantised by the caller."""
+    rng = np.random.default_rng(40)
+    T, H, I = 8, 64, 64
+    x = _rand_bf16(rng, (T, H), 1.0)
+    Wr = rng.standard_normal((1, H)).astype(np.float32)
+    Wgu = _rand_bf16(rng, (1, 2 * I, H), 0.1)
+    Wdn = _rand_bf16(rng, (1, H, I), 0.1)
+    Wgu_q, Wdn_q = Wgu.copy(), Wdn.copy()
+    oracle.mx_fakequant_bf16(Wgu_q)
+    oracle.mx_fakequant_bf16(Wdn_q)
+    L = oracle.Layer(T, H, 1, 1, I, mx=True, pure=True).set(x=x, Wr=Wr, Wgu=Wgu_q, Wdn=Wdn_q)
+    idx, w, _ = L.route()
+    y = L.fwd(idx, w)
+
+    def fq(a):
+        out = a.copy()
+        for r in range(a.shape[0]):
+            for b in range(0, a.shape[1], 32):
+                blk = a[r, b:b + 32]
+                amax = np.abs(blk).max()
+                e = -127
+                if amax > 0:
+                    e = math.frexp(amax)[1] - 10
+                    while amax > 448.0 * 2.0 ** e:
+                        e += 1
+                q = torch.from_numpy((blk / 2.0 ** e).astype(np.float32)).to(torch.float8_e4m3fn)
+                out[r, b:b + 32] = q.float().numpy() * 2.0 ** e
+        return out
+
+    xd = fq(_bits_to_f64(x))
+    g = xd @ _bits_to_f64(Wgu_q[0, :I]).T
+    u = xd @ _bits_to_f64(Wgu_q[0, I:]).T
+    hq = fq(g / (1 + np.exp(-g)) * u)
+    ref = hq @ _bits_to_f64(Wdn_q[0]).T
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+    # the fake-quantised weights are exactly the dequantised MX codes
+    q, s = oracle.mx_quantize(Wgu[0])
+    deq = np.vectorize(oracle.e4m3_value)(q) * 2.0 ** (np.repeat(s.astype(np.int64), 32, axis=1) - 127)
+    assert np.array_equal(deq, _bits_to_f64(Wgu_q[0]))
+
+
+# ------------------------------------------------------------------ gradients
+def _fd_layer(score_fn, seed):
+    """A small pure-fp64 layer with inputs chosen so that routing has margins."""
+    rng = np.random.default_rng(seed)
+    T, H, E, k, I = 6, 32, 8, 2, 16
+    S, Is = (1, 8) if score_fn else (0, 0)
+    while True:
+        x = rng.standard_normal((T, H))
+        Wr = rng.standard_normal((E, H)) / math.sqrt(H)
+        bias = 0.01 * rng.standard_normal(E) if score_fn else None
+        L = oracle.Layer(T, H, E, k, I, S=S, Is=Is, score_fn=score_fn,
+                         n_group=4 if score_fn else 1, topk_group=2 if score_fn else 1,
+                         routed_scale=1.7 if score_fn else 1.0, pure=True)
+        L.set(x=x, Wr=Wr, bias=bias, Wgu=rng.standard_normal((E, 2 * I, H)) * 0.3,
+              Wdn=rng.standard_normal((E, H, I)) * 0.3,
+              Wgu_s=rng.standard_normal((S, 2 * Is, H)) * 0.3 if S else None,
+              Wdn_s=rng.standard_normal((S, H, Is)) * 0.3 if S else None,
+              dy=rng.standard_normal((T, H)))
+        idx, w, gap = L.route()
+        if gap.min() > 1e-3:
+            return L
+
+
+def _loss(L):
+    idx, w, _ = L.route()
+    y = L.fwd(idx, w)
+    return float((y * L.arrays["dy"]).sum())
+
+
+@pytest.mark.parametrize("score_fn", [0, 1])
+def test_gradients_match_finite_differences(score_fn):
+    L = _fd_layer(score_fn, seed=50 + score_fn)
+    c = L.cfg
+    idx, w, _ = L.route()
+    dx, dl, G = L.bwd(idx, w)
+    eps = 1e-6
+    rng = np.random.default_rng(3)
+
+    def fd(name, pos):
+        a = L.arrays[name]
+        old = a[pos]
+        a[pos] = old + eps
+        L.set(**{name: a})
+        lp = _loss(L)
+        a[pos] = old - eps
+        L.set(**{name: a})
+        lm = _loss(L)
+        a[pos] = old
+        L.set(**{name: a})
+        return (lp - lm) / (2 * eps)
+
+    for _ in range(24):
+        t, h = rng.integers(c.T), rng.integers(c.H)
+        assert fd("x", (t, h)) == pytest.approx(dx[t, h], rel=1e-6, abs=1e-8)
+    dWr = L.drouter(idx, w, np.arange(c.E))
+    for _ in range(24):
+        e, h = rng.integers(c.E), rng.integers(c.H)
+        assert fd("Wr", (e, h)) == pytest.approx(dWr[e, h], rel=1e-6, abs=1e-8)
+    groups = [(e, False) for e in range(c.E)] + [(s, True) for s in range(c.S)]
+    for g, sh in groups:
+        dgu, ddn = L.dw_full(idx, w, g, sh)
+        wname_gu, wname_dn = ("Wgu_s", "Wdn_s") if sh else ("Wgu", "Wdn")
+        for _ in range(4):
+            n, h = rng.integers(dgu.shape[0]), rng.integers(c.H)
+            assert fd(wname_gu, (g, n, h)) == pytest.approx(dgu[n, h], rel=1e-6, abs=1e-8)
+            h2, i = rng.integers(c.H), rng.integers(ddn.shape[1])
+            assert fd(wname_dn, (g, h2, i)) == pytest.approx(ddn[h2, i], rel=1e-6, abs=1e-8)
+
+
+def test_dw_entries_agree_with_full():
+    rng = np.random.default_rng(60)
+    T, H, E, k, I = 24, 32, 4, 2, 32
+    x = _rand_bf16(rng, (T, H), 1.0)
+    L = oracle.Layer(T, H, E, k, I, S=1, Is=32).set(
+        x=x, Wr=rng.standard_normal((E, H)).astype(np.float32) / 6,
+        Wgu=_rand_bf16(rng, (E, 2 * I, H), 0.1), Wdn=_rand_bf16(rng, (E, H, I), 0.1),
+        Wgu_s=_rand_bf16(rng, (1, 64, H), 0.1), Wdn_s=_rand_bf16(rng, (1, H, 32), 0.1),
+        dy=_rand_bf16(rng, (T, H), 1.0))
+    idx, w, _ = L.route()
+    for g, sh in [(0, False), (3, False), (0, True)]:
+        dgu, ddn = L.dw_full(idx, w, g, sh)
+        r = rng.integers(0, dgu.shape[0], 20)
+        cc = rng.integers(0, H, 20)
+        assert np.array_equal(L.dw_entries(idx, w, g, sh, 0, r, cc), dgu[r, cc])
+        r2 = rng.integers(0, H, 20)
+        c2 = rng.integers(0, ddn.shape[1], 20)
+        assert np.array_equal(L.dw_entries(idx, w, g, sh, 1, r2, c2), ddn[r2, c2])
