@@ -1,0 +1,191 @@
+/*
+ * mok.h -- C ABI of the B200 (sm_100a) mixture-of-experts layer library (libmok.so).
+ *
+ * The layer is the one the pages centre on: a DeepSeek-V3-type MoE layer
+ * ("Cursor åpner megakernelen som ga 41 prosent flere tokens i sekundet",
+ * last paragraph), forward in BF16 and MXFP8 and backward in BF16
+ * ("Megakernels are dead and back…", section "Números de MoK"), computed
+ * deterministically with no CPU-GPU synchronisation inside the layer
+ * ("Cursor veröffentlicht MoE-Megakernel Mixture-of-Kittens als Open Source",
+ * section "Kommunikation im Kernel").  All experts live on one GPU.
+ *
+ * Conventions shared by every entry point:
+ *  - Pointers named "device" are CUDA device pointers on the current device;
+ *    pointers named "host" are host memory (pinned or pageable).
+ *  - All tensors are dense, row-major, contiguous, with the shapes given.
+ *    bf16 tensors are passed as raw 16-bit storage.  Device pointers must be
+ *    16-byte aligned.
+ *  - The caller owns every buffer, including workspaces; the library never
+ *    allocates device memory and never synchronises the host inside
+ *    moe_fwd/moe_bwd.  Work is enqueued on `stream` (a cudaStream_t, NULL =
+ *    legacy default stream).
+ *  - Outputs are overwritten, never accumulated into.
+ *  - Return value: MOK_OK (0) or a negative MOK_ERR_* code; argument errors are
+ *    detected on the host before anything is enqueued.  Errors that arise on
+ *    the device (a bounded wait that ran out) are recorded in a device status
+ *    word and reported by moe_status.
+ *  - Results are bit-identical across calls with the same inputs (fixed
+ *    reduction orders, no floating-point atomics).
+ */
+#ifndef MOK_H
+#define MOK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- error codes ---------------------------------------------------------- */
+#define MOK_OK 0
+#define MOK_ERR_INVALID (-1)      /* bad shape, pointer, alignment or option */
+#define MOK_ERR_DEVICE (-2)       /* current device is not sm_100 (B200) */
+#define MOK_ERR_WORKSPACE (-3)    /* ctx or scratch buffer too small */
+#define MOK_ERR_LAUNCH (-4)       /* a CUDA call failed while enqueueing */
+#define MOK_ERR_UNSUPPORTED (-5)  /* valid but not implemented combination */
+
+/* device status bits (moe_status) */
+#define MOK_STATUS_TIMEOUT 1      /* a bounded wait inside a kernel ran out */
+
+/* ---- configuration -------------------------------------------------------- */
+#define MOK_SCORE_SOFTMAX 0       /* softmax over all experts, top-k, renormalised */
+#define MOK_SCORE_SIGMOID 1       /* sigmoid scores + selection bias, group-limited top-k */
+
+#define MOK_DTYPE_BF16 0          /* bf16 operands, fp32 accumulation */
+#define MOK_DTYPE_MXFP8 1         /* e4m3 operands with 1x32 ue8m0 block scales (forward only) */
+
+typedef struct moe_cfg {
+    int32_t T;            /* tokens in the batch, >= 1 */
+    int32_t H;            /* hidden size, multiple of 256 */
+    int32_t E;            /* routed experts, 1..256 */
+    int32_t I;            /* expert intermediate size, multiple of 128 */
+    int32_t top_k;        /* experts per token, 1..min(E, 16) */
+    int32_t n_shared;     /* shared experts applied to every token, 0..4 */
+    int32_t I_shared;     /* shared intermediate size; must equal I when n_shared > 0 */
+    int32_t score_fn;     /* MOK_SCORE_* */
+    int32_t n_group;      /* expert groups for group-limited selection (1 = none); divides E */
+    int32_t topk_group;   /* groups kept per token, 1..n_group */
+    float routed_scale;   /* multiplies the renormalised routing weights */
+    int32_t dtype;        /* MOK_DTYPE_* */
+} moe_cfg;
+
+/*
+ * Layer parameters (device pointers).  Expert weights use the layouts
+ *   w_gate_up [E, 2I, H]: rows 0..I-1 the gate projection, rows I..2I-1 the up projection
+ *   w_down    [E, H, I]
+ *   ws_*      the same for the n_shared shared experts ([S, 2I, H], [S, H, I]).
+ * For MOK_DTYPE_BF16 the weights are bf16 and the s_* scale pointers are NULL.
+ * For MOK_DTYPE_MXFP8 the weights are e4m3 codes (one byte each, same shapes)
+ * and s_* hold one ue8m0 byte per 32 consecutive elements along the last
+ * (contraction) axis: [E, 2I, H/32], [E, H, I/32] (see moe_quantize_mxfp8).
+ */
+typedef struct moe_params {
+    const float *router_w;      /* [E, H] fp32 */
+    const float *e_bias;        /* [E] fp32 selection bias (sigmoid scoring), or NULL */
+    const float *logit_bias;    /* [E] fp32 term added to the router logits, or NULL */
+    const void *w_gate_up;
+    const void *w_down;
+    const uint8_t *s_gate_up;
+    const uint8_t *s_down;
+    const void *ws_gate_up;
+    const void *ws_down;
+    const uint8_t *ss_gate_up;
+    const uint8_t *ss_down;
+} moe_params;
+
+/* Routing record (device pointers; any may be NULL to skip that output). */
+typedef struct moe_routing {
+    int32_t *topk_idx;   /* [T, top_k] selected experts, slot order = selection order */
+    float *topk_w;       /* [T, top_k] routing weights */
+    int32_t *counts;     /* [E] tokens per expert */
+    int32_t *offsets;    /* [E+1] exclusive prefix sum of counts */
+    int32_t *perm;       /* [T*top_k] sorted row -> t*top_k + slot (expert-major, token ascending) */
+    int32_t *inv_perm;   /* [T*top_k] t*top_k + slot -> sorted row */
+} moe_routing;
+
+/* Gradients (device pointers, all overwritten).  dws_* may be NULL when n_shared == 0. */
+typedef struct moe_grads {
+    void *dx;            /* [T, H] bf16 */
+    void *dw_gate_up;    /* [E, 2I, H] bf16 */
+    void *dw_down;       /* [E, H, I] bf16 */
+    float *drouter_w;    /* [E, H] fp32 */
+    void *dws_gate_up;   /* [S, 2I, H] bf16 */
+    void *dws_down;      /* [S, H, I] bf16 */
+} moe_grads;
+
+/*
+ * Sizes of the caller-allocated buffers for a configuration.
+ *   ctx_bytes         saved forward state that moe_bwd reads (routing record,
+ *                     gate/up pre-activations, h, weighted h, per-slot rows)
+ *   fwd_scratch_bytes temporary device memory of moe_fwd
+ *   bwd_scratch_bytes temporary device memory of moe_bwd
+ * Any output pointer may be NULL.  Returns MOK_ERR_INVALID for a bad cfg.
+ */
+int moe_workspace_size(const moe_cfg *cfg, size_t *ctx_bytes, size_t *fwd_scratch_bytes,
+                       size_t *bwd_scratch_bytes);
+
+/*
+ * Forward pass.  x: [T, H] bf16 (device); y: [T, H] bf16 (device, output).
+ * routing: optional copy of the routing record (NULL = none).
+ * save_for_backward != 0 stores the state moe_bwd needs in ctx, which must then
+ * be at least ctx_bytes long; with save_for_backward == 0, ctx may be NULL.
+ * The forward follows the steps: router logits (fp32), scoring and top-k with
+ * ties to the lower expert index, deterministic counts/prefix scan/stable
+ * permutation, pull-gathered gate/up grouped GEMM with a SwiGLU epilogue,
+ * down grouped GEMM whose epilogue pushes each row into its (token, slot)
+ * row, and a fixed-order weighted sum over slots (shared experts last,
+ * weight 1).  The pull-at-dispatch / push-at-combine split follows
+ * "Cursor åpner megakernelen…" (paragraph on pulling versus pushing tokens).
+ */
+int moe_fwd(const moe_cfg *cfg, const void *x, const moe_params *params, void *y,
+            const moe_routing *routing, void *ctx, size_t ctx_bytes, int save_for_backward,
+            void *scratch, size_t scratch_bytes, void *stream);
+
+/*
+ * Backward pass (MOK_DTYPE_BF16 only).  x and dy: [T, H] bf16 (device); ctx:
+ * the buffer a moe_fwd call with save_for_backward != 0 filled for the same x
+ * and params.  Computes dx, the expert weight gradients and the router weight
+ * gradient (the selection bias gets none) with fixed reduction orders.
+ */
+int moe_bwd(const moe_cfg *cfg, const void *x, const void *dy, const moe_params *params,
+            const void *ctx, size_t ctx_bytes, const moe_grads *grads, void *scratch,
+            size_t scratch_bytes, void *stream);
+
+/*
+ * Host-buffer variants: x_host / y_host (and dy_host / dx_host) are host
+ * memory; the call copies them through the scratch buffer (which must then be
+ * at least moe_host_scratch_size bytes), runs the layer on `stream` and
+ * synchronises that stream before returning.  Parameters, ctx and the other
+ * gradients stay on the device.
+ */
+int moe_host_scratch_size(const moe_cfg *cfg, int backward, size_t *bytes);
+int moe_fwd_host(const moe_cfg *cfg, const void *x_host, const moe_params *params, void *y_host,
+                 void *ctx, size_t ctx_bytes, int save_for_backward, void *scratch,
+                 size_t scratch_bytes, void *stream);
+int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host,
+                 const moe_params *params, const void *ctx, size_t ctx_bytes, void *dx_host,
+                 const moe_grads *grads, void *scratch, size_t scratch_bytes, void *stream);
+
+/*
+ * MXFP8 quantisation along the last axis: src [rows, K] bf16 (device) ->
+ * q [rows, K] e4m3 codes and scales [rows, K/32] ue8m0 (device).  Per block of
+ * 32 consecutive elements the exponent e is the smallest integer with
+ * amax <= 448 * 2^e (clamped to [-127, 127]; an all-zero block takes -127),
+ * the scale byte is e + 127 and each element is x / 2^e rounded to nearest
+ * even e4m3 with saturation.  K must be a multiple of 32.
+ */
+int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *scales,
+                       void *stream);
+
+/* Synchronise `stream`, then read and clear the device status word of the
+ * current device (MOK_STATUS_* bits) into *device_status. */
+int moe_status(void *stream, int32_t *device_status);
+
+/* Static message for an error code. */
+const char *moe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOK_H */

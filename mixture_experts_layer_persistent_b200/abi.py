@@ -1,0 +1,149 @@
+"""ctypes binding of libmok.so -- argument marshalling only.
+
+Every name here mirrors an entry point of include/mok.h.  Device pointers
+are passed as integers (e.g. ``tensor.data_ptr()``), streams as
+``torch.cuda.Stream.cuda_stream`` integers.  Nothing in this module computes
+any part of the layer, and there is no fallback: if the library cannot be
+loaded, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmok.so")
+
+MOK_OK = 0
+MOK_ERR_INVALID = -1
+MOK_ERR_DEVICE = -2
+MOK_ERR_WORKSPACE = -3
+MOK_ERR_LAUNCH = -4
+MOK_ERR_UNSUPPORTED = -5
+MOK_STATUS_TIMEOUT = 1
+MOK_SCORE_SOFTMAX = 0
+MOK_SCORE_SIGMOID = 1
+MOK_DTYPE_BF16 = 0
+MOK_DTYPE_MXFP8 = 1
+
+_i32, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+
+
+class moe_cfg(ctypes.Structure):
+    _fields_ = [("T", _i32), ("H", _i32), ("E", _i32), ("I", _i32), ("top_k", _i32),
+                ("n_shared", _i32), ("I_shared", _i32), ("score_fn", _i32), ("n_group", _i32),
+                ("topk_group", _i32), ("routed_scale", _f32), ("dtype", _i32)]
+
+
+class moe_params(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("router_w", "e_bias", "logit_bias", "w_gate_up", "w_down",
+                                    "s_gate_up", "s_down", "ws_gate_up", "ws_down", "ss_gate_up",
+                                    "ss_down")]
+
+
+class moe_routing(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("topk_idx", "topk_w", "counts", "offsets", "perm", "inv_perm")]
+
+
+class moe_grads(ctypes.Structure):
+    _fields_ = [(n, _vp) for n in ("dx", "dw_gate_up", "dw_down", "drouter_w", "dws_gate_up",
+                                    "dws_down")]
+
+
+class MokError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__(f"{fn} failed: {moe_strerror(code)} ({code})")
+        self.code = code
+
+
+_lib = None
+
+
+def lib():
+    """Load libmok.so (raises if it is missing: the layer has no other implementation)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m mixture_experts_layer_persistent_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER
+        L.moe_workspace_size.argtypes = [P(moe_cfg), P(_sz), P(_sz), P(_sz)]
+        L.moe_fwd.argtypes = [P(moe_cfg), _vp, P(moe_params), _vp, P(moe_routing), _vp, _sz, _i32, _vp,
+                              _sz, _vp]
+        L.moe_bwd.argtypes = [P(moe_cfg), _vp, _vp, P(moe_params), _vp, _sz, P(moe_grads), _vp, _sz,
+                              _vp]
+        L.moe_host_scratch_size.argtypes = [P(moe_cfg), _i32, P(_sz)]
+        L.moe_fwd_host.argtypes = [P(moe_cfg), _vp, P(moe_params), _vp, _vp, _sz, _i32, _vp, _sz, _vp]
+        L.moe_bwd_host.argtypes = [P(moe_cfg), _vp, _vp, P(moe_params), _vp, _sz, _vp, P(moe_grads),
+                                   _vp, _sz, _vp]
+        L.moe_quantize_mxfp8.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
+        L.moe_status.argtypes = [_vp, P(_i32)]
+        L.moe_strerror.argtypes = [ctypes.c_int]
+        L.moe_strerror.restype = ctypes.c_char_p
+        for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
+                     "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_status"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(fn, rc):
+    if rc != MOK_OK:
+        raise MokError(fn, rc)
+
+
+def moe_strerror(code: int) -> str:
+    return lib().moe_strerror(int(code)).decode()
+
+
+def moe_workspace_size(cfg: moe_cfg):
+    c, f, b = _sz(), _sz(), _sz()
+    _check("moe_workspace_size", lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(c),
+                                                          ctypes.byref(f), ctypes.byref(b)))
+    return c.value, f.value, b.value
+
+
+def moe_host_scratch_size(cfg: moe_cfg, backward: bool) -> int:
+    n = _sz()
+    _check("moe_host_scratch_size", lib().moe_host_scratch_size(ctypes.byref(cfg), int(backward),
+                                                                ctypes.byref(n)))
+    return n.value
+
+
+def moe_fwd(cfg, x, params, y, routing, ctx, ctx_bytes, save_for_backward, scratch, scratch_bytes,
+            stream):
+    rc = lib().moe_fwd(ctypes.byref(cfg), x, ctypes.byref(params), y,
+                       ctypes.byref(routing) if routing is not None else None, ctx, ctx_bytes,
+                       int(save_for_backward), scratch, scratch_bytes, stream)
+    _check("moe_fwd", rc)
+
+
+def moe_bwd(cfg, x, dy, params, ctx, ctx_bytes, grads, scratch, scratch_bytes, stream):
+    rc = lib().moe_bwd(ctypes.byref(cfg), x, dy, ctypes.byref(params), ctx, ctx_bytes,
+                       ctypes.byref(grads), scratch, scratch_bytes, stream)
+    _check("moe_bwd", rc)
+
+
+def moe_fwd_host(cfg, x_host, params, y_host, ctx, ctx_bytes, save_for_backward, scratch,
+                 scratch_bytes, stream):
+    rc = lib().moe_fwd_host(ctypes.byref(cfg), x_host, ctypes.byref(params), y_host, ctx, ctx_bytes,
+                            int(save_for_backward), scratch, scratch_bytes, stream)
+    _check("moe_fwd_host", rc)
+
+
+def moe_bwd_host(cfg, x_host, dy_host, params, ctx, ctx_bytes, dx_host, grads, scratch,
+                 scratch_bytes, stream):
+    rc = lib().moe_bwd_host(ctypes.byref(cfg), x_host, dy_host, ctypes.byref(params), ctx,
+                            ctx_bytes, dx_host, ctypes.byref(grads), scratch, scratch_bytes, stream)
+    _check("moe_bwd_host", rc)
+
+
+def moe_quantize_mxfp8(src, rows, K, q, scales, stream):
+    _check("moe_quantize_mxfp8", lib().moe_quantize_mxfp8(src, rows, K, q, scales, stream))
+
+
+def moe_status(stream) -> int:
+    v = _i32()
+    _check("moe_status", lib().moe_status(stream, ctypes.byref(v)))
+    return v.value

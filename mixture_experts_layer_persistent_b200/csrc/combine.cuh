@@ -1,0 +1,204 @@
+// combine.cuh -- the HBM-bound steps: the fixed-order weighted k-sum of the
+// forward, the per-slot routing gradient, the router weight gradient and the
+// final dx sum of the backward.  All sums run in a fixed order with no
+// floating-point atomics, so results are bit-reproducible.
+#pragma once
+#include "ptx.cuh"
+
+namespace mok {
+
+__device__ __forceinline__ void unpack8(const uint4 u, float (&v)[8])
+{
+    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+    v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&v)[8])
+{
+    uint4 u;
+    u.x = pack_bf16x2(v[0], v[1]);
+    u.y = pack_bf16x2(v[2], v[3]);
+    u.z = pack_bf16x2(v[4], v[5]);
+    u.w = pack_bf16x2(v[6], v[7]);
+    return u;
+}
+
+// y[t] = sum_{j<k} w[t,j] O[t,j] (ascending j) + sum_s O[t,k+s] (ascending s), fp32, -> bf16.
+// Thread = 8 columns of one token (16-byte loads).
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16 *__restrict__ O,
+                                                      const float *__restrict__ topk_w,
+                                                      __nv_bfloat16 *__restrict__ y, int T, int H, int k, int S)
+{
+    const int cpr = H / 8;
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)T * cpr) return;
+    const int t = (int)(i / cpr), c = (int)(i % cpr) * 8;
+    const int kk = k + S;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const __nv_bfloat16 *row = O + (size_t)t * kk * H + c;
+    for (int j = 0; j < kk; ++j) {
+        const float w = j < k ? topk_w[(size_t)t * k + j] : 1.0f;
+        float v[8];
+        unpack8(*reinterpret_cast<const uint4 *>(row + (size_t)j * H), v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(w, v[q], acc[q]);
+    }
+    *reinterpret_cast<uint4 *>(y + (size_t)t * H + c) = pack8(acc);
+}
+
+// Backward, per token: G_j = <dy[t], O[t,j]> (j < k), then the logit gradient
+//   softmax: dl_j = w_j (G_j - sum_i q_i G_i),             q = w / routed_scale
+//   sigmoid: dl_j = rho/S (G_j - sum_i q_i G_i) s_j (1 - s_j), S = sum of selected s
+// One block of 256 threads per token; each thread sums a fixed column subset,
+// then a fixed-shape tree over threads.
+__global__ void __launch_bounds__(256) slot_grad_kernel(const __nv_bfloat16 *__restrict__ dy,
+                                                        const __nv_bfloat16 *__restrict__ O,
+                                                        const float *__restrict__ topk_w,
+                                                        const float *__restrict__ topk_p, float *__restrict__ dl,
+                                                        int T, int H, int k, int S, int score_fn,
+                                                        float routed_scale)
+{
+    __shared__ float s_red[8][16];
+    const int t = blockIdx.x;
+    const int kk = k + S;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float g[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) g[j] = 0.0f;
+    const __nv_bfloat16 *dyr = dy + (size_t)t * H;
+    const __nv_bfloat16 *orow = O + (size_t)t * kk * H;
+    for (int c = tid * 8; c < H; c += 256 * 8) {
+        float d[8];
+        unpack8(*reinterpret_cast<const uint4 *>(dyr + c), d);
+        for (int j = 0; j < k; ++j) {
+            float o[8];
+            unpack8(*reinterpret_cast<const uint4 *>(orow + (size_t)j * H + c), o);
+            float s = g[j];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) s = fmaf(d[q], o[q], s);
+            g[j] = s;
+        }
+    }
+    for (int j = 0; j < k; ++j) {
+        float v = g[j];
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
+        if (lane == 0) s_red[warp][j] = v;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float G[16], q[16];
+        float gbar = 0.0f, S_ = 0.0f;
+        for (int j = 0; j < k; ++j) {
+            float v = 0.0f;
+            for (int w = 0; w < 8; ++w) v += s_red[w][j];
+            G[j] = v;
+            q[j] = topk_w[(size_t)t * k + j] / routed_scale;
+            gbar = fmaf(q[j], G[j], gbar);
+            S_ += topk_p[(size_t)t * k + j];
+        }
+        for (int j = 0; j < k; ++j) {
+            float r;
+            if (score_fn == 0) {
+                r = topk_w[(size_t)t * k + j] * (G[j] - gbar);
+            } else {
+                const float s = topk_p[(size_t)t * k + j];
+                r = routed_scale / S_ * (G[j] - gbar) * s * (1.0f - s);
+            }
+            dl[(size_t)t * k + j] = r;
+        }
+    }
+}
+
+// Router weight gradient, pass 1: for each chunk of up to `chunk_rows` sorted
+// rows of one expert and 256 columns, partial[chunk, cols] = sum over the
+// chunk's rows (ascending) of dl(row) x[token(row), cols].  8 warps take rows
+// r = warp (mod 8); their sums are added in warp order.
+__global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                              const float *__restrict__ dl,
+                                                              const int *__restrict__ offsets,
+                                                              const int *__restrict__ chunk_start,
+                                                              const int *__restrict__ perm,
+                                                              float *__restrict__ partial, int H, int E, int k,
+                                                              int chunk_rows)
+{
+    __shared__ float s_acc[8][256];
+    const int chunk = blockIdx.x;
+    const int h0 = blockIdx.y * 256;
+    if (chunk >= chunk_start[E]) return;
+    int lo = 0, hi = E - 1;     // expert owning this chunk: largest e with chunk_start[e] <= chunk
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (chunk_start[mid] <= chunk) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const int r0 = offsets[e] + (chunk - chunk_start[e]) * chunk_rows;
+    const int r1 = min(offsets[e + 1], r0 + chunk_rows);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int r = r0 + warp; r < r1; r += 8) {
+        const int s = perm[r];                  // t * k + slot
+        const float d = dl[s];
+        const int tok = s / k;
+        float v[8];
+        unpack8(*reinterpret_cast<const uint4 *>(x + (size_t)tok * H + h0 + lane * 8), v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(d, v[q], acc[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) s_acc[warp][lane * 8 + q] = acc[q];
+    __syncthreads();
+    float s = 0.0f;
+    for (int w = 0; w < 8; ++w) s += s_acc[w][threadIdx.x];
+    partial[(size_t)chunk * H + h0 + threadIdx.x] = s;
+}
+
+// Router weight gradient, pass 2: dWr[e, h] = sum over the expert's chunks in order.
+__global__ void __launch_bounds__(256) drouter_reduce_kernel(const float *__restrict__ partial,
+                                                             const int *__restrict__ chunk_start,
+                                                             float *__restrict__ dWr, int H, int E)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)E * H) return;
+    const int e = (int)(i / H), h = (int)(i % H);
+    float s = 0.0f;
+    for (int c = chunk_start[e]; c < chunk_start[e + 1]; ++c) s += partial[(size_t)c * H + h];
+    dWr[i] = s;
+}
+
+// dx[t] = sum_j dXs[t, j] (ascending j over routed then shared slots)
+//         + sum_{j<k} dl[t, j] router_w[idx[t, j]]   -> bf16.
+__global__ void __launch_bounds__(256) dx_combine_kernel(const __nv_bfloat16 *__restrict__ dXs,
+                                                         const float *__restrict__ dl,
+                                                         const int *__restrict__ topk_idx,
+                                                         const float *__restrict__ router_w,
+                                                         __nv_bfloat16 *__restrict__ dx, int T, int H, int k, int S)
+{
+    const int cpr = H / 8;
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)T * cpr) return;
+    const int t = (int)(i / cpr), c = (int)(i % cpr) * 8;
+    const int kk = k + S;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const __nv_bfloat16 *row = dXs + (size_t)t * kk * H + c;
+    for (int j = 0; j < kk; ++j) {
+        float v[8];
+        unpack8(*reinterpret_cast<const uint4 *>(row + (size_t)j * H), v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] += v[q];
+    }
+    float r[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int j = 0; j < k; ++j) {
+        const float d = dl[(size_t)t * k + j];
+        const float *wr = router_w + (size_t)topk_idx[(size_t)t * k + j] * H + c;
+        const float4 w0 = *reinterpret_cast<const float4 *>(wr);
+        const float4 w1 = *reinterpret_cast<const float4 *>(wr + 4);
+        r[0] = fmaf(d, w0.x, r[0]); r[1] = fmaf(d, w0.y, r[1]); r[2] = fmaf(d, w0.z, r[2]); r[3] = fmaf(d, w0.w, r[3]);
+        r[4] = fmaf(d, w1.x, r[4]); r[5] = fmaf(d, w1.y, r[5]); r[6] = fmaf(d, w1.z, r[6]); r[7] = fmaf(d, w1.w, r[7]);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] += r[q];
+    *reinterpret_cast<uint4 *>(dx + (size_t)t * H + c) = pack8(acc);
+}
+
+}  // namespace mok

@@ -1,0 +1,466 @@
+// gemm.cuh -- persistent, warp-specialised grouped GEMM on tcgen05/TMEM (sm_100a).
+//
+// One template serves every expert contraction of the layer.  A group is one
+// expert (routed experts first, then shared experts) and owns a contiguous
+// range of "sorted rows" (the expert-major order of (token, slot) pairs).
+//
+//   ragged-M (forward, data gradients):  D[rows of g, N] = A[rows of g, K] . B_g[N, K]^T
+//   ragged-K (weight gradients):         D_g[M, N] = sum over rows r of g of A[r, M]^T B[r, N]
+//
+// A rows that belong to a token are pulled by index straight from the token
+// matrix with TMA gather4 (the pull-at-dispatch idea of "Cursor åpner
+// megakernelen…", paragraph on pulling versus pushing tokens, re-derived for
+// one GPU: the expert tile fetches its rows instead of a separate scatter
+// pass).  The push epilogue writes each output row to its (token, slot) row
+// (push at combine, same paragraph).  The shared-memory stage ring walks a
+// fixed-size buffer at tile granularity whatever the routing imbalance (the
+// fixed-size macrobatch ring of "Megakernels are dead and back…", section
+// "Números de MoK").
+//
+// Roles (192 threads): warp 0 issues TMA loads into a STAGES-deep ring, warp 1
+// allocates TMEM and issues tcgen05.mma (one elected thread), warps 2-5 drain
+// the double-buffered TMEM accumulator and run the epilogue.  Every output
+// tile is produced by exactly one CTA with a fixed K order, so results do not
+// depend on scheduling: the layer is bit-reproducible.
+#pragma once
+#include "ptx.cuh"
+
+namespace mok {
+
+constexpr int BM = 128;        // UMMA M (cta_group::1, all 128 TMEM lanes)
+constexpr int BK = 64;         // one 128-byte swizzle row of bf16
+constexpr int kMaxGroups = 264;
+
+enum Epi : int { EPI_SWIGLU = 0, EPI_PUSH = 1, EPI_DSWIGLU = 2, EPI_WGRAD = 3 };
+
+struct GemmArgs {
+    int num_groups;               // G
+    int num_routed;               // groups [0, num_routed) use tmB, the rest tmB_s / out_s
+    const int *offsets;           // [G+1] sorted-row range of every group
+    const int *gorder;            // ragged-K: group processing order (longest first), [G]
+    const int *row_token;         // [R] gather row of each sorted row
+    const int *row_slot;          // [R] destination row of each sorted row (push)
+    const float *row_w;           // [R] routing weight of each sorted row
+    int n_tiles;                  // output tiles along N
+    int m_tiles;                  // ragged-K: output tiles along M
+    int num_kb;                   // ragged-M: K / BK
+    int b_rows_per_group;         // ragged-M: rows of one group in B's 2D view
+    int b_half;                   // EPI_SWIGLU: row offset of the up projection inside a group
+    __nv_bfloat16 *out;           // main output
+    __nv_bfloat16 *out_s;         // EPI_WGRAD: output of the shared groups
+    __nv_bfloat16 *out2;          // EPI_SWIGLU: saved gate/up pre-activations [R, 2I] (or null)
+    __nv_bfloat16 *out3;          // EPI_SWIGLU: w * h [R, I] (or null)
+    const __nv_bfloat16 *aux;     // EPI_DSWIGLU: saved gate/up pre-activations [R, 2I]
+    int ldo;                      // elements per output row
+    int inter;                    // I
+    long long group_out_elems;    // EPI_WGRAD: elements of one group's output
+    int *status;                  // device status word
+};
+
+template <int BN_, bool A_MN_, bool B_MN_, bool A_GATHER_, bool B_GATHER_, bool RAGGED_K_, int EPI_>
+struct GemmCfg {
+    static constexpr int BN = BN_;
+    static constexpr bool A_MN = A_MN_, B_MN = B_MN_, A_GATHER = A_GATHER_, B_GATHER = B_GATHER_;
+    static constexpr bool RAGGED_K = RAGGED_K_;
+    static constexpr int EPI = EPI_;
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = BN == 256 ? 4 : 6;
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int AUX_BYTES = 256 + 3 * kMaxGroups * 4;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
+    static constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
+    static_assert(BN == 128 || BN == 256, "BN");
+    static_assert(!RAGGED_K || (A_MN && B_MN), "weight gradients take both operands MN-major");
+    static_assert(!RAGGED_K || (A_GATHER != B_GATHER), "one operand of a weight gradient is gathered");
+};
+
+struct Tile {
+    int g;          // group
+    int nt;         // N tile
+    int m0;         // ragged-M: first sorted row; ragged-K: first M index
+    int rows;       // ragged-M: valid rows in the tile
+    int krow0;      // ragged-K: first sorted row of the group
+    int krows;      // ragged-K: rows of the group
+    int nkb;        // K blocks
+};
+
+template <class C>
+__device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const int *s_off, const int *s_tstart,
+                                            const int *s_gorder, int G)
+{
+    Tile t;
+    if constexpr (C::RAGGED_K) {
+        const int tpg = a.m_tiles * a.n_tiles;
+        const int gi = tile / tpg, local = tile - gi * tpg;
+        t.g = s_gorder[gi];
+        const int mt = local / a.n_tiles;
+        t.nt = local - mt * a.n_tiles;
+        t.m0 = mt * BM;
+        t.rows = BM;
+        t.krow0 = s_off[t.g];
+        t.krows = s_off[t.g + 1] - t.krow0;
+        t.nkb = (t.krows + BK - 1) / BK;
+    } else {
+        int lo = 0, hi = G - 1;          // largest g with s_tstart[g] <= tile
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
+        }
+        t.g = lo;
+        const int local = tile - s_tstart[lo];
+        const int mt = local / a.n_tiles;
+        t.nt = local - mt * a.n_tiles;
+        t.m0 = s_off[lo] + mt * BM;
+        t.rows = min(BM, s_off[lo + 1] - t.m0);
+        t.krow0 = 0;
+        t.krows = 0;
+        t.nkb = a.num_kb;
+    }
+    return t;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+__device__ __forceinline__ void store_bf16x16(__nv_bfloat16 *dst, const float (&v)[16])
+{
+    uint4 lo, hi;
+    lo.x = pack_bf16x2(v[0], v[1]);   lo.y = pack_bf16x2(v[2], v[3]);
+    lo.z = pack_bf16x2(v[4], v[5]);   lo.w = pack_bf16x2(v[6], v[7]);
+    hi.x = pack_bf16x2(v[8], v[9]);   hi.y = pack_bf16x2(v[10], v[11]);
+    hi.z = pack_bf16x2(v[12], v[13]); hi.w = pack_bf16x2(v[14], v[15]);
+    reinterpret_cast<uint4 *>(dst)[0] = lo;
+    reinterpret_cast<uint4 *>(dst)[1] = hi;
+}
+
+__device__ __forceinline__ void load_bf16x16(const __nv_bfloat16 *src, float (&v)[16])
+{
+    const uint4 lo = reinterpret_cast<const uint4 *>(src)[0];
+    const uint4 hi = reinterpret_cast<const uint4 *>(src)[1];
+    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        v[2 * i] = bf16_lo(w[i]);
+        v[2 * i + 1] = bf16_hi(w[i]);
+    }
+}
+
+template <class C>
+__global__ void __launch_bounds__(192, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB_s, const GemmArgs args)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *tiles = smem;
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(tiles + C::STAGES * C::STAGE_BYTES);
+    uint64_t *empty_bar = full_bar + C::STAGES;
+    uint64_t *accf = empty_bar + C::STAGES;
+    uint64_t *acce = accf + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    int *s_off = reinterpret_cast<int *>(full_bar) + 64;
+    int *s_tstart = s_off + kMaxGroups;
+    int *s_gorder = s_tstart + kMaxGroups;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = args.num_groups;
+    int *status = args.status;
+
+    if (warp == 0) {
+        for (int i = lane; i <= G; i += 32) s_off[i] = args.offsets[i];
+        if constexpr (C::RAGGED_K) {
+            for (int i = lane; i < G; i += 32) s_gorder[i] = args.gorder[i];
+        }
+        __syncwarp();
+        if constexpr (!C::RAGGED_K) {
+            // tile prefix over groups: ceil(rows / BM) * n_tiles tiles each (warp scan)
+            int carry = 0;
+            for (int base = 0; base < G; base += 32) {
+                const int g = base + lane;
+                int v = 0;
+                if (g < G) v = ((s_off[g + 1] - s_off[g] + BM - 1) / BM) * args.n_tiles;
+                int incl = v;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+                    if (lane >= d) incl += o;
+                }
+                if (g < G) s_tstart[g] = carry + incl - v;
+                carry += __shfl_sync(0xffffffffu, incl, 31);
+            }
+            if (lane == 0) s_tstart[G] = carry;
+        }
+        if (lane == 0) {
+            for (int s = 0; s < C::STAGES; ++s) {
+                mbar_init(&full_bar[s], 1);
+                mbar_init(&empty_bar[s], 1);
+            }
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(&accf[b], 1);
+                mbar_init(&acce[b], 128);
+            }
+            *abort_flag = 0;
+            fence_barrier_init();
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            tma_prefetch_desc(&tmB_s);
+        }
+    } else if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = C::RAGGED_K ? G * args.m_tiles * args.n_tiles : s_tstart[G];
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
+            const bool routed = t.g < args.num_routed;
+            const CUtensorMap *mB = routed ? &tmB : &tmB_s;
+            const int gl = routed ? t.g : t.g - args.num_routed;
+            for (int kb = 0; kb < t.nkb; ++kb) {
+                bool ok = true;
+                if (lane == 0) {
+                    ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status);
+                    if (ok) mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) goto producer_done;
+                uint8_t *sA = tiles + stage * C::STAGE_BYTES;
+                uint8_t *sB = sA + C::A_BYTES;
+                uint64_t *fb = &full_bar[stage];
+                // ---- A
+                if constexpr (C::A_GATHER && !C::A_MN) {
+                    const int r = t.m0 + 4 * lane, end = t.m0 + t.rows;
+                    const int i0 = r + 0 < end ? args.row_token[r + 0] : 0;
+                    const int i1 = r + 1 < end ? args.row_token[r + 1] : 0;
+                    const int i2 = r + 2 < end ? args.row_token[r + 2] : 0;
+                    const int i3 = r + 3 < end ? args.row_token[r + 3] : 0;
+                    tma_gather4(sA + lane * 512, &tmA, fb, kb * BK, i0, i1, i2, i3);
+                } else if constexpr (!C::A_GATHER && !C::A_MN) {
+                    if (lane == 0) tma_load_2d(sA, &tmA, fb, kb * BK, t.m0);
+                } else if constexpr (C::A_GATHER && C::A_MN) {
+                    const int chunk = lane >> 4, q = lane & 15;
+                    const int r = t.krow0 + kb * BK + 4 * q, end = t.krow0 + t.krows;
+                    const int i0 = r + 0 < end ? args.row_token[r + 0] : 0;
+                    const int i1 = r + 1 < end ? args.row_token[r + 1] : 0;
+                    const int i2 = r + 2 < end ? args.row_token[r + 2] : 0;
+                    const int i3 = r + 3 < end ? args.row_token[r + 3] : 0;
+                    tma_gather4(sA + chunk * 8192 + q * 512, &tmA, fb, t.m0 + chunk * 64, i0, i1, i2, i3);
+                } else {
+                    if (lane < BM / 64) tma_load_2d(sA + lane * 8192, &tmA, fb, t.m0 + lane * 64, t.krow0 + kb * BK);
+                }
+                // ---- B
+                if constexpr (!C::B_MN) {
+                    if (lane == 0) {
+                        if constexpr (C::EPI == EPI_SWIGLU) {
+                            const int row = gl * args.b_rows_per_group + t.nt * 128;
+                            tma_load_2d(sB, mB, fb, kb * BK, row);
+                            tma_load_2d(sB + 128 * 128, mB, fb, kb * BK, row + args.b_half);
+                        } else {
+                            tma_load_2d(sB, mB, fb, kb * BK, gl * args.b_rows_per_group + t.nt * C::BN);
+                        }
+                    }
+                } else if constexpr (!C::B_GATHER && !C::RAGGED_K) {
+                    if (lane < C::BN / 64)
+                        tma_load_2d(sB + lane * 8192, mB, fb, t.nt * C::BN + lane * 64,
+                                    gl * args.b_rows_per_group + kb * BK);
+                } else if constexpr (!C::B_GATHER && C::RAGGED_K) {
+                    if (lane < C::BN / 64)
+                        tma_load_2d(sB + lane * 8192, &tmB, fb, t.nt * C::BN + lane * 64, t.krow0 + kb * BK);
+                } else {
+#pragma unroll
+                    for (int op = lane; op < (C::BN / 64) * 16; op += 32) {
+                        const int chunk = op >> 4, q = op & 15;
+                        const int r = t.krow0 + kb * BK + 4 * q, end = t.krow0 + t.krows;
+                        const int i0 = r + 0 < end ? args.row_token[r + 0] : 0;
+                        const int i1 = r + 1 < end ? args.row_token[r + 1] : 0;
+                        const int i2 = r + 2 < end ? args.row_token[r + 2] : 0;
+                        const int i3 = r + 3 < end ? args.row_token[r + 3] : 0;
+                        tma_gather4(sB + chunk * 8192 + q * 512, &tmB, fb, t.nt * C::BN + chunk * 64, i0, i1, i2,
+                                    i3);
+                    }
+                }
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    producer_done:;
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        int stage = 0, acc = 0;
+        uint32_t phase = 0, acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&acce[acc], acc_phase ^ 1u, abort_flag, status);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
+            for (int kb = 0; kb < t.nkb; ++kb) {
+                if (lane == 0) ok = mbar_wait(&full_bar[stage], phase, abort_flag, status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                uint8_t *sA = tiles + stage * C::STAGE_BYTES;
+                uint8_t *sB = sA + C::A_BYTES;
+                if constexpr (C::RAGGED_K) {
+                    const int valid = t.krows - kb * BK;
+                    if (valid < BK) {
+                        // rows past the group's end: zero them in the contiguous operand
+                        // (the gathered operand holds finite rows there)
+                        uint8_t *base = C::A_GATHER ? sB : sA;
+                        const int chunks = C::A_GATHER ? C::BN / 64 : BM / 64;
+                        const int n16 = (BK - valid) * 8;
+                        for (int c = 0; c < chunks; ++c) {
+                            uint4 *p = reinterpret_cast<uint4 *>(base + c * 8192 + valid * 128);
+                            for (int i = lane; i < n16; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+#pragma unroll
+                    for (int k = 0; k < BK / 16; ++k) {
+                        const uint64_t ad = C::A_MN ? smem_desc_sw128(a0 + k * 2048, 8192, 1024)
+                                                    : smem_desc_sw128(a0 + k * 32, 16, 1024);
+                        const uint64_t bd = C::B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024)
+                                                    : smem_desc_sw128(b0 + k * 32, 16, 1024);
+                        umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&empty_bar[stage]);
+                }
+                __syncwarp();
+                if (++stage == C::STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) {
+                if (t.nkb > 0) umma_commit(&accf[acc]);
+                else mbar_arrive(&accf[acc]);
+            }
+            __syncwarp();
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int eq = warp & 3;                 // TMEM lane quarter this warp may access
+        const int row = eq * 32 + lane;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
+            if (!mbar_wait(&accf[acc], acc_phase, abort_flag, status)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * C::BN) + (static_cast<uint32_t>(eq * 32) << 16);
+            if constexpr (C::EPI == EPI_SWIGLU) {
+                const int r = t.m0 + row;
+                const bool valid = row < t.rows;
+                const int I = args.inter;
+                const int n0 = t.nt * 128;
+                const float w = (valid && args.out3) ? args.row_w[r] : 0.0f;
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 16) {
+                    float g[16], u[16], h[16];
+                    tmem_ld16(taddr + c, g);
+                    tmem_ld16(taddr + 128 + c, u);
+                    tmem_ld_wait();
+                    if (valid) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) h[i] = silu_f(g[i]) * u[i];
+                        store_bf16x16(args.out + (size_t)r * I + n0 + c, h);
+                        if (args.out2) {
+                            store_bf16x16(args.out2 + (size_t)r * 2 * I + n0 + c, g);
+                            store_bf16x16(args.out2 + (size_t)r * 2 * I + I + n0 + c, u);
+                        }
+                        if (args.out3) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) h[i] = w * bf16_round(h[i]);
+                            store_bf16x16(args.out3 + (size_t)r * I + n0 + c, h);
+                        }
+                    }
+                }
+            } else if constexpr (C::EPI == EPI_PUSH) {
+                const bool valid = row < t.rows;
+                const size_t drow = valid ? static_cast<size_t>(args.row_slot[t.m0 + row]) : 0;
+#pragma unroll 1
+                for (int c = 0; c < C::BN; c += 16) {
+                    float v[16];
+                    tmem_ld16(taddr + c, v);
+                    tmem_ld_wait();
+                    if (valid) store_bf16x16(args.out + drow * args.ldo + t.nt * C::BN + c, v);
+                }
+            } else if constexpr (C::EPI == EPI_DSWIGLU) {
+                const int r = t.m0 + row;
+                const bool valid = row < t.rows;
+                const int I = args.inter;
+                const int n0 = t.nt * C::BN;
+                const float w = valid ? args.row_w[r] : 0.0f;
+#pragma unroll 1
+                for (int c = 0; c < C::BN; c += 16) {
+                    float v[16], g[16], u[16], dg[16], du[16];
+                    tmem_ld16(taddr + c, v);
+                    tmem_ld_wait();
+                    if (valid) {
+                        load_bf16x16(args.aux + (size_t)r * 2 * I + n0 + c, g);
+                        load_bf16x16(args.aux + (size_t)r * 2 * I + I + n0 + c, u);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float dh = w * v[i];
+                            const float sg = 1.0f / (1.0f + expf(-g[i]));
+                            dg[i] = dh * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
+                            du[i] = dh * g[i] * sg;
+                        }
+                        store_bf16x16(args.out + (size_t)r * 2 * I + n0 + c, dg);
+                        store_bf16x16(args.out + (size_t)r * 2 * I + I + n0 + c, du);
+                    }
+                }
+            } else {   // EPI_WGRAD
+                const bool routed = t.g < args.num_routed;
+                __nv_bfloat16 *base = routed ? args.out + (size_t)t.g * args.group_out_elems
+                                             : args.out_s + (size_t)(t.g - args.num_routed) * args.group_out_elems;
+                __nv_bfloat16 *dst = base + (size_t)(t.m0 + row) * args.ldo + t.nt * C::BN;
+#pragma unroll 1
+                for (int c = 0; c < C::BN; c += 16) {
+                    float v[16];
+                    if (t.nkb > 0) {
+                        tmem_ld16(taddr + c, v);
+                        tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+                    }
+                    store_bf16x16(dst + c, v);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&acce[acc]);
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1u;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace mok

@@ -1,0 +1,556 @@
+// mok.cu -- the C ABI of libmok (see include/mok.h): argument checks, the
+// layout of the caller's ctx/scratch buffers, TMA descriptors and the launch
+// sequence of the forward and backward passes.  All launches go to the
+// caller's stream; nothing here waits on the device except moe_status and the
+// host-buffer variants.
+#include "mok.h"
+
+#include <cudaTypedefs.h>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "combine.cuh"
+#include "gemm.cuh"
+#include "quant.cuh"
+#include "route.cuh"
+
+namespace mok {
+
+__device__ int g_status;   // device status word (MOK_STATUS_* bits)
+
+namespace {
+
+constexpr int kChunkRows = 256;   // router-gradient row chunk
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    bool init = false;
+    bool ok = false;
+    int sms = 0;
+    int *status = nullptr;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+const DeviceInfo *device_info()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.init) {
+        d.init = true;
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        void *p = nullptr;
+        const bool sym = cudaGetSymbolAddress(&p, g_status) == cudaSuccess;
+        d.status = static_cast<int *>(p);
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess)
+                g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        d.ok = major == 10 && minor == 0 && sym && g_encode != nullptr && d.sms > 0;
+    }
+    return d.ok ? &d : nullptr;
+}
+
+// 2D tensor map over a row-major [outer, inner] matrix, 128-byte swizzle.
+bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+               uint32_t box_outer, size_t elem_bytes)
+{
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * elem_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t es[2] = {1, 1};
+    const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const CUresult r = g_encode(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Offsets of the arrays inside a buffer, laid out in order with 256-byte alignment.
+struct Carver {
+    size_t off = 0;
+    char *base;
+    explicit Carver(void *b) : base(static_cast<char *>(b)) {}
+    template <class T> T *take(size_t count)
+    {
+        off = align_up(off, 256);
+        T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+        off += count * sizeof(T);
+        return p;
+    }
+};
+
+struct Shapes {
+    long long T, H, E, I, k, S, G, kk, R, TK;
+    long long max_chunks;
+};
+
+Shapes shapes(const moe_cfg &c)
+{
+    Shapes s;
+    s.T = c.T; s.H = c.H; s.E = c.E; s.I = c.I; s.k = c.top_k; s.S = c.n_shared;
+    s.G = s.E + s.S;
+    s.kk = s.k + s.S;
+    s.TK = s.T * s.k;
+    s.R = s.TK + s.S * s.T;
+    s.max_chunks = (s.TK + kChunkRows - 1) / kChunkRows + s.E;
+    return s;
+}
+
+// forward state: what the backward reads, plus what the forward needs anyway
+struct State {
+    int *topk_idx, *counts, *offsets, *gorder, *chunk_start, *perm, *inv_perm, *row_token, *row_slot;
+    float *topk_w, *topk_p, *row_w;
+    __nv_bfloat16 *gu, *h, *hw, *O;
+    uint8_t *xq, *xs, *hq, *hs;     // MXFP8 operands
+    size_t bytes;
+};
+
+State carve_state(const moe_cfg &c, void *buf, bool training)
+{
+    const Shapes s = shapes(c);
+    const bool mx = c.dtype == MOK_DTYPE_MXFP8;
+    Carver cv(buf);
+    State st{};
+    st.topk_idx = cv.take<int>(s.TK);
+    st.topk_w = cv.take<float>(s.TK);
+    st.topk_p = cv.take<float>(s.TK);
+    st.counts = cv.take<int>(s.E);
+    st.offsets = cv.take<int>(s.G + 1);
+    st.gorder = cv.take<int>(s.G);
+    st.chunk_start = cv.take<int>(s.E + 1);
+    st.perm = cv.take<int>(s.TK);
+    st.inv_perm = cv.take<int>(s.TK);
+    st.row_token = cv.take<int>(s.R);
+    st.row_slot = cv.take<int>(s.R);
+    st.row_w = cv.take<float>(s.R);
+    st.gu = training ? cv.take<__nv_bfloat16>(s.R * 2 * s.I) : nullptr;
+    st.hw = training ? cv.take<__nv_bfloat16>(s.R * s.I) : nullptr;
+    if (mx) {
+        st.h = nullptr;
+        st.hq = cv.take<uint8_t>(s.R * s.I);
+        st.hs = cv.take<uint8_t>(s.R * s.I / 32);
+        st.xq = cv.take<uint8_t>(s.T * s.H);
+        st.xs = cv.take<uint8_t>(s.T * s.H / 32);
+    } else {
+        st.h = cv.take<__nv_bfloat16>(s.R * s.I);
+        st.hq = st.hs = st.xq = st.xs = nullptr;
+    }
+    st.O = cv.take<__nv_bfloat16>(s.T * s.kk * s.H);
+    st.bytes = align_up(cv.off, 256);
+    return st;
+}
+
+struct BwdScratch {
+    float *dl, *partial;
+    __nv_bfloat16 *dgu, *dxs;
+    size_t bytes;
+};
+
+BwdScratch carve_bwd(const moe_cfg &c, void *buf)
+{
+    const Shapes s = shapes(c);
+    Carver cv(buf);
+    BwdScratch b{};
+    b.dl = cv.take<float>(s.TK);
+    b.partial = cv.take<float>(s.max_chunks * s.H);
+    b.dgu = cv.take<__nv_bfloat16>(s.R * 2 * s.I);
+    b.dxs = cv.take<__nv_bfloat16>(s.T * s.kk * s.H);
+    b.bytes = align_up(cv.off, 256);
+    return b;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cfg(const moe_cfg *c)
+{
+    if (!c) return MOK_ERR_INVALID;
+    if (c->T < 1 || c->H < 256 || c->H % 256 || c->E < 1 || c->E > 256 || c->I < 128 || c->I % 128) return MOK_ERR_INVALID;
+    if (c->top_k < 1 || c->top_k > 16 || c->top_k > c->E) return MOK_ERR_INVALID;
+    if (c->n_shared < 0 || c->n_shared > 4) return MOK_ERR_INVALID;
+    if (c->n_shared > 0 && c->I_shared != c->I) return MOK_ERR_UNSUPPORTED;
+    if (c->score_fn != MOK_SCORE_SOFTMAX && c->score_fn != MOK_SCORE_SIGMOID) return MOK_ERR_INVALID;
+    if (c->n_group < 1 || c->n_group > 32 || c->E % c->n_group) return MOK_ERR_INVALID;
+    if (c->topk_group < 1 || c->topk_group > c->n_group) return MOK_ERR_INVALID;
+    if (c->n_group > 1 && c->topk_group < c->n_group && c->top_k > c->topk_group * (c->E / c->n_group))
+        return MOK_ERR_INVALID;
+    if (!(c->routed_scale > 0.0f)) return MOK_ERR_INVALID;
+    if (c->dtype != MOK_DTYPE_BF16 && c->dtype != MOK_DTYPE_MXFP8) return MOK_ERR_INVALID;
+    const long long R = (long long)c->T * (c->top_k + c->n_shared);
+    if (R >= (1ll << 31)) return MOK_ERR_INVALID;
+    return MOK_OK;
+}
+
+template <class C>
+int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &bs, const GemmArgs &args, int grid,
+                cudaStream_t st)
+{
+    if (grid <= 0) return MOK_OK;
+    if (cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
+        cudaSuccess)
+        return MOK_ERR_LAUNCH;
+    grouped_gemm_kernel<C><<<grid, 192, C::SMEM_BYTES, st>>>(a, b, bs, args);
+    return cudaGetLastError() == cudaSuccess ? MOK_OK : MOK_ERR_LAUNCH;
+}
+
+inline int blocks_for(long long n, int per) { return static_cast<int>((n + per - 1) / per); }
+
+#define MOK_TRY(expr)                 \
+    do {                              \
+        const int rc_ = (expr);       \
+        if (rc_ != MOK_OK) return rc_; \
+    } while (0)
+
+#define MOK_LAUNCHED()                                                     \
+    do {                                                                   \
+        if (cudaGetLastError() != cudaSuccess) return MOK_ERR_LAUNCH;       \
+    } while (0)
+
+// ------------------------------------------------------------------ forward
+int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const moe_routing *routing,
+            const State &st, const DeviceInfo &dev, bool training, cudaStream_t stream)
+{
+    const Shapes s = shapes(c);
+    if (c.dtype != MOK_DTYPE_BF16) return MOK_ERR_UNSUPPORTED;
+
+    RouteArgs ra;
+    ra.x = static_cast<const __nv_bfloat16 *>(x);
+    ra.router_w = p.router_w;
+    ra.e_bias = p.e_bias;
+    ra.logit_bias = p.logit_bias;
+    ra.T = c.T; ra.H = c.H; ra.E = c.E; ra.k = c.top_k;
+    ra.score_fn = c.score_fn; ra.n_group = c.n_group; ra.topk_group = c.topk_group;
+    ra.routed_scale = c.routed_scale;
+    ra.topk_idx = st.topk_idx; ra.topk_w = st.topk_w; ra.topk_p = st.topk_p;
+    router_kernel<<<blocks_for(s.T, kRouteTokens), 256, 0, stream>>>(ra);
+    MOK_LAUNCHED();
+
+    DispatchArgs da;
+    da.topk_idx = st.topk_idx; da.topk_w = st.topk_w;
+    da.T = c.T; da.k = c.top_k; da.E = c.E; da.S = c.n_shared; da.chunk_rows = kChunkRows;
+    da.counts = st.counts; da.offsets = st.offsets; da.gorder = st.gorder; da.chunk_start = st.chunk_start;
+    da.perm = st.perm; da.inv_perm = st.inv_perm; da.row_token = st.row_token; da.row_slot = st.row_slot;
+    da.row_w = st.row_w;
+    dispatch_kernel<<<1, 1024, 0, stream>>>(da);
+    MOK_LAUNCHED();
+
+    // gate/up: pull token rows by index, SwiGLU epilogue
+    CUtensorMap tA, tB, tBs;
+    if (!make_tmap(&tA, x, s.H, s.T, BK, 1, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, BK, 128, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, BK, 128, 2))
+        return MOK_ERR_INVALID;
+    GemmArgs ga{};
+    ga.num_groups = static_cast<int>(s.G);
+    ga.num_routed = c.E;
+    ga.offsets = st.offsets;
+    ga.row_token = st.row_token;
+    ga.row_slot = st.row_slot;
+    ga.row_w = st.row_w;
+    ga.n_tiles = c.I / 128;
+    ga.num_kb = c.H / BK;
+    ga.b_rows_per_group = 2 * c.I;
+    ga.b_half = c.I;
+    ga.out = st.h;
+    ga.out2 = training ? st.gu : nullptr;
+    ga.out3 = training ? st.hw : nullptr;
+    ga.inter = c.I;
+    ga.status = dev.status;
+    using CGateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU>;
+    MOK_TRY(launch_gemm<CGateUp>(tA, tB, tBs, ga, dev.sms, stream));
+
+    // down: contiguous h rows, push epilogue into (token, slot) rows
+    if (!make_tmap(&tA, st.h, s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, BK, 256, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, BK, 256, 2))
+        return MOK_ERR_INVALID;
+    GemmArgs gd = ga;
+    gd.n_tiles = c.H / 256;
+    gd.num_kb = c.I / BK;
+    gd.b_rows_per_group = c.H;
+    gd.b_half = 0;
+    gd.out = st.O;
+    gd.out2 = gd.out3 = nullptr;
+    gd.ldo = c.H;
+    using CDown = GemmCfg<256, false, false, false, false, false, EPI_PUSH>;
+    MOK_TRY(launch_gemm<CDown>(tA, tB, tBs, gd, dev.sms, stream));
+
+    combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(st.O, st.topk_w,
+                                                                       static_cast<__nv_bfloat16 *>(y), c.T, c.H,
+                                                                       c.top_k, c.n_shared);
+    MOK_LAUNCHED();
+
+    if (routing) {
+        const size_t tk = static_cast<size_t>(s.TK);
+        if (routing->topk_idx && cudaMemcpyAsync(routing->topk_idx, st.topk_idx, tk * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
+        if (routing->topk_w && cudaMemcpyAsync(routing->topk_w, st.topk_w, tk * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
+        if (routing->counts && cudaMemcpyAsync(routing->counts, st.counts, s.E * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
+        if (routing->offsets && cudaMemcpyAsync(routing->offsets, st.offsets, (s.E + 1) * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
+        if (routing->perm && cudaMemcpyAsync(routing->perm, st.perm, tk * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
+        if (routing->inv_perm && cudaMemcpyAsync(routing->inv_perm, st.inv_perm, tk * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
+    }
+    return MOK_OK;
+}
+
+// ------------------------------------------------------------------ backward
+int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &p, const State &st,
+             const moe_grads &gr, const BwdScratch &bs, const DeviceInfo &dev, cudaStream_t stream)
+{
+    const Shapes s = shapes(c);
+    const __nv_bfloat16 *dyb = static_cast<const __nv_bfloat16 *>(dy);
+
+    slot_grad_kernel<<<c.T, 256, 0, stream>>>(dyb, st.O, st.topk_w, st.topk_p, bs.dl, c.T, c.H, c.top_k,
+                                              c.n_shared, c.score_fn, c.routed_scale);
+    MOK_LAUNCHED();
+    drouter_partial_kernel<<<dim3(static_cast<unsigned>(s.max_chunks), c.H / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(x), bs.dl, st.offsets, st.chunk_start, st.perm, bs.partial, c.H, c.E,
+        c.top_k, kChunkRows);
+    MOK_LAUNCHED();
+    drouter_reduce_kernel<<<blocks_for(s.E * s.H, 256), 256, 0, stream>>>(bs.partial, st.chunk_start,
+                                                                          gr.drouter_w, c.H, c.E);
+    MOK_LAUNCHED();
+
+    GemmArgs base{};
+    base.num_groups = static_cast<int>(s.G);
+    base.num_routed = c.E;
+    base.offsets = st.offsets;
+    base.gorder = st.gorder;
+    base.row_token = st.row_token;
+    base.row_slot = st.row_slot;
+    base.row_w = st.row_w;
+    base.inter = c.I;
+    base.status = dev.status;
+
+    CUtensorMap tA, tB, tBs;
+    // dgrad of down: dh = w * (dy[token] . W_down), SwiGLU backward epilogue -> dGU
+    if (!make_tmap(&tA, dy, s.H, s.T, BK, 1, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
+    GemmArgs g1 = base;
+    g1.n_tiles = c.I / 128;
+    g1.num_kb = c.H / BK;
+    g1.b_rows_per_group = c.H;
+    g1.aux = st.gu;
+    g1.out = bs.dgu;
+    using CDgradDown = GemmCfg<128, false, true, true, false, false, EPI_DSWIGLU>;
+    MOK_TRY(launch_gemm<CDgradDown>(tA, tB, tBs, g1, dev.sms, stream));
+
+    // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
+    if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
+    GemmArgs g2 = base;
+    g2.m_tiles = c.H / 128;
+    g2.n_tiles = c.I / 128;
+    g2.out = static_cast<__nv_bfloat16 *>(gr.dw_down);
+    g2.out_s = static_cast<__nv_bfloat16 *>(gr.dws_down);
+    g2.ldo = c.I;
+    g2.group_out_elems = s.H * s.I;
+    using CWgradDown = GemmCfg<128, true, true, true, false, true, EPI_WGRAD>;
+    const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
+    MOK_TRY(launch_gemm<CWgradDown>(tA, tB, tB, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms), stream));
+
+    // dgrad of gate/up: dX rows = dGU . W_gate_up, pushed into (token, slot) rows
+    if (!make_tmap(&tA, bs.dgu, 2 * s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, 64, 64, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 64, 64, 2))
+        return MOK_ERR_INVALID;
+    GemmArgs g3 = base;
+    g3.n_tiles = c.H / 256;
+    g3.num_kb = 2 * c.I / BK;
+    g3.b_rows_per_group = 2 * c.I;
+    g3.out = bs.dxs;
+    g3.ldo = c.H;
+    using CDgradGU = GemmCfg<256, false, true, false, false, false, EPI_PUSH>;
+    MOK_TRY(launch_gemm<CDgradGU>(tA, tB, tBs, g3, dev.sms, stream));
+
+    // wgrad of gate/up: dW_gate_up[g] = sum_r dGU_r^T x[token r]
+    if (!make_tmap(&tA, bs.dgu, 2 * s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tB, x, s.H, s.T, BK, 1, 2)) return MOK_ERR_INVALID;
+    GemmArgs g4 = base;
+    g4.m_tiles = 2 * c.I / 128;
+    g4.n_tiles = c.H / 256;
+    g4.out = static_cast<__nv_bfloat16 *>(gr.dw_gate_up);
+    g4.out_s = static_cast<__nv_bfloat16 *>(gr.dws_gate_up);
+    g4.ldo = c.H;
+    g4.group_out_elems = 2 * s.I * s.H;
+    using CWgradGU = GemmCfg<256, true, true, false, true, true, EPI_WGRAD>;
+    const long long t4 = s.G * g4.m_tiles * g4.n_tiles;
+    MOK_TRY(launch_gemm<CWgradGU>(tA, tB, tB, g4, static_cast<int>(t4 < dev.sms ? t4 : dev.sms), stream));
+
+    dx_combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(
+        bs.dxs, bs.dl, st.topk_idx, p.router_w, static_cast<__nv_bfloat16 *>(gr.dx), c.T, c.H, c.top_k,
+        c.n_shared);
+    MOK_LAUNCHED();
+    return MOK_OK;
+}
+
+int check_params(const moe_cfg &c, const moe_params *p)
+{
+    if (!p || !p->router_w || !p->w_gate_up || !p->w_down) return MOK_ERR_INVALID;
+    if (c.n_shared > 0 && (!p->ws_gate_up || !p->ws_down)) return MOK_ERR_INVALID;
+    if (c.dtype == MOK_DTYPE_MXFP8 && (!p->s_gate_up || !p->s_down || (c.n_shared > 0 && (!p->ss_gate_up || !p->ss_down))))
+        return MOK_ERR_INVALID;
+    const void *ptrs[] = {p->router_w, p->w_gate_up, p->w_down, p->ws_gate_up, p->ws_down};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return MOK_ERR_INVALID;
+    return MOK_OK;
+}
+
+}  // namespace
+}  // namespace mok
+
+using namespace mok;
+
+extern "C" {
+
+int moe_workspace_size(const moe_cfg *cfg, size_t *ctx_bytes, size_t *fwd_scratch_bytes, size_t *bwd_scratch_bytes)
+{
+    MOK_TRY(check_cfg(cfg));
+    if (ctx_bytes) *ctx_bytes = carve_state(*cfg, nullptr, true).bytes;
+    if (fwd_scratch_bytes) *fwd_scratch_bytes = carve_state(*cfg, nullptr, false).bytes;
+    if (bwd_scratch_bytes) *bwd_scratch_bytes = carve_bwd(*cfg, nullptr).bytes;
+    return MOK_OK;
+}
+
+int moe_fwd(const moe_cfg *cfg, const void *x, const moe_params *params, void *y, const moe_routing *routing,
+            void *ctx, size_t ctx_bytes, int save_for_backward, void *scratch, size_t scratch_bytes, void *stream)
+{
+    MOK_TRY(check_cfg(cfg));
+    MOK_TRY(check_params(*cfg, params));
+    if (!x || !y || !aligned16(x) || !aligned16(y)) return MOK_ERR_INVALID;
+    const DeviceInfo *dev = device_info();
+    if (!dev) return MOK_ERR_DEVICE;
+    const bool training = save_for_backward != 0;
+    void *buf = training ? ctx : scratch;
+    const size_t have = training ? ctx_bytes : scratch_bytes;
+    const State need = carve_state(*cfg, nullptr, training);
+    if (!buf || have < need.bytes) return MOK_ERR_WORKSPACE;
+    if (!aligned16(buf)) return MOK_ERR_INVALID;
+    const State st = carve_state(*cfg, buf, training);
+    return forward(*cfg, x, *params, y, routing, st, *dev, training, static_cast<cudaStream_t>(stream));
+}
+
+int moe_bwd(const moe_cfg *cfg, const void *x, const void *dy, const moe_params *params, const void *ctx,
+            size_t ctx_bytes, const moe_grads *grads, void *scratch, size_t scratch_bytes, void *stream)
+{
+    MOK_TRY(check_cfg(cfg));
+    MOK_TRY(check_params(*cfg, params));
+    if (cfg->dtype != MOK_DTYPE_BF16) return MOK_ERR_UNSUPPORTED;
+    if (!x || !dy || !grads || !grads->dx || !grads->dw_gate_up || !grads->dw_down || !grads->drouter_w)
+        return MOK_ERR_INVALID;
+    if (cfg->n_shared > 0 && (!grads->dws_gate_up || !grads->dws_down)) return MOK_ERR_INVALID;
+    const void *ptrs[] = {x, dy, grads->dx, grads->dw_gate_up, grads->dw_down, grads->drouter_w,
+                          grads->dws_gate_up, grads->dws_down};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return MOK_ERR_INVALID;
+    const DeviceInfo *dev = device_info();
+    if (!dev) return MOK_ERR_DEVICE;
+    if (!ctx || ctx_bytes < carve_state(*cfg, nullptr, true).bytes) return MOK_ERR_WORKSPACE;
+    if (!scratch || scratch_bytes < carve_bwd(*cfg, nullptr).bytes) return MOK_ERR_WORKSPACE;
+    if (!aligned16(ctx) || !aligned16(scratch)) return MOK_ERR_INVALID;
+    const State st = carve_state(*cfg, const_cast<void *>(ctx), true);
+    const BwdScratch bs = carve_bwd(*cfg, scratch);
+    return backward(*cfg, x, dy, *params, st, *grads, bs, *dev, static_cast<cudaStream_t>(stream));
+}
+
+int moe_host_scratch_size(const moe_cfg *cfg, int backward, size_t *bytes)
+{
+    MOK_TRY(check_cfg(cfg));
+    const size_t io = align_up(static_cast<size_t>(cfg->T) * cfg->H * 2, 256);
+    size_t inner = backward ? carve_bwd(*cfg, nullptr).bytes : carve_state(*cfg, nullptr, false).bytes;
+    if (bytes) *bytes = (backward ? 3 : 2) * io + inner;
+    return MOK_OK;
+}
+
+int moe_fwd_host(const moe_cfg *cfg, const void *x_host, const moe_params *params, void *y_host, void *ctx,
+                 size_t ctx_bytes, int save_for_backward, void *scratch, size_t scratch_bytes, void *stream)
+{
+    MOK_TRY(check_cfg(cfg));
+    if (!x_host || !y_host || !scratch) return MOK_ERR_INVALID;
+    size_t need = 0;
+    moe_host_scratch_size(cfg, 0, &need);
+    if (scratch_bytes < need) return MOK_ERR_WORKSPACE;
+    const size_t io = align_up(static_cast<size_t>(cfg->T) * cfg->H * 2, 256);
+    char *s = static_cast<char *>(scratch);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t nb = static_cast<size_t>(cfg->T) * cfg->H * 2;
+    if (cudaMemcpyAsync(s, x_host, nb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOK_ERR_LAUNCH;
+    MOK_TRY(moe_fwd(cfg, s, params, s + io, nullptr, ctx, ctx_bytes, save_for_backward, s + 2 * io,
+                    scratch_bytes - 2 * io, stream));
+    if (cudaMemcpyAsync(y_host, s + io, nb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOK_ERR_LAUNCH;
+    return cudaStreamSynchronize(st) == cudaSuccess ? MOK_OK : MOK_ERR_LAUNCH;
+}
+
+int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, const moe_params *params,
+                 const void *ctx, size_t ctx_bytes, void *dx_host, const moe_grads *grads, void *scratch,
+                 size_t scratch_bytes, void *stream)
+{
+    MOK_TRY(check_cfg(cfg));
+    if (!x_host || !dy_host || !dx_host || !scratch || !grads) return MOK_ERR_INVALID;
+    size_t need = 0;
+    moe_host_scratch_size(cfg, 1, &need);
+    if (scratch_bytes < need) return MOK_ERR_WORKSPACE;
+    const size_t io = align_up(static_cast<size_t>(cfg->T) * cfg->H * 2, 256);
+    char *s = static_cast<char *>(scratch);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t nb = static_cast<size_t>(cfg->T) * cfg->H * 2;
+    if (cudaMemcpyAsync(s, x_host, nb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOK_ERR_LAUNCH;
+    if (cudaMemcpyAsync(s + io, dy_host, nb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOK_ERR_LAUNCH;
+    moe_grads g = *grads;
+    g.dx = s + 2 * io;
+    MOK_TRY(moe_bwd(cfg, s, s + io, params, ctx, ctx_bytes, &g, s + 3 * io, scratch_bytes - 3 * io, stream));
+    if (cudaMemcpyAsync(dx_host, s + 2 * io, nb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOK_ERR_LAUNCH;
+    return cudaStreamSynchronize(st) == cudaSuccess ? MOK_OK : MOK_ERR_LAUNCH;
+}
+
+int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *scales, void *stream)
+{
+    if (!src || !q || !scales || rows < 0 || K <= 0 || K % 32) return MOK_ERR_INVALID;
+    if (!aligned16(src) || !aligned16(q)) return MOK_ERR_INVALID;
+    if (!device_info()) return MOK_ERR_DEVICE;
+    const long long nb = rows * (K / 32);
+    if (nb == 0) return MOK_OK;
+    quantize_mxfp8_kernel<<<blocks_for(nb, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16 *>(src), nb, static_cast<uint8_t *>(q), static_cast<uint8_t *>(scales));
+    return cudaGetLastError() == cudaSuccess ? MOK_OK : MOK_ERR_LAUNCH;
+}
+
+int moe_status(void *stream, int32_t *device_status)
+{
+    if (!device_status) return MOK_ERR_INVALID;
+    if (!device_info()) return MOK_ERR_DEVICE;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOK_ERR_LAUNCH;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MOK_ERR_LAUNCH;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MOK_ERR_LAUNCH;
+    *device_status = v;
+    return MOK_OK;
+}
+
+const char *moe_strerror(int code)
+{
+    switch (code) {
+    case MOK_OK: return "ok";
+    case MOK_ERR_INVALID: return "invalid argument (shape, pointer, alignment or option)";
+    case MOK_ERR_DEVICE: return "current device is not an sm_100 (B200) GPU";
+    case MOK_ERR_WORKSPACE: return "ctx or scratch buffer too small";
+    case MOK_ERR_LAUNCH: return "a CUDA call failed while enqueueing work";
+    case MOK_ERR_UNSUPPORTED: return "combination not supported";
+    default: return "unknown error";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// quant.cuh -- MXFP8 quantisation (e4m3 elements, one ue8m0 scale per 32
+// consecutive elements along the contraction axis), as used by the MXFP8
+// forward ("Megakernels are dead and back…", section "Números de MoK").
+//
+// Block rule: e = smallest integer with amax <= 448 * 2^e (448 = largest e4m3
+// value), clamped to [-127, 127], an all-zero block taking -127; the scale byte
+// is e + 127 and every element is x * 2^-e rounded to nearest even e4m3 with
+// saturation.  With this rule no element saturates.
+#pragma once
+#include <cuda_fp8.h>
+#include "ptx.cuh"
+
+namespace mok {
+
+// Exponent of the block from the fp32 bit pattern of amax (exact integer logic):
+// amax = (1 + f) 2^p; 448 * 2^(p-8) = 1.75 * 2^p covers it iff f <= 0.75.
+__device__ __forceinline__ int mx_exponent(float amax)
+{
+    const uint32_t b = __float_as_uint(amax);
+    const int biased = static_cast<int>(b >> 23);
+    if (biased == 0) return -127;                    // zero or subnormal: far below 448 * 2^-127
+    const int p = biased - 127;
+    int e = p - 8 + ((b & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    return max(-127, min(127, e));
+}
+
+__device__ __forceinline__ float exp2_neg(int e)   // 2^-e for e in [-127, 126]
+{
+    return __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+}
+
+// Thread = one block of 32 bf16 values: 64-byte load, 32-byte store.
+__global__ void __launch_bounds__(256) quantize_mxfp8_kernel(const __nv_bfloat16 *__restrict__ src,
+                                                             long long nblocks, uint8_t *__restrict__ q,
+                                                             uint8_t *__restrict__ scales)
+{
+    const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= nblocks) return;
+    const uint4 *p = reinterpret_cast<const uint4 *>(src + b * 32);
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 u = p[i];
+        v[8 * i + 0] = bf16_lo(u.x); v[8 * i + 1] = bf16_hi(u.x);
+        v[8 * i + 2] = bf16_lo(u.y); v[8 * i + 3] = bf16_hi(u.y);
+        v[8 * i + 4] = bf16_lo(u.z); v[8 * i + 5] = bf16_hi(u.z);
+        v[8 * i + 6] = bf16_lo(u.w); v[8 * i + 7] = bf16_hi(u.w);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int e = mx_exponent(amax);
+    const float s = exp2_neg(e);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(v[4 * i + j] * s, __NV_SATFINITE, __NV_E4M3);
+            word |= static_cast<uint32_t>(c) << (8 * j);
+        }
+        w[i] = word;
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(q + b * 32);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    scales[b] = static_cast<uint8_t>(e + 127);
+}
+
+}  // namespace mok

@@ -1,0 +1,71 @@
+"""Shared helpers of the tests: seeded cases, oracle set-up, tolerance checks."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from mixture_experts_layer_persistent_b200 import synth
+
+RTOL = 1e-2
+ATOL = 1e-2
+
+
+def bits_to_bf16(bits: np.ndarray, device="cpu") -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def oracle_layer(wl, params, x_bits, dy_bits=None, mx=False, pure=False, weights=None):
+    """Oracle layer of a workload; params are torch tensors (any device)."""
+    L = oracle.Layer(wl.T, wl.H, wl.E, wl.k, wl.I, S=wl.S, Is=wl.Is, score_fn=wl.score_fn,
+                     n_group=wl.n_group, topk_group=wl.topk_group, routed_scale=1.0, mx=mx,
+                     pure=pure)
+    f32 = lambda t: None if t is None else t.detach().float().cpu().numpy()
+    w = weights or {}
+    L.set(x=x_bits, Wr=f32(params["router_w"]), bias=f32(params.get("e_bias")),
+          lbias=f32(params.get("logit_bias")),
+          Wgu=w.get("Wgu", None) if "Wgu" in w else synth.bf16_bits(params["w_gate_up"]),
+          Wdn=w.get("Wdn", None) if "Wdn" in w else synth.bf16_bits(params["w_down"]),
+          Wgu_s=w.get("Wgu_s") if "Wgu_s" in w else (synth.bf16_bits(params["ws_gate_up"]) if wl.S else None),
+          Wdn_s=w.get("Wdn_s") if "Wdn_s" in w else (synth.bf16_bits(params["ws_down"]) if wl.S else None),
+          dy=dy_bits)
+    return L
+
+
+def make_case(wl, device="cpu", gen_device=None, mx=False):
+    """Seeded inputs of a workload with top-k margins >= 1e-3 (x rows resampled).
+
+    Returns dict: params (on `device`), x, dy (on `device`), x_bits, dy_bits,
+    oracle layer L, idx, w (oracle routing), resamples.
+    """
+    gd = gen_device or device
+    params = synth.draw_params(wl, gd)
+    x_bits = synth.bf16_bits(synth.draw_x(wl, gd))
+    dy_bits = synth.bf16_bits(synth.draw_dy(wl, gd)) if wl.backward else None
+    L = oracle_layer(wl, params, x_bits, dy_bits, mx=mx)
+    x_bits, idx, w, counts = oracle.margin_reject(
+        L, lambda a: synth.bf16_bits(synth.draw_x(wl, gd, attempt=a)))
+    params = {k: (v.to(device) if v is not None else None) for k, v in params.items()}
+    return {
+        "params": params,
+        "x": bits_to_bf16(x_bits, device),
+        "dy": bits_to_bf16(dy_bits, device) if dy_bits is not None else None,
+        "x_bits": x_bits, "dy_bits": dy_bits, "L": L, "idx": idx, "w": w, "resamples": counts,
+    }
+
+
+def assert_close(got, want, what, rtol=RTOL, atol=ATOL):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    err = np.abs(got - want)
+    bound = atol + rtol * np.abs(want)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())}/{bad.size} elements out of tolerance; worst at "
+                             f"{i}: got {got[i]!r} want {want[i]!r} (|err| {err[i]:.3g} > {bound[i]:.3g})")
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)

@@ -1,0 +1,57 @@
+"""The C-ABI library loads on a CPU-only host and exports every declared entry point."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_persistent_b200 import abi, build, make_cfg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "mok.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_library_builds_and_exports_every_symbol():
+    build.build()
+    lib = ctypes.CDLL(abi.LIB_PATH)
+    names = _declared()
+    assert "moe_fwd" in names and "moe_bwd" in names and len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_workspace_sizes_and_argument_checks():
+    c = make_cfg(4096, 7168, 256, 2048, 8, 1, 2048, 1, 8, 4)
+    ctx, fwd, bwd = abi.moe_workspace_size(c)
+    T, H, I, kk = 4096, 7168, 2048, 9
+    R = T * kk
+    # ctx holds at least g,u, h, w*h and the per-slot rows
+    assert ctx >= R * 2 * I * 2 + 2 * R * I * 2 + T * kk * H * 2
+    assert fwd >= R * I * 2 + T * kk * H * 2 and fwd < ctx
+    assert bwd >= R * 2 * I * 2 + T * kk * H * 2
+    bad = [make_cfg(64, 200, 8, 128, 2), make_cfg(64, 256, 8, 100, 2), make_cfg(64, 256, 8, 128, 9),
+           make_cfg(64, 256, 300, 128, 2), make_cfg(0, 256, 8, 128, 2),
+           make_cfg(64, 256, 8, 128, 2, score_fn=1, n_group=3, topk_group=1)]
+    for c in bad:
+        with pytest.raises(abi.MokError) as ei:
+            abi.moe_workspace_size(c)
+        assert ei.value.code == abi.MOK_ERR_INVALID
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_workspace_size(make_cfg(64, 256, 8, 128, 2, n_shared=1, I_shared=256))
+    assert ei.value.code == abi.MOK_ERR_UNSUPPORTED
+    assert abi.moe_strerror(abi.MOK_ERR_WORKSPACE).startswith("ctx or scratch")
+
+
+def test_calls_fail_loudly_without_a_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("needs a host without a usable GPU")
+    c = make_cfg(64, 256, 8, 128, 2)
+    p = abi.moe_params()
+    with pytest.raises(abi.MokError):
+        abi.moe_fwd(c, 16, p, 16, None, None, 0, 0, 16, 1 << 30, None)

@@ -1,0 +1,37 @@
+"""MXFP8 quantiser (1x32 ue8m0 scales, e4m3 codes) bit-exact against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from mixture_experts_layer_persistent_b200 import quantize_mxfp8
+from tests._support import bits_to_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _special_rows():
+    rows = np.zeros((6, 64), np.float32)
+    rows[1, :32] = 448.0 * 2.0 ** -3          # amax exactly 448 * 2^e
+    rows[1, 32:] = np.linspace(-57, 57, 32)   # just above 448 * 2^-3
+    rows[2, :] = 1e-30                        # tiny
+    rows[3, :] = np.linspace(-3e38, 3e38, 64)
+    rows[4, ::2] = 1.0
+    rows[4, 1::2] = -1.75
+    rows[5, :] = 2.0 ** -133                  # bf16 subnormal
+    return rows
+
+
+@pytest.mark.parametrize("shape", [(6, 64), (1000, 7168), (37, 2048)])
+def test_quantize_matches_oracle(shape):
+    g = torch.Generator().manual_seed(shape[0])
+    x = torch.randn(shape, generator=g) * torch.exp2(torch.randint(-20, 20, (shape[0], 1), generator=g).float())
+    if shape == (6, 64):
+        x = torch.from_numpy(_special_rows())
+    xb = x.to(torch.bfloat16)
+    bits = xb.view(torch.int16).numpy().view(np.uint16)
+    q, s = quantize_mxfp8(xb.cuda())
+    torch.cuda.synchronize()
+    oq, os_ = oracle.mx_quantize(bits)
+    assert np.array_equal(s.cpu().numpy(), os_)
+    assert np.array_equal(q.cpu().numpy(), oq)
