@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 MoE layer (libmok) -- one JSON line on rank 0.
+
+A step is one forward + backward pass of the DeepSeek-V3-shaped BF16 layer
+(T=4096, H=7168, E=256, top-8, I=2048, one shared expert, sigmoid + bias
+group-limited routing) over one batch of seeded synthetic tokens, through the
+C ABI (moe_fwd, moe_bwd).  Inputs are resident in HBM when the timed region
+starts; the 22.6 GB of expert weights exceed the 126 MB L2, so no flush is
+needed between steps.  With N GPUs (torchrun) every rank runs its own replica
+on its own tokens (the layer has no exchange step on one GPU's experts):
+value = tokens of all ranks / max-over-ranks time, scaling "weak".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl mok|reference]
+
+--impl reference times the fp64 CPU oracle on the host cores (rank 0 only) on
+a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s fwd MXFP8 & BF16, bwd BF16; % of tensor-core peak"
+FWD_PHASES = ["router", "dispatch", "gate_up_gemm", "down_gemm", "combine"]
+BWD_PHASES = ["slot_grad", "drouter_partial", "drouter_reduce", "down_dgrad_gemm", "down_wgrad_gemm",
+              "gate_up_dgrad_gemm", "gate_up_wgrad_gemm", "dx_sum"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="dsv3")
+    ap.add_argument("--impl", default="mok", choices=["mok", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16": d["bf16_tflops"],
+                "bf16_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class Clocks:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.path = tempfile.mktemp(prefix="clocks", suffix=".csv")
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ algorithmic counts
+def algorithmic(wl, counts):
+    """FLOPs and bytes of each GEMM phase (per launch) from the routing counts."""
+    T, H, I, E, S, k = wl.T, wl.H, wl.I, wl.E, wl.S, wl.k
+    R = T * (k + S)
+    groups = int((counts > 0).sum()) + S          # experts whose weights are streamed
+    wgu = groups * 2 * I * H * 2
+    wdn = groups * H * I * 2
+    G = E + S
+    out = {
+        "gate_up_gemm": (4 * H * I * R, wgu + T * H * 2 + R * I * 2 * 2 + R * 2 * I * 2),
+        "down_gemm": (2 * H * I * R, wdn + R * I * 2 + T * (k + S) * H * 2),
+        "down_dgrad_gemm": (2 * H * I * R, wdn + T * H * 2 + R * 2 * I * 2 * 2),
+        "down_wgrad_gemm": (2 * H * I * R, T * H * 2 + R * I * 2 + G * H * I * 2),
+        "gate_up_dgrad_gemm": (4 * H * I * R, wgu + R * 2 * I * 2 + T * (k + S) * H * 2),
+        "gate_up_wgrad_gemm": (4 * H * I * R, R * 2 * I * 2 + T * H * 2 + G * 2 * I * H * 2),
+    }
+    return out
+
+
+# ------------------------------------------------------------------ CPU oracle sample
+def oracle_sample(wl, params, x, dy, seconds, log=None):
+    """Time the fp64 oracle's forward + dx backward on a token sample of the workload."""
+    import numpy as np
+    import oracle
+    from mixture_experts_layer_persistent_b200 import synth
+    from tests._support import oracle_layer
+
+    L = oracle_layer(wl, params, synth.bf16_bits(x), synth.bf16_bits(dy))
+    idx, w, _ = L.route(tokens=np.arange(1))
+    t0 = time.perf_counter()
+    L.route(tokens=np.arange(1), into=(idx, w, np.zeros(wl.T)))
+    L.fwd(idx, w, tokens=[0])
+    L.bwd(idx, w, tokens=[0])
+    one = time.perf_counter() - t0
+    n = int(max(1, min(wl.T, seconds / max(one, 1e-6))))
+    toks = np.arange(n, dtype=np.int32)
+    t0 = time.perf_counter()
+    gap = np.zeros(wl.T)
+    L.route(tokens=toks, into=(idx, w, gap))
+    L.fwd(idx, w, tokens=toks)
+    L.bwd(idx, w, tokens=toks)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"routing + forward + dx backward of {n} of the {wl.T} tokens of the {wl.name} "
+                      f"workload (fp64 C oracle, OpenMP over tokens; weight gradients not in the sample)",
+            "seconds": dt}
+
+
+# ------------------------------------------------------------------ main
+def main():
+    args = parse()
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.impl == "reference":
+        if rank == 0:
+            reference_arm(args, world)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, synth, moe_trace_events
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    wl = synth.scaled(wl, seed=wl.seed + 1000 * rank)
+    params = synth.draw_params(wl, dev)
+    x = synth.draw_x(wl, dev)
+    dy = synth.draw_dy(wl, dev)
+    layer = MoELayer(cfg_for(wl), params, training=True, device=dev)
+    y = torch.empty_like(x)
+    grads = layer.new_grads()
+    routing = layer.new_routing()
+    layer.forward(x, y, routing=routing)
+    torch.cuda.synchronize()
+    counts = routing["counts"].cpu().numpy()
+
+    def step():
+        layer.forward(x, y)
+        layer.backward(x, dy, grads)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+
+    K = args.steps
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    fev = [[mk() for _ in range(abi.MOK_FWD_PHASES + 1)] for _ in range(K)]
+    bev = [[mk() for _ in range(abi.MOK_BWD_PHASES + 1)] for _ in range(K)]
+    start, end = mk(), mk()
+    uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    if not uuid.startswith("GPU-"):
+        uuid = "GPU-" + uuid
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = Clocks(uuid)
+    time.sleep(0.4)
+    start.record()
+    for i in range(K):
+        moe_trace_events([e.cuda_event for e in fev[i]], [e.cuda_event for e in bev[i]])
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    moe_trace_events(None, None)
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    t = torch.tensor([ms], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    status = layer.status()
+
+    phase = {}
+    for n_i, name in enumerate(FWD_PHASES):
+        phase[name] = statistics.mean(fev[i][n_i].elapsed_time(fev[i][n_i + 1]) for i in range(K))
+    for n_i, name in enumerate(BWD_PHASES):
+        phase[name] = statistics.mean(bev[i][n_i].elapsed_time(bev[i][n_i + 1]) for i in range(K))
+    fwd_ms = sum(phase[n] for n in FWD_PHASES)
+    bwd_ms = sum(phase[n] for n in BWD_PHASES)
+
+    pk = peaks()
+    alg = algorithmic(wl, counts)
+    dom = max(alg, key=lambda n: phase[n])
+    flops, nbytes = alg[dom]
+    t_dom = phase[dom] / 1e3
+    t_tc = flops / (pk["bf16_sustained"] * 1e12)
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    if t_hbm >= t_tc:
+        roof = {"bound": "hbm", "achieved": nbytes / t_dom / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": flops / t_dom / 1e12, "peak": pk["bf16_sustained"],
+                "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["peak_source"] = pk["source"] + (" sustained bf16" if roof["bound"] == "tensor" else " hbm copy")
+    roof["algorithmic_flops"] = flops
+    roof["algorithmic_bytes"] = nbytes
+
+    total_flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
+    tokens = wl.T * world
+    value = tokens * K / (ms_max / 1e3)
+    fwd_tps = wl.T / (fwd_ms / 1e3)
+    bwd_tps = wl.T / (bwd_ms / 1e3)
+
+    # ---------------- end to end through the host-buffer entry points
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_run(layer, wl, x, dy, grads, K, world, dist)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample(wl, {k2: v for k2, v in params.items()}, x, dy, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: DeepSeek-V3-shaped MoE layer fwd+bwd BF16, T={wl.T}, "
+                                   f"H={wl.H}, E={wl.E}, top-{wl.k}, I={wl.I}, {wl.S} shared expert, "
+                                   f"sigmoid+bias routing, {wl.n_group} groups / top-{wl.topk_group}",
+                       "tokens_per_gpu": wl.T, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (22.6 GB expert weights streamed per pass)"},
+            "gpu_launches": K * (len(FWD_PHASES) + len(BWD_PHASES)),
+            "clocks": clk, "device_status": status,
+            "phases_ms": {k2: round(v, 4) for k2, v in phase.items()},
+            "breakdown": {
+                "fwd_bf16_tokens_per_s": fwd_tps, "bwd_bf16_tokens_per_s": bwd_tps,
+                "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+                "fwd_tc_peak_frac_of_measured_burst": (6 * wl.H * wl.I * wl.T * (wl.k + wl.S) / (fwd_ms / 1e3))
+                / (pk["bf16"] * 1e12),
+                "bwd_tc_peak_frac_of_measured_burst": (12 * wl.H * wl.I * wl.T * (wl.k + wl.S) / (bwd_ms / 1e3))
+                / (pk["bf16"] * 1e12),
+                "step_tflops": 3 * total_flops / (ms_max / K / 1e3) / 1e12,
+                "expert_load_max_over_mean": float(counts.max() / counts.mean()),
+                "empty_experts": int((counts == 0).sum()),
+            },
+            "roofline": roof,
+            "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def e2e_run(layer, wl, x, dy, grads, K, world, dist):
+    import torch
+    from mixture_experts_layer_persistent_b200 import abi
+    c = layer.cfg
+    hx = x.cpu().pin_memory()
+    hdy = dy.cpu().pin_memory()
+    hy = torch.empty_like(hx).pin_memory()
+    hdx = torch.empty_like(hx).pin_memory()
+    n = max(abi.moe_host_scratch_size(c, False), abi.moe_host_scratch_size(c, True))
+    scratch = torch.empty(n, dtype=torch.uint8, device=x.device)
+    g = abi.moe_grads(None, grads["dw_gate_up"].data_ptr(), grads["dw_down"].data_ptr(),
+                      grads["drouter_w"].data_ptr(),
+                      grads["dws_gate_up"].data_ptr() if grads["dws_gate_up"] is not None else None,
+                      grads["dws_down"].data_ptr() if grads["dws_down"] is not None else None)
+    st = layer.stream()
+
+    def step():
+        abi.moe_fwd_host(c, hx.data_ptr(), layer.cparams, hy.data_ptr(), layer.ctx.data_ptr(),
+                         layer.ctx_bytes, 1, scratch.data_ptr(), n, st)
+        abi.moe_bwd_host(c, hx.data_ptr(), hdy.data_ptr(), layer.cparams, layer.ctx.data_ptr(),
+                         layer.ctx_bytes, hdx.data_ptr(), g, scratch.data_ptr(), n, st)
+
+    step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    t = torch.tensor([s.elapsed_time(e)], device=x.device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    nb = wl.T * wl.H * 2
+    return {"value": wl.T * world * K / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * nb,
+            "d2h_bytes_per_step": 2 * nb, "ms_per_step": ms / K,
+            "api": "moe_fwd_host + moe_bwd_host (pinned host x, dy -> y, dx)"}
+
+
+def reference_arm(args, world):
+    """The fp64 oracle on the host cores, bounded token sample per step."""
+    import torch
+    from mixture_experts_layer_persistent_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    gdev = "cuda" if torch.cuda.is_available() else "cpu"
+    params = synth.draw_params(wl, gdev)
+    x = synth.draw_x(wl, gdev)
+    dy = synth.draw_dy(wl, gdev)
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    res = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample(wl, params, x, dy, per_step)
+        if i >= args.warmup:
+            res.append(r)
+    value = statistics.mean(r["value"] for r in res)
+    ms = statistics.mean(r["seconds"] for r in res) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{wl.name} (oracle on a token sample)", "tokens_per_gpu": wl.T},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": res[0]["cores"], "kind": "oracle",
+                         "sample": res[0]["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

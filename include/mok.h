@@ -178,6 +178,24 @@ int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host,
 int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *scales,
                        void *stream);
 
+/*
+ * Phase tracing.  When events are set, every later moe_fwd (moe_bwd) records
+ * fwd_events[i] (bwd_events[i]) on its stream just before launching phase i
+ * and the last event after its final launch, so that elapsed times between
+ * consecutive events time each phase on the launching stream.  Events are
+ * cudaEvent_t handles owned by the caller.  Phases:
+ *   forward  (MOK_FWD_PHASES = 5, needs 6 events): router, dispatch,
+ *            gate/up GEMM, down GEMM, combine
+ *   backward (MOK_BWD_PHASES = 8, needs 9 events): slot gradient,
+ *            router-gradient partial sums, router-gradient reduction,
+ *            down dgrad GEMM, down wgrad GEMM, gate/up dgrad GEMM,
+ *            gate/up wgrad GEMM, dx sum
+ * Pass n = 0 to stop tracing.  The setting is per host thread.
+ */
+#define MOK_FWD_PHASES 5
+#define MOK_BWD_PHASES 8
+int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events, int n_bwd);
+
 /* Synchronise `stream`, then read and clear the device status word of the
  * current device (MOK_STATUS_* bits) into *device_status. */
 int moe_status(void *stream, int32_t *device_status);

@@ -25,6 +25,8 @@ MOK_SCORE_SOFTMAX = 0
 MOK_SCORE_SIGMOID = 1
 MOK_DTYPE_BF16 = 0
 MOK_DTYPE_MXFP8 = 1
+MOK_FWD_PHASES = 5
+MOK_BWD_PHASES = 8
 
 _i32, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -79,10 +81,12 @@ def lib():
                                    _vp, _sz, _vp]
         L.moe_quantize_mxfp8.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
         L.moe_status.argtypes = [_vp, P(_i32)]
+        L.moe_trace_events.argtypes = [P(_vp), ctypes.c_int, P(_vp), ctypes.c_int]
         L.moe_strerror.argtypes = [ctypes.c_int]
         L.moe_strerror.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
-                     "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_status"):
+                     "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_status",
+                     "moe_trace_events"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -147,3 +151,11 @@ def moe_status(stream) -> int:
     v = _i32()
     _check("moe_status", lib().moe_status(stream, ctypes.byref(v)))
     return v.value
+
+
+def moe_trace_events(fwd_events, bwd_events):
+    """fwd_events / bwd_events: lists of raw cudaEvent_t handles (ints), or None to stop."""
+    fa = (_vp * len(fwd_events))(*fwd_events) if fwd_events else None
+    ba = (_vp * len(bwd_events))(*bwd_events) if bwd_events else None
+    _check("moe_trace_events", lib().moe_trace_events(fa, len(fwd_events or ()), ba,
+                                                      len(bwd_events or ())))
