@@ -154,6 +154,8 @@ def oracle_sample(wl, params, x, dy, seconds, log=None):
 # ------------------------------------------------------------------ main
 def main():
     args = parse()
+    from mixture_experts_layer_persistent_b200 import build as _build
+    _build.build()          # no-op unless a source is newer than libmok.so
     import torch
     import torch.distributed as dist
 
