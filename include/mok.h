@@ -203,6 +203,11 @@ int moe_status(void *stream, int32_t *device_status);
 /* Static message for an error code. */
 const char *moe_strerror(int code);
 
+/* Description of the last failure of a call made by this host thread (which
+ * CUDA call failed and the CUDA error string); "" if none.  Valid until the
+ * thread's next failing call. */
+const char *moe_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -54,7 +54,8 @@ class moe_grads(ctypes.Structure):
 
 class MokError(RuntimeError):
     def __init__(self, fn, code):
-        super().__init__(f"{fn} failed: {moe_strerror(code)} ({code})")
+        detail = lib().moe_last_error().decode()
+        super().__init__(f"{fn} failed: {moe_strerror(code)} ({code})" + (f": {detail}" if detail else ""))
         self.code = code
 
 
@@ -84,6 +85,8 @@ def lib():
         L.moe_trace_events.argtypes = [P(_vp), ctypes.c_int, P(_vp), ctypes.c_int]
         L.moe_strerror.argtypes = [ctypes.c_int]
         L.moe_strerror.restype = ctypes.c_char_p
+        L.moe_last_error.argtypes = []
+        L.moe_last_error.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
                      "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_status",
                      "moe_trace_events"):

@@ -35,6 +35,19 @@ std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// per-thread description of the last failure (moe_last_error)
+thread_local char t_last_error[256] = "";
+
+int fail(int code, const char *what, cudaError_t e = cudaSuccess)
+{
+    if (e != cudaSuccess)
+        snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%s)", what, cudaGetErrorString(e),
+                 cudaGetErrorName(e));
+    else
+        snprintf(t_last_error, sizeof(t_last_error), "%s", what);
+    return code;
+}
+
 // per-thread phase tracing (moe_trace_events)
 thread_local cudaEvent_t t_fwd_ev[MOK_FWD_PHASES + 1];
 thread_local cudaEvent_t t_bwd_ev[MOK_BWD_PHASES + 1];
@@ -213,11 +226,12 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b
                 cudaStream_t st)
 {
     if (grid <= 0) return MOK_OK;
-    if (cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) !=
-        cudaSuccess)
-        return MOK_ERR_LAUNCH;
+    cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(grouped_gemm_kernel)", e);
     grouped_gemm_kernel<C><<<grid, 192, C::SMEM_BYTES, st>>>(a, b, bs, args);
-    return cudaGetLastError() == cudaSuccess ? MOK_OK : MOK_ERR_LAUNCH;
+    e = cudaGetLastError();
+    return e == cudaSuccess ? MOK_OK : fail(MOK_ERR_LAUNCH, "grouped_gemm_kernel launch", e);
 }
 
 inline int blocks_for(long long n, int per) { return static_cast<int>((n + per - 1) / per); }
@@ -228,9 +242,10 @@ inline int blocks_for(long long n, int per) { return static_cast<int>((n + per -
         if (rc_ != MOK_OK) return rc_; \
     } while (0)
 
-#define MOK_LAUNCHED()                                                     \
-    do {                                                                   \
-        if (cudaGetLastError() != cudaSuccess) return MOK_ERR_LAUNCH;       \
+#define MOK_LAUNCHED()                                                              \
+    do {                                                                            \
+        const cudaError_t e_ = cudaGetLastError();                                  \
+        if (e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "kernel launch", e_);    \
     } while (0)
 
 // ------------------------------------------------------------------ forward
@@ -315,12 +330,12 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
 
     if (routing) {
         const size_t tk = static_cast<size_t>(s.TK);
-        if (routing->topk_idx && cudaMemcpyAsync(routing->topk_idx, st.topk_idx, tk * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
-        if (routing->topk_w && cudaMemcpyAsync(routing->topk_w, st.topk_w, tk * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
-        if (routing->counts && cudaMemcpyAsync(routing->counts, st.counts, s.E * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
-        if (routing->offsets && cudaMemcpyAsync(routing->offsets, st.offsets, (s.E + 1) * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
-        if (routing->perm && cudaMemcpyAsync(routing->perm, st.perm, tk * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
-        if (routing->inv_perm && cudaMemcpyAsync(routing->inv_perm, st.inv_perm, tk * 4, cudaMemcpyDeviceToDevice, stream)) return MOK_ERR_LAUNCH;
+        if (routing->topk_idx) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->topk_idx, st.topk_idx, tk * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
+        if (routing->topk_w) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->topk_w, st.topk_w, tk * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
+        if (routing->counts) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->counts, st.counts, s.E * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
+        if (routing->offsets) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->offsets, st.offsets, (s.E + 1) * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
+        if (routing->perm) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->perm, st.perm, tk * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
+        if (routing->inv_perm) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->inv_perm, st.inv_perm, tk * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
     }
     return MOK_OK;
 }
@@ -515,11 +530,13 @@ int moe_fwd_host(const moe_cfg *cfg, const void *x_host, const moe_params *param
     char *s = static_cast<char *>(scratch);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t nb = static_cast<size_t>(cfg->T) * cfg->H * 2;
-    if (cudaMemcpyAsync(s, x_host, nb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOK_ERR_LAUNCH;
+    if (const cudaError_t e_ = cudaMemcpyAsync(s, x_host, nb, cudaMemcpyHostToDevice, st); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync", e_);
     MOK_TRY(moe_fwd(cfg, s, params, s + io, nullptr, ctx, ctx_bytes, save_for_backward, s + 2 * io,
                     scratch_bytes - 2 * io, stream));
-    if (cudaMemcpyAsync(y_host, s + io, nb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOK_ERR_LAUNCH;
-    return cudaStreamSynchronize(st) == cudaSuccess ? MOK_OK : MOK_ERR_LAUNCH;
+    if (const cudaError_t e_ = cudaMemcpyAsync(y_host, s + io, nb, cudaMemcpyDeviceToHost, st); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync", e_);
+    if (const cudaError_t e_ = cudaStreamSynchronize(st); e_ != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaStreamSynchronize", e_);
+    return MOK_OK;
 }
 
 int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, const moe_params *params,
@@ -535,13 +552,15 @@ int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, co
     char *s = static_cast<char *>(scratch);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t nb = static_cast<size_t>(cfg->T) * cfg->H * 2;
-    if (cudaMemcpyAsync(s, x_host, nb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOK_ERR_LAUNCH;
-    if (cudaMemcpyAsync(s + io, dy_host, nb, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOK_ERR_LAUNCH;
+    if (const cudaError_t e_ = cudaMemcpyAsync(s, x_host, nb, cudaMemcpyHostToDevice, st); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync", e_);
+    if (const cudaError_t e_ = cudaMemcpyAsync(s + io, dy_host, nb, cudaMemcpyHostToDevice, st); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync", e_);
     moe_grads g = *grads;
     g.dx = s + 2 * io;
     MOK_TRY(moe_bwd(cfg, s, s + io, params, ctx, ctx_bytes, &g, s + 3 * io, scratch_bytes - 3 * io, stream));
-    if (cudaMemcpyAsync(dx_host, s + 2 * io, nb, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOK_ERR_LAUNCH;
-    return cudaStreamSynchronize(st) == cudaSuccess ? MOK_OK : MOK_ERR_LAUNCH;
+    if (const cudaError_t e_ = cudaMemcpyAsync(dx_host, s + 2 * io, nb, cudaMemcpyDeviceToHost, st); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync", e_);
+    if (const cudaError_t e_ = cudaStreamSynchronize(st); e_ != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaStreamSynchronize", e_);
+    return MOK_OK;
 }
 
 int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *scales, void *stream)
@@ -553,7 +572,9 @@ int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *
     if (nb == 0) return MOK_OK;
     quantize_mxfp8_kernel<<<blocks_for(nb, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const __nv_bfloat16 *>(src), nb, static_cast<uint8_t *>(q), static_cast<uint8_t *>(scales));
-    return cudaGetLastError() == cudaSuccess ? MOK_OK : MOK_ERR_LAUNCH;
+    if (const cudaError_t e_ = cudaGetLastError(); e_ != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "quantize_mxfp8_kernel launch", e_);
+    return MOK_OK;
 }
 
 int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events, int n_bwd)
@@ -572,14 +593,16 @@ int moe_status(void *stream, int32_t *device_status)
 {
     if (!device_status) return MOK_ERR_INVALID;
     if (!device_info()) return MOK_ERR_DEVICE;
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOK_ERR_LAUNCH;
+    if (const cudaError_t e_ = cudaStreamSynchronize(static_cast<cudaStream_t>(stream)); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaStreamSynchronize", e_);
     int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MOK_ERR_LAUNCH;
+    if (const cudaError_t e_ = cudaMemcpyFromSymbol(&v, g_status, sizeof(int)); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyFromSymbol", e_);
     const int zero = 0;
-    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return MOK_ERR_LAUNCH;
+    if (const cudaError_t e_ = cudaMemcpyToSymbol(g_status, &zero, sizeof(int)); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyToSymbol", e_);
     *device_status = v;
     return MOK_OK;
 }
+
+const char *moe_last_error(void) { return t_last_error; }
 
 const char *moe_strerror(int code)
 {
