@@ -204,6 +204,9 @@ def main():
     fev = [[mk() for _ in range(abi.MOK_FWD_PHASES + 1)] for _ in range(K)]
     bev = [[mk() for _ in range(abi.MOK_BWD_PHASES + 1)] for _ in range(K)]
     start, end = mk(), mk()
+    for e in [e for ev in fev + bev for e in ev]:
+        e.record()              # torch creates the CUDA event on its first record
+    torch.cuda.synchronize()
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     if not uuid.startswith("GPU-"):
         uuid = "GPU-" + uuid

@@ -53,13 +53,17 @@ thread_local cudaEvent_t t_fwd_ev[MOK_FWD_PHASES + 1];
 thread_local cudaEvent_t t_bwd_ev[MOK_BWD_PHASES + 1];
 thread_local bool t_fwd_on = false, t_bwd_on = false;
 
-inline void mark_fwd(int i, cudaStream_t s)
+inline int mark_fwd(int i, cudaStream_t s)
 {
-    if (t_fwd_on) cudaEventRecord(t_fwd_ev[i], s);
+    if (!t_fwd_on) return MOK_OK;
+    const cudaError_t e = cudaEventRecord(t_fwd_ev[i], s);
+    return e == cudaSuccess ? MOK_OK : fail(MOK_ERR_LAUNCH, "cudaEventRecord(trace event)", e);
 }
-inline void mark_bwd(int i, cudaStream_t s)
+inline int mark_bwd(int i, cudaStream_t s)
 {
-    if (t_bwd_on) cudaEventRecord(t_bwd_ev[i], s);
+    if (!t_bwd_on) return MOK_OK;
+    const cudaError_t e = cudaEventRecord(t_bwd_ev[i], s);
+    return e == cudaSuccess ? MOK_OK : fail(MOK_ERR_LAUNCH, "cudaEventRecord(trace event)", e);
 }
 
 const DeviceInfo *device_info()
@@ -264,7 +268,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     ra.score_fn = c.score_fn; ra.n_group = c.n_group; ra.topk_group = c.topk_group;
     ra.routed_scale = c.routed_scale;
     ra.topk_idx = st.topk_idx; ra.topk_w = st.topk_w; ra.topk_p = st.topk_p;
-    mark_fwd(0, stream);
+    MOK_TRY(mark_fwd(0, stream));
     router_kernel<<<blocks_for(s.T, kRouteTokens), 256, 0, stream>>>(ra);
     MOK_LAUNCHED();
 
@@ -274,7 +278,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     da.counts = st.counts; da.offsets = st.offsets; da.gorder = st.gorder; da.chunk_start = st.chunk_start;
     da.perm = st.perm; da.inv_perm = st.inv_perm; da.row_token = st.row_token; da.row_slot = st.row_slot;
     da.row_w = st.row_w;
-    mark_fwd(1, stream);
+    MOK_TRY(mark_fwd(1, stream));
     dispatch_kernel<<<1, 1024, 0, stream>>>(da);
     MOK_LAUNCHED();
 
@@ -301,7 +305,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     ga.inter = c.I;
     ga.status = dev.status;
     using CGateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU>;
-    mark_fwd(2, stream);
+    MOK_TRY(mark_fwd(2, stream));
     MOK_TRY(launch_gemm<CGateUp>(tA, tB, tBs, ga, dev.sms, stream));
 
     // down: contiguous h rows, push epilogue into (token, slot) rows
@@ -318,15 +322,15 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     gd.out2 = gd.out3 = nullptr;
     gd.ldo = c.H;
     using CDown = GemmCfg<256, false, false, false, false, false, EPI_PUSH>;
-    mark_fwd(3, stream);
+    MOK_TRY(mark_fwd(3, stream));
     MOK_TRY(launch_gemm<CDown>(tA, tB, tBs, gd, dev.sms, stream));
 
-    mark_fwd(4, stream);
+    MOK_TRY(mark_fwd(4, stream));
     combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(st.O, st.topk_w,
                                                                        static_cast<__nv_bfloat16 *>(y), c.T, c.H,
                                                                        c.top_k, c.n_shared);
     MOK_LAUNCHED();
-    mark_fwd(5, stream);
+    MOK_TRY(mark_fwd(5, stream));
 
     if (routing) {
         const size_t tk = static_cast<size_t>(s.TK);
@@ -347,16 +351,16 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     const Shapes s = shapes(c);
     const __nv_bfloat16 *dyb = static_cast<const __nv_bfloat16 *>(dy);
 
-    mark_bwd(0, stream);
+    MOK_TRY(mark_bwd(0, stream));
     slot_grad_kernel<<<c.T, 256, 0, stream>>>(dyb, st.O, st.topk_w, st.topk_p, bs.dl, c.T, c.H, c.top_k,
                                               c.n_shared, c.score_fn, c.routed_scale);
     MOK_LAUNCHED();
-    mark_bwd(1, stream);
+    MOK_TRY(mark_bwd(1, stream));
     drouter_partial_kernel<<<dim3(static_cast<unsigned>(s.max_chunks), c.H / 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(x), bs.dl, st.offsets, st.chunk_start, st.perm, bs.partial, c.H, c.E,
         c.top_k, kChunkRows);
     MOK_LAUNCHED();
-    mark_bwd(2, stream);
+    MOK_TRY(mark_bwd(2, stream));
     drouter_reduce_kernel<<<blocks_for(s.E * s.H, 256), 256, 0, stream>>>(bs.partial, st.chunk_start,
                                                                           gr.drouter_w, c.H, c.E);
     MOK_LAUNCHED();
@@ -384,7 +388,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g1.aux = st.gu;
     g1.out = bs.dgu;
     using CDgradDown = GemmCfg<128, false, true, true, false, false, EPI_DSWIGLU>;
-    mark_bwd(3, stream);
+    MOK_TRY(mark_bwd(3, stream));
     MOK_TRY(launch_gemm<CDgradDown>(tA, tB, tBs, g1, dev.sms, stream));
 
     // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
@@ -398,7 +402,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g2.group_out_elems = s.H * s.I;
     using CWgradDown = GemmCfg<128, true, true, true, false, true, EPI_WGRAD>;
     const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
-    mark_bwd(4, stream);
+    MOK_TRY(mark_bwd(4, stream));
     MOK_TRY(launch_gemm<CWgradDown>(tA, tB, tB, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms), stream));
 
     // dgrad of gate/up: dX rows = dGU . W_gate_up, pushed into (token, slot) rows
@@ -413,7 +417,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g3.out = bs.dxs;
     g3.ldo = c.H;
     using CDgradGU = GemmCfg<256, false, true, false, false, false, EPI_PUSH>;
-    mark_bwd(5, stream);
+    MOK_TRY(mark_bwd(5, stream));
     MOK_TRY(launch_gemm<CDgradGU>(tA, tB, tBs, g3, dev.sms, stream));
 
     // wgrad of gate/up: dW_gate_up[g] = sum_r dGU_r^T x[token r]
@@ -428,15 +432,15 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g4.group_out_elems = 2 * s.I * s.H;
     using CWgradGU = GemmCfg<256, true, true, false, true, true, EPI_WGRAD>;
     const long long t4 = s.G * g4.m_tiles * g4.n_tiles;
-    mark_bwd(6, stream);
+    MOK_TRY(mark_bwd(6, stream));
     MOK_TRY(launch_gemm<CWgradGU>(tA, tB, tB, g4, static_cast<int>(t4 < dev.sms ? t4 : dev.sms), stream));
 
-    mark_bwd(7, stream);
+    MOK_TRY(mark_bwd(7, stream));
     dx_combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(
         bs.dxs, bs.dl, st.topk_idx, p.router_w, static_cast<__nv_bfloat16 *>(gr.dx), c.T, c.H, c.top_k,
         c.n_shared);
     MOK_LAUNCHED();
-    mark_bwd(8, stream);
+    MOK_TRY(mark_bwd(8, stream));
     return MOK_OK;
 }
 
@@ -582,6 +586,10 @@ int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events
     if (n_fwd < 0 || n_bwd < 0) return MOK_ERR_INVALID;
     if (n_fwd > 0 && (n_fwd < MOK_FWD_PHASES + 1 || !fwd_events)) return MOK_ERR_INVALID;
     if (n_bwd > 0 && (n_bwd < MOK_BWD_PHASES + 1 || !bwd_events)) return MOK_ERR_INVALID;
+    for (int i = 0; i < (n_fwd > 0 ? MOK_FWD_PHASES + 1 : 0); ++i)
+        if (!fwd_events[i]) return fail(MOK_ERR_INVALID, "moe_trace_events: NULL event handle");
+    for (int i = 0; i < (n_bwd > 0 ? MOK_BWD_PHASES + 1 : 0); ++i)
+        if (!bwd_events[i]) return fail(MOK_ERR_INVALID, "moe_trace_events: NULL event handle");
     t_fwd_on = n_fwd > 0;
     t_bwd_on = n_bwd > 0;
     for (int i = 0; t_fwd_on && i <= MOK_FWD_PHASES; ++i) t_fwd_ev[i] = static_cast<cudaEvent_t>(fwd_events[i]);
