@@ -1,11 +1,12 @@
 // gemm.cuh -- persistent, warp-specialised grouped GEMM on tcgen05/TMEM (sm_100a).
 //
-// One template serves every expert contraction of the layer.  A group is one
-// expert (routed experts first, then shared experts) and owns a contiguous
-// range of "sorted rows" (the expert-major order of (token, slot) pairs).
+// One template serves every contraction of the layer.  A group is one expert
+// (routed experts first, then shared experts) and owns a contiguous range of
+// "sorted rows" (the expert-major order of (token, slot) pairs).
 //
 //   ragged-M (forward, data gradients):  D[rows of g, N] = A[rows of g, K] . B_g[N, K]^T
 //   ragged-K (weight gradients):         D_g[M, N] = sum over rows r of g of A[r, M]^T B[r, N]
+//   router (one group of all tokens, split over K): partial logits of x . [Wr_hi|Wr_mid|Wr_lo]^T
 //
 // A rows that belong to a token are pulled by index straight from the token
 // matrix with TMA gather4 (the pull-at-dispatch idea of "Cursor åpner
@@ -19,9 +20,10 @@
 //
 // Roles (192 threads): warp 0 issues TMA loads into a STAGES-deep ring, warp 1
 // allocates TMEM and issues tcgen05.mma (one elected thread), warps 2-5 drain
-// the double-buffered TMEM accumulator and run the epilogue.  Every output
-// tile is produced by exactly one CTA with a fixed K order, so results do not
-// depend on scheduling: the layer is bit-reproducible.
+// the double-buffered TMEM accumulator and run the epilogue, staging each
+// 32-row block through shared memory so that global stores cover whole lines.
+// Every output tile is produced by exactly one CTA with a fixed K order, so
+// results do not depend on scheduling: the layer is bit-reproducible.
 #pragma once
 #include "ptx.cuh"
 
@@ -31,7 +33,7 @@ constexpr int BM = 128;        // UMMA M (cta_group::1, all 128 TMEM lanes)
 constexpr int BK = 64;         // one 128-byte swizzle row of bf16
 constexpr int kMaxGroups = 264;
 
-enum Epi : int { EPI_SWIGLU = 0, EPI_PUSH = 1, EPI_DSWIGLU = 2, EPI_WGRAD = 3 };
+enum Epi : int { EPI_SWIGLU = 0, EPI_PUSH = 1, EPI_DSWIGLU = 2, EPI_WGRAD = 3, EPI_ROUTER = 4 };
 
 struct GemmArgs {
     int num_groups;               // G
@@ -41,18 +43,21 @@ struct GemmArgs {
     const int *row_token;         // [R] gather row of each sorted row
     const int *row_slot;          // [R] destination row of each sorted row (push)
     const float *row_w;           // [R] routing weight of each sorted row
-    int n_tiles;                  // output tiles along N
+    int n_tiles;                  // output tiles along N (router: K splits)
     int m_tiles;                  // ragged-K: output tiles along M
-    int num_kb;                   // ragged-M: K / BK
+    int num_kb;                   // ragged-M: K / BK (router: K blocks per split)
     int b_rows_per_group;         // ragged-M: rows of one group in B's 2D view
     int b_half;                   // EPI_SWIGLU: row offset of the up projection inside a group
+    int a_k_mod;                  // EPI_ROUTER: A's K coordinate wraps at this many elements (H)
     __nv_bfloat16 *out;           // main output
     __nv_bfloat16 *out_s;         // EPI_WGRAD: output of the shared groups
     __nv_bfloat16 *out2;          // EPI_SWIGLU: saved gate/up pre-activations [R, 2I] (or null)
     __nv_bfloat16 *out3;          // EPI_SWIGLU: w * h [R, I] (or null)
+    float *out_f32;               // EPI_ROUTER: partial logits [n_tiles, rows, 256]
     const __nv_bfloat16 *aux;     // EPI_DSWIGLU: saved gate/up pre-activations [R, 2I]
     int ldo;                      // elements per output row
     int inter;                    // I
+    int rows_total;               // EPI_ROUTER: rows of one partial-logit slab (T)
     long long group_out_elems;    // EPI_WGRAD: elements of one group's output
     int *status;                  // device status word
 };
@@ -68,17 +73,20 @@ struct GemmCfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = BN == 256 ? 4 : 6;
     static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int STAGE_WORDS = 36;                       // padded u32 per staged row (32 + 4)
+    static constexpr int EPI_STAGE_BYTES = 4 * 32 * STAGE_WORDS * 4;
     static constexpr int AUX_BYTES = 256 + 3 * kMaxGroups * 4;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_STAGE_BYTES + AUX_BYTES;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
     static_assert(BN == 128 || BN == 256, "BN");
     static_assert(!RAGGED_K || (A_MN && B_MN), "weight gradients take both operands MN-major");
     static_assert(!RAGGED_K || (A_GATHER != B_GATHER), "one operand of a weight gradient is gathered");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 struct Tile {
     int g;          // group
-    int nt;         // N tile
+    int nt;         // N tile (router: K split)
     int m0;         // ragged-M: first sorted row; ragged-K: first M index
     int rows;       // ragged-M: valid rows in the tile
     int krow0;      // ragged-K: first sorted row of the group
@@ -123,27 +131,73 @@ __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const i
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
-__device__ __forceinline__ void store_bf16x16(__nv_bfloat16 *dst, const float (&v)[16])
+// Token rows of the four consecutive sorted rows r .. r+3 (rows at or past `end`
+// take row 0: their products are masked or multiplied by zeroed operand rows).
+__device__ __forceinline__ void gather_rows4(const int *row_token, int r, int end, int (&i)[4])
 {
-    uint4 lo, hi;
-    lo.x = pack_bf16x2(v[0], v[1]);   lo.y = pack_bf16x2(v[2], v[3]);
-    lo.z = pack_bf16x2(v[4], v[5]);   lo.w = pack_bf16x2(v[6], v[7]);
-    hi.x = pack_bf16x2(v[8], v[9]);   hi.y = pack_bf16x2(v[10], v[11]);
-    hi.z = pack_bf16x2(v[12], v[13]); hi.w = pack_bf16x2(v[14], v[15]);
-    reinterpret_cast<uint4 *>(dst)[0] = lo;
-    reinterpret_cast<uint4 *>(dst)[1] = hi;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) i[q] = r + q < end ? __ldg(row_token + r + q) : 0;
 }
 
-__device__ __forceinline__ void load_bf16x16(const __nv_bfloat16 *src, float (&v)[16])
+// Warp-cooperative store of a 32-row block: lane l supplies row l as W u32
+// words (W = 16 or 32) and that row's destination (null = skip the row).
+// The block goes through a padded per-warp staging buffer so that each store
+// instruction writes 32 / (W/4) whole rows of 4W contiguous bytes.
+template <int W>
+__device__ __forceinline__ void warp_store_rows(uint32_t *stage, const uint32_t (&p)[W], void *dst, int lane)
 {
-    const uint4 lo = reinterpret_cast<const uint4 *>(src)[0];
-    const uint4 hi = reinterpret_cast<const uint4 *>(src)[1];
-    const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+    constexpr int S = 36;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        v[2 * i] = bf16_lo(w[i]);
-        v[2 * i + 1] = bf16_hi(w[i]);
+    for (int i = 0; i < W; i += 4)
+        *reinterpret_cast<uint4 *>(stage + lane * S + i) = make_uint4(p[i], p[i + 1], p[i + 2], p[i + 3]);
+    __syncwarp();
+    constexpr int LPR = W / 4;        // lanes per row
+    constexpr int RPI = 32 / LPR;     // rows per store instruction
+    const uint64_t d = reinterpret_cast<uint64_t>(dst);
+#pragma unroll
+    for (int it = 0; it < 32 / RPI; ++it) {
+        const int row = it * RPI + lane / LPR, ch = lane % LPR;
+        const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d), row);
+        const uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d >> 32), row);
+        const uint4 v = *reinterpret_cast<const uint4 *>(stage + row * S + ch * 4);
+        const uint64_t rd = (static_cast<uint64_t>(hi) << 32) | lo;
+        if (rd) reinterpret_cast<uint4 *>(rd)[ch] = v;
     }
+    __syncwarp();
+}
+
+// Warp-cooperative load of a 32-row block (inverse of warp_store_rows): lane l
+// receives row l (W u32 words) read from `src` (null = zeros).
+template <int W>
+__device__ __forceinline__ void warp_load_rows(uint32_t *stage, uint32_t (&p)[W], const void *src, int lane)
+{
+    constexpr int S = 36;
+    constexpr int LPR = W / 4;
+    constexpr int RPI = 32 / LPR;
+    const uint64_t d = reinterpret_cast<uint64_t>(src);
+#pragma unroll
+    for (int it = 0; it < 32 / RPI; ++it) {
+        const int row = it * RPI + lane / LPR, ch = lane % LPR;
+        const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d), row);
+        const uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d >> 32), row);
+        const uint64_t rs = (static_cast<uint64_t>(hi) << 32) | lo;
+        const uint4 v = rs ? reinterpret_cast<const uint4 *>(rs)[ch] : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(stage + row * S + ch * 4) = v;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < W; i += 4) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(stage + lane * S + i);
+        p[i] = v.x; p[i + 1] = v.y; p[i + 2] = v.z; p[i + 3] = v.w;
+    }
+    __syncwarp();
+}
+
+template <int N>
+__device__ __forceinline__ void pack_bf16(const float *v, uint32_t (&p)[N / 2])
+{
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) p[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
 }
 
 template <class C>
@@ -154,7 +208,8 @@ __global__ void __launch_bounds__(192, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *tiles = smem;
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(tiles + C::STAGES * C::STAGE_BYTES);
+    uint32_t *epi_stage = reinterpret_cast<uint32_t *>(tiles + C::STAGES * C::STAGE_BYTES);
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(epi_stage) + C::EPI_STAGE_BYTES);
     uint64_t *empty_bar = full_bar + C::STAGES;
     uint64_t *accf = empty_bar + C::STAGES;
     uint64_t *acce = accf + 2;
@@ -225,6 +280,11 @@ __global__ void __launch_bounds__(192, 1)
             const bool routed = t.g < args.num_routed;
             const CUtensorMap *mB = routed ? &tmB : &tmB_s;
             const int gl = routed ? t.g : t.g - args.num_routed;
+            int ga[4] = {0, 0, 0, 0};       // gather rows of this lane (ragged-M: whole tile)
+            int gk[4] = {0, 0, 0, 0};       // gather rows of this lane for the current K block (ragged-K)
+            if constexpr (C::A_GATHER && !C::A_MN) gather_rows4(args.row_token, t.m0 + 4 * lane, t.m0 + t.rows, ga);
+            if constexpr (C::RAGGED_K)
+                if (t.nkb > 0) gather_rows4(args.row_token, t.krow0 + 4 * (lane & 15), t.krow0 + t.krows, gk);
             for (int kb = 0; kb < t.nkb; ++kb) {
                 bool ok = true;
                 if (lane == 0) {
@@ -236,24 +296,18 @@ __global__ void __launch_bounds__(192, 1)
                 uint8_t *sA = tiles + stage * C::STAGE_BYTES;
                 uint8_t *sB = sA + C::A_BYTES;
                 uint64_t *fb = &full_bar[stage];
+                const int kg = C::EPI == EPI_ROUTER ? t.nt * args.num_kb + kb : kb;   // global K block
                 // ---- A
                 if constexpr (C::A_GATHER && !C::A_MN) {
-                    const int r = t.m0 + 4 * lane, end = t.m0 + t.rows;
-                    const int i0 = r + 0 < end ? args.row_token[r + 0] : 0;
-                    const int i1 = r + 1 < end ? args.row_token[r + 1] : 0;
-                    const int i2 = r + 2 < end ? args.row_token[r + 2] : 0;
-                    const int i3 = r + 3 < end ? args.row_token[r + 3] : 0;
-                    tma_gather4(sA + lane * 512, &tmA, fb, kb * BK, i0, i1, i2, i3);
+                    tma_gather4(sA + lane * 512, &tmA, fb, kb * BK, ga[0], ga[1], ga[2], ga[3]);
                 } else if constexpr (!C::A_GATHER && !C::A_MN) {
-                    if (lane == 0) tma_load_2d(sA, &tmA, fb, kb * BK, t.m0);
+                    if (lane == 0) {
+                        const int kc = C::EPI == EPI_ROUTER ? (kg * BK) % args.a_k_mod : kb * BK;
+                        tma_load_2d(sA, &tmA, fb, kc, t.m0);
+                    }
                 } else if constexpr (C::A_GATHER && C::A_MN) {
                     const int chunk = lane >> 4, q = lane & 15;
-                    const int r = t.krow0 + kb * BK + 4 * q, end = t.krow0 + t.krows;
-                    const int i0 = r + 0 < end ? args.row_token[r + 0] : 0;
-                    const int i1 = r + 1 < end ? args.row_token[r + 1] : 0;
-                    const int i2 = r + 2 < end ? args.row_token[r + 2] : 0;
-                    const int i3 = r + 3 < end ? args.row_token[r + 3] : 0;
-                    tma_gather4(sA + chunk * 8192 + q * 512, &tmA, fb, t.m0 + chunk * 64, i0, i1, i2, i3);
+                    tma_gather4(sA + chunk * 8192 + q * 512, &tmA, fb, t.m0 + chunk * 64, gk[0], gk[1], gk[2], gk[3]);
                 } else {
                     if (lane < BM / 64) tma_load_2d(sA + lane * 8192, &tmA, fb, t.m0 + lane * 64, t.krow0 + kb * BK);
                 }
@@ -264,6 +318,8 @@ __global__ void __launch_bounds__(192, 1)
                             const int row = gl * args.b_rows_per_group + t.nt * 128;
                             tma_load_2d(sB, mB, fb, kb * BK, row);
                             tma_load_2d(sB + 128 * 128, mB, fb, kb * BK, row + args.b_half);
+                        } else if constexpr (C::EPI == EPI_ROUTER) {
+                            tma_load_2d(sB, mB, fb, kg * BK, 0);
                         } else {
                             tma_load_2d(sB, mB, fb, kb * BK, gl * args.b_rows_per_group + t.nt * C::BN);
                         }
@@ -279,15 +335,14 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
                     for (int op = lane; op < (C::BN / 64) * 16; op += 32) {
                         const int chunk = op >> 4, q = op & 15;
-                        const int r = t.krow0 + kb * BK + 4 * q, end = t.krow0 + t.krows;
-                        const int i0 = r + 0 < end ? args.row_token[r + 0] : 0;
-                        const int i1 = r + 1 < end ? args.row_token[r + 1] : 0;
-                        const int i2 = r + 2 < end ? args.row_token[r + 2] : 0;
-                        const int i3 = r + 3 < end ? args.row_token[r + 3] : 0;
-                        tma_gather4(sB + chunk * 8192 + q * 512, &tmB, fb, t.nt * C::BN + chunk * 64, i0, i1, i2,
-                                    i3);
+                        tma_gather4(sB + chunk * 8192 + q * 512, &tmB, fb, t.nt * C::BN + chunk * 64, gk[0], gk[1],
+                                    gk[2], gk[3]);
                     }
                 }
+                // next K block's gather rows, fetched while this block is in flight
+                if constexpr (C::RAGGED_K)
+                    if (kb + 1 < t.nkb)
+                        gather_rows4(args.row_token, t.krow0 + (kb + 1) * BK + 4 * (lane & 15), t.krow0 + t.krows, gk);
                 if (++stage == C::STAGES) {
                     stage = 0;
                     phase ^= 1u;
@@ -361,6 +416,7 @@ __global__ void __launch_bounds__(192, 1)
         // ------------------------------------------------------------ epilogue
         const int eq = warp & 3;                 // TMEM lane quarter this warp may access
         const int row = eq * 32 + lane;
+        uint32_t *stg = epi_stage + (warp - 2) * 32 * C::STAGE_WORDS;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -375,35 +431,55 @@ __global__ void __launch_bounds__(192, 1)
                 const int n0 = t.nt * 128;
                 const float w = (valid && args.out3) ? args.row_w[r] : 0.0f;
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 16) {
-                    float g[16], u[16], h[16];
-                    tmem_ld16(taddr + c, g);
-                    tmem_ld16(taddr + 128 + c, u);
+                for (int c = 0; c < 128; c += 32) {
+                    float g[32], u[32], h[32];
+                    uint32_t p[16];
+                    tmem_ld32(taddr + c, g);
+                    tmem_ld32(taddr + 128 + c, u);
                     tmem_ld_wait();
-                    if (valid) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) h[i] = silu_f(g[i]) * u[i];
-                        store_bf16x16(args.out + (size_t)r * I + n0 + c, h);
-                        if (args.out2) {
-                            store_bf16x16(args.out2 + (size_t)r * 2 * I + n0 + c, g);
-                            store_bf16x16(args.out2 + (size_t)r * 2 * I + I + n0 + c, u);
-                        }
-                        if (args.out3) {
+                    for (int i = 0; i < 32; ++i) h[i] = silu_f(g[i]) * u[i];
+                    pack_bf16<32>(h, p);
+                    warp_store_rows<16>(stg, p, valid ? args.out + (size_t)r * I + n0 + c : nullptr, lane);
+                    if (args.out2) {
+                        pack_bf16<32>(g, p);
+                        warp_store_rows<16>(stg, p, valid ? args.out2 + (size_t)r * 2 * I + n0 + c : nullptr, lane);
+                        pack_bf16<32>(u, p);
+                        warp_store_rows<16>(stg, p, valid ? args.out2 + (size_t)r * 2 * I + I + n0 + c : nullptr,
+                                            lane);
+                    }
+                    if (args.out3) {
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) h[i] = w * bf16_round(h[i]);
-                            store_bf16x16(args.out3 + (size_t)r * I + n0 + c, h);
-                        }
+                        for (int i = 0; i < 32; ++i) h[i] = w * bf16_round(h[i]);
+                        pack_bf16<32>(h, p);
+                        warp_store_rows<16>(stg, p, valid ? args.out3 + (size_t)r * I + n0 + c : nullptr, lane);
                     }
                 }
-            } else if constexpr (C::EPI == EPI_PUSH) {
-                const bool valid = row < t.rows;
-                const size_t drow = valid ? static_cast<size_t>(args.row_slot[t.m0 + row]) : 0;
+            } else if constexpr (C::EPI == EPI_PUSH || C::EPI == EPI_WGRAD) {
+                __nv_bfloat16 *dst = nullptr;
+                if constexpr (C::EPI == EPI_PUSH) {
+                    if (row < t.rows)
+                        dst = args.out + (size_t)args.row_slot[t.m0 + row] * args.ldo + t.nt * C::BN;
+                } else {
+                    const bool routed = t.g < args.num_routed;
+                    __nv_bfloat16 *base = routed ? args.out + (size_t)t.g * args.group_out_elems
+                                                 : args.out_s + (size_t)(t.g - args.num_routed) * args.group_out_elems;
+                    dst = base + (size_t)(t.m0 + row) * args.ldo + t.nt * C::BN;
+                }
 #pragma unroll 1
-                for (int c = 0; c < C::BN; c += 16) {
-                    float v[16];
-                    tmem_ld16(taddr + c, v);
-                    tmem_ld_wait();
-                    if (valid) store_bf16x16(args.out + drow * args.ldo + t.nt * C::BN + c, v);
+                for (int c = 0; c < C::BN; c += 64) {
+                    float v[64];
+                    uint32_t p[32];
+                    if (C::EPI == EPI_PUSH || t.nkb > 0) {
+                        tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
+                        tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                        tmem_ld_wait();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 64; ++i) v[i] = 0.0f;
+                    }
+                    pack_bf16<64>(v, p);
+                    warp_store_rows<32>(stg, p, dst ? dst + c : nullptr, lane);
                 }
             } else if constexpr (C::EPI == EPI_DSWIGLU) {
                 const int r = t.m0 + row;
@@ -411,41 +487,42 @@ __global__ void __launch_bounds__(192, 1)
                 const int I = args.inter;
                 const int n0 = t.nt * C::BN;
                 const float w = valid ? args.row_w[r] : 0.0f;
+                const __nv_bfloat16 *gsrc = valid ? args.aux + (size_t)r * 2 * I + n0 : nullptr;
+                __nv_bfloat16 *gdst = valid ? args.out + (size_t)r * 2 * I + n0 : nullptr;
 #pragma unroll 1
-                for (int c = 0; c < C::BN; c += 16) {
-                    float v[16], g[16], u[16], dg[16], du[16];
-                    tmem_ld16(taddr + c, v);
+                for (int c = 0; c < C::BN; c += 32) {
+                    float v[32], dg[32], du[32];
+                    uint32_t gp[16], up[16], p[16];
+                    tmem_ld32(taddr + c, v);
+                    warp_load_rows<16>(stg, gp, gsrc ? gsrc + c : nullptr, lane);
+                    warp_load_rows<16>(stg, up, gsrc ? gsrc + I + c : nullptr, lane);
                     tmem_ld_wait();
-                    if (valid) {
-                        load_bf16x16(args.aux + (size_t)r * 2 * I + n0 + c, g);
-                        load_bf16x16(args.aux + (size_t)r * 2 * I + I + n0 + c, u);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float dh = w * v[i];
-                            const float sg = 1.0f / (1.0f + expf(-g[i]));
-                            dg[i] = dh * u[i] * sg * (1.0f + g[i] * (1.0f - sg));
-                            du[i] = dh * g[i] * sg;
-                        }
-                        store_bf16x16(args.out + (size_t)r * 2 * I + n0 + c, dg);
-                        store_bf16x16(args.out + (size_t)r * 2 * I + I + n0 + c, du);
+                    for (int i = 0; i < 32; ++i) {
+                        const float gi = (i & 1) ? bf16_hi(gp[i >> 1]) : bf16_lo(gp[i >> 1]);
+                        const float ui = (i & 1) ? bf16_hi(up[i >> 1]) : bf16_lo(up[i >> 1]);
+                        const float dh = w * v[i];
+                        const float sg = 1.0f / (1.0f + expf(-gi));
+                        dg[i] = dh * ui * sg * (1.0f + gi * (1.0f - sg));
+                        du[i] = dh * gi * sg;
                     }
+                    pack_bf16<32>(dg, p);
+                    warp_store_rows<16>(stg, p, gdst ? gdst + c : nullptr, lane);
+                    pack_bf16<32>(du, p);
+                    warp_store_rows<16>(stg, p, gdst ? gdst + I + c : nullptr, lane);
                 }
-            } else {   // EPI_WGRAD
-                const bool routed = t.g < args.num_routed;
-                __nv_bfloat16 *base = routed ? args.out + (size_t)t.g * args.group_out_elems
-                                             : args.out_s + (size_t)(t.g - args.num_routed) * args.group_out_elems;
-                __nv_bfloat16 *dst = base + (size_t)(t.m0 + row) * args.ldo + t.nt * C::BN;
+            } else {   // EPI_ROUTER: fp32 partial logits of this K split
+                const int r = t.m0 + row;
+                float *dst = row < t.rows ? args.out_f32 + ((size_t)t.nt * args.rows_total + r) * 256 : nullptr;
 #pragma unroll 1
-                for (int c = 0; c < C::BN; c += 16) {
-                    float v[16];
-                    if (t.nkb > 0) {
-                        tmem_ld16(taddr + c, v);
-                        tmem_ld_wait();
-                    } else {
+                for (int c = 0; c < 256; c += 32) {
+                    float v[32];
+                    uint32_t p[32];
+                    tmem_ld32(taddr + c, v);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) v[i] = 0.0f;
-                    }
-                    store_bf16x16(dst + c, v);
+                    for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
+                    warp_store_rows<32>(stg, p, dst ? dst + c : nullptr, lane);
                 }
             }
             tc_fence_before();

@@ -127,7 +127,23 @@ struct Carver {
 struct Shapes {
     long long T, H, E, I, k, S, G, kk, R, TK;
     long long max_chunks;
+    int n_split;              // K splits of the router contraction
 };
+
+// Router contraction: one M tile per 128 tokens, K = 3H (three bf16 terms of
+// the fp32 router weights).  Split K so that about one wave of 148 SMs is busy;
+// the split count divides the number of K blocks.
+int router_splits(long long T, long long H)
+{
+    const long long m_tiles = (T + BM - 1) / BM;
+    const long long kb = 3 * H / BK;
+    long long target = 148 / m_tiles;
+    if (target > 8) target = 8;
+    int best = 1;
+    for (int d = 1; d <= target; ++d)
+        if (kb % d == 0) best = d;
+    return best;
+}
 
 Shapes shapes(const moe_cfg &c)
 {
@@ -138,13 +154,16 @@ Shapes shapes(const moe_cfg &c)
     s.TK = s.T * s.k;
     s.R = s.TK + s.S * s.T;
     s.max_chunks = (s.TK + kChunkRows - 1) / kChunkRows + s.E;
+    s.n_split = router_splits(s.T, s.H);
     return s;
 }
 
 // forward state: what the backward reads, plus what the forward needs anyway
 struct State {
     int *topk_idx, *counts, *offsets, *gorder, *chunk_start, *perm, *inv_perm, *row_token, *row_slot;
-    float *topk_w, *topk_p, *row_w;
+    int *all_rows;
+    float *topk_w, *topk_p, *row_w, *rpart;
+    __nv_bfloat16 *wr3;
     __nv_bfloat16 *gu, *h, *hw, *O;
     uint8_t *xq, *xs, *hq, *hs;     // MXFP8 operands
     size_t bytes;
@@ -168,6 +187,9 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
     st.row_token = cv.take<int>(s.R);
     st.row_slot = cv.take<int>(s.R);
     st.row_w = cv.take<float>(s.R);
+    st.all_rows = cv.take<int>(2);
+    st.wr3 = cv.take<__nv_bfloat16>(s.E * 3 * s.H);
+    st.rpart = cv.take<float>(static_cast<size_t>(s.n_split) * s.T * 256);
     st.gu = training ? cv.take<__nv_bfloat16>(s.R * 2 * s.I) : nullptr;
     st.hw = training ? cv.take<__nv_bfloat16>(s.R * s.I) : nullptr;
     if (mx) {
@@ -259,17 +281,38 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     const Shapes s = shapes(c);
     if (c.dtype != MOK_DTYPE_BF16) return MOK_ERR_UNSUPPORTED;
 
-    RouteArgs ra;
-    ra.x = static_cast<const __nv_bfloat16 *>(x);
-    ra.router_w = p.router_w;
-    ra.e_bias = p.e_bias;
-    ra.logit_bias = p.logit_bias;
-    ra.T = c.T; ra.H = c.H; ra.E = c.E; ra.k = c.top_k;
-    ra.score_fn = c.score_fn; ra.n_group = c.n_group; ra.topk_group = c.topk_group;
-    ra.routed_scale = c.routed_scale;
-    ra.topk_idx = st.topk_idx; ra.topk_w = st.topk_w; ra.topk_p = st.topk_p;
+    // router logits on the tensor cores: x . [Wr_hi | Wr_mid | Wr_lo]^T, split over K
     MOK_TRY(mark_fwd(0, stream));
-    router_kernel<<<blocks_for(s.T, kRouteTokens), 256, 0, stream>>>(ra);
+    router_split_kernel<<<blocks_for(s.E * s.H, 256), 256, 0, stream>>>(p.router_w, st.wr3, c.E, c.H, st.all_rows,
+                                                                         c.T);
+    MOK_LAUNCHED();
+    {
+        CUtensorMap rA, rB;
+        if (!make_tmap(&rA, x, s.H, s.T, BK, 128, 2)) return fail(MOK_ERR_INVALID, "tensor map (x)");
+        if (!make_tmap(&rB, st.wr3, 3 * s.H, s.E, BK, 256, 2)) return fail(MOK_ERR_INVALID, "tensor map (router)");
+        GemmArgs gr{};
+        gr.num_groups = 1;
+        gr.num_routed = 1;
+        gr.offsets = st.all_rows;
+        gr.n_tiles = s.n_split;
+        gr.num_kb = static_cast<int>(3 * s.H / BK / s.n_split);
+        gr.a_k_mod = c.H;
+        gr.out_f32 = st.rpart;
+        gr.rows_total = c.T;
+        gr.status = dev.status;
+        using CRouter = GemmCfg<256, false, false, false, false, false, EPI_ROUTER>;
+        MOK_TRY(launch_gemm<CRouter>(rA, rB, rB, gr, dev.sms, stream));
+    }
+    SelectArgs sa;
+    sa.partial = st.rpart;
+    sa.n_split = s.n_split;
+    sa.e_bias = p.e_bias;
+    sa.logit_bias = p.logit_bias;
+    sa.T = c.T; sa.E = c.E; sa.k = c.top_k;
+    sa.score_fn = c.score_fn; sa.n_group = c.n_group; sa.topk_group = c.topk_group;
+    sa.routed_scale = c.routed_scale;
+    sa.topk_idx = st.topk_idx; sa.topk_w = st.topk_w; sa.topk_p = st.topk_p;
+    router_select_kernel<<<blocks_for(s.T, 8), 256, 0, stream>>>(sa);
     MOK_LAUNCHED();
 
     DispatchArgs da;

@@ -1,4 +1,4 @@
-// route.cuh -- router logits, scoring and top-k selection, and the
+// route.cuh -- router weight split, scoring and top-k selection, and the
 // deterministic counting sort that turns the selection into per-expert row
 // ranges (counts, prefix offsets, stable permutation, row maps).
 //
@@ -14,22 +14,46 @@
 
 namespace mok {
 
-struct RouteArgs {
-    const __nv_bfloat16 *x;     // [T, H]
-    const float *router_w;      // [E, H]
+// Router weights as three bf16 terms: Wr = hi + mid + lo to within 2^-25
+// relative, laid out [E, 3H] = [hi | mid | lo] along K, so that the tensor-core
+// contraction of x (bf16, exact) with the three terms reproduces the fp32
+// router logits.  Each difference below is exact in fp32.
+// It also writes the one-group row range {0, T} the router contraction reads.
+__global__ void __launch_bounds__(256) router_split_kernel(const float *__restrict__ Wr,
+                                                           __nv_bfloat16 *__restrict__ Wr3, int E, int H,
+                                                           int *__restrict__ all_rows, int T)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i == 0) {
+        all_rows[0] = 0;
+        all_rows[1] = T;
+    }
+    if (i >= (long long)E * H) return;
+    const int e = (int)(i / H), h = (int)(i % H);
+    const float w = Wr[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+    __nv_bfloat16 *row = Wr3 + (size_t)e * 3 * H;
+    row[h] = hi;
+    row[H + h] = mid;
+    row[2 * H + h] = lo;
+}
+
+struct SelectArgs {
+    const float *partial;       // [n_split, T, 256] partial logits (tensor-core K splits)
+    int n_split;
     const float *e_bias;        // [E] or null
     const float *logit_bias;    // [E] or null
-    int T, H, E, k;
+    int T, E, k;
     int score_fn, n_group, topk_group;
     float routed_scale;
     int *topk_idx;              // [T, k]
     float *topk_w;              // [T, k]
     float *topk_p;              // [T, k] sigmoid score s (sigmoid) or w / routed_scale (softmax)
 };
-
-constexpr int kRouteTokens = 32;   // tokens per block
-constexpr int kRouteHC = 32;       // H chunk staged in shared memory
-constexpr int kRoutePad = 36;      // padded row stride (floats)
 
 // one (value, index) candidate; larger value wins, then lower index
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib)
@@ -50,182 +74,110 @@ __device__ __forceinline__ void warp_argmax(float &v, int &i)
     }
 }
 
-// Block: 256 threads, 32 tokens.  Thread (eg = tid % 64, tg = tid / 64) owns
-// experts eg + 64 i (i < 4) and tokens 8 tg .. 8 tg + 7: 32 fp32 dot products
-// over H, each accumulated in ascending h.
-__global__ void __launch_bounds__(256) router_kernel(const RouteArgs a)
+// One warp per token.  Lane l holds experts l + 32 i.  The logit is the sum of
+// the K-split partials in split order plus logit_bias; selection as above.
+__global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a)
 {
-    __shared__ __align__(16) float s_w[256 * kRoutePad];              // router rows chunk, later logits
-    __shared__ __align__(16) float s_x[kRouteTokens * kRoutePad];
-    const int tid = threadIdx.x;
-    const int t0 = blockIdx.x * kRouteTokens;
-    const int eg = tid & 63, tg = tid >> 6;
-    const int E = a.E, H = a.H;
-    float acc[4][8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-
-    for (int h0 = 0; h0 < H; h0 += kRouteHC) {
-        // stage router rows [E, 32] and x rows [32, 32] (as fp32)
-        for (int q = tid; q < E * (kRouteHC / 4); q += 256) {
-            const int e = q / (kRouteHC / 4), c4 = q % (kRouteHC / 4);
-            const float4 v = *reinterpret_cast<const float4 *>(a.router_w + (size_t)e * H + h0 + c4 * 4);
-            *reinterpret_cast<float4 *>(&s_w[e * kRoutePad + c4 * 4]) = v;
-        }
-        for (int q = tid; q < kRouteTokens * (kRouteHC / 8); q += 256) {
-            const int tt = q / (kRouteHC / 8), c8 = q % (kRouteHC / 8);
-            const int t = t0 + tt;
-            float v[8];
-            if (t < a.T) {
-                const uint4 u = *reinterpret_cast<const uint4 *>(a.x + (size_t)t * H + h0 + c8 * 8);
-                v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
-                v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) s_x[tt * kRoutePad + c8 * 8 + i] = v[i];
-        }
-        __syncthreads();
-#pragma unroll
-        for (int hh = 0; hh < kRouteHC; hh += 4) {
-            float4 xv[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) xv[j] = *reinterpret_cast<const float4 *>(&s_x[(tg * 8 + j) * kRoutePad + hh]);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int e = eg + 64 * i;
-                if (e < E) {
-                    const float4 wv = *reinterpret_cast<const float4 *>(&s_w[e * kRoutePad + hh]);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        float s = acc[i][j];
-                        s = fmaf(xv[j].x, wv.x, s);
-                        s = fmaf(xv[j].y, wv.y, s);
-                        s = fmaf(xv[j].z, wv.z, s);
-                        s = fmaf(xv[j].w, wv.w, s);
-                        acc[i][j] = s;
-                    }
-                }
-            }
-        }
-        __syncthreads();
-    }
-    // logits to shared memory: s_w[tt * 257 + e]
-    float *s_lg = s_w;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int e = eg + 64 * i;
-        if (e < E) {
-            const float lb = a.logit_bias ? a.logit_bias[e] : 0.0f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) s_lg[(tg * 8 + j) * 257 + e] = acc[i][j] + lb;
-        }
-    }
-    __syncthreads();
-
-    // selection: warp w handles tokens w, w + 8, w + 16, w + 24
-    const int warp = tid >> 5, lane = tid & 31;
+    __shared__ float s_row[8][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= a.T) return;
+    const int E = a.E;
     const int npl = (E + 31) / 32;
-    for (int tt = warp; tt < kRouteTokens; tt += 8) {
-        const int t = t0 + tt;
-        if (t >= a.T) break;
-        float *lg = s_lg + tt * 257;
-        float sel[8], sc[8];
+    float *row = s_row[warp];
+    float lgv[8], sel[8], sc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        lgv[i] = 0.0f;
+        sel[i] = -INFINITY;
+        sc[i] = 0.0f;
+        if (i < npl && e < E) {
+            float lg = 0.0f;
+            for (int s = 0; s < a.n_split; ++s) lg += a.partial[((size_t)s * a.T + t) * 256 + e];
+            if (a.logit_bias) lg += a.logit_bias[e];
+            lgv[i] = lg;
+            if (a.score_fn == 0) {
+                sel[i] = lg;
+            } else {
+                const float sg = 1.0f / (1.0f + expf(-lg));
+                sc[i] = sg;
+                sel[i] = sg + (a.e_bias ? a.e_bias[e] : 0.0f);
+            }
+        }
+    }
+    if (a.n_group > 1 && a.topk_group < a.n_group) {
+        // group score: sum of the two best selection scores of the group
+        const int gs = E / a.n_group;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int e = lane + 32 * i;
-            sel[i] = -INFINITY;
-            sc[i] = 0.0f;
-            if (i < npl && e < E) {
-                if (a.score_fn == 0) {
-                    sel[i] = lg[e];
-                } else {
-                    const float s = 1.0f / (1.0f + expf(-lg[e]));
-                    sc[i] = s;
-                    sel[i] = s + (a.e_bias ? a.e_bias[e] : 0.0f);
-                }
+            if (i < npl && e < E) row[e] = sel[i];
+        }
+        __syncwarp();
+        float gsc = -INFINITY;
+        if (lane < a.n_group) {
+            float b1 = -INFINITY, b2 = -INFINITY;
+            for (int m = 0; m < gs; ++m) {
+                const float v = row[lane * gs + m];
+                if (v > b1) { b2 = b1; b1 = v; }
+                else if (v > b2) { b2 = v; }
+            }
+            gsc = gs > 1 ? b1 + b2 : b1;
+        }
+        unsigned keep = 0;   // bit g set: group g kept
+        for (int r = 0; r < a.topk_group; ++r) {
+            float v = lane < a.n_group ? gsc : -INFINITY;
+            int gi = lane < a.n_group ? lane : 1 << 30;
+            if (keep & (1u << (lane & 31))) v = -INFINITY;
+            warp_argmax(v, gi);
+            keep |= 1u << gi;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            if (i < npl && e < E && !(keep & (1u << (e / gs)))) sel[i] = -INFINITY;
+        }
+    }
+    // top-k by repeated warp argmax
+    int my_idx[16];
+    float my_val[16];
+    for (int j = 0; j < a.k; ++j) {
+        float bv = -INFINITY;
+        int bi = 1 << 30;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int e = lane + 32 * i;
+            if (i < npl && e < E && better(sel[i], e, bv, bi)) {
+                bv = sel[i];
+                bi = e;
             }
         }
-        if (a.n_group > 1 && a.topk_group < a.n_group) {
-            // group score: sum of the two best selection scores of the group
-            const int gs = E / a.n_group;
-            __syncwarp();
+        warp_argmax(bv, bi);
+        my_idx[j] = bi;
+        float wv = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int e = lane + 32 * i;
-                if (i < npl && e < E) lg[e] = sel[i];   // reuse the logit row for selection scores
+        for (int i = 0; i < 8; ++i)
+            if (lane + 32 * i == bi) {
+                sel[i] = -INFINITY;                                   // the owner retires the winner
+                wv = a.score_fn == 0 ? lgv[i] : sc[i];               // logit (softmax) or sigmoid score
             }
-            __syncwarp();
-            float gsc = -INFINITY;
-            if (lane < a.n_group) {
-                float b1 = -INFINITY, b2 = -INFINITY;
-                for (int m = 0; m < gs; ++m) {
-                    const float v = lg[lane * gs + m];
-                    if (v > b1) { b2 = b1; b1 = v; }
-                    else if (v > b2) { b2 = v; }
-                }
-                gsc = gs > 1 ? b1 + b2 : b1;
-            }
-            unsigned keep = 0;   // bit g set: group g kept
-            for (int r = 0; r < a.topk_group; ++r) {
-                float v = lane < a.n_group ? gsc : -INFINITY;
-                int gi = lane < a.n_group ? lane : 1 << 30;
-                if (keep & (1u << (lane & 31))) v = -INFINITY;
-                warp_argmax(v, gi);
-                keep |= 1u << gi;
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int e = lane + 32 * i;
-                if (i < npl && e < E && !(keep & (1u << (e / gs)))) sel[i] = -INFINITY;
-            }
+        my_val[j] = __shfl_sync(0xffffffffu, wv, bi & 31);
+    }
+    if (lane == 0) {
+        float wsum = 0.0f;
+        float p[16];
+        if (a.score_fn == 0) {
+            const float m = my_val[0];
+            for (int j = 0; j < a.k; ++j) { p[j] = expf(my_val[j] - m); wsum += p[j]; }
+        } else {
+            for (int j = 0; j < a.k; ++j) { p[j] = my_val[j]; wsum += p[j]; }
         }
-        // top-k by repeated warp argmax
-        int my_idx[16];
-        float my_val[16];
         for (int j = 0; j < a.k; ++j) {
-            float bv = -INFINITY;
-            int bi = 1 << 30;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int e = lane + 32 * i;
-                if (i < npl && e < E && better(sel[i], e, bv, bi)) {
-                    bv = sel[i];
-                    bi = e;
-                }
-            }
-            warp_argmax(bv, bi);
-            my_idx[j] = bi;
-            // owner retires the winner
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (lane + 32 * i == bi) sel[i] = -INFINITY;
-            // the winner's weight ingredient: logit (softmax) or sigmoid score
-            float wv = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (lane + 32 * i == bi) wv = a.score_fn == 0 ? s_lg[tt * 257 + bi] : sc[i];
-            my_val[j] = __shfl_sync(0xffffffffu, wv, bi & 31);
-        }
-        if (lane == 0) {
-            float wsum = 0.0f;
-            float p[16];
-            if (a.score_fn == 0) {
-                const float m = my_val[0];
-                for (int j = 0; j < a.k; ++j) { p[j] = expf(my_val[j] - m); wsum += p[j]; }
-            } else {
-                for (int j = 0; j < a.k; ++j) { p[j] = my_val[j]; wsum += p[j]; }
-            }
-            for (int j = 0; j < a.k; ++j) {
-                const float q = p[j] / wsum;
-                a.topk_idx[(size_t)t * a.k + j] = my_idx[j];
-                a.topk_w[(size_t)t * a.k + j] = a.routed_scale * q;
-                a.topk_p[(size_t)t * a.k + j] = a.score_fn == 0 ? q : my_val[j];
-            }
+            const float q = p[j] / wsum;
+            a.topk_idx[(size_t)t * a.k + j] = my_idx[j];
+            a.topk_w[(size_t)t * a.k + j] = a.routed_scale * q;
+            a.topk_p[(size_t)t * a.k + j] = a.score_fn == 0 ? q : my_val[j];
         }
     }
 }
