@@ -8,8 +8,9 @@
 //   ragged-K (weight gradients):         D_g[M, N] = sum over rows r of g of A[r, M]^T B[r, N]
 //   router (one group of all tokens, split over K): partial logits of x . [Wr_hi|Wr_mid|Wr_lo]^T
 //
-// A rows that belong to a token are pulled by index straight from the token
-// matrix with TMA gather4 (the pull-at-dispatch idea of "Cursor åpner
+// Operand rows that belong to a token are pulled by index straight from the
+// token matrix into the shared-memory ring by four pull warps issuing 16-byte
+// cp.async copies (the pull-at-dispatch idea of "Cursor åpner
 // megakernelen…", paragraph on pulling versus pushing tokens, re-derived for
 // one GPU: the expert tile fetches its rows instead of a separate scatter
 // pass).  The push epilogue writes each output row to its (token, slot) row
@@ -18,10 +19,13 @@
 // fixed-size macrobatch ring of "Megakernels are dead and back…", section
 // "Números de MoK").
 //
-// Roles (192 threads): warp 0 issues TMA loads into a STAGES-deep ring, warp 1
-// allocates TMEM and issues tcgen05.mma (one elected thread), warps 2-5 drain
-// the double-buffered TMEM accumulator and run the epilogue, staging each
-// 32-row block through shared memory so that global stores cover whole lines.
+// Roles: warp 0 issues TMA loads of the contiguous operands into a
+// STAGES-deep ring, warp 1 allocates TMEM and issues tcgen05.mma (one elected
+// thread), warps 2-5 drain the double-buffered TMEM accumulator and run the
+// epilogue, staging each 32-row block through shared memory so that global
+// stores cover whole lines, and warps 6-9 (kernels with a gathered operand)
+// pull the gathered rows.  TMA gather4 would also serve, but at four 128-byte
+// rows per instruction it issues too slowly to keep the tensor core fed.
 // Every output tile is produced by exactly one CTA with a fixed K order, so
 // results do not depend on scheduling: the layer is bit-reproducible.
 #pragma once
@@ -49,6 +53,8 @@ struct GemmArgs {
     int b_rows_per_group;         // ragged-M: rows of one group in B's 2D view
     int b_half;                   // EPI_SWIGLU: row offset of the up projection inside a group
     int a_k_mod;                  // EPI_ROUTER: A's K coordinate wraps at this many elements (H)
+    const __nv_bfloat16 *gather_src; // token matrix the pull warps gather rows from (x or dy)
+    int gather_ld;                // elements per token row of gather_src
     __nv_bfloat16 *out;           // main output
     __nv_bfloat16 *out_s;         // EPI_WGRAD: output of the shared groups
     __nv_bfloat16 *out2;          // EPI_SWIGLU: saved gate/up pre-activations [R, 2I] (or null)
@@ -72,6 +78,10 @@ struct GemmCfg {
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = BN == 256 ? 4 : 6;
+    static constexpr int PULL_WARPS = (A_GATHER || B_GATHER) ? 4 : 0;   // cp.async gather warps
+    static constexpr int THREADS = 192 + 32 * PULL_WARPS;
+    static constexpr int GATHER_BYTES = A_GATHER ? A_BYTES : (B_GATHER ? B_BYTES : 0);
+    static constexpr int TMA_BYTES = STAGE_BYTES - GATHER_BYTES;
     static constexpr int TMEM_COLS = 2 * BN;
     static constexpr int STAGE_WORDS = 36;                       // padded u32 per staged row (32 + 4)
     static constexpr int EPI_STAGE_BYTES = 4 * 32 * STAGE_WORDS * 4;
@@ -130,14 +140,6 @@ __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const i
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
-
-// Token rows of the four consecutive sorted rows r .. r+3 (rows at or past `end`
-// take row 0: their products are masked or multiplied by zeroed operand rows).
-__device__ __forceinline__ void gather_rows4(const int *row_token, int r, int end, int (&i)[4])
-{
-#pragma unroll
-    for (int q = 0; q < 4; ++q) i[q] = r + q < end ? __ldg(row_token + r + q) : 0;
-}
 
 // Warp-cooperative store of a 32-row block: lane l supplies row l as W u32
 // words (W = 16 or 32) and that row's destination (null = skip the row).
@@ -201,7 +203,7 @@ __device__ __forceinline__ void pack_bf16(const float *v, uint32_t (&p)[N / 2])
 }
 
 template <class C>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(C::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmB_s, const GemmArgs args)
 {
@@ -249,7 +251,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (lane == 0) {
             for (int s = 0; s < C::STAGES; ++s) {
-                mbar_init(&full_bar[s], 1);
+                mbar_init(&full_bar[s], 1 + 32 * C::PULL_WARPS);
                 mbar_init(&empty_bar[s], 1);
             }
             for (int b = 0; b < 2; ++b) {
@@ -280,16 +282,11 @@ __global__ void __launch_bounds__(192, 1)
             const bool routed = t.g < args.num_routed;
             const CUtensorMap *mB = routed ? &tmB : &tmB_s;
             const int gl = routed ? t.g : t.g - args.num_routed;
-            int ga[4] = {0, 0, 0, 0};       // gather rows of this lane (ragged-M: whole tile)
-            int gk[4] = {0, 0, 0, 0};       // gather rows of this lane for the current K block (ragged-K)
-            if constexpr (C::A_GATHER && !C::A_MN) gather_rows4(args.row_token, t.m0 + 4 * lane, t.m0 + t.rows, ga);
-            if constexpr (C::RAGGED_K)
-                if (t.nkb > 0) gather_rows4(args.row_token, t.krow0 + 4 * (lane & 15), t.krow0 + t.krows, gk);
             for (int kb = 0; kb < t.nkb; ++kb) {
                 bool ok = true;
                 if (lane == 0) {
                     ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status);
-                    if (ok) mbar_arrive_expect_tx(&full_bar[stage], C::STAGE_BYTES);
+                    if (ok) mbar_arrive_expect_tx(&full_bar[stage], C::TMA_BYTES);
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) goto producer_done;
@@ -297,18 +294,13 @@ __global__ void __launch_bounds__(192, 1)
                 uint8_t *sB = sA + C::A_BYTES;
                 uint64_t *fb = &full_bar[stage];
                 const int kg = C::EPI == EPI_ROUTER ? t.nt * args.num_kb + kb : kb;   // global K block
-                // ---- A
-                if constexpr (C::A_GATHER && !C::A_MN) {
-                    tma_gather4(sA + lane * 512, &tmA, fb, kb * BK, ga[0], ga[1], ga[2], ga[3]);
-                } else if constexpr (!C::A_GATHER && !C::A_MN) {
+                // ---- A (gathered A rows come from the pull warps)
+                if constexpr (!C::A_GATHER && !C::A_MN) {
                     if (lane == 0) {
                         const int kc = C::EPI == EPI_ROUTER ? (kg * BK) % args.a_k_mod : kb * BK;
                         tma_load_2d(sA, &tmA, fb, kc, t.m0);
                     }
-                } else if constexpr (C::A_GATHER && C::A_MN) {
-                    const int chunk = lane >> 4, q = lane & 15;
-                    tma_gather4(sA + chunk * 8192 + q * 512, &tmA, fb, t.m0 + chunk * 64, gk[0], gk[1], gk[2], gk[3]);
-                } else {
+                } else if constexpr (!C::A_GATHER && C::A_MN) {
                     if (lane < BM / 64) tma_load_2d(sA + lane * 8192, &tmA, fb, t.m0 + lane * 64, t.krow0 + kb * BK);
                 }
                 // ---- B
@@ -331,18 +323,7 @@ __global__ void __launch_bounds__(192, 1)
                 } else if constexpr (!C::B_GATHER && C::RAGGED_K) {
                     if (lane < C::BN / 64)
                         tma_load_2d(sB + lane * 8192, &tmB, fb, t.nt * C::BN + lane * 64, t.krow0 + kb * BK);
-                } else {
-#pragma unroll
-                    for (int op = lane; op < (C::BN / 64) * 16; op += 32) {
-                        const int chunk = op >> 4, q = op & 15;
-                        tma_gather4(sB + chunk * 8192 + q * 512, &tmB, fb, t.nt * C::BN + chunk * 64, gk[0], gk[1],
-                                    gk[2], gk[3]);
-                    }
                 }
-                // next K block's gather rows, fetched while this block is in flight
-                if constexpr (C::RAGGED_K)
-                    if (kb + 1 < t.nkb)
-                        gather_rows4(args.row_token, t.krow0 + (kb + 1) * BK + 4 * (lane & 15), t.krow0 + t.krows, gk);
                 if (++stage == C::STAGES) {
                     stage = 0;
                     phase ^= 1u;
@@ -350,6 +331,83 @@ __global__ void __launch_bounds__(192, 1)
             }
         }
     producer_done:;
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ pull warps
+        // Gathered operand: each 128-byte row is copied by index from the token
+        // matrix with 16-byte cp.async into the 128-byte-swizzled layout the MMA
+        // descriptors expect (16-byte chunk c of row r lands at chunk c ^ (r & 7)).
+        if constexpr (C::PULL_WARPS > 0) {
+            const int p = threadIdx.x - 192;
+            const int c16 = p & 7;
+            const int r0 = p >> 3;                      // 0..15
+            const __nv_bfloat16 *src = args.gather_src;
+            const size_t ld = static_cast<size_t>(args.gather_ld);
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+                const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
+                if constexpr (!C::RAGGED_K) {
+                    // K-major A: the tile's 128 rows, this thread's rows r0 + 16 i
+                    int tok[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = r0 + 16 * i;
+                        tok[i] = r < t.rows ? __ldg(args.row_token + t.m0 + r) : 0;
+                    }
+                    for (int kb = 0; kb < t.nkb; ++kb) {
+                        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status)) goto pull_done;
+                        uint8_t *dst = tiles + stage * C::STAGE_BYTES;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int r = r0 + 16 * i;
+                            cp_async16(dst + r * 128 + ((c16 ^ (r & 7)) << 4), src + tok[i] * ld + kb * BK + c16 * 8);
+                        }
+                        cp_async_arrive_noinc(&full_bar[stage]);
+                        if (++stage == C::STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                } else {
+                    // MN-major operand: 64 gathered K rows per block, this thread's rows r0 + 16 i
+                    constexpr int CH = (C::A_GATHER ? BM : C::BN) / 64;
+                    constexpr int OFF = C::A_GATHER ? 0 : C::A_BYTES;
+                    const int mn0 = C::A_GATHER ? t.m0 : t.nt * C::BN;
+                    const int end = t.krow0 + t.krows;
+                    int tok[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int kr = t.krow0 + r0 + 16 * i;
+                        tok[i] = kr < end ? __ldg(args.row_token + kr) : 0;
+                    }
+                    for (int kb = 0; kb < t.nkb; ++kb) {
+                        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status)) goto pull_done;
+                        uint8_t *dst = tiles + stage * C::STAGE_BYTES + OFF;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int r = r0 + 16 * i;
+                            const __nv_bfloat16 *row = src + tok[i] * ld + mn0 + c16 * 8;
+#pragma unroll
+                            for (int j = 0; j < CH; ++j)
+                                cp_async16(dst + j * 8192 + r * 128 + ((c16 ^ (r & 7)) << 4), row + j * 64);
+                        }
+                        cp_async_arrive_noinc(&full_bar[stage]);
+                        if (kb + 1 < t.nkb) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int kr = t.krow0 + (kb + 1) * BK + r0 + 16 * i;
+                                tok[i] = kr < end ? __ldg(args.row_token + kr) : 0;
+                            }
+                        }
+                        if (++stage == C::STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                }
+            }
+        pull_done:;
+        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         int stage = 0, acc = 0;
@@ -386,6 +444,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 tc_fence_after();
                 if (lane == 0) {
+                    if constexpr (C::PULL_WARPS > 0) fence_proxy_async_smem();   // cp.async data -> tensor core
                     const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
 #pragma unroll
                     for (int k = 0; k < BK / 16; ++k) {

@@ -255,7 +255,7 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(grouped_gemm_kernel)", e);
-    grouped_gemm_kernel<C><<<grid, 192, C::SMEM_BYTES, st>>>(a, b, bs, args);
+    grouped_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, bs, args);
     e = cudaGetLastError();
     return e == cudaSuccess ? MOK_OK : fail(MOK_ERR_LAUNCH, "grouped_gemm_kernel launch", e);
 }
@@ -327,7 +327,6 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
 
     // gate/up: pull token rows by index, SwiGLU epilogue
     CUtensorMap tA, tB, tBs;
-    if (!make_tmap(&tA, x, s.H, s.T, BK, 1, 2)) return MOK_ERR_INVALID;
     if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, BK, 128, 2)) return MOK_ERR_INVALID;
     if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, BK, 128, 2))
         return MOK_ERR_INVALID;
@@ -346,10 +345,12 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     ga.out2 = training ? st.gu : nullptr;
     ga.out3 = training ? st.hw : nullptr;
     ga.inter = c.I;
+    ga.gather_src = static_cast<const __nv_bfloat16 *>(x);
+    ga.gather_ld = c.H;
     ga.status = dev.status;
     using CGateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU>;
     MOK_TRY(mark_fwd(2, stream));
-    MOK_TRY(launch_gemm<CGateUp>(tA, tB, tBs, ga, dev.sms, stream));
+    MOK_TRY(launch_gemm<CGateUp>(tB, tB, tBs, ga, dev.sms, stream));
 
     // down: contiguous h rows, push epilogue into (token, slot) rows
     if (!make_tmap(&tA, st.h, s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
@@ -417,11 +418,12 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     base.row_slot = st.row_slot;
     base.row_w = st.row_w;
     base.inter = c.I;
+    base.gather_src = dyb;
+    base.gather_ld = c.H;
     base.status = dev.status;
 
     CUtensorMap tA, tB, tBs;
     // dgrad of down: dh = w * (dy[token] . W_down), SwiGLU backward epilogue -> dGU
-    if (!make_tmap(&tA, dy, s.H, s.T, BK, 1, 2)) return MOK_ERR_INVALID;
     if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
     if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
     GemmArgs g1 = base;
@@ -432,7 +434,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g1.out = bs.dgu;
     using CDgradDown = GemmCfg<128, false, true, true, false, false, EPI_DSWIGLU>;
     MOK_TRY(mark_bwd(3, stream));
-    MOK_TRY(launch_gemm<CDgradDown>(tA, tB, tBs, g1, dev.sms, stream));
+    MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, g1, dev.sms, stream));
 
     // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
     if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
@@ -446,7 +448,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     using CWgradDown = GemmCfg<128, true, true, true, false, true, EPI_WGRAD>;
     const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
     MOK_TRY(mark_bwd(4, stream));
-    MOK_TRY(launch_gemm<CWgradDown>(tA, tB, tB, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms), stream));
+    MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms), stream));
 
     // dgrad of gate/up: dX rows = dGU . W_gate_up, pushed into (token, slot) rows
     if (!make_tmap(&tA, bs.dgu, 2 * s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
@@ -465,8 +467,8 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
 
     // wgrad of gate/up: dW_gate_up[g] = sum_r dGU_r^T x[token r]
     if (!make_tmap(&tA, bs.dgu, 2 * s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tB, x, s.H, s.T, BK, 1, 2)) return MOK_ERR_INVALID;
     GemmArgs g4 = base;
+    g4.gather_src = static_cast<const __nv_bfloat16 *>(x);
     g4.m_tiles = 2 * c.I / 128;
     g4.n_tiles = c.H / 256;
     g4.out = static_cast<__nv_bfloat16 *>(gr.dw_gate_up);
@@ -476,7 +478,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     using CWgradGU = GemmCfg<256, true, true, false, true, true, EPI_WGRAD>;
     const long long t4 = s.G * g4.m_tiles * g4.n_tiles;
     MOK_TRY(mark_bwd(6, stream));
-    MOK_TRY(launch_gemm<CWgradGU>(tA, tB, tB, g4, static_cast<int>(t4 < dev.sms ? t4 : dev.sms), stream));
+    MOK_TRY(launch_gemm<CWgradGU>(tA, tA, tA, g4, static_cast<int>(t4 < dev.sms ? t4 : dev.sms), stream));
 
     MOK_TRY(mark_bwd(7, stream));
     dx_combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(

@@ -1,5 +1,5 @@
-// ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA (tiled and
-// gather4), tcgen05 (TMEM allocation, UMMA issue/commit, TMEM loads) and the
+// ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA tiles,
+// cp.async, tcgen05 (TMEM allocation, UMMA issue/commit, TMEM loads) and the
 // shared-memory / instruction descriptors those take.
 #pragma once
 #include <cstdint>
@@ -95,16 +95,17 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, ui
         : "memory");
 }
 
-// Gather of four rows r0..r3 (box one row high, `col` the inner start) into four
-// consecutive 128-byte shared-memory rows at dst.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *tm, uint64_t *bar, int32_t col, int32_t r0,
-                                            int32_t r1, int32_t r2, int32_t r3)
+// 16-byte asynchronous global->shared copy, cached in L2 only.
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
 {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+
+// Arrive on `bar` once all cp.async copies issued so far by this thread have
+// landed (the arrival is counted in the barrier's initial count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
