@@ -279,9 +279,11 @@ def main():
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{wl.name}: DeepSeek-V3-shaped MoE layer fwd+bwd BF16, T={wl.T}, "
-                                   f"H={wl.H}, E={wl.E}, top-{wl.k}, I={wl.I}, {wl.S} shared expert, "
-                                   f"sigmoid+bias routing, {wl.n_group} groups / top-{wl.topk_group}",
+            "config": {"workload": f"{wl.name}: MoE layer fwd+bwd BF16, T={wl.T}, H={wl.H}, E={wl.E}, "
+                                   f"top-{wl.k}, I={wl.I}, {wl.S} shared expert(s), "
+                                   + (f"sigmoid+bias routing, {wl.n_group} groups / top-{wl.topk_group}"
+                                      if wl.score_fn else "softmax routing")
+                                   + (f", Zipf({wl.zipf}) logit term" if wl.zipf else ""),
                        "tokens_per_gpu": wl.T, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (22.6 GB expert weights streamed per pass)"},
             "gpu_launches": K * (len(FWD_PHASES) + len(BWD_PHASES)),

@@ -54,6 +54,10 @@ WORKLOADS = {
                            seed=3),
     "dsv3_zipf": Workload("dsv3_zipf", T=16384, H=7168, E=256, k=8, I=2048, S=1, Is=2048,
                           score_fn=1, n_group=8, topk_group=4, zipf=1.2, seed=4),
+    # DeepSeek-V3 expert shape with 32 experts: small enough for kernel captures
+    # (about 6 GB on the device with gradients) while every operand exceeds L2
+    "dsv3_e32": Workload("dsv3_e32", T=1024, H=7168, E=32, k=8, I=2048, S=1, Is=2048,
+                         score_fn=1, n_group=8, topk_group=4, seed=5),
 }
 
 
