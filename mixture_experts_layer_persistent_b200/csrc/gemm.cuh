@@ -374,11 +374,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     constexpr int OFF = C::A_GATHER ? 0 : C::A_BYTES;
                     const int mn0 = C::A_GATHER ? t.m0 : t.nt * C::BN;
                     const int end = t.krow0 + t.krows;
-                    int tok[4];
+                    // token rows of K blocks kb, kb+1, kb+2: fetched three blocks ahead so
+                    // that the index loads never stall the copies
+                    int tk0[4], tk1[4], tk2[4];
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int kr = t.krow0 + r0 + 16 * i;
-                        tok[i] = kr < end ? __ldg(args.row_token + kr) : 0;
+                        tk0[i] = kr < end ? __ldg(args.row_token + kr) : 0;
+                        tk1[i] = kr + BK < end ? __ldg(args.row_token + kr + BK) : 0;
+                        tk2[i] = kr + 2 * BK < end ? __ldg(args.row_token + kr + 2 * BK) : 0;
                     }
                     for (int kb = 0; kb < t.nkb; ++kb) {
                         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status)) goto pull_done;
@@ -386,18 +390,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const int r = r0 + 16 * i;
-                            const __nv_bfloat16 *row = src + tok[i] * ld + mn0 + c16 * 8;
+                            const __nv_bfloat16 *row = src + tk0[i] * ld + mn0 + c16 * 8;
 #pragma unroll
                             for (int j = 0; j < CH; ++j)
                                 cp_async16(dst + j * 8192 + r * 128 + ((c16 ^ (r & 7)) << 4), row + j * 64);
                         }
                         cp_async_arrive_noinc(&full_bar[stage]);
-                        if (kb + 1 < t.nkb) {
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int kr = t.krow0 + (kb + 1) * BK + r0 + 16 * i;
-                                tok[i] = kr < end ? __ldg(args.row_token + kr) : 0;
-                            }
+                        for (int i = 0; i < 4; ++i) {
+                            const int kr = t.krow0 + (kb + 3) * BK + r0 + 16 * i;
+                            tk0[i] = tk1[i];
+                            tk1[i] = tk2[i];
+                            tk2[i] = kr < end ? __ldg(args.row_token + kr) : 0;
                         }
                         if (++stage == C::STAGES) {
                             stage = 0;

@@ -437,18 +437,26 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, g1, dev.sms, stream));
 
     // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
-    if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
     GemmArgs g2 = base;
     g2.m_tiles = c.H / 128;
-    g2.n_tiles = c.I / 128;
     g2.out = static_cast<__nv_bfloat16 *>(gr.dw_down);
     g2.out_s = static_cast<__nv_bfloat16 *>(gr.dws_down);
     g2.ldo = c.I;
     g2.group_out_elems = s.H * s.I;
-    using CWgradDown = GemmCfg<128, true, true, true, false, true, EPI_WGRAD>;
-    const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
     MOK_TRY(mark_bwd(4, stream));
-    MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms), stream));
+    if (c.I % 256 == 0) {
+        if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
+        g2.n_tiles = c.I / 256;
+        using CWgradDown = GemmCfg<256, true, true, true, false, true, EPI_WGRAD>;
+        const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
+        MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms), stream));
+    } else {
+        if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
+        g2.n_tiles = c.I / 128;
+        using CWgradDown = GemmCfg<128, true, true, true, false, true, EPI_WGRAD>;
+        const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
+        MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms), stream));
+    }
 
     // dgrad of gate/up: dX rows = dGU . W_gate_up, pushed into (token, slot) rows
     if (!make_tmap(&tA, bs.dgu, 2 * s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
