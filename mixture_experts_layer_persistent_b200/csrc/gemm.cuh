@@ -36,6 +36,7 @@ namespace mok {
 constexpr int BM = 128;        // UMMA M (cta_group::1, all 128 TMEM lanes)
 constexpr int BK = 64;         // one 128-byte swizzle row of bf16
 constexpr int kMaxGroups = 264;
+constexpr int kPanelM = 8;     // ragged-M raster panel height (M tiles)
 
 enum Epi : int { EPI_SWIGLU = 0, EPI_PUSH = 1, EPI_DSWIGLU = 2, EPI_WGRAD = 3, EPI_ROUTER = 4 };
 
@@ -127,9 +128,17 @@ __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const i
             if (s_tstart[mid] <= tile) lo = mid; else hi = mid - 1;
         }
         t.g = lo;
+        // Raster inside a group: panels of up to kPanelM M tiles; within a panel
+        // the N tiles are outer and the M tiles inner, so the CTAs that run at
+        // the same time share one weight strip (read from HBM once) while the
+        // panel's activation rows stay in L2.
         const int local = tile - s_tstart[lo];
-        const int mt = local / a.n_tiles;
-        t.nt = local - mt * a.n_tiles;
+        const int mtiles = (s_off[lo + 1] - s_off[lo] + BM - 1) / BM;
+        const int per_panel = kPanelM * a.n_tiles;
+        const int pnl = local / per_panel, rem = local - pnl * per_panel;
+        const int ps = min(kPanelM, mtiles - pnl * kPanelM);
+        t.nt = rem / ps;
+        const int mt = pnl * kPanelM + (rem - t.nt * ps);
         t.m0 = s_off[lo] + mt * BM;
         t.rows = min(BM, s_off[lo + 1] - t.m0);
         t.krow0 = 0;
