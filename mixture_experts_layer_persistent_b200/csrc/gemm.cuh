@@ -84,8 +84,7 @@ struct GemmCfg {
     static constexpr int GATHER_BYTES = A_GATHER ? A_BYTES : (B_GATHER ? B_BYTES : 0);
     static constexpr int TMA_BYTES = STAGE_BYTES - GATHER_BYTES;
     static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int STAGE_WORDS = 36;                       // padded u32 per staged row (32 + 4)
-    static constexpr int EPI_STAGE_BYTES = 4 * 32 * STAGE_WORDS * 4;
+    static constexpr int EPI_STAGE_BYTES = 4 * 4096;             // one 32 x 128-byte block per epilogue warp
     static constexpr int AUX_BYTES = 256 + 3 * kMaxGroups * 4;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_STAGE_BYTES + AUX_BYTES;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
@@ -150,71 +149,96 @@ __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const i
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
-// Warp-cooperative store of a 32-row block: lane l supplies row l as W u32
-// words (W = 16 or 32) and that row's destination (null = skip the row).
-// The block goes through a padded per-warp staging buffer so that each store
-// instruction writes 32 / (W/4) whole rows of 4W contiguous bytes.
-template <int W>
-__device__ __forceinline__ void warp_store_rows(uint32_t *stage, const uint32_t (&p)[W], void *dst, int lane)
-{
-    constexpr int S = 36;
-#pragma unroll
-    for (int i = 0; i < W; i += 4)
-        *reinterpret_cast<uint4 *>(stage + lane * S + i) = make_uint4(p[i], p[i + 1], p[i + 2], p[i + 3]);
-    __syncwarp();
-    constexpr int LPR = W / 4;        // lanes per row
-    constexpr int RPI = 32 / LPR;     // rows per store instruction
-    const uint64_t d = reinterpret_cast<uint64_t>(dst);
-#pragma unroll
-    for (int it = 0; it < 32 / RPI; ++it) {
-        const int row = it * RPI + lane / LPR, ch = lane % LPR;
-        const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d), row);
-        const uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d >> 32), row);
-        const uint4 v = *reinterpret_cast<const uint4 *>(stage + row * S + ch * 4);
-        const uint64_t rd = (static_cast<uint64_t>(hi) << 32) | lo;
-        if (rd) reinterpret_cast<uint4 *>(rd)[ch] = v;
-    }
-    __syncwarp();
-}
-
-// Warp-cooperative load of a 32-row block (inverse of warp_store_rows): lane l
-// receives row l (W u32 words) read from `src` (null = zeros).
-template <int W>
-__device__ __forceinline__ void warp_load_rows(uint32_t *stage, uint32_t (&p)[W], const void *src, int lane)
-{
-    constexpr int S = 36;
-    constexpr int LPR = W / 4;
-    constexpr int RPI = 32 / LPR;
-    const uint64_t d = reinterpret_cast<uint64_t>(src);
-#pragma unroll
-    for (int it = 0; it < 32 / RPI; ++it) {
-        const int row = it * RPI + lane / LPR, ch = lane % LPR;
-        const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d), row);
-        const uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d >> 32), row);
-        const uint64_t rs = (static_cast<uint64_t>(hi) << 32) | lo;
-        const uint4 v = rs ? reinterpret_cast<const uint4 *>(rs)[ch] : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4 *>(stage + row * S + ch * 4) = v;
-    }
-    __syncwarp();
-#pragma unroll
-    for (int i = 0; i < W; i += 4) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(stage + lane * S + i);
-        p[i] = v.x; p[i + 1] = v.y; p[i + 2] = v.z; p[i + 3] = v.w;
-    }
-    __syncwarp();
-}
-
 template <int N>
-__device__ __forceinline__ void pack_bf16(const float *v, uint32_t (&p)[N / 2])
+__device__ __forceinline__ void pack_bf16(const float *v, uint32_t *p)
 {
 #pragma unroll
     for (int i = 0; i < N / 2; ++i) p[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
 }
 
+// ---- epilogue block I/O --------------------------------------------------
+// A warp moves 32 rows x 128 bytes at a time through its 4 KB staging buffer,
+// laid out like a 128-byte-swizzled TMA box (16-byte chunk c of row r at
+// chunk c ^ (r & 7)), so the TMA store engine writes whole lines while the
+// warp moves on; the stores stay in flight without occupying the warp.
+
+__device__ __forceinline__ void stage_block(uint32_t *stg, const uint32_t *p, int lane)
+{
+    if (lane == 0) bulk_wait_read0();     // the previous store from this buffer has read it
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4 *>(stg + lane * 32 + ((c ^ (lane & 7)) << 2)) =
+            make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+}
+
+// 32 full rows to rows row0..row0+31 of a row-major tensor, starting at column col
+__device__ __forceinline__ void store_block_tile(uint32_t *stg, const uint32_t *p, int lane, const CUtensorMap *tm,
+                                                 int col, int row0)
+{
+    stage_block(stg, p, lane);
+    if (lane == 0) {
+        tma_store_2d(tm, stg, col, row0);
+        bulk_commit();
+    }
+}
+
+// 32 full rows, row `lane` to row dst_row (this lane's value), starting at column col
+__device__ __forceinline__ void store_block_scatter(uint32_t *stg, const uint32_t *p, int lane, const CUtensorMap *tm,
+                                                    int col, int dst_row)
+{
+    stage_block(stg, p, lane);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const int r0 = __shfl_sync(0xffffffffu, dst_row, 4 * q + 0);
+        const int r1 = __shfl_sync(0xffffffffu, dst_row, 4 * q + 1);
+        const int r2 = __shfl_sync(0xffffffffu, dst_row, 4 * q + 2);
+        const int r3 = __shfl_sync(0xffffffffu, dst_row, 4 * q + 3);
+        if (lane == 0) tma_scatter4(tm, stg + q * 128, col, r0, r1, r2, r3);
+    }
+    if (lane == 0) bulk_commit();
+}
+
+// one lane's 128-byte row with plain stores (blocks that are only partly valid)
+__device__ __forceinline__ void store_row_direct(void *dst, const uint32_t *p)
+{
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) d[c] = make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+}
+
+// cooperative load of 32 rows x 128 bytes (row `lane` from src, null = zeros) into p
+__device__ __forceinline__ void load_block(uint32_t *stg, uint32_t *p, const void *src, int lane)
+{
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
+    const uint64_t d = reinterpret_cast<uint64_t>(src);
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+        const int row = it * 4 + (lane >> 3), ch = lane & 7;
+        const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d), row);
+        const uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d >> 32), row);
+        const uint64_t rs = (static_cast<uint64_t>(hi) << 32) | lo;
+        const uint4 v = rs ? reinterpret_cast<const uint4 *>(rs)[ch] : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(stg + row * 32 + ((ch ^ (row & 7)) << 2)) = v;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(stg + lane * 32 + ((c ^ (lane & 7)) << 2));
+        p[4 * c] = v.x; p[4 * c + 1] = v.y; p[4 * c + 2] = v.z; p[4 * c + 3] = v.w;
+    }
+    __syncwarp();
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmB_s, const GemmArgs args)
+                        const __grid_constant__ CUtensorMap tmB_s, const __grid_constant__ CUtensorMap tmO,
+                        const __grid_constant__ CUtensorMap tmO2, const __grid_constant__ CUtensorMap tmO3,
+                        const GemmArgs args)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -272,6 +296,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
             tma_prefetch_desc(&tmB_s);
+            tma_prefetch_desc(&tmO);
         }
     } else if (warp == 1) {
         tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -487,8 +512,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int eq = warp & 3;                 // TMEM lane quarter this warp may access
-        const int row = eq * 32 + lane;
-        uint32_t *stg = epi_stage + (warp - 2) * 32 * C::STAGE_WORDS;
+        const int row = eq * 32 + lane;          // tile row of this thread
+        uint32_t *stg = reinterpret_cast<uint32_t *>(epi_stage) + (warp - 2) * 1024;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -496,53 +521,74 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (!mbar_wait(&accf[acc], acc_phase, abort_flag, status)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * C::BN) + (static_cast<uint32_t>(eq * 32) << 16);
+            const bool valid = row < t.rows;
+            const bool full = eq * 32 + 31 < t.rows;        // all 32 rows of this warp's block valid
+            const int row0 = t.m0 + eq * 32;                // first row of the block (ragged-M)
             if constexpr (C::EPI == EPI_SWIGLU) {
                 const int r = t.m0 + row;
-                const bool valid = row < t.rows;
                 const int I = args.inter;
                 const int n0 = t.nt * 128;
                 const float w = (valid && args.out3) ? args.row_w[r] : 0.0f;
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 32) {
-                    float g[32], u[32], h[32];
-                    uint32_t p[16];
-                    tmem_ld32(taddr + c, g);
-                    tmem_ld32(taddr + 128 + c, u);
-                    tmem_ld_wait();
+                for (int c = 0; c < 128; c += 64) {
+                    uint32_t hp[32], wp[32];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) h[i] = silu_f(g[i]) * u[i];
-                    pack_bf16<32>(h, p);
-                    warp_store_rows<16>(stg, p, valid ? args.out + (size_t)r * I + n0 + c : nullptr, lane);
-                    if (args.out2) {
-                        pack_bf16<32>(g, p);
-                        warp_store_rows<16>(stg, p, valid ? args.out2 + (size_t)r * 2 * I + n0 + c : nullptr, lane);
-                        pack_bf16<32>(u, p);
-                        warp_store_rows<16>(stg, p, valid ? args.out2 + (size_t)r * 2 * I + I + n0 + c : nullptr,
-                                            lane);
+                    for (int half = 0; half < 2; ++half) {
+                        float g[32], u[32];
+                        tmem_ld32(taddr + c + 32 * half, g);
+                        tmem_ld32(taddr + 128 + c + 32 * half, u);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
+                        pack_bf16<32>(g, hp + 16 * half);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) g[i] = w * bf16_round(g[i]);
+                        pack_bf16<32>(g, wp + 16 * half);
                     }
+                    if (full) store_block_tile(stg, hp, lane, &tmO, n0 + c, row0);
+                    else if (valid) store_row_direct(args.out + (size_t)r * I + n0 + c, hp);
                     if (args.out3) {
+                        if (full) store_block_tile(stg, wp, lane, &tmO3, n0 + c, row0);
+                        else if (valid) store_row_direct(args.out3 + (size_t)r * I + n0 + c, wp);
+                    }
+                    if (args.out2) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) h[i] = w * bf16_round(h[i]);
-                        pack_bf16<32>(h, p);
-                        warp_store_rows<16>(stg, p, valid ? args.out3 + (size_t)r * I + n0 + c : nullptr, lane);
+                        for (int part = 0; part < 2; ++part) {       // gate, then up pre-activations
+                            float v[64];
+                            uint32_t p[32];
+                            tmem_ld32(taddr + 128 * part + c, *reinterpret_cast<float(*)[32]>(v));
+                            tmem_ld32(taddr + 128 * part + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                            tmem_ld_wait();
+                            pack_bf16<64>(v, p);
+                            const int col = part * I + n0 + c;
+                            if (full) store_block_tile(stg, p, lane, &tmO2, col, row0);
+                            else if (valid) store_row_direct(args.out2 + (size_t)r * 2 * I + col, p);
+                        }
                     }
                 }
-            } else if constexpr (C::EPI == EPI_PUSH || C::EPI == EPI_WGRAD) {
-                __nv_bfloat16 *dst = nullptr;
-                if constexpr (C::EPI == EPI_PUSH) {
-                    if (row < t.rows)
-                        dst = args.out + (size_t)args.row_slot[t.m0 + row] * args.ldo + t.nt * C::BN;
-                } else {
-                    const bool routed = t.g < args.num_routed;
-                    __nv_bfloat16 *base = routed ? args.out + (size_t)t.g * args.group_out_elems
-                                                 : args.out_s + (size_t)(t.g - args.num_routed) * args.group_out_elems;
-                    dst = base + (size_t)(t.m0 + row) * args.ldo + t.nt * C::BN;
-                }
+            } else if constexpr (C::EPI == EPI_PUSH) {
+                const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
+                __nv_bfloat16 *dst = args.out + (size_t)dst_row * args.ldo + t.nt * C::BN;
 #pragma unroll 1
                 for (int c = 0; c < C::BN; c += 64) {
                     float v[64];
                     uint32_t p[32];
-                    if (C::EPI == EPI_PUSH || t.nkb > 0) {
+                    tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
+                    tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                    tmem_ld_wait();
+                    pack_bf16<64>(v, p);
+                    if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
+                    else if (valid) store_row_direct(dst + c, p);
+                }
+            } else if constexpr (C::EPI == EPI_WGRAD) {
+                const bool routed = t.g < args.num_routed;
+                const int gl = routed ? t.g : t.g - args.num_routed;
+                const int grow0 = gl * args.m_tiles * BM + t.m0 + eq * 32;   // row in the [groups * M, N] view
+#pragma unroll 1
+                for (int c = 0; c < C::BN; c += 64) {
+                    float v[64];
+                    uint32_t p[32];
+                    if (t.nkb > 0) {
                         tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
                         tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
                         tmem_ld_wait();
@@ -551,41 +597,47 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         for (int i = 0; i < 64; ++i) v[i] = 0.0f;
                     }
                     pack_bf16<64>(v, p);
-                    warp_store_rows<32>(stg, p, dst ? dst + c : nullptr, lane);
+                    store_block_tile(stg, p, lane, routed ? &tmO : &tmO2, t.nt * C::BN + c, grow0);
                 }
             } else if constexpr (C::EPI == EPI_DSWIGLU) {
                 const int r = t.m0 + row;
-                const bool valid = row < t.rows;
                 const int I = args.inter;
                 const int n0 = t.nt * C::BN;
                 const float w = valid ? args.row_w[r] : 0.0f;
                 const __nv_bfloat16 *gsrc = valid ? args.aux + (size_t)r * 2 * I + n0 : nullptr;
-                __nv_bfloat16 *gdst = valid ? args.out + (size_t)r * 2 * I + n0 : nullptr;
 #pragma unroll 1
-                for (int c = 0; c < C::BN; c += 32) {
-                    float v[32], dg[32], du[32];
-                    uint32_t gp[16], up[16], p[16];
-                    tmem_ld32(taddr + c, v);
-                    warp_load_rows<16>(stg, gp, gsrc ? gsrc + c : nullptr, lane);
-                    warp_load_rows<16>(stg, up, gsrc ? gsrc + I + c : nullptr, lane);
-                    tmem_ld_wait();
+                for (int c = 0; c < C::BN; c += 64) {
+                    uint32_t gp[32], up[32], dgp[32], dup[32];
+                    load_block(stg, gp, gsrc ? gsrc + c : nullptr, lane);
+                    load_block(stg, up, gsrc ? gsrc + I + c : nullptr, lane);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const float gi = (i & 1) ? bf16_hi(gp[i >> 1]) : bf16_lo(gp[i >> 1]);
-                        const float ui = (i & 1) ? bf16_hi(up[i >> 1]) : bf16_lo(up[i >> 1]);
-                        const float dh = w * v[i];
-                        const float sg = 1.0f / (1.0f + expf(-gi));
-                        dg[i] = dh * ui * sg * (1.0f + gi * (1.0f - sg));
-                        du[i] = dh * gi * sg;
+                    for (int half = 0; half < 2; ++half) {
+                        float v[32], dg[32], du[32];
+                        tmem_ld32(taddr + c + 32 * half, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const uint32_t gw = gp[16 * half + (i >> 1)], uw = up[16 * half + (i >> 1)];
+                            const float gi = (i & 1) ? bf16_hi(gw) : bf16_lo(gw);
+                            const float ui = (i & 1) ? bf16_hi(uw) : bf16_lo(uw);
+                            const float dh = w * v[i];
+                            const float sg = 1.0f / (1.0f + expf(-gi));
+                            dg[i] = dh * ui * sg * (1.0f + gi * (1.0f - sg));
+                            du[i] = dh * gi * sg;
+                        }
+                        pack_bf16<32>(dg, dgp + 16 * half);
+                        pack_bf16<32>(du, dup + 16 * half);
                     }
-                    pack_bf16<32>(dg, p);
-                    warp_store_rows<16>(stg, p, gdst ? gdst + c : nullptr, lane);
-                    pack_bf16<32>(du, p);
-                    warp_store_rows<16>(stg, p, gdst ? gdst + I + c : nullptr, lane);
+                    if (full) {
+                        store_block_tile(stg, dgp, lane, &tmO, n0 + c, row0);
+                        store_block_tile(stg, dup, lane, &tmO, I + n0 + c, row0);
+                    } else if (valid) {
+                        store_row_direct(args.out + (size_t)r * 2 * I + n0 + c, dgp);
+                        store_row_direct(args.out + (size_t)r * 2 * I + I + n0 + c, dup);
+                    }
                 }
             } else {   // EPI_ROUTER: fp32 partial logits of this K split
                 const int r = t.m0 + row;
-                float *dst = row < t.rows ? args.out_f32 + ((size_t)t.nt * args.rows_total + r) * 256 : nullptr;
 #pragma unroll 1
                 for (int c = 0; c < 256; c += 32) {
                     float v[32];
@@ -594,7 +646,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
-                    warp_store_rows<32>(stg, p, dst ? dst + c : nullptr, lane);
+                    if (full) store_block_tile(stg, p, lane, &tmO, c, t.nt * args.rows_total + row0);
+                    else if (valid) store_row_direct(args.out_f32 + ((size_t)t.nt * args.rows_total + r) * 256 + c, p);
                 }
             }
             tc_fence_before();
@@ -602,6 +655,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1u;
         }
+        if (lane == 0) bulk_wait0();             // every bulk store of this warp has completed
     }
 
     tc_fence_before();

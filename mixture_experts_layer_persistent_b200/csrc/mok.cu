@@ -101,7 +101,9 @@ bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
     const cuuint64_t strides[1] = {inner * elem_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t es[2] = {1, 1};
-    const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const CUtensorMapDataType dt = elem_bytes == 2   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : elem_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                                     : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     const CUresult r = g_encode(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -247,15 +249,16 @@ int check_cfg(const moe_cfg *c)
     return MOK_OK;
 }
 
+// Operand maps a, b, bs (B of the shared groups) and output maps o, o2, o3.
 template <class C>
-int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &bs, const GemmArgs &args, int grid,
-                cudaStream_t st)
+int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &bs, const CUtensorMap &o,
+                const CUtensorMap &o2, const CUtensorMap &o3, const GemmArgs &args, int grid, cudaStream_t st)
 {
     if (grid <= 0) return MOK_OK;
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(grouped_gemm_kernel)", e);
-    grouped_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, bs, args);
+    grouped_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, bs, o, o2, o3, args);
     e = cudaGetLastError();
     return e == cudaSuccess ? MOK_OK : fail(MOK_ERR_LAUNCH, "grouped_gemm_kernel launch", e);
 }
@@ -287,9 +290,10 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
                                                                          c.T);
     MOK_LAUNCHED();
     {
-        CUtensorMap rA, rB;
+        CUtensorMap rA, rB, rO;
         if (!make_tmap(&rA, x, s.H, s.T, BK, 128, 2)) return fail(MOK_ERR_INVALID, "tensor map (x)");
         if (!make_tmap(&rB, st.wr3, 3 * s.H, s.E, BK, 256, 2)) return fail(MOK_ERR_INVALID, "tensor map (router)");
+        if (!make_tmap(&rO, st.rpart, 256, s.n_split * s.T, 32, 32, 4)) return fail(MOK_ERR_INVALID, "tensor map (logits)");
         GemmArgs gr{};
         gr.num_groups = 1;
         gr.num_routed = 1;
@@ -301,7 +305,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         gr.rows_total = c.T;
         gr.status = dev.status;
         using CRouter = GemmCfg<256, false, false, false, false, false, EPI_ROUTER>;
-        MOK_TRY(launch_gemm<CRouter>(rA, rB, rB, gr, dev.sms, stream));
+        MOK_TRY(launch_gemm<CRouter>(rA, rB, rB, rO, rO, rO, gr, dev.sms, stream));
     }
     SelectArgs sa;
     sa.partial = st.rpart;
@@ -326,8 +330,11 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     MOK_LAUNCHED();
 
     // gate/up: pull token rows by index, SwiGLU epilogue
-    CUtensorMap tA, tB, tBs;
+    CUtensorMap tA, tB, tBs, tO, tO2, tO3;
     if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, BK, 128, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tO, st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tO2, training ? st.gu : st.h, training ? 2 * s.I : s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tO3, training ? st.hw : st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
     if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, BK, 128, 2))
         return MOK_ERR_INVALID;
     GemmArgs ga{};
@@ -350,7 +357,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     ga.status = dev.status;
     using CGateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU>;
     MOK_TRY(mark_fwd(2, stream));
-    MOK_TRY(launch_gemm<CGateUp>(tB, tB, tBs, ga, dev.sms, stream));
+    MOK_TRY(launch_gemm<CGateUp>(tB, tB, tBs, tO, tO2, tO3, ga, dev.sms, stream));
 
     // down: contiguous h rows, push epilogue into (token, slot) rows
     if (!make_tmap(&tA, st.h, s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
@@ -367,7 +374,8 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     gd.ldo = c.H;
     using CDown = GemmCfg<256, false, false, false, false, false, EPI_PUSH>;
     MOK_TRY(mark_fwd(3, stream));
-    MOK_TRY(launch_gemm<CDown>(tA, tB, tBs, gd, dev.sms, stream));
+    if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;
+    MOK_TRY(launch_gemm<CDown>(tA, tB, tBs, tO, tO, tO, gd, dev.sms, stream));
 
     MOK_TRY(mark_fwd(4, stream));
     combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(st.O, st.topk_w,
@@ -422,7 +430,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     base.gather_ld = c.H;
     base.status = dev.status;
 
-    CUtensorMap tA, tB, tBs;
+    CUtensorMap tA, tB, tBs, tO, tO2;
     // dgrad of down: dh = w * (dy[token] . W_down), SwiGLU backward epilogue -> dGU
     if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
     if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
@@ -434,7 +442,8 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g1.out = bs.dgu;
     using CDgradDown = GemmCfg<128, false, true, true, false, false, EPI_DSWIGLU>;
     MOK_TRY(mark_bwd(3, stream));
-    MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, g1, dev.sms, stream));
+    if (!make_tmap(&tO, bs.dgu, 2 * s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+    MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, tO, tO, tO, g1, dev.sms, stream));
 
     // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
     GemmArgs g2 = base;
@@ -444,18 +453,23 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g2.ldo = c.I;
     g2.group_out_elems = s.H * s.I;
     MOK_TRY(mark_bwd(4, stream));
+    if (!make_tmap(&tO, gr.dw_down, s.I, s.E * s.H, 64, 32, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tO2, s.S ? gr.dws_down : gr.dw_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 32, 2))
+        return MOK_ERR_INVALID;
     if (c.I % 256 == 0) {
         if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
         g2.n_tiles = c.I / 256;
         using CWgradDown = GemmCfg<256, true, true, true, false, true, EPI_WGRAD>;
         const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
-        MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms), stream));
+        MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, tO, tO2, tO, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms),
+                                        stream));
     } else {
         if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
         g2.n_tiles = c.I / 128;
         using CWgradDown = GemmCfg<128, true, true, true, false, true, EPI_WGRAD>;
         const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
-        MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms), stream));
+        MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, tO, tO2, tO, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms),
+                                        stream));
     }
 
     // dgrad of gate/up: dX rows = dGU . W_gate_up, pushed into (token, slot) rows
@@ -471,7 +485,8 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g3.ldo = c.H;
     using CDgradGU = GemmCfg<256, false, true, false, false, false, EPI_PUSH>;
     MOK_TRY(mark_bwd(5, stream));
-    MOK_TRY(launch_gemm<CDgradGU>(tA, tB, tBs, g3, dev.sms, stream));
+    if (!make_tmap(&tO, bs.dxs, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;
+    MOK_TRY(launch_gemm<CDgradGU>(tA, tB, tBs, tO, tO, tO, g3, dev.sms, stream));
 
     // wgrad of gate/up: dW_gate_up[g] = sum_r dGU_r^T x[token r]
     if (!make_tmap(&tA, bs.dgu, 2 * s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
@@ -486,7 +501,10 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     using CWgradGU = GemmCfg<256, true, true, false, true, true, EPI_WGRAD>;
     const long long t4 = s.G * g4.m_tiles * g4.n_tiles;
     MOK_TRY(mark_bwd(6, stream));
-    MOK_TRY(launch_gemm<CWgradGU>(tA, tA, tA, g4, static_cast<int>(t4 < dev.sms ? t4 : dev.sms), stream));
+    if (!make_tmap(&tO, gr.dw_gate_up, s.H, s.E * 2 * s.I, 64, 32, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tO2, s.S ? gr.dws_gate_up : gr.dw_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 64, 32, 2))
+        return MOK_ERR_INVALID;
+    MOK_TRY(launch_gemm<CWgradGU>(tA, tA, tA, tO, tO2, tO, g4, static_cast<int>(t4 < dev.sms ? t4 : dev.sms), stream));
 
     MOK_TRY(mark_bwd(7, stream));
     dx_combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(

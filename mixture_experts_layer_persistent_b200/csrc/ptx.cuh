@@ -95,6 +95,33 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, ui
         : "memory");
 }
 
+// 2D tiled TMA store of a shared-memory box to global memory (bulk group).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *tm, const void *src, int32_t c0, int32_t c1)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+
+// TMA store of four consecutive 128-byte shared-memory rows to rows r0..r3
+// (box one row high, `col` the inner start).
+__device__ __forceinline__ void tma_scatter4(const CUtensorMap *tm, const void *src, int32_t col, int32_t r0,
+                                             int32_t r1, int32_t r2, int32_t r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.tile::scatter4.bulk_group [%0, {%2, %3, %4, %5, %6}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(tm)),
+        "r"(smem_u32(src)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until this thread's bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until this thread's bulk stores have completed
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // 16-byte asynchronous global->shared copy, cached in L2 only.
 __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
 {
