@@ -30,6 +30,7 @@
 // results do not depend on scheduling: the layer is bit-reproducible.
 #pragma once
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace mok {
 
@@ -56,6 +57,12 @@ struct GemmArgs {
     int a_k_mod;                  // EPI_ROUTER: A's K coordinate wraps at this many elements (H)
     const __nv_bfloat16 *gather_src; // token matrix the pull warps gather rows from (x or dy)
     int gather_ld;                // elements per token row of gather_src
+    // MXFP8 (block-scaled) operands: ue8m0 scales, one byte per 32 K-elements, rows of sf_ld bytes
+    const uint8_t *sfa_src;       // scales of A's rows (token rows when A is gathered, sorted rows otherwise)
+    const uint8_t *sfb_src;       // scales of the routed groups' B rows
+    const uint8_t *sfb_src_s;     // scales of the shared groups' B rows
+    int sf_ld;                    // scale bytes per row (K / 32)
+    uint8_t *out_scales;          // MXFP8 SwiGLU epilogue: scales of h [R, I/32]
     __nv_bfloat16 *out;           // main output
     __nv_bfloat16 *out_s;         // EPI_WGRAD: output of the shared groups
     __nv_bfloat16 *out2;          // EPI_SWIGLU: saved gate/up pre-activations [R, 2I] (or null)
@@ -69,25 +76,35 @@ struct GemmArgs {
     int *status;                  // device status word
 };
 
-template <int BN_, bool A_MN_, bool B_MN_, bool A_GATHER_, bool B_GATHER_, bool RAGGED_K_, int EPI_>
+template <int BN_, bool A_MN_, bool B_MN_, bool A_GATHER_, bool B_GATHER_, bool RAGGED_K_, int EPI_,
+          bool MX_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;
     static constexpr bool A_MN = A_MN_, B_MN = B_MN_, A_GATHER = A_GATHER_, B_GATHER = B_GATHER_;
     static constexpr bool RAGGED_K = RAGGED_K_;
     static constexpr int EPI = EPI_;
-    static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr bool MX = MX_;                              // e4m3 operands with ue8m0 block scales
+    static constexpr int ESIZE = MX ? 1 : 2;                     // operand bytes per element
+    static constexpr int KB_ELEMS = 128 / ESIZE;                 // K elements per 128-byte block row
+    static constexpr int A_BYTES = BM * 128;
+    static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int SF_BYTES = MX ? 512 + BN * 4 : 0;       // SFA (128 rows) + SFB (BN rows), 4 bytes each
     static constexpr int STAGES = BN == 256 ? 4 : 6;
-    static constexpr int PULL_WARPS = (A_GATHER || B_GATHER) ? 4 : 0;   // cp.async gather warps
+    static constexpr int PULL_WARPS = (A_GATHER || B_GATHER || MX) ? 4 : 0;   // cp.async warps
     static constexpr int THREADS = 192 + 32 * PULL_WARPS;
     static constexpr int GATHER_BYTES = A_GATHER ? A_BYTES : (B_GATHER ? B_BYTES : 0);
     static constexpr int TMA_BYTES = STAGE_BYTES - GATHER_BYTES;
-    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int ACC_BUFS = MX ? 1 : 2;                  // MXFP8 needs TMEM columns for the scales
+    static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
+    static constexpr int SF_TMEM_COL = 256;                      // SFA at 256..259, SFB at 260..
     static constexpr int EPI_STAGE_BYTES = 4 * 4096;             // one 32 x 128-byte block per epilogue warp
     static constexpr int AUX_BYTES = 256 + 3 * kMaxGroups * 4;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_STAGE_BYTES + AUX_BYTES;
+    static constexpr int SMEM_BYTES =
+        1024 + STAGES * STAGE_BYTES + STAGES * SF_BYTES + EPI_STAGE_BYTES + AUX_BYTES;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
+    static_assert(!MX || (!A_MN && !B_MN && !RAGGED_K && BN == 256 && (EPI == EPI_SWIGLU || EPI == EPI_PUSH)),
+                  "MXFP8 serves the forward expert GEMMs");
     static_assert(BN == 128 || BN == 256, "BN");
     static_assert(!RAGGED_K || (A_MN && B_MN), "weight gradients take both operands MN-major");
     static_assert(!RAGGED_K || (A_GATHER != B_GATHER), "one operand of a weight gradient is gathered");
@@ -243,7 +260,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *tiles = smem;
-    uint32_t *epi_stage = reinterpret_cast<uint32_t *>(tiles + C::STAGES * C::STAGE_BYTES);
+    uint8_t *sf_tiles = tiles + C::STAGES * C::STAGE_BYTES;     // MXFP8 scale blocks, one per stage
+    uint32_t *epi_stage = reinterpret_cast<uint32_t *>(sf_tiles + C::STAGES * C::SF_BYTES);
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(epi_stage) + C::EPI_STAGE_BYTES);
     uint64_t *empty_bar = full_bar + C::STAGES;
     uint64_t *accf = empty_bar + C::STAGES;
@@ -328,10 +346,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 uint8_t *sB = sA + C::A_BYTES;
                 uint64_t *fb = &full_bar[stage];
                 const int kg = C::EPI == EPI_ROUTER ? t.nt * args.num_kb + kb : kb;   // global K block
+                constexpr int KE = C::KB_ELEMS;
                 // ---- A (gathered A rows come from the pull warps)
                 if constexpr (!C::A_GATHER && !C::A_MN) {
                     if (lane == 0) {
-                        const int kc = C::EPI == EPI_ROUTER ? (kg * BK) % args.a_k_mod : kb * BK;
+                        const int kc = C::EPI == EPI_ROUTER ? (kg * BK) % args.a_k_mod : kb * KE;
                         tma_load_2d(sA, &tmA, fb, kc, t.m0);
                     }
                 } else if constexpr (!C::A_GATHER && C::A_MN) {
@@ -342,12 +361,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     if (lane == 0) {
                         if constexpr (C::EPI == EPI_SWIGLU) {
                             const int row = gl * args.b_rows_per_group + t.nt * 128;
-                            tma_load_2d(sB, mB, fb, kb * BK, row);
-                            tma_load_2d(sB + 128 * 128, mB, fb, kb * BK, row + args.b_half);
+                            tma_load_2d(sB, mB, fb, kb * KE, row);
+                            tma_load_2d(sB + 128 * 128, mB, fb, kb * KE, row + args.b_half);
                         } else if constexpr (C::EPI == EPI_ROUTER) {
                             tma_load_2d(sB, mB, fb, kg * BK, 0);
                         } else {
-                            tma_load_2d(sB, mB, fb, kb * BK, gl * args.b_rows_per_group + t.nt * C::BN);
+                            tma_load_2d(sB, mB, fb, kb * KE, gl * args.b_rows_per_group + t.nt * C::BN);
                         }
                     }
                 } else if constexpr (!C::B_GATHER && !C::RAGGED_K) {
@@ -374,8 +393,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const int p = threadIdx.x - 192;
             const int c16 = p & 7;
             const int r0 = p >> 3;                      // 0..15
-            const __nv_bfloat16 *src = args.gather_src;
-            const size_t ld = static_cast<size_t>(args.gather_ld);
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(args.gather_src);
+            const size_t ld = static_cast<size_t>(args.gather_ld) * C::ESIZE;   // bytes per token row
             int stage = 0;
             uint32_t phase = 0;
             for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -383,18 +402,50 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 if constexpr (!C::RAGGED_K) {
                     // K-major A: the tile's 128 rows, this thread's rows r0 + 16 i
                     int tok[8];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int r = r0 + 16 * i;
-                        tok[i] = r < t.rows ? __ldg(args.row_token + t.m0 + r) : 0;
-                    }
-                    for (int kb = 0; kb < t.nkb; ++kb) {
-                        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status)) goto pull_done;
-                        uint8_t *dst = tiles + stage * C::STAGE_BYTES;
+                    if constexpr (C::A_GATHER) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const int r = r0 + 16 * i;
-                            cp_async16(dst + r * 128 + ((c16 ^ (r & 7)) << 4), src + tok[i] * ld + kb * BK + c16 * 8);
+                            tok[i] = r < t.rows ? __ldg(args.row_token + t.m0 + r) : 0;
+                        }
+                    }
+                    // MXFP8 scales: SFA row p (its token row when A is gathered), SFB rows p and p + 128
+                    const uint8_t *sfa = nullptr, *sfb0 = nullptr, *sfb1 = nullptr;
+                    if constexpr (C::MX) {
+                        const int ar = p < t.rows ? (C::A_GATHER ? __ldg(args.row_token + t.m0 + p) : t.m0 + p)
+                                                  : (C::A_GATHER ? 0 : t.m0);
+                        sfa = args.sfa_src + (size_t)ar * args.sf_ld;
+                        const bool routed = t.g < args.num_routed;
+                        const int gl = routed ? t.g : t.g - args.num_routed;
+                        const uint8_t *sb = routed ? args.sfb_src : args.sfb_src_s;
+                        int b0, b1;
+                        if constexpr (C::EPI == EPI_SWIGLU) {
+                            b0 = t.nt * 128 + p;                 // gate row
+                            b1 = args.b_half + t.nt * 128 + p;   // matching up row
+                        } else {
+                            b0 = t.nt * C::BN + p;
+                            b1 = t.nt * C::BN + 128 + p;
+                        }
+                        sfb0 = sb + ((size_t)gl * args.b_rows_per_group + b0) * args.sf_ld;
+                        sfb1 = sb + ((size_t)gl * args.b_rows_per_group + b1) * args.sf_ld;
+                    }
+                    for (int kb = 0; kb < t.nkb; ++kb) {
+                        if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status)) goto pull_done;
+                        if constexpr (C::A_GATHER) {
+                            uint8_t *dst = tiles + stage * C::STAGE_BYTES;
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const int r = r0 + 16 * i;
+                                cp_async16(dst + r * 128 + ((c16 ^ (r & 7)) << 4), src + tok[i] * ld + kb * 128 + c16 * 16);
+                            }
+                        }
+                        if constexpr (C::MX) {
+                            // SF atom layout: the 4 scales of row m at byte 16 (m % 32) + 4 (m / 32) of its 128-row block
+                            uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
+                            const int at = 16 * (p & 31) + 4 * (p >> 5);
+                            cp_async4(sf + at, sfa + kb * 4);
+                            cp_async4(sf + 512 + at, sfb0 + kb * 4);
+                            cp_async4(sf + 1024 + at, sfb1 + kb * 4);
                         }
                         cp_async_arrive_noinc(&full_bar[stage]);
                         if (++stage == C::STAGES) {
@@ -424,10 +475,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const int r = r0 + 16 * i;
-                            const __nv_bfloat16 *row = src + tk0[i] * ld + mn0 + c16 * 8;
+                            const uint8_t *row = src + tk0[i] * ld + mn0 * C::ESIZE + c16 * 16;
 #pragma unroll
                             for (int j = 0; j < CH; ++j)
-                                cp_async16(dst + j * 8192 + r * 128 + ((c16 ^ (r & 7)) << 4), row + j * 64);
+                                cp_async16(dst + j * 8192 + r * 128 + ((c16 ^ (r & 7)) << 4), row + j * 128);
                         }
                         cp_async_arrive_noinc(&full_bar[stage]);
 #pragma unroll
@@ -484,13 +535,30 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 if (lane == 0) {
                     if constexpr (C::PULL_WARPS > 0) fence_proxy_async_smem();   // cp.async data -> tensor core
                     const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+                    if constexpr (C::MX) {
+                        // scales of this K block into TMEM (issued before, so ordered with, the MMAs)
+                        const uint32_t sf0 = smem_u32(sf_tiles + stage * C::SF_BYTES);
+                        const uint32_t tsfa = tmem_base + C::SF_TMEM_COL, tsfb = tsfa + 4;
+                        tmem_cp_32x128b_x4(tsfa, smem_desc_plain(sf0));
 #pragma unroll
-                    for (int k = 0; k < BK / 16; ++k) {
-                        const uint64_t ad = C::A_MN ? smem_desc_sw128(a0 + k * 2048, 8192, 1024)
-                                                    : smem_desc_sw128(a0 + k * 32, 16, 1024);
-                        const uint64_t bd = C::B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024)
-                                                    : smem_desc_sw128(b0 + k * 32, 16, 1024);
-                        umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                        for (int b = 0; b < C::BN / 128; ++b) tmem_cp_32x128b_x4(tsfb + 4 * b, smem_desc_plain(sf0 + 512 + 512 * b));
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t ad = smem_desc_sw128(a0 + k * 32, 16, 1024);
+                            const uint64_t bd = smem_desc_sw128(b0 + k * 32, 16, 1024);
+                            const uint32_t j = static_cast<uint32_t>(k);
+                            umma_mxf8(d_tmem, ad, bd, idesc_mxf8(BM, C::BN, j), tsfa | (j << 30), tsfb | (j << 30),
+                                      (kb | k) != 0 ? 1u : 0u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < BK / 16; ++k) {
+                            const uint64_t ad = C::A_MN ? smem_desc_sw128(a0 + k * 2048, 8192, 1024)
+                                                        : smem_desc_sw128(a0 + k * 32, 16, 1024);
+                            const uint64_t bd = C::B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024)
+                                                        : smem_desc_sw128(b0 + k * 32, 16, 1024);
+                            umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                        }
                     }
                     umma_commit(&empty_bar[stage]);
                 }
@@ -506,8 +574,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 else mbar_arrive(&accf[acc]);
             }
             __syncwarp();
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1u;
+            if (++acc == C::ACC_BUFS) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -524,7 +594,43 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const bool valid = row < t.rows;
             const bool full = eq * 32 + 31 < t.rows;        // all 32 rows of this warp's block valid
             const int row0 = t.m0 + eq * 32;                // first row of the block (ragged-M)
-            if constexpr (C::EPI == EPI_SWIGLU) {
+            if constexpr (C::EPI == EPI_SWIGLU && C::MX) {
+                // h = silu(g) u quantised per 32 columns: e4m3 codes [R, I] and ue8m0 scales [R, I/32]
+                const int r = t.m0 + row;
+                const int I = args.inter;
+                const int n0 = t.nt * 128;
+                uint32_t q[32];
+                uint32_t sc = 0;
+#pragma unroll
+                for (int blk = 0; blk < 4; ++blk) {
+                    float g[32], u[32];
+                    tmem_ld32(taddr + 32 * blk, g);
+                    tmem_ld32(taddr + 128 + 32 * blk, u);
+                    tmem_ld_wait();
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        g[i] = silu_f(g[i]) * u[i];
+                        amax = fmaxf(amax, fabsf(g[i]));
+                    }
+                    const int e = mx_exponent(amax);
+                    const float sf = exp2_neg(e);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        uint32_t word = 0;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            word |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(g[4 * i + j] * sf, __NV_SATFINITE, __NV_E4M3))
+                                    << (8 * j);
+                        q[8 * blk + i] = word;
+                    }
+                    sc |= static_cast<uint32_t>(e + 127) << (8 * blk);
+                }
+                uint8_t *qout = reinterpret_cast<uint8_t *>(args.out);
+                if (full) store_block_tile(stg, q, lane, &tmO, n0, row0);
+                else if (valid) store_row_direct(qout + (size_t)r * I + n0, q);
+                if (valid) *reinterpret_cast<uint32_t *>(args.out_scales + (size_t)r * (I / 32) + t.nt * 4) = sc;
+            } else if constexpr (C::EPI == EPI_SWIGLU) {
                 const int r = t.m0 + row;
                 const int I = args.inter;
                 const int n0 = t.nt * 128;
@@ -652,8 +758,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
             tc_fence_before();
             mbar_arrive(&acce[acc]);
-            acc ^= 1;
-            if (acc == 0) acc_phase ^= 1u;
+            if (++acc == C::ACC_BUFS) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
         }
         if (lane == 0) bulk_wait0();             // every bulk store of this warp has completed
     }

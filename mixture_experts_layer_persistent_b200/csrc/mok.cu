@@ -282,7 +282,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
             const State &st, const DeviceInfo &dev, bool training, cudaStream_t stream)
 {
     const Shapes s = shapes(c);
-    if (c.dtype != MOK_DTYPE_BF16) return MOK_ERR_UNSUPPORTED;
+    const bool mx = c.dtype == MOK_DTYPE_MXFP8;
 
     // router logits on the tensor cores: x . [Wr_hi | Wr_mid | Wr_lo]^T, split over K
     MOK_TRY(mark_fwd(0, stream));
@@ -329,53 +329,113 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     dispatch_kernel<<<1, 1024, 0, stream>>>(da);
     MOK_LAUNCHED();
 
-    // gate/up: pull token rows by index, SwiGLU epilogue
-    CUtensorMap tA, tB, tBs, tO, tO2, tO3;
-    if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, BK, 128, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tO, st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tO2, training ? st.gu : st.h, training ? 2 * s.I : s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tO3, training ? st.hw : st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, BK, 128, 2))
-        return MOK_ERR_INVALID;
-    GemmArgs ga{};
-    ga.num_groups = static_cast<int>(s.G);
-    ga.num_routed = c.E;
-    ga.offsets = st.offsets;
-    ga.row_token = st.row_token;
-    ga.row_slot = st.row_slot;
-    ga.row_w = st.row_w;
-    ga.n_tiles = c.I / 128;
-    ga.num_kb = c.H / BK;
-    ga.b_rows_per_group = 2 * c.I;
-    ga.b_half = c.I;
-    ga.out = st.h;
-    ga.out2 = training ? st.gu : nullptr;
-    ga.out3 = training ? st.hw : nullptr;
-    ga.inter = c.I;
-    ga.gather_src = static_cast<const __nv_bfloat16 *>(x);
-    ga.gather_ld = c.H;
-    ga.status = dev.status;
-    using CGateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU>;
-    MOK_TRY(mark_fwd(2, stream));
-    MOK_TRY(launch_gemm<CGateUp>(tB, tB, tBs, tO, tO2, tO3, ga, dev.sms, stream));
+    if (mx) {
+        // MXFP8: quantise x (1x32 ue8m0 blocks along H), then block-scaled expert GEMMs
+        MOK_TRY(mark_fwd(2, stream));
+        const long long xb = s.T * s.H / 32;
+        quantize_mxfp8_kernel<<<blocks_for(xb, 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(x), xb,
+                                                                        st.xq, st.xs);
+        MOK_LAUNCHED();
+        CUtensorMap tA, tB, tBs, tO;
+        if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, 128, 128, 1)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 128, 128, 1))
+            return MOK_ERR_INVALID;
+        if (!make_tmap(&tO, st.hq, s.I, s.R, 128, 32, 1)) return MOK_ERR_INVALID;
+        GemmArgs ga{};
+        ga.num_groups = static_cast<int>(s.G);
+        ga.num_routed = c.E;
+        ga.offsets = st.offsets;
+        ga.row_token = st.row_token;
+        ga.row_slot = st.row_slot;
+        ga.row_w = st.row_w;
+        ga.n_tiles = c.I / 128;
+        ga.num_kb = c.H / 128;
+        ga.b_rows_per_group = 2 * c.I;
+        ga.b_half = c.I;
+        ga.out = reinterpret_cast<__nv_bfloat16 *>(st.hq);
+        ga.out_scales = st.hs;
+        ga.inter = c.I;
+        ga.gather_src = reinterpret_cast<const __nv_bfloat16 *>(st.xq);
+        ga.gather_ld = c.H;
+        ga.sfa_src = st.xs;
+        ga.sfb_src = p.s_gate_up;
+        ga.sfb_src_s = s.S ? p.ss_gate_up : p.s_gate_up;
+        ga.sf_ld = c.H / 32;
+        ga.status = dev.status;
+        using CGateUpMx = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU, true>;
+        MOK_TRY(launch_gemm<CGateUpMx>(tB, tB, tBs, tO, tO, tO, ga, dev.sms, stream));
 
-    // down: contiguous h rows, push epilogue into (token, slot) rows
-    if (!make_tmap(&tA, st.h, s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, BK, 256, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, BK, 256, 2))
-        return MOK_ERR_INVALID;
-    GemmArgs gd = ga;
-    gd.n_tiles = c.H / 256;
-    gd.num_kb = c.I / BK;
-    gd.b_rows_per_group = c.H;
-    gd.b_half = 0;
-    gd.out = st.O;
-    gd.out2 = gd.out3 = nullptr;
-    gd.ldo = c.H;
-    using CDown = GemmCfg<256, false, false, false, false, false, EPI_PUSH>;
-    MOK_TRY(mark_fwd(3, stream));
-    if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;
-    MOK_TRY(launch_gemm<CDown>(tA, tB, tBs, tO, tO, tO, gd, dev.sms, stream));
+        if (!make_tmap(&tA, st.hq, s.I, s.R, 128, 128, 1)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 128, 256, 1)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 128, 256, 1))
+            return MOK_ERR_INVALID;
+        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;
+        GemmArgs gd = ga;
+        gd.n_tiles = c.H / 256;
+        gd.num_kb = c.I / 128;
+        gd.b_rows_per_group = c.H;
+        gd.b_half = 0;
+        gd.out = st.O;
+        gd.out_scales = nullptr;
+        gd.ldo = c.H;
+        gd.gather_src = nullptr;
+        gd.sfa_src = st.hs;
+        gd.sfb_src = p.s_down;
+        gd.sfb_src_s = s.S ? p.ss_down : p.s_down;
+        gd.sf_ld = c.I / 32;
+        using CDownMx = GemmCfg<256, false, false, false, false, false, EPI_PUSH, true>;
+        MOK_TRY(mark_fwd(3, stream));
+        MOK_TRY(launch_gemm<CDownMx>(tA, tB, tBs, tO, tO, tO, gd, dev.sms, stream));
+    } else {
+        // gate/up: pull token rows by index, SwiGLU epilogue
+        CUtensorMap tA, tB, tBs, tO, tO2, tO3;
+        if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, BK, 128, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tO, st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tO2, training ? st.gu : st.h, training ? 2 * s.I : s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tO3, training ? st.hw : st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, BK, 128, 2))
+            return MOK_ERR_INVALID;
+        GemmArgs ga{};
+        ga.num_groups = static_cast<int>(s.G);
+        ga.num_routed = c.E;
+        ga.offsets = st.offsets;
+        ga.row_token = st.row_token;
+        ga.row_slot = st.row_slot;
+        ga.row_w = st.row_w;
+        ga.n_tiles = c.I / 128;
+        ga.num_kb = c.H / BK;
+        ga.b_rows_per_group = 2 * c.I;
+        ga.b_half = c.I;
+        ga.out = st.h;
+        ga.out2 = training ? st.gu : nullptr;
+        ga.out3 = training ? st.hw : nullptr;
+        ga.inter = c.I;
+        ga.gather_src = static_cast<const __nv_bfloat16 *>(x);
+        ga.gather_ld = c.H;
+        ga.status = dev.status;
+        using CGateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU>;
+        MOK_TRY(mark_fwd(2, stream));
+        MOK_TRY(launch_gemm<CGateUp>(tB, tB, tBs, tO, tO2, tO3, ga, dev.sms, stream));
+
+        // down: contiguous h rows, push epilogue into (token, slot) rows
+        if (!make_tmap(&tA, st.h, s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, BK, 256, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, BK, 256, 2))
+            return MOK_ERR_INVALID;
+        GemmArgs gd = ga;
+        gd.n_tiles = c.H / 256;
+        gd.num_kb = c.I / BK;
+        gd.b_rows_per_group = c.H;
+        gd.b_half = 0;
+        gd.out = st.O;
+        gd.out2 = gd.out3 = nullptr;
+        gd.ldo = c.H;
+        using CDown = GemmCfg<256, false, false, false, false, false, EPI_PUSH>;
+        MOK_TRY(mark_fwd(3, stream));
+        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;
+        MOK_TRY(launch_gemm<CDown>(tA, tB, tBs, tO, tO, tO, gd, dev.sms, stream));
+
+    }
 
     MOK_TRY(mark_fwd(4, stream));
     combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(st.O, st.topk_w,
@@ -552,6 +612,7 @@ int moe_fwd(const moe_cfg *cfg, const void *x, const moe_params *params, void *y
     const DeviceInfo *dev = device_info();
     if (!dev) return MOK_ERR_DEVICE;
     const bool training = save_for_backward != 0;
+    if (training && cfg->dtype == MOK_DTYPE_MXFP8) return fail(MOK_ERR_UNSUPPORTED, "MXFP8 is forward-only (no saved state)");
     void *buf = training ? ctx : scratch;
     const size_t have = training ? ctx_bytes : scratch_bytes;
     const State need = carve_state(*cfg, nullptr, training);

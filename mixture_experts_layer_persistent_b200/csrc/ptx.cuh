@@ -1,5 +1,5 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarriers, TMA tiles,
-// cp.async, tcgen05 (TMEM allocation, UMMA issue/commit, TMEM loads) and the
+// cp.async, tcgen05 (including the block-scaled MXFP8 MMA and tcgen05.cp) (TMEM allocation, UMMA issue/commit, TMEM loads) and the
 // shared-memory / instruction descriptors those take.
 #pragma once
 #include <cstdint>
@@ -122,6 +122,12 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 // wait until this thread's bulk stores have completed
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// 4-byte asynchronous global->shared copy.
+__device__ __forceinline__ void cp_async4(void *dst_smem, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+
 // 16-byte asynchronous global->shared copy, cached in L2 only.
 __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
 {
@@ -169,6 +175,39 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// D[tmem] (+)= (A * SFA) . (B * SFB)^T with e4m3 A/B and ue8m0 scales per 32
+// K-elements held in TMEM (kind::mxf8f6f4, block scaled, K = 32 per instruction).
+__device__ __forceinline__ void umma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Copy 32 rows x 16 bytes of shared memory (descriptor) into TMEM at taddr,
+// replicated into all four 32-lane quarters (the scale-factor layout the
+// block-scaled MMA reads).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of an unswizzled K-major block whose 16-byte rows are
+// contiguous (8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t smem_desc_plain(uint32_t saddr)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1) << 16;          // leading byte offset (unused: one 16-byte column)
+    d |= static_cast<uint64_t>(128 >> 4) << 32;   // stride byte offset: next 8-row core matrix
+    d |= static_cast<uint64_t>(1) << 46;          // descriptor version for sm_100
+    return d;                                     // layout type 0: no swizzle
 }
 
 // Arrive once on `bar` when all previously issued tcgen05.mma of this thread complete.
@@ -238,6 +277,19 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
            | (static_cast<uint32_t>(b_mn_major) << 16) // B major
            | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
            | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor of kind::mxf8f6f4 block-scaled MMA: e4m3 A and B,
+// ue8m0 scales, fp32 accumulator, K-major operands; sf_id selects the byte of
+// the 32-bit TMEM scale word (the 32-element K block within a 128-element group).
+__host__ __device__ constexpr uint32_t idesc_mxf8(int M, int N, uint32_t sf_id)
+{
+    return (sf_id << 4)                                 // B scale factor id
+           | (0u << 7) | (0u << 10)                     // A, B format: e4m3
+           | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+           | (1u << 23)                                 // scale format: ue8m0
+           | (static_cast<uint32_t>(M >> 4) << 24)      // M / 16
+           | (sf_id << 29);                             // A scale factor id
 }
 
 // ------------------------------------------------------------------ bf16 helpers

@@ -92,3 +92,52 @@ def test_reruns_bit_identical(ran):
             a = g1[k].view(torch.int32) if v.dtype == torch.float32 else g1[k].view(torch.int16)
             b = v.view(torch.int32) if v.dtype == torch.float32 else v.view(torch.int16)
             assert torch.equal(a, b), k
+
+
+# ---------------------------------------------------------------- MXFP8 forward
+MEDIUM_MX = synth.Workload("medium_mx", T=700, H=512, E=16, k=4, I=256, S=1, Is=256, score_fn=1,
+                           n_group=4, topk_group=2, mxfp8=True, backward=False, seed=21)
+
+
+def _mx_params(params):
+    from mixture_experts_layer_persistent_b200 import quantize_mxfp8
+    out = {k: params[k] for k in ("router_w", "e_bias", "logit_bias")}
+    for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
+                        ("ws_down", "ss_down")):
+        if params.get(name) is None:
+            out[name] = out[sname] = None
+            continue
+        out[name], out[sname] = quantize_mxfp8(params[name])
+    return out
+
+
+def _rel_rms(got, want):
+    return float(np.sqrt(np.mean((got - want) ** 2)) / np.sqrt(np.mean(want ** 2)))
+
+
+@pytest.mark.parametrize("wl", [MEDIUM_MX, synth.scaled(MEDIUM_MX, name="medium_mx_softmax", score_fn=0,
+                                                        n_group=1, topk_group=1, S=0, Is=0, T=333,
+                                                        seed=22)], ids=lambda w: w.name)
+def test_mxfp8_forward_matches_oracle(wl):
+    import oracle
+    case = make_case(wl, device="cuda", gen_device="cpu", mx=True)
+    params = _mx_params(case["params"])
+    layer = MoELayer(cfg_for(wl), params, training=False, device=torch.device("cuda"))
+    routing = layer.new_routing()
+    y = layer.forward(case["x"], routing=routing)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    assert np.array_equal(routing["topk_idx"].cpu().numpy(), case["idx"])
+    L = case["L"]
+    for name in ("Wgu", "Wdn", "Wgu_s", "Wdn_s"):
+        if L.arrays.get(name) is not None:
+            a = L.arrays[name].copy()
+            oracle.mx_fakequant_bf16(a)
+            L.set(**{name: a})
+    yo = L.fwd(case["idx"], case["w"])
+    err = _rel_rms(to_np(y), yo)
+    assert err <= 2e-2, err
+    # reruns are bit-identical
+    y2 = layer.forward(case["x"])
+    torch.cuda.synchronize()
+    assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
