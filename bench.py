@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--mx-workload", default="dsv3_mxfp8",
+                    help="MXFP8 forward workload measured after the main one ('' to skip)")
     return ap.parse_args()
 
 
@@ -265,6 +267,17 @@ def main():
     fwd_tps = wl.T / (fwd_ms / 1e3)
     bwd_tps = wl.T / (bwd_ms / 1e3)
 
+    # ---------------- MXFP8 forward (block-scaled e4m3) on its own workload
+    mx = None
+    if args.mx_workload:
+        del layer, grads, params
+        torch.cuda.empty_cache()
+        mx = mxfp8_run(synth.scaled(synth.WORKLOADS[args.mx_workload],
+                                    seed=synth.WORKLOADS[args.mx_workload].seed + 1000 * rank),
+                       dev, K, args.warmup, world, dist, pk)
+        layer = MoELayer(cfg_for(wl), synth.draw_params(wl, dev), training=True, device=dev)
+        grads = layer.new_grads()
+
     # ---------------- end to end through the host-buffer entry points
     e2e = None
     if not args.no_e2e:
@@ -301,11 +314,68 @@ def main():
                 "empty_experts": int((counts == 0).sum()),
             },
             "roofline": roof,
+            "mxfp8": mx,
             "e2e": e2e, "cpu_baseline": cpu,
         }
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()
+
+
+def mxfp8_run(wl, dev, K, warmup, world, dist, pk):
+    """Forward tokens/s of the MXFP8 layer (weights quantised once, outside the timed region)."""
+    import torch
+    from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, moe_trace_events, quantize_mxfp8, synth
+    p = synth.draw_params(wl, dev)
+    params = {k: p[k] for k in ("router_w", "e_bias", "logit_bias")}
+    for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
+                        ("ws_down", "ss_down")):
+        if p.get(name) is None:
+            params[name] = params[sname] = None
+        else:
+            params[name], params[sname] = quantize_mxfp8(p[name])
+            p[name] = None
+    del p
+    torch.cuda.empty_cache()
+    x = synth.draw_x(wl, dev)
+    layer = MoELayer(cfg_for(wl), params, training=False, device=dev)
+    y = torch.empty_like(x)
+    for _ in range(warmup):
+        layer.forward(x, y)
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    fev = [[mk() for _ in range(abi.MOK_FWD_PHASES + 1)] for _ in range(K)]
+    for e in [e for ev in fev for e in ev]:
+        e.record()
+    start, end = mk(), mk()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    start.record()
+    for i in range(K):
+        moe_trace_events([e.cuda_event for e in fev[i]], None)
+        layer.forward(x, y)
+    end.record()
+    torch.cuda.synchronize()
+    moe_trace_events(None, None)
+    status = layer.status()
+    t = torch.tensor([start.elapsed_time(end)], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / K
+    phases = {n: statistics.mean(fev[i][j].elapsed_time(fev[i][j + 1]) for i in range(K))
+              for j, n in enumerate(FWD_PHASES)}
+    flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
+    fp8_peak = 2 * pk["bf16_sustained"]          # measured bf16 x the nominal dense fp8/bf16 ratio
+    gemm_ms = phases["gate_up_gemm"] + phases["down_gemm"]
+    return {"workload": f"{wl.name}: MoE layer fwd MXFP8 (e4m3, 1x32 ue8m0), T={wl.T}, H={wl.H}, E={wl.E}, "
+                        f"top-{wl.k}, I={wl.I}, {wl.S} shared",
+            "tokens_per_s": wl.T * world / (ms / 1e3), "ms_per_fwd": ms, "phases_ms": {k: round(v, 4) for k, v in phases.items()},
+            "layer_tflops": flops / (ms / 1e3) / 1e12,
+            "fp8_peak_tflops": fp8_peak, "fp8_peak_source": "measured sustained bf16 x 2 (nominal fp8/bf16 dense ratio)",
+            "tc_peak_frac": flops / (ms / 1e3) / 1e12 / fp8_peak,
+            "expert_gemm_tc_peak_frac": flops / (gemm_ms / 1e3) / 1e12 / fp8_peak,
+            "device_status": status}
 
 
 def e2e_run(layer, wl, x, dy, grads, K, world, dist):
