@@ -115,10 +115,10 @@ def algorithmic(wl, counts):
     G = E + S
     out = {
         "gate_up_gemm": (4 * H * I * R, wgu + T * H * 2 + R * I * 2 * 2 + R * 2 * I * 2),
-        "down_gemm": (2 * H * I * R, wdn + R * I * 2 + T * (k + S) * H * 2),
+        "down_gemm": (2 * H * I * R, wdn + R * I * 2 + T * (k + S) * H * 4),
         "down_dgrad_gemm": (2 * H * I * R, wdn + T * H * 2 + R * 2 * I * 2 * 2),
         "down_wgrad_gemm": (2 * H * I * R, T * H * 2 + R * I * 2 + G * H * I * 2),
-        "gate_up_dgrad_gemm": (4 * H * I * R, wgu + R * 2 * I * 2 + T * (k + S) * H * 2),
+        "gate_up_dgrad_gemm": (4 * H * I * R, wgu + R * 2 * I * 2 + T * (k + S) * H * 4),
         "gate_up_wgrad_gemm": (4 * H * I * R, R * 2 * I * 2 + T * H * 2 + G * 2 * I * H * 2),
     }
     return out

@@ -13,6 +13,12 @@ __device__ __forceinline__ void unpack8(const uint4 u, float (&v)[8])
     v[4] = bf16_lo(u.z); v[5] = bf16_hi(u.z); v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
 }
 
+__device__ __forceinline__ void load8(const float *p, float (&v)[8])
+{
+    const float4 a = reinterpret_cast<const float4 *>(p)[0], b = reinterpret_cast<const float4 *>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 __device__ __forceinline__ uint4 pack8(const float (&v)[8])
 {
     uint4 u;
@@ -25,7 +31,7 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8])
 
 // y[t] = sum_{j<k} w[t,j] O[t,j] (ascending j) + sum_s O[t,k+s] (ascending s), fp32, -> bf16.
 // Thread = 8 columns of one token (16-byte loads).
-__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16 *__restrict__ O,
+__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ O,
                                                       const float *__restrict__ topk_w,
                                                       __nv_bfloat16 *__restrict__ y, int T, int H, int k, int S)
 {
@@ -35,11 +41,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16 *__res
     const int t = (int)(i / cpr), c = (int)(i % cpr) * 8;
     const int kk = k + S;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const __nv_bfloat16 *row = O + (size_t)t * kk * H + c;
+    const float *row = O + (size_t)t * kk * H + c;
     for (int j = 0; j < kk; ++j) {
         const float w = j < k ? topk_w[(size_t)t * k + j] : 1.0f;
         float v[8];
-        unpack8(*reinterpret_cast<const uint4 *>(row + (size_t)j * H), v);
+        load8(row + (size_t)j * H, v);
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = fmaf(w, v[q], acc[q]);
     }
@@ -52,7 +58,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16 *__res
 // One block of 256 threads per token; each thread sums a fixed column subset,
 // then a fixed-shape tree over threads.
 __global__ void __launch_bounds__(256) slot_grad_kernel(const __nv_bfloat16 *__restrict__ dy,
-                                                        const __nv_bfloat16 *__restrict__ O,
+                                                        const float *__restrict__ O,
                                                         const float *__restrict__ topk_w,
                                                         const float *__restrict__ topk_p, float *__restrict__ dl,
                                                         int T, int H, int k, int S, int score_fn,
@@ -66,13 +72,13 @@ __global__ void __launch_bounds__(256) slot_grad_kernel(const __nv_bfloat16 *__r
 #pragma unroll
     for (int j = 0; j < 16; ++j) g[j] = 0.0f;
     const __nv_bfloat16 *dyr = dy + (size_t)t * H;
-    const __nv_bfloat16 *orow = O + (size_t)t * kk * H;
+    const float *orow = O + (size_t)t * kk * H;
     for (int c = tid * 8; c < H; c += 256 * 8) {
         float d[8];
         unpack8(*reinterpret_cast<const uint4 *>(dyr + c), d);
         for (int j = 0; j < k; ++j) {
             float o[8];
-            unpack8(*reinterpret_cast<const uint4 *>(orow + (size_t)j * H + c), o);
+            load8(orow + (size_t)j * H + c, o);
             float s = g[j];
 #pragma unroll
             for (int q = 0; q < 8; ++q) s = fmaf(d[q], o[q], s);
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(256) drouter_reduce_kernel(const float *__rest
 
 // dx[t] = sum_j dXs[t, j] (ascending j over routed then shared slots)
 //         + sum_{j<k} dl[t, j] router_w[idx[t, j]]   -> bf16.
-__global__ void __launch_bounds__(256) dx_combine_kernel(const __nv_bfloat16 *__restrict__ dXs,
+__global__ void __launch_bounds__(256) dx_combine_kernel(const float *__restrict__ dXs,
                                                          const float *__restrict__ dl,
                                                          const int *__restrict__ topk_idx,
                                                          const float *__restrict__ router_w,
@@ -180,10 +186,10 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const __nv_bfloat16 *__
     const int t = (int)(i / cpr), c = (int)(i % cpr) * 8;
     const int kk = k + S;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const __nv_bfloat16 *row = dXs + (size_t)t * kk * H + c;
+    const float *row = dXs + (size_t)t * kk * H + c;
     for (int j = 0; j < kk; ++j) {
         float v[8];
-        unpack8(*reinterpret_cast<const uint4 *>(row + (size_t)j * H), v);
+        load8(row + (size_t)j * H, v);
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] += v[q];
     }

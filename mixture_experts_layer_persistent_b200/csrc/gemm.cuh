@@ -67,7 +67,7 @@ struct GemmArgs {
     __nv_bfloat16 *out_s;         // EPI_WGRAD: output of the shared groups
     __nv_bfloat16 *out2;          // EPI_SWIGLU: saved gate/up pre-activations [R, 2I] (or null)
     __nv_bfloat16 *out3;          // EPI_SWIGLU: w * h [R, I] (or null)
-    float *out_f32;               // EPI_ROUTER: partial logits [n_tiles, rows, 256]
+    float *out_f32;               // EPI_ROUTER: partial logits [n_tiles, rows, 256]; EPI_PUSH: fp32 slot rows
     const __nv_bfloat16 *aux;     // EPI_DSWIGLU: saved gate/up pre-activations [R, 2I]
     int ldo;                      // elements per output row
     int inter;                    // I
@@ -673,16 +673,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                 }
             } else if constexpr (C::EPI == EPI_PUSH) {
+                // fp32 rows pushed into their (token, slot) row of the slot buffer
                 const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
-                __nv_bfloat16 *dst = args.out + (size_t)dst_row * args.ldo + t.nt * C::BN;
+                float *dst = args.out_f32 + (size_t)dst_row * args.ldo + t.nt * C::BN;
 #pragma unroll 1
-                for (int c = 0; c < C::BN; c += 64) {
-                    float v[64];
+                for (int c = 0; c < C::BN; c += 32) {
+                    float v[32];
                     uint32_t p[32];
-                    tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
-                    tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                    tmem_ld32(taddr + c, v);
                     tmem_ld_wait();
-                    pack_bf16<64>(v, p);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
                     if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
                     else if (valid) store_row_direct(dst + c, p);
                 }

@@ -166,7 +166,8 @@ struct State {
     int *all_rows;
     float *topk_w, *topk_p, *row_w, *rpart;
     __nv_bfloat16 *wr3;
-    __nv_bfloat16 *gu, *h, *hw, *O;
+    __nv_bfloat16 *gu, *h, *hw;
+    float *O;                       // per-(token, slot) rows, fp32
     uint8_t *xq, *xs, *hq, *hs;     // MXFP8 operands
     size_t bytes;
 };
@@ -204,14 +205,14 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
         st.h = cv.take<__nv_bfloat16>(s.R * s.I);
         st.hq = st.hs = st.xq = st.xs = nullptr;
     }
-    st.O = cv.take<__nv_bfloat16>(s.T * s.kk * s.H);
+    st.O = cv.take<float>(s.T * s.kk * s.H);
     st.bytes = align_up(cv.off, 256);
     return st;
 }
 
 struct BwdScratch {
-    float *dl, *partial;
-    __nv_bfloat16 *dgu, *dxs;
+    float *dl, *partial, *dxs;    // dxs: per-(token, slot) dx rows, fp32
+    __nv_bfloat16 *dgu;
     size_t bytes;
 };
 
@@ -223,7 +224,7 @@ BwdScratch carve_bwd(const moe_cfg &c, void *buf)
     b.dl = cv.take<float>(s.TK);
     b.partial = cv.take<float>(s.max_chunks * s.H);
     b.dgu = cv.take<__nv_bfloat16>(s.R * 2 * s.I);
-    b.dxs = cv.take<__nv_bfloat16>(s.T * s.kk * s.H);
+    b.dxs = cv.take<float>(s.T * s.kk * s.H);
     b.bytes = align_up(cv.off, 256);
     return b;
 }
@@ -369,13 +370,14 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 128, 256, 1)) return MOK_ERR_INVALID;
         if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 128, 256, 1))
             return MOK_ERR_INVALID;
-        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 32, 1, 4)) return MOK_ERR_INVALID;
         GemmArgs gd = ga;
         gd.n_tiles = c.H / 256;
         gd.num_kb = c.I / 128;
         gd.b_rows_per_group = c.H;
         gd.b_half = 0;
-        gd.out = st.O;
+        gd.out = nullptr;
+        gd.out_f32 = st.O;
         gd.out_scales = nullptr;
         gd.ldo = c.H;
         gd.gather_src = nullptr;
@@ -427,12 +429,13 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         gd.num_kb = c.I / BK;
         gd.b_rows_per_group = c.H;
         gd.b_half = 0;
-        gd.out = st.O;
+        gd.out = nullptr;
+        gd.out_f32 = st.O;
         gd.out2 = gd.out3 = nullptr;
         gd.ldo = c.H;
         using CDown = GemmCfg<256, false, false, false, false, false, EPI_PUSH>;
         MOK_TRY(mark_fwd(3, stream));
-        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 32, 1, 4)) return MOK_ERR_INVALID;
         MOK_TRY(launch_gemm<CDown>(tA, tB, tBs, tO, tO, tO, gd, dev.sms, stream));
 
     }
@@ -541,11 +544,11 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g3.n_tiles = c.H / 256;
     g3.num_kb = 2 * c.I / BK;
     g3.b_rows_per_group = 2 * c.I;
-    g3.out = bs.dxs;
+    g3.out_f32 = bs.dxs;
     g3.ldo = c.H;
     using CDgradGU = GemmCfg<256, false, true, false, false, false, EPI_PUSH>;
     MOK_TRY(mark_bwd(5, stream));
-    if (!make_tmap(&tO, bs.dxs, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&tO, bs.dxs, s.H, s.T * s.kk, 32, 1, 4)) return MOK_ERR_INVALID;
     MOK_TRY(launch_gemm<CDgradGU>(tA, tB, tBs, tO, tO, tO, g3, dev.sms, stream));
 
     // wgrad of gate/up: dW_gate_up[g] = sum_r dGU_r^T x[token r]

@@ -26,10 +26,11 @@
  *
  * Rounding mirrors.  Unless cfg->pure is set, the oracle rounds to bf16
  * (round-to-nearest-even, computed directly from fp64) exactly where the
- * layer stores a tensor: h, the per-(token, slot) rows o, y, the saved
- * gate/up pre-activations read by the backward, the weighted h used by the
- * down-projection weight gradient, dGU, the per-slot dx rows, dx and the
- * weight gradients.  In MXFP8 mode x and h are quantised with the 1x32 ue8m0
+ * layer stores a tensor in bf16: h, y, the saved gate/up pre-activations read
+ * by the backward, the weighted h used by the down-projection weight
+ * gradient, dGU, dx and the weight gradients.  The per-(token, slot) rows of
+ * the forward (o) and of the backward (per-slot dx) are stored in fp32, so
+ * they are not rounded.  In MXFP8 mode x and h are quantised with the 1x32 ue8m0
  * block rule below; weights are fake-quantised by the caller with
  * orc_mx_fakequant_bf16 before use.
  *
@@ -404,13 +405,13 @@ static void swiglu_h(const orc_cfg *c, const double *g, const double *u, int I, 
     }
 }
 
-/* o = h Wd^T, stored (mirrored) as bf16 */
+/* o = h Wd^T (the per-(token, slot) rows are stored in fp32: no bf16 mirror) */
 static void down(const orc_cfg *c, const slot_w *s, const double *h, double *o)
 {
     for (int n = 0; n < c->H; n++) {
         double a = 0.0;
         for (int i = 0; i < s->I; i++) a += h[i] * ld(s->Wdn, s->dn_off + (int64_t)n * s->I + i, c->w_kind);
-        o[n] = mirror(c, a);
+        o[n] = a;
     }
 }
 
@@ -537,7 +538,7 @@ int orc_bwd_tokens(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, c
             for (int q = 0; q < H; q++) {
                 double a = 0.0;
                 for (int i = 0; i < 2 * s.I; i++) a += dgu[i] * ld(s.Wgu, s.gu_off + (int64_t)i * H + q, c->w_kind);
-                acc[q] += mirror(c, a);
+                acc[q] += a;                      /* per-slot dx rows are stored in fp32 */
             }
         }
         dlogits_token(c, prob, id, ww, G, dl);

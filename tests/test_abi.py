@@ -31,9 +31,9 @@ def test_workspace_sizes_and_argument_checks():
     T, H, I, kk = 4096, 7168, 2048, 9
     R = T * kk
     # ctx holds at least g,u, h, w*h and the per-slot rows
-    assert ctx >= R * 2 * I * 2 + 2 * R * I * 2 + T * kk * H * 2
-    assert fwd >= R * I * 2 + T * kk * H * 2 and fwd < ctx
-    assert bwd >= R * 2 * I * 2 + T * kk * H * 2
+    assert ctx >= R * 2 * I * 2 + 2 * R * I * 2 + T * kk * H * 4
+    assert fwd >= R * I * 2 + T * kk * H * 4 and fwd < ctx
+    assert bwd >= R * 2 * I * 2 + T * kk * H * 4
     bad = [make_cfg(64, 200, 8, 128, 2), make_cfg(64, 256, 8, 100, 2), make_cfg(64, 256, 8, 128, 9),
            make_cfg(64, 256, 300, 128, 2), make_cfg(0, 256, 8, 128, 2),
            make_cfg(64, 256, 8, 128, 2, score_fn=1, n_group=3, topk_group=1)]
