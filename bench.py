@@ -139,7 +139,8 @@ def oracle_sample(wl, params, x, dy, seconds, log=None):
     L.fwd(idx, w, tokens=[0])
     L.bwd(idx, w, tokens=[0])
     one = time.perf_counter() - t0
-    n = int(max(1, min(wl.T, seconds / max(one, 1e-6))))
+    cores = oracle.num_threads()          # the oracle parallelises over tokens
+    n = int(max(cores, min(wl.T, cores * int(seconds / max(one, 1e-6)))))
     toks = np.arange(n, dtype=np.int32)
     t0 = time.perf_counter()
     gap = np.zeros(wl.T)
@@ -267,17 +268,6 @@ def main():
     fwd_tps = wl.T / (fwd_ms / 1e3)
     bwd_tps = wl.T / (bwd_ms / 1e3)
 
-    # ---------------- MXFP8 forward (block-scaled e4m3) on its own workload
-    mx = None
-    if args.mx_workload:
-        del layer, grads, params
-        torch.cuda.empty_cache()
-        mx = mxfp8_run(synth.scaled(synth.WORKLOADS[args.mx_workload],
-                                    seed=synth.WORKLOADS[args.mx_workload].seed + 1000 * rank),
-                       dev, K, args.warmup, world, dist, pk)
-        layer = MoELayer(cfg_for(wl), synth.draw_params(wl, dev), training=True, device=dev)
-        grads = layer.new_grads()
-
     # ---------------- end to end through the host-buffer entry points
     e2e = None
     if not args.no_e2e:
@@ -285,7 +275,15 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_sample(wl, {k2: v for k2, v in params.items()}, x, dy, args.cpu_seconds)
+        cpu = oracle_sample(wl, params, x, dy, args.cpu_seconds)
+
+    # ---------------- MXFP8 forward (block-scaled e4m3) on its own workload
+    mx = None
+    if args.mx_workload:
+        del layer, grads, params
+        torch.cuda.empty_cache()
+        mwl = synth.WORKLOADS[args.mx_workload]
+        mx = mxfp8_run(synth.scaled(mwl, seed=mwl.seed + 1000 * rank), dev, K, args.warmup, world, dist, pk)
 
     if rank == 0:
         line = {
