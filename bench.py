@@ -46,7 +46,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--mx-workload", default="dsv3_mxfp8",
-                    help="MXFP8 forward workload measured after the main one ('' to skip)")
+                    help="MXFP8 forward workload measured after the main one ('none' to skip)")
     return ap.parse_args()
 
 
@@ -279,7 +279,7 @@ def main():
 
     # ---------------- MXFP8 forward (block-scaled e4m3) on its own workload
     mx = None
-    if args.mx_workload:
+    if args.mx_workload and args.mx_workload != "none":
         del layer, grads, params
         torch.cuda.empty_cache()
         mwl = synth.WORKLOADS[args.mx_workload]
