@@ -104,6 +104,22 @@ class Clocks:
                 "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ replicas
+def replica_throughput(ms_local: float, tokens_local: int, dist=None, device=None):
+    """Whole-job throughput of independent replicas: every rank's tokens over the
+    slowest rank's time (max over ranks).  Returns (tokens/s, max ms, total tokens)."""
+    import torch
+    t = torch.tensor([ms_local, float(tokens_local)], dtype=torch.float64, device=device)
+    if dist is not None and dist.is_initialized() and dist.get_world_size() > 1:
+        mx = t[:1].clone()
+        dist.all_reduce(mx, op=dist.ReduceOp.MAX)
+        tok = t[1:].clone()
+        dist.all_reduce(tok, op=dist.ReduceOp.SUM)
+        t = torch.cat([mx, tok])
+    ms, tokens = float(t[0]), int(t[1])
+    return tokens / (ms / 1e3), ms, tokens
+
+
 # ------------------------------------------------------------------ algorithmic counts
 def algorithmic(wl, counts):
     """FLOPs and bytes of each GEMM phase (per launch) from the routing counts."""
@@ -228,11 +244,7 @@ def main():
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
-    ms = start.elapsed_time(end)
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    value, ms_max, _ = replica_throughput(start.elapsed_time(end), wl.T * K, dist, dev)
     status = layer.status()
 
     phase = {}
@@ -263,8 +275,6 @@ def main():
     roof["algorithmic_bytes"] = nbytes
 
     total_flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
-    tokens = wl.T * world
-    value = tokens * K / (ms_max / 1e3)
     fwd_tps = wl.T / (fwd_ms / 1e3)
     bwd_tps = wl.T / (bwd_ms / 1e3)
 
