@@ -196,6 +196,35 @@ int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *
 #define MOK_BWD_PHASES 8
 int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events, int n_bwd);
 
+/*
+ * Forward pass that allocates nothing and takes no workspace.
+ *
+ * The pages describe no such call; it exists for callers that cannot hand the
+ * layer a device buffer: runtimes that plan every byte of device memory ahead
+ * of time and forbid allocation once running, plug-in hosts that give a layer
+ * only its inputs and outputs, and processes whose device memory is already
+ * fully reserved by another allocator.
+ *
+ * It runs the same kernels as moe_fwd without saved state (inference; BF16 or
+ * MXFP8), with its intermediate buffers placed in one static device array of
+ * MOK_STATIC_SCRATCH_BYTES that the library declares at file scope.  Every GPU
+ * that loads the library holds that array until the process exits.
+ *   - x, y and the parameters are device pointers as for moe_fwd; the caller
+ *     still owns them.
+ *   - Shapes whose forward scratch (the fwd_scratch_bytes of
+ *     moe_workspace_size) exceeds MOK_STATIC_SCRATCH_BYTES are rejected with
+ *     MOK_ERR_WORKSPACE before anything is enqueued.
+ *   - The first call on a device looks up the array's device address (a host
+ *     runtime call); make that first call before any stream capture.
+ *   - All calls on a device share the one array, and each call overwrites what
+ *     the previous one left there (nothing in it needs to start at zero).  Two
+ *     calls that overlap on the GPU, from different streams or threads, race on
+ *     it: serialise them.
+ * No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define MOK_STATIC_SCRATCH_BYTES (32u << 20)
+int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, void *y, void *stream);
+
 /* Synchronise `stream`, then read and clear the device status word of the
  * current device (MOK_STATUS_* bits) into *device_status. */
 int moe_status(void *stream, int32_t *device_status);

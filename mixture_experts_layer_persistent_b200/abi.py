@@ -27,6 +27,7 @@ MOK_DTYPE_BF16 = 0
 MOK_DTYPE_MXFP8 = 1
 MOK_FWD_PHASES = 5
 MOK_BWD_PHASES = 8
+MOK_STATIC_SCRATCH_BYTES = 32 << 20
 
 _i32, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -83,13 +84,14 @@ def lib():
         L.moe_quantize_mxfp8.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
         L.moe_status.argtypes = [_vp, P(_i32)]
         L.moe_trace_events.argtypes = [P(_vp), ctypes.c_int, P(_vp), ctypes.c_int]
+        L.moe_fwd_static.argtypes = [P(moe_cfg), _vp, P(moe_params), _vp, _vp]
         L.moe_strerror.argtypes = [ctypes.c_int]
         L.moe_strerror.restype = ctypes.c_char_p
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
                      "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_status",
-                     "moe_trace_events"):
+                     "moe_trace_events", "moe_fwd_static"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -162,3 +164,8 @@ def moe_trace_events(fwd_events, bwd_events):
     ba = (_vp * len(bwd_events))(*bwd_events) if bwd_events else None
     _check("moe_trace_events", lib().moe_trace_events(fa, len(fwd_events or ()), ba,
                                                       len(bwd_events or ())))
+
+
+def moe_fwd_static(cfg, x, params, y, stream):
+    """Forward pass using the library's static scratch (no workspace argument)."""
+    _check("moe_fwd_static", lib().moe_fwd_static(ctypes.byref(cfg), x, ctypes.byref(params), y, stream))

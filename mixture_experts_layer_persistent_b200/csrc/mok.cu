@@ -19,6 +19,11 @@ namespace mok {
 
 __device__ int g_status;   // device status word (MOK_STATUS_* bits)
 
+// Scratch of moe_fwd_static: the library's own storage, so that callers who
+// cannot allocate still get a forward pass.  Host code must not use the symbol
+// itself as a pointer; it looks up the device address once per device.
+static __device__ __align__(256) unsigned char g_static_scratch[MOK_STATIC_SCRATCH_BYTES];
+
 namespace {
 
 constexpr int kChunkRows = 256;   // router-gradient row chunk
@@ -743,6 +748,39 @@ int moe_status(void *stream, int32_t *device_status)
     if (const cudaError_t e_ = cudaMemcpyToSymbol(g_status, &zero, sizeof(int)); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyToSymbol", e_);
     *device_status = v;
     return MOK_OK;
+}
+
+int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, void *y, void *stream)
+{
+    MOK_TRY(check_cfg(cfg));
+    MOK_TRY(check_params(*cfg, params));
+    if (!x || !y || !aligned16(x) || !aligned16(y)) return fail(MOK_ERR_INVALID, "moe_fwd_static: x or y");
+    const size_t need = carve_state(*cfg, nullptr, false).bytes;
+    if (need > MOK_STATIC_SCRATCH_BYTES) {
+        snprintf(t_last_error, sizeof(t_last_error),
+                 "moe_fwd_static: this shape needs %zu bytes of scratch; the static scratch holds %u bytes",
+                 need, MOK_STATIC_SCRATCH_BYTES);
+        return MOK_ERR_WORKSPACE;
+    }
+    const DeviceInfo *dev = device_info();
+    if (!dev) return MOK_ERR_DEVICE;
+    // once per device, with that device current: the array's device address
+    static void *s_static_ptr[kMaxDevices] = {};
+    int d = 0;
+    if (const cudaError_t e = cudaGetDevice(&d); e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaGetDevice", e);
+    void *ptr = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!s_static_ptr[d]) {
+            void *p = nullptr;
+            if (const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch); e != cudaSuccess)
+                return fail(MOK_ERR_LAUNCH, "cudaGetSymbolAddress(static scratch)", e);
+            s_static_ptr[d] = p;
+        }
+        ptr = s_static_ptr[d];
+    }
+    const State st = carve_state(*cfg, ptr, false);
+    return forward(*cfg, x, *params, y, nullptr, st, *dev, false, static_cast<cudaStream_t>(stream));
 }
 
 const char *moe_last_error(void) { return t_last_error; }
