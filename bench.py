@@ -140,6 +140,23 @@ def algorithmic(wl, counts):
     return out
 
 
+def measured_traffic(wl, phase):
+    """DRAM bytes per launch of `phase` from the committed ncu capture, or None
+    when the workload differs or the kernel sources changed since the capture."""
+    import glob
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic_dsv3.json")
+    if wl.name != "dsv3" or not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "mixture_experts_layer_persistent_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    if h.hexdigest() != rec["source_sha256"]:
+        return None
+    return rec["per_launch_bytes"].get(phase)
+
+
 # ------------------------------------------------------------------ CPU oracle sample
 def oracle_sample(wl, params, x, dy, seconds, log=None):
     """Time the fp64 oracle's forward + dx backward on a token sample of the workload."""
@@ -268,7 +285,7 @@ def main():
         roof = {"bound": "tensor", "achieved": flops / t_dom / 1e12, "peak": pk["bf16_sustained"],
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(wl, dom)
     roof["kernel"] = dom
     roof["peak_source"] = pk["source"] + (" sustained bf16" if roof["bound"] == "tensor" else " hbm copy")
     roof["algorithmic_flops"] = flops
