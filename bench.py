@@ -324,7 +324,9 @@ def main():
                                    + (f", Zipf({wl.zipf}) logit term" if wl.zipf else ""),
                        "tokens_per_gpu": wl.T, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (22.6 GB expert weights streamed per pass)"},
-            "gpu_launches": K * (len(FWD_PHASES) + len(BWD_PHASES)),
+            # forward: router split, router GEMM, select, 3 dispatch kernels, gate/up, down,
+            # combine (9); backward: slot grad, 2 router-gradient kernels, 4 GEMMs, dx sum (8)
+            "gpu_launches": K * (9 + 8),
             "clocks": clk, "device_status": status,
             "phases_ms": {k2: round(v, 4) for k2, v in phase.items()},
             "breakdown": {

@@ -90,18 +90,28 @@ struct GemmCfg {
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int SF_BYTES = MX ? 512 + BN * 4 : 0;       // SFA (128 rows) + SFB (BN rows), 4 bytes each
-    static constexpr int STAGES = BN == 256 ? 4 : 6;
+    // Tuning: weight-streaming kernels want a deep operand ring; MXFP8 (single
+    // accumulator buffer) and the weight gradients (short K per tile) want the
+    // epilogue to overlap its stores, so they trade a stage for a second
+    // staging buffer, and the weight gradients split each tile's columns over
+    // eight epilogue warps (two per TMEM lane quarter).
+    static constexpr int STAGES = (MX || RAGGED_K) ? 3 : (BN == 256 ? 4 : 5);
+    static constexpr int EPI_BUFS = (BN == 256 && !MX && !RAGGED_K) ? 1 : 2;
+    static constexpr int EPI_WARPS = RAGGED_K ? 8 : 4;
     static constexpr int PULL_WARPS = (A_GATHER || B_GATHER || MX) ? 4 : 0;   // cp.async warps
-    static constexpr int THREADS = 192 + 32 * PULL_WARPS;
+    static constexpr int PULL_WARP0 = 2 + EPI_WARPS;
+    static constexpr int THREADS = 64 + 32 * (EPI_WARPS + PULL_WARPS);
     static constexpr int GATHER_BYTES = A_GATHER ? A_BYTES : (B_GATHER ? B_BYTES : 0);
     static constexpr int TMA_BYTES = STAGE_BYTES - GATHER_BYTES;
     static constexpr int ACC_BUFS = MX ? 1 : 2;                  // MXFP8 needs TMEM columns for the scales
     static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
     static constexpr int SF_TMEM_COL = 256;                      // SFA at 256..259, SFB at 260..
-    static constexpr int EPI_STAGE_BYTES = 4 * 4096;             // one 32 x 128-byte block per epilogue warp
+    static constexpr int EPI_STAGE_BYTES = EPI_WARPS * EPI_BUFS * 4096;   // 32 x 128-byte blocks per epilogue warp
     static constexpr int AUX_BYTES = 256 + 3 * kMaxGroups * 4;
-    static constexpr int SMEM_BYTES =
-        1024 + STAGES * STAGE_BYTES + STAGES * SF_BYTES + EPI_STAGE_BYTES + AUX_BYTES;
+    // the epilogue staging blocks follow the scale region and must stay 1024-byte
+    // aligned (their 128-byte swizzle phase comes from the address)
+    static constexpr int SF_REGION = (STAGES * SF_BYTES + 1023) / 1024 * 1024;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + SF_REGION + EPI_STAGE_BYTES + AUX_BYTES;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
     static_assert(!MX || (!A_MN && !B_MN && !RAGGED_K && BN == 256 && (EPI == EPI_SWIGLU || EPI == EPI_PUSH)),
                   "MXFP8 serves the forward expert GEMMs");
@@ -109,6 +119,7 @@ struct GemmCfg {
     static_assert(!RAGGED_K || (A_MN && B_MN), "weight gradients take both operands MN-major");
     static_assert(!RAGGED_K || (A_GATHER != B_GATHER), "one operand of a weight gradient is gathered");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert((STAGES * STAGE_BYTES) % 1024 == 0, "stage ring keeps 1024-byte alignment");
 };
 
 struct Tile {
@@ -179,9 +190,24 @@ __device__ __forceinline__ void pack_bf16(const float *v, uint32_t *p)
 // chunk c ^ (r & 7)), so the TMA store engine writes whole lines while the
 // warp moves on; the stores stay in flight without occupying the warp.
 
-__device__ __forceinline__ void stage_block(uint32_t *stg, const uint32_t *p, int lane)
+// Two staging buffers per warp alternate: before a buffer is rewritten, the
+// store issued from it two blocks earlier must have read it (at most one store
+// group, the other buffer's, may still be reading).
+struct EpiStage {
+    uint32_t *buf;      // bufs x 1024 words
+    int bufs;           // 1 or 2
+    int n;              // blocks staged so far
+    __device__ __forceinline__ uint32_t *next() { return buf + ((n++ & (bufs - 1)) << 10); }
+};
+
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
+__device__ __forceinline__ void stage_block(const EpiStage &es, uint32_t *stg, const uint32_t *p, int lane)
 {
-    if (lane == 0) bulk_wait_read0();     // the previous store from this buffer has read it
+    if (lane == 0) {                      // the store that last used this buffer has read it
+        if (es.bufs == 2) bulk_wait_read1();
+        else bulk_wait_read0();
+    }
     __syncwarp();
 #pragma unroll
     for (int c = 0; c < 8; ++c)
@@ -192,10 +218,11 @@ __device__ __forceinline__ void stage_block(uint32_t *stg, const uint32_t *p, in
 }
 
 // 32 full rows to rows row0..row0+31 of a row-major tensor, starting at column col
-__device__ __forceinline__ void store_block_tile(uint32_t *stg, const uint32_t *p, int lane, const CUtensorMap *tm,
+__device__ __forceinline__ void store_block_tile(EpiStage &es, const uint32_t *p, int lane, const CUtensorMap *tm,
                                                  int col, int row0)
 {
-    stage_block(stg, p, lane);
+    uint32_t *stg = es.next();
+    stage_block(es, stg, p, lane);
     if (lane == 0) {
         tma_store_2d(tm, stg, col, row0);
         bulk_commit();
@@ -203,10 +230,11 @@ __device__ __forceinline__ void store_block_tile(uint32_t *stg, const uint32_t *
 }
 
 // 32 full rows, row `lane` to row dst_row (this lane's value), starting at column col
-__device__ __forceinline__ void store_block_scatter(uint32_t *stg, const uint32_t *p, int lane, const CUtensorMap *tm,
+__device__ __forceinline__ void store_block_scatter(EpiStage &es, const uint32_t *p, int lane, const CUtensorMap *tm,
                                                     int col, int dst_row)
 {
-    stage_block(stg, p, lane);
+    uint32_t *stg = es.next();
+    stage_block(es, stg, p, lane);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
         const int r0 = __shfl_sync(0xffffffffu, dst_row, 4 * q + 0);
@@ -227,9 +255,10 @@ __device__ __forceinline__ void store_row_direct(void *dst, const uint32_t *p)
 }
 
 // cooperative load of 32 rows x 128 bytes (row `lane` from src, null = zeros) into p
-__device__ __forceinline__ void load_block(uint32_t *stg, uint32_t *p, const void *src, int lane)
+__device__ __forceinline__ void load_block(EpiStage &es, uint32_t *p, const void *src, int lane)
 {
-    if (lane == 0) bulk_wait_read0();
+    uint32_t *stg = es.next();
+    if (lane == 0) bulk_wait_read0();     // loads commit no store group: wait for every store to have read
     __syncwarp();
     const uint64_t d = reinterpret_cast<uint64_t>(src);
 #pragma unroll
@@ -261,7 +290,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *tiles = smem;
     uint8_t *sf_tiles = tiles + C::STAGES * C::STAGE_BYTES;     // MXFP8 scale blocks, one per stage
-    uint32_t *epi_stage = reinterpret_cast<uint32_t *>(sf_tiles + C::STAGES * C::SF_BYTES);
+    uint32_t *epi_stage = reinterpret_cast<uint32_t *>(sf_tiles + C::SF_REGION);
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(epi_stage) + C::EPI_STAGE_BYTES);
     uint64_t *empty_bar = full_bar + C::STAGES;
     uint64_t *accf = empty_bar + C::STAGES;
@@ -307,7 +336,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
             for (int b = 0; b < 2; ++b) {
                 mbar_init(&accf[b], 1);
-                mbar_init(&acce[b], 128);
+                mbar_init(&acce[b], 32 * C::EPI_WARPS);
             }
             *abort_flag = 0;
             fence_barrier_init();
@@ -384,13 +413,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
         }
     producer_done:;
-    } else if (warp >= 6) {
+    } else if (warp >= C::PULL_WARP0) {
         // ------------------------------------------------------------ pull warps
         // Gathered operand: each 128-byte row is copied by index from the token
         // matrix with 16-byte cp.async into the 128-byte-swizzled layout the MMA
         // descriptors expect (16-byte chunk c of row r lands at chunk c ^ (r & 7)).
         if constexpr (C::PULL_WARPS > 0) {
-            const int p = threadIdx.x - 192;
+            const int p = threadIdx.x - 32 * C::PULL_WARP0;
             const int c16 = p & 7;
             const int r0 = p >> 3;                      // 0..15
             const uint8_t *src = reinterpret_cast<const uint8_t *>(args.gather_src);
@@ -583,7 +612,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // ------------------------------------------------------------ epilogue
         const int eq = warp & 3;                 // TMEM lane quarter this warp may access
         const int row = eq * 32 + lane;          // tile row of this thread
-        uint32_t *stg = reinterpret_cast<uint32_t *>(epi_stage) + (warp - 2) * 1024;
+        const int ew = warp - 2;                 // epilogue warp index
+        EpiStage stg{reinterpret_cast<uint32_t *>(epi_stage) + ew * C::EPI_BUFS * 1024, C::EPI_BUFS, 0};
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -691,20 +721,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const bool routed = t.g < args.num_routed;
                 const int gl = routed ? t.g : t.g - args.num_routed;
                 const int grow0 = gl * args.m_tiles * BM + t.m0 + eq * 32;   // row in the [groups * M, N] view
+                constexpr int COLS = C::BN * 4 / C::EPI_WARPS;               // columns of this warp
+                const int c0 = (ew >> 2) * COLS;
+                float v[64];
+                if (t.nkb > 0) {
+                    tmem_ld32(taddr + c0, *reinterpret_cast<float(*)[32]>(v));
+                    tmem_ld32(taddr + c0 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                    tmem_ld_wait();
+                }
 #pragma unroll 1
-                for (int c = 0; c < C::BN; c += 64) {
-                    float v[64];
+                for (int c = c0; c < c0 + COLS; c += 64) {
                     uint32_t p[32];
                     if (t.nkb > 0) {
-                        tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
-                        tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-                        tmem_ld_wait();
+                        pack_bf16<64>(v, p);
+                        if (c + 64 < c0 + COLS) {          // next block's TMEM load overlaps this block's store
+                            tmem_ld32(taddr + c + 64, *reinterpret_cast<float(*)[32]>(v));
+                            tmem_ld32(taddr + c + 96, *reinterpret_cast<float(*)[32]>(v + 32));
+                        }
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 64; ++i) v[i] = 0.0f;
+                        for (int i = 0; i < 32; ++i) p[i] = 0u;
                     }
-                    pack_bf16<64>(v, p);
                     store_block_tile(stg, p, lane, routed ? &tmO : &tmO2, t.nt * C::BN + c, grow0);
+                    if (t.nkb > 0 && c + 64 < c0 + COLS) tmem_ld_wait();
                 }
             } else if constexpr (C::EPI == EPI_DSWIGLU) {
                 const int r = t.m0 + row;

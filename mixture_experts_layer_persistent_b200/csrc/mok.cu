@@ -169,6 +169,7 @@ Shapes shapes(const moe_cfg &c)
 struct State {
     int *topk_idx, *counts, *offsets, *gorder, *chunk_start, *perm, *inv_perm, *row_token, *row_slot;
     int *all_rows;
+    int *hist;                      // [dispatch chunks, E] per-chunk counts, then base rows
     float *topk_w, *topk_p, *row_w, *rpart;
     __nv_bfloat16 *wr3;
     __nv_bfloat16 *gu, *h, *hw;
@@ -196,6 +197,7 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
     st.row_slot = cv.take<int>(s.R);
     st.row_w = cv.take<float>(s.R);
     st.all_rows = cv.take<int>(2);
+    st.hist = cv.take<int>(((s.T + kDispatchChunk - 1) / kDispatchChunk) * s.E);
     st.wr3 = cv.take<__nv_bfloat16>(s.E * 3 * s.H);
     st.rpart = cv.take<float>(static_cast<size_t>(s.n_split) * s.T * 256);
     st.gu = training ? cv.take<__nv_bfloat16>(s.R * 2 * s.I) : nullptr;
@@ -331,9 +333,17 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     da.counts = st.counts; da.offsets = st.offsets; da.gorder = st.gorder; da.chunk_start = st.chunk_start;
     da.perm = st.perm; da.inv_perm = st.inv_perm; da.row_token = st.row_token; da.row_slot = st.row_slot;
     da.row_w = st.row_w;
+    da.hist = st.hist;
     MOK_TRY(mark_fwd(1, stream));
-    dispatch_kernel<<<1, 1024, 0, stream>>>(da);
-    MOK_LAUNCHED();
+    {
+        const int n_chunks = static_cast<int>((s.T + kDispatchChunk - 1) / kDispatchChunk);
+        dispatch_count_kernel<<<n_chunks, 1024, 0, stream>>>(da);
+        MOK_LAUNCHED();
+        dispatch_scan_kernel<<<1, 256, 0, stream>>>(da, n_chunks);
+        MOK_LAUNCHED();
+        dispatch_place_kernel<<<n_chunks, 1024, 0, stream>>>(da);
+        MOK_LAUNCHED();
+    }
 
     if (mx) {
         // MXFP8: quantise x (1x32 ue8m0 blocks along H), then block-scaled expert GEMMs

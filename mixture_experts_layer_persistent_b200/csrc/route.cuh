@@ -188,6 +188,7 @@ struct DispatchArgs {
     const float *topk_w;   // [T, k]
     int T, k, E, S;
     int chunk_rows;        // row chunk of the router-gradient partial sums
+    int *hist;             // [C, E] (tokens of chunk c choosing e), then the chunk's base row
     int *counts;           // [E]
     int *offsets;          // [E + S + 1] sorted-row ranges (routed, then shared)
     int *gorder;           // [E + S] groups by rows descending, index ascending
@@ -199,36 +200,61 @@ struct DispatchArgs {
     float *row_w;          // [R]
 };
 
-// One block of 1024 threads: integer counting sort, bit-exact and stable in
-// token order.  Chunks of 1024 tokens: per-expert token bitmasks give each
-// (token, slot) its rank among earlier tokens of the chunk.
-__global__ void __launch_bounds__(1024) dispatch_kernel(const DispatchArgs a)
+constexpr int kDispatchChunk = 1024;   // tokens per chunk (one block of 1024 threads)
+
+// Integer counting sort of the T*k (token, slot) pairs by expert, stable in
+// token order, in three launches: per-chunk histograms, a per-expert scan over
+// chunks and experts, and per-chunk placement.  Every count is an integer, so
+// the result is the same whatever the order of the atomics.
+__global__ void __launch_bounds__(1024) dispatch_count_kernel(const DispatchArgs a)
 {
     __shared__ int s_cnt[256];
-    __shared__ int s_base[256];
-    __shared__ uint32_t s_mask[256][32];
-    const int tid = threadIdx.x;
-    const int E = a.E, k = a.k, T = a.T, kk = a.k + a.S;
-    const long long TK = (long long)T * k;
-    for (int e = tid; e < E; e += 1024) s_cnt[e] = 0;
+    const int c = blockIdx.x, tid = threadIdx.x;
+    for (int e = tid; e < a.E; e += 1024) s_cnt[e] = 0;
     __syncthreads();
-    for (long long i = tid; i < TK; i += 1024) atomicAdd(&s_cnt[a.topk_idx[i]], 1);
+    const int t = c * kDispatchChunk + tid;
+    if (t < a.T)
+        for (int j = 0; j < a.k; ++j) atomicAdd(&s_cnt[a.topk_idx[(size_t)t * a.k + j]], 1);
     __syncthreads();
-    if (tid == 0) {
+    for (int e = tid; e < a.E; e += 1024) a.hist[(size_t)c * a.E + e] = s_cnt[e];
+}
+
+// One block: counts, exclusive offsets, each chunk's first row per expert (in
+// place of its histogram), router-gradient chunk starts and the group order.
+__global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a, int n_chunks)
+{
+    __shared__ int s_cnt[256];
+    __shared__ int s_off[257];
+    const int e = threadIdx.x, E = a.E, T = a.T;
+    int total = 0;
+    if (e < E)
+        for (int c = 0; c < n_chunks; ++c) total += a.hist[(size_t)c * E + e];
+    s_cnt[e] = e < E ? total : 0;
+    __syncthreads();
+    if (e == 0) {
         int acc = 0, cacc = 0;
-        for (int e = 0; e < E; ++e) {
-            a.counts[e] = s_cnt[e];
-            a.offsets[e] = acc;
-            a.chunk_start[e] = cacc;
-            s_base[e] = acc;
-            acc += s_cnt[e];
-            cacc += (s_cnt[e] + a.chunk_rows - 1) / a.chunk_rows;
+        for (int q = 0; q < E; ++q) {
+            s_off[q] = acc;
+            a.counts[q] = s_cnt[q];
+            a.offsets[q] = acc;
+            a.chunk_start[q] = cacc;
+            acc += s_cnt[q];
+            cacc += (s_cnt[q] + a.chunk_rows - 1) / a.chunk_rows;
         }
         a.chunk_start[E] = cacc;
         for (int s = 0; s <= a.S; ++s) a.offsets[E + s] = acc + s * T;
     }
+    __syncthreads();
+    if (e < E) {
+        int run = s_off[e];
+        for (int c = 0; c < n_chunks; ++c) {
+            const int h = a.hist[(size_t)c * E + e];
+            a.hist[(size_t)c * E + e] = run;
+            run += h;
+        }
+    }
     // group order: longest first, lower index on ties
-    for (int g = tid; g < E + a.S; g += 1024) {
+    for (int g = e; g < E + a.S; g += 256) {
         const int cg = g < E ? s_cnt[g] : T;
         int rank = 0;
         for (int h = 0; h < E + a.S; ++h) {
@@ -237,44 +263,43 @@ __global__ void __launch_bounds__(1024) dispatch_kernel(const DispatchArgs a)
         }
         a.gorder[rank] = g;
     }
+}
+
+// Per chunk: per-expert token bitmasks give each (token, slot) its rank among
+// the chunk's earlier tokens of that expert; row = chunk base + rank.
+__global__ void __launch_bounds__(1024) dispatch_place_kernel(const DispatchArgs a)
+{
+    __shared__ uint32_t s_mask[256][32];
+    const int c = blockIdx.x, tid = threadIdx.x;
+    const int E = a.E, k = a.k, kk = a.k + a.S, T = a.T;
+    for (int q = tid; q < E * 32; q += 1024) (&s_mask[0][0])[q] = 0u;
     __syncthreads();
-    for (int c0 = 0; c0 < T; c0 += 1024) {
-        for (int q = tid; q < E * 32; q += 1024) (&s_mask[0][0])[q] = 0u;
-        __syncthreads();
-        const int t = c0 + tid;
-        const int word = tid >> 5, bit = tid & 31;
-        if (t < T)
-            for (int j = 0; j < k; ++j) atomicOr(&s_mask[a.topk_idx[(size_t)t * k + j]][word], 1u << bit);
-        __syncthreads();
-        if (t < T) {
-            for (int j = 0; j < k; ++j) {
-                const int e = a.topk_idx[(size_t)t * k + j];
-                int rank = __popc(s_mask[e][word] & ((1u << bit) - 1u));
-                for (int w = 0; w < word; ++w) rank += __popc(s_mask[e][w]);
-                const int pos = s_base[e] + rank;
-                const int s = t * k + j;
-                a.perm[pos] = s;
-                a.inv_perm[s] = pos;
-                a.row_token[pos] = t;
-                a.row_slot[pos] = t * kk + j;
-                a.row_w[pos] = a.topk_w[s];
-            }
+    const int t = c * kDispatchChunk + tid;
+    const int word = tid >> 5, bit = tid & 31;
+    if (t < T)
+        for (int j = 0; j < k; ++j) atomicOr(&s_mask[a.topk_idx[(size_t)t * k + j]][word], 1u << bit);
+    __syncthreads();
+    if (t < T) {
+        for (int j = 0; j < k; ++j) {
+            const int e = a.topk_idx[(size_t)t * k + j];
+            int rank = __popc(s_mask[e][word] & ((1u << bit) - 1u));
+            for (int w = 0; w < word; ++w) rank += __popc(s_mask[e][w]);
+            const int pos = a.hist[(size_t)c * E + e] + rank;
+            const int sl = t * k + j;
+            a.perm[pos] = sl;
+            a.inv_perm[sl] = pos;
+            a.row_token[pos] = t;
+            a.row_slot[pos] = t * kk + j;
+            a.row_w[pos] = a.topk_w[sl];
         }
-        __syncthreads();
-        for (int e = tid; e < E; e += 1024) {
-            int n = 0;
-            for (int w = 0; w < 32; ++w) n += __popc(s_mask[e][w]);
-            s_base[e] += n;
+        // shared experts: every token, in token order, weight 1
+        const long long TK = (long long)T * k;
+        for (int s = 0; s < a.S; ++s) {
+            const long long pos = TK + (long long)s * T + t;
+            a.row_token[pos] = t;
+            a.row_slot[pos] = t * kk + k + s;
+            a.row_w[pos] = 1.0f;
         }
-        __syncthreads();
-    }
-    // shared experts: every token, in token order, weight 1
-    for (long long r = tid; r < (long long)a.S * T; r += 1024) {
-        const int s = (int)(r / T), t = (int)(r % T);
-        const long long pos = TK + r;
-        a.row_token[pos] = t;
-        a.row_slot[pos] = t * kk + k + s;
-        a.row_w[pos] = 1.0f;
     }
 }
 
