@@ -225,6 +225,16 @@ int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events
 #define MOK_STATIC_SCRATCH_BYTES (32u << 20)
 int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, void *y, void *stream);
 
+/*
+ * Fault-injection hook for testing the bounded waits.  While enabled (non-zero),
+ * every forward launched by this host thread makes CTA 0 of the gate/up GEMM
+ * skip the signal that hands its first accumulator to the epilogue; the
+ * epilogue's wait then runs out after about 2 s, the kernel records
+ * MOK_STATUS_TIMEOUT and returns (no trap, no fault).  Results of such a call
+ * are meaningless.  Off by default.
+ */
+int moe_test_drop_signal(int enable);
+
 /* Synchronise `stream`, then read and clear the device status word of the
  * current device (MOK_STATUS_* bits) into *device_status. */
 int moe_status(void *stream, int32_t *device_status);

@@ -85,13 +85,14 @@ def lib():
         L.moe_status.argtypes = [_vp, P(_i32)]
         L.moe_trace_events.argtypes = [P(_vp), ctypes.c_int, P(_vp), ctypes.c_int]
         L.moe_fwd_static.argtypes = [P(moe_cfg), _vp, P(moe_params), _vp, _vp]
+        L.moe_test_drop_signal.argtypes = [ctypes.c_int]
         L.moe_strerror.argtypes = [ctypes.c_int]
         L.moe_strerror.restype = ctypes.c_char_p
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
                      "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_status",
-                     "moe_trace_events", "moe_fwd_static"):
+                     "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -169,3 +170,8 @@ def moe_trace_events(fwd_events, bwd_events):
 def moe_fwd_static(cfg, x, params, y, stream):
     """Forward pass using the library's static scratch (no workspace argument)."""
     _check("moe_fwd_static", lib().moe_fwd_static(ctypes.byref(cfg), x, ctypes.byref(params), y, stream))
+
+
+def moe_test_drop_signal(enable: bool):
+    """Fault injection for the bounded waits (see include/mok.h)."""
+    _check("moe_test_drop_signal", lib().moe_test_drop_signal(int(enable)))

@@ -74,6 +74,7 @@ struct GemmArgs {
     int rows_total;               // EPI_ROUTER: rows of one partial-logit slab (T)
     long long group_out_elems;    // EPI_WGRAD: elements of one group's output
     int *status;                  // device status word
+    int test_drop_signal;         // fault injection: CTA 0 skips its first accumulator signal
 };
 
 template <int BN_, bool A_MN_, bool B_MN_, bool A_GATHER_, bool B_GATHER_, bool RAGGED_K_, int EPI_,
@@ -622,7 +623,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
             }
             if (!ok) break;
-            if (lane == 0) {
+            if (lane == 0 && !(args.test_drop_signal && blockIdx.x == 0 && tile == 0)) {
                 if (t.nkb > 0) umma_commit(&accf[acc]);
                 else mbar_arrive(&accf[acc]);
             }

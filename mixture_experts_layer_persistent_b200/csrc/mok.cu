@@ -57,6 +57,7 @@ int fail(int code, const char *what, cudaError_t e = cudaSuccess)
 thread_local cudaEvent_t t_fwd_ev[MOK_FWD_PHASES + 1];
 thread_local cudaEvent_t t_bwd_ev[MOK_BWD_PHASES + 1];
 thread_local bool t_fwd_on = false, t_bwd_on = false;
+thread_local int t_drop_signal = 0;     // moe_test_drop_signal
 
 inline int mark_fwd(int i, cudaStream_t s)
 {
@@ -430,6 +431,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         ga.gather_src = static_cast<const __nv_bfloat16 *>(x);
         ga.gather_ld = c.H;
         ga.status = dev.status;
+        ga.test_drop_signal = t_drop_signal;
         using CGateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU>;
         MOK_TRY(mark_fwd(2, stream));
         MOK_TRY(launch_gemm<CGateUp>(tB, tB, tBs, tO, tO2, tO3, ga, dev.sms, stream));
@@ -791,6 +793,12 @@ int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, 
     }
     const State st = carve_state(*cfg, ptr, false);
     return forward(*cfg, x, *params, y, nullptr, st, *dev, false, static_cast<cudaStream_t>(stream));
+}
+
+int moe_test_drop_signal(int enable)
+{
+    t_drop_signal = enable != 0;
+    return MOK_OK;
 }
 
 const char *moe_last_error(void) { return t_last_error; }
