@@ -91,18 +91,14 @@ struct GemmCfg {
     static constexpr int B_BYTES = BN * 128;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int SF_BYTES = MX ? 512 + BN * 4 : 0;       // SFA (128 rows) + SFB (BN rows), 4 bytes each
-    // Tuning: weight-streaming kernels want a deep operand ring; MXFP8 (single
-    // accumulator buffer) and the weight gradients (short K per tile) want the
-    // epilogue to overlap its stores, so they trade a stage for a second
-    // staging buffer, and the weight gradients split each tile's columns over
-    // eight epilogue warps (two per TMEM lane quarter).
-    static constexpr int STAGES = (MX || RAGGED_K) ? 3 : (BN == 256 ? 4 : 5);
-    static constexpr int EPI_BUFS = (BN == 256 && !MX && !RAGGED_K) ? 1 : 2;
-    static constexpr int EPI_WARPS = RAGGED_K ? 8 : 4;
+    // Tuning (measured at the DeepSeek-V3 shape): the weight-streaming kernels
+    // want a deep operand ring; BN = 128 and MXFP8 trade a stage for a second
+    // epilogue staging buffer so that one block's store overlaps the next
+    // block's conversion; the weight gradients keep a deep ring.
+    static constexpr int STAGES = MX ? 3 : (BN == 256 ? 4 : (RAGGED_K ? 6 : 5));
+    static constexpr int EPI_BUFS = (MX || (!RAGGED_K && BN != 256)) ? 2 : 1;
+    static constexpr int EPI_WARPS = 4;
     static constexpr int PULL_WARPS = (A_GATHER || B_GATHER || MX) ? 4 : 0;   // cp.async warps
-    // K blocks of weights prefetched into L2 ahead of their TMA load: more HBM
-    // requests in flight than the shared-memory ring alone can hold
-    static constexpr int B_PREFETCH = (!RAGGED_K && EPI != EPI_ROUTER) ? 8 : 0;
     static constexpr int PULL_WARP0 = 2 + EPI_WARPS;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + PULL_WARPS);
     static constexpr int GATHER_BYTES = A_GATHER ? A_BYTES : (B_GATHER ? B_BYTES : 0);
@@ -367,25 +363,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const bool routed = t.g < args.num_routed;
             const CUtensorMap *mB = routed ? &tmB : &tmB_s;
             const int gl = routed ? t.g : t.g - args.num_routed;
-            // L2 prefetch of the weight boxes of K block kb (the same boxes the loads below read)
-            auto prefetch_b = [&](int kb) {
-                constexpr int KE = C::KB_ELEMS;
-                if constexpr (!C::B_MN) {
-                    if constexpr (C::EPI == EPI_SWIGLU) {
-                        const int row = gl * args.b_rows_per_group + t.nt * 128;
-                        tma_prefetch_2d(mB, kb * KE, row);
-                        tma_prefetch_2d(mB, kb * KE, row + args.b_half);
-                    } else {
-                        tma_prefetch_2d(mB, kb * KE, gl * args.b_rows_per_group + t.nt * C::BN);
-                    }
-                } else {
-                    for (int c = 0; c < C::BN / 64; ++c)
-                        tma_prefetch_2d(mB, t.nt * C::BN + c * 64, gl * args.b_rows_per_group + kb * BK);
-                }
-            };
-            if constexpr (C::B_PREFETCH > 0)
-                if (lane == 0)
-                    for (int kb = 0; kb < min(C::B_PREFETCH, t.nkb); ++kb) prefetch_b(kb);
             for (int kb = 0; kb < t.nkb; ++kb) {
                 bool ok = true;
                 if (lane == 0) {
@@ -429,8 +406,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     if (lane < C::BN / 64)
                         tma_load_2d(sB + lane * 8192, &tmB, fb, t.nt * C::BN + lane * 64, t.krow0 + kb * BK);
                 }
-                if constexpr (C::B_PREFETCH > 0)
-                    if (lane == 0 && kb + C::B_PREFETCH < t.nkb) prefetch_b(kb + C::B_PREFETCH);
                 if (++stage == C::STAGES) {
                     stage = 0;
                     phase ^= 1u;

@@ -95,15 +95,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, ui
         : "memory");
 }
 
-// Prefetch a 2D box into L2 (no shared memory, no completion tracking).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap *tm, int32_t c0, int32_t c1)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(tm)),
-                 "r"(c0), "r"(c1)
-                 : "memory");
-}
-
 // 2D tiled TMA store of a shared-memory box to global memory (bulk group).
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *tm, const void *src, int32_t c0, int32_t c1)
 {
