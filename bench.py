@@ -226,9 +226,13 @@ def main():
     torch.cuda.synchronize()
     counts = routing["counts"].cpu().numpy()
 
+    launches = [0, 0]               # kernels per forward, per backward (counted by the library)
+
     def step():
         layer.forward(x, y)
+        launches[0] = abi.moe_launch_count()
         layer.backward(x, dy, grads)
+        launches[1] = abi.moe_launch_count()
 
     for _ in range(args.warmup):
         step()
@@ -325,8 +329,9 @@ def main():
                        "tokens_per_gpu": wl.T, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (22.6 GB expert weights streamed per pass)"},
             # forward: router split, router GEMM, select, 3 dispatch kernels, gate/up, down,
-            # combine (9); backward: slot grad, 2 router-gradient kernels, 4 GEMMs, dx sum (8)
-            "gpu_launches": K * (9 + 8),
+            # combine (9); backward: slot grad, 2 router-gradient kernels, 4 GEMMs plus the
+            # resident weight-gradient kernels, dx sum (10)
+            "gpu_launches": K * (launches[0] + launches[1]),
             "clocks": clk, "device_status": status,
             "phases_ms": {k2: round(v, 4) for k2, v in phase.items()},
             "breakdown": {

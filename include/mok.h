@@ -226,6 +226,14 @@ int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events
 int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, void *y, void *stream);
 
 /*
+ * Number of CUDA kernels launched by the last moe_fwd / moe_bwd (or their
+ * _host / _static variants) called on this host thread; 0 before the first.
+ * The count depends on the configuration (dtype, whether I is a multiple of
+ * 256) but not on the data.  Returns MOK_ERR_INVALID for a NULL `count`.
+ */
+int moe_launch_count(int *count);
+
+/*
  * Fault-injection hook for testing the bounded waits.  While enabled (non-zero),
  * every forward launched by this host thread makes CTA 0 of the gate/up GEMM
  * skip the signal that hands its first accumulator to the epilogue; the

@@ -86,6 +86,7 @@ def lib():
         L.moe_trace_events.argtypes = [P(_vp), ctypes.c_int, P(_vp), ctypes.c_int]
         L.moe_fwd_static.argtypes = [P(moe_cfg), _vp, P(moe_params), _vp, _vp]
         L.moe_test_drop_signal.argtypes = [ctypes.c_int]
+        L.moe_launch_count.argtypes = [P(_i32)]
         L.moe_strerror.argtypes = [ctypes.c_int]
         L.moe_strerror.restype = ctypes.c_char_p
         L.moe_last_error.argtypes = []
@@ -170,6 +171,13 @@ def moe_trace_events(fwd_events, bwd_events):
 def moe_fwd_static(cfg, x, params, y, stream):
     """Forward pass using the library's static scratch (no workspace argument)."""
     _check("moe_fwd_static", lib().moe_fwd_static(ctypes.byref(cfg), x, ctypes.byref(params), y, stream))
+
+
+def moe_launch_count() -> int:
+    """Kernels launched by the last forward or backward called on this thread."""
+    n = _i32(0)
+    _check("moe_launch_count", lib().moe_launch_count(ctypes.byref(n)))
+    return n.value
 
 
 def moe_test_drop_signal(enable: bool):

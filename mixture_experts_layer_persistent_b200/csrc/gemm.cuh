@@ -75,6 +75,9 @@ struct GemmArgs {
     long long group_out_elems;    // EPI_WGRAD: elements of one group's output
     int *status;                  // device status word
     int test_drop_signal;         // fault injection: CTA 0 skips its first accumulator signal
+    int k_split;                  // ragged-K: > 0 limits the streaming kernel to groups with more rows
+                                  // (a prefix of gorder); the resident kernel takes the rest
+    int m_per_unit;               // resident weight-gradient kernel: M tiles per work unit
 };
 
 template <int BN_, bool A_MN_, bool B_MN_, bool A_GATHER_, bool B_GATHER_, bool RAGGED_K_, int EPI_,
@@ -131,6 +134,20 @@ struct Tile {
     int krows;      // ragged-K: rows of the group
     int nkb;        // K blocks
 };
+
+// gorder lists groups by rows descending: the first `nbig` have more than k_split rows
+// (k_split <= 0: every group)
+__device__ __forceinline__ int count_big_groups(const int *s_off, const int *s_gorder, int G, int k_split)
+{
+    if (k_split <= 0) return G;
+    int lo = 0, hi = G;                   // first position whose group has <= k_split rows
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        const int g = s_gorder[mid];
+        if (s_off[g + 1] - s_off[g] > k_split) lo = mid + 1; else hi = mid;
+    }
+    return lo;
+}
 
 template <class C>
 __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const int *s_off, const int *s_tstart,
@@ -352,7 +369,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int total = C::RAGGED_K ? G * args.m_tiles * args.n_tiles : s_tstart[G];
+    const int total = C::RAGGED_K ? count_big_groups(s_off, s_gorder, G, args.k_split) * args.m_tiles * args.n_tiles
+                                  : s_tstart[G];
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer

@@ -14,6 +14,7 @@
 #include "gemm.cuh"
 #include "quant.cuh"
 #include "route.cuh"
+#include "wgrad.cuh"
 
 namespace mok {
 
@@ -58,6 +59,7 @@ thread_local cudaEvent_t t_fwd_ev[MOK_FWD_PHASES + 1];
 thread_local cudaEvent_t t_bwd_ev[MOK_BWD_PHASES + 1];
 thread_local bool t_fwd_on = false, t_bwd_on = false;
 thread_local int t_drop_signal = 0;     // moe_test_drop_signal
+thread_local int t_launches = 0;        // kernels launched by the current / last forward or backward
 
 inline int mark_fwd(int i, cudaStream_t s)
 {
@@ -260,6 +262,28 @@ int check_cfg(const moe_cfg *c)
 
 // Operand maps a, b, bs (B of the shared groups) and output maps o, o2, o3.
 template <class C>
+int launch_wgrad_resident(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &o, const CUtensorMap &o2,
+                          const GemmArgs &args, int grid, cudaStream_t st)
+{
+    if (grid <= 0) return MOK_OK;
+    cudaError_t e = cudaFuncSetAttribute(wgrad_resident_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(wgrad_resident_kernel)", e);
+    wgrad_resident_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, o, o2, args);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "wgrad_resident_kernel launch", e);
+    ++t_launches;
+    return MOK_OK;
+}
+
+// M tiles per resident work unit: runs of at most 16, split evenly
+int resident_m_per_unit(int m_tiles)
+{
+    const int chunks = (m_tiles + 15) / 16;
+    return (m_tiles + chunks - 1) / chunks;
+}
+
+template <class C>
 int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &bs, const CUtensorMap &o,
                 const CUtensorMap &o2, const CUtensorMap &o3, const GemmArgs &args, int grid, cudaStream_t st)
 {
@@ -269,7 +293,9 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b
     if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(grouped_gemm_kernel)", e);
     grouped_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, bs, o, o2, o3, args);
     e = cudaGetLastError();
-    return e == cudaSuccess ? MOK_OK : fail(MOK_ERR_LAUNCH, "grouped_gemm_kernel launch", e);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "grouped_gemm_kernel launch", e);
+    ++t_launches;
+    return MOK_OK;
 }
 
 inline int blocks_for(long long n, int per) { return static_cast<int>((n + per - 1) / per); }
@@ -284,6 +310,7 @@ inline int blocks_for(long long n, int per) { return static_cast<int>((n + per -
     do {                                                                            \
         const cudaError_t e_ = cudaGetLastError();                                  \
         if (e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "kernel launch", e_);    \
+        ++t_launches;                                                               \
     } while (0)
 
 // ------------------------------------------------------------------ forward
@@ -291,6 +318,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
             const State &st, const DeviceInfo &dev, bool training, cudaStream_t stream)
 {
     const Shapes s = shapes(c);
+    t_launches = 0;
     const bool mx = c.dtype == MOK_DTYPE_MXFP8;
 
     // router logits on the tensor cores: x . [Wr_hi | Wr_mid | Wr_lo]^T, split over K
@@ -481,6 +509,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
              const moe_grads &gr, const BwdScratch &bs, const DeviceInfo &dev, cudaStream_t stream)
 {
     const Shapes s = shapes(c);
+    t_launches = 0;
     const __nv_bfloat16 *dyb = static_cast<const __nv_bfloat16 *>(dy);
 
     MOK_TRY(mark_bwd(0, stream));
@@ -515,15 +544,21 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
     if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
     GemmArgs g1 = base;
-    g1.n_tiles = c.I / 128;
     g1.num_kb = c.H / BK;
     g1.b_rows_per_group = c.H;
     g1.aux = st.gu;
     g1.out = bs.dgu;
-    using CDgradDown = GemmCfg<128, false, true, true, false, false, EPI_DSWIGLU>;
     MOK_TRY(mark_bwd(3, stream));
     if (!make_tmap(&tO, bs.dgu, 2 * s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
-    MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, tO, tO, tO, g1, dev.sms, stream));
+    if (c.I % 256 == 0) {      // N = 256 halves the gathered dy rows per weight byte
+        g1.n_tiles = c.I / 256;
+        using CDgradDown = GemmCfg<256, false, true, true, false, false, EPI_DSWIGLU>;
+        MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, tO, tO, tO, g1, dev.sms, stream));
+    } else {
+        g1.n_tiles = c.I / 128;
+        using CDgradDown = GemmCfg<128, false, true, true, false, false, EPI_DSWIGLU>;
+        MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, tO, tO, tO, g1, dev.sms, stream));
+    }
 
     // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
     GemmArgs g2 = base;
@@ -537,12 +572,19 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     if (!make_tmap(&tO2, s.S ? gr.dws_down : gr.dw_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 32, 2))
         return MOK_ERR_INVALID;
     if (c.I % 256 == 0) {
+        // groups of more than kResidentRows rows stream both operands; the rest keep
+        // their (w h) slab resident and stream gathered dy
         if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
         g2.n_tiles = c.I / 256;
+        g2.k_split = kResidentRows;
+        g2.m_per_unit = resident_m_per_unit(g2.m_tiles);
         using CWgradDown = GemmCfg<256, true, true, true, false, true, EPI_WGRAD>;
         const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
         MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, tO, tO2, tO, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms),
                                         stream));
+        const long long u2 = s.G * g2.n_tiles * ((g2.m_tiles + g2.m_per_unit - 1) / g2.m_per_unit);
+        MOK_TRY(launch_wgrad_resident<WgradResCfg<true>>(tB, tB, tO, tO2, g2,
+                                                         static_cast<int>(u2 < dev.sms ? u2 : dev.sms), stream));
     } else {
         if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
         g2.n_tiles = c.I / 128;
@@ -578,6 +620,8 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g4.out_s = static_cast<__nv_bfloat16 *>(gr.dws_gate_up);
     g4.ldo = c.H;
     g4.group_out_elems = 2 * s.I * s.H;
+    g4.k_split = kResidentRows;            // larger groups stream; the rest keep their x slab resident
+    g4.m_per_unit = resident_m_per_unit(g4.m_tiles);
     using CWgradGU = GemmCfg<256, true, true, false, true, true, EPI_WGRAD>;
     const long long t4 = s.G * g4.m_tiles * g4.n_tiles;
     MOK_TRY(mark_bwd(6, stream));
@@ -585,6 +629,9 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     if (!make_tmap(&tO2, s.S ? gr.dws_gate_up : gr.dw_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 64, 32, 2))
         return MOK_ERR_INVALID;
     MOK_TRY(launch_gemm<CWgradGU>(tA, tA, tA, tO, tO2, tO, g4, static_cast<int>(t4 < dev.sms ? t4 : dev.sms), stream));
+    const long long u4 = s.G * g4.n_tiles * ((g4.m_tiles + g4.m_per_unit - 1) / g4.m_per_unit);
+    MOK_TRY(launch_wgrad_resident<WgradResCfg<false>>(tA, tA, tO, tO2, g4, static_cast<int>(u4 < dev.sms ? u4 : dev.sms),
+                                                      stream));
 
     MOK_TRY(mark_bwd(7, stream));
     dx_combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(
@@ -793,6 +840,13 @@ int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, 
     }
     const State st = carve_state(*cfg, ptr, false);
     return forward(*cfg, x, *params, y, nullptr, st, *dev, false, static_cast<cudaStream_t>(stream));
+}
+
+int moe_launch_count(int *count)
+{
+    if (!count) return MOK_ERR_INVALID;
+    *count = t_launches;
+    return MOK_OK;
 }
 
 int moe_test_drop_signal(int enable)
