@@ -137,14 +137,14 @@ struct Tile {
 
 // gorder lists groups by rows descending: the first `nbig` have more than k_split rows
 // (k_split <= 0: every group)
-__device__ __forceinline__ int count_big_groups(const int *s_off, const int *s_gorder, int G, int k_split)
+__device__ __forceinline__ int count_big_groups(const int *off, const int *order, int G, int k_split)
 {
     if (k_split <= 0) return G;
     int lo = 0, hi = G;                   // first position whose group has <= k_split rows
     while (lo < hi) {
         const int mid = (lo + hi) >> 1;
-        const int g = s_gorder[mid];
-        if (s_off[g + 1] - s_off[g] > k_split) lo = mid + 1; else hi = mid;
+        const int g = order[mid];
+        if (off[g + 1] - off[g] > k_split) lo = mid + 1; else hi = mid;
     }
     return lo;
 }

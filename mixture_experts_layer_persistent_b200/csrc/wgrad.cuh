@@ -43,16 +43,17 @@ struct WgradResCfg {
     static constexpr int B_KB_BYTES = BN * BK * 2;           // 256 N x 64 K, four 8 KB chunks
     static constexpr int B_BYTES = KB_MAX * B_KB_BYTES;
     static constexpr int STAGES = 4;
-    static constexpr int EPI_WARPS = 4;
-    static constexpr int EPI_BUFS = 1;
+    static constexpr int EPI_WARPS = 4;                      // 4 or 8 (two per TMEM lane quarter)
+    static constexpr int EPI_BUFS = 2;
     static constexpr int PULL_WARPS = 4;
     static constexpr int PULL_WARP0 = 2 + EPI_WARPS;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + PULL_WARPS);
     static constexpr int TMEM_COLS = 2 * BN;                 // two accumulators
     static constexpr int EPI_STAGE_BYTES = EPI_WARPS * EPI_BUFS * 4096;
     static constexpr int BAR_BYTES = 256;
-    static constexpr int AUX_BYTES = BAR_BYTES + (2 * kMaxGroups + 1) * 4;
-    static constexpr int SMEM_BYTES = 1024 + B_BYTES + STAGES * A_BYTES + EPI_STAGE_BYTES + AUX_BYTES;
+    // the group tables (offsets, order) are read through L1, not staged: the
+    // shared memory goes to the resident slab, the ring and the store staging
+    static constexpr int SMEM_BYTES = 1024 + B_BYTES + STAGES * A_BYTES + EPI_STAGE_BYTES + BAR_BYTES;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, true, true);
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert((2 * STAGES + KB_MAX + 5) * 8 + 8 <= BAR_BYTES, "barrier block");
@@ -67,8 +68,7 @@ struct WUnit {
     int nkb;        // K blocks
 };
 
-__device__ __forceinline__ WUnit decode_unit(int u, const GemmArgs &a, const int *s_off, const int *s_gorder, int nbig,
-                                             int m_chunks)
+__device__ __forceinline__ WUnit decode_unit(int u, const GemmArgs &a, int nbig, int m_chunks)
 {
     WUnit w;
     const int per_group = a.n_tiles * m_chunks;
@@ -76,11 +76,11 @@ __device__ __forceinline__ WUnit decode_unit(int u, const GemmArgs &a, const int
     const int rem = u - (gi - nbig) * per_group;
     w.nt = rem / m_chunks;
     const int mc = rem - w.nt * m_chunks;
-    w.g = s_gorder[gi];
+    w.g = __ldg(a.gorder + gi);
     w.mt0 = mc * a.m_per_unit;
     w.mt1 = min(w.mt0 + a.m_per_unit, a.m_tiles);
-    w.krow0 = s_off[w.g];
-    w.krows = s_off[w.g + 1] - w.krow0;
+    w.krow0 = __ldg(a.offsets + w.g);
+    w.krows = __ldg(a.offsets + w.g + 1) - w.krow0;
     w.nkb = (w.krows + BK - 1) / BK;
     return w;
 }
@@ -114,16 +114,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t *acce = accf + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    int *s_off = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(afull) + C::BAR_BYTES);
-    int *s_gorder = s_off + kMaxGroups + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = args.num_groups;
     int *status = args.status;
 
     if (warp == 0) {
-        for (int i = lane; i <= G; i += 32) s_off[i] = args.offsets[i];
-        for (int i = lane; i < G; i += 32) s_gorder[i] = args.gorder[i];
         if (lane == 0) {
             for (int s = 0; s < C::STAGES; ++s) {
                 mbar_init(&afull[s], C::A_GATHER ? 32 * C::PULL_WARPS : 1);
@@ -149,7 +145,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    const int nbig = count_big_groups(s_off, s_gorder, G, args.k_split);
+    const int nbig = count_big_groups(args.offsets, args.gorder, G, args.k_split);
     const int m_chunks = (args.m_tiles + args.m_per_unit - 1) / args.m_per_unit;
     const int total = (G - nbig) * args.n_tiles * m_chunks;
 
@@ -158,7 +154,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         int stage = 0;
         uint32_t phase = 0, bphase = 0;
         for (int u = blockIdx.x; u < total; u += gridDim.x) {
-            const WUnit w = decode_unit(u, args, s_off, s_gorder, nbig, m_chunks);
+            const WUnit w = decode_unit(u, args, nbig, m_chunks);
             if (w.nkb == 0) continue;
             bool ok = true;
             if constexpr (!C::B_GATHER) {
@@ -210,7 +206,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         uint32_t phase = 0, bphase = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-            const WUnit w = decode_unit(u, args, s_off, s_gorder, nbig, m_chunks);
+            const WUnit w = decode_unit(u, args, nbig, m_chunks);
             if (w.nkb == 0) continue;
             int tok[C::KB_MAX][4];
 #pragma unroll
@@ -283,7 +279,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         uint32_t phase = 0, acc_phase = 0, bph = 0;     // bph: parity bit of bfull[kb]
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-            const WUnit w = decode_unit(u, args, s_off, s_gorder, nbig, m_chunks);
+            const WUnit w = decode_unit(u, args, nbig, m_chunks);
             for (int mt = w.mt0; mt < w.mt1; ++mt) {
                 if (lane == 0) ok = mbar_wait(&acce[acc], acc_phase ^ 1u, abort_flag, status);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -357,7 +353,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         uint32_t acc_phase = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
-            const WUnit w = decode_unit(u, args, s_off, s_gorder, nbig, m_chunks);
+            const WUnit w = decode_unit(u, args, nbig, m_chunks);
             const bool routed = w.g < args.num_routed;
             const int gl = routed ? w.g : w.g - args.num_routed;
             for (int mt = w.mt0; mt < w.mt1; ++mt) {
@@ -366,18 +362,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 tc_fence_after();
                 const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * C::BN) + (static_cast<uint32_t>(eq * 32) << 16);
                 const int grow0 = gl * args.m_tiles * BM + mt * BM + eq * 32;
+                constexpr int COLS = C::BN * 4 / C::EPI_WARPS;       // columns of this warp
+                const int c0 = (ew >> 2) * COLS;
                 float v[64];
                 if (w.nkb > 0) {
-                    tmem_ld32(taddr, *reinterpret_cast<float(*)[32]>(v));
-                    tmem_ld32(taddr + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                    tmem_ld32(taddr + c0, *reinterpret_cast<float(*)[32]>(v));
+                    tmem_ld32(taddr + c0 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
                     tmem_ld_wait();
                 }
 #pragma unroll 1
-                for (int c = 0; c < C::BN; c += 64) {
+                for (int c = c0; c < c0 + COLS; c += 64) {
                     uint32_t pk[32];
                     if (w.nkb > 0) {
                         pack_bf16<64>(v, pk);
-                        if (c + 64 < C::BN) {              // next block's TMEM load overlaps this block's store
+                        if (c + 64 < c0 + COLS) {          // next block's TMEM load overlaps this block's store
                             tmem_ld32(taddr + c + 64, *reinterpret_cast<float(*)[32]>(v));
                             tmem_ld32(taddr + c + 96, *reinterpret_cast<float(*)[32]>(v + 32));
                         }
@@ -386,7 +384,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         for (int i = 0; i < 32; ++i) pk[i] = 0u;
                     }
                     store_block_tile(stg, pk, lane, routed ? &tmO : &tmO2, w.nt * C::BN + c, grow0);
-                    if (w.nkb > 0 && c + 64 < C::BN) tmem_ld_wait();
+                    if (w.nkb > 0 && c + 64 < c0 + COLS) tmem_ld_wait();
                 }
                 tc_fence_before();
                 mbar_arrive(&acce[acc]);
