@@ -98,8 +98,14 @@ struct GemmCfg {
     // want a deep operand ring; BN = 128 and MXFP8 trade a stage for a second
     // epilogue staging buffer so that one block's store overlaps the next
     // block's conversion; the weight gradients keep a deep ring.
-    static constexpr int STAGES = MX ? 3 : (BN == 256 ? 4 : (RAGGED_K ? 6 : 5));
-    static constexpr int EPI_BUFS = (MX || (!RAGGED_K && BN != 256)) ? 2 : 1;
+    // Kernels whose epilogue moves several blocks per warp and tile (SwiGLU
+    // backward, weight gradients at N = 256, MXFP8) do better with a second
+    // staging buffer in place of a fourth stage; the plain weight streamers keep
+    // four.  (MXFP8 measured slower with a fourth stage and one staging buffer.)
+    static constexpr bool MX_SWIGLU = MX && EPI == EPI_SWIGLU;
+    static constexpr bool HEAVY_EPI = BN == 256 && (MX || EPI == EPI_DSWIGLU || RAGGED_K);
+    static constexpr int STAGES = HEAVY_EPI ? 3 : (BN == 256 ? 4 : (RAGGED_K ? 6 : 5));
+    static constexpr int EPI_BUFS = (HEAVY_EPI || (!RAGGED_K && BN != 256)) ? 2 : 1;
     static constexpr int EPI_WARPS = 4;
     static constexpr int PULL_WARPS = (A_GATHER || B_GATHER || MX) ? 4 : 0;   // cp.async warps
     static constexpr int PULL_WARP0 = 2 + EPI_WARPS;
@@ -649,12 +655,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const int n0 = t.nt * 128;
                 uint32_t q[32];
                 uint32_t sc = 0;
+                // the single accumulator is handed back to the MMA warp as soon as its
+                // last columns are in registers: the loads of block b + 1 overlap the
+                // math of block b
+                float gb[2][32], ub[2][32];
+                tmem_ld32(taddr, gb[0]);
+                tmem_ld32(taddr + 128, ub[0]);
+                tmem_ld_wait();
 #pragma unroll
                 for (int blk = 0; blk < 4; ++blk) {
-                    float g[32], u[32];
-                    tmem_ld32(taddr + 32 * blk, g);
-                    tmem_ld32(taddr + 128 + 32 * blk, u);
-                    tmem_ld_wait();
+                    float *g = gb[blk & 1], *u = ub[blk & 1];
+                    if (blk < 3) {
+                        tmem_ld32(taddr + 32 * (blk + 1), gb[(blk + 1) & 1]);
+                        tmem_ld32(taddr + 128 + 32 * (blk + 1), ub[(blk + 1) & 1]);
+                    }
                     float amax = 0.0f;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -673,6 +687,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         q[8 * blk + i] = word;
                     }
                     sc |= static_cast<uint32_t>(e + 127) << (8 * blk);
+                    if (blk < 3) tmem_ld_wait();
+                    if (blk == 2) {
+                        tc_fence_before();
+                        mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
+                    }
                 }
                 uint8_t *qout = reinterpret_cast<uint8_t *>(args.out);
                 if (full) store_block_tile(stg, q, lane, &tmO, n0, row0);
@@ -814,8 +833,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     else if (valid) store_row_direct(args.out_f32 + ((size_t)t.nt * args.rows_total + r) * 256 + c, p);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&acce[acc]);
+            if constexpr (!C::MX_SWIGLU) {
+                tc_fence_before();
+                mbar_arrive(&acce[acc]);
+            }
             if (++acc == C::ACC_BUFS) {
                 acc = 0;
                 acc_phase ^= 1u;
