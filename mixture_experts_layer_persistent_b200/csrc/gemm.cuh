@@ -98,12 +98,12 @@ struct GemmCfg {
     // want a deep operand ring; BN = 128 and MXFP8 trade a stage for a second
     // epilogue staging buffer so that one block's store overlaps the next
     // block's conversion; the weight gradients keep a deep ring.
-    // Kernels whose epilogue moves several blocks per warp and tile (SwiGLU
-    // backward, weight gradients at N = 256, MXFP8) do better with a second
+    // Kernels whose epilogue moves several blocks per warp and tile (weight
+    // gradients at N = 256, MXFP8) do better with a second
     // staging buffer in place of a fourth stage; the plain weight streamers keep
     // four.  (MXFP8 measured slower with a fourth stage and one staging buffer.)
     static constexpr bool MX_SWIGLU = MX && EPI == EPI_SWIGLU;
-    static constexpr bool HEAVY_EPI = BN == 256 && (MX || EPI == EPI_DSWIGLU || RAGGED_K);
+    static constexpr bool HEAVY_EPI = BN == 256 && (MX || RAGGED_K);
     static constexpr int STAGES = HEAVY_EPI ? 3 : (BN == 256 ? 4 : (RAGGED_K ? 6 : 5));
     static constexpr int EPI_BUFS = (HEAVY_EPI || (!RAGGED_K && BN != 256)) ? 2 : 1;
     static constexpr int EPI_WARPS = 4;
@@ -277,29 +277,16 @@ __device__ __forceinline__ void store_row_direct(void *dst, const uint32_t *p)
     for (int c = 0; c < 8; ++c) d[c] = make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
 }
 
-// cooperative load of 32 rows x 128 bytes (row `lane` from src, null = zeros) into p
-__device__ __forceinline__ void load_block(EpiStage &es, uint32_t *p, const void *src, int lane)
+// 128 bytes of this lane's own row (null = zeros) straight into registers: the
+// first 16-byte load brings the line into L1 and the other seven hit it
+__device__ __forceinline__ void load_row_direct(uint32_t *p, const void *src)
 {
-    uint32_t *stg = es.next();
-    if (lane == 0) bulk_wait_read0();     // loads commit no store group: wait for every store to have read
-    __syncwarp();
-    const uint64_t d = reinterpret_cast<uint64_t>(src);
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-        const int row = it * 4 + (lane >> 3), ch = lane & 7;
-        const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d), row);
-        const uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(d >> 32), row);
-        const uint64_t rs = (static_cast<uint64_t>(hi) << 32) | lo;
-        const uint4 v = rs ? reinterpret_cast<const uint4 *>(rs)[ch] : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4 *>(stg + row * 32 + ((ch ^ (row & 7)) << 2)) = v;
-    }
-    __syncwarp();
+    const uint4 *q = reinterpret_cast<const uint4 *>(src);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(stg + lane * 32 + ((c ^ (lane & 7)) << 2));
+        const uint4 v = src ? __ldg(q + c) : make_uint4(0u, 0u, 0u, 0u);
         p[4 * c] = v.x; p[4 * c + 1] = v.y; p[4 * c + 2] = v.z; p[4 * c + 3] = v.w;
     }
-    __syncwarp();
 }
 
 template <class C>
@@ -791,8 +778,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll 1
                 for (int c = 0; c < C::BN; c += 64) {
                     uint32_t gp[32], up[32], dgp[32], dup[32];
-                    load_block(stg, gp, gsrc ? gsrc + c : nullptr, lane);
-                    load_block(stg, up, gsrc ? gsrc + I + c : nullptr, lane);
+                    load_row_direct(gp, gsrc ? gsrc + c : nullptr);
+                    load_row_direct(up, gsrc ? gsrc + I + c : nullptr);
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         float v[32], dg[32], du[32];
