@@ -213,24 +213,35 @@ __device__ __forceinline__ void pack_bf16(const float *v, uint32_t *p)
 // chunk c ^ (r & 7)), so the TMA store engine writes whole lines while the
 // warp moves on; the stores stay in flight without occupying the warp.
 
-// Two staging buffers per warp alternate: before a buffer is rewritten, the
-// store issued from it two blocks earlier must have read it (at most one store
-// group, the other buffer's, may still be reading).
+// The staging buffers of a warp rotate: before a buffer is rewritten, the store
+// issued from it `bufs` blocks earlier must have read it (the bufs - 1 later
+// store groups, one per block, may still be reading theirs).
 struct EpiStage {
     uint32_t *buf;      // bufs x 1024 words
-    int bufs;           // 1 or 2
-    int n;              // blocks staged so far
-    __device__ __forceinline__ uint32_t *next() { return buf + ((n++ & (bufs - 1)) << 10); }
+    int bufs;           // 1 to 4
+    int cur;            // buffer of the next block
+    __device__ __forceinline__ uint32_t *next()
+    {
+        uint32_t *b = buf + (cur << 10);
+        cur = cur + 1 == bufs ? 0 : cur + 1;
+        return b;
+    }
 };
 
-__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+// wait until at most `pending` bulk store groups of this thread still read shared memory
+__device__ __forceinline__ void bulk_wait_read(int pending)
+{
+    switch (pending) {
+    case 0: asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.bulk.wait_group.read 2;" ::: "memory"); break;
+    default: asm volatile("cp.async.bulk.wait_group.read 3;" ::: "memory"); break;
+    }
+}
 
 __device__ __forceinline__ void stage_block(const EpiStage &es, uint32_t *stg, const uint32_t *p, int lane)
 {
-    if (lane == 0) {                      // the store that last used this buffer has read it
-        if (es.bufs == 2) bulk_wait_read1();
-        else bulk_wait_read0();
-    }
+    if (lane == 0) bulk_wait_read(es.bufs - 1);     // the store that last used this buffer has read it
     __syncwarp();
 #pragma unroll
     for (int c = 0; c < 8; ++c)

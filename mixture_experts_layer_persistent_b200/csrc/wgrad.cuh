@@ -56,6 +56,7 @@ struct WgradResCfg {
     static constexpr int SMEM_BYTES = 1024 + B_BYTES + STAGES * A_BYTES + EPI_STAGE_BYTES + BAR_BYTES;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, true, true);
     static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(EPI_BUFS >= 1 && EPI_BUFS <= 4, "staging buffers per warp");
     static_assert((2 * STAGES + KB_MAX + 5) * 8 + 8 <= BAR_BYTES, "barrier block");
 };
 

@@ -61,6 +61,9 @@ WORKLOADS = {
     # the same with 128 rows per routed expert on average, as in dsv3
     "dsv3_e32_r128": Workload("dsv3_e32_r128", T=512, H=7168, E=32, k=8, I=2048, S=1, Is=2048,
                               score_fn=1, n_group=8, topk_group=4, seed=6),
+    # MXFP8 forward with 256 rows per routed expert on average, as in dsv3_mxfp8
+    "dsv3_mxfp8_e32": Workload("dsv3_mxfp8_e32", T=1024, H=7168, E=32, k=8, I=2048, S=1, Is=2048,
+                               score_fn=1, n_group=8, topk_group=4, mxfp8=True, backward=False, seed=7),
 }
 
 
