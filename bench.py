@@ -357,7 +357,7 @@ def main():
 def mxfp8_run(wl, dev, K, warmup, world, dist, pk):
     """Forward tokens/s of the MXFP8 layer (weights quantised once, outside the timed region)."""
     import torch
-    from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, moe_trace_events, quantize_mxfp8, synth
+    from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, moe_trace_events, quantize_mxfp8_weights, synth
     p = synth.draw_params(wl, dev)
     params = {k: p[k] for k in ("router_w", "e_bias", "logit_bias")}
     for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
@@ -365,7 +365,7 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk):
         if p.get(name) is None:
             params[name] = params[sname] = None
         else:
-            params[name], params[sname] = quantize_mxfp8(p[name])
+            params[name], params[sname] = quantize_mxfp8_weights(p[name])
             p[name] = None
     del p
     torch.cuda.empty_cache()

@@ -78,7 +78,9 @@ typedef struct moe_cfg {
  * For MOK_DTYPE_BF16 the weights are bf16 and the s_* scale pointers are NULL.
  * For MOK_DTYPE_MXFP8 the weights are e4m3 codes (one byte each, same shapes)
  * and s_* hold one ue8m0 byte per 32 consecutive elements along the last
- * (contraction) axis: [E, 2I, H/32], [E, H, I/32] (see moe_quantize_mxfp8).
+ * (contraction) axis, for the tensors [E*2I, H] and [E*H, I] (S in place of E
+ * for the shared experts), in the packed weight-scale layout that
+ * moe_quantize_mxfp8_weights writes.
  */
 typedef struct moe_params {
     const float *router_w;      /* [E, H] fp32 */
@@ -177,6 +179,21 @@ int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host,
  */
 int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *scales,
                        void *stream);
+
+/*
+ * The same quantisation for expert weights, with the scales in the packed
+ * weight-scale layout the MXFP8 layer reads: (K/128) x (rows/128) tiles of
+ * 512 bytes, tile (kb, rb) at byte offset (kb * rows/128 + rb) * 512, holding
+ * for row r = 128 rb + 32 q + i (0 <= q < 4, 0 <= i < 32) and 32-element block
+ * j = 4 kb + s (0 <= s < 4) the scale byte at 16 i + 4 q + s.  This is the
+ * block-scaled MMA's scale-factor layout for a 128-row block, so the layer
+ * fetches one K block of a weight tile's scales as one 512-byte copy per 128
+ * rows.  q is [rows, K] e4m3 as for moe_quantize_mxfp8; scales holds
+ * rows * K / 32 bytes.  rows and K must be multiples of 128 (MOK_ERR_INVALID
+ * otherwise).
+ */
+int moe_quantize_mxfp8_weights(const void *src, int64_t rows, int64_t K, void *q, void *scales,
+                               void *stream);
 
 /*
  * Phase tracing.  When events are set, every later moe_fwd (moe_bwd) records

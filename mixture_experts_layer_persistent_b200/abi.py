@@ -82,6 +82,7 @@ def lib():
         L.moe_bwd_host.argtypes = [P(moe_cfg), _vp, _vp, P(moe_params), _vp, _sz, _vp, P(moe_grads),
                                    _vp, _sz, _vp]
         L.moe_quantize_mxfp8.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
+        L.moe_quantize_mxfp8_weights.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
         L.moe_status.argtypes = [_vp, P(_i32)]
         L.moe_trace_events.argtypes = [P(_vp), ctypes.c_int, P(_vp), ctypes.c_int]
         L.moe_fwd_static.argtypes = [P(moe_cfg), _vp, P(moe_params), _vp, _vp]
@@ -92,7 +93,7 @@ def lib():
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
-                     "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_status",
+                     "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_quantize_mxfp8_weights", "moe_status",
                      "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -152,6 +153,10 @@ def moe_bwd_host(cfg, x_host, dy_host, params, ctx, ctx_bytes, dx_host, grads, s
 
 def moe_quantize_mxfp8(src, rows, K, q, scales, stream):
     _check("moe_quantize_mxfp8", lib().moe_quantize_mxfp8(src, rows, K, q, scales, stream))
+
+
+def moe_quantize_mxfp8_weights(src, rows, K, q, scales, stream):
+    _check("moe_quantize_mxfp8_weights", lib().moe_quantize_mxfp8_weights(src, rows, K, q, scales, stream))
 
 
 def moe_status(stream) -> int:

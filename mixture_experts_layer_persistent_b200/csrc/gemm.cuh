@@ -59,9 +59,11 @@ struct GemmArgs {
     int gather_ld;                // elements per token row of gather_src
     // MXFP8 (block-scaled) operands: ue8m0 scales, one byte per 32 K-elements, rows of sf_ld bytes
     const uint8_t *sfa_src;       // scales of A's rows (token rows when A is gathered, sorted rows otherwise)
-    const uint8_t *sfb_src;       // scales of the routed groups' B rows
-    const uint8_t *sfb_src_s;     // scales of the shared groups' B rows
-    int sf_ld;                    // scale bytes per row (K / 32)
+    const uint8_t *sfb_src;       // scales of the routed groups' B rows (packed weight-scale layout)
+    const uint8_t *sfb_src_s;     // scales of the shared groups' B rows (packed weight-scale layout)
+    int sf_ld;                    // A scale bytes per row (K / 32)
+    int sfb_row_tiles;            // 128-row blocks of the routed weight tensor
+    int sfb_row_tiles_s;          // 128-row blocks of the shared weight tensor
     uint8_t *out_scales;          // MXFP8 SwiGLU epilogue: scales of h [R, I/32]
     __nv_bfloat16 *out;           // main output
     __nv_bfloat16 *out_s;         // EPI_WGRAD: output of the shared groups
@@ -99,11 +101,12 @@ struct GemmCfg {
     // epilogue staging buffer so that one block's store overlaps the next
     // block's conversion; the weight gradients keep a deep ring.
     // Kernels whose epilogue moves several blocks per warp and tile (weight
-    // gradients at N = 256, MXFP8) do better with a second
-    // staging buffer in place of a fourth stage; the plain weight streamers keep
-    // four.  (MXFP8 measured slower with a fourth stage and one staging buffer.)
+    // gradients at N = 256, the MXFP8 down GEMM's fp32 pushes) do better with a
+    // second staging buffer in place of a fourth stage; the plain weight
+    // streamers, the MXFP8 gate/up GEMM among them (one block per warp and
+    // tile), keep four.
     static constexpr bool MX_SWIGLU = MX && EPI == EPI_SWIGLU;
-    static constexpr bool HEAVY_EPI = BN == 256 && (MX || RAGGED_K);
+    static constexpr bool HEAVY_EPI = BN == 256 && ((MX && !MX_SWIGLU) || RAGGED_K);
     static constexpr int STAGES = HEAVY_EPI ? 3 : (BN == 256 ? 4 : (RAGGED_K ? 6 : 5));
     static constexpr int EPI_BUFS = (HEAVY_EPI || (!RAGGED_K && BN != 256)) ? 2 : 1;
     static constexpr int EPI_WARPS = 4;
@@ -111,7 +114,8 @@ struct GemmCfg {
     static constexpr int PULL_WARP0 = 2 + EPI_WARPS;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + PULL_WARPS);
     static constexpr int GATHER_BYTES = A_GATHER ? A_BYTES : (B_GATHER ? B_BYTES : 0);
-    static constexpr int TMA_BYTES = STAGE_BYTES - GATHER_BYTES;
+    // MXFP8: the weight scales of a K block (two 512-byte tiles) come with B
+    static constexpr int TMA_BYTES = STAGE_BYTES - GATHER_BYTES + (MX ? 1024 : 0);
     static constexpr int ACC_BUFS = MX ? 1 : 2;                  // MXFP8 needs TMEM columns for the scales
     static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
     static constexpr int SF_TMEM_COL = 256;                      // SFA at 256..259, SFB at 260..
@@ -428,6 +432,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     if (lane < C::BN / 64)
                         tma_load_2d(sB + lane * 8192, &tmB, fb, t.nt * C::BN + lane * 64, t.krow0 + kb * BK);
                 }
+                if constexpr (C::MX) {
+                    // the weight scales of this K block: one packed 512-byte tile per 128 B rows
+                    if (lane == 0) {
+                        const uint8_t *sb = routed ? args.sfb_src : args.sfb_src_s;
+                        const long long rt = routed ? args.sfb_row_tiles : args.sfb_row_tiles_s;
+                        const int r0 = gl * args.b_rows_per_group + (C::EPI == EPI_SWIGLU ? t.nt * 128 : t.nt * C::BN);
+                        const int r1 = C::EPI == EPI_SWIGLU ? r0 + args.b_half : r0 + 128;
+                        uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
+                        bulk_load(sf + 512, sb + (static_cast<long long>(kb) * rt + (r0 >> 7)) * 512, 512, fb);
+                        bulk_load(sf + 1024, sb + (static_cast<long long>(kb) * rt + (r1 >> 7)) * 512, 512, fb);
+                    }
+                }
                 if (++stage == C::STAGES) {
                     stage = 0;
                     phase ^= 1u;
@@ -460,25 +476,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             tok[i] = r < t.rows ? __ldg(args.row_token + t.m0 + r) : 0;
                         }
                     }
-                    // MXFP8 scales: SFA row p (its token row when A is gathered), SFB rows p and p + 128
-                    const uint8_t *sfa = nullptr, *sfb0 = nullptr, *sfb1 = nullptr;
+                    // MXFP8 scales of A: row p (its token row when A is gathered); the weight
+                    // scales come with B from the producer
+                    const uint8_t *sfa = nullptr;
                     if constexpr (C::MX) {
                         const int ar = p < t.rows ? (C::A_GATHER ? __ldg(args.row_token + t.m0 + p) : t.m0 + p)
                                                   : (C::A_GATHER ? 0 : t.m0);
                         sfa = args.sfa_src + (size_t)ar * args.sf_ld;
-                        const bool routed = t.g < args.num_routed;
-                        const int gl = routed ? t.g : t.g - args.num_routed;
-                        const uint8_t *sb = routed ? args.sfb_src : args.sfb_src_s;
-                        int b0, b1;
-                        if constexpr (C::EPI == EPI_SWIGLU) {
-                            b0 = t.nt * 128 + p;                 // gate row
-                            b1 = args.b_half + t.nt * 128 + p;   // matching up row
-                        } else {
-                            b0 = t.nt * C::BN + p;
-                            b1 = t.nt * C::BN + 128 + p;
-                        }
-                        sfb0 = sb + ((size_t)gl * args.b_rows_per_group + b0) * args.sf_ld;
-                        sfb1 = sb + ((size_t)gl * args.b_rows_per_group + b1) * args.sf_ld;
                     }
                     for (int kb = 0; kb < t.nkb; ++kb) {
                         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status)) goto pull_done;
@@ -495,8 +499,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                             uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
                             const int at = 16 * (p & 31) + 4 * (p >> 5);
                             cp_async4(sf + at, sfa + kb * 4);
-                            cp_async4(sf + 512 + at, sfb0 + kb * 4);
-                            cp_async4(sf + 1024 + at, sfb1 + kb * 4);
                         }
                         cp_async_arrive_noinc(&full_bar[stage]);
                         if (++stage == C::STAGES) {

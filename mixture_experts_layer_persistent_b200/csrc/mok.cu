@@ -379,7 +379,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         MOK_TRY(mark_fwd(2, stream));
         const long long xb = s.T * s.H / 32;
         quantize_mxfp8_kernel<<<blocks_for(xb, 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(x), xb,
-                                                                        st.xq, st.xs);
+                                                                        st.xq, st.xs, s.H / 32, 0);
         MOK_LAUNCHED();
         CUtensorMap tA, tB, tBs, tO;
         if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, 128, 128, 1)) return MOK_ERR_INVALID;
@@ -406,6 +406,8 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         ga.sfb_src = p.s_gate_up;
         ga.sfb_src_s = s.S ? p.ss_gate_up : p.s_gate_up;
         ga.sf_ld = c.H / 32;
+        ga.sfb_row_tiles = static_cast<int>(s.E * 2 * s.I / 128);
+        ga.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : s.E) * 2 * s.I / 128);
         ga.status = dev.status;
         using CGateUpMx = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU, true>;
         MOK_TRY(launch_gemm<CGateUpMx>(tB, tB, tBs, tO, tO, tO, ga, dev.sms, stream));
@@ -429,6 +431,8 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         gd.sfb_src = p.s_down;
         gd.sfb_src_s = s.S ? p.ss_down : p.s_down;
         gd.sf_ld = c.I / 32;
+        gd.sfb_row_tiles = static_cast<int>(s.E * s.H / 128);
+        gd.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : s.E) * s.H / 128);
         using CDownMx = GemmCfg<256, false, false, false, false, false, EPI_PUSH, true>;
         MOK_TRY(mark_fwd(3, stream));
         MOK_TRY(launch_gemm<CDownMx>(tA, tB, tBs, tO, tO, tO, gd, dev.sms, stream));
@@ -766,18 +770,30 @@ int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, co
     return MOK_OK;
 }
 
-int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *scales, void *stream)
+static int quantize(const void *src, int64_t rows, int64_t K, void *q, void *scales, bool packed, void *stream)
 {
     if (!src || !q || !scales || rows < 0 || K <= 0 || K % 32) return MOK_ERR_INVALID;
+    if (packed && (rows % 128 || K % 128)) return fail(MOK_ERR_INVALID, "moe_quantize_mxfp8_weights: rows and K must be multiples of 128");
     if (!aligned16(src) || !aligned16(q)) return MOK_ERR_INVALID;
     if (!device_info()) return MOK_ERR_DEVICE;
     const long long nb = rows * (K / 32);
     if (nb == 0) return MOK_OK;
     quantize_mxfp8_kernel<<<blocks_for(nb, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const __nv_bfloat16 *>(src), nb, static_cast<uint8_t *>(q), static_cast<uint8_t *>(scales));
+        static_cast<const __nv_bfloat16 *>(src), nb, static_cast<uint8_t *>(q), static_cast<uint8_t *>(scales), K / 32,
+        packed ? rows / 128 : 0);
     if (const cudaError_t e_ = cudaGetLastError(); e_ != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "quantize_mxfp8_kernel launch", e_);
     return MOK_OK;
+}
+
+int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *scales, void *stream)
+{
+    return quantize(src, rows, K, q, scales, false, stream);
+}
+
+int moe_quantize_mxfp8_weights(const void *src, int64_t rows, int64_t K, void *q, void *scales, void *stream)
+{
+    return quantize(src, rows, K, q, scales, true, stream);
 }
 
 int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events, int n_bwd)

@@ -30,9 +30,22 @@ __device__ __forceinline__ float exp2_neg(int e)   // 2^-e for e in [-127, 126]
 }
 
 // Thread = one block of 32 bf16 values: 64-byte load, 32-byte store.
+// Byte offset of scale (row, j) (j = 32-element block along K) in the packed
+// weight-scale layout: (K/128) x (rows/128) tiles of 512 bytes, tile (kb, rb)
+// holding for row r = 128 rb + 32 q + i and block j = 4 kb + s the byte at
+// 16 i + 4 q + s.  That is the layout the block-scaled MMA's scale-factor
+// copy reads for a 128-row block, so one K block of a weight tile's scales
+// is one contiguous 512-byte copy per 128 rows.
+__device__ __forceinline__ long long packed_scale_offset(long long row, long long j, long long row_tiles)
+{
+    return ((j >> 2) * row_tiles + (row >> 7)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (j & 3);
+}
+
+// row_tiles = 0: scales [rows, K/32] row-major; row_tiles = rows / 128: packed layout
 __global__ void __launch_bounds__(256) quantize_mxfp8_kernel(const __nv_bfloat16 *__restrict__ src,
                                                              long long nblocks, uint8_t *__restrict__ q,
-                                                             uint8_t *__restrict__ scales)
+                                                             uint8_t *__restrict__ scales, long long kb32,
+                                                             long long row_tiles)
 {
     const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (b >= nblocks) return;
@@ -65,7 +78,8 @@ __global__ void __launch_bounds__(256) quantize_mxfp8_kernel(const __nv_bfloat16
     uint4 *dst = reinterpret_cast<uint4 *>(q + b * 32);
     dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
     dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    scales[b] = static_cast<uint8_t>(e + 127);
+    const long long at = row_tiles ? packed_scale_offset(b / kb32, b % kb32, row_tiles) : b;
+    scales[at] = static_cast<uint8_t>(e + 127);
 }
 
 }  // namespace mok

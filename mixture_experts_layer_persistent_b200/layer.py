@@ -124,3 +124,15 @@ def quantize_mxfp8(src: torch.Tensor):
     abi.moe_quantize_mxfp8(src.data_ptr(), rows, K, q.data_ptr(), s.data_ptr(),
                            torch.cuda.current_stream(src.device).cuda_stream)
     return q, s
+
+
+def quantize_mxfp8_weights(src: torch.Tensor):
+    """Expert weights bf16 [..., K] -> (e4m3 codes uint8 [..., K], ue8m0 scales as a flat uint8
+    tensor in the packed weight-scale layout of include/mok.h) via libmok."""
+    K = src.shape[-1]
+    rows = src.numel() // K
+    q = torch.empty(src.shape, dtype=torch.uint8, device=src.device)
+    s = torch.empty(rows * (K // 32), dtype=torch.uint8, device=src.device)
+    abi.moe_quantize_mxfp8_weights(src.data_ptr(), rows, K, q.data_ptr(), s.data_ptr(),
+                                   torch.cuda.current_stream(src.device).cuda_stream)
+    return q, s

@@ -69,3 +69,13 @@ def assert_close(got, want, what, rtol=RTOL, atol=ATOL):
 
 def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def packed_scale_offsets(rows, kb32, total_rows):
+    """Byte offsets [len(rows), kb32] of the scales of `rows` in the packed weight-scale
+    layout of include/mok.h (moe_quantize_mxfp8_weights): (K/128) x (total_rows/128)
+    tiles of 512 bytes; row r = 128 rb + 32 q + i, block j = 4 kb + s at byte
+    (kb * total_rows/128 + rb) * 512 + 16 i + 4 q + s."""
+    r = np.asarray(rows, dtype=np.int64)[:, None]
+    j = np.arange(kb32, dtype=np.int64)[None, :]
+    return ((j // 4) * (total_rows // 128) + r // 128) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + (j % 4)

@@ -13,8 +13,8 @@ import pytest
 import torch
 
 import oracle
-from mixture_experts_layer_persistent_b200 import MoELayer, cfg_for, quantize_mxfp8, synth
-from tests._support import assert_close, bits_to_bf16, oracle_layer, to_np
+from mixture_experts_layer_persistent_b200 import MoELayer, cfg_for, quantize_mxfp8_weights, synth
+from tests._support import assert_close, bits_to_bf16, oracle_layer, packed_scale_offsets, to_np
 
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 
@@ -107,13 +107,14 @@ def test_mxfp8_full_size():
     qp = {k: params[k] for k in ("router_w", "e_bias", "logit_bias")}
     for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
                         ("ws_down", "ss_down")):
-        qp[name], qp[sname] = quantize_mxfp8(params[name])
+        qp[name], qp[sname] = quantize_mxfp8_weights(params[name])
     torch.cuda.synchronize()
     # weight quantisation is bit-exact against the oracle's (sampled rows)
     rows = np.array([0, 1, 777, 2 * wl.I * wl.E - 1])
     wq, ws = oracle.mx_quantize(L.arrays["Wgu"].reshape(-1, wl.H)[rows])
     assert np.array_equal(qp["w_gate_up"].view(-1, wl.H)[torch.from_numpy(rows).cuda()].cpu().numpy(), wq)
-    assert np.array_equal(qp["s_gate_up"].view(-1, wl.H // 32)[torch.from_numpy(rows).cuda()].cpu().numpy(), ws)
+    at = packed_scale_offsets(rows, wl.H // 32, 2 * wl.I * wl.E)
+    assert np.array_equal(qp["s_gate_up"][torch.from_numpy(at.ravel()).cuda()].cpu().numpy().reshape(at.shape), ws)
     del params
     layer = MoELayer(cfg_for(wl), qp, training=False, device=torch.device("cuda"))
     routing = layer.new_routing()

@@ -111,14 +111,14 @@ MEDIUM_MX = synth.Workload("medium_mx", T=700, H=512, E=16, k=4, I=256, S=1, Is=
 
 
 def _mx_params(params):
-    from mixture_experts_layer_persistent_b200 import quantize_mxfp8
+    from mixture_experts_layer_persistent_b200 import quantize_mxfp8_weights
     out = {k: params[k] for k in ("router_w", "e_bias", "logit_bias")}
     for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
                         ("ws_down", "ss_down")):
         if params.get(name) is None:
             out[name] = out[sname] = None
             continue
-        out[name], out[sname] = quantize_mxfp8(params[name])
+        out[name], out[sname] = quantize_mxfp8_weights(params[name])
     return out
 
 

@@ -35,3 +35,22 @@ def test_quantize_matches_oracle(shape):
     oq, os_ = oracle.mx_quantize(bits)
     assert np.array_equal(s.cpu().numpy(), os_)
     assert np.array_equal(q.cpu().numpy(), oq)
+
+
+@pytest.mark.parametrize("shape", [(256, 512), (384, 7168)])
+def test_weight_quantize_packs_the_same_scales(shape):
+    """moe_quantize_mxfp8_weights: the same codes as the oracle, and the oracle's scales
+    at the packed weight-scale offsets (every byte of the packed buffer written once)."""
+    from mixture_experts_layer_persistent_b200 import quantize_mxfp8_weights
+    from tests._support import packed_scale_offsets
+    g = torch.Generator().manual_seed(shape[1])
+    x = torch.randn(shape, generator=g) * torch.exp2(torch.randint(-20, 20, (shape[0], 1), generator=g).float())
+    xb = x.to(torch.bfloat16)
+    bits = xb.view(torch.int16).numpy().view(np.uint16)
+    q, s = quantize_mxfp8_weights(xb.cuda())
+    torch.cuda.synchronize()
+    oq, os_ = oracle.mx_quantize(bits)
+    assert np.array_equal(q.cpu().numpy(), oq)
+    at = packed_scale_offsets(np.arange(shape[0]), shape[1] // 32, shape[0])
+    assert np.array_equal(np.sort(at.ravel()), np.arange(s.numel()))
+    assert np.array_equal(s.cpu().numpy()[at], os_)
