@@ -19,6 +19,11 @@ __device__ __forceinline__ void load8(const float *p, float (&v)[8])
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
+__device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&v)[8])
+{
+    unpack8(*reinterpret_cast<const uint4 *>(p), v);
+}
+
 __device__ __forceinline__ uint4 pack8(const float (&v)[8])
 {
     uint4 u;
@@ -31,7 +36,9 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8])
 
 // y[t] = sum_{j<k} w[t,j] O[t,j] (ascending j) + sum_s O[t,k+s] (ascending s), fp32, -> bf16.
 // Thread = 8 columns of one token (16-byte loads).
-__global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ O,
+// O: fp32 slot rows (BF16 layer) or bf16 slot rows (MXFP8 forward)
+template <class Slot>
+__global__ void __launch_bounds__(256) combine_kernel(const Slot *__restrict__ O,
                                                       const float *__restrict__ topk_w,
                                                       __nv_bfloat16 *__restrict__ y, int T, int H, int k, int S)
 {
@@ -41,7 +48,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float *__restrict__ 
     const int t = (int)(i / cpr), c = (int)(i % cpr) * 8;
     const int kk = k + S;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const float *row = O + (size_t)t * kk * H + c;
+    const Slot *row = O + (size_t)t * kk * H + c;
     for (int j = 0; j < kk; ++j) {
         const float w = j < k ? topk_w[(size_t)t * k + j] : 1.0f;
         float v[8];

@@ -739,6 +739,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         }
                     }
                 }
+            } else if constexpr (C::EPI == EPI_PUSH && C::MX) {
+                // MXFP8 forward: bf16 rows pushed into their (token, slot) row
+                const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
+                __nv_bfloat16 *dst = args.out + (size_t)dst_row * args.ldo + t.nt * C::BN;
+#pragma unroll 1
+                for (int c = 0; c < C::BN; c += 64) {
+                    float v[64];
+                    uint32_t p[32];
+                    tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
+                    tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                    tmem_ld_wait();
+                    pack_bf16<64>(v, p);
+                    if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
+                    else if (valid) store_row_direct(dst + c, p);
+                }
             } else if constexpr (C::EPI == EPI_PUSH) {
                 // fp32 rows pushed into their (token, slot) row of the slot buffer
                 const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;

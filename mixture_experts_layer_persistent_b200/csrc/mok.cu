@@ -176,7 +176,7 @@ struct State {
     float *topk_w, *topk_p, *row_w, *rpart;
     __nv_bfloat16 *wr3;
     __nv_bfloat16 *gu, *h, *hw;
-    float *O;                       // per-(token, slot) rows, fp32
+    float *O;                       // per-(token, slot) rows: fp32 (BF16), bf16 (MXFP8 forward)
     uint8_t *xq, *xs, *hq, *hs;     // MXFP8 operands
     size_t bytes;
 };
@@ -215,7 +215,7 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
         st.h = cv.take<__nv_bfloat16>(s.R * s.I);
         st.hq = st.hs = st.xq = st.xs = nullptr;
     }
-    st.O = cv.take<float>(s.T * s.kk * s.H);
+    st.O = mx ? reinterpret_cast<float *>(cv.take<__nv_bfloat16>(s.T * s.kk * s.H)) : cv.take<float>(s.T * s.kk * s.H);
     st.bytes = align_up(cv.off, 256);
     return st;
 }
@@ -416,14 +416,14 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 128, 256, 1)) return MOK_ERR_INVALID;
         if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 128, 256, 1))
             return MOK_ERR_INVALID;
-        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 32, 1, 4)) return MOK_ERR_INVALID;
+        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;   // bf16 slot rows
         GemmArgs gd = ga;
         gd.n_tiles = c.H / 256;
         gd.num_kb = c.I / 128;
         gd.b_rows_per_group = c.H;
         gd.b_half = 0;
-        gd.out = nullptr;
-        gd.out_f32 = st.O;
+        gd.out = reinterpret_cast<__nv_bfloat16 *>(st.O);
+        gd.out_f32 = nullptr;
         gd.out_scales = nullptr;
         gd.ldo = c.H;
         gd.gather_src = nullptr;
@@ -490,9 +490,13 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     }
 
     MOK_TRY(mark_fwd(4, stream));
-    combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(st.O, st.topk_w,
-                                                                       static_cast<__nv_bfloat16 *>(y), c.T, c.H,
-                                                                       c.top_k, c.n_shared);
+    if (mx)
+        combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(
+            reinterpret_cast<const __nv_bfloat16 *>(st.O), st.topk_w, static_cast<__nv_bfloat16 *>(y), c.T, c.H,
+            c.top_k, c.n_shared);
+    else
+        combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(
+            st.O, st.topk_w, static_cast<__nv_bfloat16 *>(y), c.T, c.H, c.top_k, c.n_shared);
     MOK_LAUNCHED();
     MOK_TRY(mark_fwd(5, stream));
 
