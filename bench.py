@@ -429,7 +429,8 @@ def e2e_run(layer, wl, x, dy, grads, K, world, dist):
     def step():
         abi.moe_fwd_host(c, hx.data_ptr(), layer.cparams, hy.data_ptr(), layer.ctx.data_ptr(),
                          layer.ctx_bytes, 1, scratch.data_ptr(), n, st)
-        abi.moe_bwd_host(c, hx.data_ptr(), hdy.data_ptr(), layer.cparams, layer.ctx.data_ptr(),
+        # x stays in the scratch between the two calls (x_host = NULL): uploaded once per step
+        abi.moe_bwd_host(c, None, hdy.data_ptr(), layer.cparams, layer.ctx.data_ptr(),
                          layer.ctx_bytes, hdx.data_ptr(), g, scratch.data_ptr(), n, st)
 
     step()
@@ -449,7 +450,7 @@ def e2e_run(layer, wl, x, dy, grads, K, world, dist):
     nb = wl.T * wl.H * 2
     return {"value": wl.T * world * K / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": 2 * nb,
             "d2h_bytes_per_step": 2 * nb, "ms_per_step": ms / K,
-            "api": "moe_fwd_host + moe_bwd_host (pinned host x, dy -> y, dx)"}
+            "api": "moe_fwd_host + moe_bwd_host (pinned host x, dy -> y, dx; x uploaded once per step)"}
 
 
 def reference_arm(args, world):

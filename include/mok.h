@@ -159,7 +159,10 @@ int moe_bwd(const moe_cfg *cfg, const void *x, const void *dy, const moe_params 
  * memory; the call copies them through the scratch buffer (which must then be
  * at least moe_host_scratch_size bytes), runs the layer on `stream` and
  * synchronises that stream before returning.  Parameters, ctx and the other
- * gradients stay on the device.
+ * gradients stay on the device.  moe_bwd_host takes x_host = NULL to reuse the
+ * x that the preceding moe_fwd_host on the same stream left in the first
+ * T*H*2 bytes of the same scratch buffer (nothing else may have written that
+ * buffer in between): the second upload of x is then skipped.
  */
 int moe_host_scratch_size(const moe_cfg *cfg, int backward, size_t *bytes);
 int moe_fwd_host(const moe_cfg *cfg, const void *x_host, const moe_params *params, void *y_host,

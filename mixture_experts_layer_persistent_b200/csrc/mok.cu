@@ -755,7 +755,7 @@ int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, co
                  size_t scratch_bytes, void *stream)
 {
     MOK_TRY(check_cfg(cfg));
-    if (!x_host || !dy_host || !dx_host || !scratch || !grads) return MOK_ERR_INVALID;
+    if (!dy_host || !dx_host || !scratch || !grads) return MOK_ERR_INVALID;
     size_t need = 0;
     moe_host_scratch_size(cfg, 1, &need);
     if (scratch_bytes < need) return MOK_ERR_WORKSPACE;
@@ -763,7 +763,8 @@ int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, co
     char *s = static_cast<char *>(scratch);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t nb = static_cast<size_t>(cfg->T) * cfg->H * 2;
-    if (const cudaError_t e_ = cudaMemcpyAsync(s, x_host, nb, cudaMemcpyHostToDevice, st); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync", e_);
+    if (x_host)                 // NULL: x is still in the scratch from the preceding moe_fwd_host
+        if (const cudaError_t e_ = cudaMemcpyAsync(s, x_host, nb, cudaMemcpyHostToDevice, st); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync", e_);
     if (const cudaError_t e_ = cudaMemcpyAsync(s + io, dy_host, nb, cudaMemcpyHostToDevice, st); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync", e_);
     moe_grads g = *grads;
     g.dx = s + 2 * io;

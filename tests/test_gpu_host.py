@@ -1,0 +1,51 @@
+"""The host-buffer entry points (moe_fwd_host, moe_bwd_host) against the device API.
+
+They run the same kernels on copies of the same inputs, so y, dx and the weight
+gradients must match the device-pointer calls byte for byte, both when
+moe_bwd_host uploads x itself and when it reuses the x that moe_fwd_host left in
+the scratch buffer (x_host = NULL).
+"""
+import pytest
+import torch
+
+from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, synth
+from tests._support import make_case
+
+pytestmark = pytest.mark.gpu
+
+WL = synth.Workload("host_medium", T=333, H=768, E=12, k=3, I=384, S=2, Is=384, seed=41)
+
+
+@pytest.mark.parametrize("reuse_x", [False, True], ids=["upload_x", "reuse_x"])
+def test_host_entry_points_match_device_api(reuse_x):
+    case = make_case(WL, device="cuda", gen_device="cpu")
+    dev = torch.device("cuda")
+    layer = MoELayer(cfg_for(WL), case["params"], training=True, device=dev)
+    y_ref = layer.forward(case["x"]).clone()
+    g_ref = {k: (v.clone() if v is not None else None) for k, v in layer.backward(case["x"], case["dy"]).items()}
+    torch.cuda.synchronize()
+
+    c = layer.cfg
+    hx = case["x"].cpu().pin_memory()
+    hdy = case["dy"].cpu().pin_memory()
+    hy = torch.empty_like(hx).pin_memory()
+    hdx = torch.empty_like(hx).pin_memory()
+    n = max(abi.moe_host_scratch_size(c, False), abi.moe_host_scratch_size(c, True))
+    scratch = torch.empty(n, dtype=torch.uint8, device=dev)
+    grads = layer.new_grads()
+    g = abi.moe_grads(None, grads["dw_gate_up"].data_ptr(), grads["dw_down"].data_ptr(),
+                      grads["drouter_w"].data_ptr(),
+                      grads["dws_gate_up"].data_ptr() if grads["dws_gate_up"] is not None else None,
+                      grads["dws_down"].data_ptr() if grads["dws_down"] is not None else None)
+    st = layer.stream()
+    abi.moe_fwd_host(c, hx.data_ptr(), layer.cparams, hy.data_ptr(), layer.ctx.data_ptr(), layer.ctx_bytes, 1,
+                     scratch.data_ptr(), n, st)
+    abi.moe_bwd_host(c, None if reuse_x else hx.data_ptr(), hdy.data_ptr(), layer.cparams, layer.ctx.data_ptr(),
+                     layer.ctx_bytes, hdx.data_ptr(), g, scratch.data_ptr(), n, st)
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    assert torch.equal(hy.view(torch.int16), y_ref.cpu().view(torch.int16))
+    assert torch.equal(hdx.view(torch.int16), g_ref["dx"].cpu().view(torch.int16))
+    for k in ("dw_gate_up", "dw_down", "dws_gate_up", "dws_down"):
+        assert torch.equal(grads[k].view(torch.int16), g_ref[k].view(torch.int16)), k
+    assert torch.equal(grads["drouter_w"].view(torch.int32), g_ref["drouter_w"].view(torch.int32))
