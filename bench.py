@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--extra-workloads", default="small,dsv3_zipf",
+                    help="BF16 workloads also measured, comma-separated ('none' to skip)")
     ap.add_argument("--mx-workload", default="dsv3_mxfp8",
                     help="MXFP8 forward workload measured after the main one ('none' to skip)")
     return ap.parse_args()
@@ -308,11 +310,20 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_sample(wl, params, x, dy, args.cpu_seconds)
 
+    del layer, grads, params
+    torch.cuda.empty_cache()
+
+    # ---------------- the other BF16 workloads (the small forward, the skewed fwd+bwd)
+    extra = {}
+    for name in ([] if args.extra_workloads in ("", "none") else args.extra_workloads.split(",")):
+        ewl = synth.WORKLOADS[name]
+        extra[name] = bf16_workload_run(synth.scaled(ewl, seed=ewl.seed + 1000 * rank), dev, K, args.warmup, world,
+                                        dist, pk)
+        torch.cuda.empty_cache()
+
     # ---------------- MXFP8 forward (block-scaled e4m3) on its own workload
     mx = None
     if args.mx_workload and args.mx_workload != "none":
-        del layer, grads, params
-        torch.cuda.empty_cache()
         mwl = synth.WORKLOADS[args.mx_workload]
         mx = mxfp8_run(synth.scaled(mwl, seed=mwl.seed + 1000 * rank), dev, K, args.warmup, world, dist, pk)
 
@@ -347,11 +358,75 @@ def main():
             },
             "roofline": roof,
             "mxfp8": mx,
+            "bf16_workloads": extra,
             "e2e": e2e, "cpu_baseline": cpu,
         }
         print(json.dumps(line))
     if world > 1:
         dist.destroy_process_group()
+
+
+def bf16_workload_run(wl, dev, K, warmup, world, dist, pk):
+    """Tokens/s and tensor-core fractions of the BF16 layer on another workload (forward, and
+    backward when the workload has one), per-phase CUDA events on the layer's stream."""
+    import torch
+    from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, moe_trace_events, synth
+    params = synth.draw_params(wl, dev)
+    x = synth.draw_x(wl, dev)
+    dy = synth.draw_dy(wl, dev) if wl.backward else None
+    layer = MoELayer(cfg_for(wl), params, training=wl.backward, device=dev)
+    y = torch.empty_like(x)
+    grads = layer.new_grads() if wl.backward else None
+    routing = layer.new_routing()
+    layer.forward(x, y, routing=routing)
+    counts = routing["counts"].cpu().numpy()
+    for _ in range(warmup):
+        layer.forward(x, y)
+        if wl.backward:
+            layer.backward(x, dy, grads)
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    fev = [[mk() for _ in range(abi.MOK_FWD_PHASES + 1)] for _ in range(K)]
+    bev = [[mk() for _ in range(abi.MOK_BWD_PHASES + 1)] for _ in range(K)]
+    for e in [e for ev in fev + bev for e in ev]:
+        e.record()
+    start, end = mk(), mk()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    start.record()
+    for i in range(K):
+        moe_trace_events([e.cuda_event for e in fev[i]], [e.cuda_event for e in bev[i]] if wl.backward else None)
+        layer.forward(x, y)
+        if wl.backward:
+            layer.backward(x, dy, grads)
+    end.record()
+    torch.cuda.synchronize()
+    moe_trace_events(None, None)
+    status = layer.status()
+    t = torch.tensor([start.elapsed_time(end)], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / K
+    fwd_ms = statistics.mean(fev[i][0].elapsed_time(fev[i][-1]) for i in range(K))
+    bwd_ms = statistics.mean(bev[i][0].elapsed_time(bev[i][-1]) for i in range(K)) if wl.backward else 0.0
+    fwd_flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
+    out = {"workload": f"{wl.name}: MoE layer {'fwd+bwd' if wl.backward else 'fwd'} BF16, T={wl.T}, H={wl.H}, "
+                       f"E={wl.E}, top-{wl.k}, I={wl.I}, {wl.S} shared"
+                       + (f", Zipf({wl.zipf}) logit term" if wl.zipf else ""),
+           "tokens_per_s": wl.T * world / (ms / 1e3), "ms_per_step": ms,
+           "fwd_ms": fwd_ms, "fwd_tokens_per_s": wl.T / (fwd_ms / 1e3),
+           "fwd_tc_peak_frac_of_measured_burst": fwd_flops / (fwd_ms / 1e3) / 1e12 / pk["bf16"],
+           "fwd_tc_peak_frac_of_measured_sustained": fwd_flops / (fwd_ms / 1e3) / 1e12 / pk["bf16_sustained"],
+           "expert_load_max_over_mean": float(counts.max() / max(1e-9, counts.mean())),
+           "empty_experts": int((counts == 0).sum()), "device_status": status}
+    if wl.backward:
+        out.update({"bwd_ms": bwd_ms, "bwd_tokens_per_s": wl.T / (bwd_ms / 1e3),
+                    "bwd_tc_peak_frac_of_measured_burst": 2 * fwd_flops / (bwd_ms / 1e3) / 1e12 / pk["bf16"],
+                    "bwd_tc_peak_frac_of_measured_sustained":
+                        2 * fwd_flops / (bwd_ms / 1e3) / 1e12 / pk["bf16_sustained"]})
+    del layer, params, grads
+    return out
 
 
 def mxfp8_run(wl, dev, K, warmup, world, dist, pk):
