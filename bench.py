@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/s fwd MXFP8 & BF16, bwd BF16; % of tensor-core peak"
 FWD_PHASES = ["router", "dispatch", "gate_up_gemm", "down_gemm", "combine"]
-BWD_PHASES = ["slot_grad", "drouter_partial", "drouter_reduce", "down_dgrad_gemm", "down_wgrad_gemm",
+BWD_PHASES = ["down_dgrad_gemm", "slot_grad", "drouter_partial", "drouter_reduce", "down_wgrad_gemm",
               "gate_up_dgrad_gemm", "gate_up_wgrad_gemm", "dx_sum"]
 
 

@@ -206,10 +206,11 @@ int moe_quantize_mxfp8_weights(const void *src, int64_t rows, int64_t K, void *q
  * cudaEvent_t handles owned by the caller.  Phases:
  *   forward  (MOK_FWD_PHASES = 5, needs 6 events): router, dispatch,
  *            gate/up GEMM, down GEMM, combine
- *   backward (MOK_BWD_PHASES = 8, needs 9 events): slot gradient,
- *            router-gradient partial sums, router-gradient reduction,
- *            down dgrad GEMM, down wgrad GEMM, gate/up dgrad GEMM,
- *            gate/up wgrad GEMM, dx sum
+ *   backward (MOK_BWD_PHASES = 8, needs 9 events): down dgrad GEMM (its
+ *            epilogue also forms the slot-gradient partial sums), slot
+ *            gradient, router-gradient partial sums, router-gradient
+ *            reduction, down wgrad GEMM, gate/up dgrad GEMM, gate/up wgrad
+ *            GEMM, dx sum
  * Pass n = 0 to stop tracing.  The setting is per host thread.
  */
 #define MOK_FWD_PHASES 5

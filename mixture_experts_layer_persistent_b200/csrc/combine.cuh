@@ -59,67 +59,41 @@ __global__ void __launch_bounds__(256) combine_kernel(const Slot *__restrict__ O
     *reinterpret_cast<uint4 *>(y + (size_t)t * H + c) = pack8(acc);
 }
 
-// Backward, per token: G_j = <dy[t], O[t,j]> (j < k), then the logit gradient
+// Backward, per token: G_j = <dy[t], o_j> (j < k), summed in a fixed order from the
+// per-N-tile partials <dy W_down, h> that the down dgrad GEMM's epilogue wrote for
+// the slot's sorted row (o_j = h_j W_down^T, so the two are equal), then the logit
+// gradient
 //   softmax: dl_j = w_j (G_j - sum_i q_i G_i),             q = w / routed_scale
 //   sigmoid: dl_j = rho/S (G_j - sum_i q_i G_i) s_j (1 - s_j), S = sum of selected s
-// One block of 256 threads per token; each thread sums a fixed column subset,
-// then a fixed-shape tree over threads.
-__global__ void __launch_bounds__(256) slot_grad_kernel(const __nv_bfloat16 *__restrict__ dy,
-                                                        const float *__restrict__ O,
+// One thread per token.
+__global__ void __launch_bounds__(256) slot_grad_kernel(const float *__restrict__ gpart, int n_parts,
+                                                        const int *__restrict__ inv_perm,
                                                         const float *__restrict__ topk_w,
                                                         const float *__restrict__ topk_p, float *__restrict__ dl,
-                                                        int T, int H, int k, int S, int score_fn,
-                                                        float routed_scale)
+                                                        int T, int k, int score_fn, float routed_scale)
 {
-    __shared__ float s_red[8][16];
-    const int t = blockIdx.x;
-    const int kk = k + S;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    float g[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) g[j] = 0.0f;
-    const __nv_bfloat16 *dyr = dy + (size_t)t * H;
-    const float *orow = O + (size_t)t * kk * H;
-    for (int c = tid * 8; c < H; c += 256 * 8) {
-        float d[8];
-        unpack8(*reinterpret_cast<const uint4 *>(dyr + c), d);
-        for (int j = 0; j < k; ++j) {
-            float o[8];
-            load8(orow + (size_t)j * H + c, o);
-            float s = g[j];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) s = fmaf(d[q], o[q], s);
-            g[j] = s;
-        }
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    float G[16], q[16];
+    float gbar = 0.0f, S_ = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        const float *gp = gpart + (size_t)inv_perm[(size_t)t * k + j] * n_parts;
+        float v = 0.0f;
+        for (int p = 0; p < n_parts; ++p) v += gp[p];
+        G[j] = v;
+        q[j] = topk_w[(size_t)t * k + j] / routed_scale;
+        gbar = fmaf(q[j], G[j], gbar);
+        S_ += topk_p[(size_t)t * k + j];
     }
     for (int j = 0; j < k; ++j) {
-        float v = g[j];
-#pragma unroll
-        for (int d = 16; d >= 1; d >>= 1) v += __shfl_xor_sync(0xffffffffu, v, d);
-        if (lane == 0) s_red[warp][j] = v;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        float G[16], q[16];
-        float gbar = 0.0f, S_ = 0.0f;
-        for (int j = 0; j < k; ++j) {
-            float v = 0.0f;
-            for (int w = 0; w < 8; ++w) v += s_red[w][j];
-            G[j] = v;
-            q[j] = topk_w[(size_t)t * k + j] / routed_scale;
-            gbar = fmaf(q[j], G[j], gbar);
-            S_ += topk_p[(size_t)t * k + j];
+        float r;
+        if (score_fn == 0) {
+            r = topk_w[(size_t)t * k + j] * (G[j] - gbar);
+        } else {
+            const float s = topk_p[(size_t)t * k + j];
+            r = routed_scale / S_ * (G[j] - gbar) * s * (1.0f - s);
         }
-        for (int j = 0; j < k; ++j) {
-            float r;
-            if (score_fn == 0) {
-                r = topk_w[(size_t)t * k + j] * (G[j] - gbar);
-            } else {
-                const float s = topk_p[(size_t)t * k + j];
-                r = routed_scale / S_ * (G[j] - gbar) * s * (1.0f - s);
-            }
-            dl[(size_t)t * k + j] = r;
-        }
+        dl[(size_t)t * k + j] = r;
     }
 }
 

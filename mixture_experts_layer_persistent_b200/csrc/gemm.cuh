@@ -71,6 +71,8 @@ struct GemmArgs {
     __nv_bfloat16 *out3;          // EPI_SWIGLU: w * h [R, I] (or null)
     float *out_f32;               // EPI_ROUTER: partial logits [n_tiles, rows, 256]; EPI_PUSH: fp32 slot rows
     const __nv_bfloat16 *aux;     // EPI_DSWIGLU: saved gate/up pre-activations [R, 2I]
+    const __nv_bfloat16 *aux_h;   // EPI_DSWIGLU: saved h [R, I] (the down GEMM's A operand)
+    float *gpart;                 // EPI_DSWIGLU: <dy W_down, h> of each routed row over each N tile [R_routed, n_tiles]
     int ldo;                      // elements per output row
     int inter;                    // I
     int rows_total;               // EPI_ROUTER: rows of one partial-logit slab (T)
@@ -803,11 +805,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const int n0 = t.nt * C::BN;
                 const float w = valid ? args.row_w[r] : 0.0f;
                 const __nv_bfloat16 *gsrc = valid ? args.aux + (size_t)r * 2 * I + n0 : nullptr;
+                // slot gradient of a routed row: G = <dy, o> = <dy W_down, h>, summed here over
+                // this tile's columns (v before the routing weight) against the saved h
+                const bool routed_row = valid && t.g < args.num_routed;
+                const __nv_bfloat16 *hsrc = routed_row ? args.aux_h + (size_t)r * I + n0 : nullptr;
+                float gsum = 0.0f;
 #pragma unroll 1
                 for (int c = 0; c < C::BN; c += 64) {
-                    uint32_t gp[32], up[32], dgp[32], dup[32];
+                    uint32_t gp[32], up[32], dgp[32], dup[32], hp[32];
                     load_row_direct(gp, gsrc ? gsrc + c : nullptr);
                     load_row_direct(up, gsrc ? gsrc + I + c : nullptr);
+                    load_row_direct(hp, hsrc ? hsrc + c : nullptr);
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         float v[32], dg[32], du[32];
@@ -816,8 +824,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
                             const uint32_t gw = gp[16 * half + (i >> 1)], uw = up[16 * half + (i >> 1)];
+                            const uint32_t hw = hp[16 * half + (i >> 1)];
                             const float gi = (i & 1) ? bf16_hi(gw) : bf16_lo(gw);
                             const float ui = (i & 1) ? bf16_hi(uw) : bf16_lo(uw);
+                            gsum = fmaf(v[i], (i & 1) ? bf16_hi(hw) : bf16_lo(hw), gsum);
                             const float dh = w * v[i];
                             const float sg = 1.0f / (1.0f + expf(-gi));
                             dg[i] = dh * ui * sg * (1.0f + gi * (1.0f - sg));
@@ -834,6 +844,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         store_row_direct(args.out + (size_t)r * 2 * I + I + n0 + c, dup);
                     }
                 }
+                if (routed_row) args.gpart[(size_t)r * args.n_tiles + t.nt] = gsum;
             } else {   // EPI_ROUTER: fp32 partial logits of this K split
                 const int r = t.m0 + row;
 #pragma unroll 1

@@ -222,6 +222,7 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
 
 struct BwdScratch {
     float *dl, *partial, *dxs;    // dxs: per-(token, slot) dx rows, fp32
+    float *gpart;                 // per routed row and N tile of the down dgrad: <dy W_down, h>
     __nv_bfloat16 *dgu;
     size_t bytes;
 };
@@ -232,6 +233,7 @@ BwdScratch carve_bwd(const moe_cfg &c, void *buf)
     Carver cv(buf);
     BwdScratch b{};
     b.dl = cv.take<float>(s.TK);
+    b.gpart = cv.take<float>(s.TK * (s.I / 128));
     b.partial = cv.take<float>(s.max_chunks * s.H);
     b.dgu = cv.take<__nv_bfloat16>(s.R * 2 * s.I);
     b.dxs = cv.take<float>(s.T * s.kk * s.H);
@@ -520,20 +522,6 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     t_launches = 0;
     const __nv_bfloat16 *dyb = static_cast<const __nv_bfloat16 *>(dy);
 
-    MOK_TRY(mark_bwd(0, stream));
-    slot_grad_kernel<<<c.T, 256, 0, stream>>>(dyb, st.O, st.topk_w, st.topk_p, bs.dl, c.T, c.H, c.top_k,
-                                              c.n_shared, c.score_fn, c.routed_scale);
-    MOK_LAUNCHED();
-    MOK_TRY(mark_bwd(1, stream));
-    drouter_partial_kernel<<<dim3(static_cast<unsigned>(s.max_chunks), c.H / 256), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(x), bs.dl, st.offsets, st.chunk_start, st.perm, bs.partial, c.H, c.E,
-        c.top_k, kChunkRows);
-    MOK_LAUNCHED();
-    MOK_TRY(mark_bwd(2, stream));
-    drouter_reduce_kernel<<<blocks_for(s.E * s.H, 256), 256, 0, stream>>>(bs.partial, st.chunk_start,
-                                                                          gr.drouter_w, c.H, c.E);
-    MOK_LAUNCHED();
-
     GemmArgs base{};
     base.num_groups = static_cast<int>(s.G);
     base.num_routed = c.E;
@@ -555,8 +543,10 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g1.num_kb = c.H / BK;
     g1.b_rows_per_group = c.H;
     g1.aux = st.gu;
+    g1.aux_h = st.h;
+    g1.gpart = bs.gpart;
     g1.out = bs.dgu;
-    MOK_TRY(mark_bwd(3, stream));
+    MOK_TRY(mark_bwd(0, stream));
     if (!make_tmap(&tO, bs.dgu, 2 * s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
     if (c.I % 256 == 0) {      // N = 256 halves the gathered dy rows per weight byte
         g1.n_tiles = c.I / 256;
@@ -567,6 +557,22 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
         using CDgradDown = GemmCfg<128, false, true, true, false, false, EPI_DSWIGLU>;
         MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, tO, tO, tO, g1, dev.sms, stream));
     }
+
+    // slot gradients from the down dgrad's partials, then the router weight gradient
+    MOK_TRY(mark_bwd(1, stream));
+    slot_grad_kernel<<<blocks_for(s.T, 256), 256, 0, stream>>>(bs.gpart, g1.n_tiles, st.inv_perm, st.topk_w,
+                                                              st.topk_p, bs.dl, c.T, c.top_k, c.score_fn,
+                                                              c.routed_scale);
+    MOK_LAUNCHED();
+    MOK_TRY(mark_bwd(2, stream));
+    drouter_partial_kernel<<<dim3(static_cast<unsigned>(s.max_chunks), c.H / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(x), bs.dl, st.offsets, st.chunk_start, st.perm, bs.partial, c.H, c.E,
+        c.top_k, kChunkRows);
+    MOK_LAUNCHED();
+    MOK_TRY(mark_bwd(3, stream));
+    drouter_reduce_kernel<<<blocks_for(s.E * s.H, 256), 256, 0, stream>>>(bs.partial, st.chunk_start,
+                                                                          gr.drouter_w, c.H, c.E);
+    MOK_LAUNCHED();
 
     // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
     GemmArgs g2 = base;
