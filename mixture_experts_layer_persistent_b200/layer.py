@@ -26,7 +26,7 @@ def cfg_for(wl, dtype=None) -> abi.moe_cfg:
     if dtype is None:
         dtype = abi.MOK_DTYPE_MXFP8 if wl.mxfp8 else abi.MOK_DTYPE_BF16
     return make_cfg(wl.T, wl.H, wl.E, wl.I, wl.k, wl.S, wl.Is, wl.score_fn, wl.n_group,
-                    wl.topk_group, 1.0, dtype)
+                    wl.topk_group, wl.routed_scale, dtype)
 
 
 class MoELayer:

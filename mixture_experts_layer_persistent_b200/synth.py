@@ -38,6 +38,7 @@ class Workload:
     n_group: int = 1
     topk_group: int = 1
     zipf: float = 0.0          # >0: add -zipf*ln(rank) to the logits
+    routed_scale: float = 1.0  # factor on the renormalised routing weights
     mxfp8: bool = False
     backward: bool = True
     seed: int = 0

@@ -18,7 +18,7 @@ def bits_to_bf16(bits: np.ndarray, device="cpu") -> torch.Tensor:
 def oracle_layer(wl, params, x_bits, dy_bits=None, mx=False, pure=False, weights=None):
     """Oracle layer of a workload; params are torch tensors (any device)."""
     L = oracle.Layer(wl.T, wl.H, wl.E, wl.k, wl.I, S=wl.S, Is=wl.Is, score_fn=wl.score_fn,
-                     n_group=wl.n_group, topk_group=wl.topk_group, routed_scale=1.0, mx=mx,
+                     n_group=wl.n_group, topk_group=wl.topk_group, routed_scale=wl.routed_scale, mx=mx,
                      pure=pure)
     f32 = lambda t: None if t is None else t.detach().float().cpu().numpy()
     w = weights or {}
