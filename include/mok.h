@@ -256,11 +256,11 @@ int moe_launch_count(int *count);
 
 /*
  * Fault-injection hook for testing the bounded waits.  While enabled (non-zero),
- * every forward launched by this host thread makes CTA 0 of the gate/up GEMM
- * skip the signal that hands its first accumulator to the epilogue; the
- * epilogue's wait then runs out after about 2 s, the kernel records
- * MOK_STATUS_TIMEOUT and returns (no trap, no fault).  Results of such a call
- * are meaningless.  Off by default.
+ * every BF16 forward launched by this host thread makes CTA 0 of the gate/up
+ * GEMM and CTA 0 of the down GEMM skip the signal that hands their first
+ * accumulator to the epilogue; each epilogue's wait then runs out after about
+ * 2 s, the kernel records MOK_STATUS_TIMEOUT and returns (no trap, no fault).
+ * Results of such a call are meaningless.  Off by default.
  */
 int moe_test_drop_signal(int enable);
 
