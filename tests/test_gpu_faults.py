@@ -1,10 +1,10 @@
 """Failure detection without a GPU fault: a signal that never comes.
 
-With the fault-injection hook on, CTA 0 of the gate/up GEMM skips the signal
-that hands its first accumulator to the epilogue.  The epilogue's bounded wait
-must run out (about 2 s), record MOK_STATUS_TIMEOUT in the device status word
-and let the kernel return; the context stays usable and the next forward is
-correct.  The tiny workload gives every CTA a single tile, so nothing of CTA 0
+With the fault-injection hook on, CTA 0 of the gate/up GEMM (and of the down
+GEMM) skips the signal that hands its first accumulator to the epilogue.  The
+epilogue's bounded wait must run out (about 2 s), record MOK_STATUS_TIMEOUT in
+the device status word and let the kernel return; the context stays usable and
+the next forward is correct.  The tiny workload gives every CTA a single tile, so nothing of CTA 0
 is still in flight when its wait runs out.
 """
 import time
