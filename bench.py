@@ -296,6 +296,12 @@ def main():
     roof["peak_source"] = pk["source"] + (" sustained bf16" if roof["bound"] == "tensor" else " hbm copy")
     roof["algorithmic_flops"] = flops
     roof["algorithmic_bytes"] = nbytes
+    # every GEMM phase against both measured peaks (algorithmic bytes and FLOPs / its event time)
+    phase_roofline = {}
+    for name, (fl, nb) in alg.items():
+        t = phase[name] / 1e3
+        phase_roofline[name] = {"ms": round(phase[name], 4), "hbm_frac": round(nb / t / 1e9 / pk["hbm_gbs"], 4),
+                                "tc_frac_sustained": round(fl / t / 1e12 / pk["bf16_sustained"], 4)}
 
     total_flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
     fwd_tps = wl.T / (fwd_ms / 1e3)
@@ -357,6 +363,7 @@ def main():
                 "empty_experts": int((counts == 0).sum()),
             },
             "roofline": roof,
+            "phase_roofline": phase_roofline,
             "mxfp8": mx,
             "bf16_workloads": extra,
             "e2e": e2e, "cpu_baseline": cpu,
