@@ -122,6 +122,10 @@ typedef struct moe_grads {
  *                     gate/up pre-activations, h, weighted h, per-slot rows)
  *   fwd_scratch_bytes temporary device memory of moe_fwd
  *   bwd_scratch_bytes temporary device memory of moe_bwd
+ * The forward's buffer (ctx or forward scratch) and the backward scratch also
+ * hold the tile counters of that pass's grouped GEMMs.  The pass zeroes them
+ * on its stream before its first launch, so nothing needs to start at zero.
+ * Two passes that overlap on the GPU need separate buffers.
  * Any output pointer may be NULL.  Returns MOK_ERR_INVALID for a bad cfg.
  */
 int moe_workspace_size(const moe_cfg *cfg, size_t *ctx_bytes, size_t *fwd_scratch_bytes,

@@ -82,6 +82,7 @@ struct GemmArgs {
     int k_split;                  // ragged-K: > 0 limits the streaming kernel to groups with more rows
                                   // (a prefix of gorder); the resident kernel takes the rest
     int m_per_unit;               // resident weight-gradient kernel: M tiles per work unit
+    int *sched;                   // tile counter of this launch, zero before it (one per launch)
 };
 
 template <int BN_, bool A_MN_, bool B_MN_, bool A_GATHER_, bool B_GATHER_, bool RAGGED_K_, int EPI_,
@@ -213,6 +214,48 @@ __device__ __forceinline__ void pack_bf16(const float *v, uint32_t *p)
     for (int i = 0; i < N / 2; ++i) p[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
 }
 
+// ---- tile schedule ----------------------------------------------------------
+// Tiles start in index order.  CTA b takes tile b first; afterwards its
+// producer claims the next index from the launch's counter kClaimAhead K blocks
+// before the last load of its current tile (so the atomic's latency hides
+// behind those loads) and hands it to the other roles through a ring of
+// shared-memory slots.  The tiles that share a weight strip
+// (an expert's M tiles of one N strip, adjacent in the raster) therefore start
+// within about a microsecond of each other and read the strip from HBM once,
+// where a fixed stride of gridDim.x lets the CTAs drift apart over the waves.
+// A tile's result does not depend on the CTA that computes it.
+constexpr int kSchedSlots = 4;
+constexpr int kClaimAhead = 8;     // K blocks before a tile's last load at which the next tile is claimed
+
+struct Sched {
+    uint64_t *full;     // [kSchedSlots] slot written (one producer arrival)
+    uint64_t *empty;    // [kSchedSlots] slot read by every consuming warp
+    int *slot;          // [kSchedSlots] tile indices
+};
+
+// producer lane 0: publish the tile of turn `it` (total = no more work)
+__device__ __forceinline__ bool sched_put(const Sched &s, int it, int tile, volatile int *abort_flag, int *status)
+{
+    const int k = it % kSchedSlots;
+    if (!mbar_wait(&s.empty[k], (static_cast<uint32_t>(it / kSchedSlots) & 1u) ^ 1u, abort_flag, status)) return false;
+    s.slot[k] = tile;
+    mbar_arrive(&s.full[k]);             // release: the slot is visible to the waiters
+    return true;
+}
+
+// a consuming warp: the tile of turn `it` (total when the work is out or a wait gave up)
+__device__ __forceinline__ int sched_take(const Sched &s, int it, int total, int lane, volatile int *abort_flag,
+                                          int *status)
+{
+    const int k = it % kSchedSlots;
+    int tile = total;
+    if (lane == 0) {
+        if (mbar_wait(&s.full[k], static_cast<uint32_t>(it / kSchedSlots) & 1u, abort_flag, status)) tile = s.slot[k];
+        mbar_arrive(&s.empty[k]);
+    }
+    return __shfl_sync(0xffffffffu, tile, 0);
+}
+
 // ---- epilogue block I/O --------------------------------------------------
 // A warp moves 32 rows x 128 bytes at a time through its 4 KB staging buffer,
 // laid out like a 128-byte-swizzled TMA box (16-byte chunk c of row r at
@@ -324,6 +367,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint64_t *acce = accf + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    const Sched sch{acce + 3, acce + 3 + kSchedSlots, reinterpret_cast<int *>(acce + 3 + 2 * kSchedSlots)};
+    static_assert(8 * (2 * C::STAGES + 5 + 2 * kSchedSlots) + 4 * kSchedSlots <= 256, "barrier region");
     int *s_off = reinterpret_cast<int *>(full_bar) + 64;
     int *s_tstart = s_off + kMaxGroups;
     int *s_gorder = s_tstart + kMaxGroups;
@@ -365,6 +410,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 mbar_init(&accf[b], 1);
                 mbar_init(&acce[b], 32 * C::EPI_WARPS);
             }
+            for (int i = 0; i < kSchedSlots; ++i) {
+                mbar_init(&sch.full[i], 1);
+                mbar_init(&sch.empty[i], 1 + C::EPI_WARPS + C::PULL_WARPS);
+            }
             *abort_flag = 0;
             fence_barrier_init();
             tma_prefetch_desc(&tmA);
@@ -386,12 +435,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // ------------------------------------------------------------ producer
         int stage = 0;
         uint32_t phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        int tile = blockIdx.x;
+        for (int it = 0;; ++it) {
+            bool put = true;
+            if (lane == 0) put = sched_put(sch, it, tile, abort_flag, status);
+            put = __shfl_sync(0xffffffffu, put, 0);
+            if (!put || tile >= total) break;
             const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
             const bool routed = t.g < args.num_routed;
             const CUtensorMap *mB = routed ? &tmB : &tmB_s;
             const int gl = routed ? t.g : t.g - args.num_routed;
+            const int claim_kb = t.nkb > kClaimAhead ? t.nkb - kClaimAhead : 0;
+            int next = 0;
+            if (t.nkb == 0 && lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(args.sched, 1);
             for (int kb = 0; kb < t.nkb; ++kb) {
+                if (kb == claim_kb && lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(args.sched, 1);
                 bool ok = true;
                 if (lane == 0) {
                     ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status);
@@ -451,6 +509,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     phase ^= 1u;
                 }
             }
+            tile = __shfl_sync(0xffffffffu, next, 0);
         }
     producer_done:;
     } else if (warp >= C::PULL_WARP0) {
@@ -466,7 +525,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const size_t ld = static_cast<size_t>(args.gather_ld) * C::ESIZE;   // bytes per token row
             int stage = 0;
             uint32_t phase = 0;
-            for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+            for (int it = 0;; ++it) {
+                const int tile = sched_take(sch, it, total, lane, abort_flag, status);
+                if (tile >= total) break;
                 const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
                 if constexpr (!C::RAGGED_K) {
                     // K-major A: the tile's 128 rows, this thread's rows r0 + 16 i
@@ -556,7 +617,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // ------------------------------------------------------------ MMA issuer
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        for (int it = 0;; ++it) {
+            const int tile = sched_take(sch, it, total, lane, abort_flag, status);
+            if (tile >= total) break;
             const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
             bool ok = true;
             if (lane == 0) ok = mbar_wait(&acce[acc], acc_phase ^ 1u, abort_flag, status);
@@ -642,7 +705,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         EpiStage stg{reinterpret_cast<uint32_t *>(epi_stage) + ew * C::EPI_BUFS * 1024, C::EPI_BUFS, 0};
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        for (int it = 0;; ++it) {
+            const int tile = sched_take(sch, it, total, lane, abort_flag, status);
+            if (tile >= total) break;
             const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
             if (!mbar_wait(&accf[acc], acc_phase, abort_flag, status)) break;
             tc_fence_after();

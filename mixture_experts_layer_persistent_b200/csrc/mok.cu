@@ -120,6 +120,10 @@ bool make_tmap(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Tile counters of the grouped GEMMs, one per launch of a pass; the pass zeroes
+// them on its stream before the first launch.
+constexpr int kSchedCounters = 8;
+
 // Offsets of the arrays inside a buffer, laid out in order with 256-byte alignment.
 struct Carver {
     size_t off = 0;
@@ -178,6 +182,7 @@ struct State {
     __nv_bfloat16 *gu, *h, *hw;
     float *O;                       // per-(token, slot) rows: fp32 (BF16), bf16 (MXFP8 forward)
     uint8_t *xq, *xs, *hq, *hs;     // MXFP8 operands
+    int *sched;                     // [kSchedCounters] forward GEMM tile counters
     size_t bytes;
 };
 
@@ -216,6 +221,7 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
         st.hq = st.hs = st.xq = st.xs = nullptr;
     }
     st.O = mx ? reinterpret_cast<float *>(cv.take<__nv_bfloat16>(s.T * s.kk * s.H)) : cv.take<float>(s.T * s.kk * s.H);
+    st.sched = cv.take<int>(kSchedCounters);
     st.bytes = align_up(cv.off, 256);
     return st;
 }
@@ -224,6 +230,7 @@ struct BwdScratch {
     float *dl, *partial, *dxs;    // dxs: per-(token, slot) dx rows, fp32
     float *gpart;                 // per routed row and N tile of the down dgrad: <dy W_down, h>
     __nv_bfloat16 *dgu;
+    int *sched;                   // [kSchedCounters] backward GEMM tile counters
     size_t bytes;
 };
 
@@ -237,6 +244,7 @@ BwdScratch carve_bwd(const moe_cfg &c, void *buf)
     b.partial = cv.take<float>(s.max_chunks * s.H);
     b.dgu = cv.take<__nv_bfloat16>(s.R * 2 * s.I);
     b.dxs = cv.take<float>(s.T * s.kk * s.H);
+    b.sched = cv.take<int>(kSchedCounters);
     b.bytes = align_up(cv.off, 256);
     return b;
 }
@@ -290,6 +298,7 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b
                 const CUtensorMap &o2, const CUtensorMap &o3, const GemmArgs &args, int grid, cudaStream_t st)
 {
     if (grid <= 0) return MOK_OK;
+    if (!args.sched) return fail(MOK_ERR_INVALID, "grouped GEMM launch without a tile counter");
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(grouped_gemm_kernel)", e);
@@ -322,6 +331,8 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     const Shapes s = shapes(c);
     t_launches = 0;
     const bool mx = c.dtype == MOK_DTYPE_MXFP8;
+    if (const cudaError_t e = cudaMemsetAsync(st.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
 
     // router logits on the tensor cores: x . [Wr_hi | Wr_mid | Wr_lo]^T, split over K
     MOK_TRY(mark_fwd(0, stream));
@@ -343,6 +354,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         gr.out_f32 = st.rpart;
         gr.rows_total = c.T;
         gr.status = dev.status;
+        gr.sched = st.sched + 0;
         using CRouter = GemmCfg<256, false, false, false, false, false, EPI_ROUTER>;
         MOK_TRY(launch_gemm<CRouter>(rA, rB, rB, rO, rO, rO, gr, dev.sms, stream));
     }
@@ -389,6 +401,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
             return MOK_ERR_INVALID;
         if (!make_tmap(&tO, st.hq, s.I, s.R, 128, 32, 1)) return MOK_ERR_INVALID;
         GemmArgs ga{};
+        ga.sched = st.sched + 1;
         ga.num_groups = static_cast<int>(s.G);
         ga.num_routed = c.E;
         ga.offsets = st.offsets;
@@ -420,6 +433,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
             return MOK_ERR_INVALID;
         if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;   // bf16 slot rows
         GemmArgs gd = ga;
+        gd.sched = st.sched + 2;
         gd.n_tiles = c.H / 256;
         gd.num_kb = c.I / 128;
         gd.b_rows_per_group = c.H;
@@ -448,6 +462,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, BK, 128, 2))
             return MOK_ERR_INVALID;
         GemmArgs ga{};
+        ga.sched = st.sched + 1;
         ga.num_groups = static_cast<int>(s.G);
         ga.num_routed = c.E;
         ga.offsets = st.offsets;
@@ -476,6 +491,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, BK, 256, 2))
             return MOK_ERR_INVALID;
         GemmArgs gd = ga;
+        gd.sched = st.sched + 2;
         gd.n_tiles = c.H / 256;
         gd.num_kb = c.I / BK;
         gd.b_rows_per_group = c.H;
@@ -521,6 +537,8 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     const Shapes s = shapes(c);
     t_launches = 0;
     const __nv_bfloat16 *dyb = static_cast<const __nv_bfloat16 *>(dy);
+    if (const cudaError_t e = cudaMemsetAsync(bs.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
 
     GemmArgs base{};
     base.num_groups = static_cast<int>(s.G);
@@ -540,6 +558,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
     if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
     GemmArgs g1 = base;
+    g1.sched = bs.sched + 0;
     g1.num_kb = c.H / BK;
     g1.b_rows_per_group = c.H;
     g1.aux = st.gu;
@@ -576,6 +595,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
 
     // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
     GemmArgs g2 = base;
+    g2.sched = bs.sched + 1;
     g2.m_tiles = c.H / 128;
     g2.out = static_cast<__nv_bfloat16 *>(gr.dw_down);
     g2.out_s = static_cast<__nv_bfloat16 *>(gr.dws_down);
@@ -614,6 +634,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 64, 64, 2))
         return MOK_ERR_INVALID;
     GemmArgs g3 = base;
+    g3.sched = bs.sched + 2;
     g3.n_tiles = c.H / 256;
     g3.num_kb = 2 * c.I / BK;
     g3.b_rows_per_group = 2 * c.I;
@@ -627,6 +648,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     // wgrad of gate/up: dW_gate_up[g] = sum_r dGU_r^T x[token r]
     if (!make_tmap(&tA, bs.dgu, 2 * s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
     GemmArgs g4 = base;
+    g4.sched = bs.sched + 3;
     g4.gather_src = static_cast<const __nv_bfloat16 *>(x);
     g4.m_tiles = 2 * c.I / 128;
     g4.n_tiles = c.H / 256;
