@@ -49,11 +49,15 @@ class Inputs(ctypes.Structure):
 
 _lib = None
 
+# Path of another build of the oracle to load instead of liboracle.so.  The
+# planted-mistake tests set it to run the pins against a deliberately broken copy.
+LIB_ENV = "MOK_ORACLE_LIB"
+
 
 def lib():
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
+        _lib = ctypes.CDLL(os.environ.get(LIB_ENV) or build())
         d, p, i, i64 = ctypes.c_double, ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
         _lib.orc_round_bf16.restype = d
         _lib.orc_round_bf16.argtypes = [d]

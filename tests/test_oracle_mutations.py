@@ -1,0 +1,172 @@
+"""Planted mistakes in the oracle are caught by its pins (CPU only).
+
+Each case copies oracle/oracle.c, plants one plausible mistake in the copy (a
+flipped sign, a dropped term, a wrong index, a transposed operand, a wrong
+rounding rule), compiles it, and runs the pin tests of test_oracle_pins.py
+against that build.  The case passes only if the pin named beside the mistake
+fails; a mistake that no pin notices would mean that part of the oracle is
+unpinned.  The control case runs the pins on an unmodified copy built the same
+way and needs them all to pass.
+
+The copies live in a temporary directory; the committed oracle is never
+touched.  Rounding placements in the backward (which stored tensors the
+oracle rounds to bf16 there) are a reading of the layer's storage precision,
+not arithmetic, and are not planted here.
+"""
+import concurrent.futures
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ORACLE_C = os.path.join(ROOT, "oracle", "oracle.c")
+PINS = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+
+# (id, text in oracle.c (occurs exactly once), replacement, pin that must fail)
+MUTATIONS = [
+    # expert arithmetic
+    ("silu_sign",
+     "return g / (1.0 + exp(-g)); }", "return g / (1.0 + exp(g)); }",
+     "test_single_expert_equals_dense_swiglu"),
+    ("swiglu_operands_swapped",
+     "h[i] = silu(g[i]) * u[i];\n    if (c->mx)", "h[i] = silu(u[i]) * g[i];\n    if (c->mx)",
+     "test_single_expert_equals_dense_swiglu"),
+    ("up_rows_read_from_gate_half",
+     "b += xd[h] * ld(s->Wgu, s->gu_off + (int64_t)(s->I + i) * H + h, c->w_kind);",
+     "b += xd[h] * ld(s->Wgu, s->gu_off + (int64_t)i * H + h, c->w_kind);",
+     "test_single_expert_equals_dense_swiglu"),
+    ("down_weight_transposed",
+     "a += h[i] * ld(s->Wdn, s->dn_off + (int64_t)n * s->I + i, c->w_kind);",
+     "a += h[i] * ld(s->Wdn, s->dn_off + (int64_t)i * c->H + n, c->w_kind);",
+     "test_single_expert_equals_dense_swiglu"),
+    ("shared_expert_dropped",
+     "double wj = shared ? 1.0 : w[(int64_t)t * k + j];\n            gate_up(c, &s, xd, g, u);\n            swiglu_h",
+     "double wj = shared ? 0.0 : w[(int64_t)t * k + j];\n            gate_up(c, &s, xd, g, u);\n            swiglu_h",
+     "test_single_expert_equals_dense_swiglu"),
+    ("routing_weight_not_applied",
+     "acc[n2] += wj * o[n2];", "acc[n2] += o[n2];",
+     "test_mirrors_sit_at_stored_tensors"),
+    ("y_not_rounded_to_bf16",
+     "y[(int64_t)ti * H + n2] = mirror(c, acc[n2]);", "y[(int64_t)ti * H + n2] = acc[n2];",
+     "test_mirrors_sit_at_stored_tensors"),
+    ("h_not_rounded_to_bf16",
+     "for (int i = 0; i < I; i++) h[i] = mirror(c, h[i]);", "for (int i = 0; i < I; i++) h[i] = h[i];",
+     "test_mirrors_sit_at_stored_tensors"),
+    # routing
+    ("weights_not_renormalised",
+     "w[j] = c->routed_scale * prob[ord[j]] / tot;", "w[j] = c->routed_scale * prob[ord[j]];",
+     "test_softmax_topk_bruteforce"),
+    ("routed_scale_dropped",
+     "w[j] = c->routed_scale * prob[ord[j]] / tot;", "w[j] = prob[ord[j]] / tot;",
+     "test_sigmoid_group_limited_bruteforce"),
+    ("selection_bias_in_weights",
+     "w[j] = c->routed_scale * prob[ord[j]] / tot;", "w[j] = c->routed_scale * sc[ord[j]] / tot;",
+     "test_sigmoid_group_limited_bruteforce"),
+    ("ties_to_higher_index",
+     "(key[idx[j]] == key[v] && idx[j] > v)", "(key[idx[j]] == key[v] && idx[j] < v)",
+     "test_ties_go_to_lower_index"),
+    ("group_score_best_only",
+     "gsc[g] = sc[g * gs + wo[0]] + (gs > 1 ? sc[g * gs + wo[1]] : 0.0);", "gsc[g] = sc[g * gs + wo[0]];",
+     "test_sigmoid_group_limited_bruteforce"),
+    ("dispatch_tokens_descending",
+     "for (int t = 0; t < T; t++)\n        for (int j = 0; j < k; j++) {\n            int64_t s",
+     "for (int t = T - 1; t >= 0; t--)\n        for (int j = 0; j < k; j++) {\n            int64_t s",
+     "test_dispatch_invariants"),
+    # backward
+    ("softmax_dlogit_sign",
+     "dl[j] = w[j] * (G[j] - gbar);", "dl[j] = w[j] * (gbar - G[j]);",
+     "test_gradients_match_finite_differences"),
+    ("sigmoid_derivative_term_dropped",
+     "dl[j] = rho / S * (G[j] - gbar) * s * (1.0 - s);", "dl[j] = rho / S * (G[j] - gbar) * s;",
+     "test_gradients_match_finite_differences"),
+    ("silu_derivative_term_dropped",
+     "dgu[i] = mirror(c, dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)));", "dgu[i] = mirror(c, dh[i] * ub * sg);",
+     "test_gradients_match_finite_differences"),
+    ("du_uses_g_not_silu",
+     "dgu[I + i] = mirror(c, dh[i] * gb * sg);", "dgu[I + i] = mirror(c, dh[i] * gb);",
+     "test_gradients_match_finite_differences"),
+    ("dx_misses_router_path",
+     "dx[(int64_t)ti * H + q] = mirror(c, acc[q] + r);", "dx[(int64_t)ti * H + q] = mirror(c, acc[q]);",
+     "test_gradients_match_finite_differences"),
+    ("drouter_wrong_slot",
+     "a += dl[(int64_t)r * k + slot[r]] * ld(", "a += dl[(int64_t)r * k] * ld(",
+     "test_gradients_match_finite_differences"),
+    ("down_dgrad_transposed",
+     "dh[i] += d * ld(s->Wdn, s->dn_off + (int64_t)n * s->I + i, c->w_kind);",
+     "dh[i] += d * ld(s->Wdn, s->dn_off + (int64_t)i * c->H + n, c->w_kind);",
+     "test_gradients_match_finite_differences"),
+    ("dw_down_unweighted_h",
+     "HW[(int64_t)r * I + i] = mirror(c, wr[r] * hh);", "HW[(int64_t)r * I + i] = mirror(c, hh);",
+     "test_gradients_match_finite_differences"),
+    # number formats
+    ("bf16_truncates",
+     "double r = ldexp(nearbyint(ldexp(a, -q)), q);\n    if (r > 3.3895313892515355e38)",
+     "double r = ldexp(trunc(ldexp(a, -q)), q);\n    if (r > 3.3895313892515355e38)",
+     "test_bf16_rounding_matches_torch"),
+    ("e4m3_ties_away_from_zero",
+     "double r = ldexp(nearbyint(ldexp(a, -q)), q);\n    if (r > 448.0)",
+     "double r = ldexp(round(ldexp(a, -q)), q);\n    if (r > 448.0)",
+     "test_e4m3_rounding_matches_torch"),
+    ("e4m3_no_saturation",
+     "if (r > 448.0) r = 448.0;", "if (r > 1e300) r = 448.0;",
+     "test_e4m3_rounding_matches_torch"),
+    ("mx_scale_boundary",
+     "while (amax > ldexp(448.0, e)) e++;", "while (amax >= ldexp(448.0, e)) e++;",
+     "test_mx_scale_golden"),
+    ("mx_x_not_quantised",
+     "if (c->mx)\n        for (int b = 0; b < c->H; b += 32)", "if (0)\n        for (int b = 0; b < c->H; b += 32)",
+     "test_mxfp8_single_expert_matches_fakequant_mlp"),
+    ("mx_h_not_quantised",
+     "for (int b = 0; b < I; b += 32) mx_block(h + b, 32, NULL, NULL);",
+     "for (int b = 0; b < 0; b += 32) mx_block(h + b, 32, NULL, NULL);",
+     "test_mxfp8_single_expert_matches_fakequant_mlp"),
+]
+CONTROL = ("control", None, None, None)
+
+
+def _build_and_run(tmp, case):
+    name, old, new, _ = case
+    src = open(ORACLE_C).read()
+    if old is not None:
+        if src.count(old) != 1:
+            return name, ("bad-site", src.count(old))
+        src = src.replace(old, new)
+    d = os.path.join(tmp, name)
+    os.makedirs(d, exist_ok=True)
+    c_path, so_path = os.path.join(d, "oracle.c"), os.path.join(d, "liboracle.so")
+    open(c_path, "w").write(src)
+    cc = subprocess.run(["gcc", "-O1", "-fopenmp", "-shared", "-fPIC", c_path, "-o", so_path, "-lm"],
+                        capture_output=True, text=True)
+    if cc.returncode != 0:
+        return name, ("compile", cc.stderr[-2000:])
+    env = dict(os.environ, **{oracle.LIB_ENV: so_path, "OMP_NUM_THREADS": "2"})
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-p", "no:cacheprovider", "-rf", PINS],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    failed = sorted(set(re.findall(r"FAILED \S+::(test_\w+)", r.stdout)))
+    return name, (r.returncode, failed, r.stdout[-3000:])
+
+
+@pytest.fixture(scope="module")
+def outcomes(tmp_path_factory):
+    tmp = str(tmp_path_factory.mktemp("planted"))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        return dict(ex.map(lambda c: _build_and_run(tmp, c), MUTATIONS + [CONTROL]))
+
+
+def test_control_copy_passes_every_pin(outcomes):
+    rc, failed, out = outcomes["control"]
+    assert rc == 0 and not failed, out
+
+
+@pytest.mark.parametrize("name,old,new,pin", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(outcomes, name, old, new, pin):
+    res = outcomes[name]
+    assert res[0] not in ("bad-site", "compile"), res
+    rc, failed, out = res
+    assert rc == 1, out          # 1: tests ran and some failed (not a collection or usage error)
+    assert pin in failed, (failed, out)

@@ -235,15 +235,25 @@ def test_single_expert_equals_dense_swiglu(shared):
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
 
 
-def _bf16_round_via_torch(a):
-    # double -> float32 -> bf16 may round twice; agreement is checked to 1 ulp
-    return torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).double().numpy()
+def _assert_nearest_bf16(got, exact):
+    """`got` holds bf16 values, each the nearest one to `exact`: exactly
+    representable in bf16 (checked with torch's conversion, exact for such
+    values) and within half a bf16 ulp (2^(e-8) for |exact| in [2^e, 2^(e+1)))."""
+    got = np.asarray(got, np.float64)
+    exact = np.asarray(exact, np.float64)
+    f32 = got.astype(np.float32)
+    assert np.array_equal(f32.astype(np.float64), got)
+    assert np.array_equal(torch.from_numpy(f32).to(torch.bfloat16).float().numpy(), f32)
+    nz = exact != 0
+    assert np.all(got[~nz] == 0)
+    half_ulp = 2.0 ** (np.floor(np.log2(np.abs(exact[nz]))) - 8)
+    assert np.all(np.abs(got[nz] - exact[nz]) <= half_ulp)
 
 
 def test_mirrors_sit_at_stored_tensors():
     """With mirrors on, the two-expert forward equals the weighted sum of per-expert
-    MLPs with bf16 rounding of h and y (computed here with torch's rounding); the
-    per-slot rows o are kept unrounded (they are stored in fp32)."""
+    MLPs with h and y rounded to the nearest bf16 (the layer stores them in bf16);
+    the per-slot rows o are kept unrounded (they are stored in fp32)."""
     rng = np.random.default_rng(30)
     T, H, E, k, I = 16, 64, 4, 2, 64
     x = _rand_bf16(rng, (T, H), 1.0)
@@ -260,12 +270,11 @@ def test_mirrors_sit_at_stored_tensors():
             e = idx[t, j]
             g = xd[t] @ _bits_to_f64(Wgu[e, :I]).T
             u = xd[t] @ _bits_to_f64(Wgu[e, I:]).T
-            hh = _bf16_round_via_torch(g / (1 + np.exp(-g)) * u)
-            np.testing.assert_allclose(h[t, j], hh, rtol=2 ** -8, atol=0)
+            _assert_nearest_bf16(h[t, j], g / (1 + np.exp(-g)) * u)
             o = h[t, j] @ _bits_to_f64(Wdn[e]).T
             np.testing.assert_allclose(O[t, j], o, rtol=1e-12, atol=1e-12)
             acc += w[t, j] * O[t, j]
-        np.testing.assert_allclose(y[t], _bf16_round_via_torch(acc), rtol=2 ** -8, atol=0)
+        _assert_nearest_bf16(y[t], acc)
 
 
 def test_mxfp8_single_expert_matches_fakequant_mlp():
