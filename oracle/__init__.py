@@ -78,6 +78,7 @@ def lib():
         _lib.orc_route.argtypes = [cp, p, p, p, p, p, i, p, p, p, p, p]
         _lib.orc_dispatch.argtypes = [cp, p, p, p, p, p]
         _lib.orc_fwd_tokens.argtypes = [cp, ip, p, p, p, i, p, p, p]
+        _lib.orc_h_mx.argtypes = [cp, ip, p, p, i, p, p, p]
         _lib.orc_bwd_tokens.argtypes = [cp, ip, p, p, p, i, p, p, p]
         _lib.orc_drouter.argtypes = [cp, ip, p, p, p, i, p]
         _lib.orc_dw_entries.argtypes = [cp, ip, p, p, i, i, i, p, p, i, p]
@@ -177,6 +178,21 @@ class Layer:
         lib().orc_fwd_tokens(ctypes.byref(c), ctypes.byref(self.inp), _ptr(idx), _ptr(w),
                              _ptr(tokens), n, _ptr(y), _ptr(O), _ptr(h))
         return (y, O, h) if want_slots else y
+
+    def h_mx(self, idx, tokens):
+        """MXFP8 mode: (h unrounded [n, k+S, Im] fp64, e4m3 codes [n, k+S, Im] uint8,
+        ue8m0 scales [n, k+S, Im/32] uint8) of the listed tokens' slots."""
+        c = self.cfg
+        tokens = np.ascontiguousarray(tokens, np.int32)
+        n, kk, Im = len(tokens), c.k + c.S, max(c.I, c.Is)
+        hraw = np.zeros((n, kk, Im))
+        hq = np.zeros((n, kk, Im), np.uint8)
+        hs = np.zeros((n, kk, Im // 32), np.uint8)
+        rc = lib().orc_h_mx(ctypes.byref(c), ctypes.byref(self.inp),
+                            _ptr(np.ascontiguousarray(idx, np.int32)), _ptr(tokens), n, _ptr(hraw),
+                            _ptr(hq), _ptr(hs))
+        assert rc == 0
+        return hraw, hq, hs
 
     def bwd(self, idx, w, tokens=None):
         c = self.cfg

@@ -242,10 +242,12 @@ static double route_token(const orc_cfg *c, const void *x, const void *Wr, const
         lg[e] = s;
     }
     if (c->score_fn == 0) {
-        double mx = lg[0];
-        for (int e = 1; e < E; e++) if (lg[e] > mx) mx = lg[e];
+        /* a NaN logit (non-finite input) stays NaN and is left out of the
+         * normaliser, so the other experts' probabilities do not depend on it */
+        double mx = -INFINITY;
+        for (int e = 0; e < E; e++) if (lg[e] > mx) mx = lg[e];
         double z = 0.0;
-        for (int e = 0; e < E; e++) { prob[e] = exp(lg[e] - mx); z += prob[e]; }
+        for (int e = 0; e < E; e++) { prob[e] = exp(lg[e] - mx); if (!isnan(prob[e])) z += prob[e]; }
         for (int e = 0; e < E; e++) { prob[e] /= z; sc[e] = prob[e]; }
     } else {
         for (int e = 0; e < E; e++) {
@@ -253,6 +255,9 @@ static double route_token(const orc_cfg *c, const void *x, const void *Wr, const
             sc[e] = prob[e] + (bias ? ld(bias, e, c->r_kind) : 0.0);
         }
     }
+    /* a NaN selection score (non-finite input) ranks below every other score,
+     * like -inf; the order (score descending, index ascending) stays total */
+    for (int e = 0; e < E; e++) if (isnan(sc[e])) sc[e] = -INFINITY;
     double gap = INFINITY;
     /* group limiting: keep the topk_group groups with the best top-2 sums */
     int G = c->n_group, gs = E / G;
@@ -264,6 +269,7 @@ static double route_token(const orc_cfg *c, const void *x, const void *Wr, const
         for (int g = 0; g < G; g++) {
             order_desc(sc + g * gs, wo, gs);
             gsc[g] = sc[g * gs + wo[0]] + (gs > 1 ? sc[g * gs + wo[1]] : 0.0);
+            if (isnan(gsc[g])) gsc[g] = -INFINITY;      /* -inf + inf */
         }
         order_desc(gsc, gord, G);
         memset(keep, 0, E);
@@ -443,6 +449,37 @@ int orc_fwd_tokens(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, c
         }
         for (int n2 = 0; n2 < H; n2++) y[(int64_t)ti * H + n2] = mirror(c, acc[n2]);
         free(o);
+        free(xd);
+    }
+    return 0;
+}
+
+/* MXFP8 mode: the quantised h of each (token, slot) of n tokens, as the down
+ * projection reads it.  hraw: [n, k+S, max(I,Is)] the unrounded h = silu(g) u
+ * (fp64); hq: e4m3 codes, same shape; hs: [n, k+S, max(I,Is)/32] ue8m0 scale
+ * bytes.  Any output may be NULL. */
+int orc_h_mx(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, const int32_t *tokens, int n,
+             double *hraw, uint8_t *hq, uint8_t *hs)
+{
+    const int H = c->H, k = c->k, kk = c->k + c->S;
+    const int Im = c->I > c->Is ? c->I : c->Is;
+    if (!c->mx || (c->I % 32) || (c->S && (c->Is % 32))) return -1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int ti = 0; ti < n; ti++) {
+        int t = tokens[ti];
+        double *xd = (double *)malloc(sizeof(double) * (H + 3 * Im));
+        double *g = xd + H, *u = g + Im, *h = u + Im;
+        load_x(c, in->x, t, xd);
+        for (int j = 0; j < kk; j++) {
+            int shared = j >= k;
+            slot_w s = slot_weights(c, in, shared ? j - k : idx[(int64_t)t * k + j], shared);
+            gate_up(c, &s, xd, g, u);
+            for (int i = 0; i < s.I; i++) h[i] = silu(g[i]) * u[i];
+            int64_t row = (int64_t)ti * kk + j;
+            if (hraw) memcpy(hraw + row * Im, h, sizeof(double) * s.I);
+            for (int b = 0; b < s.I; b += 32)
+                mx_block(h + b, 32, hq ? hq + row * Im + b : NULL, hs ? hs + row * (Im / 32) + b / 32 : NULL);
+        }
         free(xd);
     }
     return 0;

@@ -9,9 +9,10 @@ unpinned.  The control case runs the pins on an unmodified copy built the same
 way and needs them all to pass.
 
 The copies live in a temporary directory; the committed oracle is never
-touched.  Rounding placements in the backward (which stored tensors the
-oracle rounds to bf16 there) are a reading of the layer's storage precision,
-not arithmetic, and are not planted here.
+touched.  The mistakes cover the expert arithmetic, the routing and its top-k
+margins, the backward, the number formats and the placement of the bf16
+rounding mirrors in the forward and the backward (a mirror dropped, moved or
+added where the layer keeps fp32).
 """
 import concurrent.futures
 import os
@@ -103,6 +104,41 @@ MUTATIONS = [
     ("dw_down_unweighted_h",
      "HW[(int64_t)r * I + i] = mirror(c, wr[r] * hh);", "HW[(int64_t)r * I + i] = mirror(c, hh);",
      "test_gradients_match_finite_differences"),
+    # top-k margins (the gap margin rejection reads) and non-finite scores
+    ("gap_on_unbiased_scores",
+     "double d = tmp[ord[j]] - tmp[ord[j + 1]];", "double d = prob[ord[j]] - prob[ord[j + 1]];",
+     "test_margin_gap_sigmoid_groups_bruteforce"),
+    ("group_gap_dropped",
+     "double d = gsc[gord[i]] - gsc[gord[i + 1]];\n            if (d < gap) gap = d;",
+     "double d = gsc[gord[i]] - gsc[gord[i + 1]];\n            (void)d;",
+     "test_margin_gap_sigmoid_groups_bruteforce"),
+    ("gap_misses_kth_neighbour",
+     "for (int j = 0; j < k && j + 1 < ncand; j++) {", "for (int j = 0; j + 1 < k && j + 1 < ncand; j++) {",
+     "test_margin_gap_softmax_bruteforce"),
+    ("nan_score_not_ranked_last",
+     "for (int e = 0; e < E; e++) if (isnan(sc[e])) sc[e] = -INFINITY;", "",
+     "test_nan_scores_rank_last"),
+    # where the backward rounds to bf16 (the stored tensors)
+    ("saved_gu_not_rounded",
+     "double gb = mirror(c, g[i]), ub = mirror(c, u[i]);", "double gb = g[i], ub = u[i];",
+     "test_backward_mirrors_sit_at_stored_tensors"),
+    ("dh_rounded_instead_of_dgu",
+     "dgu[i] = mirror(c, dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)));\n        dgu[I + i] = mirror(c, dh[i] * gb * sg);",
+     "dgu[i] = mirror(c, dh[i]) * ub * sg * (1.0 + gb * (1.0 - sg));\n        dgu[I + i] = mirror(c, dh[i]) * gb * sg;",
+     "test_backward_mirrors_sit_at_stored_tensors"),
+    ("wh_not_rounded",
+     "HW[(int64_t)r * I + i] = mirror(c, wr[r] * hh);", "HW[(int64_t)r * I + i] = wr[r] * hh;",
+     "test_backward_mirrors_sit_at_stored_tensors"),
+    ("dx_not_rounded",
+     "dx[(int64_t)ti * H + q] = mirror(c, acc[q] + r);", "dx[(int64_t)ti * H + q] = acc[q] + r;",
+     "test_backward_mirrors_sit_at_stored_tensors"),
+    ("dw_gate_up_not_rounded",
+     "dWgu[(int64_t)n * H + q] = mirror(c, a);", "dWgu[(int64_t)n * H + q] = a;",
+     "test_backward_mirrors_sit_at_stored_tensors"),
+    ("slot_dx_rows_rounded",
+     "acc[q] += a;                      /* per-slot dx rows are stored in fp32 */",
+     "acc[q] += mirror(c, a);",
+     "test_backward_mirrors_sit_at_stored_tensors"),
     # number formats
     ("bf16_truncates",
      "double r = ldexp(nearbyint(ldexp(a, -q)), q);\n    if (r > 3.3895313892515355e38)",

@@ -311,9 +311,26 @@ def test_mxfp8_single_expert_matches_fakequant_mlp():
     xd = fq(_bits_to_f64(x))
     g = xd @ _bits_to_f64(Wgu_q[0, :I]).T
     u = xd @ _bits_to_f64(Wgu_q[0, I:]).T
-    hq = fq(g / (1 + np.exp(-g)) * u)
+    hraw = g / (1 + np.exp(-g)) * u
+    hq = fq(hraw)
     ref = hq @ _bits_to_f64(Wdn_q[0]).T
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+    # the quantised h the down projection reads (h_mx): unrounded h, then per block
+    # the scale byte of the golden rule and torch's e4m3 codes of h / 2^e
+    oraw, ocodes, oscales = L.h_mx(idx, np.arange(T))
+    np.testing.assert_allclose(oraw[:, 0], hraw, rtol=1e-12, atol=1e-15)
+    for t in range(T):
+        for b in range(I // 32):
+            blk = oraw[t, 0, 32 * b:32 * b + 32]
+            amax = np.abs(blk).max()
+            e = -127
+            if amax > 0:
+                e = math.frexp(amax)[1] - 10
+                while amax > 448.0 * 2.0 ** e:
+                    e += 1
+            assert oscales[t, 0, b] == e + 127
+            codes = torch.from_numpy((blk / 2.0 ** e).astype(np.float32)).to(torch.float8_e4m3fn)
+            assert np.array_equal(ocodes[t, 0, 32 * b:32 * b + 32], codes.view(torch.uint8).numpy())
     # the fake-quantised weights are exactly the dequantised MX codes
     q, s = oracle.mx_quantize(Wgu[0])
     deq = np.vectorize(oracle.e4m3_value)(q) * 2.0 ** (np.repeat(s.astype(np.int64), 32, axis=1) - 127)
@@ -407,3 +424,182 @@ def test_dw_entries_agree_with_full():
         r2 = rng.integers(0, H, 20)
         c2 = rng.integers(0, ddn.shape[1], 20)
         assert np.array_equal(L.dw_entries(idx, w, g, sh, 1, r2, c2), ddn[r2, c2])
+
+
+# ------------------------------------------------------------------ top-k margins
+def _sorted_desc(vals):
+    """Indices by (value descending, index ascending), as the layer orders candidates."""
+    return sorted(range(len(vals)), key=lambda e: (-vals[e], e))
+
+
+def _gap_bruteforce(lg_t, k, score_fn, bias=None, n_group=1, topk_group=1):
+    """Smallest adjacent gap among the top k+1 selection scores of one token and,
+    with group-limited selection, among the top topk_group+1 group scores.  The
+    group score is the best pair sum of the group (enumerated), the candidates
+    are the experts of the kept groups."""
+    E = len(lg_t)
+    if score_fn == 0:
+        p = np.exp(lg_t - lg_t.max())
+        sc = p / p.sum()
+    else:
+        sc = 1 / (1 + np.exp(-lg_t)) + (0.0 if bias is None else bias.astype(np.float64))
+    gap = math.inf
+    cand = list(range(E))
+    if n_group > 1 and topk_group < n_group:
+        gs = E // n_group
+        gsc = [max(sc[g * gs + a] + sc[g * gs + b] for a, b in itertools.combinations(range(gs), 2))
+               if gs > 1 else sc[g * gs] for g in range(n_group)]
+        go = _sorted_desc(gsc)
+        for i in range(min(topk_group, n_group - 1)):
+            gap = min(gap, gsc[go[i]] - gsc[go[i + 1]])
+        cand = [g * gs + i for g in go[:topk_group] for i in range(gs)]
+    order = sorted(cand, key=lambda e: (-sc[e], e))
+    for j in range(min(k, len(order) - 1)):
+        gap = min(gap, sc[order[j]] - sc[order[j + 1]])
+    return gap
+
+
+@pytest.mark.parametrize("k", [1, 3])
+def test_margin_gap_softmax_bruteforce(k):
+    """The gap that margin rejection reads is the smallest adjacent difference
+    among the top k+1 softmax probabilities (not only the top k), ties giving 0."""
+    T, H, E = 40, 16, 8
+    x, Wr = _tiny_router(T, H, E, seed=70 + k)
+    Wr[1] *= 3.0
+    Wr[7] = Wr[1]                              # a tied pair, often on top: those tokens have gap 0
+    L = oracle.Layer(T, H, E, k, 8).set(x=x, Wr=Wr)
+    _, _, gap = L.route()
+    lg = _logits_np(x, Wr)
+    want = np.array([_gap_bruteforce(lg[t], k, 0) for t in range(T)])
+    np.testing.assert_allclose(gap, want, rtol=1e-9, atol=1e-13)
+    assert (want == 0).any() and (want > 0).any()
+
+
+@pytest.mark.parametrize("k,TG", [(2, 2), (4, 3)])
+def test_margin_gap_sigmoid_groups_bruteforce(k, TG):
+    """Group-limited sigmoid routing: the gap covers the biased expert scores among
+    the kept groups' experts and the group scores around the kept/dropped boundary,
+    with the additive logit term in the logits."""
+    T, H, E, G = 48, 16, 16, 4
+    x, Wr = _tiny_router(T, H, E, seed=80 + k)
+    bias = (0.2 * np.random.default_rng(81).standard_normal(E)).astype(np.float32)
+    lb = (0.3 * np.random.default_rng(82).standard_normal(E)).astype(np.float32)
+    L = oracle.Layer(T, H, E, k, 8, score_fn=1, n_group=G, topk_group=TG, routed_scale=1.3)
+    L.set(x=x, Wr=Wr, bias=bias, lbias=lb)
+    _, _, gap = L.route()
+    lg = _logits_np(x, Wr, lb)
+    want = np.array([_gap_bruteforce(lg[t], k, 1, bias, G, TG) for t in range(T)])
+    np.testing.assert_allclose(gap, want, rtol=1e-9, atol=1e-13)
+    # the group term decides the gap of some tokens and the expert term of others
+    exp_only = np.array([_gap_bruteforce(lg[t], k, 1, bias) for t in range(T)])
+    assert (want < exp_only).any()
+
+
+def test_nan_scores_rank_last():
+    """A NaN selection score ranks below every other score (as -inf), so the
+    top-k stays k distinct experts with ties to the lower index: a token whose
+    logits are all NaN takes experts 0..k-1; an expert whose logit term is NaN is
+    never chosen while k other experts remain, and under softmax the other
+    experts' weights stay the softmax over the selected logits.  (The GPU path
+    follows the same rule; these inputs are not run there.)"""
+    T, H, E, k = 12, 16, 8, 3
+    x, Wr = _tiny_router(T, H, E, seed=90)
+    x[4] = 0x7FC0                              # bf16 NaN: every logit of token 4 is NaN
+    lb = np.zeros(E, np.float32)
+    lb[2] = np.nan
+    for score_fn, G, TG in [(0, 1, 1), (1, 4, 2)]:
+        L = oracle.Layer(T, H, E, k, 8, score_fn=score_fn, n_group=G, topk_group=TG).set(x=x, Wr=Wr, lbias=lb)
+        idx, w, _ = L.route()
+        assert list(idx[4]) == [0, 1, 2]        # every score -inf: the lowest indices
+        lg = _logits_np(x, Wr, lb)
+        for t in range(T):
+            if t == 4:
+                continue
+            assert 2 not in idx[t]
+            sc = lg[t].copy() if score_fn == 0 else 1 / (1 + np.exp(-lg[t]))
+            sc[2] = -np.inf
+            if G > 1:
+                gs = E // G
+                gsc = [max(sc[g * gs + a] + sc[g * gs + b] for a, b in itertools.combinations(range(gs), 2))
+                       for g in range(G)]
+                gsc = [-np.inf if np.isnan(v) else v for v in gsc]
+                keep = _sorted_desc(gsc)[:TG]
+                sc = np.array([sc[e] if e // gs in keep else -np.inf for e in range(E)])
+            assert list(idx[t]) == _sorted_desc(list(sc))[:k]
+            if score_fn == 0:
+                sel = lg[t, idx[t]]
+                np.testing.assert_allclose(w[t], np.exp(sel - sel.max()) / np.exp(sel - sel.max()).sum(),
+                                           rtol=1e-12)
+
+
+# ------------------------------------------------------------------ backward rounding mirrors
+def _rb(v):
+    """Nearest bf16 value of fp64 values, ties to even (8 significant bits), by
+    exact scaling: v = m 2^e with m in [0.5, 1) -> round m 2^8 to an integer."""
+    v = np.asarray(v, np.float64)
+    m, e = np.frexp(v)
+    e = np.maximum(e, -125)                    # subnormal bf16 spacing 2^-133
+    return np.ldexp(np.rint(np.ldexp(v, 8 - e)), e - 8)
+
+
+def test_backward_mirrors_sit_at_stored_tensors():
+    """With mirrors on, dx and the weight gradients equal a numpy restatement of
+    the backward that rounds to the nearest bf16 exactly where the layer stores a
+    bf16 tensor -- the saved g and u read by the SwiGLU backward, dGU, h, w*h, dx
+    and dW -- and nowhere else: dh, the per-slot dx rows and the routing-gradient
+    path stay unrounded.  Routing from the oracle (pinned above); softmax scoring
+    and one shared expert."""
+    rng = np.random.default_rng(95)
+    T, H, E, k, I, Is = 16, 64, 4, 2, 32, 32
+    x = _rand_bf16(rng, (T, H), 1.0)
+    dy = _rand_bf16(rng, (T, H), 1.0)
+    Wr = rng.standard_normal((E, H)).astype(np.float32) / 8
+    Wgu = _rand_bf16(rng, (E, 2 * I, H), 0.1)
+    Wdn = _rand_bf16(rng, (E, H, I), 0.1)
+    Wgu_s = _rand_bf16(rng, (1, 2 * Is, H), 0.1)
+    Wdn_s = _rand_bf16(rng, (1, H, Is), 0.1)
+    L = oracle.Layer(T, H, E, k, I, S=1, Is=Is).set(x=x, Wr=Wr, Wgu=Wgu, Wdn=Wdn, Wgu_s=Wgu_s,
+                                                     Wdn_s=Wdn_s, dy=dy)
+    idx, w, _ = L.route()
+    dx, _, _ = L.bwd(idx, w)
+    xd, dyd = _bits_to_f64(x), _bits_to_f64(dy)
+    Wr64 = Wr.astype(np.float64)
+
+    def expert(shared, e):
+        gu = _bits_to_f64(Wgu_s[e] if shared else Wgu[e])
+        dn = _bits_to_f64(Wdn_s[e] if shared else Wdn[e])
+        return gu[:len(gu) // 2], gu[len(gu) // 2:], dn
+
+    def slot(t, shared, e, wj):
+        Wg, Wu, Wd = expert(shared, e)
+        g, u = Wg @ xd[t], Wu @ xd[t]                           # unrounded accumulators
+        h = _rb(g / (1 + np.exp(-g)) * u)                        # stored h
+        dh = Wd.T @ (wj * dyd[t])                                # dh: not stored, unrounded
+        gb, ub = _rb(g), _rb(u)                                  # saved g, u
+        sg = 1 / (1 + np.exp(-gb))
+        dgu = np.concatenate([_rb(dh * ub * sg * (1 + gb * (1 - sg))), _rb(dh * gb * sg)])   # stored dGU
+        return h, dgu, np.concatenate([Wg, Wu]).T @ dgu           # per-slot dx row: fp32, unrounded
+
+    want_dx = np.zeros((T, H))
+    rows = {g: [] for g in [(False, e) for e in range(E)] + [(True, 0)]}
+    for t in range(T):
+        G, acc = np.zeros(k), np.zeros(H)
+        for j in range(k + 1):
+            shared = j == k
+            e = 0 if shared else idx[t, j]
+            wj = 1.0 if shared else w[t, j]
+            h, dgu, dxs = slot(t, shared, e, wj)
+            acc += dxs
+            if not shared:
+                G[j] = dyd[t] @ (expert(False, e)[2] @ h)           # <dy, o_j>, o_j unrounded (fp32 slot row)
+            rows[(shared, e)].append((t, wj, h, dgu))
+        dl = w[t] * (G - (w[t] * G).sum())
+        want_dx[t] = _rb(acc + dl @ Wr64[idx[t]])
+    np.testing.assert_allclose(dx, want_dx, rtol=1e-9, atol=1e-12)
+    for (shared, e), rs in rows.items():
+        dgu_full, ddn_full = L.dw_full(idx, w, e, shared)
+        toks = [r[0] for r in rs]
+        DGU = np.array([r[3] for r in rs]).reshape(len(rs), -1)
+        HW = _rb(np.array([r[1] * r[2] for r in rs]).reshape(len(rs), -1))     # stored w*h
+        np.testing.assert_allclose(dgu_full, _rb(DGU.T @ xd[toks]), rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(ddn_full, _rb(dyd[toks].T @ HW), rtol=1e-9, atol=1e-12)
