@@ -47,6 +47,8 @@ extern "C" {
 
 /* device status bits (moe_status) */
 #define MOK_STATUS_TIMEOUT 1      /* a bounded wait inside a kernel ran out */
+#define MOK_STATUS_BAD_INDEX 2    /* a routing index outside [0, E) reached the dispatch (it was
+                                     placed as expert 0; the layer's own selection never makes one) */
 
 /* ---- configuration -------------------------------------------------------- */
 #define MOK_SCORE_SOFTMAX 0       /* softmax over all experts, top-k, renormalised */
@@ -143,6 +145,10 @@ int moe_workspace_size(const moe_cfg *cfg, size_t *ctx_bytes, size_t *fwd_scratc
  * row, and a fixed-order weighted sum over slots (shared experts last,
  * weight 1).  The pull-at-dispatch / push-at-combine split follows
  * "Cursor åpner megakernelen…" (paragraph on pulling versus pushing tokens).
+ * Non-finite input: a selection score that is NaN ranks below every other
+ * score (as -inf), so every token still gets top_k distinct experts in
+ * [0, E) (ties to the lower index); such a token's weights and outputs are
+ * NaN.  Other tokens are unaffected.
  */
 int moe_fwd(const moe_cfg *cfg, const void *x, const moe_params *params, void *y,
             const moe_routing *routing, void *ctx, size_t ctx_bytes, int save_for_backward,
@@ -249,6 +255,34 @@ int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events
  */
 #define MOK_STATIC_SCRATCH_BYTES (32u << 20)
 int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, void *y, void *stream);
+
+/*
+ * Where the forward keeps one of its intermediate tensors inside its buffer
+ * (ctx when save_for_backward != 0, the forward scratch otherwise), for
+ * inspection and tests: *offset = byte offset from the buffer's start, *bytes =
+ * size.  The contents are valid once the forward on the stream has completed
+ * and until that buffer is next written.  R = T * (top_k + n_shared) sorted
+ * rows: the routed rows expert-major (the order of moe_routing.perm), then
+ * n_shared blocks of T rows (shared expert s, token t at row T*top_k + s*T + t).
+ *   MOK_SAVED_H          [R, I] bf16 h = silu(g) u (BF16 layer)
+ *   MOK_SAVED_HQ         [R, I] e4m3 codes of h (MXFP8 layer)
+ *   MOK_SAVED_HS         [R, I/32] ue8m0 scale bytes of h, row-major (MXFP8 layer)
+ *   MOK_SAVED_GU         [R, 2I] bf16 gate and up pre-activations (BF16, save_for_backward)
+ *   MOK_SAVED_HW         [R, I] bf16 routing weight times h (BF16, save_for_backward)
+ *   MOK_SAVED_ROW_TOKEN  [R] int32 token of each sorted row
+ *   MOK_SAVED_ROW_W      [R] fp32 routing weight of each sorted row (1 for shared rows)
+ * Returns MOK_ERR_UNSUPPORTED when the configuration keeps no such tensor and
+ * MOK_ERR_INVALID for an unknown `which` or a bad cfg.  The pages have no
+ * counterpart; this is a window on the saved state for the library's users.
+ */
+#define MOK_SAVED_H 0
+#define MOK_SAVED_HQ 1
+#define MOK_SAVED_HS 2
+#define MOK_SAVED_GU 3
+#define MOK_SAVED_HW 4
+#define MOK_SAVED_ROW_TOKEN 5
+#define MOK_SAVED_ROW_W 6
+int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_t *offset, size_t *bytes);
 
 /*
  * Number of CUDA kernels launched by the last moe_fwd / moe_bwd (or their

@@ -21,6 +21,7 @@ MOK_ERR_WORKSPACE = -3
 MOK_ERR_LAUNCH = -4
 MOK_ERR_UNSUPPORTED = -5
 MOK_STATUS_TIMEOUT = 1
+MOK_STATUS_BAD_INDEX = 2
 MOK_SCORE_SOFTMAX = 0
 MOK_SCORE_SIGMOID = 1
 MOK_DTYPE_BF16 = 0
@@ -28,6 +29,7 @@ MOK_DTYPE_MXFP8 = 1
 MOK_FWD_PHASES = 5
 MOK_BWD_PHASES = 8
 MOK_STATIC_SCRATCH_BYTES = 32 << 20
+MOK_SAVED_H, MOK_SAVED_HQ, MOK_SAVED_HS, MOK_SAVED_GU, MOK_SAVED_HW, MOK_SAVED_ROW_TOKEN, MOK_SAVED_ROW_W = range(7)
 
 _i32, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -88,13 +90,14 @@ def lib():
         L.moe_fwd_static.argtypes = [P(moe_cfg), _vp, P(moe_params), _vp, _vp]
         L.moe_test_drop_signal.argtypes = [ctypes.c_int]
         L.moe_launch_count.argtypes = [P(_i32)]
+        L.moe_saved_tensor.argtypes = [P(moe_cfg), _i32, _i32, P(_sz), P(_sz)]
         L.moe_strerror.argtypes = [ctypes.c_int]
         L.moe_strerror.restype = ctypes.c_char_p
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
                      "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_quantize_mxfp8_weights", "moe_status",
-                     "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal"):
+                     "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal", "moe_saved_tensor"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -114,6 +117,14 @@ def moe_workspace_size(cfg: moe_cfg):
     _check("moe_workspace_size", lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(c),
                                                           ctypes.byref(f), ctypes.byref(b)))
     return c.value, f.value, b.value
+
+
+def moe_saved_tensor(cfg: moe_cfg, save_for_backward: bool, which: int):
+    """(byte offset, bytes) of a saved tensor inside the forward's buffer."""
+    off, n = _sz(), _sz()
+    _check("moe_saved_tensor", lib().moe_saved_tensor(ctypes.byref(cfg), int(save_for_backward), int(which),
+                                                      ctypes.byref(off), ctypes.byref(n)))
+    return off.value, n.value
 
 
 def moe_host_scratch_size(cfg: moe_cfg, backward: bool) -> int:

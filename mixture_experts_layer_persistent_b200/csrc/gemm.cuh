@@ -368,7 +368,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     const Sched sch{acce + 3, acce + 3 + kSchedSlots, reinterpret_cast<int *>(acce + 3 + 2 * kSchedSlots)};
-    static_assert(8 * (2 * C::STAGES + 5 + 2 * kSchedSlots) + 4 * kSchedSlots <= 256, "barrier region");
+    uint64_t *drain_bar = acce + 3 + 2 * kSchedSlots + (4 * kSchedSlots + 7) / 8;   // MMA drain on abort
+    static_assert(8 * (2 * C::STAGES + 6 + 2 * kSchedSlots) + 4 * kSchedSlots <= 256, "barrier region");
     int *s_off = reinterpret_cast<int *>(full_bar) + 64;
     int *s_tstart = s_off + kMaxGroups;
     int *s_gorder = s_tstart + kMaxGroups;
@@ -414,6 +415,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 mbar_init(&sch.full[i], 1);
                 mbar_init(&sch.empty[i], 1 + C::EPI_WARPS + C::PULL_WARPS);
             }
+            mbar_init(drain_bar, 1);
             *abort_flag = 0;
             fence_barrier_init();
             tma_prefetch_desc(&tmA);
@@ -435,6 +437,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // ------------------------------------------------------------ producer
         int stage = 0;
         uint32_t phase = 0;
+        int fills = 0;                   // stages whose loads this producer issued
         int tile = blockIdx.x;
         for (int it = 0;; ++it) {
             bool put = true;
@@ -504,6 +507,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         bulk_load(sf + 1024, sb + (static_cast<long long>(kb) * rt + (r1 >> 7)) * 512, 512, fb);
                     }
                 }
+                ++fills;
                 if (++stage == C::STAGES) {
                     stage = 0;
                     phase ^= 1u;
@@ -511,7 +515,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
             tile = __shfl_sync(0xffffffffu, next, 0);
         }
-    producer_done:;
+    producer_done:
+        if (*abort_flag && lane == 0) {
+            // another role gave up: let the last STAGES fills land (bounded) before the
+            // CTA releases its shared memory
+            int s2 = stage;
+            uint32_t ph = phase;
+            for (int i = 0; i < min(fills, C::STAGES); ++i) {
+                if (--s2 < 0) {
+                    s2 = C::STAGES - 1;
+                    ph ^= 1u;
+                }
+                mbar_drain(&full_bar[s2], ph);
+            }
+        }
     } else if (warp >= C::PULL_WARP0) {
         // ------------------------------------------------------------ pull warps
         // Gathered operand: each 128-byte row is copied by index from the token
@@ -611,7 +628,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     }
                 }
             }
-        pull_done:;
+        pull_done:
+            cp_async_wait_all();         // nothing of this thread still lands in shared memory
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -696,6 +714,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 acc = 0;
                 acc_phase ^= 1u;
             }
+        }
+        if (__shfl_sync(0xffffffffu, *abort_flag, 0)) {
+            // the MMAs (and scale copies) this warp issued complete before TMEM is released
+            if (lane == 0) {
+                umma_commit(drain_bar);
+                mbar_drain(drain_bar, 0);
+            }
+            __syncwarp();
         }
     } else {
         // ------------------------------------------------------------ epilogue

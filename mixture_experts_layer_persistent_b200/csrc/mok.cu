@@ -377,6 +377,7 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     da.perm = st.perm; da.inv_perm = st.inv_perm; da.row_token = st.row_token; da.row_slot = st.row_slot;
     da.row_w = st.row_w;
     da.hist = st.hist;
+    da.status = dev.status;
     MOK_TRY(mark_fwd(1, stream));
     {
         const int n_chunks = static_cast<int>((s.T + kDispatchChunk - 1) / kDispatchChunk);
@@ -889,6 +890,33 @@ int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, 
     }
     const State st = carve_state(*cfg, ptr, false);
     return forward(*cfg, x, *params, y, nullptr, st, *dev, false, static_cast<cudaStream_t>(stream));
+}
+
+int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_t *offset, size_t *bytes)
+{
+    MOK_TRY(check_cfg(cfg));
+    const bool training = save_for_backward != 0;
+    if (training && cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
+    // carve over a stand-in base address: only the differences are used
+    char *const base = reinterpret_cast<char *>(uintptr_t(1) << 40);
+    const State st = carve_state(*cfg, base, training);
+    const Shapes s = shapes(*cfg);
+    const void *p = nullptr;
+    size_t n = 0;
+    switch (which) {
+    case MOK_SAVED_H: p = st.h; n = s.R * s.I * 2; break;
+    case MOK_SAVED_HQ: p = st.hq; n = s.R * s.I; break;
+    case MOK_SAVED_HS: p = st.hs; n = s.R * s.I / 32; break;
+    case MOK_SAVED_GU: p = st.gu; n = s.R * 2 * s.I * 2; break;
+    case MOK_SAVED_HW: p = st.hw; n = s.R * s.I * 2; break;
+    case MOK_SAVED_ROW_TOKEN: p = st.row_token; n = s.R * 4; break;
+    case MOK_SAVED_ROW_W: p = st.row_w; n = s.R * 4; break;
+    default: return MOK_ERR_INVALID;
+    }
+    if (!p) return MOK_ERR_UNSUPPORTED;
+    if (offset) *offset = static_cast<size_t>(static_cast<const char *>(p) - base);
+    if (bytes) *bytes = n;
+    return MOK_OK;
 }
 
 int moe_launch_count(int *count)

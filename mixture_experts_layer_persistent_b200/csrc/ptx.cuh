@@ -12,6 +12,7 @@ namespace mok {
 // Bounded waits give up after this many nanoseconds and flag the device status.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kStatusTimeout = 1;
+constexpr int kStatusBadIndex = 2;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -79,6 +80,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+// After a role of the CTA has given up: wait for the phase of `parity` to
+// complete, ignoring the abort flag, for at most kDrainLimitNs.  Used so that
+// copies and MMAs a role already issued land before the CTA releases its shared
+// memory and TMEM.  An operation in flight completes within microseconds; the
+// limit only bounds the wait when a phase can no longer complete because
+// another role stopped contributing to it.
+constexpr uint64_t kDrainLimitNs = 20000000ull;
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity)
+{
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > kDrainLimitNs) return false;
+    return true;
+}
+
+// Wait until every cp.async this thread issued has completed.
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *tm)
 {
@@ -127,8 +146,7 @@ __device__ __forceinline__ void tma_scatter4(const CUtensorMap *tm, const void *
 }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// wait until this thread's bulk stores have finished reading shared memory
-// wait until this thread's bulk stores have completed
+// wait until this thread's bulk stores have completed (their writes are done)
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // 4-byte asynchronous global->shared copy.

@@ -74,17 +74,18 @@ __device__ __forceinline__ void warp_argmax(float &v, int &i)
     }
 }
 
-// One warp per token.  Lane l holds experts l + 32 i.  The logit is the sum of
-// the K-split partials in split order plus logit_bias; selection as above.
-__global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a)
+// A selection score that is NaN (a non-finite activation or bias) ranks below
+// every other score, as -inf does; the selection below still returns k distinct
+// experts in [0, E), ties going to the lower index.
+__device__ __forceinline__ float rank_score(float v) { return v == v ? v : -INFINITY; }
+
+// Selection of one token by one warp.  Lane l holds experts l + 32 i.  The
+// logit is the sum of the K-split partials in split order plus logit_bias;
+// selection as above.  row: 256 floats of shared memory owned by the warp.
+__device__ __forceinline__ void select_token(const SelectArgs &a, int t, int lane, float *row)
 {
-    __shared__ float s_row[8][256];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t = blockIdx.x * 8 + warp;
-    if (t >= a.T) return;
     const int E = a.E;
     const int npl = (E + 31) / 32;
-    float *row = s_row[warp];
     float lgv[8], sel[8], sc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -98,11 +99,11 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a)
             if (a.logit_bias) lg += a.logit_bias[e];
             lgv[i] = lg;
             if (a.score_fn == 0) {
-                sel[i] = lg;
+                sel[i] = rank_score(lg);
             } else {
                 const float sg = 1.0f / (1.0f + expf(-lg));
                 sc[i] = sg;
-                sel[i] = sg + (a.e_bias ? a.e_bias[e] : 0.0f);
+                sel[i] = rank_score(sg + (a.e_bias ? a.e_bias[e] : 0.0f));
             }
         }
     }
@@ -123,15 +124,17 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a)
                 if (v > b1) { b2 = b1; b1 = v; }
                 else if (v > b2) { b2 = v; }
             }
-            gsc = gs > 1 ? b1 + b2 : b1;
+            gsc = rank_score(gs > 1 ? b1 + b2 : b1);
         }
         unsigned keep = 0;   // bit g set: group g kept
         for (int r = 0; r < a.topk_group; ++r) {
-            float v = lane < a.n_group ? gsc : -INFINITY;
-            int gi = lane < a.n_group ? lane : 1 << 30;
-            if (keep & (1u << (lane & 31))) v = -INFINITY;
+            // groups already kept and lanes past the last group never win, so the
+            // topk_group kept groups are distinct even when their scores are -inf
+            const bool cand = lane < a.n_group && !(keep & (1u << lane));
+            float v = cand ? gsc : -INFINITY;
+            int gi = cand ? lane : 1 << 30;
             warp_argmax(v, gi);
-            keep |= 1u << gi;
+            if (gi < a.n_group) keep |= 1u << gi;
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -139,16 +142,18 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a)
             if (i < npl && e < E && !(keep & (1u << (e / gs)))) sel[i] = -INFINITY;
         }
     }
-    // top-k by repeated warp argmax
+    // top-k by repeated warp argmax over the experts not yet taken; k <= E, so
+    // every round finds a candidate and bi is always an expert index below E
     int my_idx[16];
     float my_val[16];
+    unsigned taken = 0;      // bit i: expert lane + 32 i already selected
     for (int j = 0; j < a.k; ++j) {
         float bv = -INFINITY;
         int bi = 1 << 30;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int e = lane + 32 * i;
-            if (i < npl && e < E && better(sel[i], e, bv, bi)) {
+            if (i < npl && e < E && !(taken & (1u << i)) && better(sel[i], e, bv, bi)) {
                 bv = sel[i];
                 bi = e;
             }
@@ -159,7 +164,7 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a)
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             if (lane + 32 * i == bi) {
-                sel[i] = -INFINITY;                                   // the owner retires the winner
+                taken |= 1u << i;                                     // the owner retires the winner
                 wv = a.score_fn == 0 ? lgv[i] : sc[i];               // logit (softmax) or sigmoid score
             }
         my_val[j] = __shfl_sync(0xffffffffu, wv, bi & 31);
@@ -182,6 +187,16 @@ __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a)
     }
 }
 
+// One warp per token.
+__global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a)
+{
+    __shared__ float s_row[8][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= a.T) return;
+    select_token(a, t, lane, s_row[warp]);
+}
+
 // ------------------------------------------------------------------ dispatch
 struct DispatchArgs {
     const int *topk_idx;   // [T, k]
@@ -198,7 +213,19 @@ struct DispatchArgs {
     int *row_token;        // [R]
     int *row_slot;         // [R]
     float *row_w;          // [R]
+    int *status;           // device status word
 };
+
+// A routing index outside [0, E) cannot come out of the selection above; if one
+// is ever met, it is counted and placed as expert 0 (both dispatch kernels map
+// it the same way, so every row range stays consistent and in bounds) and the
+// status word records MOK_STATUS_BAD_INDEX.
+__device__ __forceinline__ int checked_expert(int e, int E, int *status)
+{
+    if (static_cast<unsigned>(e) < static_cast<unsigned>(E)) return e;
+    atomicOr(status, kStatusBadIndex);
+    return 0;
+}
 
 constexpr int kDispatchChunk = 1024;   // tokens per chunk (one block of 1024 threads)
 
@@ -214,7 +241,7 @@ __global__ void __launch_bounds__(1024) dispatch_count_kernel(const DispatchArgs
     __syncthreads();
     const int t = c * kDispatchChunk + tid;
     if (t < a.T)
-        for (int j = 0; j < a.k; ++j) atomicAdd(&s_cnt[a.topk_idx[(size_t)t * a.k + j]], 1);
+        for (int j = 0; j < a.k; ++j) atomicAdd(&s_cnt[checked_expert(a.topk_idx[(size_t)t * a.k + j], a.E, a.status)], 1);
     __syncthreads();
     for (int e = tid; e < a.E; e += 1024) a.hist[(size_t)c * a.E + e] = s_cnt[e];
 }
@@ -277,11 +304,11 @@ __global__ void __launch_bounds__(1024) dispatch_place_kernel(const DispatchArgs
     const int t = c * kDispatchChunk + tid;
     const int word = tid >> 5, bit = tid & 31;
     if (t < T)
-        for (int j = 0; j < k; ++j) atomicOr(&s_mask[a.topk_idx[(size_t)t * k + j]][word], 1u << bit);
+        for (int j = 0; j < k; ++j) atomicOr(&s_mask[checked_expert(a.topk_idx[(size_t)t * k + j], E, a.status)][word], 1u << bit);
     __syncthreads();
     if (t < T) {
         for (int j = 0; j < k; ++j) {
-            const int e = a.topk_idx[(size_t)t * k + j];
+            const int e = checked_expert(a.topk_idx[(size_t)t * k + j], E, a.status);
             int rank = __popc(s_mask[e][word] & ((1u << bit) - 1u));
             for (int w = 0; w < word; ++w) rank += __popc(s_mask[e][w]);
             const int pos = a.hist[(size_t)c * E + e] + rank;

@@ -111,6 +111,13 @@ class MoELayer:
                     self.ctx_bytes, cg, self.bwd_scratch.data_ptr(), self.bwd_bytes, self.stream())
         return grads
 
+    def saved(self, which: int, dtype=torch.uint8) -> torch.Tensor:
+        """A view of one tensor the last forward kept in this layer's buffer
+        (abi.MOK_SAVED_*), flat, of the given dtype."""
+        off, n = abi.moe_saved_tensor(self.cfg, self.training, which)
+        buf = self.ctx if self.training else self.scratch
+        return buf[off:off + n].view(dtype)
+
     def status(self) -> int:
         return abi.moe_status(self.stream())
 

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 from mixture_experts_layer_persistent_b200 import MoELayer, cfg_for, synth
-from tests._support import assert_close, make_case, to_np
+from tests._support import assert_close, check_mx_h, make_case, rel_rms_per_token, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -122,14 +122,20 @@ def _mx_params(params):
     return out
 
 
-def _rel_rms(got, want):
-    return float(np.sqrt(np.mean((got - want) ** 2)) / np.sqrt(np.mean(want ** 2)))
+MX_CASES = [MEDIUM_MX,
+            synth.scaled(MEDIUM_MX, name="medium_mx_softmax", score_fn=0, n_group=1, topk_group=1, S=0, Is=0,
+                         T=333, seed=22),
+            # I = 384: not a multiple of 256 (three 128-column h tiles, a K of three blocks in the
+            # down GEMM), two shared experts, groups ending in partial 32-row blocks
+            synth.scaled(MEDIUM_MX, name="medium_mx_i384", T=411, H=768, E=12, k=3, I=384, S=2, Is=384,
+                         n_group=4, topk_group=2, seed=23)]
 
 
-@pytest.mark.parametrize("wl", [MEDIUM_MX, synth.scaled(MEDIUM_MX, name="medium_mx_softmax", score_fn=0,
-                                                        n_group=1, topk_group=1, S=0, Is=0, T=333,
-                                                        seed=22)], ids=lambda w: w.name)
+@pytest.mark.parametrize("wl", MX_CASES, ids=lambda w: w.name)
 def test_mxfp8_forward_matches_oracle(wl):
+    """MXFP8 forward: routing bit-exact; the h codes and scales the gate/up epilogue
+    stored agree with the oracle's quantisation of h (see check_mx_h); y within
+    2e-2 relative RMS (the acceptance of record), pooled and for every token."""
     import oracle
     case = make_case(wl, device="cuda", gen_device="cpu", mx=True)
     params = _mx_params(case["params"])
@@ -145,9 +151,12 @@ def test_mxfp8_forward_matches_oracle(wl):
             a = L.arrays[name].copy()
             oracle.mx_fakequant_bf16(a)
             L.set(**{name: a})
+    hstat = check_mx_h(layer, L, case["idx"], np.arange(wl.T), routing["inv_perm"].cpu().numpy())
     yo = L.fwd(case["idx"], case["w"])
-    err = _rel_rms(to_np(y), yo)
+    err, worst = rel_rms_per_token(to_np(y), yo)
+    print(f"{wl.name}: relative RMS of y {err:.3g} pooled, {worst:.3g} worst token; h {hstat}")
     assert err <= 2e-2, err
+    assert worst <= 2e-2, worst
     # reruns are bit-identical
     y2 = layer.forward(case["x"])
     torch.cuda.synchronize()
