@@ -65,6 +65,14 @@ WORKLOADS = {
     # MXFP8 forward with 256 rows per routed expert on average, as in dsv3_mxfp8
     "dsv3_mxfp8_e32": Workload("dsv3_mxfp8_e32", T=1024, H=7168, E=32, k=8, I=2048, S=1, Is=2048,
                                score_fn=1, n_group=8, topk_group=4, mxfp8=True, backward=False, seed=7),
+    # 16 routed experts of the DeepSeek-V3 shape, 128 rows each on average (as dsv3), for
+    # per-kernel counter captures: about 3 GB on the device with gradients, every weight
+    # tensor larger than L2
+    "dsv3_e16_r128": Workload("dsv3_e16_r128", T=256, H=7168, E=16, k=8, I=2048, S=1, Is=2048,
+                              score_fn=1, n_group=8, topk_group=4, seed=8),
+    # the MXFP8 forward of the same shape with 256 rows per routed expert (as dsv3_mxfp8)
+    "dsv3_mxfp8_e16": Workload("dsv3_mxfp8_e16", T=512, H=7168, E=16, k=8, I=2048, S=1, Is=2048,
+                               score_fn=1, n_group=8, topk_group=4, mxfp8=True, backward=False, seed=9),
 }
 
 
