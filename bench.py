@@ -180,6 +180,79 @@ def algorithmic(wl, counts):
     return out
 
 
+def forward_algorithmic(wl, counts):
+    """FLOPs and bytes of one whole forward (the persistent kernel's work): the two
+    expert GEMMs plus the router (x read, three bf16 router terms written and read,
+    partial logits) and the combine (slot rows read, y written)."""
+    alg = algorithmic(wl, counts)
+    T, H, E, k, S = wl.T, wl.H, wl.E, wl.k, wl.S
+    slot_bytes = 2 if wl.mxfp8 else 4
+    fl = alg["gate_up_gemm"][0] + alg["down_gemm"][0] + 2 * 3 * H * E * T
+    nb = (alg["gate_up_gemm"][1] + alg["down_gemm"][1] + T * H * 2 + 2 * E * 3 * H * 2
+          + T * (k + S) * H * slot_bytes + T * H * 2)
+    return fl, nb
+
+
+STAMP_PHASES = ["p0_zero_split_quant", "router_gemm", "select", "dispatch", "gate_up_gemm", "down_after_gate_up",
+                "combine"]
+
+
+def stamp_phases(bufs, sms):
+    """Phase spans (ms) of the persistent forward from its device stamps, averaged over
+    steps: a phase runs from the last CTA's end of the previous phase (the barrier
+    release) to the last CTA's end of its own; the down GEMM overlaps the gate/up
+    tail, so its span counts only the part after the last gate/up tile."""
+    import numpy as np
+    acc = np.zeros(len(STAMP_PHASES))
+    for b in bufs:
+        t = b.view(-1, sms).cpu().numpy().astype(np.float64)
+        ends = t.max(axis=1)
+        acc[0] += ends[1] - t[0].min()
+        acc[1:] += np.diff(ends[1:])
+    return {n: round(float(v) / len(bufs) / 1e6, 4) for n, v in zip(STAMP_PHASES, acc)}
+
+
+def forward_ab(layer, x, y, K):
+    """Forward only, K steps each: the split schedule with an event per step, then the
+    persistent schedule (one launch) with its device stamps."""
+    import torch
+    from mixture_experts_layer_persistent_b200 import abi, moe_trace_events
+    dev = x.device
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    out = {}
+    for name, sched in (("split", abi.MOK_SCHEDULE_SPLIT), ("persistent", abi.MOK_SCHEDULE_PERSISTENT)):
+        abi.moe_set_schedule(sched)
+        for _ in range(2):
+            layer.forward(x, y)
+        fev = [[mk() for _ in range(abi.MOK_FWD_PHASES + 1)] for _ in range(K)]
+        for e in [e for ev in fev for e in ev]:
+            e.record()
+        bufs = [torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) for _ in range(K)]
+        torch.cuda.synchronize()
+        s, e = mk(), mk()
+        s.record()
+        for i in range(K):
+            moe_trace_events([ev.cuda_event for ev in fev[i]], None)
+            abi.moe_trace_device(bufs[i].data_ptr(), bufs[i].numel() * 8)
+            layer.forward(x, y)
+            launches = abi.moe_launch_count()
+        e.record()
+        torch.cuda.synchronize()
+        moe_trace_events(None, None)
+        abi.moe_trace_device(None, 0)
+        r = {"ms_per_fwd": s.elapsed_time(e) / K, "launches_per_fwd": launches}
+        if name == "split":
+            r["phases_ms"] = {n: round(statistics.mean(fev[i][j].elapsed_time(fev[i][j + 1]) for i in range(K)), 4)
+                              for j, n in enumerate(FWD_PHASES)}
+        else:
+            r["device_phases_ms"] = stamp_phases(bufs, sms)
+        out[name] = r
+    abi.moe_set_schedule(abi.MOK_SCHEDULE_PERSISTENT)
+    out["persistent_over_split_speedup"] = out["split"]["ms_per_fwd"] / out["persistent"]["ms_per_fwd"]
+    return out
+
+
 def measured_traffic(wl, phase):
     """DRAM bytes per launch of `phase` from the committed ncu capture, or None
     when the workload differs or the kernel sources changed since the capture."""
@@ -286,6 +359,8 @@ def main():
     start, end = mk(), mk()
     for e in [e for ev in fev + bev for e in ev]:
         e.record()              # torch creates the CUDA event on its first record
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    stamps = [torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) for _ in range(K)]
     torch.cuda.synchronize()
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     if not uuid.startswith("GPU-"):
@@ -298,28 +373,39 @@ def main():
     start.record()
     for i in range(K):
         moe_trace_events([e.cuda_event for e in fev[i]], [e.cuda_event for e in bev[i]])
+        abi.moe_trace_device(stamps[i].data_ptr(), stamps[i].numel() * 8)
         step()
     end.record()
     torch.cuda.synchronize()
     moe_trace_events(None, None)
+    abi.moe_trace_device(None, 0)
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
     value, ms_max, _ = replica_throughput(start.elapsed_time(end), wl.T * K, dist, dev)
     status = layer.status()
 
-    phase = {}
-    for n_i, name in enumerate(FWD_PHASES):
-        phase[name] = statistics.mean(fev[i][n_i].elapsed_time(fev[i][n_i + 1]) for i in range(K))
+    # the forward is one persistent launch (events around it); the backward's steps are
+    # separate launches with an event each
+    phase = {"fwd_persistent": statistics.mean(fev[i][0].elapsed_time(fev[i][-1]) for i in range(K))}
     for n_i, name in enumerate(BWD_PHASES):
         phase[name] = statistics.mean(bev[i][n_i].elapsed_time(bev[i][n_i + 1]) for i in range(K))
-    fwd_ms = sum(phase[n] for n in FWD_PHASES)
+    fwd_ms = phase["fwd_persistent"]
     bwd_ms = sum(phase[n] for n in BWD_PHASES)
+    fwd_device_phases = stamp_phases(stamps, sms)
+
+    # forward A/B: split schedule (events per step, the per-GEMM attribution below) against
+    # the persistent one, forward only
+    ab = forward_ab(layer, x, y, K)
+    for n_i, name in enumerate(FWD_PHASES):
+        phase["split_" + name] = ab["split"]["phases_ms"][name]
 
     pk = peaks()
     alg = algorithmic(wl, counts)
-    dom = max(alg, key=lambda n: phase[n])
-    flops, nbytes = alg[dom]
+    kern = {"fwd_persistent": forward_algorithmic(wl, counts)}
+    kern.update({n: alg[n] for n in alg if n in phase})
+    dom = max(kern, key=lambda n: phase[n])
+    flops, nbytes = kern[dom]
     t_dom = phase[dom] / 1e3
     t_tc = flops / (pk["bf16_sustained"] * 1e12)
     t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
@@ -336,8 +422,8 @@ def main():
     roof["algorithmic_bytes"] = nbytes
     # every GEMM phase against both measured peaks (algorithmic bytes and FLOPs / its event time)
     phase_roofline = {}
-    for name, (fl, nb) in alg.items():
-        t = phase[name] / 1e3
+    for name, (fl, nb) in list(alg.items()) + [("fwd_persistent", kern["fwd_persistent"])]:
+        t = (phase[name] if name in phase else phase["split_" + name]) / 1e3
         phase_roofline[name] = {"ms": round(phase[name], 4), "hbm_frac": round(nb / t / 1e9 / pk["hbm_gbs"], 4),
                                 "tc_frac_sustained": round(fl / t / 1e12 / pk["bf16_sustained"], 4)}
 
@@ -383,12 +469,13 @@ def main():
                                    + (f", Zipf({wl.zipf}) logit term" if wl.zipf else ""),
                        "tokens_per_gpu": wl.T, "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (22.6 GB expert weights streamed per pass)"},
-            # forward: router split, router GEMM, select, 3 dispatch kernels, gate/up, down,
-            # combine (9); backward: slot grad, 2 router-gradient kernels, 4 GEMMs plus the
-            # resident weight-gradient kernels, dx sum (10)
+            # forward: one persistent kernel; backward: down dgrad, slot grad, 2 router-gradient
+            # kernels, 4 GEMMs plus the resident weight-gradient kernels, dx sum (10)
             "gpu_launches": K * (launches[0] + launches[1]),
             "clocks": clk, "device_status": status,
             "phases_ms": {k2: round(v, 4) for k2, v in phase.items()},
+            "fwd_device_phases_ms": fwd_device_phases,
+            "forward_schedule_ab": ab,
             "breakdown": {
                 "fwd_bf16_tokens_per_s": fwd_tps, "bwd_bf16_tokens_per_s": bwd_tps,
                 "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
@@ -455,8 +542,10 @@ def bf16_workload_run(wl, dev, K, warmup, world, dist, pk):
     ms = float(t.item()) / K
     fwd_ms = statistics.mean(fev[i][0].elapsed_time(fev[i][-1]) for i in range(K))
     bwd_ms = statistics.mean(bev[i][0].elapsed_time(bev[i][-1]) for i in range(K)) if wl.backward else 0.0
+    ab = forward_ab(layer, x, y, K)
     fwd_flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
-    out = {"workload": f"{wl.name}: MoE layer {'fwd+bwd' if wl.backward else 'fwd'} BF16, T={wl.T}, H={wl.H}, "
+    out = {"forward_schedule_ab": ab,
+           "workload": f"{wl.name}: MoE layer {'fwd+bwd' if wl.backward else 'fwd'} BF16, T={wl.T}, H={wl.H}, "
                        f"E={wl.E}, top-{wl.k}, I={wl.I}, {wl.S} shared"
                        + (f", Zipf({wl.zipf}) logit term" if wl.zipf else ""),
            "tokens_per_s": wl.T * world / (ms / 1e3), "ms_per_step": ms,
@@ -515,8 +604,8 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item()) / K
-    phases = {n: statistics.mean(fev[i][j].elapsed_time(fev[i][j + 1]) for i in range(K))
-              for j, n in enumerate(FWD_PHASES)}
+    ab = forward_ab(layer, x, y, K)
+    phases = ab["split"]["phases_ms"]              # per-step times: the split schedule's events
     flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
     gemm_ms = phases["gate_up_gemm"] + phases["down_gemm"]
     del layer, params, x, y
@@ -527,7 +616,8 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk):
     peak = fp8["burst_tflops"]
     return {"workload": f"{wl.name}: MoE layer fwd MXFP8 (e4m3, 1x32 ue8m0), T={wl.T}, H={wl.H}, E={wl.E}, "
                         f"top-{wl.k}, I={wl.I}, {wl.S} shared",
-            "tokens_per_s": wl.T * world / (ms / 1e3), "ms_per_fwd": ms, "phases_ms": {k: round(v, 4) for k, v in phases.items()},
+            "tokens_per_s": wl.T * world / (ms / 1e3), "ms_per_fwd": ms, "split_phases_ms": phases,
+            "forward_schedule_ab": ab,
             "layer_tflops": flops / (ms / 1e3) / 1e12,
             "fp8_peak": fp8, "fp8_peak_tflops": peak,
             "fp8_peak_source": "measured burst (torch._scaled_mm e4m3 8192^3 on this GPU)",

@@ -212,7 +212,9 @@ int moe_quantize_mxfp8_weights(const void *src, int64_t rows, int64_t K, void *q
  * Phase tracing.  When events are set, every later moe_fwd (moe_bwd) records
  * fwd_events[i] (bwd_events[i]) on its stream just before launching phase i
  * and the last event after its final launch, so that elapsed times between
- * consecutive events time each phase on the launching stream.  Events are
+ * consecutive events time each phase on the launching stream.  Under the
+ * persistent forward schedule the forward is one launch: fwd_events[0] is
+ * recorded before it and the others after it (see moe_trace_device).  Events are
  * cudaEvent_t handles owned by the caller.  Phases:
  *   forward  (MOK_FWD_PHASES = 5, needs 6 events): router, dispatch,
  *            gate/up GEMM, down GEMM, combine
@@ -283,6 +285,36 @@ int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, 
 #define MOK_SAVED_ROW_TOKEN 5
 #define MOK_SAVED_ROW_W 6
 int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_t *offset, size_t *bytes);
+
+/*
+ * Schedule of the forward pass (per host thread; default PERSISTENT).
+ *   MOK_SCHEDULE_PERSISTENT  the whole forward is one cooperative launch of one
+ *       persistent kernel, one CTA per SM: router, top-k, dispatch, the two
+ *       expert GEMMs and the combine are phases separated by grid barriers,
+ *       except that the down GEMM starts an M tile as soon as every gate/up tile
+ *       of its rows is in memory (per-tile readiness counters) -- the fusion of
+ *       the layer into one kernel that "Cursor åpner megakernelen…" (the quoted
+ *       paragraph) describes.  No memset or other launch precedes it.
+ *   MOK_SCHEDULE_SPLIT  one launch per step in stream order (router split,
+ *       router GEMM, select, three dispatch kernels, [MXFP8: quantise x], gate/up,
+ *       down, combine) after a memset of the tile counters: the comparison point.
+ * Both schedules give byte-identical results.  The backward is always split.
+ */
+#define MOK_SCHEDULE_PERSISTENT 0
+#define MOK_SCHEDULE_SPLIT 1
+int moe_set_schedule(int schedule);
+int moe_get_schedule(int *schedule);
+
+/*
+ * Device-side phase stamps of the persistent forward (per host thread).  When
+ * buf (device memory, at least MOK_TRACE_POINTS * SMs * 8 bytes) is set, every
+ * later persistent forward writes, for each point p and CTA b, the globaltimer
+ * value (ns) at buf[p * SMs + b]: p = 0 start, then the end of the zeroing /
+ * router-split / quantisation phase, the router GEMM, the top-k, the dispatch,
+ * the gate/up GEMM, the down GEMM and the combine.  NULL stops it.
+ */
+#define MOK_TRACE_POINTS 8
+int moe_trace_device(void *buf, size_t bytes);
 
 /*
  * Number of CUDA kernels launched by the last moe_fwd / moe_bwd (or their

@@ -29,6 +29,9 @@ MOK_DTYPE_MXFP8 = 1
 MOK_FWD_PHASES = 5
 MOK_BWD_PHASES = 8
 MOK_STATIC_SCRATCH_BYTES = 32 << 20
+MOK_SCHEDULE_PERSISTENT = 0
+MOK_SCHEDULE_SPLIT = 1
+MOK_TRACE_POINTS = 8
 MOK_SAVED_H, MOK_SAVED_HQ, MOK_SAVED_HS, MOK_SAVED_GU, MOK_SAVED_HW, MOK_SAVED_ROW_TOKEN, MOK_SAVED_ROW_W = range(7)
 
 _i32, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
@@ -91,13 +94,17 @@ def lib():
         L.moe_test_drop_signal.argtypes = [ctypes.c_int]
         L.moe_launch_count.argtypes = [P(_i32)]
         L.moe_saved_tensor.argtypes = [P(moe_cfg), _i32, _i32, P(_sz), P(_sz)]
+        L.moe_set_schedule.argtypes = [ctypes.c_int]
+        L.moe_get_schedule.argtypes = [P(_i32)]
+        L.moe_trace_device.argtypes = [_vp, _sz]
         L.moe_strerror.argtypes = [ctypes.c_int]
         L.moe_strerror.restype = ctypes.c_char_p
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
                      "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_quantize_mxfp8_weights", "moe_status",
-                     "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal", "moe_saved_tensor"):
+                     "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal", "moe_saved_tensor",
+                     "moe_set_schedule", "moe_get_schedule", "moe_trace_device"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -117,6 +124,20 @@ def moe_workspace_size(cfg: moe_cfg):
     _check("moe_workspace_size", lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(c),
                                                           ctypes.byref(f), ctypes.byref(b)))
     return c.value, f.value, b.value
+
+
+def moe_set_schedule(schedule: int) -> None:
+    _check("moe_set_schedule", lib().moe_set_schedule(int(schedule)))
+
+
+def moe_get_schedule() -> int:
+    v = _i32()
+    _check("moe_get_schedule", lib().moe_get_schedule(ctypes.byref(v)))
+    return v.value
+
+
+def moe_trace_device(buf, nbytes: int) -> None:
+    _check("moe_trace_device", lib().moe_trace_device(buf, int(nbytes)))
 
 
 def moe_saved_tensor(cfg: moe_cfg, save_for_backward: bool, which: int):

@@ -38,13 +38,11 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8])
 // Thread = 8 columns of one token (16-byte loads).
 // O: fp32 slot rows (BF16 layer) or bf16 slot rows (MXFP8 forward)
 template <class Slot>
-__global__ void __launch_bounds__(256) combine_kernel(const Slot *__restrict__ O,
-                                                      const float *__restrict__ topk_w,
-                                                      __nv_bfloat16 *__restrict__ y, int T, int H, int k, int S)
+__device__ __forceinline__ void combine_elem(long long i, const Slot *__restrict__ O,
+                                             const float *__restrict__ topk_w, __nv_bfloat16 *__restrict__ y,
+                                             int H, int k, int S)
 {
     const int cpr = H / 8;
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (long long)T * cpr) return;
     const int t = (int)(i / cpr), c = (int)(i % cpr) * 8;
     const int kk = k + S;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -57,6 +55,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const Slot *__restrict__ O
         for (int q = 0; q < 8; ++q) acc[q] = fmaf(w, v[q], acc[q]);
     }
     *reinterpret_cast<uint4 *>(y + (size_t)t * H + c) = pack8(acc);
+}
+
+template <class Slot>
+__global__ void __launch_bounds__(256) combine_kernel(const Slot *__restrict__ O,
+                                                      const float *__restrict__ topk_w,
+                                                      __nv_bfloat16 *__restrict__ y, int T, int H, int k, int S)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < (long long)T * (H / 8)) combine_elem(i, O, topk_w, y, H, k, S);
 }
 
 // Backward, per token: G_j = <dy[t], o_j> (j < k), summed in a fixed order from the

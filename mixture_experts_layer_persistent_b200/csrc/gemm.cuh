@@ -41,6 +41,9 @@ constexpr int kPanelM = 8;     // ragged-M raster panel height (M tiles)
 
 enum Epi : int { EPI_SWIGLU = 0, EPI_PUSH = 1, EPI_DSWIGLU = 2, EPI_WGRAD = 3, EPI_ROUTER = 4 };
 
+constexpr int kGemmBarBytes = 256;                 // mbarriers, abort flag, schedule slots of one phase
+constexpr int kGemmAuxBytes = 3 * kMaxGroups * 4;  // group offsets, tile starts, group order
+
 struct GemmArgs {
     int num_groups;               // G
     int num_routed;               // groups [0, num_routed) use tmB, the rest tmB_s / out_s
@@ -83,7 +86,17 @@ struct GemmArgs {
                                   // (a prefix of gorder); the resident kernel takes the rest
     int m_per_unit;               // resident weight-gradient kernel: M tiles per work unit
     int *sched;                   // tile counter of this launch, zero before it (one per launch)
+    // Per-M-tile readiness between two ragged-M GEMMs of one persistent launch (the
+    // gate/up GEMM produces the rows the down GEMM reads).  Counter of the M tile
+    // (g, mt) = ready[tstart(g) / n_tiles + mt], zero before the producing phase.
+    int *ready;                   // null: no readiness tracking
+    int ready_role;               // kReadySignal: each epilogue warp adds 1 per tile once its stores
+                                  // are complete; kReadyWait: the producer waits for ready_target
+                                  // before it hands a tile to the other roles
+    int ready_target;
 };
+
+constexpr int kReadyNone = 0, kReadySignal = 1, kReadyWait = 2;
 
 template <int BN_, bool A_MN_, bool B_MN_, bool A_GATHER_, bool B_GATHER_, bool RAGGED_K_, int EPI_,
           bool MX_ = false>
@@ -123,11 +136,13 @@ struct GemmCfg {
     static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
     static constexpr int SF_TMEM_COL = 256;                      // SFA at 256..259, SFB at 260..
     static constexpr int EPI_STAGE_BYTES = EPI_WARPS * EPI_BUFS * 4096;   // 32 x 128-byte blocks per epilogue warp
-    static constexpr int AUX_BYTES = 256 + 3 * kMaxGroups * 4;
     // the epilogue staging blocks follow the scale region and must stay 1024-byte
     // aligned (their 128-byte swizzle phase comes from the address)
     static constexpr int SF_REGION = (STAGES * SF_BYTES + 1023) / 1024 * 1024;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + SF_REGION + EPI_STAGE_BYTES + AUX_BYTES;
+    // ring, scale blocks and staging: the part of shared memory a GEMM phase carves
+    static constexpr int RING_BYTES = STAGES * STAGE_BYTES + SF_REGION + EPI_STAGE_BYTES;
+    // standalone kernel: ring, then the phase's barrier block, group tables and TMEM slot
+    static constexpr int SMEM_BYTES = 1024 + RING_BYTES + kGemmBarBytes + kGemmAuxBytes + 16;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
     static_assert(!MX || (!A_MN && !B_MN && !RAGGED_K && BN == 256 && (EPI == EPI_SWIGLU || EPI == EPI_PUSH)),
                   "MXFP8 serves the forward expert GEMMs");
@@ -349,28 +364,83 @@ __device__ __forceinline__ void load_row_direct(uint32_t *p, const void *src)
     }
 }
 
-template <class C>
-__global__ void __launch_bounds__(C::THREADS, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmB_s, const __grid_constant__ CUtensorMap tmO,
-                        const __grid_constant__ CUtensorMap tmO2, const __grid_constant__ CUtensorMap tmO3,
-                        const GemmArgs args)
+// ---- readiness between the phases of one persistent launch --------------------
+__device__ __forceinline__ void red_release_gpu_add(int *p, int v)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *p)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Order this thread's generic-proxy accesses with its async-proxy (TMA) accesses of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Producer lane: wait until the M tile's counter reaches the target (bounded;
+// gives up as mbar_wait does).  Loads the tile's rows only after this returns true.
+__device__ __forceinline__ bool wait_ready(const int *ctr, int target, volatile int *abort, int *status)
+{
+    if (ld_acquire_gpu(ctr) >= target) {
+        fence_proxy_async_global();
+        return true;
+    }
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (ld_acquire_gpu(ctr) >= target) {
+            fence_proxy_async_global();
+            return true;
+        }
+        if ((i & 63u) == 0u && (*abort || globaltimer() - t0 > kWaitLimitNs)) {
+            *abort = 1;
+            atomicOr(status, kStatusTimeout);
+            return false;
+        }
+    }
+}
+
+// Epilogue warp: this warp's rows of the tile are in global memory (its TMA stores
+// complete, its plain stores fenced); count it on the tile's readiness counter.
+__device__ __forceinline__ void signal_ready(int *ctr, int lane)
+{
+    __syncwarp();
+    if (lane == 0) {
+        bulk_wait0();
+        fence_proxy_async_global();
+        __threadfence();
+        red_release_gpu_add(ctr, 1);
+    }
+    __syncwarp();
+}
+
+// One grouped-GEMM phase run by every thread of the CTA.
+//   smem       1024-byte aligned: C::RING_BYTES of stage ring, scale blocks and staging
+//   bar_block  kGemmBarBytes of barriers for this phase alone (not reused by another phase)
+//   aux        kGemmAuxBytes of group tables
+//   tmem_base  TMEM columns [0, C::TMEM_COLS) allocated by the caller
+// Starts and ends with a CTA-wide barrier.  A standalone launch wraps one phase;
+// the persistent forward runs several in one launch.
+template <class C>
+__device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, int *aux, uint32_t tmem_base,
+                                           const CUtensorMap &tmA, const CUtensorMap &tmB, const CUtensorMap &tmB_s,
+                                           const CUtensorMap &tmO, const CUtensorMap &tmO2, const CUtensorMap &tmO3,
+                                           const GemmArgs &args)
+{
     uint8_t *tiles = smem;
     uint8_t *sf_tiles = tiles + C::STAGES * C::STAGE_BYTES;     // MXFP8 scale blocks, one per stage
     uint32_t *epi_stage = reinterpret_cast<uint32_t *>(sf_tiles + C::SF_REGION);
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(epi_stage) + C::EPI_STAGE_BYTES);
+    uint64_t *full_bar = bar_block;
     uint64_t *empty_bar = full_bar + C::STAGES;
     uint64_t *accf = empty_bar + C::STAGES;
     uint64_t *acce = accf + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(acce + 2);
     const Sched sch{acce + 3, acce + 3 + kSchedSlots, reinterpret_cast<int *>(acce + 3 + 2 * kSchedSlots)};
     uint64_t *drain_bar = acce + 3 + 2 * kSchedSlots + (4 * kSchedSlots + 7) / 8;   // MMA drain on abort
-    static_assert(8 * (2 * C::STAGES + 6 + 2 * kSchedSlots) + 4 * kSchedSlots <= 256, "barrier region");
-    int *s_off = reinterpret_cast<int *>(full_bar) + 64;
+    static_assert(8 * (2 * C::STAGES + 6 + 2 * kSchedSlots) + 4 * kSchedSlots <= kGemmBarBytes, "barrier region");
+    int *s_off = aux;
     int *s_tstart = s_off + kMaxGroups;
     int *s_gorder = s_tstart + kMaxGroups;
 
@@ -423,13 +493,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tma_prefetch_desc(&tmB_s);
             tma_prefetch_desc(&tmO);
         }
-    } else if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    // data an earlier phase of the same launch wrote with plain stores is read here
+    // by TMA and cp.async: order the two proxies (free in a standalone launch)
+    fence_proxy_async_global();
     const int total = C::RAGGED_K ? count_big_groups(s_off, s_gorder, G, args.k_split) * args.m_tiles * args.n_tiles
                                   : s_tstart[G];
 
@@ -441,8 +511,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         int tile = blockIdx.x;
         for (int it = 0;; ++it) {
             bool put = true;
-            if (lane == 0) put = sched_put(sch, it, tile, abort_flag, status);
-            put = __shfl_sync(0xffffffffu, put, 0);
+            if constexpr (!C::RAGGED_K) {
+                if (args.ready_role == kReadyWait && tile < total) {
+                    // the rows this tile reads are produced by an earlier phase of the launch
+                    const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
+                    const int mt = s_tstart[t.g] / args.n_tiles + (t.m0 - s_off[t.g]) / BM;
+                    if (lane == 0) put = wait_ready(args.ready + mt, args.ready_target, abort_flag, status);
+                    put = __shfl_sync(0xffffffffu, put, 0);
+                    if (!put) tile = total;          // publish "no more work" to the other roles
+                }
+            }
+            bool put2 = true;
+            if (lane == 0) put2 = sched_put(sch, it, tile, abort_flag, status);
+            put = __shfl_sync(0xffffffffu, put2, 0) && put;
             if (!put || tile >= total) break;
             const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
             const bool routed = t.g < args.num_routed;
@@ -954,17 +1035,44 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 tc_fence_before();
                 mbar_arrive(&acce[acc]);
             }
+            if constexpr (!C::RAGGED_K) {
+                if (args.ready_role == kReadySignal)
+                    signal_ready(args.ready + s_tstart[t.g] / args.n_tiles + (t.m0 - s_off[t.g]) / BM, lane);
+            }
             if (++acc == C::ACC_BUFS) {
                 acc = 0;
                 acc_phase ^= 1u;
             }
         }
-        if (lane == 0) bulk_wait0();             // every bulk store of this warp has completed
+        if (lane == 0) {
+            bulk_wait0();                        // every bulk store of this warp has completed
+            fence_proxy_async_global();          // ... and is ordered before later plain accesses
+        }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB_s, const __grid_constant__ CUtensorMap tmO,
+                        const __grid_constant__ CUtensorMap tmO2, const __grid_constant__ CUtensorMap tmO3,
+                        const GemmArgs args)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::RING_BYTES);
+    int *aux = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(bars) + kGemmBarBytes);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(aux) + kGemmAuxBytes);
+    if ((threadIdx.x >> 5) == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    gemm_phase<C>(smem, bars, aux, tmem_base, tmA, tmB, tmB_s, tmO, tmO2, tmO3, args);
+    if ((threadIdx.x >> 5) == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
     }

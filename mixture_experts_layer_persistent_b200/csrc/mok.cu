@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "combine.cuh"
+#include "fused.cuh"
 #include "gemm.cuh"
 #include "quant.cuh"
 #include "route.cuh"
@@ -59,6 +60,9 @@ thread_local cudaEvent_t t_fwd_ev[MOK_FWD_PHASES + 1];
 thread_local cudaEvent_t t_bwd_ev[MOK_BWD_PHASES + 1];
 thread_local bool t_fwd_on = false, t_bwd_on = false;
 thread_local int t_drop_signal = 0;     // moe_test_drop_signal
+thread_local int t_schedule = MOK_SCHEDULE_PERSISTENT;   // moe_set_schedule
+thread_local unsigned long long *t_dev_trace = nullptr;   // moe_trace_device
+thread_local size_t t_dev_trace_bytes = 0;
 thread_local int t_launches = 0;        // kernels launched by the current / last forward or backward
 
 inline int mark_fwd(int i, cudaStream_t s)
@@ -183,6 +187,10 @@ struct State {
     float *O;                       // per-(token, slot) rows: fp32 (BF16), bf16 (MXFP8 forward)
     uint8_t *xq, *xs, *hq, *hs;     // MXFP8 operands
     int *sched;                     // [kSchedCounters] forward GEMM tile counters
+    int *ready;                     // [n_mtiles] per-M-tile readiness (persistent forward)
+    int *zero;                      // sched, ready and hist: the counters the persistent forward zeroes
+    int n_zero, n_mtiles;
+    unsigned long long *gs_flags;   // [kMaxFusedCtas] grid-barrier arrival tags, then release tag, epoch
     size_t bytes;
 };
 
@@ -205,7 +213,17 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
     st.row_slot = cv.take<int>(s.R);
     st.row_w = cv.take<float>(s.R);
     st.all_rows = cv.take<int>(2);
-    st.hist = cv.take<int>(((s.T + kDispatchChunk - 1) / kDispatchChunk) * s.E);
+    // tile counters, readiness counters and dispatch histograms in one range, zeroed
+    // at the start of the persistent forward (the split forward zeroes the tile
+    // counters with a memset; its histograms are written, not accumulated)
+    st.n_mtiles = static_cast<int>(s.R / BM + s.G + 1);
+    const long long n_hist = ((s.T + kDispatchChunk - 1) / kDispatchChunk) * s.E;
+    st.n_zero = static_cast<int>(kSchedCounters + st.n_mtiles + n_hist);
+    st.zero = cv.take<int>(st.n_zero);
+    st.sched = st.zero;
+    st.ready = st.zero + kSchedCounters;
+    st.hist = st.ready + st.n_mtiles;
+    st.gs_flags = cv.take<unsigned long long>(kMaxFusedCtas + 2);
     st.wr3 = cv.take<__nv_bfloat16>(s.E * 3 * s.H);
     st.rpart = cv.take<float>(static_cast<size_t>(s.n_split) * s.T * 256);
     st.gu = training ? cv.take<__nv_bfloat16>(s.R * 2 * s.I) : nullptr;
@@ -221,7 +239,6 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
         st.hq = st.hs = st.xq = st.xs = nullptr;
     }
     st.O = mx ? reinterpret_cast<float *>(cv.take<__nv_bfloat16>(s.T * s.kk * s.H)) : cv.take<float>(s.T * s.kk * s.H);
-    st.sched = cv.take<int>(kSchedCounters);
     st.bytes = align_up(cv.off, 256);
     return st;
 }
@@ -325,40 +342,39 @@ inline int blocks_for(long long n, int per) { return static_cast<int>((n + per -
     } while (0)
 
 // ------------------------------------------------------------------ forward
-int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const moe_routing *routing,
-            const State &st, const DeviceInfo &dev, bool training, cudaStream_t stream)
+// Tensor maps and arguments of every step of the forward, shared by the split
+// schedule (one launch per step) and the persistent one (one launch).
+struct FwdPlan {
+    FusedMaps m;
+    GemmArgs gr, ga, gd;
+    SelectArgs sa;
+    DispatchArgs da;
+    int n_chunks;
+};
+
+int build_fwd_plan(const moe_cfg &c, const void *x, const moe_params &p, const State &st, const DeviceInfo &dev,
+                   bool training, FwdPlan &pl)
 {
     const Shapes s = shapes(c);
-    t_launches = 0;
     const bool mx = c.dtype == MOK_DTYPE_MXFP8;
-    if (const cudaError_t e = cudaMemsetAsync(st.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
-        return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
-
     // router logits on the tensor cores: x . [Wr_hi | Wr_mid | Wr_lo]^T, split over K
-    MOK_TRY(mark_fwd(0, stream));
-    router_split_kernel<<<blocks_for(s.E * s.H, 256), 256, 0, stream>>>(p.router_w, st.wr3, c.E, c.H, st.all_rows,
-                                                                         c.T);
-    MOK_LAUNCHED();
-    {
-        CUtensorMap rA, rB, rO;
-        if (!make_tmap(&rA, x, s.H, s.T, BK, 128, 2)) return fail(MOK_ERR_INVALID, "tensor map (x)");
-        if (!make_tmap(&rB, st.wr3, 3 * s.H, s.E, BK, 256, 2)) return fail(MOK_ERR_INVALID, "tensor map (router)");
-        if (!make_tmap(&rO, st.rpart, 256, s.n_split * s.T, 32, 32, 4)) return fail(MOK_ERR_INVALID, "tensor map (logits)");
-        GemmArgs gr{};
-        gr.num_groups = 1;
-        gr.num_routed = 1;
-        gr.offsets = st.all_rows;
-        gr.n_tiles = s.n_split;
-        gr.num_kb = static_cast<int>(3 * s.H / BK / s.n_split);
-        gr.a_k_mod = c.H;
-        gr.out_f32 = st.rpart;
-        gr.rows_total = c.T;
-        gr.status = dev.status;
-        gr.sched = st.sched + 0;
-        using CRouter = GemmCfg<256, false, false, false, false, false, EPI_ROUTER>;
-        MOK_TRY(launch_gemm<CRouter>(rA, rB, rB, rO, rO, rO, gr, dev.sms, stream));
-    }
-    SelectArgs sa;
+    if (!make_tmap(&pl.m.rA, x, s.H, s.T, BK, 128, 2)) return fail(MOK_ERR_INVALID, "tensor map (x)");
+    if (!make_tmap(&pl.m.rB, st.wr3, 3 * s.H, s.E, BK, 256, 2)) return fail(MOK_ERR_INVALID, "tensor map (router)");
+    if (!make_tmap(&pl.m.rO, st.rpart, 256, s.n_split * s.T, 32, 32, 4)) return fail(MOK_ERR_INVALID, "tensor map (logits)");
+    GemmArgs &gr = pl.gr;
+    gr = GemmArgs{};
+    gr.num_groups = 1;
+    gr.num_routed = 1;
+    gr.offsets = st.all_rows;
+    gr.n_tiles = s.n_split;
+    gr.num_kb = static_cast<int>(3 * s.H / BK / s.n_split);
+    gr.a_k_mod = c.H;
+    gr.out_f32 = st.rpart;
+    gr.rows_total = c.T;
+    gr.status = dev.status;
+    gr.sched = st.sched + 0;
+
+    SelectArgs &sa = pl.sa;
     sa.partial = st.rpart;
     sa.n_split = s.n_split;
     sa.e_bias = p.e_bias;
@@ -367,10 +383,9 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     sa.score_fn = c.score_fn; sa.n_group = c.n_group; sa.topk_group = c.topk_group;
     sa.routed_scale = c.routed_scale;
     sa.topk_idx = st.topk_idx; sa.topk_w = st.topk_w; sa.topk_p = st.topk_p;
-    router_select_kernel<<<blocks_for(s.T, 8), 256, 0, stream>>>(sa);
-    MOK_LAUNCHED();
+    sa.hist = nullptr;
 
-    DispatchArgs da;
+    DispatchArgs &da = pl.da;
     da.topk_idx = st.topk_idx; da.topk_w = st.topk_w;
     da.T = c.T; da.k = c.top_k; da.E = c.E; da.S = c.n_shared; da.chunk_rows = kChunkRows;
     da.counts = st.counts; da.offsets = st.offsets; da.gorder = st.gorder; da.chunk_start = st.chunk_start;
@@ -378,62 +393,50 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     da.row_w = st.row_w;
     da.hist = st.hist;
     da.status = dev.status;
-    MOK_TRY(mark_fwd(1, stream));
-    {
-        const int n_chunks = static_cast<int>((s.T + kDispatchChunk - 1) / kDispatchChunk);
-        dispatch_count_kernel<<<n_chunks, 1024, 0, stream>>>(da);
-        MOK_LAUNCHED();
-        dispatch_scan_kernel<<<1, 256, 0, stream>>>(da, n_chunks);
-        MOK_LAUNCHED();
-        dispatch_place_kernel<<<n_chunks, 1024, 0, stream>>>(da);
-        MOK_LAUNCHED();
-    }
+    pl.n_chunks = static_cast<int>((s.T + kDispatchChunk - 1) / kDispatchChunk);
 
+    GemmArgs &ga = pl.ga;
+    GemmArgs &gd = pl.gd;
+    ga = GemmArgs{};
+    ga.sched = st.sched + 1;
+    ga.num_groups = static_cast<int>(s.G);
+    ga.num_routed = c.E;
+    ga.offsets = st.offsets;
+    ga.row_token = st.row_token;
+    ga.row_slot = st.row_slot;
+    ga.row_w = st.row_w;
+    ga.n_tiles = c.I / 128;
+    ga.b_rows_per_group = 2 * c.I;
+    ga.b_half = c.I;
+    ga.inter = c.I;
+    ga.gather_ld = c.H;
+    ga.status = dev.status;
+    ga.test_drop_signal = t_drop_signal;
+    ga.ready = st.ready;
     if (mx) {
-        // MXFP8: quantise x (1x32 ue8m0 blocks along H), then block-scaled expert GEMMs
-        MOK_TRY(mark_fwd(2, stream));
-        const long long xb = s.T * s.H / 32;
-        quantize_mxfp8_kernel<<<blocks_for(xb, 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(x), xb,
-                                                                        st.xq, st.xs, s.H / 32, 0);
-        MOK_LAUNCHED();
-        CUtensorMap tA, tB, tBs, tO;
-        if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, 128, 128, 1)) return MOK_ERR_INVALID;
-        if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 128, 128, 1))
+        // MXFP8: block-scaled expert GEMMs on the quantised x (1x32 ue8m0 blocks along H)
+        if (!make_tmap(&pl.m.gB, p.w_gate_up, s.H, s.E * 2 * s.I, 128, 128, 1)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.gBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 128, 128, 1))
             return MOK_ERR_INVALID;
-        if (!make_tmap(&tO, st.hq, s.I, s.R, 128, 32, 1)) return MOK_ERR_INVALID;
-        GemmArgs ga{};
-        ga.sched = st.sched + 1;
-        ga.num_groups = static_cast<int>(s.G);
-        ga.num_routed = c.E;
-        ga.offsets = st.offsets;
-        ga.row_token = st.row_token;
-        ga.row_slot = st.row_slot;
-        ga.row_w = st.row_w;
-        ga.n_tiles = c.I / 128;
+        if (!make_tmap(&pl.m.gO, st.hq, s.I, s.R, 128, 32, 1)) return MOK_ERR_INVALID;
+        pl.m.gO2 = pl.m.gO3 = pl.m.gO;
         ga.num_kb = c.H / 128;
-        ga.b_rows_per_group = 2 * c.I;
-        ga.b_half = c.I;
         ga.out = reinterpret_cast<__nv_bfloat16 *>(st.hq);
         ga.out_scales = st.hs;
-        ga.inter = c.I;
         ga.gather_src = reinterpret_cast<const __nv_bfloat16 *>(st.xq);
-        ga.gather_ld = c.H;
         ga.sfa_src = st.xs;
         ga.sfb_src = p.s_gate_up;
         ga.sfb_src_s = s.S ? p.ss_gate_up : p.s_gate_up;
         ga.sf_ld = c.H / 32;
         ga.sfb_row_tiles = static_cast<int>(s.E * 2 * s.I / 128);
         ga.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : s.E) * 2 * s.I / 128);
-        ga.status = dev.status;
-        using CGateUpMx = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU, true>;
-        MOK_TRY(launch_gemm<CGateUpMx>(tB, tB, tBs, tO, tO, tO, ga, dev.sms, stream));
 
-        if (!make_tmap(&tA, st.hq, s.I, s.R, 128, 128, 1)) return MOK_ERR_INVALID;
-        if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 128, 256, 1)) return MOK_ERR_INVALID;
-        if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 128, 256, 1))
+        if (!make_tmap(&pl.m.dA, st.hq, s.I, s.R, 128, 128, 1)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.dB, p.w_down, s.I, s.E * s.H, 128, 256, 1)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.dBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 128, 256, 1))
             return MOK_ERR_INVALID;
-        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;   // bf16 slot rows
-        GemmArgs gd = ga;
+        if (!make_tmap(&pl.m.dO, st.O, s.H, s.T * s.kk, 64, 1, 2)) return MOK_ERR_INVALID;   // bf16 slot rows
+        gd = ga;
         gd.sched = st.sched + 2;
         gd.n_tiles = c.H / 256;
         gd.num_kb = c.I / 128;
@@ -450,48 +453,27 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         gd.sf_ld = c.I / 32;
         gd.sfb_row_tiles = static_cast<int>(s.E * s.H / 128);
         gd.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : s.E) * s.H / 128);
-        using CDownMx = GemmCfg<256, false, false, false, false, false, EPI_PUSH, true>;
-        MOK_TRY(mark_fwd(3, stream));
-        MOK_TRY(launch_gemm<CDownMx>(tA, tB, tBs, tO, tO, tO, gd, dev.sms, stream));
     } else {
         // gate/up: pull token rows by index, SwiGLU epilogue
-        CUtensorMap tA, tB, tBs, tO, tO2, tO3;
-        if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, BK, 128, 2)) return MOK_ERR_INVALID;
-        if (!make_tmap(&tO, st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
-        if (!make_tmap(&tO2, training ? st.gu : st.h, training ? 2 * s.I : s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
-        if (!make_tmap(&tO3, training ? st.hw : st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
-        if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, BK, 128, 2))
+        if (!make_tmap(&pl.m.gB, p.w_gate_up, s.H, s.E * 2 * s.I, BK, 128, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.gO, st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.gO2, training ? st.gu : st.h, training ? 2 * s.I : s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.gO3, training ? st.hw : st.h, s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.gBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, BK, 128, 2))
             return MOK_ERR_INVALID;
-        GemmArgs ga{};
-        ga.sched = st.sched + 1;
-        ga.num_groups = static_cast<int>(s.G);
-        ga.num_routed = c.E;
-        ga.offsets = st.offsets;
-        ga.row_token = st.row_token;
-        ga.row_slot = st.row_slot;
-        ga.row_w = st.row_w;
-        ga.n_tiles = c.I / 128;
         ga.num_kb = c.H / BK;
-        ga.b_rows_per_group = 2 * c.I;
-        ga.b_half = c.I;
         ga.out = st.h;
         ga.out2 = training ? st.gu : nullptr;
         ga.out3 = training ? st.hw : nullptr;
-        ga.inter = c.I;
         ga.gather_src = static_cast<const __nv_bfloat16 *>(x);
-        ga.gather_ld = c.H;
-        ga.status = dev.status;
-        ga.test_drop_signal = t_drop_signal;
-        using CGateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU>;
-        MOK_TRY(mark_fwd(2, stream));
-        MOK_TRY(launch_gemm<CGateUp>(tB, tB, tBs, tO, tO2, tO3, ga, dev.sms, stream));
 
         // down: contiguous h rows, push epilogue into (token, slot) rows
-        if (!make_tmap(&tA, st.h, s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
-        if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, BK, 256, 2)) return MOK_ERR_INVALID;
-        if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, BK, 256, 2))
+        if (!make_tmap(&pl.m.dA, st.h, s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.dB, p.w_down, s.I, s.E * s.H, BK, 256, 2)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.dBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, BK, 256, 2))
             return MOK_ERR_INVALID;
-        GemmArgs gd = ga;
+        if (!make_tmap(&pl.m.dO, st.O, s.H, s.T * s.kk, 32, 1, 4)) return MOK_ERR_INVALID;
+        gd = ga;
         gd.sched = st.sched + 2;
         gd.n_tiles = c.H / 256;
         gd.num_kb = c.I / BK;
@@ -501,11 +483,71 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         gd.out_f32 = st.O;
         gd.out2 = gd.out3 = nullptr;
         gd.ldo = c.H;
-        using CDown = GemmCfg<256, false, false, false, false, false, EPI_PUSH>;
-        MOK_TRY(mark_fwd(3, stream));
-        if (!make_tmap(&tO, st.O, s.H, s.T * s.kk, 32, 1, 4)) return MOK_ERR_INVALID;
-        MOK_TRY(launch_gemm<CDown>(tA, tB, tBs, tO, tO, tO, gd, dev.sms, stream));
+    }
+    gd.ready_target = 4 * (c.I / 128);    // four epilogue warps per gate/up tile, I/128 tiles per M tile
+    return MOK_OK;
+}
 
+int copy_routing(const moe_routing *routing, const State &st, const Shapes &s, cudaStream_t stream)
+{
+    if (!routing) return MOK_OK;
+    const size_t tk = static_cast<size_t>(s.TK);
+    struct { void *dst; const void *src; size_t n; } cp[] = {
+        {routing->topk_idx, st.topk_idx, tk * 4}, {routing->topk_w, st.topk_w, tk * 4},
+        {routing->counts, st.counts, static_cast<size_t>(s.E) * 4},
+        {routing->offsets, st.offsets, static_cast<size_t>(s.E + 1) * 4},
+        {routing->perm, st.perm, tk * 4}, {routing->inv_perm, st.inv_perm, tk * 4}};
+    for (const auto &q : cp)
+        if (q.dst)
+            if (const cudaError_t e = cudaMemcpyAsync(q.dst, q.src, q.n, cudaMemcpyDeviceToDevice, stream); e != cudaSuccess)
+                return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e);
+    return MOK_OK;
+}
+
+// Split schedule: one launch per step, in stream order.
+int forward_split(const moe_cfg &c, const void *x, const moe_params &p, void *y, const State &st,
+                  const DeviceInfo &dev, const FwdPlan &pl, cudaStream_t stream)
+{
+    const Shapes s = shapes(c);
+    const bool mx = c.dtype == MOK_DTYPE_MXFP8;
+    if (const cudaError_t e = cudaMemsetAsync(st.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
+    MOK_TRY(mark_fwd(0, stream));
+    router_split_kernel<<<blocks_for(s.E * s.H, 256), 256, 0, stream>>>(p.router_w, st.wr3, c.E, c.H, st.all_rows,
+                                                                         c.T);
+    MOK_LAUNCHED();
+    MOK_TRY(launch_gemm<typename FusedCfg<false>::Router>(pl.m.rA, pl.m.rB, pl.m.rB, pl.m.rO, pl.m.rO, pl.m.rO, pl.gr,
+                                                         dev.sms, stream));
+    router_select_kernel<<<blocks_for(s.T, 8), 256, 0, stream>>>(pl.sa);
+    MOK_LAUNCHED();
+
+    MOK_TRY(mark_fwd(1, stream));
+    dispatch_count_kernel<<<pl.n_chunks, 1024, 0, stream>>>(pl.da);
+    MOK_LAUNCHED();
+    dispatch_scan_kernel<<<1, 256, 0, stream>>>(pl.da, pl.n_chunks);
+    MOK_LAUNCHED();
+    dispatch_place_kernel<<<pl.n_chunks, 1024, 0, stream>>>(pl.da);
+    MOK_LAUNCHED();
+
+    MOK_TRY(mark_fwd(2, stream));
+    GemmArgs ga = pl.ga, gd = pl.gd;
+    ga.ready_role = gd.ready_role = kReadyNone;
+    if (mx) {
+        const long long xb = s.T * s.H / 32;
+        quantize_mxfp8_kernel<<<blocks_for(xb, 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(x), xb,
+                                                                        st.xq, st.xs, s.H / 32, 0);
+        MOK_LAUNCHED();
+        MOK_TRY(launch_gemm<typename FusedCfg<true>::GateUp>(pl.m.gB, pl.m.gB, pl.m.gBs, pl.m.gO, pl.m.gO2, pl.m.gO3,
+                                                            ga, dev.sms, stream));
+        MOK_TRY(mark_fwd(3, stream));
+        MOK_TRY(launch_gemm<typename FusedCfg<true>::Down>(pl.m.dA, pl.m.dB, pl.m.dBs, pl.m.dO, pl.m.dO, pl.m.dO, gd,
+                                                          dev.sms, stream));
+    } else {
+        MOK_TRY(launch_gemm<typename FusedCfg<false>::GateUp>(pl.m.gB, pl.m.gB, pl.m.gBs, pl.m.gO, pl.m.gO2, pl.m.gO3,
+                                                             ga, dev.sms, stream));
+        MOK_TRY(mark_fwd(3, stream));
+        MOK_TRY(launch_gemm<typename FusedCfg<false>::Down>(pl.m.dA, pl.m.dB, pl.m.dBs, pl.m.dO, pl.m.dO, pl.m.dO, gd,
+                                                           dev.sms, stream));
     }
 
     MOK_TRY(mark_fwd(4, stream));
@@ -517,18 +559,83 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
         combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(
             st.O, st.topk_w, static_cast<__nv_bfloat16 *>(y), c.T, c.H, c.top_k, c.n_shared);
     MOK_LAUNCHED();
-    MOK_TRY(mark_fwd(5, stream));
+    return mark_fwd(5, stream);
+}
 
-    if (routing) {
-        const size_t tk = static_cast<size_t>(s.TK);
-        if (routing->topk_idx) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->topk_idx, st.topk_idx, tk * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
-        if (routing->topk_w) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->topk_w, st.topk_w, tk * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
-        if (routing->counts) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->counts, st.counts, s.E * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
-        if (routing->offsets) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->offsets, st.offsets, (s.E + 1) * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
-        if (routing->perm) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->perm, st.perm, tk * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
-        if (routing->inv_perm) { if (const cudaError_t e_ = cudaMemcpyAsync(routing->inv_perm, st.inv_perm, tk * 4, cudaMemcpyDeviceToDevice, stream); e_ != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaMemcpyAsync(routing)", e_); }
-    }
+// Persistent schedule: the whole forward as one cooperative launch (fused.cuh).
+// Cooperative, so that every CTA is resident at once (the grid barriers and the
+// readiness waits need that) or the launch fails; one CTA per SM.
+template <bool MX>
+int launch_fused(const moe_cfg &c, const void *x, const moe_params &p, void *y, const State &st,
+                 const DeviceInfo &dev, const FwdPlan &pl, cudaStream_t stream)
+{
+    using F = FusedCfg<MX>;
+    if (dev.sms > kMaxFusedCtas) return fail(MOK_ERR_UNSUPPORTED, "more SMs than the grid barrier holds");
+    FusedFwdArgs a{};
+    a.gs.flags = st.gs_flags;
+    a.gs.go = st.gs_flags + kMaxFusedCtas;
+    a.gs.epoch = st.gs_flags + kMaxFusedCtas + 1;
+    a.status = dev.status;
+    a.zero = st.zero;
+    a.n_zero = st.n_zero;
+    a.router_w = p.router_w;
+    a.wr3 = st.wr3;
+    a.all_rows = st.all_rows;
+    a.T = c.T; a.H = c.H; a.E = c.E; a.k = c.top_k; a.S = c.n_shared;
+    a.x = static_cast<const __nv_bfloat16 *>(x);
+    a.xq = st.xq;
+    a.xs = st.xs;
+    a.gr = pl.gr;
+    a.ga = pl.ga;
+    a.gd = pl.gd;
+    a.ga.ready_role = kReadySignal;
+    a.gd.ready_role = kReadyWait;
+    a.sa = pl.sa;
+    a.sa.hist = st.hist;
+    a.da = pl.da;
+    a.n_chunks = pl.n_chunks;
+    a.O = st.O;
+    a.y = static_cast<__nv_bfloat16 *>(y);
+    a.trace = (t_dev_trace && t_dev_trace_bytes >= sizeof(unsigned long long) * kFusedTracePoints * dev.sms)
+                  ? t_dev_trace : nullptr;
+
+    cudaError_t e = cudaFuncSetAttribute(moe_fwd_fused_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         F::SMEM_BYTES);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(moe_fwd_fused_kernel)", e);
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(static_cast<unsigned>(dev.sms));
+    lc.blockDim = dim3(kFusedThreads);
+    lc.dynamicSmemBytes = F::SMEM_BYTES;
+    lc.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    MOK_TRY(mark_fwd(0, stream));
+    e = cudaLaunchKernelEx(&lc, moe_fwd_fused_kernel<MX>, pl.m, a);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaLaunchKernelEx(moe_fwd_fused_kernel, cooperative)", e);
+    ++t_launches;
+    // one launch: the per-step events all mark its end (phase times come from moe_trace_device)
+    for (int i = 1; i <= MOK_FWD_PHASES; ++i) MOK_TRY(mark_fwd(i, stream));
     return MOK_OK;
+}
+
+int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const moe_routing *routing,
+            const State &st, const DeviceInfo &dev, bool training, cudaStream_t stream)
+{
+    t_launches = 0;
+    FwdPlan pl;
+    MOK_TRY(build_fwd_plan(c, x, p, st, dev, training, pl));
+    const bool mx = c.dtype == MOK_DTYPE_MXFP8;
+    if (t_schedule == MOK_SCHEDULE_SPLIT) {
+        MOK_TRY(forward_split(c, x, p, y, st, dev, pl, stream));
+    } else if (mx) {
+        MOK_TRY(launch_fused<true>(c, x, p, y, st, dev, pl, stream));
+    } else {
+        MOK_TRY(launch_fused<false>(c, x, p, y, st, dev, pl, stream));
+    }
+    return copy_routing(routing, st, shapes(c), stream);
 }
 
 // ------------------------------------------------------------------ backward
@@ -916,6 +1023,28 @@ int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_
     if (!p) return MOK_ERR_UNSUPPORTED;
     if (offset) *offset = static_cast<size_t>(static_cast<const char *>(p) - base);
     if (bytes) *bytes = n;
+    return MOK_OK;
+}
+
+int moe_set_schedule(int schedule)
+{
+    if (schedule != MOK_SCHEDULE_PERSISTENT && schedule != MOK_SCHEDULE_SPLIT) return MOK_ERR_INVALID;
+    t_schedule = schedule;
+    return MOK_OK;
+}
+
+int moe_get_schedule(int *schedule)
+{
+    if (!schedule) return MOK_ERR_INVALID;
+    *schedule = t_schedule;
+    return MOK_OK;
+}
+
+int moe_trace_device(void *buf, size_t bytes)
+{
+    if (buf && !aligned16(buf)) return MOK_ERR_INVALID;
+    t_dev_trace = static_cast<unsigned long long *>(buf);
+    t_dev_trace_bytes = buf ? bytes : 0;
     return MOK_OK;
 }
 

@@ -41,14 +41,12 @@ __device__ __forceinline__ long long packed_scale_offset(long long row, long lon
     return ((j >> 2) * row_tiles + (row >> 7)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (j & 3);
 }
 
-// row_tiles = 0: scales [rows, K/32] row-major; row_tiles = rows / 128: packed layout
-__global__ void __launch_bounds__(256) quantize_mxfp8_kernel(const __nv_bfloat16 *__restrict__ src,
-                                                             long long nblocks, uint8_t *__restrict__ q,
-                                                             uint8_t *__restrict__ scales, long long kb32,
-                                                             long long row_tiles)
+// Block b (32 elements) of src.  row_tiles = 0: scales [rows, K/32] row-major;
+// row_tiles = rows / 128: packed layout
+__device__ __forceinline__ void quantize_block(long long b, const __nv_bfloat16 *__restrict__ src,
+                                               uint8_t *__restrict__ q, uint8_t *__restrict__ scales, long long kb32,
+                                               long long row_tiles)
 {
-    const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (b >= nblocks) return;
     const uint4 *p = reinterpret_cast<const uint4 *>(src + b * 32);
     float v[32];
 #pragma unroll
@@ -80,6 +78,15 @@ __global__ void __launch_bounds__(256) quantize_mxfp8_kernel(const __nv_bfloat16
     dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     const long long at = row_tiles ? packed_scale_offset(b / kb32, b % kb32, row_tiles) : b;
     scales[at] = static_cast<uint8_t>(e + 127);
+}
+
+__global__ void __launch_bounds__(256) quantize_mxfp8_kernel(const __nv_bfloat16 *__restrict__ src,
+                                                             long long nblocks, uint8_t *__restrict__ q,
+                                                             uint8_t *__restrict__ scales, long long kb32,
+                                                             long long row_tiles)
+{
+    const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (b < nblocks) quantize_block(b, src, q, scales, kb32, row_tiles);
 }
 
 }  // namespace mok

@@ -19,16 +19,9 @@ namespace mok {
 // contraction of x (bf16, exact) with the three terms reproduces the fp32
 // router logits.  Each difference below is exact in fp32.
 // It also writes the one-group row range {0, T} the router contraction reads.
-__global__ void __launch_bounds__(256) router_split_kernel(const float *__restrict__ Wr,
-                                                           __nv_bfloat16 *__restrict__ Wr3, int E, int H,
-                                                           int *__restrict__ all_rows, int T)
+__device__ __forceinline__ void router_split_elem(long long i, const float *__restrict__ Wr,
+                                                  __nv_bfloat16 *__restrict__ Wr3, int H)
 {
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i == 0) {
-        all_rows[0] = 0;
-        all_rows[1] = T;
-    }
-    if (i >= (long long)E * H) return;
     const int e = (int)(i / H), h = (int)(i % H);
     const float w = Wr[i];
     const __nv_bfloat16 hi = __float2bfloat16_rn(w);
@@ -42,6 +35,18 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float *__restri
     row[2 * H + h] = lo;
 }
 
+__global__ void __launch_bounds__(256) router_split_kernel(const float *__restrict__ Wr,
+                                                           __nv_bfloat16 *__restrict__ Wr3, int E, int H,
+                                                           int *__restrict__ all_rows, int T)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i == 0) {
+        all_rows[0] = 0;
+        all_rows[1] = T;
+    }
+    if (i < (long long)E * H) router_split_elem(i, Wr, Wr3, H);
+}
+
 struct SelectArgs {
     const float *partial;       // [n_split, T, 256] partial logits (tensor-core K splits)
     int n_split;
@@ -53,7 +58,11 @@ struct SelectArgs {
     int *topk_idx;              // [T, k]
     float *topk_w;              // [T, k]
     float *topk_p;              // [T, k] sigmoid score s (sigmoid) or w / routed_scale (softmax)
+    int *hist;                  // null, or [chunks of kDispatchChunk tokens, E] counts, zero
+                                // before: the selection also counts each (token, slot) there
 };
+
+constexpr int kDispatchChunk = 1024;   // tokens per dispatch chunk
 
 // one (value, index) candidate; larger value wins, then lower index
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib)
@@ -183,6 +192,7 @@ __device__ __forceinline__ void select_token(const SelectArgs &a, int t, int lan
             a.topk_idx[(size_t)t * a.k + j] = my_idx[j];
             a.topk_w[(size_t)t * a.k + j] = a.routed_scale * q;
             a.topk_p[(size_t)t * a.k + j] = a.score_fn == 0 ? q : my_val[j];
+            if (a.hist) atomicAdd(&a.hist[(size_t)(t / kDispatchChunk) * E + my_idx[j]], 1);
         }
     }
 }
@@ -226,8 +236,6 @@ __device__ __forceinline__ int checked_expert(int e, int E, int *status)
     atomicOr(status, kStatusBadIndex);
     return 0;
 }
-
-constexpr int kDispatchChunk = 1024;   // tokens per chunk (one block of 1024 threads)
 
 // Integer counting sort of the T*k (token, slot) pairs by expert, stable in
 // token order, in three launches: per-chunk histograms, a per-expert scan over
@@ -290,6 +298,92 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
         }
         a.gorder[rank] = g;
     }
+}
+
+// The scan and the placement of one chunk in one CTA (any block size >= 256),
+// for the persistent forward: every CTA that owns a chunk derives its own base
+// rows from the per-chunk counts (exclusive offsets over experts plus the
+// counts of the earlier chunks), so no grid-wide step sits between the scan
+// and the placement; CTA `writer` also writes counts, offsets, the
+// router-gradient chunk starts and the group order.  The placement is the one
+// of dispatch_place_kernel below, with the token of a thread strided by the
+// block size.  s_mask: [256][32] words, s_base / s_cnt: 256 ints each.
+__device__ __forceinline__ void dispatch_scan_place_chunk(const DispatchArgs &a, int c, int n_chunks, bool writer,
+                                                          uint32_t (*s_mask)[32], int *s_base, int *s_cnt)
+{
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int E = a.E, k = a.k, kk = a.k + a.S, T = a.T;
+    for (int q = tid; q < E * 32; q += nthr) (&s_mask[0][0])[q] = 0u;
+    if (tid < E) {
+        int total = 0, before = 0;
+        for (int cc = 0; cc < n_chunks; ++cc) {
+            const int h = a.hist[(size_t)cc * E + tid];
+            if (cc < c) before += h;
+            total += h;
+        }
+        s_cnt[tid] = total;
+        s_base[tid] = before;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int acc = 0, cacc = 0;
+        for (int q = 0; q < E; ++q) {
+            const int cnt = s_cnt[q];
+            s_base[q] += acc;
+            if (writer) {
+                a.counts[q] = cnt;
+                a.offsets[q] = acc;
+                a.chunk_start[q] = cacc;
+            }
+            acc += cnt;
+            cacc += (cnt + a.chunk_rows - 1) / a.chunk_rows;
+        }
+        if (writer) {
+            a.chunk_start[E] = cacc;
+            for (int s2 = 0; s2 <= a.S; ++s2) a.offsets[E + s2] = acc + s2 * T;
+        }
+    }
+    if (writer) {
+        for (int g = tid; g < E + a.S; g += nthr) {
+            const int cg = g < E ? s_cnt[g] : T;
+            int rank = 0;
+            for (int h = 0; h < E + a.S; ++h) {
+                const int ch = h < E ? s_cnt[h] : T;
+                rank += (ch > cg) || (ch == cg && h < g);
+            }
+            a.gorder[rank] = g;
+        }
+    }
+    __syncthreads();
+    const int t0 = c * kDispatchChunk;
+    const int nt = min(kDispatchChunk, T - t0);
+    for (int l = tid; l < nt; l += nthr)
+        for (int j = 0; j < k; ++j)
+            atomicOr(&s_mask[checked_expert(a.topk_idx[(size_t)(t0 + l) * k + j], E, a.status)][l >> 5], 1u << (l & 31));
+    __syncthreads();
+    for (int l = tid; l < nt; l += nthr) {
+        const int t = t0 + l, word = l >> 5, bit = l & 31;
+        for (int j = 0; j < k; ++j) {
+            const int e = checked_expert(a.topk_idx[(size_t)t * k + j], E, a.status);
+            int rank = __popc(s_mask[e][word] & ((1u << bit) - 1u));
+            for (int w = 0; w < word; ++w) rank += __popc(s_mask[e][w]);
+            const int pos = s_base[e] + rank;
+            const int sl = t * k + j;
+            a.perm[pos] = sl;
+            a.inv_perm[sl] = pos;
+            a.row_token[pos] = t;
+            a.row_slot[pos] = t * kk + j;
+            a.row_w[pos] = a.topk_w[sl];
+        }
+        const long long TK = (long long)T * k;
+        for (int s2 = 0; s2 < a.S; ++s2) {
+            const long long pos = TK + (long long)s2 * T + t;
+            a.row_token[pos] = t;
+            a.row_slot[pos] = t * kk + k + s2;
+            a.row_w[pos] = 1.0f;
+        }
+    }
+    __syncthreads();
 }
 
 // Per chunk: per-expert token bitmasks give each (token, slot) its rank among
