@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="dsv3")
     ap.add_argument("--impl", default="mok", choices=["mok", "reference"])
+    ap.add_argument("--schedule", default="persistent", choices=["persistent", "split"],
+                    help="forward schedule of the timed steps (the A/B leg runs both)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -221,6 +223,7 @@ def forward_ab(layer, x, y, K):
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     mk = lambda: torch.cuda.Event(enable_timing=True)
     out = {}
+    restore = abi.moe_get_schedule()
     for name, sched in (("split", abi.MOK_SCHEDULE_SPLIT), ("persistent", abi.MOK_SCHEDULE_PERSISTENT)):
         abi.moe_set_schedule(sched)
         for _ in range(2):
@@ -248,7 +251,7 @@ def forward_ab(layer, x, y, K):
         else:
             r["device_phases_ms"] = stamp_phases(bufs, sms)
         out[name] = r
-    abi.moe_set_schedule(abi.MOK_SCHEDULE_PERSISTENT)
+    abi.moe_set_schedule(restore)
     out["persistent_over_split_speedup"] = out["split"]["ms_per_fwd"] / out["persistent"]["ms_per_fwd"]
     return out
 
@@ -326,6 +329,8 @@ def main():
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    sched = abi.MOK_SCHEDULE_SPLIT if args.schedule == "split" else abi.MOK_SCHEDULE_PERSISTENT
+    abi.moe_set_schedule(sched)
     wl = synth.WORKLOADS[args.workload]
     wl = synth.scaled(wl, seed=wl.seed + 1000 * rank)
     params = synth.draw_params(wl, dev)
@@ -387,12 +392,13 @@ def main():
 
     # the forward is one persistent launch (events around it); the backward's steps are
     # separate launches with an event each
-    phase = {"fwd_persistent": statistics.mean(fev[i][0].elapsed_time(fev[i][-1]) for i in range(K))}
+    fwd_name = "fwd_persistent" if sched == abi.MOK_SCHEDULE_PERSISTENT else "fwd_split"
+    phase = {fwd_name: statistics.mean(fev[i][0].elapsed_time(fev[i][-1]) for i in range(K))}
     for n_i, name in enumerate(BWD_PHASES):
         phase[name] = statistics.mean(bev[i][n_i].elapsed_time(bev[i][n_i + 1]) for i in range(K))
-    fwd_ms = phase["fwd_persistent"]
+    fwd_ms = phase[fwd_name]
     bwd_ms = sum(phase[n] for n in BWD_PHASES)
-    fwd_device_phases = stamp_phases(stamps, sms)
+    fwd_device_phases = stamp_phases(stamps, sms) if sched == abi.MOK_SCHEDULE_PERSISTENT else None
 
     # forward A/B: split schedule (events per step, the per-GEMM attribution below) against
     # the persistent one, forward only
@@ -402,7 +408,7 @@ def main():
 
     pk = peaks()
     alg = algorithmic(wl, counts)
-    kern = {"fwd_persistent": forward_algorithmic(wl, counts)}
+    kern = {fwd_name: forward_algorithmic(wl, counts)}
     kern.update({n: alg[n] for n in alg if n in phase})
     dom = max(kern, key=lambda n: phase[n])
     flops, nbytes = kern[dom]
@@ -422,7 +428,7 @@ def main():
     roof["algorithmic_bytes"] = nbytes
     # every GEMM phase against both measured peaks (algorithmic bytes and FLOPs / its event time)
     phase_roofline = {}
-    for name, (fl, nb) in list(alg.items()) + [("fwd_persistent", kern["fwd_persistent"])]:
+    for name, (fl, nb) in list(alg.items()) + [(fwd_name, kern[fwd_name])]:
         t = (phase[name] if name in phase else phase["split_" + name]) / 1e3
         phase_roofline[name] = {"ms": round(phase[name], 4), "hbm_frac": round(nb / t / 1e9 / pk["hbm_gbs"], 4),
                                 "tc_frac_sustained": round(fl / t / 1e12 / pk["bf16_sustained"], 4)}
@@ -468,6 +474,7 @@ def main():
                                       if wl.score_fn else "softmax routing")
                                    + (f", Zipf({wl.zipf}) logit term" if wl.zipf else ""),
                        "tokens_per_gpu": wl.T, "parallelism": f"replicas x{world}",
+                       "forward_schedule": args.schedule,
                        "l2": "inputs larger than L2 (22.6 GB expert weights streamed per pass)"},
             # forward: one persistent kernel; backward: down dgrad, slot grad, 2 router-gradient
             # kernels, 4 GEMMs plus the resident weight-gradient kernels, dx sum (10)
