@@ -287,21 +287,28 @@ int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, 
 int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_t *offset, size_t *bytes);
 
 /*
- * Schedule of the forward pass (per host thread; default PERSISTENT).
+ * Schedule of the passes (per host thread; default PERSISTENT).
  *   MOK_SCHEDULE_PERSISTENT  the whole forward is one cooperative launch of one
  *       persistent kernel, one CTA per SM: router, top-k, dispatch, the two
  *       expert GEMMs and the combine are phases separated by grid barriers,
  *       except that the down GEMM starts an M tile as soon as every gate/up tile
  *       of its rows is in memory (per-tile readiness counters) -- the fusion of
  *       the layer into one kernel that "Cursor åpner megakernelen…" (the quoted
- *       paragraph) describes.  No memset or other launch precedes it.
+ *       paragraph) describes.  No memset or other launch precedes it.  The
+ *       backward runs split with programmatic dependent launch.
  *   MOK_SCHEDULE_SPLIT  one launch per step in stream order (router split,
  *       router GEMM, select, three dispatch kernels, [MXFP8: quantise x], gate/up,
- *       down, combine) after a memset of the tile counters: the comparison point.
- * Both schedules give byte-identical results.  The backward is always split.
+ *       down, combine) after a memset of the tile counters; the backward the same.
+ *   MOK_SCHEDULE_SPLIT_PDL  the split launches with programmatic dependent
+ *       launch: each launch's CTAs are placed as soon as the previous launch's
+ *       CTAs leave their SMs and wait on the device for its completion (the
+ *       kernel-boundary alternative to one fused kernel that "Megakernels are
+ *       dead and back…", the case against megakernels, argues for).
+ * All schedules give byte-identical results.
  */
 #define MOK_SCHEDULE_PERSISTENT 0
 #define MOK_SCHEDULE_SPLIT 1
+#define MOK_SCHEDULE_SPLIT_PDL 2
 int moe_set_schedule(int schedule);
 int moe_get_schedule(int *schedule);
 

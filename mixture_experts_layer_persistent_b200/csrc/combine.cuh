@@ -62,6 +62,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const Slot *__restrict__ O
                                                       const float *__restrict__ topk_w,
                                                       __nv_bfloat16 *__restrict__ y, int T, int H, int k, int S)
 {
+    griddep_enter();
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < (long long)T * (H / 8)) combine_elem(i, O, topk_w, y, H, k, S);
 }
@@ -79,6 +80,7 @@ __global__ void __launch_bounds__(256) slot_grad_kernel(const float *__restrict_
                                                         const float *__restrict__ topk_p, float *__restrict__ dl,
                                                         int T, int k, int score_fn, float routed_scale)
 {
+    griddep_enter();
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= T) return;
     float G[16], q[16];
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat1
                                                               float *__restrict__ partial, int H, int E, int k,
                                                               int chunk_rows)
 {
+    griddep_enter();
     __shared__ float s_acc[8][256];
     const int chunk = blockIdx.x;
     const int h0 = blockIdx.y * 256;
@@ -152,6 +155,7 @@ __global__ void __launch_bounds__(256) drouter_reduce_kernel(const float *__rest
                                                              const int *__restrict__ chunk_start,
                                                              float *__restrict__ dWr, int H, int E)
 {
+    griddep_enter();
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (long long)E * H) return;
     const int e = (int)(i / H), h = (int)(i % H);
@@ -168,6 +172,7 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *__restrict
                                                          const float *__restrict__ router_w,
                                                          __nv_bfloat16 *__restrict__ dx, int T, int H, int k, int S)
 {
+    griddep_enter();
     const int cpr = H / 8;
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= (long long)T * cpr) return;

@@ -64,6 +64,7 @@ thread_local int t_schedule = MOK_SCHEDULE_PERSISTENT;   // moe_set_schedule
 thread_local unsigned long long *t_dev_trace = nullptr;   // moe_trace_device
 thread_local size_t t_dev_trace_bytes = 0;
 thread_local int t_launches = 0;        // kernels launched by the current / last forward or backward
+thread_local bool t_pdl = false;        // launches of the current pass use programmatic dependent launch
 
 inline int mark_fwd(int i, cudaStream_t s)
 {
@@ -287,6 +288,31 @@ int check_cfg(const moe_cfg *c)
     return MOK_OK;
 }
 
+// One kernel launch on the pass's stream, with the programmatic stream
+// serialisation attribute when the pass runs with PDL (the kernels begin with
+// griddep_enter, so the attribute only lets a launch's CTAs start early).
+template <typename... KArgs, typename... Args>
+int launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, const char *what,
+             Args &&...args)
+{
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (t_pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 1;
+    }
+    const cudaError_t e = cudaLaunchKernelEx(&lc, kern, std::forward<Args>(args)...);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, what, e);
+    ++t_launches;
+    return MOK_OK;
+}
+
 // Operand maps a, b, bs (B of the shared groups) and output maps o, o2, o3.
 template <class C>
 int launch_wgrad_resident(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &o, const CUtensorMap &o2,
@@ -296,11 +322,8 @@ int launch_wgrad_resident(const CUtensorMap &a, const CUtensorMap &b, const CUte
     cudaError_t e = cudaFuncSetAttribute(wgrad_resident_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(wgrad_resident_kernel)", e);
-    wgrad_resident_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, o, o2, args);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "wgrad_resident_kernel launch", e);
-    ++t_launches;
-    return MOK_OK;
+    return launch_k(wgrad_resident_kernel<C>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st,
+                    "wgrad_resident_kernel launch", a, b, o, o2, args);
 }
 
 // M tiles per resident work unit: runs of at most 16, split evenly
@@ -319,11 +342,8 @@ int launch_gemm(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &b
     cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(grouped_gemm_kernel)", e);
-    grouped_gemm_kernel<C><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, bs, o, o2, o3, args);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "grouped_gemm_kernel launch", e);
-    ++t_launches;
-    return MOK_OK;
+    return launch_k(grouped_gemm_kernel<C>, dim3(grid), dim3(C::THREADS), C::SMEM_BYTES, st,
+                    "grouped_gemm_kernel launch", a, b, bs, o, o2, o3, args);
 }
 
 inline int blocks_for(long long n, int per) { return static_cast<int>((n + per - 1) / per); }
@@ -513,30 +533,24 @@ int forward_split(const moe_cfg &c, const void *x, const moe_params &p, void *y,
     if (const cudaError_t e = cudaMemsetAsync(st.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
     MOK_TRY(mark_fwd(0, stream));
-    router_split_kernel<<<blocks_for(s.E * s.H, 256), 256, 0, stream>>>(p.router_w, st.wr3, c.E, c.H, st.all_rows,
-                                                                         c.T);
-    MOK_LAUNCHED();
+    MOK_TRY(launch_k(router_split_kernel, dim3(blocks_for(s.E * s.H, 256)), dim3(256), 0, stream, "router_split_kernel",
+                     p.router_w, st.wr3, c.E, c.H, st.all_rows, c.T));
     MOK_TRY(launch_gemm<typename FusedCfg<false>::Router>(pl.m.rA, pl.m.rB, pl.m.rB, pl.m.rO, pl.m.rO, pl.m.rO, pl.gr,
                                                          dev.sms, stream));
-    router_select_kernel<<<blocks_for(s.T, 8), 256, 0, stream>>>(pl.sa);
-    MOK_LAUNCHED();
+    MOK_TRY(launch_k(router_select_kernel, dim3(blocks_for(s.T, 8)), dim3(256), 0, stream, "router_select_kernel", pl.sa));
 
     MOK_TRY(mark_fwd(1, stream));
-    dispatch_count_kernel<<<pl.n_chunks, 1024, 0, stream>>>(pl.da);
-    MOK_LAUNCHED();
-    dispatch_scan_kernel<<<1, 256, 0, stream>>>(pl.da, pl.n_chunks);
-    MOK_LAUNCHED();
-    dispatch_place_kernel<<<pl.n_chunks, 1024, 0, stream>>>(pl.da);
-    MOK_LAUNCHED();
+    MOK_TRY(launch_k(dispatch_count_kernel, dim3(pl.n_chunks), dim3(1024), 0, stream, "dispatch_count_kernel", pl.da));
+    MOK_TRY(launch_k(dispatch_scan_kernel, dim3(1), dim3(256), 0, stream, "dispatch_scan_kernel", pl.da, pl.n_chunks));
+    MOK_TRY(launch_k(dispatch_place_kernel, dim3(pl.n_chunks), dim3(1024), 0, stream, "dispatch_place_kernel", pl.da));
 
     MOK_TRY(mark_fwd(2, stream));
     GemmArgs ga = pl.ga, gd = pl.gd;
     ga.ready_role = gd.ready_role = kReadyNone;
     if (mx) {
         const long long xb = s.T * s.H / 32;
-        quantize_mxfp8_kernel<<<blocks_for(xb, 256), 256, 0, stream>>>(static_cast<const __nv_bfloat16 *>(x), xb,
-                                                                        st.xq, st.xs, s.H / 32, 0);
-        MOK_LAUNCHED();
+        MOK_TRY(launch_k(quantize_mxfp8_kernel, dim3(blocks_for(xb, 256)), dim3(256), 0, stream, "quantize_mxfp8_kernel",
+                         static_cast<const __nv_bfloat16 *>(x), xb, st.xq, st.xs, static_cast<long long>(s.H / 32), 0ll));
         MOK_TRY(launch_gemm<typename FusedCfg<true>::GateUp>(pl.m.gB, pl.m.gB, pl.m.gBs, pl.m.gO, pl.m.gO2, pl.m.gO3,
                                                             ga, dev.sms, stream));
         MOK_TRY(mark_fwd(3, stream));
@@ -552,13 +566,14 @@ int forward_split(const moe_cfg &c, const void *x, const moe_params &p, void *y,
 
     MOK_TRY(mark_fwd(4, stream));
     if (mx)
-        combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(
-            reinterpret_cast<const __nv_bfloat16 *>(st.O), st.topk_w, static_cast<__nv_bfloat16 *>(y), c.T, c.H,
-            c.top_k, c.n_shared);
+        MOK_TRY(launch_k(combine_kernel<__nv_bfloat16>, dim3(blocks_for(s.T * s.H / 8, 256)), dim3(256), 0, stream,
+                         "combine_kernel", reinterpret_cast<const __nv_bfloat16 *>(st.O),
+                         static_cast<const float *>(st.topk_w), static_cast<__nv_bfloat16 *>(y), c.T, c.H, c.top_k,
+                         c.n_shared));
     else
-        combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(
-            st.O, st.topk_w, static_cast<__nv_bfloat16 *>(y), c.T, c.H, c.top_k, c.n_shared);
-    MOK_LAUNCHED();
+        MOK_TRY(launch_k(combine_kernel<float>, dim3(blocks_for(s.T * s.H / 8, 256)), dim3(256), 0, stream,
+                         "combine_kernel", static_cast<const float *>(st.O), static_cast<const float *>(st.topk_w),
+                         static_cast<__nv_bfloat16 *>(y), c.T, c.H, c.top_k, c.n_shared));
     return mark_fwd(5, stream);
 }
 
@@ -628,7 +643,8 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
     FwdPlan pl;
     MOK_TRY(build_fwd_plan(c, x, p, st, dev, training, pl));
     const bool mx = c.dtype == MOK_DTYPE_MXFP8;
-    if (t_schedule == MOK_SCHEDULE_SPLIT) {
+    t_pdl = t_schedule == MOK_SCHEDULE_SPLIT_PDL;
+    if (t_schedule == MOK_SCHEDULE_SPLIT || t_schedule == MOK_SCHEDULE_SPLIT_PDL) {
         MOK_TRY(forward_split(c, x, p, y, st, dev, pl, stream));
     } else if (mx) {
         MOK_TRY(launch_fused<true>(c, x, p, y, st, dev, pl, stream));
@@ -644,6 +660,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
 {
     const Shapes s = shapes(c);
     t_launches = 0;
+    t_pdl = t_schedule != MOK_SCHEDULE_SPLIT;       // the backward is split; PDL unless plain split is asked
     const __nv_bfloat16 *dyb = static_cast<const __nv_bfloat16 *>(dy);
     if (const cudaError_t e = cudaMemsetAsync(bs.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
@@ -687,19 +704,19 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
 
     // slot gradients from the down dgrad's partials, then the router weight gradient
     MOK_TRY(mark_bwd(1, stream));
-    slot_grad_kernel<<<blocks_for(s.T, 256), 256, 0, stream>>>(bs.gpart, g1.n_tiles, st.inv_perm, st.topk_w,
-                                                              st.topk_p, bs.dl, c.T, c.top_k, c.score_fn,
-                                                              c.routed_scale);
-    MOK_LAUNCHED();
+    MOK_TRY(launch_k(slot_grad_kernel, dim3(blocks_for(s.T, 256)), dim3(256), 0, stream, "slot_grad_kernel",
+                     static_cast<const float *>(bs.gpart), g1.n_tiles, static_cast<const int *>(st.inv_perm),
+                     static_cast<const float *>(st.topk_w), static_cast<const float *>(st.topk_p), bs.dl, c.T,
+                     c.top_k, c.score_fn, c.routed_scale));
     MOK_TRY(mark_bwd(2, stream));
-    drouter_partial_kernel<<<dim3(static_cast<unsigned>(s.max_chunks), c.H / 256), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(x), bs.dl, st.offsets, st.chunk_start, st.perm, bs.partial, c.H, c.E,
-        c.top_k, kChunkRows);
-    MOK_LAUNCHED();
+    MOK_TRY(launch_k(drouter_partial_kernel, dim3(static_cast<unsigned>(s.max_chunks), c.H / 256), dim3(256), 0, stream,
+                     "drouter_partial_kernel", static_cast<const __nv_bfloat16 *>(x), static_cast<const float *>(bs.dl),
+                     static_cast<const int *>(st.offsets), static_cast<const int *>(st.chunk_start),
+                     static_cast<const int *>(st.perm), bs.partial, c.H, c.E, c.top_k, kChunkRows));
     MOK_TRY(mark_bwd(3, stream));
-    drouter_reduce_kernel<<<blocks_for(s.E * s.H, 256), 256, 0, stream>>>(bs.partial, st.chunk_start,
-                                                                          gr.drouter_w, c.H, c.E);
-    MOK_LAUNCHED();
+    MOK_TRY(launch_k(drouter_reduce_kernel, dim3(blocks_for(s.E * s.H, 256)), dim3(256), 0, stream,
+                     "drouter_reduce_kernel", static_cast<const float *>(bs.partial),
+                     static_cast<const int *>(st.chunk_start), gr.drouter_w, c.H, c.E));
 
     // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
     GemmArgs g2 = base;
@@ -778,10 +795,10 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
                                                       stream));
 
     MOK_TRY(mark_bwd(7, stream));
-    dx_combine_kernel<<<blocks_for(s.T * s.H / 8, 256), 256, 0, stream>>>(
-        bs.dxs, bs.dl, st.topk_idx, p.router_w, static_cast<__nv_bfloat16 *>(gr.dx), c.T, c.H, c.top_k,
-        c.n_shared);
-    MOK_LAUNCHED();
+    MOK_TRY(launch_k(dx_combine_kernel, dim3(blocks_for(s.T * s.H / 8, 256)), dim3(256), 0, stream,
+                     "dx_combine_kernel", static_cast<const float *>(bs.dxs), static_cast<const float *>(bs.dl),
+                     static_cast<const int *>(st.topk_idx), p.router_w, static_cast<__nv_bfloat16 *>(gr.dx), c.T, c.H,
+                     c.top_k, c.n_shared));
     MOK_TRY(mark_bwd(8, stream));
     return MOK_OK;
 }
@@ -1028,7 +1045,8 @@ int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_
 
 int moe_set_schedule(int schedule)
 {
-    if (schedule != MOK_SCHEDULE_PERSISTENT && schedule != MOK_SCHEDULE_SPLIT) return MOK_ERR_INVALID;
+    if (schedule != MOK_SCHEDULE_PERSISTENT && schedule != MOK_SCHEDULE_SPLIT && schedule != MOK_SCHEDULE_SPLIT_PDL)
+        return MOK_ERR_INVALID;
     t_schedule = schedule;
     return MOK_OK;
 }

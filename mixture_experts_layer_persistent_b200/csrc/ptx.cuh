@@ -98,6 +98,20 @@ __device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity)
 // Wait until every cp.async this thread issued has completed.
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Every kernel of the split schedules starts with these two: wait until the
+// grids this launch depends on have completed and their writes are visible,
+// then let the next launch in the stream place its CTAs as soon as SMs free up
+// (they wait here in turn).  Both are no-ops in a launch without the
+// programmatic stream serialisation attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void griddep_enter()
+{
+    griddep_wait();
+    griddep_launch_dependents();
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *tm)
 {

@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(256) quantize_mxfp8_kernel(const __nv_bfloat16
                                                              uint8_t *__restrict__ scales, long long kb32,
                                                              long long row_tiles)
 {
+    griddep_enter();
     const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (b < nblocks) quantize_block(b, src, q, scales, kb32, row_tiles);
 }

@@ -39,6 +39,7 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float *__restri
                                                            __nv_bfloat16 *__restrict__ Wr3, int E, int H,
                                                            int *__restrict__ all_rows, int T)
 {
+    griddep_enter();
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i == 0) {
         all_rows[0] = 0;
@@ -200,6 +201,7 @@ __device__ __forceinline__ void select_token(const SelectArgs &a, int t, int lan
 // One warp per token.
 __global__ void __launch_bounds__(256) router_select_kernel(const SelectArgs a)
 {
+    griddep_enter();
     __shared__ float s_row[8][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t = blockIdx.x * 8 + warp;
@@ -243,6 +245,7 @@ __device__ __forceinline__ int checked_expert(int e, int E, int *status)
 // the result is the same whatever the order of the atomics.
 __global__ void __launch_bounds__(1024) dispatch_count_kernel(const DispatchArgs a)
 {
+    griddep_enter();
     __shared__ int s_cnt[256];
     const int c = blockIdx.x, tid = threadIdx.x;
     for (int e = tid; e < a.E; e += 1024) s_cnt[e] = 0;
@@ -258,6 +261,7 @@ __global__ void __launch_bounds__(1024) dispatch_count_kernel(const DispatchArgs
 // place of its histogram), router-gradient chunk starts and the group order.
 __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a, int n_chunks)
 {
+    griddep_enter();
     __shared__ int s_cnt[256];
     __shared__ int s_off[257];
     const int e = threadIdx.x, E = a.E, T = a.T;
@@ -390,6 +394,7 @@ __device__ __forceinline__ void dispatch_scan_place_chunk(const DispatchArgs &a,
 // the chunk's earlier tokens of that expert; row = chunk base + rank.
 __global__ void __launch_bounds__(1024) dispatch_place_kernel(const DispatchArgs a)
 {
+    griddep_enter();
     __shared__ uint32_t s_mask[256][32];
     const int c = blockIdx.x, tid = threadIdx.x;
     const int E = a.E, k = a.k, kk = a.k + a.S, T = a.T;

@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                           const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                           const GemmArgs args)
 {
+    griddep_enter();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sB = smem;                                        // resident B: KB_MAX blocks

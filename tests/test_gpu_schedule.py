@@ -1,5 +1,8 @@
 """The persistent (one-launch) forward against the split (one launch per step) forward.
 
+The split schedule also runs with programmatic dependent launch (PDL); the
+backward after a persistent forward uses PDL, after a split forward it does not.
+
 Both schedules run the same device code with the same fixed reduction orders,
 so every output and every saved tensor must agree byte for byte: y, the routing
 record, the saved h / g,u / w*h (or the MXFP8 h codes and scales), and the
@@ -84,7 +87,18 @@ def test_persistent_forward_equals_split_forward(wl):
     g_s = None
     if training:
         dy = synth.draw_dy(wl, "cpu").to(dev)
-        g_s = {k: v.clone() for k, v in layer.backward(x, dy).items() if v is not None}
+        abi.moe_set_schedule(abi.MOK_SCHEDULE_SPLIT)          # plain launches, no PDL
+        try:
+            g_s = {k: v.clone() for k, v in layer.backward(x, dy).items() if v is not None}
+            torch.cuda.synchronize()
+        finally:
+            abi.moe_set_schedule(abi.MOK_SCHEDULE_PERSISTENT)
+    # the split launches with programmatic dependent launch: the same bytes
+    y_d, r_d, n_d = _forward(layer, x, abi.MOK_SCHEDULE_SPLIT_PDL)
+    assert n_d == n_s
+    assert _same(y_d, y_s), "y differs between the split and the PDL-split schedules"
+    for k in r_s:
+        assert _same(r_d[k], r_s[k]), k
     y_p, r_p, n_p = _forward(layer, x, abi.MOK_SCHEDULE_PERSISTENT)
     assert n_p == 1, n_p
     assert n_s >= 9, n_s
@@ -94,7 +108,7 @@ def test_persistent_forward_equals_split_forward(wl):
     for k, v in _saved(layer, wl.mxfp8).items():
         assert _same(v, saved_s[k]), f"saved tensor {k} differs"
     if training:
-        g_p = layer.backward(x, dy)
+        g_p = layer.backward(x, dy)        # persistent schedule: the backward's launches use PDL
         torch.cuda.synchronize()
         for k, v in g_s.items():
             assert _same(g_p[k], v), f"gradient {k} differs"
