@@ -224,7 +224,8 @@ def forward_ab(layer, x, y, K):
     mk = lambda: torch.cuda.Event(enable_timing=True)
     out = {}
     restore = abi.moe_get_schedule()
-    for name, sched in (("split", abi.MOK_SCHEDULE_SPLIT), ("persistent", abi.MOK_SCHEDULE_PERSISTENT)):
+    for name, sched in (("split", abi.MOK_SCHEDULE_SPLIT), ("split_pdl", abi.MOK_SCHEDULE_SPLIT_PDL),
+                        ("persistent", abi.MOK_SCHEDULE_PERSISTENT)):
         abi.moe_set_schedule(sched)
         for _ in range(2):
             layer.forward(x, y)
@@ -236,7 +237,8 @@ def forward_ab(layer, x, y, K):
         s, e = mk(), mk()
         s.record()
         for i in range(K):
-            moe_trace_events([ev.cuda_event for ev in fev[i]], None)
+            if name == "split":          # events between the steps (they would cut the PDL overlap)
+                moe_trace_events([ev.cuda_event for ev in fev[i]], None)
             abi.moe_trace_device(bufs[i].data_ptr(), bufs[i].numel() * 8)
             layer.forward(x, y)
             launches = abi.moe_launch_count()
@@ -248,11 +250,35 @@ def forward_ab(layer, x, y, K):
         if name == "split":
             r["phases_ms"] = {n: round(statistics.mean(fev[i][j].elapsed_time(fev[i][j + 1]) for i in range(K)), 4)
                               for j, n in enumerate(FWD_PHASES)}
-        else:
+        elif name == "persistent":
             r["device_phases_ms"] = stamp_phases(bufs, sms)
         out[name] = r
     abi.moe_set_schedule(restore)
     out["persistent_over_split_speedup"] = out["split"]["ms_per_fwd"] / out["persistent"]["ms_per_fwd"]
+    out["persistent_over_split_pdl_speedup"] = out["split_pdl"]["ms_per_fwd"] / out["persistent"]["ms_per_fwd"]
+    return out
+
+
+def backward_ab(layer, x, dy, grads, K):
+    """Backward only, K steps each: plain split launches against PDL launches."""
+    import torch
+    from mixture_experts_layer_persistent_b200 import abi
+    restore = abi.moe_get_schedule()
+    out = {}
+    for name, sched in (("split", abi.MOK_SCHEDULE_SPLIT), ("split_pdl", abi.MOK_SCHEDULE_SPLIT_PDL)):
+        abi.moe_set_schedule(sched)
+        for _ in range(2):
+            layer.backward(x, dy, grads)
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(K):
+            layer.backward(x, dy, grads)
+        e.record()
+        torch.cuda.synchronize()
+        out[name] = {"ms_per_bwd": s.elapsed_time(e) / K, "launches_per_bwd": abi.moe_launch_count()}
+    abi.moe_set_schedule(restore)
+    out["pdl_speedup"] = out["split"]["ms_per_bwd"] / out["split_pdl"]["ms_per_bwd"]
     return out
 
 
@@ -405,6 +431,8 @@ def main():
     ab = forward_ab(layer, x, y, K)
     for n_i, name in enumerate(FWD_PHASES):
         phase["split_" + name] = ab["split"]["phases_ms"][name]
+    layer.forward(x, y)
+    bab = backward_ab(layer, x, dy, grads, K)
 
     pk = peaks()
     alg = algorithmic(wl, counts)
@@ -483,6 +511,7 @@ def main():
             "phases_ms": {k2: round(v, 4) for k2, v in phase.items()},
             "fwd_device_phases_ms": fwd_device_phases,
             "forward_schedule_ab": ab,
+            "backward_schedule_ab": bab,
             "breakdown": {
                 "fwd_bf16_tokens_per_s": fwd_tps, "bwd_bf16_tokens_per_s": bwd_tps,
                 "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
