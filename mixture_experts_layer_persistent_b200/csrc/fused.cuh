@@ -18,7 +18,8 @@
 //       in its dispatch chunk's histogram (integer atomics)
 //   --- grid barrier
 //   P3  per dispatch chunk: scan of the histograms and stable placement of the
-//       chunk's (token, slot) rows (every CTA derives its own chunk's base rows)
+//       chunk's (token, slot) rows (every CTA derives its own chunk's base rows);
+//       MXFP8: then (after a grid barrier) x's scales packed per M tile
 //   --- grid barrier
 //   P4  gate/up GEMM with the SwiGLU epilogue, then the down GEMM with the push
 //       epilogue.  No barrier between them: each gate/up epilogue warp counts
@@ -222,14 +223,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (long long b = gtid; b < nb; b += gstride) quantize_block(b, a.x, a.xq, a.xs, a.H / 32, 0);
     }
     fused_stamp(a, 1);
-    bool alive = grid_sync(a.gs, epoch, 0, true, a.status, s_flag);
+    int nb = 0;                                      // barriers passed
+    bool alive = grid_sync(a.gs, epoch, nb++, true, a.status, s_flag);
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.gs.epoch = (epoch + 1) & kEpochMask;   // every CTA has read it
 
     // ---------------------------------------------------------------- P1
     if (alive)
         gemm_phase<typename F::Router>(smem, bars, aux, tmem_base, m.rA, m.rB, m.rB, m.rO, m.rO, m.rO, a.gr);
     fused_stamp(a, 2);
-    alive = grid_sync(a.gs, epoch, 1, alive, a.status, s_flag);
+    alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
 
     // ---------------------------------------------------------------- P2
     if (alive) {
@@ -238,7 +240,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int t = blockIdx.x * nw + warp; t < a.T; t += gridDim.x * nw) select_token(a.sa, t, lane, row);
     }
     fused_stamp(a, 3);
-    alive = grid_sync(a.gs, epoch, 2, alive, a.status, s_flag);
+    alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
 
     // ---------------------------------------------------------------- P3
     if (alive) {
@@ -248,8 +250,22 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (int c = blockIdx.x; c < a.n_chunks; c += gridDim.x)
             dispatch_scan_place_chunk(a.da, c, a.n_chunks, c == 0, s_mask, s_base, s_cnt);
     }
+    if constexpr (MX) {
+        // x's scales packed per M tile of the gate/up GEMM, once every row is placed
+        alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
+        if (alive) {
+            int *s_off = reinterpret_cast<int *>(smem);
+            int *s_mt = s_off + kMaxGroupsQ + 1;
+            if (threadIdx.x == 0) load_tile_tables(a.ga.offsets, a.ga.num_groups, s_off, s_mt);
+            __syncthreads();
+            const long long R = static_cast<long long>(a.T) * (a.k + a.S);
+            for (long long r = gtid; r < R; r += gstride)
+                pack_row_scales(r, a.ga.num_groups, s_off, s_mt, a.ga.row_token, a.xs, a.H / 32,
+                                const_cast<uint8_t *>(a.ga.sfa_packed));
+        }
+    }
     fused_stamp(a, 4);
-    alive = grid_sync(a.gs, epoch, 3, alive, a.status, s_flag);
+    alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
 
     // ---------------------------------------------------------------- P4
     if (alive) {
@@ -263,7 +279,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         fused_stamp(a, 5);
     }
     fused_stamp(a, 6);
-    alive = grid_sync(a.gs, epoch, 4, alive, a.status, s_flag);
+    alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
 
     // ---------------------------------------------------------------- P5
     if (alive) {
