@@ -458,7 +458,7 @@ def main():
     phase_roofline = {}
     for name, (fl, nb) in list(alg.items()) + [(fwd_name, kern[fwd_name])]:
         t = (phase[name] if name in phase else phase["split_" + name]) / 1e3
-        phase_roofline[name] = {"ms": round(phase[name], 4), "hbm_frac": round(nb / t / 1e9 / pk["hbm_gbs"], 4),
+        phase_roofline[name] = {"ms": round(t * 1e3, 4), "hbm_frac": round(nb / t / 1e9 / pk["hbm_gbs"], 4),
                                 "tc_frac_sustained": round(fl / t / 1e12 / pk["bf16_sustained"], 4)}
 
     total_flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
