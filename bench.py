@@ -323,7 +323,8 @@ def oracle_sample(wl, params, x, dy, seconds, log=None):
     L.fwd(idx, w, tokens=toks)
     L.bwd(idx, w, tokens=toks)
     dt = time.perf_counter() - t0
-    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+    return {"value": n / dt, "unit": "tokens/s (routing + forward + dx backward; weight gradients excluded)",
+            "cores": oracle.num_threads(), "kind": "oracle",
             "sample": f"routing + forward + dx backward of {n} of the {wl.T} tokens of the {wl.name} "
                       f"workload (fp64 C oracle, OpenMP over tokens; weight gradients not in the sample)",
             "seconds": dt}
@@ -729,7 +730,7 @@ def reference_arm(args, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{wl.name} (oracle on a token sample)", "tokens_per_gpu": wl.T},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": res[0]["cores"], "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": res[0]["unit"], "cores": res[0]["cores"], "kind": "oracle",
                          "sample": res[0]["sample"]},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
