@@ -195,23 +195,39 @@ def forward_algorithmic(wl, counts):
     return fl, nb
 
 
+def backward_algorithmic(wl, counts):
+    """FLOPs and bytes of one whole backward (the persistent kernel's work): the four
+    expert GEMMs plus the slot and router gradients (x read) and the dx sum (slot rows
+    read, dx written)."""
+    alg = algorithmic(wl, counts)
+    T, H, E, k, S = wl.T, wl.H, wl.E, wl.k, wl.S
+    names = ["down_dgrad_gemm", "down_wgrad_gemm", "gate_up_dgrad_gemm", "gate_up_wgrad_gemm"]
+    fl = sum(alg[n][0] for n in names) + 2 * T * k * H
+    nb = sum(alg[n][1] for n in names) + T * H * 2 + T * (k + S) * H * 4 + T * H * 2 + E * H * 4
+    return fl, nb
+
+
+BWD_STAMP_PHASES = ["q0_zero", "down_dgrad_gemm", "gate_up_dgrad_gemm", "down_wgrad_gemm", "slot_grad",
+                    "router_partial_dx_gate_up_wgrad", "router_reduce"]
+
+
 STAMP_PHASES = ["p0_zero_split_quant", "router_gemm", "select", "dispatch", "gate_up_gemm", "down_after_gate_up",
                 "combine"]
 
 
-def stamp_phases(bufs, sms):
+def stamp_phases(bufs, sms, names=None):
     """Phase spans (ms) of the persistent forward from its device stamps, averaged over
     steps: a phase runs from the last CTA's end of the previous phase (the barrier
     release) to the last CTA's end of its own; the down GEMM overlaps the gate/up
     tail, so its span counts only the part after the last gate/up tile."""
     import numpy as np
-    acc = np.zeros(len(STAMP_PHASES))
+    acc = np.zeros(len(names or STAMP_PHASES))
     for b in bufs:
         t = b.view(-1, sms).cpu().numpy().astype(np.float64)
         ends = t.max(axis=1)
         acc[0] += ends[1] - t[0].min()
         acc[1:] += np.diff(ends[1:])
-    return {n: round(float(v) / len(bufs) / 1e6, 4) for n, v in zip(STAMP_PHASES, acc)}
+    return {n: round(float(v) / len(bufs) / 1e6, 4) for n, v in zip(names or STAMP_PHASES, acc)}
 
 
 def forward_ab(layer, x, y, K):
@@ -260,25 +276,47 @@ def forward_ab(layer, x, y, K):
 
 
 def backward_ab(layer, x, dy, grads, K):
-    """Backward only, K steps each: plain split launches against PDL launches."""
+    """Backward only, K steps each: plain split launches (an event per step), PDL split
+    launches, and the persistent launch (device stamps)."""
     import torch
-    from mixture_experts_layer_persistent_b200 import abi
+    from mixture_experts_layer_persistent_b200 import abi, moe_trace_events
+    dev = x.device
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    mk = lambda: torch.cuda.Event(enable_timing=True)
     restore = abi.moe_get_schedule()
     out = {}
-    for name, sched in (("split", abi.MOK_SCHEDULE_SPLIT), ("split_pdl", abi.MOK_SCHEDULE_SPLIT_PDL)):
+    for name, sched in (("split", abi.MOK_SCHEDULE_SPLIT), ("split_pdl", abi.MOK_SCHEDULE_SPLIT_PDL),
+                        ("persistent", abi.MOK_SCHEDULE_PERSISTENT)):
         abi.moe_set_schedule(sched)
         for _ in range(2):
             layer.backward(x, dy, grads)
+        bev = [[mk() for _ in range(abi.MOK_BWD_PHASES + 1)] for _ in range(K)]
+        for e in [e for ev in bev for e in ev]:
+            e.record()
+        bufs = [torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) for _ in range(K)]
         torch.cuda.synchronize()
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s, e = mk(), mk()
         s.record()
-        for _ in range(K):
+        for i in range(K):
+            if name == "split":
+                moe_trace_events(None, [ev.cuda_event for ev in bev[i]])
+            abi.moe_trace_device(None, 0, bufs[i].data_ptr(), bufs[i].numel() * 8)
             layer.backward(x, dy, grads)
+            launches = abi.moe_launch_count()
         e.record()
         torch.cuda.synchronize()
-        out[name] = {"ms_per_bwd": s.elapsed_time(e) / K, "launches_per_bwd": abi.moe_launch_count()}
+        moe_trace_events(None, None)
+        abi.moe_trace_device(None, 0)
+        r = {"ms_per_bwd": s.elapsed_time(e) / K, "launches_per_bwd": launches}
+        if name == "split":
+            r["phases_ms"] = {n: round(statistics.mean(bev[i][j].elapsed_time(bev[i][j + 1]) for i in range(K)), 4)
+                              for j, n in enumerate(BWD_PHASES)}
+        elif name == "persistent":
+            r["device_phases_ms"] = stamp_phases(bufs, sms, BWD_STAMP_PHASES)
+        out[name] = r
     abi.moe_set_schedule(restore)
-    out["pdl_speedup"] = out["split"]["ms_per_bwd"] / out["split_pdl"]["ms_per_bwd"]
+    out["persistent_over_split_speedup"] = out["split"]["ms_per_bwd"] / out["persistent"]["ms_per_bwd"]
+    out["split_pdl_over_split_speedup"] = out["split"]["ms_per_bwd"] / out["split_pdl"]["ms_per_bwd"]
     return out
 
 
@@ -393,6 +431,7 @@ def main():
         e.record()              # torch creates the CUDA event on its first record
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     stamps = [torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) for _ in range(K)]
+    bstamps = [torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) for _ in range(K)]
     torch.cuda.synchronize()
     uuid = str(torch.cuda.get_device_properties(dev).uuid)
     if not uuid.startswith("GPU-"):
@@ -405,7 +444,8 @@ def main():
     start.record()
     for i in range(K):
         moe_trace_events([e.cuda_event for e in fev[i]], [e.cuda_event for e in bev[i]])
-        abi.moe_trace_device(stamps[i].data_ptr(), stamps[i].numel() * 8)
+        abi.moe_trace_device(stamps[i].data_ptr(), stamps[i].numel() * 8, bstamps[i].data_ptr(),
+                             bstamps[i].numel() * 8)
         step()
     end.record()
     torch.cuda.synchronize()
@@ -419,13 +459,20 @@ def main():
 
     # the forward is one persistent launch (events around it); the backward's steps are
     # separate launches with an event each
-    fwd_name = "fwd_persistent" if sched == abi.MOK_SCHEDULE_PERSISTENT else "fwd_split"
-    phase = {fwd_name: statistics.mean(fev[i][0].elapsed_time(fev[i][-1]) for i in range(K))}
-    for n_i, name in enumerate(BWD_PHASES):
-        phase[name] = statistics.mean(bev[i][n_i].elapsed_time(bev[i][n_i + 1]) for i in range(K))
+    # each pass is one persistent launch (events around it), or split launches with an
+    # event each (--schedule split)
+    persistent = sched == abi.MOK_SCHEDULE_PERSISTENT
+    fwd_name = "fwd_persistent" if persistent else "fwd_split"
+    bwd_name = "bwd_persistent" if persistent else "bwd_split"
+    phase = {fwd_name: statistics.mean(fev[i][0].elapsed_time(fev[i][-1]) for i in range(K)),
+             bwd_name: statistics.mean(bev[i][0].elapsed_time(bev[i][-1]) for i in range(K))}
+    if not persistent:
+        for n_i, name in enumerate(BWD_PHASES):
+            phase[name] = statistics.mean(bev[i][n_i].elapsed_time(bev[i][n_i + 1]) for i in range(K))
     fwd_ms = phase[fwd_name]
-    bwd_ms = sum(phase[n] for n in BWD_PHASES)
-    fwd_device_phases = stamp_phases(stamps, sms) if sched == abi.MOK_SCHEDULE_PERSISTENT else None
+    bwd_ms = phase[bwd_name]
+    fwd_device_phases = stamp_phases(stamps, sms) if persistent else None
+    bwd_device_phases = stamp_phases(bstamps, sms, BWD_STAMP_PHASES) if persistent else None
 
     # forward A/B: split schedule (events per step, the per-GEMM attribution below) against
     # the persistent one, forward only
@@ -434,10 +481,12 @@ def main():
         phase["split_" + name] = ab["split"]["phases_ms"][name]
     layer.forward(x, y)
     bab = backward_ab(layer, x, dy, grads, K)
+    for name in BWD_PHASES:
+        phase["split_" + name] = bab["split"]["phases_ms"][name]
 
     pk = peaks()
     alg = algorithmic(wl, counts)
-    kern = {fwd_name: forward_algorithmic(wl, counts)}
+    kern = {fwd_name: forward_algorithmic(wl, counts), bwd_name: backward_algorithmic(wl, counts)}
     kern.update({n: alg[n] for n in alg if n in phase})
     dom = max(kern, key=lambda n: phase[n])
     flops, nbytes = kern[dom]
@@ -457,7 +506,7 @@ def main():
     roof["algorithmic_bytes"] = nbytes
     # every GEMM phase against both measured peaks (algorithmic bytes and FLOPs / its event time)
     phase_roofline = {}
-    for name, (fl, nb) in list(alg.items()) + [(fwd_name, kern[fwd_name])]:
+    for name, (fl, nb) in list(alg.items()) + [(fwd_name, kern[fwd_name]), (bwd_name, kern[bwd_name])]:
         t = (phase[name] if name in phase else phase["split_" + name]) / 1e3
         phase_roofline[name] = {"ms": round(t * 1e3, 4), "hbm_frac": round(nb / t / 1e9 / pk["hbm_gbs"], 4),
                                 "tc_frac_sustained": round(fl / t / 1e12 / pk["bf16_sustained"], 4)}
@@ -505,12 +554,12 @@ def main():
                        "tokens_per_gpu": wl.T, "parallelism": f"replicas x{world}",
                        "forward_schedule": args.schedule,
                        "l2": "inputs larger than L2 (22.6 GB expert weights streamed per pass)"},
-            # forward: one persistent kernel; backward: down dgrad, slot grad, 2 router-gradient
-            # kernels, 4 GEMMs plus the resident weight-gradient kernels, dx sum (10)
+            # persistent schedule: one kernel per pass (split: 9 + 10)
             "gpu_launches": K * (launches[0] + launches[1]),
             "clocks": clk, "device_status": status,
             "phases_ms": {k2: round(v, 4) for k2, v in phase.items()},
             "fwd_device_phases_ms": fwd_device_phases,
+            "bwd_device_phases_ms": bwd_device_phases,
             "forward_schedule_ab": ab,
             "backward_schedule_ab": bab,
             "breakdown": {
@@ -580,8 +629,12 @@ def bf16_workload_run(wl, dev, K, warmup, world, dist, pk):
     fwd_ms = statistics.mean(fev[i][0].elapsed_time(fev[i][-1]) for i in range(K))
     bwd_ms = statistics.mean(bev[i][0].elapsed_time(bev[i][-1]) for i in range(K)) if wl.backward else 0.0
     ab = forward_ab(layer, x, y, K)
+    bab = None
+    if wl.backward:
+        layer.forward(x, y)
+        bab = backward_ab(layer, x, dy, grads, K)
     fwd_flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
-    out = {"forward_schedule_ab": ab,
+    out = {"forward_schedule_ab": ab, "backward_schedule_ab": bab,
            "workload": f"{wl.name}: MoE layer {'fwd+bwd' if wl.backward else 'fwd'} BF16, T={wl.T}, H={wl.H}, "
                        f"E={wl.E}, top-{wl.k}, I={wl.I}, {wl.S} shared"
                        + (f", Zipf({wl.zipf}) logit term" if wl.zipf else ""),

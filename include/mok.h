@@ -288,14 +288,16 @@ int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_
 
 /*
  * Schedule of the passes (per host thread; default PERSISTENT).
- *   MOK_SCHEDULE_PERSISTENT  the whole forward is one cooperative launch of one
- *       persistent kernel, one CTA per SM: router, top-k, dispatch, the two
- *       expert GEMMs and the combine are phases separated by grid barriers,
- *       except that the down GEMM starts an M tile as soon as every gate/up tile
- *       of its rows is in memory (per-tile readiness counters) -- the fusion of
- *       the layer into one kernel that "Cursor åpner megakernelen…" (the quoted
- *       paragraph) describes.  No memset or other launch precedes it.  The
- *       backward runs split with programmatic dependent launch.
+ *   MOK_SCHEDULE_PERSISTENT  each pass is one cooperative launch of one
+ *       persistent kernel, one CTA per SM -- the fusion of the layer into one
+ *       kernel that "Cursor åpner megakernelen…" (the quoted paragraph)
+ *       describes.  Forward: router, top-k, dispatch, the two expert GEMMs and
+ *       the combine are phases separated by grid barriers, except that the down
+ *       GEMM starts an M tile as soon as every gate/up tile of its rows is in
+ *       memory (per-tile readiness counters).  Backward: down dgrad, gate/up
+ *       dgrad (started per M tile the same way), the weight gradients, the slot
+ *       and router gradients and the dx sum.  No memset or other launch precedes
+ *       either.
  *   MOK_SCHEDULE_SPLIT  one launch per step in stream order (router split,
  *       router GEMM, select, three dispatch kernels, [MXFP8: quantise x], gate/up,
  *       down, combine) after a memset of the tile counters; the backward the same.
@@ -313,15 +315,19 @@ int moe_set_schedule(int schedule);
 int moe_get_schedule(int *schedule);
 
 /*
- * Device-side phase stamps of the persistent forward (per host thread).  When
- * buf (device memory, at least MOK_TRACE_POINTS * SMs * 8 bytes) is set, every
- * later persistent forward writes, for each point p and CTA b, the globaltimer
- * value (ns) at buf[p * SMs + b]: p = 0 start, then the end of the zeroing /
- * router-split / quantisation phase, the router GEMM, the top-k, the dispatch,
- * the gate/up GEMM, the down GEMM and the combine.  NULL stops it.
+ * Device-side phase stamps of the persistent passes (per host thread).  When
+ * buf (bwd_buf) -- device memory of at least MOK_TRACE_POINTS * SMs * 8 bytes --
+ * is set, every later persistent forward (backward) writes, for each point p
+ * and CTA b, the globaltimer value (ns) at buf[p * SMs + b].  Forward points:
+ * p = 0 start, then the end of the zeroing / router-split / quantisation
+ * phase, the router GEMM, the top-k, the dispatch, the gate/up GEMM, the down
+ * GEMM and the combine.  Backward points: p = 0 start, then the end of the
+ * zeroing, the down dgrad GEMM, the gate/up dgrad GEMM, the down weight
+ * gradient, the slot gradients, the router partial sums + dx + gate/up weight
+ * gradient, and the router-gradient reduction.  NULL stops the stamps.
  */
 #define MOK_TRACE_POINTS 8
-int moe_trace_device(void *buf, size_t bytes);
+int moe_trace_device(void *buf, size_t bytes, void *bwd_buf, size_t bwd_bytes);
 
 /*
  * Number of CUDA kernels launched by the last moe_fwd / moe_bwd (or their

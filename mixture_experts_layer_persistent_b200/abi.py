@@ -97,7 +97,7 @@ def lib():
         L.moe_saved_tensor.argtypes = [P(moe_cfg), _i32, _i32, P(_sz), P(_sz)]
         L.moe_set_schedule.argtypes = [ctypes.c_int]
         L.moe_get_schedule.argtypes = [P(_i32)]
-        L.moe_trace_device.argtypes = [_vp, _sz]
+        L.moe_trace_device.argtypes = [_vp, _sz, _vp, _sz]
         L.moe_strerror.argtypes = [ctypes.c_int]
         L.moe_strerror.restype = ctypes.c_char_p
         L.moe_last_error.argtypes = []
@@ -137,8 +137,8 @@ def moe_get_schedule() -> int:
     return v.value
 
 
-def moe_trace_device(buf, nbytes: int) -> None:
-    _check("moe_trace_device", lib().moe_trace_device(buf, int(nbytes)))
+def moe_trace_device(buf, nbytes: int, bwd_buf=None, bwd_nbytes: int = 0) -> None:
+    _check("moe_trace_device", lib().moe_trace_device(buf, int(nbytes), bwd_buf, int(bwd_nbytes)))
 
 
 def moe_saved_tensor(cfg: moe_cfg, save_for_backward: bool, which: int):

@@ -74,15 +74,11 @@ __global__ void __launch_bounds__(256) combine_kernel(const Slot *__restrict__ O
 //   softmax: dl_j = w_j (G_j - sum_i q_i G_i),             q = w / routed_scale
 //   sigmoid: dl_j = rho/S (G_j - sum_i q_i G_i) s_j (1 - s_j), S = sum of selected s
 // One thread per token.
-__global__ void __launch_bounds__(256) slot_grad_kernel(const float *__restrict__ gpart, int n_parts,
-                                                        const int *__restrict__ inv_perm,
-                                                        const float *__restrict__ topk_w,
-                                                        const float *__restrict__ topk_p, float *__restrict__ dl,
-                                                        int T, int k, int score_fn, float routed_scale)
+__device__ __forceinline__ void slot_grad_token(int t, const float *__restrict__ gpart, int n_parts,
+                                                const int *__restrict__ inv_perm, const float *__restrict__ topk_w,
+                                                const float *__restrict__ topk_p, float *__restrict__ dl, int k,
+                                                int score_fn, float routed_scale)
 {
-    griddep_enter();
-    const int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= T) return;
     float G[16], q[16];
     float gbar = 0.0f, S_ = 0.0f;
     for (int j = 0; j < k; ++j) {
@@ -106,23 +102,31 @@ __global__ void __launch_bounds__(256) slot_grad_kernel(const float *__restrict_
     }
 }
 
+__global__ void __launch_bounds__(256) slot_grad_kernel(const float *__restrict__ gpart, int n_parts,
+                                                        const int *__restrict__ inv_perm,
+                                                        const float *__restrict__ topk_w,
+                                                        const float *__restrict__ topk_p, float *__restrict__ dl,
+                                                        int T, int k, int score_fn, float routed_scale)
+{
+    griddep_enter();
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t < T) slot_grad_token(t, gpart, n_parts, inv_perm, topk_w, topk_p, dl, k, score_fn, routed_scale);
+}
+
 // Router weight gradient, pass 1: for each chunk of up to `chunk_rows` sorted
 // rows of one expert and 256 columns, partial[chunk, cols] = sum over the
 // chunk's rows (ascending) of dl(row) x[token(row), cols].  8 warps take rows
 // r = warp (mod 8); their sums are added in warp order.
-__global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat16 *__restrict__ x,
-                                                              const float *__restrict__ dl,
-                                                              const int *__restrict__ offsets,
-                                                              const int *__restrict__ chunk_start,
-                                                              const int *__restrict__ perm,
-                                                              float *__restrict__ partial, int H, int E, int k,
-                                                              int chunk_rows)
+// One (chunk, 256-column block) item by the first 256 threads of the CTA
+// (s_acc: 8 x 256 floats of shared memory).  Every thread of the CTA calls it:
+// it contains a CTA-wide barrier.
+__device__ __forceinline__ void drouter_partial_item(int chunk, int h0, const __nv_bfloat16 *__restrict__ x,
+                                                     const float *__restrict__ dl, const int *__restrict__ offsets,
+                                                     const int *__restrict__ chunk_start,
+                                                     const int *__restrict__ perm, float *__restrict__ partial,
+                                                     int H, int E, int k, int chunk_rows, float (*s_acc)[256])
 {
-    griddep_enter();
-    __shared__ float s_acc[8][256];
-    const int chunk = blockIdx.x;
-    const int h0 = blockIdx.y * 256;
-    if (chunk >= chunk_start[E]) return;
+    const bool active = threadIdx.x < 256;
     int lo = 0, hi = E - 1;     // expert owning this chunk: largest e with chunk_start[e] <= chunk
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -133,7 +137,7 @@ __global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat1
     const int r1 = min(offsets[e + 1], r0 + chunk_rows);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int r = r0 + warp; r < r1; r += 8) {
+    for (int r = r0 + warp; active && r < r1; r += 8) {
         const int s = perm[r];                  // t * k + slot
         const float d = dl[s];
         const int tok = s / k;
@@ -142,40 +146,61 @@ __global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat1
 #pragma unroll
         for (int q = 0; q < 8; ++q) acc[q] = fmaf(d, v[q], acc[q]);
     }
+    if (active) {
 #pragma unroll
-    for (int q = 0; q < 8; ++q) s_acc[warp][lane * 8 + q] = acc[q];
+        for (int q = 0; q < 8; ++q) s_acc[warp][lane * 8 + q] = acc[q];
+    }
     __syncthreads();
-    float s = 0.0f;
-    for (int w = 0; w < 8; ++w) s += s_acc[w][threadIdx.x];
-    partial[(size_t)chunk * H + h0 + threadIdx.x] = s;
+    if (active) {
+        float s = 0.0f;
+        for (int w = 0; w < 8; ++w) s += s_acc[w][threadIdx.x];
+        partial[(size_t)chunk * H + h0 + threadIdx.x] = s;
+    }
+    __syncthreads();                            // s_acc is free again
+}
+
+__global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat16 *__restrict__ x,
+                                                              const float *__restrict__ dl,
+                                                              const int *__restrict__ offsets,
+                                                              const int *__restrict__ chunk_start,
+                                                              const int *__restrict__ perm,
+                                                              float *__restrict__ partial, int H, int E, int k,
+                                                              int chunk_rows)
+{
+    griddep_enter();
+    __shared__ float s_acc[8][256];
+    if (static_cast<int>(blockIdx.x) >= chunk_start[E]) return;
+    drouter_partial_item(blockIdx.x, blockIdx.y * 256, x, dl, offsets, chunk_start, perm, partial, H, E, k, chunk_rows,
+                         s_acc);
 }
 
 // Router weight gradient, pass 2: dWr[e, h] = sum over the expert's chunks in order.
-__global__ void __launch_bounds__(256) drouter_reduce_kernel(const float *__restrict__ partial,
-                                                             const int *__restrict__ chunk_start,
-                                                             float *__restrict__ dWr, int H, int E)
+__device__ __forceinline__ void drouter_reduce_elem(long long i, const float *__restrict__ partial,
+                                                   const int *__restrict__ chunk_start, float *__restrict__ dWr, int H)
 {
-    griddep_enter();
-    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (long long)E * H) return;
     const int e = (int)(i / H), h = (int)(i % H);
     float s = 0.0f;
     for (int c = chunk_start[e]; c < chunk_start[e + 1]; ++c) s += partial[(size_t)c * H + h];
     dWr[i] = s;
 }
 
-// dx[t] = sum_j dXs[t, j] (ascending j over routed then shared slots)
-//         + sum_{j<k} dl[t, j] router_w[idx[t, j]]   -> bf16.
-__global__ void __launch_bounds__(256) dx_combine_kernel(const float *__restrict__ dXs,
-                                                         const float *__restrict__ dl,
-                                                         const int *__restrict__ topk_idx,
-                                                         const float *__restrict__ router_w,
-                                                         __nv_bfloat16 *__restrict__ dx, int T, int H, int k, int S)
+__global__ void __launch_bounds__(256) drouter_reduce_kernel(const float *__restrict__ partial,
+                                                             const int *__restrict__ chunk_start,
+                                                             float *__restrict__ dWr, int H, int E)
 {
     griddep_enter();
-    const int cpr = H / 8;
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (long long)T * cpr) return;
+    if (i < (long long)E * H) drouter_reduce_elem(i, partial, chunk_start, dWr, H);
+}
+
+// dx[t] = sum_j dXs[t, j] (ascending j over routed then shared slots)
+//         + sum_{j<k} dl[t, j] router_w[idx[t, j]]   -> bf16.
+__device__ __forceinline__ void dx_combine_elem(long long i, const float *__restrict__ dXs,
+                                                const float *__restrict__ dl, const int *__restrict__ topk_idx,
+                                                const float *__restrict__ router_w, __nv_bfloat16 *__restrict__ dx,
+                                                int H, int k, int S)
+{
+    const int cpr = H / 8;
     const int t = (int)(i / cpr), c = (int)(i % cpr) * 8;
     const int kk = k + S;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -198,6 +223,17 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *__restrict
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] += r[q];
     *reinterpret_cast<uint4 *>(dx + (size_t)t * H + c) = pack8(acc);
+}
+
+__global__ void __launch_bounds__(256) dx_combine_kernel(const float *__restrict__ dXs,
+                                                         const float *__restrict__ dl,
+                                                         const int *__restrict__ topk_idx,
+                                                         const float *__restrict__ router_w,
+                                                         __nv_bfloat16 *__restrict__ dx, int T, int H, int k, int S)
+{
+    griddep_enter();
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < (long long)T * (H / 8)) dx_combine_elem(i, dXs, dl, topk_idx, router_w, dx, H, k, S);
 }
 
 }  // namespace mok

@@ -605,9 +605,12 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
             tile = __shfl_sync(0xffffffffu, next, 0);
         }
     producer_done:
-        if (*abort_flag && lane == 0) {
-            // another role gave up: let the last STAGES fills land (bounded) before the
-            // CTA releases its shared memory
+        if (lane == 0) {
+            // the last STAGES fills: after an abort, let their loads land (bounded) before
+            // the CTA releases its shared memory; otherwise wait until the MMA has released
+            // them, so that no arrival on this phase's barriers is still in flight when the
+            // phase ends (a later phase of the launch may reuse the memory)
+            const bool aborted = *abort_flag != 0;
             int s2 = stage;
             uint32_t ph = phase;
             for (int i = 0; i < min(fills, C::STAGES); ++i) {
@@ -615,7 +618,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                     s2 = C::STAGES - 1;
                     ph ^= 1u;
                 }
-                mbar_drain(&full_bar[s2], ph);
+                mbar_drain(aborted ? &full_bar[s2] : &empty_bar[s2], ph);
             }
         }
     } else if (warp >= C::PULL_WARP0) {

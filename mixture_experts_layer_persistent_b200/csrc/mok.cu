@@ -12,6 +12,7 @@
 
 #include "combine.cuh"
 #include "fused.cuh"
+#include "fused_bwd.cuh"
 #include "gemm.cuh"
 #include "quant.cuh"
 #include "route.cuh"
@@ -61,8 +62,10 @@ thread_local cudaEvent_t t_bwd_ev[MOK_BWD_PHASES + 1];
 thread_local bool t_fwd_on = false, t_bwd_on = false;
 thread_local int t_drop_signal = 0;     // moe_test_drop_signal
 thread_local int t_schedule = MOK_SCHEDULE_PERSISTENT;   // moe_set_schedule
-thread_local unsigned long long *t_dev_trace = nullptr;   // moe_trace_device
+thread_local unsigned long long *t_dev_trace = nullptr;   // moe_trace_device (forward)
 thread_local size_t t_dev_trace_bytes = 0;
+thread_local unsigned long long *t_dev_trace_bwd = nullptr;   // moe_trace_device (backward)
+thread_local size_t t_dev_trace_bwd_bytes = 0;
 thread_local int t_launches = 0;        // kernels launched by the current / last forward or backward
 thread_local bool t_pdl = false;        // launches of the current pass use programmatic dependent launch
 
@@ -251,6 +254,10 @@ struct BwdScratch {
     float *gpart;                 // per routed row and N tile of the down dgrad: <dy W_down, h>
     __nv_bfloat16 *dgu;
     int *sched;                   // [kSchedCounters] backward GEMM tile counters
+    int *ready;                   // [n_mtiles] per-M-tile readiness of dGU (persistent backward)
+    int *zero;                    // sched and ready: the counters the persistent backward zeroes
+    int n_zero;
+    unsigned long long *gs_flags; // grid-barrier tags, release tag, epoch
     size_t bytes;
 };
 
@@ -264,7 +271,12 @@ BwdScratch carve_bwd(const moe_cfg &c, void *buf)
     b.partial = cv.take<float>(s.max_chunks * s.H);
     b.dgu = cv.take<__nv_bfloat16>(s.R * 2 * s.I);
     b.dxs = cv.take<float>(s.T * s.kk * s.H);
-    b.sched = cv.take<int>(kSchedCounters);
+    const int n_mtiles = static_cast<int>(s.R / BM + s.G + 1);
+    b.n_zero = kSchedCounters + n_mtiles;
+    b.zero = cv.take<int>(b.n_zero);
+    b.sched = b.zero;
+    b.ready = b.zero + kSchedCounters;
+    b.gs_flags = cv.take<unsigned long long>(kMaxFusedCtas + 2);
     b.bytes = align_up(cv.off, 256);
     return b;
 }
@@ -664,16 +676,21 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
 }
 
 // ------------------------------------------------------------------ backward
-int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &p, const State &st,
-             const moe_grads &gr, const BwdScratch &bs, const DeviceInfo &dev, cudaStream_t stream)
+// Tensor maps and arguments of every step of the backward, shared by the split
+// schedule and the persistent one.
+struct BwdPlan {
+    FusedBwdMaps m;
+    GemmArgs g1, g2, g3, g4;
+    int g2_grid, g4_grid;       // split launches of the streaming weight gradients
+    int g2_units, g4_units;     // resident weight-gradient work units (0: none)
+    bool n256;                  // I is a multiple of 256
+};
+
+int build_bwd_plan(const moe_cfg &c, const void *x, const void *dy, const moe_params &p, const State &st,
+                   const moe_grads &gr, const BwdScratch &bs, const DeviceInfo &dev, BwdPlan &pl)
 {
     const Shapes s = shapes(c);
-    t_launches = 0;
-    t_pdl = t_schedule != MOK_SCHEDULE_SPLIT;       // the backward is split; PDL unless plain split is asked
-    const __nv_bfloat16 *dyb = static_cast<const __nv_bfloat16 *>(dy);
-    if (const cudaError_t e = cudaMemsetAsync(bs.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
-        return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
-
+    pl.n256 = c.I % 256 == 0;
     GemmArgs base{};
     base.num_groups = static_cast<int>(s.G);
     base.num_routed = c.E;
@@ -683,15 +700,18 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     base.row_slot = st.row_slot;
     base.row_w = st.row_w;
     base.inter = c.I;
-    base.gather_src = dyb;
+    base.gather_src = static_cast<const __nv_bfloat16 *>(dy);
     base.gather_ld = c.H;
     base.status = dev.status;
+    base.ready = bs.ready;
 
-    CUtensorMap tA, tB, tBs, tO, tO2;
     // dgrad of down: dh = w * (dy[token] . W_down), SwiGLU backward epilogue -> dGU
-    if (!make_tmap(&tB, p.w_down, s.I, s.E * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
-    GemmArgs g1 = base;
+    if (!make_tmap(&pl.m.d1B, p.w_down, s.I, s.E * s.H, 64, 64, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&pl.m.d1Bs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 64, 2))
+        return MOK_ERR_INVALID;
+    if (!make_tmap(&pl.m.d1O, bs.dgu, 2 * s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
+    GemmArgs &g1 = pl.g1;
+    g1 = base;
     g1.sched = bs.sched + 0;
     g1.num_kb = c.H / BK;
     g1.b_rows_per_group = c.H;
@@ -699,17 +719,94 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     g1.aux_h = st.h;
     g1.gpart = bs.gpart;
     g1.out = bs.dgu;
-    MOK_TRY(mark_bwd(0, stream));
-    if (!make_tmap(&tO, bs.dgu, 2 * s.I, s.R, 64, 32, 2)) return MOK_ERR_INVALID;
-    if (c.I % 256 == 0) {      // N = 256 halves the gathered dy rows per weight byte
-        g1.n_tiles = c.I / 256;
-        using CDgradDown = GemmCfg<256, false, true, true, false, false, EPI_DSWIGLU>;
-        MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, tO, tO, tO, g1, dev.sms, stream));
+    g1.n_tiles = pl.n256 ? c.I / 256 : c.I / 128;   // N = 256 halves the gathered dy rows per weight byte
+
+    // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
+    if (!make_tmap(&pl.m.w2O, gr.dw_down, s.I, s.E * s.H, 64, 32, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&pl.m.w2O2, s.S ? gr.dws_down : gr.dw_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 32, 2))
+        return MOK_ERR_INVALID;
+    if (!make_tmap(&pl.m.w2B, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
+    GemmArgs &g2 = pl.g2;
+    g2 = base;
+    g2.sched = bs.sched + 1;
+    g2.m_tiles = c.H / 128;
+    g2.out = static_cast<__nv_bfloat16 *>(gr.dw_down);
+    g2.out_s = static_cast<__nv_bfloat16 *>(gr.dws_down);
+    g2.ldo = c.I;
+    g2.group_out_elems = s.H * s.I;
+    if (pl.n256) {
+        // groups of more than kResidentRows rows stream both operands; the rest keep
+        // their (w h) slab resident and stream gathered dy
+        g2.n_tiles = c.I / 256;
+        g2.k_split = kResidentRows;
+        g2.m_per_unit = resident_m_per_unit(g2.m_tiles);
+        pl.g2_units = static_cast<int>(s.G * g2.n_tiles * ((g2.m_tiles + g2.m_per_unit - 1) / g2.m_per_unit));
     } else {
-        g1.n_tiles = c.I / 128;
-        using CDgradDown = GemmCfg<128, false, true, true, false, false, EPI_DSWIGLU>;
-        MOK_TRY(launch_gemm<CDgradDown>(tB, tB, tBs, tO, tO, tO, g1, dev.sms, stream));
+        g2.n_tiles = c.I / 128;
+        pl.g2_units = 0;
     }
+    const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
+    pl.g2_grid = static_cast<int>(t2 < dev.sms ? t2 : dev.sms);
+
+    // dgrad of gate/up: dX rows = dGU . W_gate_up, pushed into (token, slot) rows
+    if (!make_tmap(&pl.m.d3A, bs.dgu, 2 * s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&pl.m.d3B, p.w_gate_up, s.H, s.E * 2 * s.I, 64, 64, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&pl.m.d3Bs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 64, 64, 2))
+        return MOK_ERR_INVALID;
+    if (!make_tmap(&pl.m.d3O, bs.dxs, s.H, s.T * s.kk, 32, 1, 4)) return MOK_ERR_INVALID;
+    GemmArgs &g3 = pl.g3;
+    g3 = base;
+    g3.sched = bs.sched + 2;
+    g3.n_tiles = c.H / 256;
+    g3.num_kb = 2 * c.I / BK;
+    g3.b_rows_per_group = 2 * c.I;
+    g3.out_f32 = bs.dxs;
+    g3.ldo = c.H;
+    g3.ready_target = 4 * g1.n_tiles;     // four epilogue warps per down-dgrad tile, its N tiles per M tile
+
+    // wgrad of gate/up: dW_gate_up[g] = sum_r dGU_r^T x[token r]
+    if (!make_tmap(&pl.m.w4A, bs.dgu, 2 * s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&pl.m.w4O, gr.dw_gate_up, s.H, s.E * 2 * s.I, 64, 32, 2)) return MOK_ERR_INVALID;
+    if (!make_tmap(&pl.m.w4O2, s.S ? gr.dws_gate_up : gr.dw_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 64, 32, 2))
+        return MOK_ERR_INVALID;
+    GemmArgs &g4 = pl.g4;
+    g4 = base;
+    g4.sched = bs.sched + 3;
+    g4.gather_src = static_cast<const __nv_bfloat16 *>(x);
+    g4.m_tiles = 2 * c.I / 128;
+    g4.n_tiles = c.H / 256;
+    g4.out = static_cast<__nv_bfloat16 *>(gr.dw_gate_up);
+    g4.out_s = static_cast<__nv_bfloat16 *>(gr.dws_gate_up);
+    g4.ldo = c.H;
+    g4.group_out_elems = 2 * s.I * s.H;
+    g4.k_split = kResidentRows;            // larger groups stream; the rest keep their x slab resident
+    g4.m_per_unit = resident_m_per_unit(g4.m_tiles);
+    const long long t4 = s.G * g4.m_tiles * g4.n_tiles;
+    pl.g4_grid = static_cast<int>(t4 < dev.sms ? t4 : dev.sms);
+    pl.g4_units = static_cast<int>(s.G * g4.n_tiles * ((g4.m_tiles + g4.m_per_unit - 1) / g4.m_per_unit));
+    return MOK_OK;
+}
+
+// Split schedule: one launch per step, in stream order (with PDL unless the plain
+// split schedule is asked for).
+int backward_split(const moe_cfg &c, const void *x, const moe_params &p, const State &st, const moe_grads &gr,
+                   const BwdScratch &bs, const DeviceInfo &dev, const BwdPlan &pl, cudaStream_t stream)
+{
+    const Shapes s = shapes(c);
+    t_pdl = t_schedule != MOK_SCHEDULE_SPLIT;
+    if (const cudaError_t e = cudaMemsetAsync(bs.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
+    GemmArgs g1 = pl.g1, g2 = pl.g2, g3 = pl.g3, g4 = pl.g4;
+    g1.ready_role = g3.ready_role = kReadyNone;
+    const FusedBwdMaps &m = pl.m;
+
+    MOK_TRY(mark_bwd(0, stream));
+    if (pl.n256)
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradDown>(m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1,
+                                                                  dev.sms, stream));
+    else
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<false>::DgradDown>(m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1,
+                                                                   dev.sms, stream));
 
     // slot gradients from the down dgrad's partials, then the router weight gradient
     MOK_TRY(mark_bwd(1, stream));
@@ -727,89 +824,115 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
                      "drouter_reduce_kernel", static_cast<const float *>(bs.partial),
                      static_cast<const int *>(st.chunk_start), gr.drouter_w, c.H, c.E));
 
-    // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
-    GemmArgs g2 = base;
-    g2.sched = bs.sched + 1;
-    g2.m_tiles = c.H / 128;
-    g2.out = static_cast<__nv_bfloat16 *>(gr.dw_down);
-    g2.out_s = static_cast<__nv_bfloat16 *>(gr.dws_down);
-    g2.ldo = c.I;
-    g2.group_out_elems = s.H * s.I;
     MOK_TRY(mark_bwd(4, stream));
-    if (!make_tmap(&tO, gr.dw_down, s.I, s.E * s.H, 64, 32, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tO2, s.S ? gr.dws_down : gr.dw_down, s.I, (s.S ? s.S : s.E) * s.H, 64, 32, 2))
-        return MOK_ERR_INVALID;
-    if (c.I % 256 == 0) {
-        // groups of more than kResidentRows rows stream both operands; the rest keep
-        // their (w h) slab resident and stream gathered dy
-        if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
-        g2.n_tiles = c.I / 256;
-        g2.k_split = kResidentRows;
-        g2.m_per_unit = resident_m_per_unit(g2.m_tiles);
-        using CWgradDown = GemmCfg<256, true, true, true, false, true, EPI_WGRAD>;
-        const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
-        MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, tO, tO2, tO, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms),
-                                        stream));
-        const long long u2 = s.G * g2.n_tiles * ((g2.m_tiles + g2.m_per_unit - 1) / g2.m_per_unit);
-        MOK_TRY(launch_wgrad_resident<WgradResCfg<true>>(tB, tB, tO, tO2, g2,
-                                                         static_cast<int>(u2 < dev.sms ? u2 : dev.sms), stream));
+    if (pl.n256) {
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::WgradDown>(m.w2B, m.w2B, m.w2B, m.w2O, m.w2O2, m.w2O, g2,
+                                                                  pl.g2_grid, stream));
+        MOK_TRY(launch_wgrad_resident<WgradResCfg<true>>(m.w2B, m.w2B, m.w2O, m.w2O2, g2,
+                                                         pl.g2_units < dev.sms ? pl.g2_units : dev.sms, stream));
     } else {
-        if (!make_tmap(&tB, st.hw, s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
-        g2.n_tiles = c.I / 128;
-        using CWgradDown = GemmCfg<128, true, true, true, false, true, EPI_WGRAD>;
-        const long long t2 = s.G * g2.m_tiles * g2.n_tiles;
-        MOK_TRY(launch_gemm<CWgradDown>(tB, tB, tB, tO, tO2, tO, g2, static_cast<int>(t2 < dev.sms ? t2 : dev.sms),
-                                        stream));
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<false>::WgradDown>(m.w2B, m.w2B, m.w2B, m.w2O, m.w2O2, m.w2O, g2,
+                                                                   pl.g2_grid, stream));
     }
 
-    // dgrad of gate/up: dX rows = dGU . W_gate_up, pushed into (token, slot) rows
-    if (!make_tmap(&tA, bs.dgu, 2 * s.I, s.R, BK, 128, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tB, p.w_gate_up, s.H, s.E * 2 * s.I, 64, 64, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 64, 64, 2))
-        return MOK_ERR_INVALID;
-    GemmArgs g3 = base;
-    g3.sched = bs.sched + 2;
-    g3.n_tiles = c.H / 256;
-    g3.num_kb = 2 * c.I / BK;
-    g3.b_rows_per_group = 2 * c.I;
-    g3.out_f32 = bs.dxs;
-    g3.ldo = c.H;
-    using CDgradGU = GemmCfg<256, false, true, false, false, false, EPI_PUSH>;
     MOK_TRY(mark_bwd(5, stream));
-    if (!make_tmap(&tO, bs.dxs, s.H, s.T * s.kk, 32, 1, 4)) return MOK_ERR_INVALID;
-    MOK_TRY(launch_gemm<CDgradGU>(tA, tB, tBs, tO, tO, tO, g3, dev.sms, stream));
+    MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradGU>(m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O, g3, dev.sms,
+                                                            stream));
 
-    // wgrad of gate/up: dW_gate_up[g] = sum_r dGU_r^T x[token r]
-    if (!make_tmap(&tA, bs.dgu, 2 * s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
-    GemmArgs g4 = base;
-    g4.sched = bs.sched + 3;
-    g4.gather_src = static_cast<const __nv_bfloat16 *>(x);
-    g4.m_tiles = 2 * c.I / 128;
-    g4.n_tiles = c.H / 256;
-    g4.out = static_cast<__nv_bfloat16 *>(gr.dw_gate_up);
-    g4.out_s = static_cast<__nv_bfloat16 *>(gr.dws_gate_up);
-    g4.ldo = c.H;
-    g4.group_out_elems = 2 * s.I * s.H;
-    g4.k_split = kResidentRows;            // larger groups stream; the rest keep their x slab resident
-    g4.m_per_unit = resident_m_per_unit(g4.m_tiles);
-    using CWgradGU = GemmCfg<256, true, true, false, true, true, EPI_WGRAD>;
-    const long long t4 = s.G * g4.m_tiles * g4.n_tiles;
     MOK_TRY(mark_bwd(6, stream));
-    if (!make_tmap(&tO, gr.dw_gate_up, s.H, s.E * 2 * s.I, 64, 32, 2)) return MOK_ERR_INVALID;
-    if (!make_tmap(&tO2, s.S ? gr.dws_gate_up : gr.dw_gate_up, s.H, (s.S ? s.S : s.E) * 2 * s.I, 64, 32, 2))
-        return MOK_ERR_INVALID;
-    MOK_TRY(launch_gemm<CWgradGU>(tA, tA, tA, tO, tO2, tO, g4, static_cast<int>(t4 < dev.sms ? t4 : dev.sms), stream));
-    const long long u4 = s.G * g4.n_tiles * ((g4.m_tiles + g4.m_per_unit - 1) / g4.m_per_unit);
-    MOK_TRY(launch_wgrad_resident<WgradResCfg<false>>(tA, tA, tO, tO2, g4, static_cast<int>(u4 < dev.sms ? u4 : dev.sms),
-                                                      stream));
+    MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::WgradGU>(m.w4A, m.w4A, m.w4A, m.w4O, m.w4O2, m.w4O, g4, pl.g4_grid,
+                                                            stream));
+    MOK_TRY(launch_wgrad_resident<WgradResCfg<false>>(m.w4A, m.w4A, m.w4O, m.w4O2, g4,
+                                                      pl.g4_units < dev.sms ? pl.g4_units : dev.sms, stream));
 
     MOK_TRY(mark_bwd(7, stream));
     MOK_TRY(launch_k(dx_combine_kernel, dim3(blocks_for(s.T * s.H / 8, 256)), dim3(256), 0, stream,
                      "dx_combine_kernel", static_cast<const float *>(bs.dxs), static_cast<const float *>(bs.dl),
                      static_cast<const int *>(st.topk_idx), p.router_w, static_cast<__nv_bfloat16 *>(gr.dx), c.T, c.H,
                      c.top_k, c.n_shared));
-    MOK_TRY(mark_bwd(8, stream));
+    return mark_bwd(8, stream);
+}
+
+// Persistent schedule: the whole backward as one cooperative launch (fused_bwd.cuh).
+template <bool N256>
+int launch_fused_bwd(const moe_cfg &c, const void *x, const moe_params &p, const State &st, const moe_grads &gr,
+                     const BwdScratch &bs, const DeviceInfo &dev, const BwdPlan &pl, cudaStream_t stream)
+{
+    using F = FusedBwdCfg<N256>;
+    if (dev.sms > kMaxFusedCtas) return fail(MOK_ERR_UNSUPPORTED, "more SMs than the grid barrier holds");
+    const Shapes s = shapes(c);
+    FusedBwdArgs a{};
+    a.gs.flags = bs.gs_flags;
+    a.gs.go = bs.gs_flags + kMaxFusedCtas;
+    a.gs.epoch = bs.gs_flags + kMaxFusedCtas + 1;
+    a.status = dev.status;
+    a.zero = bs.zero;
+    a.n_zero = bs.n_zero;
+    a.g1 = pl.g1;
+    a.g1.ready_role = kReadySignal;
+    a.g2 = a.g2r = pl.g2;
+    a.g3 = pl.g3;
+    a.g3.ready_role = kReadyWait;
+    a.g4 = a.g4r = pl.g4;
+    a.g2_units = pl.g2_units;
+    a.g4_units = pl.g4_units;
+    a.gpart = bs.gpart;
+    a.n_parts = pl.g1.n_tiles;
+    a.inv_perm = st.inv_perm;
+    a.topk_idx = st.topk_idx;
+    a.offsets = st.offsets;
+    a.chunk_start = st.chunk_start;
+    a.perm = st.perm;
+    a.topk_w = st.topk_w;
+    a.topk_p = st.topk_p;
+    a.router_w = p.router_w;
+    a.dl = bs.dl;
+    a.partial = bs.partial;
+    a.drouter_w = gr.drouter_w;
+    a.x = static_cast<const __nv_bfloat16 *>(x);
+    a.T = c.T; a.H = c.H; a.E = c.E; a.k = c.top_k; a.S = c.n_shared;
+    a.score_fn = c.score_fn;
+    a.chunk_rows = kChunkRows;
+    a.max_chunks = static_cast<int>(s.max_chunks);
+    a.routed_scale = c.routed_scale;
+    a.dxs = bs.dxs;
+    a.dx = static_cast<__nv_bfloat16 *>(gr.dx);
+    a.trace = (t_dev_trace_bwd && t_dev_trace_bwd_bytes >= sizeof(unsigned long long) * kFusedBwdTracePoints * dev.sms)
+                  ? t_dev_trace_bwd : nullptr;
+
+    cudaError_t e = cudaFuncSetAttribute(moe_bwd_fused_kernel<N256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         F::SMEM_BYTES);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(moe_bwd_fused_kernel)", e);
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(static_cast<unsigned>(dev.sms));
+    lc.blockDim = dim3(kFusedThreads);
+    lc.dynamicSmemBytes = F::SMEM_BYTES;
+    lc.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    MOK_TRY(mark_bwd(0, stream));
+    e = cudaLaunchKernelEx(&lc, moe_bwd_fused_kernel<N256>, pl.m, a);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaLaunchKernelEx(moe_bwd_fused_kernel, cooperative)", e);
+    ++t_launches;
+    for (int i = 1; i <= MOK_BWD_PHASES; ++i) MOK_TRY(mark_bwd(i, stream));
     return MOK_OK;
+}
+
+int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &p, const State &st,
+             const moe_grads &gr, const BwdScratch &bs, const DeviceInfo &dev, cudaStream_t stream)
+{
+    t_launches = 0;
+    BwdPlan pl;
+    MOK_TRY(build_bwd_plan(c, x, dy, p, st, gr, bs, dev, pl));
+    if (t_schedule == MOK_SCHEDULE_PERSISTENT) {
+        t_pdl = false;
+        return pl.n256 ? launch_fused_bwd<true>(c, x, p, st, gr, bs, dev, pl, stream)
+                       : launch_fused_bwd<false>(c, x, p, st, gr, bs, dev, pl, stream);
+    }
+    return backward_split(c, x, p, st, gr, bs, dev, pl, stream);
 }
 
 int check_params(const moe_cfg &c, const moe_params *p)
@@ -1067,11 +1190,13 @@ int moe_get_schedule(int *schedule)
     return MOK_OK;
 }
 
-int moe_trace_device(void *buf, size_t bytes)
+int moe_trace_device(void *buf, size_t bytes, void *bwd_buf, size_t bwd_bytes)
 {
-    if (buf && !aligned16(buf)) return MOK_ERR_INVALID;
+    if ((buf && !aligned16(buf)) || (bwd_buf && !aligned16(bwd_buf))) return MOK_ERR_INVALID;
     t_dev_trace = static_cast<unsigned long long *>(buf);
     t_dev_trace_bytes = buf ? bytes : 0;
+    t_dev_trace_bwd = static_cast<unsigned long long *>(bwd_buf);
+    t_dev_trace_bwd_bytes = bwd_buf ? bwd_bytes : 0;
     return MOK_OK;
 }
 

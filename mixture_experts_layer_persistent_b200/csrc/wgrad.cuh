@@ -54,11 +54,12 @@ struct WgradResCfg {
     static constexpr int BAR_BYTES = 256;
     // the group tables (offsets, order) are read through L1, not staged: the
     // shared memory goes to the resident slab, the ring and the store staging
-    static constexpr int SMEM_BYTES = 1024 + B_BYTES + STAGES * A_BYTES + EPI_STAGE_BYTES + BAR_BYTES;
+    static constexpr int DATA_BYTES = B_BYTES + STAGES * A_BYTES + EPI_STAGE_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + DATA_BYTES + BAR_BYTES + 16;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, true, true);
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert(EPI_BUFS >= 1 && EPI_BUFS <= 4, "staging buffers per warp");
-    static_assert((2 * STAGES + KB_MAX + 6) * 8 + 8 <= BAR_BYTES, "barrier block");
+    static_assert((2 * STAGES + KB_MAX + 7) * 8 <= BAR_BYTES, "barrier block");
 };
 
 struct WUnit {
@@ -97,26 +98,27 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t *blk, int chunks, int val
     }
 }
 
+// One resident weight-gradient phase run by every thread of the CTA.
+//   smem       1024-byte aligned: C::DATA_BYTES of resident slab, A ring and staging
+//   bar_block  C::BAR_BYTES of barriers for this phase
+//   tmem_base  TMEM columns [0, C::TMEM_COLS) allocated by the caller
+// Starts and ends with a CTA-wide barrier.
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, 1)
-    wgrad_resident_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                          const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
-                          const GemmArgs args)
+__device__ __forceinline__ void wgrad_resident_phase(uint8_t *smem, uint64_t *bar_block, uint32_t tmem_base,
+                                                     const CUtensorMap &tmA, const CUtensorMap &tmB,
+                                                     const CUtensorMap &tmO, const CUtensorMap &tmO2,
+                                                     const GemmArgs &args)
 {
-    griddep_enter();
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sB = smem;                                        // resident B: KB_MAX blocks
     uint8_t *sA = sB + C::B_BYTES;                             // A ring: STAGES blocks
     uint32_t *epi_stage = reinterpret_cast<uint32_t *>(sA + C::STAGES * C::A_BYTES);
-    uint64_t *afull = reinterpret_cast<uint64_t *>(reinterpret_cast<uint8_t *>(epi_stage) + C::EPI_STAGE_BYTES);
+    uint64_t *afull = bar_block;
     uint64_t *aempty = afull + C::STAGES;
     uint64_t *bfull = aempty + C::STAGES;
     uint64_t *bempty = bfull + C::KB_MAX;
     uint64_t *accf = bempty + 1;
     uint64_t *acce = accf + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acce + 2);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(acce + 2);
     uint64_t *drain_bar = acce + 3;                            // MMA drain on abort
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,13 +145,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tma_prefetch_desc(&tmO);
             tma_prefetch_desc(&tmO2);
         }
-    } else if (warp == 1) {
-        tmem_alloc(tmem_slot, C::TMEM_COLS);
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+    fence_proxy_async_global();          // operands an earlier phase of the launch wrote
     const int nbig = count_big_groups(args.offsets, args.gorder, G, args.k_split);
     const int m_chunks = (args.m_tiles + args.m_per_unit - 1) / args.m_per_unit;
     const int total = (G - nbig) * args.n_tiles * m_chunks;
@@ -203,9 +203,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 if (!ok) break;
             }
         }
-        if (*abort_flag && lane == 0) {
-            // another role gave up: let this producer's last loads land (bounded) before
-            // the CTA releases its shared memory
+        if (lane == 0) {
+            // the last fills: after an abort, let their loads land (bounded) before the CTA
+            // releases its shared memory; otherwise wait until the MMA has released them, so
+            // that no arrival on this phase's barriers is still in flight when it ends
+            const bool aborted = *abort_flag != 0;
             int s2 = stage;
             uint32_t ph = phase;
             for (int i = 0; i < min(fills, C::STAGES); ++i) {
@@ -213,10 +215,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     s2 = C::STAGES - 1;
                     ph ^= 1u;
                 }
-                mbar_drain(&afull[s2], ph);
+                mbar_drain(aborted ? &afull[s2] : &aempty[s2], ph);
             }
-            for (int kb = 0; kb < C::KB_MAX; ++kb)
-                if (bfilled & (1u << kb)) mbar_drain(&bfull[kb], ((bfill >> kb) & 1u) ^ 1u);
+            if (aborted) {
+                for (int kb = 0; kb < C::KB_MAX; ++kb)
+                    if (bfilled & (1u << kb)) mbar_drain(&bfull[kb], ((bfill >> kb) & 1u) ^ 1u);
+            } else if (bfilled) {
+                mbar_drain(bempty, bphase ^ 1u);      // the resident block of the last unit released
+            }
         }
     } else if (warp >= C::PULL_WARP0) {
         // ------------------------------------------------------------ pull warps (gathered operand)
@@ -230,6 +236,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const size_t ld = static_cast<size_t>(args.gather_ld) * 2;
         int stage = 0;
         uint32_t phase = 0, bphase = 0;
+        int pfills = 0;                  // A ring stages these warps filled
+        bool pfilled = false;            // resident block filled at least once
         bool ok = true;
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             const WUnit w = decode_unit(u, args, nbig, m_chunks);
@@ -246,6 +254,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 ok = mbar_wait(bempty, bphase ^ 1u, abort_flag, status);
                 if (!ok) break;
                 bphase ^= 1u;
+                pfilled = true;
 #pragma unroll
                 for (int kb = 0; kb < C::KB_MAX; ++kb) {
                     if (kb >= w.nkb) break;
@@ -291,6 +300,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                         }
                         fence_proxy_async_smem();
                         cp_async_arrive_noinc(&afull[stage]);
+                        ++pfills;
                         if (++stage == C::STAGES) {
                             stage = 0;
                             phase ^= 1u;
@@ -300,6 +310,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             }
         }
         cp_async_wait_all();             // nothing of this thread still lands in shared memory
+        if (p == 0 && !*abort_flag) {
+            // what the pull warps filled last has been released by the MMA (see the producer)
+            if constexpr (C::B_GATHER) {
+                if (pfilled) mbar_drain(bempty, bphase ^ 1u);
+            } else {
+                int s2 = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < min(pfills, C::STAGES); ++i) {
+                    if (--s2 < 0) {
+                        s2 = C::STAGES - 1;
+                        ph ^= 1u;
+                    }
+                    mbar_drain(&aempty[s2], ph);
+                }
+            }
+        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         int stage = 0, acc = 0;
@@ -429,12 +455,34 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 }
             }
         }
-        if (lane == 0) bulk_wait0();
+        if (lane == 0) {
+            bulk_wait0();
+            fence_proxy_async_global();
+        }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    wgrad_resident_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
+                          const GemmArgs args)
+{
+    griddep_enter();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::DATA_BYTES);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(bars) + C::BAR_BYTES);
+    if ((threadIdx.x >> 5) == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    wgrad_resident_phase<C>(smem, bars, tmem_base, tmA, tmB, tmO, tmO2, args);
+    if ((threadIdx.x >> 5) == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
     }

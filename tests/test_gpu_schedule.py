@@ -108,10 +108,20 @@ def test_persistent_forward_equals_split_forward(wl):
     for k, v in _saved(layer, wl.mxfp8).items():
         assert _same(v, saved_s[k]), f"saved tensor {k} differs"
     if training:
-        g_p = layer.backward(x, dy)        # persistent schedule: the backward's launches use PDL
+        g_p = layer.backward(x, dy)        # persistent schedule: one launch
+        assert abi.moe_launch_count() == 1
         torch.cuda.synchronize()
+        assert layer.status() == 0
         for k, v in g_s.items():
-            assert _same(g_p[k], v), f"gradient {k} differs"
+            assert _same(g_p[k], v), f"gradient {k} differs (persistent backward)"
+        abi.moe_set_schedule(abi.MOK_SCHEDULE_SPLIT_PDL)
+        try:
+            g_d = layer.backward(x, dy)    # split launches with PDL
+            torch.cuda.synchronize()
+        finally:
+            abi.moe_set_schedule(abi.MOK_SCHEDULE_PERSISTENT)
+        for k, v in g_s.items():
+            assert _same(g_d[k], v), f"gradient {k} differs (PDL split backward)"
     # reruns of the persistent forward: byte-identical (a fresh launch epoch each time)
     for _ in range(3):
         y2, _, _ = _forward(layer, x, abi.MOK_SCHEDULE_PERSISTENT)
@@ -141,16 +151,21 @@ def test_device_phase_stamps():
     dev = torch.device("cuda")
     layer = MoELayer(cfg_for(wl), _params(wl, dev), training=True, device=dev)
     x = synth.draw_x(wl, "cpu").to(dev)
+    dy = synth.draw_dy(wl, "cpu").to(dev)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     buf = torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev)
-    abi.moe_trace_device(buf.data_ptr(), buf.numel() * 8)
+    bbuf = torch.zeros_like(buf)
+    abi.moe_trace_device(buf.data_ptr(), buf.numel() * 8, bbuf.data_ptr(), bbuf.numel() * 8)
     try:
         layer.forward(x)
+        layer.backward(x, dy)
         torch.cuda.synchronize()
     finally:
         abi.moe_trace_device(None, 0)
-    t = buf.view(abi.MOK_TRACE_POINTS, sms).cpu().numpy()
-    assert (t > 0).all()
-    assert (np.diff(t, axis=0) >= 0).all()           # every CTA passes the points in order
-    # the phases behind the first grid barrier end after every CTA finished the first phase
-    assert (t[2:].min(axis=1) >= t[1].max()).all()
+    for b in (buf, bbuf):
+        t = b.view(abi.MOK_TRACE_POINTS, sms).cpu().numpy()
+        assert (t > 0).all()
+        assert (np.diff(t, axis=0) >= 0).all()           # every CTA passes the points in order
+        # the phases behind the first grid barrier end after every CTA finished the first phase
+        assert (t[2:].min(axis=1) >= t[1].max()).all()
+    assert buf.view(abi.MOK_TRACE_POINTS, sms).max() <= bbuf.view(abi.MOK_TRACE_POINTS, sms).min()
