@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--schedule", default="persistent", choices=["persistent", "split"],
                     help="forward schedule of the timed steps (the A/B leg runs both)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-ab", action="store_true", help="skip the schedule A/B legs (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--extra-workloads", default="small,dsv3_zipf",
@@ -476,13 +477,15 @@ def main():
 
     # forward A/B: split schedule (events per step, the per-GEMM attribution below) against
     # the persistent one, forward only
-    ab = forward_ab(layer, x, y, K)
-    for n_i, name in enumerate(FWD_PHASES):
-        phase["split_" + name] = ab["split"]["phases_ms"][name]
-    layer.forward(x, y)
-    bab = backward_ab(layer, x, dy, grads, K)
-    for name in BWD_PHASES:
-        phase["split_" + name] = bab["split"]["phases_ms"][name]
+    ab = bab = None
+    if not args.no_ab:
+        ab = forward_ab(layer, x, y, K)
+        for n_i, name in enumerate(FWD_PHASES):
+            phase["split_" + name] = ab["split"]["phases_ms"][name]
+        layer.forward(x, y)
+        bab = backward_ab(layer, x, dy, grads, K)
+        for name in BWD_PHASES:
+            phase["split_" + name] = bab["split"]["phases_ms"][name]
 
     pk = peaks()
     alg = algorithmic(wl, counts)
@@ -507,6 +510,8 @@ def main():
     # every GEMM phase against both measured peaks (algorithmic bytes and FLOPs / its event time)
     phase_roofline = {}
     for name, (fl, nb) in list(alg.items()) + [(fwd_name, kern[fwd_name]), (bwd_name, kern[bwd_name])]:
+        if name not in phase and "split_" + name not in phase:
+            continue
         t = (phase[name] if name in phase else phase["split_" + name]) / 1e3
         phase_roofline[name] = {"ms": round(t * 1e3, 4), "hbm_frac": round(nb / t / 1e9 / pk["hbm_gbs"], 4),
                                 "tc_frac_sustained": round(fl / t / 1e12 / pk["bf16_sustained"], 4)}
@@ -532,14 +537,15 @@ def main():
     for name in ([] if args.extra_workloads in ("", "none") else args.extra_workloads.split(",")):
         ewl = synth.WORKLOADS[name]
         extra[name] = bf16_workload_run(synth.scaled(ewl, seed=ewl.seed + 1000 * rank), dev, K, args.warmup, world,
-                                        dist, pk)
+                                        dist, pk, not args.no_ab)
         torch.cuda.empty_cache()
 
     # ---------------- MXFP8 forward (block-scaled e4m3) on its own workload
     mx = None
     if args.mx_workload and args.mx_workload != "none":
         mwl = synth.WORKLOADS[args.mx_workload]
-        mx = mxfp8_run(synth.scaled(mwl, seed=mwl.seed + 1000 * rank), dev, K, args.warmup, world, dist, pk)
+        mx = mxfp8_run(synth.scaled(mwl, seed=mwl.seed + 1000 * rank), dev, K, args.warmup, world, dist, pk,
+                       not args.no_ab)
 
     if rank == 0:
         line = {
@@ -584,7 +590,7 @@ def main():
         dist.destroy_process_group()
 
 
-def bf16_workload_run(wl, dev, K, warmup, world, dist, pk):
+def bf16_workload_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
     """Tokens/s and tensor-core fractions of the BF16 layer on another workload (forward, and
     backward when the workload has one), per-phase CUDA events on the layer's stream."""
     import torch
@@ -628,9 +634,9 @@ def bf16_workload_run(wl, dev, K, warmup, world, dist, pk):
     ms = float(t.item()) / K
     fwd_ms = statistics.mean(fev[i][0].elapsed_time(fev[i][-1]) for i in range(K))
     bwd_ms = statistics.mean(bev[i][0].elapsed_time(bev[i][-1]) for i in range(K)) if wl.backward else 0.0
-    ab = forward_ab(layer, x, y, K)
+    ab = forward_ab(layer, x, y, K) if do_ab else None
     bab = None
-    if wl.backward:
+    if wl.backward and do_ab:
         layer.forward(x, y)
         bab = backward_ab(layer, x, dy, grads, K)
     fwd_flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
@@ -653,7 +659,7 @@ def bf16_workload_run(wl, dev, K, warmup, world, dist, pk):
     return out
 
 
-def mxfp8_run(wl, dev, K, warmup, world, dist, pk):
+def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
     """Forward tokens/s of the MXFP8 layer (weights quantised once, outside the timed region)."""
     import torch
     from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, moe_trace_events, quantize_mxfp8_weights, synth
@@ -694,10 +700,15 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk):
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item()) / K
-    ab = forward_ab(layer, x, y, K)
-    phases = ab["split"]["phases_ms"]              # per-step times: the split schedule's events
+    if do_ab:
+        ab = forward_ab(layer, x, y, K)
+        phases = ab["split"]["phases_ms"]          # per-step times: the split schedule's events
+    else:
+        ab = None
+        phases = {n: statistics.mean(fev[i][j].elapsed_time(fev[i][j + 1]) for i in range(K))
+                  for j, n in enumerate(FWD_PHASES)}
     flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
-    gemm_ms = phases["gate_up_gemm"] + phases["down_gemm"]
+    gemm_ms = max(1e-9, phases["gate_up_gemm"] + phases["down_gemm"])
     del layer, params, x, y
     torch.cuda.empty_cache()
     # the FP8 denominator: a library FP8 GEMM measured on this GPU in this run; the MXFP8
@@ -714,7 +725,8 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk):
             "tc_peak_frac": flops / (ms / 1e3) / 1e12 / peak,
             "tc_peak_frac_of_sustained": flops / (ms / 1e3) / 1e12 / fp8["sustained_tflops"],
             "expert_gemm_tc_peak_frac": flops / (gemm_ms / 1e3) / 1e12 / peak,
-            "gate_up_tc_peak_frac": 4 * wl.H * wl.I * wl.T * (wl.k + wl.S) / (phases["gate_up_gemm"] / 1e3) / 1e12 / peak,
+            "gate_up_tc_peak_frac": 4 * wl.H * wl.I * wl.T * (wl.k + wl.S) / (max(1e-9, phases["gate_up_gemm"]) / 1e3)
+            / 1e12 / peak,
             "device_status": status}
 
 
