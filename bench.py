@@ -231,93 +231,96 @@ def stamp_phases(bufs, sms, names=None):
     return {n: round(float(v) / len(bufs) / 1e6, 4) for n, v in zip(names or STAMP_PHASES, acc)}
 
 
-def forward_ab(layer, x, y, K):
-    """Forward only, K steps each: the split schedule with an event per step, then the
-    persistent schedule (one launch) with its device stamps."""
+def _ab(layer, run, K, legs, trace_split, stamp_names):
+    """Interleaved A/B of the schedules: in each of K rounds every leg runs once, timed
+    with CUDA events around the pass (power and clock drift then hits every leg
+    alike).  The split leg also records an event per step, the persistent leg its
+    device stamps."""
     import torch
-    from mixture_experts_layer_persistent_b200 import abi, moe_trace_events
-    dev = x.device
+    from mixture_experts_layer_persistent_b200 import abi
+    dev = layer.device
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     mk = lambda: torch.cuda.Event(enable_timing=True)
-    out = {}
     restore = abi.moe_get_schedule()
-    for name, sched in (("split", abi.MOK_SCHEDULE_SPLIT), ("split_pdl", abi.MOK_SCHEDULE_SPLIT_PDL),
-                        ("persistent", abi.MOK_SCHEDULE_PERSISTENT)):
+    for name, sched in legs:                       # warm-up of every leg
         abi.moe_set_schedule(sched)
-        for _ in range(2):
-            layer.forward(x, y)
-        fev = [[mk() for _ in range(abi.MOK_FWD_PHASES + 1)] for _ in range(K)]
-        for e in [e for ev in fev for e in ev]:
+        run(None, None)
+        run(None, None)
+    n_ev = (abi.MOK_FWD_PHASES if trace_split == "fwd" else abi.MOK_BWD_PHASES) + 1
+    rec = {name: {"t": [], "ev": [], "st": []} for name, _ in legs}
+    for i in range(K):
+        for name, sched in legs:
+            abi.moe_set_schedule(sched)
+            s, e = mk(), mk()
+            ev = [mk() for _ in range(n_ev)] if name == "split" else None
+            st = torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) if name == "persistent" else None
+            s.record()
+            run(ev, st)
             e.record()
-        bufs = [torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) for _ in range(K)]
-        torch.cuda.synchronize()
-        s, e = mk(), mk()
-        s.record()
-        for i in range(K):
-            if name == "split":          # events between the steps (they would cut the PDL overlap)
-                moe_trace_events([ev.cuda_event for ev in fev[i]], None)
-            abi.moe_trace_device(bufs[i].data_ptr(), bufs[i].numel() * 8)
-            layer.forward(x, y)
-            launches = abi.moe_launch_count()
-        e.record()
-        torch.cuda.synchronize()
+            rec[name]["t"].append((s, e))
+            rec[name]["ev"].append(ev)
+            rec[name]["st"].append(st)
+            rec[name]["launches"] = abi.moe_launch_count()
+    torch.cuda.synchronize()
+    abi.moe_set_schedule(restore)
+    out = {}
+    for name, _ in legs:
+        r = rec[name]
+        o = {"ms": statistics.mean(a.elapsed_time(b) for a, b in r["t"]), "launches": r["launches"]}
+        if name == "split":
+            names = FWD_PHASES if trace_split == "fwd" else BWD_PHASES
+            o["phases_ms"] = {n: round(statistics.mean(ev[j].elapsed_time(ev[j + 1]) for ev in r["ev"]), 4)
+                              for j, n in enumerate(names)}
+        if name == "persistent":
+            o["device_phases_ms"] = stamp_phases(r["st"], sms, stamp_names)
+        out[name] = o
+    out["persistent_over_split_speedup"] = out["split"]["ms"] / out["persistent"]["ms"]
+    out["split_pdl_over_split_speedup"] = out["split"]["ms"] / out["split_pdl"]["ms"]
+    out["order"] = "interleaved: each round runs split, split_pdl, persistent once"
+    return out
+
+
+def _legs():
+    from mixture_experts_layer_persistent_b200 import abi
+    return (("split", abi.MOK_SCHEDULE_SPLIT), ("split_pdl", abi.MOK_SCHEDULE_SPLIT_PDL),
+            ("persistent", abi.MOK_SCHEDULE_PERSISTENT))
+
+
+def forward_ab(layer, x, y, K):
+    """Forward only: split, PDL-split and persistent schedules, interleaved."""
+    from mixture_experts_layer_persistent_b200 import abi, moe_trace_events
+
+    def run(ev, st):
+        if ev is not None:
+            moe_trace_events([e.cuda_event for e in ev], None)
+        if st is not None:
+            abi.moe_trace_device(st.data_ptr(), st.numel() * 8)
+        layer.forward(x, y)
         moe_trace_events(None, None)
         abi.moe_trace_device(None, 0)
-        r = {"ms_per_fwd": s.elapsed_time(e) / K, "launches_per_fwd": launches}
-        if name == "split":
-            r["phases_ms"] = {n: round(statistics.mean(fev[i][j].elapsed_time(fev[i][j + 1]) for i in range(K)), 4)
-                              for j, n in enumerate(FWD_PHASES)}
-        elif name == "persistent":
-            r["device_phases_ms"] = stamp_phases(bufs, sms)
-        out[name] = r
-    abi.moe_set_schedule(restore)
-    out["persistent_over_split_speedup"] = out["split"]["ms_per_fwd"] / out["persistent"]["ms_per_fwd"]
-    out["persistent_over_split_pdl_speedup"] = out["split_pdl"]["ms_per_fwd"] / out["persistent"]["ms_per_fwd"]
+
+    out = _ab(layer, run, K, _legs(), "fwd", STAMP_PHASES)
+    for leg in ("split", "split_pdl", "persistent"):     # names kept for readers of earlier lines
+        out[leg]["ms_per_fwd"] = out[leg]["ms"]
     return out
 
 
 def backward_ab(layer, x, dy, grads, K):
-    """Backward only, K steps each: plain split launches (an event per step), PDL split
-    launches, and the persistent launch (device stamps)."""
-    import torch
+    """Backward only: split, PDL-split and persistent schedules, interleaved."""
     from mixture_experts_layer_persistent_b200 import abi, moe_trace_events
-    dev = x.device
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    mk = lambda: torch.cuda.Event(enable_timing=True)
-    restore = abi.moe_get_schedule()
-    out = {}
-    for name, sched in (("split", abi.MOK_SCHEDULE_SPLIT), ("split_pdl", abi.MOK_SCHEDULE_SPLIT_PDL),
-                        ("persistent", abi.MOK_SCHEDULE_PERSISTENT)):
-        abi.moe_set_schedule(sched)
-        for _ in range(2):
-            layer.backward(x, dy, grads)
-        bev = [[mk() for _ in range(abi.MOK_BWD_PHASES + 1)] for _ in range(K)]
-        for e in [e for ev in bev for e in ev]:
-            e.record()
-        bufs = [torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) for _ in range(K)]
-        torch.cuda.synchronize()
-        s, e = mk(), mk()
-        s.record()
-        for i in range(K):
-            if name == "split":
-                moe_trace_events(None, [ev.cuda_event for ev in bev[i]])
-            abi.moe_trace_device(None, 0, bufs[i].data_ptr(), bufs[i].numel() * 8)
-            layer.backward(x, dy, grads)
-            launches = abi.moe_launch_count()
-        e.record()
-        torch.cuda.synchronize()
+
+    def run(ev, st):
+        if ev is not None:
+            moe_trace_events(None, [e.cuda_event for e in ev])
+        if st is not None:
+            abi.moe_trace_device(None, 0, st.data_ptr(), st.numel() * 8)
+        layer.backward(x, dy, grads)
         moe_trace_events(None, None)
         abi.moe_trace_device(None, 0)
-        r = {"ms_per_bwd": s.elapsed_time(e) / K, "launches_per_bwd": launches}
-        if name == "split":
-            r["phases_ms"] = {n: round(statistics.mean(bev[i][j].elapsed_time(bev[i][j + 1]) for i in range(K)), 4)
-                              for j, n in enumerate(BWD_PHASES)}
-        elif name == "persistent":
-            r["device_phases_ms"] = stamp_phases(bufs, sms, BWD_STAMP_PHASES)
-        out[name] = r
-    abi.moe_set_schedule(restore)
-    out["persistent_over_split_speedup"] = out["split"]["ms_per_bwd"] / out["persistent"]["ms_per_bwd"]
-    out["split_pdl_over_split_speedup"] = out["split"]["ms_per_bwd"] / out["split_pdl"]["ms_per_bwd"]
+
+    out = _ab(layer, run, K, _legs(), "bwd", BWD_STAMP_PHASES)
+    for leg in ("split", "split_pdl", "persistent"):
+        out[leg]["ms_per_bwd"] = out[leg]["ms"]
     return out
 
 

@@ -47,7 +47,22 @@ __device__ __forceinline__ void combine_elem(long long i, const Slot *__restrict
     const int kk = k + S;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const Slot *row = O + (size_t)t * kk * H + c;
-    for (int j = 0; j < kk; ++j) {
+    // slots in groups of four: the four rows' loads are issued before their sums,
+    // which still run in ascending j
+    int j = 0;
+    for (; j + 4 <= kk; j += 4) {
+        float v[4][8], w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            w[u] = j + u < k ? topk_w[(size_t)t * k + j + u] : 1.0f;
+            load8(row + (size_t)(j + u) * H, v[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = fmaf(w[u], v[u][q], acc[q]);
+    }
+    for (; j < kk; ++j) {
         const float w = j < k ? topk_w[(size_t)t * k + j] : 1.0f;
         float v[8];
         load8(row + (size_t)j * H, v);
@@ -115,18 +130,15 @@ __global__ void __launch_bounds__(256) slot_grad_kernel(const float *__restrict_
 
 // Router weight gradient, pass 1: for each chunk of up to `chunk_rows` sorted
 // rows of one expert and 256 columns, partial[chunk, cols] = sum over the
-// chunk's rows (ascending) of dl(row) x[token(row), cols].  8 warps take rows
-// r = warp (mod 8); their sums are added in warp order.
-// One (chunk, 256-column block) item by the first 256 threads of the CTA
-// (s_acc: 8 x 256 floats of shared memory).  Every thread of the CTA calls it:
-// it contains a CTA-wide barrier.
-__device__ __forceinline__ void drouter_partial_item(int chunk, int h0, const __nv_bfloat16 *__restrict__ x,
+// chunk's rows of dl(row) x[token(row), cols], in a fixed order: the rows
+// r0 + w, r0 + w + 8, ... (w = 0..7) are summed separately in ascending order,
+// then the eight sums in order of w.  One warp per item; lane = 8 columns.
+__device__ __forceinline__ void drouter_partial_item(int chunk, int h0, int lane, const __nv_bfloat16 *__restrict__ x,
                                                      const float *__restrict__ dl, const int *__restrict__ offsets,
                                                      const int *__restrict__ chunk_start,
                                                      const int *__restrict__ perm, float *__restrict__ partial,
-                                                     int H, int E, int k, int chunk_rows, float (*s_acc)[256])
+                                                     int H, int E, int k, int chunk_rows)
 {
-    const bool active = threadIdx.x < 256;
     int lo = 0, hi = E - 1;     // expert owning this chunk: largest e with chunk_start[e] <= chunk
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -135,30 +147,42 @@ __device__ __forceinline__ void drouter_partial_item(int chunk, int h0, const __
     const int e = lo;
     const int r0 = offsets[e] + (chunk - chunk_start[e]) * chunk_rows;
     const int r1 = min(offsets[e + 1], r0 + chunk_rows);
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int r = r0 + warp; active && r < r1; r += 8) {
-        const int s = perm[r];                  // t * k + slot
-        const float d = dl[s];
-        const int tok = s / k;
-        float v[8];
-        unpack8(*reinterpret_cast<const uint4 *>(x + (size_t)tok * H + h0 + lane * 8), v);
+    float acc[8][8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] = fmaf(d, v[q], acc[q]);
-    }
-    if (active) {
+    for (int w = 0; w < 8; ++w)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) s_acc[warp][lane * 8 + q] = acc[q];
+        for (int q = 0; q < 8; ++q) acc[w][q] = 0.0f;
+    for (int r = r0; r < r1; r += 8) {
+        float v[8][8], d[8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {             // eight rows' loads in flight
+            if (r + w < r1) {
+                const int s = perm[r + w];        // t * k + slot
+                d[w] = dl[s];
+                unpack8(*reinterpret_cast<const uint4 *>(x + (size_t)(s / k) * H + h0 + lane * 8), v[w]);
+            }
+        }
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+            if (r + w < r1)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[w][q] = fmaf(d[w], v[w][q], acc[w][q]);
     }
-    __syncthreads();
-    if (active) {
+    float out[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
         float s = 0.0f;
-        for (int w = 0; w < 8; ++w) s += s_acc[w][threadIdx.x];
-        partial[(size_t)chunk * H + h0 + threadIdx.x] = s;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) s += acc[w][q];
+        out[q] = s;
     }
-    __syncthreads();                            // s_acc is free again
+    float4 *dst = reinterpret_cast<float4 *>(partial + (size_t)chunk * H + h0 + lane * 8);
+    dst[0] = make_float4(out[0], out[1], out[2], out[3]);
+    dst[1] = make_float4(out[4], out[5], out[6], out[7]);
 }
 
+// items = (chunk, 256-column block) pairs, one warp each; grid covers an upper bound
+// of the chunk count
 __global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat16 *__restrict__ x,
                                                               const float *__restrict__ dl,
                                                               const int *__restrict__ offsets,
@@ -168,13 +192,13 @@ __global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat1
                                                               int chunk_rows)
 {
     griddep_enter();
-    __shared__ float s_acc[8][256];
-    if (static_cast<int>(blockIdx.x) >= chunk_start[E]) return;
-    drouter_partial_item(blockIdx.x, blockIdx.y * 256, x, dl, offsets, chunk_start, perm, partial, H, E, k, chunk_rows,
-                         s_acc);
+    const int hb = H / 256;
+    const int item = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (item >= chunk_start[E] * hb) return;
+    drouter_partial_item(item / hb, (item % hb) * 256, threadIdx.x & 31, x, dl, offsets, chunk_start, perm, partial, H,
+                         E, k, chunk_rows);
 }
 
-// Router weight gradient, pass 2: dWr[e, h] = sum over the expert's chunks in order.
 __device__ __forceinline__ void drouter_reduce_elem(long long i, const float *__restrict__ partial,
                                                    const int *__restrict__ chunk_start, float *__restrict__ dWr, int H)
 {
@@ -205,7 +229,17 @@ __device__ __forceinline__ void dx_combine_elem(long long i, const float *__rest
     const int kk = k + S;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const float *row = dXs + (size_t)t * kk * H + c;
-    for (int j = 0; j < kk; ++j) {
+    int j = 0;
+    for (; j + 4 <= kk; j += 4) {                  // four rows' loads in flight, sums in ascending j
+        float v[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) load8(row + (size_t)(j + u) * H, v[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] += v[u][q];
+    }
+    for (; j < kk; ++j) {
         float v[8];
         load8(row + (size_t)j * H, v);
 #pragma unroll

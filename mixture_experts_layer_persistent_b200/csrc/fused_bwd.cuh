@@ -89,7 +89,6 @@ struct FusedBwdCfg {
     static_assert(DgradDown::THREADS <= kFusedThreads && WgradDown::THREADS <= kFusedThreads &&
                   DgradGU::THREADS <= kFusedThreads && WgradGU::THREADS <= kFusedThreads &&
                   ResDown::THREADS <= kFusedThreads && ResGU::THREADS <= kFusedThreads, "phase roles fit the launch");
-    static_assert(8 * 256 * 4 <= REGION, "router-gradient scratch");
 };
 
 __device__ __forceinline__ void fused_bwd_stamp(const FusedBwdArgs &a, int point)
@@ -165,16 +164,15 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     // ---------------------------------------------------------------- Q5
     if (alive) {
-        float(*s_acc)[256] = reinterpret_cast<float(*)[256]>(smem);
-        const int n_chunks = a.chunk_start[a.E];
+        const int n_items = a.chunk_start[a.E] * (a.H / 256);
         const int hb = a.H / 256;
-        for (int item = blockIdx.x; item < n_chunks * hb; item += gridDim.x)
-            drouter_partial_item(item / hb, (item % hb) * 256, a.x, a.dl, a.offsets, a.chunk_start, a.perm, a.partial,
-                                 a.H, a.E, a.k, a.chunk_rows, s_acc);
+        const int nw = kFusedThreads / 32;
+        for (int item = blockIdx.x * nw + warp; item < n_items; item += gridDim.x * nw)
+            drouter_partial_item(item / hb, (item % hb) * 256, threadIdx.x & 31, a.x, a.dl, a.offsets, a.chunk_start,
+                                 a.perm, a.partial, a.H, a.E, a.k, a.chunk_rows);
         const long long n = static_cast<long long>(a.T) * (a.H / 8);
         for (long long i = gtid; i < n; i += gstride)
             dx_combine_elem(i, a.dxs, a.dl, a.topk_idx, a.router_w, a.dx, a.H, a.k, a.S);
-        __syncthreads();                            // the router-gradient scratch is free again
         tc_fence_after();
         gemm_phase<typename F::WgradGU>(smem, gbars + 3 * GB, aux, tmem_base, m.w4A, m.w4A, m.w4A, m.w4O, m.w4O2,
                                         m.w4O, a.g4);
