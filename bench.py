@@ -248,12 +248,19 @@ def _ab(layer, run, K, legs, trace_split, stamp_names):
         run(None, None)
     n_ev = (abi.MOK_FWD_PHASES if trace_split == "fwd" else abi.MOK_BWD_PHASES) + 1
     rec = {name: {"t": [], "ev": [], "st": []} for name, _ in legs}
+    # events and stamp buffers made before the rounds; torch creates a CUDA event at its
+    # first record, so every event is recorded once before the library records it
+    evs = [[mk() for _ in range(n_ev)] for _ in range(K)]
+    for e in [e for ev in evs for e in ev]:
+        e.record()
+    sts = [torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) for _ in range(K)]
+    torch.cuda.synchronize()
     for i in range(K):
         for name, sched in legs:
             abi.moe_set_schedule(sched)
             s, e = mk(), mk()
-            ev = [mk() for _ in range(n_ev)] if name == "split" else None
-            st = torch.zeros(abi.MOK_TRACE_POINTS * sms, dtype=torch.int64, device=dev) if name == "persistent" else None
+            ev = evs[i] if name == "split" else None
+            st = sts[i] if name == "persistent" else None
             s.record()
             run(ev, st)
             e.record()
@@ -324,21 +331,30 @@ def backward_ab(layer, x, dy, grads, K):
     return out
 
 
-def measured_traffic(wl, phase):
-    """DRAM bytes per launch of `phase` from the committed ncu capture, or None
-    when the workload differs or the kernel sources changed since the capture."""
+def source_hash():
+    """sha256 over the CUDA sources: DRAM counters are reported only for the sources they
+    were taken from."""
     import glob
     import hashlib
-    path = os.path.join(ROOT, "profiles", "dram_traffic_dsv3.json")
-    if wl.name != "dsv3" or not os.path.exists(path):
-        return None
-    rec = json.load(open(path))
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "mixture_experts_layer_persistent_b200", "csrc", "*"))):
         h.update(open(f, "rb").read())
-    if h.hexdigest() != rec["source_sha256"]:
+    return h.hexdigest()
+
+
+def measured_traffic(wl, kernel):
+    """DRAM bytes per launch of `kernel` on this workload, from the committed ncu capture of
+    the 16-expert workload of the same expert shape and rows per expert (dsv3_e16_r128,
+    profiles/dram_traffic_dsv3_e16.json) scaled by the ratio of tokens (every expert-,
+    row- and token-proportional stream scales with it), or None when the workload differs
+    or the kernel sources changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic_dsv3_e16.json")
+    if wl.name != "dsv3" or not os.path.exists(path):
         return None
-    return rec["per_launch_bytes"].get(phase)
+    rec = json.load(open(path))
+    if rec.get("source_sha256") != source_hash() or kernel not in rec["per_launch_bytes"]:
+        return None
+    return int(rec["per_launch_bytes"][kernel] * wl.T / rec["tokens"])
 
 
 # ------------------------------------------------------------------ CPU oracle sample

@@ -18,8 +18,7 @@
 //       in its dispatch chunk's histogram (integer atomics)
 //   --- grid barrier
 //   P3  per dispatch chunk: scan of the histograms and stable placement of the
-//       chunk's (token, slot) rows (every CTA derives its own chunk's base rows);
-//       MXFP8: then (after a grid barrier) x's scales packed per M tile
+//       chunk's (token, slot) rows (every CTA derives its own chunk's base rows)
 //   --- grid barrier
 //   P4  gate/up GEMM with the SwiGLU epilogue, then the down GEMM with the push
 //       epilogue.  No barrier between them: each gate/up epilogue warp counts
@@ -249,20 +248,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         int *s_cnt = s_base + 256;
         for (int c = blockIdx.x; c < a.n_chunks; c += gridDim.x)
             dispatch_scan_place_chunk(a.da, c, a.n_chunks, c == 0, s_mask, s_base, s_cnt);
-    }
-    if constexpr (MX) {
-        // x's scales packed per M tile of the gate/up GEMM, once every row is placed
-        alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
-        if (alive) {
-            int *s_off = reinterpret_cast<int *>(smem);
-            int *s_mt = s_off + kMaxGroupsQ + 1;
-            if (threadIdx.x == 0) load_tile_tables(a.ga.offsets, a.ga.num_groups, s_off, s_mt);
-            __syncthreads();
-            const long long R = static_cast<long long>(a.T) * (a.k + a.S);
-            for (long long r = gtid; r < R; r += gstride)
-                pack_row_scales(r, a.ga.num_groups, s_off, s_mt, a.ga.row_token, a.xs, a.H / 32,
-                                const_cast<uint8_t *>(a.ga.sfa_packed));
-        }
     }
     fused_stamp(a, 4);
     alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);

@@ -62,9 +62,6 @@ struct GemmArgs {
     int gather_ld;                // elements per token row of gather_src
     // MXFP8 (block-scaled) operands: ue8m0 scales, one byte per 32 K-elements, rows of sf_ld bytes
     const uint8_t *sfa_src;       // scales of A's rows (token rows when A is gathered, sorted rows otherwise)
-    const uint8_t *sfa_packed;    // or null: A's scales already packed per M tile (pack_row_scales), one
-                                  // 512-byte block per (M tile, K block), fetched by the producer
-    int sfa_kb;                   // K blocks of A (blocks per M tile in sfa_packed)
     const uint8_t *sfb_src;       // scales of the routed groups' B rows (packed weight-scale layout)
     const uint8_t *sfb_src_s;     // scales of the shared groups' B rows (packed weight-scale layout)
     int sf_ld;                    // A scale bytes per row (K / 32)
@@ -540,7 +537,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                 bool ok = true;
                 if (lane == 0) {
                     ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status);
-                    if (ok) mbar_arrive_expect_tx(&full_bar[stage], C::TMA_BYTES + (C::MX && args.sfa_packed ? 512 : 0));
+                    if (ok) mbar_arrive_expect_tx(&full_bar[stage], C::TMA_BYTES);
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) goto producer_done;
@@ -589,11 +586,6 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
                         bulk_load(sf + 512, sb + (static_cast<long long>(kb) * rt + (r0 >> 7)) * 512, 512, fb);
                         bulk_load(sf + 1024, sb + (static_cast<long long>(kb) * rt + (r1 >> 7)) * 512, 512, fb);
-                        if (args.sfa_packed) {
-                            // A's scales of this K block: the M tile's packed 512-byte block
-                            const long long mt = s_tstart[t.g] / args.n_tiles + (t.m0 - s_off[t.g]) / BM;
-                            bulk_load(sf, args.sfa_packed + (mt * args.sfa_kb + kb) * 512, 512, fb);
-                        }
                     }
                 }
                 ++fills;
@@ -652,11 +644,9 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                     // scales come with B from the producer
                     const uint8_t *sfa = nullptr;
                     if constexpr (C::MX) {
-                        if (!args.sfa_packed) {
                         const int ar = p < t.rows ? (C::A_GATHER ? __ldg(args.row_token + t.m0 + p) : t.m0 + p)
                                                   : (C::A_GATHER ? 0 : t.m0);
                         sfa = args.sfa_src + (size_t)ar * args.sf_ld;
-                        }
                     }
                     for (int kb = 0; kb < t.nkb; ++kb) {
                         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status)) goto pull_done;
@@ -670,11 +660,9 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         }
                         if constexpr (C::MX) {
                             // SF atom layout: the 4 scales of row m at byte 16 (m % 32) + 4 (m / 32) of its 128-row block
-                            if (sfa) {
-                                uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
-                                const int at = 16 * (p & 31) + 4 * (p >> 5);
-                                cp_async4(sf + at, sfa + kb * 4);
-                            }
+                            uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
+                            const int at = 16 * (p & 31) + 4 * (p >> 5);
+                            cp_async4(sf + at, sfa + kb * 4);
                         }
                         cp_async_arrive_noinc(&full_bar[stage]);
                         if (++stage == C::STAGES) {

@@ -190,7 +190,6 @@ struct State {
     __nv_bfloat16 *gu, *h, *hw;
     float *O;                       // per-(token, slot) rows: fp32 (BF16), bf16 (MXFP8 forward)
     uint8_t *xq, *xs, *hq, *hs;     // MXFP8 operands
-    uint8_t *sfx;                   // MXFP8: x's scales packed per M tile of the gate/up GEMM
     int *sched;                     // [kSchedCounters] forward GEMM tile counters
     int *ready;                     // [n_mtiles] per-M-tile readiness (persistent forward)
     int *zero;                      // sched, ready and hist: the counters the persistent forward zeroes
@@ -239,10 +238,9 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
         st.hs = cv.take<uint8_t>(s.R * s.I / 32);
         st.xq = cv.take<uint8_t>(s.T * s.H);
         st.xs = cv.take<uint8_t>(s.T * s.H / 32);
-        st.sfx = cv.take<uint8_t>(static_cast<size_t>(s.R / BM + s.G + 1) * (s.H / 128) * 512);
     } else {
         st.h = cv.take<__nv_bfloat16>(s.R * s.I);
-        st.hq = st.hs = st.xq = st.xs = st.sfx = nullptr;
+        st.hq = st.hs = st.xq = st.xs = nullptr;
     }
     st.O = mx ? reinterpret_cast<float *>(cv.take<__nv_bfloat16>(s.T * s.kk * s.H)) : cv.take<float>(s.T * s.kk * s.H);
     st.bytes = align_up(cv.off, 256);
@@ -459,8 +457,6 @@ int build_fwd_plan(const moe_cfg &c, const void *x, const moe_params &p, const S
         ga.out_scales = st.hs;
         ga.gather_src = reinterpret_cast<const __nv_bfloat16 *>(st.xq);
         ga.sfa_src = st.xs;
-        ga.sfa_packed = st.sfx;
-        ga.sfa_kb = c.H / 128;
         ga.sfb_src = p.s_gate_up;
         ga.sfb_src_s = s.S ? p.ss_gate_up : p.s_gate_up;
         ga.sf_ld = c.H / 32;
@@ -484,7 +480,6 @@ int build_fwd_plan(const moe_cfg &c, const void *x, const moe_params &p, const S
         gd.ldo = c.H;
         gd.gather_src = nullptr;
         gd.sfa_src = st.hs;
-        gd.sfa_packed = nullptr;
         gd.sfb_src = p.s_down;
         gd.sfb_src_s = s.S ? p.ss_down : p.s_down;
         gd.sf_ld = c.I / 32;
@@ -568,10 +563,6 @@ int forward_split(const moe_cfg &c, const void *x, const moe_params &p, void *y,
         const long long xb = s.T * s.H / 32;
         MOK_TRY(launch_k(quantize_mxfp8_kernel, dim3(blocks_for(xb, 256)), dim3(256), 0, stream, "quantize_mxfp8_kernel",
                          static_cast<const __nv_bfloat16 *>(x), xb, st.xq, st.xs, static_cast<long long>(s.H / 32), 0ll));
-        MOK_TRY(launch_k(pack_row_scales_kernel, dim3(blocks_for(s.R, 256)), dim3(256), 0, stream,
-                         "pack_row_scales_kernel", static_cast<const int *>(st.offsets), static_cast<int>(s.G), s.R,
-                         static_cast<const int *>(st.row_token), static_cast<const uint8_t *>(st.xs),
-                         static_cast<int>(s.H / 32), st.sfx));
         MOK_TRY(launch_gemm<typename FusedCfg<true>::GateUp>(pl.m.gB, pl.m.gB, pl.m.gBs, pl.m.gO, pl.m.gO2, pl.m.gO3,
                                                             ga, dev.sms, stream));
         MOK_TRY(mark_fwd(3, stream));

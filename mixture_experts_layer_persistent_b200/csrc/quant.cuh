@@ -12,8 +12,6 @@
 
 namespace mok {
 
-constexpr int kMaxGroupsQ = 264;      // groups (routed + shared experts) a scale packing handles
-
 // Exponent of the block from the fp32 bit pattern of amax (exact integer logic):
 // amax = (1 + f) 2^p; 448 * 2^(p-8) = 1.75 * 2^p covers it iff f <= 0.75.
 __device__ __forceinline__ int mx_exponent(float amax)
@@ -80,56 +78,6 @@ __device__ __forceinline__ void quantize_block(long long b, const __nv_bfloat16 
     dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     const long long at = row_tiles ? packed_scale_offset(b / kb32, b % kb32, row_tiles) : b;
     scales[at] = static_cast<uint8_t>(e + 127);
-}
-
-// MXFP8 activation scales packed per M tile of the grouped GEMM: sorted row r of
-// group g (rows [off[g], off[g+1])) sits in M tile mt = mt_base[g] + (r -
-// off[g]) / 128 as row i = (r - off[g]) % 128, and the four scale bytes of its
-// 128-element K block kb go to byte (mt * KB + kb) * 512 + 16 (i % 32) + 4 (i / 32)
-// of sfx (KB = K / 128): the block-scaled MMA's scale-factor layout of a
-// 128-row block, so that a tile's K block of scales is one 512-byte copy.  The
-// bytes come from the token's row of the row-major scales xs [T, K/32].
-// off, mt_base: [G + 1] group offsets and M-tile prefix (shared memory).
-__device__ __forceinline__ void pack_row_scales(long long r, int G, const int *off, const int *mt_base,
-                                                const int *__restrict__ row_token, const uint8_t *__restrict__ xs,
-                                                int kb32, uint8_t *__restrict__ sfx)
-{
-    int lo = 0, hi = G - 1;                   // largest g with off[g] <= r
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (off[mid] <= r) lo = mid; else hi = mid - 1;
-    }
-    const int local = static_cast<int>(r - off[lo]);
-    const long long mt = mt_base[lo] + local / 128;
-    const int i = local % 128;
-    const int KB = kb32 / 4;
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(xs + static_cast<size_t>(row_token[r]) * kb32);
-    uint8_t *dst = sfx + mt * KB * 512 + (i % 32) * 16 + (i / 32) * 4;
-    for (int kb = 0; kb < KB; ++kb) *reinterpret_cast<uint32_t *>(dst + static_cast<size_t>(kb) * 512) = src[kb];
-}
-
-// group offsets and the M-tile prefix of the groups into shared memory (one thread)
-__device__ __forceinline__ void load_tile_tables(const int *__restrict__ offsets, int G, int *off, int *mt_base)
-{
-    int acc = 0;
-    for (int g = 0; g <= G; ++g) {
-        off[g] = offsets[g];
-        mt_base[g] = acc;
-        if (g < G) acc += (offsets[g + 1] - offsets[g] + 127) / 128;
-    }
-}
-
-__global__ void __launch_bounds__(256) pack_row_scales_kernel(const int *__restrict__ offsets, int G, long long R,
-                                                              const int *__restrict__ row_token,
-                                                              const uint8_t *__restrict__ xs, int kb32,
-                                                              uint8_t *__restrict__ sfx)
-{
-    griddep_enter();
-    __shared__ int s_off[kMaxGroupsQ + 1], s_mt[kMaxGroupsQ + 1];
-    if (threadIdx.x == 0) load_tile_tables(offsets, G, s_off, s_mt);
-    __syncthreads();
-    const long long r = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (r < R) pack_row_scales(r, G, s_off, s_mt, row_token, xs, kb32, sfx);
 }
 
 __global__ void __launch_bounds__(256) quantize_mxfp8_kernel(const __nv_bfloat16 *__restrict__ src,
