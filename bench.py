@@ -208,8 +208,8 @@ def backward_algorithmic(wl, counts):
     return fl, nb
 
 
-BWD_STAMP_PHASES = ["q0_zero", "down_dgrad_gemm", "gate_up_dgrad_gemm", "down_wgrad_gemm", "slot_grad",
-                    "router_partial_dx_gate_up_wgrad", "router_reduce"]
+BWD_STAMP_PHASES = ["q0_zero", "dgrads_with_early_down_wgrad", "late_down_wgrad", "gate_up_wgrad", "slot_grad",
+                    "router_partial_dx", "router_reduce"]
 
 
 STAMP_PHASES = ["p0_zero_split_quant", "router_gemm", "select", "dispatch", "gate_up_gemm", "down_after_gate_up",

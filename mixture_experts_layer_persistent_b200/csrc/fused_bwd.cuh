@@ -6,7 +6,7 @@
 // backward among the measured passes).  One cooperative launch, one CTA per SM,
 // 320 threads; phases, with the grid barriers of fused.cuh:
 //
-//   Q0  zero the launch's tile and readiness counters
+//   Q0  zero the launch's tile and readiness counters; the groups' first M tiles
 //   --- grid barrier
 //   Q1  down dgrad GEMM with the SwiGLU-backward epilogue (dGU, slot-gradient
 //       partials); each epilogue warp counts its finished tile on the M tile's
@@ -14,14 +14,17 @@
 //   Q2  gate/up dgrad GEMM (dX slot rows): its producer starts an M tile once
 //       every down-dgrad tile of those rows is in memory -- no barrier
 //   Q3  down weight gradient: streaming kernel for groups of more than 256 rows,
-//       then the resident kernel for the rest (no dependency on Q1/Q2)
+//       then the resident kernel for the rest.  It depends on nothing of the
+//       pass, so every second CTA runs it BEFORE Q1/Q2: its dW stores (store
+//       bound) overlap the dgrads' weight reads (read bound) on other SMs
+//   Q5  gate/up weight gradient (streaming, then resident): each work unit
+//       waits until every dGU tile of its group is in memory -- no barrier
 //   --- grid barrier
 //   Q4  slot gradients and routing-logit gradients (one thread per token)
 //   --- grid barrier
-//   Q5  router-gradient partial sums, the dx sum, then the gate/up weight
-//       gradient (streaming, then resident)
+//   Q6  router-gradient partial sums and the dx sum
 //   --- grid barrier
-//   Q6  router-gradient reduction
+//   Q7  router-gradient reduction
 //
 // Every phase runs the device code of the split schedule's kernels, so the two
 // schedules give byte-identical gradients.  The resident weight-gradient phases
@@ -55,10 +58,18 @@ struct FusedBwdArgs {
     const float *dxs;
     __nv_bfloat16 *dx;
     unsigned long long *trace;     // null, or [kFusedBwdTracePoints][gridDim.x] globaltimer stamps
+    const int *offsets_all;        // [G + 1] row ranges of all groups (routed, then shared)
+    int *mt_base;                  // [G + 1] first M tile of each group (written in Q0)
 };
 
-// trace points: start, then the end of Q0, Q1, Q2, Q3, Q4, Q5 and Q6
+// trace points: start, end of Q0, end of the dgrads (for every second CTA after its
+// down weight gradient), end of the down weight gradient (the others), end of the
+// gate/up weight gradient, end of the slot gradients, of the router partials + dx,
+// of the router-gradient reduction
 constexpr int kFusedBwdTracePoints = 8;
+
+// every kDownWgradFirst-th CTA runs the down weight gradient before the dgrads (0: none)
+constexpr int kDownWgradFirst = 2;
 
 struct FusedBwdMaps {
     CUtensorMap d1B, d1Bs, d1O;              // down dgrad: W_down (MN-major), shared, dGU out
@@ -125,27 +136,63 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     // ---------------------------------------------------------------- Q0
     for (long long i = gtid; i < a.n_zero; i += gstride) a.zero[i] = 0;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        // first M tile of every group in the down dgrad's tiling (readiness counters)
+        int acc = 0;
+        for (int g = 0; g <= a.g1.num_groups; ++g) {
+            a.mt_base[g] = acc;
+            if (g < a.g1.num_groups) acc += (a.offsets_all[g + 1] - a.offsets_all[g] + BM - 1) / BM;
+        }
+    }
     fused_bwd_stamp(a, 1);
     int nb = 0;
     bool alive = grid_sync(a.gs, epoch, nb++, true, a.status, s_flag);
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.gs.epoch = (epoch + 1) & kEpochMask;
 
-    // ---------------------------------------------------------------- Q1, Q2, Q3
+    // ---------------------------------------------------------------- Q1, Q2, Q3, Q5
+    // The down weight gradient depends on nothing of this pass: every kDownWgradFirst-th
+    // CTA runs it first, so its dW stores overlap the dgrads' weight reads on other SMs.
+    // The gate/up weight gradient waits per group for that group's dGU (readiness).
     if (alive) {
-        gemm_phase<typename F::DgradDown>(smem, gbars, aux, tmem_base, m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, a.g1);
-        fused_bwd_stamp(a, 2);
+        const bool dw_first = kDownWgradFirst > 0 && blockIdx.x % kDownWgradFirst == kDownWgradFirst - 1;
+        if (dw_first) {
+            tc_fence_after();
+            gemm_phase<typename F::WgradDown>(smem, gbars + 2 * GB, aux, tmem_base, m.w2B, m.w2B, m.w2B, m.w2O,
+                                              m.w2O2, m.w2O, a.g2);
+            if constexpr (N256) {
+                if (a.g2_units > 0) {
+                    tc_fence_after();
+                    wgrad_resident_phase<typename F::ResDown>(smem, rbars, tmem_base, m.w2B, m.w2B, m.w2O, m.w2O2,
+                                                              a.g2r);
+                }
+            }
+        }
+        tc_fence_after();
+        gemm_phase<typename F::DgradDown>(smem, gbars, aux, tmem_base, m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O,
+                                          a.g1);
         tc_fence_after();
         gemm_phase<typename F::DgradGU>(smem, gbars + GB, aux, tmem_base, m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O,
                                         a.g3);
+        fused_bwd_stamp(a, 2);
+        if (!dw_first) {
+            tc_fence_after();
+            gemm_phase<typename F::WgradDown>(smem, gbars + 2 * GB, aux, tmem_base, m.w2B, m.w2B, m.w2B, m.w2O,
+                                              m.w2O2, m.w2O, a.g2);
+            if constexpr (N256) {
+                if (a.g2_units > 0) {
+                    tc_fence_after();
+                    wgrad_resident_phase<typename F::ResDown>(smem, rbars, tmem_base, m.w2B, m.w2B, m.w2O, m.w2O2,
+                                                              a.g2r);
+                }
+            }
+        }
         fused_bwd_stamp(a, 3);
         tc_fence_after();
-        gemm_phase<typename F::WgradDown>(smem, gbars + 2 * GB, aux, tmem_base, m.w2B, m.w2B, m.w2B, m.w2O, m.w2O2,
-                                          m.w2O, a.g2);
-        if constexpr (N256) {
-            if (a.g2_units > 0) {
-                tc_fence_after();
-                wgrad_resident_phase<typename F::ResDown>(smem, rbars, tmem_base, m.w2B, m.w2B, m.w2O, m.w2O2, a.g2r);
-            }
+        gemm_phase<typename F::WgradGU>(smem, gbars + 3 * GB, aux, tmem_base, m.w4A, m.w4A, m.w4A, m.w4O, m.w4O2,
+                                        m.w4O, a.g4);
+        if (a.g4_units > 0) {
+            tc_fence_after();
+            wgrad_resident_phase<typename F::ResGU>(smem, rbars + RB, tmem_base, m.w4A, m.w4A, m.w4O, m.w4O2, a.g4r);
         }
     } else {
         fused_bwd_stamp(a, 2);
@@ -173,13 +220,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const long long n = static_cast<long long>(a.T) * (a.H / 8);
         for (long long i = gtid; i < n; i += gstride)
             dx_combine_elem(i, a.dxs, a.dl, a.topk_idx, a.router_w, a.dx, a.H, a.k, a.S);
-        tc_fence_after();
-        gemm_phase<typename F::WgradGU>(smem, gbars + 3 * GB, aux, tmem_base, m.w4A, m.w4A, m.w4A, m.w4O, m.w4O2,
-                                        m.w4O, a.g4);
-        if (a.g4_units > 0) {
-            tc_fence_after();
-            wgrad_resident_phase<typename F::ResGU>(smem, rbars + RB, tmem_base, m.w4A, m.w4A, m.w4O, m.w4O2, a.g4r);
-        }
     }
     fused_bwd_stamp(a, 6);
     alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);

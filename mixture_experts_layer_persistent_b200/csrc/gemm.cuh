@@ -94,9 +94,13 @@ struct GemmArgs {
                                   // are complete; kReadyWait: the producer waits for ready_target
                                   // before it hands a tile to the other roles
     int ready_target;
+    const int *mt_base;           // kReadyWaitGroup: [G + 1] first M tile of each group in the producing
+                                  // GEMM's tiling (the group's counters are mt_base[g] .. mt_base[g+1]-1)
 };
 
-constexpr int kReadyNone = 0, kReadySignal = 1, kReadyWait = 2;
+// kReadyWaitGroup: a weight-gradient phase waits, before it loads a group's rows,
+// until every M tile of the group has reached ready_target
+constexpr int kReadyNone = 0, kReadySignal = 1, kReadyWait = 2, kReadyWaitGroup = 3;
 
 template <int BN_, bool A_MN_, bool B_MN_, bool A_GATHER_, bool B_GATHER_, bool RAGGED_K_, int EPI_,
           bool MX_ = false>
@@ -416,6 +420,15 @@ __device__ __forceinline__ void signal_ready(int *ctr, int lane)
     __syncwarp();
 }
 
+// Producer lane: wait for every M tile of group g (bounded, as wait_ready).
+__device__ __forceinline__ bool wait_group_ready(const GemmArgs &a, int g, volatile int *abort, int *status)
+{
+    const int m0 = a.mt_base[g], m1 = a.mt_base[g + 1];
+    for (int mt = m0; mt < m1; ++mt)
+        if (!wait_ready(a.ready + mt, a.ready_target, abort, status)) return false;
+    return true;
+}
+
 // One grouped-GEMM phase run by every thread of the CTA.
 //   smem       1024-byte aligned: C::RING_BYTES of stage ring, scale blocks and staging
 //   bar_block  kGemmBarBytes of barriers for this phase alone (not reused by another phase)
@@ -511,7 +524,15 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
         int tile = blockIdx.x;
         for (int it = 0;; ++it) {
             bool put = true;
-            if constexpr (!C::RAGGED_K) {
+            if constexpr (C::RAGGED_K) {
+                if (args.ready_role == kReadyWaitGroup && tile < total) {
+                    // the group's rows of the contiguous operand come from an earlier phase
+                    const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
+                    if (lane == 0) put = wait_group_ready(args, t.g, abort_flag, status);
+                    put = __shfl_sync(0xffffffffu, put, 0);
+                    if (!put) tile = total;
+                }
+            } else {
                 if (args.ready_role == kReadyWait && tile < total) {
                     // the rows this tile reads are produced by an earlier phase of the launch
                     const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);

@@ -256,6 +256,7 @@ struct BwdScratch {
     int *zero;                    // sched and ready: the counters the persistent backward zeroes
     int n_zero;
     unsigned long long *gs_flags; // grid-barrier tags, release tag, epoch
+    int *mt_base;                 // [G + 1] first M tile of each group (persistent backward)
     size_t bytes;
 };
 
@@ -275,6 +276,7 @@ BwdScratch carve_bwd(const moe_cfg &c, void *buf)
     b.sched = b.zero;
     b.ready = b.zero + kSchedCounters;
     b.gs_flags = cv.take<unsigned long long>(kMaxFusedCtas + 2);
+    b.mt_base = cv.take<int>(s.G + 1);
     b.bytes = align_up(cv.off, 256);
     return b;
 }
@@ -865,6 +867,11 @@ int launch_fused_bwd(const moe_cfg &c, const void *x, const moe_params &p, const
     a.g3 = pl.g3;
     a.g3.ready_role = kReadyWait;
     a.g4 = a.g4r = pl.g4;
+    a.g4.ready_role = a.g4r.ready_role = kReadyWaitGroup;
+    a.g4.ready_target = a.g4r.ready_target = 4 * pl.g1.n_tiles;
+    a.g4.mt_base = a.g4r.mt_base = bs.mt_base;
+    a.offsets_all = st.offsets;
+    a.mt_base = bs.mt_base;
     a.g2_units = pl.g2_units;
     a.g4_units = pl.g4_units;
     a.gpart = bs.gpart;

@@ -181,6 +181,12 @@ __device__ __forceinline__ void wgrad_resident_phase(uint8_t *smem, uint64_t *ba
                     bfilled |= 1u << kb;
                 }
             } else {
+                if (args.ready_role == kReadyWaitGroup) {
+                    // the group's A rows come from an earlier phase of the launch
+                    if (lane == 0) ok = wait_group_ready(args, w.g, abort_flag, status);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                }
                 // A = rows krow0.. of the contiguous [R, M] matrix, columns of M tile mt
                 for (int mt = w.mt0; mt < w.mt1 && ok; ++mt) {
                     for (int kb = 0; kb < w.nkb; ++kb) {
