@@ -37,7 +37,10 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8])
 // y[t] = sum_{j<k} w[t,j] O[t,j] (ascending j) + sum_s O[t,k+s] (ascending s), fp32, -> bf16.
 // Thread = 8 columns of one token (16-byte loads).
 // O: fp32 slot rows (BF16 layer) or bf16 slot rows (MXFP8 forward)
-template <class Slot>
+// B slot rows' loads are issued before their sums, which still run in ascending j
+// (B = 4 in the split kernel, where occupancy keeps many threads in flight; 8 in
+// the persistent kernel, whose 320 threads per SM need more loads each)
+template <class Slot, int B = 4>
 __device__ __forceinline__ void combine_elem(long long i, const Slot *__restrict__ O,
                                              const float *__restrict__ topk_w, __nv_bfloat16 *__restrict__ y,
                                              int H, int k, int S)
@@ -47,18 +50,16 @@ __device__ __forceinline__ void combine_elem(long long i, const Slot *__restrict
     const int kk = k + S;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const Slot *row = O + (size_t)t * kk * H + c;
-    // slots in groups of four: the four rows' loads are issued before their sums,
-    // which still run in ascending j
     int j = 0;
-    for (; j + 4 <= kk; j += 4) {
-        float v[4][8], w[4];
+    for (; j + B <= kk; j += B) {
+        float v[B][8], w[B];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < B; ++u) {
             w[u] = j + u < k ? topk_w[(size_t)t * k + j + u] : 1.0f;
             load8(row + (size_t)(j + u) * H, v[u]);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < B; ++u)
 #pragma unroll
             for (int q = 0; q < 8; ++q) acc[q] = fmaf(w[u], v[u][q], acc[q]);
     }
@@ -132,57 +133,24 @@ __global__ void __launch_bounds__(256) slot_grad_kernel(const float *__restrict_
 // rows of one expert and 256 columns, partial[chunk, cols] = sum over the
 // chunk's rows of dl(row) x[token(row), cols], in a fixed order: the rows
 // r0 + w, r0 + w + 8, ... (w = 0..7) are summed separately in ascending order,
-// then the eight sums in order of w.  One warp per item; lane = 8 columns.
-__device__ __forceinline__ void drouter_partial_item(int chunk, int h0, int lane, const __nv_bfloat16 *__restrict__ x,
-                                                     const float *__restrict__ dl, const int *__restrict__ offsets,
-                                                     const int *__restrict__ chunk_start,
-                                                     const int *__restrict__ perm, float *__restrict__ partial,
-                                                     int H, int E, int k, int chunk_rows)
+// then the eight sums in order of w.  Two implementations with that same order
+// (so the same bits): eight warps per item for the split schedule's kernel, a
+// team of two warps per item for the persistent kernel.
+
+__device__ __forceinline__ int drouter_chunk_rows(int chunk, const int *__restrict__ offsets,
+                                                  const int *__restrict__ chunk_start, int E, int chunk_rows, int &r1)
 {
     int lo = 0, hi = E - 1;     // expert owning this chunk: largest e with chunk_start[e] <= chunk
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (chunk_start[mid] <= chunk) lo = mid; else hi = mid - 1;
     }
-    const int e = lo;
-    const int r0 = offsets[e] + (chunk - chunk_start[e]) * chunk_rows;
-    const int r1 = min(offsets[e + 1], r0 + chunk_rows);
-    float acc[8][8];
-#pragma unroll
-    for (int w = 0; w < 8; ++w)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[w][q] = 0.0f;
-    for (int r = r0; r < r1; r += 8) {
-        float v[8][8], d[8];
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {             // eight rows' loads in flight
-            if (r + w < r1) {
-                const int s = perm[r + w];        // t * k + slot
-                d[w] = dl[s];
-                unpack8(*reinterpret_cast<const uint4 *>(x + (size_t)(s / k) * H + h0 + lane * 8), v[w]);
-            }
-        }
-#pragma unroll
-        for (int w = 0; w < 8; ++w)
-            if (r + w < r1)
-#pragma unroll
-                for (int q = 0; q < 8; ++q) acc[w][q] = fmaf(d[w], v[w][q], acc[w][q]);
-    }
-    float out[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        float s = 0.0f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) s += acc[w][q];
-        out[q] = s;
-    }
-    float4 *dst = reinterpret_cast<float4 *>(partial + (size_t)chunk * H + h0 + lane * 8);
-    dst[0] = make_float4(out[0], out[1], out[2], out[3]);
-    dst[1] = make_float4(out[4], out[5], out[6], out[7]);
+    const int r0 = offsets[lo] + (chunk - chunk_start[lo]) * chunk_rows;
+    r1 = min(offsets[lo + 1], r0 + chunk_rows);
+    return r0;
 }
 
-// items = (chunk, 256-column block) pairs, one warp each; grid covers an upper bound
-// of the chunk count
+// split schedule: one item per block of 256 threads, warp w sums the rows of residue w
 __global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat16 *__restrict__ x,
                                                               const float *__restrict__ dl,
                                                               const int *__restrict__ offsets,
@@ -192,11 +160,74 @@ __global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat1
                                                               int chunk_rows)
 {
     griddep_enter();
-    const int hb = H / 256;
-    const int item = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (item >= chunk_start[E] * hb) return;
-    drouter_partial_item(item / hb, (item % hb) * 256, threadIdx.x & 31, x, dl, offsets, chunk_start, perm, partial, H,
-                         E, k, chunk_rows);
+    __shared__ float s_acc[8][256];
+    const int chunk = blockIdx.x;
+    const int h0 = blockIdx.y * 256;
+    if (chunk >= chunk_start[E]) return;
+    int r1;
+    const int r0 = drouter_chunk_rows(chunk, offsets, chunk_start, E, chunk_rows, r1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    for (int r = r0 + warp; r < r1; r += 8) {
+        const int s = perm[r];                  // t * k + slot
+        const float d = dl[s];
+        float v[8];
+        unpack8(*reinterpret_cast<const uint4 *>(x + (size_t)(s / k) * H + h0 + lane * 8), v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = fmaf(d, v[q], acc[q]);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) s_acc[warp][lane * 8 + q] = acc[q];
+    __syncthreads();
+    float s = 0.0f;
+    for (int w = 0; w < 8; ++w) s += s_acc[w][threadIdx.x];
+    partial[(size_t)chunk * H + h0 + threadIdx.x] = s;
+}
+
+// persistent schedule: a team of two warps per item (warp half h sums residues
+// 4h .. 4h+3, four rows in flight); s_acc: the team's [8][256] floats of shared
+// memory; bar: the team's named barrier (64 threads)
+__device__ __forceinline__ void drouter_partial_team(int chunk, int h0, int half, int lane, int bar,
+                                                     const __nv_bfloat16 *__restrict__ x, const float *__restrict__ dl,
+                                                     const int *__restrict__ offsets,
+                                                     const int *__restrict__ chunk_start,
+                                                     const int *__restrict__ perm, float *__restrict__ partial,
+                                                     int H, int E, int k, int chunk_rows, float (*s_acc)[256])
+{
+    int r1;
+    const int r0 = drouter_chunk_rows(chunk, offsets, chunk_start, E, chunk_rows, r1);
+    float acc[4][8];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[w][q] = 0.0f;
+    for (int r = r0 + 4 * half; r < r1; r += 8) {
+        float v[4][8], d[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            if (r + w < r1) {
+                const int s = perm[r + w];
+                d[w] = dl[s];
+                unpack8(*reinterpret_cast<const uint4 *>(x + (size_t)(s / k) * H + h0 + lane * 8), v[w]);
+            }
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+            if (r + w < r1)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[w][q] = fmaf(d[w], v[w][q], acc[w][q]);
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) s_acc[4 * half + w][lane * 8 + q] = acc[w][q];
+    asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
+    for (int c = half * 32 + lane; c < 256; c += 64) {
+        float s = 0.0f;
+        for (int w = 0; w < 8; ++w) s += s_acc[w][c];
+        partial[(size_t)chunk * H + h0 + c] = s;
+    }
+    asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void drouter_reduce_elem(long long i, const float *__restrict__ partial,
@@ -219,6 +250,7 @@ __global__ void __launch_bounds__(256) drouter_reduce_kernel(const float *__rest
 
 // dx[t] = sum_j dXs[t, j] (ascending j over routed then shared slots)
 //         + sum_{j<k} dl[t, j] router_w[idx[t, j]]   -> bf16.
+template <int B = 4>
 __device__ __forceinline__ void dx_combine_elem(long long i, const float *__restrict__ dXs,
                                                 const float *__restrict__ dl, const int *__restrict__ topk_idx,
                                                 const float *__restrict__ router_w, __nv_bfloat16 *__restrict__ dx,
@@ -230,12 +262,12 @@ __device__ __forceinline__ void dx_combine_elem(long long i, const float *__rest
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     const float *row = dXs + (size_t)t * kk * H + c;
     int j = 0;
-    for (; j + 4 <= kk; j += 4) {                  // four rows' loads in flight, sums in ascending j
-        float v[4][8];
+    for (; j + B <= kk; j += B) {                  // B rows' loads in flight, sums in ascending j
+        float v[B][8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) load8(row + (size_t)(j + u) * H, v[u]);
+        for (int u = 0; u < B; ++u) load8(row + (size_t)(j + u) * H, v[u]);
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < B; ++u)
 #pragma unroll
             for (int q = 0; q < 8; ++q) acc[q] += v[u][q];
     }

@@ -271,9 +271,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         const long long n = static_cast<long long>(a.T) * (a.H / 8);
         for (long long i = gtid; i < n; i += gstride) {
             if constexpr (MX)
-                combine_elem(i, static_cast<const __nv_bfloat16 *>(a.O), a.sa.topk_w, a.y, a.H, a.k, a.S);
+                combine_elem<__nv_bfloat16, 8>(i, static_cast<const __nv_bfloat16 *>(a.O), a.sa.topk_w, a.y, a.H,
+                                               a.k, a.S);
             else
-                combine_elem(i, static_cast<const float *>(a.O), a.sa.topk_w, a.y, a.H, a.k, a.S);
+                combine_elem<float, 8>(i, static_cast<const float *>(a.O), a.sa.topk_w, a.y, a.H, a.k, a.S);
         }
     }
     fused_stamp(a, 7);

@@ -211,15 +211,19 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     // ---------------------------------------------------------------- Q5
     if (alive) {
+        // router-gradient partials: five teams of two warps per CTA, one item each
         const int n_items = a.chunk_start[a.E] * (a.H / 256);
         const int hb = a.H / 256;
-        const int nw = kFusedThreads / 32;
-        for (int item = blockIdx.x * nw + warp; item < n_items; item += gridDim.x * nw)
-            drouter_partial_item(item / hb, (item % hb) * 256, threadIdx.x & 31, a.x, a.dl, a.offsets, a.chunk_start,
-                                 a.perm, a.partial, a.H, a.E, a.k, a.chunk_rows);
+        constexpr int teams = kFusedThreads / 64;
+        const int team = warp >> 1;
+        float(*s_acc)[256] = reinterpret_cast<float(*)[256]>(smem) + team * 8;
+        for (int item = blockIdx.x * teams + team; item < n_items; item += gridDim.x * teams)
+            drouter_partial_team(item / hb, (item % hb) * 256, warp & 1, threadIdx.x & 31, 1 + team, a.x, a.dl,
+                                 a.offsets, a.chunk_start, a.perm, a.partial, a.H, a.E, a.k, a.chunk_rows, s_acc);
+        __syncthreads();                       // the teams' scratch is free again
         const long long n = static_cast<long long>(a.T) * (a.H / 8);
         for (long long i = gtid; i < n; i += gstride)
-            dx_combine_elem(i, a.dxs, a.dl, a.topk_idx, a.router_w, a.dx, a.H, a.k, a.S);
+            dx_combine_elem<8>(i, a.dxs, a.dl, a.topk_idx, a.router_w, a.dx, a.H, a.k, a.S);
     }
     fused_bwd_stamp(a, 6);
     alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);

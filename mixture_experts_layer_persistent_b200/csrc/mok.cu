@@ -808,7 +808,7 @@ int backward_split(const moe_cfg &c, const void *x, const moe_params &p, const S
                      static_cast<const float *>(st.topk_w), static_cast<const float *>(st.topk_p), bs.dl, c.T,
                      c.top_k, c.score_fn, c.routed_scale));
     MOK_TRY(mark_bwd(2, stream));
-    MOK_TRY(launch_k(drouter_partial_kernel, dim3(blocks_for(s.max_chunks * (c.H / 256), 8)), dim3(256), 0, stream,
+    MOK_TRY(launch_k(drouter_partial_kernel, dim3(static_cast<unsigned>(s.max_chunks), c.H / 256), dim3(256), 0, stream,
                      "drouter_partial_kernel", static_cast<const __nv_bfloat16 *>(x), static_cast<const float *>(bs.dl),
                      static_cast<const int *>(st.offsets), static_cast<const int *>(st.chunk_start),
                      static_cast<const int *>(st.perm), bs.partial, c.H, c.E, c.top_k, kChunkRows));
