@@ -208,7 +208,7 @@ def backward_algorithmic(wl, counts):
     return fl, nb
 
 
-BWD_STAMP_PHASES = ["q0_zero", "dgrads_with_early_down_wgrad", "late_down_wgrad", "gate_up_wgrad", "slot_grad",
+BWD_STAMP_PHASES = ["q0_zero", "dgrads", "down_wgrad_after_dgrads", "gate_up_wgrad_after_down_wgrad", "slot_grad",
                     "router_partial_dx", "router_reduce"]
 
 

@@ -322,11 +322,9 @@ int moe_get_schedule(int *schedule);
  * p = 0 start, then the end of the zeroing / router-split / quantisation
  * phase, the router GEMM, the top-k, the dispatch, the gate/up GEMM, the down
  * GEMM and the combine.  Backward points: p = 0 start, then the end of the
- * zeroing, of the two dgrads (on every second CTA preceded by its share of the
- * down weight gradient, which then overlaps the other CTAs' dgrads), of the
- * down weight gradient (the other CTAs), of the gate/up weight gradient, of
- * the slot gradients, of the router partial sums + dx, and of the
- * router-gradient reduction.  NULL stops the stamps.
+ * zeroing, of the two dgrads, of the down weight gradient, of the gate/up
+ * weight gradient, of the slot gradients, of the router partial sums + dx, and
+ * of the router-gradient reduction.  NULL stops the stamps.
  */
 #define MOK_TRACE_POINTS 8
 int moe_trace_device(void *buf, size_t bytes, void *bwd_buf, size_t bwd_bytes);

@@ -38,8 +38,6 @@ __device__ __forceinline__ uint4 pack8(const float (&v)[8])
 // Thread = 8 columns of one token (16-byte loads).
 // O: fp32 slot rows (BF16 layer) or bf16 slot rows (MXFP8 forward)
 // B slot rows' loads are issued before their sums, which still run in ascending j
-// (B = 4 in the split kernel, where occupancy keeps many threads in flight; 8 in
-// the persistent kernel, whose 320 threads per SM need more loads each)
 template <class Slot, int B = 4>
 __device__ __forceinline__ void combine_elem(long long i, const Slot *__restrict__ O,
                                              const float *__restrict__ topk_w, __nv_bfloat16 *__restrict__ y,
@@ -134,8 +132,9 @@ __global__ void __launch_bounds__(256) slot_grad_kernel(const float *__restrict_
 // chunk's rows of dl(row) x[token(row), cols], in a fixed order: the rows
 // r0 + w, r0 + w + 8, ... (w = 0..7) are summed separately in ascending order,
 // then the eight sums in order of w.  Two implementations with that same order
-// (so the same bits): eight warps per item for the split schedule's kernel, a
-// team of two warps per item for the persistent kernel.
+// (so the same bits): eight warps per item for the split schedule's kernel
+// below, one warp per item streaming through shared memory for the persistent
+// kernel (drouter_stream, at the end of this file).
 
 __device__ __forceinline__ int drouter_chunk_rows(int chunk, const int *__restrict__ offsets,
                                                   const int *__restrict__ chunk_start, int E, int chunk_rows, int &r1)
@@ -182,52 +181,6 @@ __global__ void __launch_bounds__(256) drouter_partial_kernel(const __nv_bfloat1
     float s = 0.0f;
     for (int w = 0; w < 8; ++w) s += s_acc[w][threadIdx.x];
     partial[(size_t)chunk * H + h0 + threadIdx.x] = s;
-}
-
-// persistent schedule: a team of two warps per item (warp half h sums residues
-// 4h .. 4h+3, four rows in flight); s_acc: the team's [8][256] floats of shared
-// memory; bar: the team's named barrier (64 threads)
-__device__ __forceinline__ void drouter_partial_team(int chunk, int h0, int half, int lane, int bar,
-                                                     const __nv_bfloat16 *__restrict__ x, const float *__restrict__ dl,
-                                                     const int *__restrict__ offsets,
-                                                     const int *__restrict__ chunk_start,
-                                                     const int *__restrict__ perm, float *__restrict__ partial,
-                                                     int H, int E, int k, int chunk_rows, float (*s_acc)[256])
-{
-    int r1;
-    const int r0 = drouter_chunk_rows(chunk, offsets, chunk_start, E, chunk_rows, r1);
-    float acc[4][8];
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[w][q] = 0.0f;
-    for (int r = r0 + 4 * half; r < r1; r += 8) {
-        float v[4][8], d[4];
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            if (r + w < r1) {
-                const int s = perm[r + w];
-                d[w] = dl[s];
-                unpack8(*reinterpret_cast<const uint4 *>(x + (size_t)(s / k) * H + h0 + lane * 8), v[w]);
-            }
-        }
-#pragma unroll
-        for (int w = 0; w < 4; ++w)
-            if (r + w < r1)
-#pragma unroll
-                for (int q = 0; q < 8; ++q) acc[w][q] = fmaf(d[w], v[w][q], acc[w][q]);
-    }
-#pragma unroll
-    for (int w = 0; w < 4; ++w)
-#pragma unroll
-        for (int q = 0; q < 8; ++q) s_acc[4 * half + w][lane * 8 + q] = acc[w][q];
-    asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
-    for (int c = half * 32 + lane; c < 256; c += 64) {
-        float s = 0.0f;
-        for (int w = 0; w < 8; ++w) s += s_acc[w][c];
-        partial[(size_t)chunk * H + h0 + c] = s;
-    }
-    asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void drouter_reduce_elem(long long i, const float *__restrict__ partial,
@@ -300,6 +253,294 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *__restrict
     griddep_enter();
     const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (i < (long long)T * (H / 8)) dx_combine_elem(i, dXs, dl, topk_idx, router_w, dx, H, k, S);
+}
+
+
+// ---- the same sums in the persistent kernels --------------------------------
+// A persistent CTA has 10 warps per SM, far too few to hide HBM latency with the
+// one-thread-per-element code above (the split kernels rely on 64 resident warps
+// per SM).  Here every thread streams its own 16-byte pieces through a private
+// ring of shared-memory slots with cp.async, NS units deep, so the loads of the
+// next NS-1 units are in flight while a unit is summed.  A thread reads back only
+// the bytes it copied itself, so no barrier is needed between copy and use.  The
+// arithmetic per output column is that of combine_elem / dx_combine_elem /
+// drouter_partial_kernel, in the same order (same bits).
+//   ring: `ring_bytes` of shared memory; slot (stage s, row j) of thread tid at
+//   ring + ((s * R + j) * blockDim.x + tid) * 16 for R rows per unit.
+
+__device__ __forceinline__ uint8_t *stream_slot(uint8_t *ring, int s, int R, int j)
+{
+    return ring + ((static_cast<size_t>(s) * R + j) * blockDim.x + threadIdx.x) * 16;
+}
+
+// stages that fit: units of R rows of 16 bytes per thread, at most 4
+__device__ __forceinline__ int stream_stages(int R, int ring_bytes)
+{
+    const int ns = ring_bytes / (R * 16 * static_cast<int>(blockDim.x));
+    return ns < 1 ? 1 : (ns > 4 ? 4 : ns);
+}
+
+template <int EPU>
+__device__ __forceinline__ void slot_values(const uint8_t *p, float (&v)[EPU])
+{
+    if constexpr (EPU == 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(p);
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    } else {
+        unpack8(*reinterpret_cast<const uint4 *>(p), v);
+    }
+}
+
+template <int EPU>
+__device__ __forceinline__ void store_bf16(__nv_bfloat16 *dst, const float (&v)[EPU])
+{
+    if constexpr (EPU == 4) {
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+    } else {
+        *reinterpret_cast<uint4 *>(dst) = pack8(v);
+    }
+}
+
+// Forward combine: warp = token (warps take tokens in turn), lane = 16-byte column
+// units lane, lane + 32, ...  The token's routing weights sit in lanes 0..k-1; the
+// next token's are loaded while this one streams.
+template <class Slot, int NS>
+__device__ __forceinline__ void combine_stream_ns(const Slot *__restrict__ O, const float *__restrict__ topk_w,
+                                                  __nv_bfloat16 *__restrict__ y, int T, int H, int k, int S,
+                                                  uint8_t *ring)
+{
+    constexpr int EPU = 16 / sizeof(Slot);
+    const int lane = threadIdx.x & 31;
+    const int nw = gridDim.x * (blockDim.x >> 5);
+    const int kk = k + S, units = H / (32 * EPU);
+    int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    float wn = t < T && lane < k ? topk_w[static_cast<size_t>(t) * k + lane] : 0.0f;
+    for (; t < T; t += nw) {
+        const float wc = wn;
+        if (t + nw < T && lane < k) wn = topk_w[static_cast<size_t>(t + nw) * k + lane];
+        const Slot *rows = O + static_cast<size_t>(t) * kk * H + lane * EPU;
+        auto issue = [&](int u) {
+            for (int j = 0; j < kk; ++j)
+                cp_async16(stream_slot(ring, u % NS, kk, j), rows + static_cast<size_t>(j) * H + u * 32 * EPU);
+        };
+#pragma unroll
+        for (int u = 0; u < NS - 1; ++u) {
+            if (u < units) issue(u);
+            cp_async_commit();
+        }
+        for (int u = 0; u < units; ++u) {
+            if (u + NS - 1 < units) issue(u + NS - 1);
+            cp_async_commit();
+            cp_async_wait<NS - 1>();
+            float acc[EPU];
+#pragma unroll
+            for (int q = 0; q < EPU; ++q) acc[q] = 0.0f;
+            for (int j = 0; j < kk; ++j) {
+                const float w = __shfl_sync(0xffffffffu, wc, j < k ? j : 0);
+                float v[EPU];
+                slot_values<EPU>(stream_slot(ring, u % NS, kk, j), v);
+#pragma unroll
+                for (int q = 0; q < EPU; ++q) acc[q] = fmaf(j < k ? w : 1.0f, v[q], acc[q]);
+            }
+            store_bf16<EPU>(y + static_cast<size_t>(t) * H + u * 32 * EPU + lane * EPU, acc);
+        }
+    }
+    cp_async_wait<0>();
+}
+
+template <class Slot>
+__device__ __forceinline__ void combine_stream(const Slot *__restrict__ O, const float *__restrict__ topk_w,
+                                               __nv_bfloat16 *__restrict__ y, int T, int H, int k, int S,
+                                               uint8_t *ring, int ring_bytes)
+{
+    switch (stream_stages(k + S, ring_bytes)) {
+    case 1: combine_stream_ns<Slot, 1>(O, topk_w, y, T, H, k, S, ring); break;
+    case 2: combine_stream_ns<Slot, 2>(O, topk_w, y, T, H, k, S, ring); break;
+    case 3: combine_stream_ns<Slot, 3>(O, topk_w, y, T, H, k, S, ring); break;
+    default: combine_stream_ns<Slot, 4>(O, topk_w, y, T, H, k, S, ring); break;
+    }
+}
+
+// dx sum: as combine_stream, with the token's k router-weight rows Wr[idx_j]
+// streamed beside its k + S dX slot rows (R = 2k + S rows per unit).
+template <int NS>
+__device__ __forceinline__ void dx_stream_ns(const float *__restrict__ dXs, const float *__restrict__ dl,
+                                             const int *__restrict__ topk_idx, const float *__restrict__ router_w,
+                                             __nv_bfloat16 *__restrict__ dx, int T, int H, int k, int S,
+                                             uint8_t *ring)
+{
+    const int lane = threadIdx.x & 31;
+    const int nw = gridDim.x * (blockDim.x >> 5);
+    const int kk = k + S, R = kk + k, units = H / 128;
+    int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    float dn = 0.0f;
+    int en = 0;
+    if (t < T && lane < k) {
+        dn = dl[static_cast<size_t>(t) * k + lane];
+        en = topk_idx[static_cast<size_t>(t) * k + lane];
+    }
+    for (; t < T; t += nw) {
+        const float dc = dn;
+        const int ec = en;
+        if (t + nw < T && lane < k) {
+            dn = dl[static_cast<size_t>(t + nw) * k + lane];
+            en = topk_idx[static_cast<size_t>(t + nw) * k + lane];
+        }
+        const float *rows = dXs + static_cast<size_t>(t) * kk * H + lane * 4;
+        auto issue = [&](int u) {
+            for (int j = 0; j < kk; ++j)
+                cp_async16(stream_slot(ring, u % NS, R, j), rows + static_cast<size_t>(j) * H + u * 128);
+            for (int j = 0; j < k; ++j) {
+                const int e = __shfl_sync(0xffffffffu, ec, j);
+                cp_async16(stream_slot(ring, u % NS, R, kk + j), router_w + static_cast<size_t>(e) * H + u * 128 +
+                                                                     lane * 4);
+            }
+        };
+#pragma unroll
+        for (int u = 0; u < NS - 1; ++u) {
+            if (u < units) issue(u);
+            cp_async_commit();
+        }
+        for (int u = 0; u < units; ++u) {
+            if (u + NS - 1 < units) issue(u + NS - 1);
+            cp_async_commit();
+            cp_async_wait<NS - 1>();
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, r[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int j = 0; j < kk; ++j) {
+                float v[4];
+                slot_values<4>(stream_slot(ring, u % NS, R, j), v);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[q] += v[q];
+            }
+            for (int j = 0; j < k; ++j) {
+                const float d = __shfl_sync(0xffffffffu, dc, j);
+                float w[4];
+                slot_values<4>(stream_slot(ring, u % NS, R, kk + j), w);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) r[q] = fmaf(d, w[q], r[q]);
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] += r[q];
+            store_bf16<4>(dx + static_cast<size_t>(t) * H + u * 128 + lane * 4, acc);
+        }
+    }
+    cp_async_wait<0>();
+}
+
+__device__ __forceinline__ void dx_stream(const float *__restrict__ dXs, const float *__restrict__ dl,
+                                          const int *__restrict__ topk_idx, const float *__restrict__ router_w,
+                                          __nv_bfloat16 *__restrict__ dx, int T, int H, int k, int S, uint8_t *ring,
+                                          int ring_bytes)
+{
+    switch (stream_stages(2 * k + S, ring_bytes)) {
+    case 1: dx_stream_ns<1>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
+    case 2: dx_stream_ns<2>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
+    case 3: dx_stream_ns<3>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
+    default: dx_stream_ns<4>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
+    }
+}
+
+// Router-gradient partial sums: warp = item (row chunk, 256 columns), lane = 8
+// columns.  The item's rows run in units of 8 (one row per residue r0 + w mod 8),
+// four units deep; a warp-private table in shared memory holds each row's token
+// and dl, loaded once per item.  Sums per residue in ascending row order, then
+// over the residues in order of w, as drouter_partial_kernel.
+//   smem: the ring (4 stages x 8 rows x 16 bytes per thread), then the warps'
+//   row tables (kDrouterMaxRows x 8 bytes per warp), then chunk_start and offsets
+//   ((E + 1) ints each).  Needs drouter_stream_bytes(E) bytes.
+constexpr int kDrouterMaxRows = 256;             // rows per chunk at most
+constexpr int kDrouterStages = 4;
+__host__ __device__ constexpr int drouter_stream_bytes(int threads, int E)
+{
+    return kDrouterStages * 8 * 16 * threads + threads / 32 * kDrouterMaxRows * 8 + 2 * (E + 1) * 4;
+}
+
+__device__ __forceinline__ void drouter_stream(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ dl,
+                                               const int *__restrict__ offsets, const int *__restrict__ chunk_start,
+                                               const int *__restrict__ perm, float *__restrict__ partial, int H, int E,
+                                               int k, int chunk_rows, uint8_t *smem)
+{
+    constexpr int NS = kDrouterStages;
+    const int nthr = blockDim.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint8_t *ring = smem;
+    int *tab_tok = reinterpret_cast<int *>(smem + NS * 8 * 16 * nthr) + warp * 2 * kDrouterMaxRows;
+    float *tab_d = reinterpret_cast<float *>(tab_tok + kDrouterMaxRows);
+    int *s_cs = reinterpret_cast<int *>(smem + NS * 8 * 16 * nthr) + (nthr >> 5) * 2 * kDrouterMaxRows;
+    int *s_off = s_cs + E + 1;
+    for (int i = threadIdx.x; i <= E; i += nthr) {
+        s_cs[i] = chunk_start[i];
+        s_off[i] = offsets[i];
+    }
+    __syncthreads();
+    const int hb = H / 256;
+    const int n_items = s_cs[E] * hb;
+    const int nw = gridDim.x * (nthr >> 5);
+    for (int item = blockIdx.x * (nthr >> 5) + warp; item < n_items; item += nw) {
+        const int chunk = item / hb, h0 = (item - chunk * hb) * 256;
+        int r1;
+        const int r0 = drouter_chunk_rows(chunk, s_off, s_cs, E, chunk_rows, r1);
+        const int nrows = r1 - r0, units = (nrows + 7) >> 3;
+        int sv[kDrouterMaxRows / 32];
+        float dv[kDrouterMaxRows / 32];
+#pragma unroll
+        for (int m = 0; m < kDrouterMaxRows / 32; ++m)
+            sv[m] = lane + 32 * m < nrows ? perm[r0 + lane + 32 * m] : 0;
+#pragma unroll
+        for (int m = 0; m < kDrouterMaxRows / 32; ++m) dv[m] = lane + 32 * m < nrows ? dl[sv[m]] : 0.0f;
+        __syncwarp();                              // the previous item's table reads are done
+#pragma unroll
+        for (int m = 0; m < kDrouterMaxRows / 32; ++m)
+            if (lane + 32 * m < nrows) {
+                tab_tok[lane + 32 * m] = sv[m] / k;
+                tab_d[lane + 32 * m] = dv[m];
+            }
+        __syncwarp();
+        const __nv_bfloat16 *xc = x + h0 + lane * 8;
+        auto issue = [&](int u) {
+            for (int w = 0; w < 8; ++w) {
+                const int i = u * 8 + w;
+                if (i < nrows) cp_async16(stream_slot(ring, u % NS, 8, w), xc + static_cast<size_t>(tab_tok[i]) * H);
+            }
+        };
+        float acc[8][8];
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[w][q] = 0.0f;
+#pragma unroll
+        for (int u = 0; u < NS - 1; ++u) {
+            if (u < units) issue(u);
+            cp_async_commit();
+        }
+        for (int u = 0; u < units; ++u) {
+            if (u + NS - 1 < units) issue(u + NS - 1);
+            cp_async_commit();
+            cp_async_wait<NS - 1>();
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                const int i = u * 8 + w;
+                if (i < nrows) {
+                    const float d = tab_d[i];
+                    float v[8];
+                    slot_values<8>(stream_slot(ring, u % NS, 8, w), v);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) acc[w][q] = fmaf(d, v[q], acc[w][q]);
+                }
+            }
+        }
+        float sum[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            float s = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) s += acc[w][q];
+            sum[q] = s;
+        }
+        float *dst = partial + static_cast<size_t>(chunk) * H + h0 + lane * 8;
+        reinterpret_cast<float4 *>(dst)[0] = make_float4(sum[0], sum[1], sum[2], sum[3]);
+        reinterpret_cast<float4 *>(dst)[1] = make_float4(sum[4], sum[5], sum[6], sum[7]);
+    }
+    cp_async_wait<0>();
 }
 
 }  // namespace mok

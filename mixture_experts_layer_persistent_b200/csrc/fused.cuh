@@ -267,15 +267,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
 
     // ---------------------------------------------------------------- P5
+    // (the GEMM ring's shared memory streams the slot rows: combine_stream)
     if (alive) {
-        const long long n = static_cast<long long>(a.T) * (a.H / 8);
-        for (long long i = gtid; i < n; i += gstride) {
-            if constexpr (MX)
-                combine_elem<__nv_bfloat16, 8>(i, static_cast<const __nv_bfloat16 *>(a.O), a.sa.topk_w, a.y, a.H,
-                                               a.k, a.S);
-            else
-                combine_elem<float, 8>(i, static_cast<const float *>(a.O), a.sa.topk_w, a.y, a.H, a.k, a.S);
-        }
+        if constexpr (MX)
+            combine_stream<__nv_bfloat16>(static_cast<const __nv_bfloat16 *>(a.O), a.sa.topk_w, a.y, a.T, a.H, a.k,
+                                          a.S, smem, F::RING);
+        else
+            combine_stream<float>(static_cast<const float *>(a.O), a.sa.topk_w, a.y, a.T, a.H, a.k, a.S, smem,
+                                  F::RING);
     }
     fused_stamp(a, 7);
 

@@ -14,9 +14,7 @@
 //   Q2  gate/up dgrad GEMM (dX slot rows): its producer starts an M tile once
 //       every down-dgrad tile of those rows is in memory -- no barrier
 //   Q3  down weight gradient: streaming kernel for groups of more than 256 rows,
-//       then the resident kernel for the rest.  It depends on nothing of the
-//       pass, so every second CTA runs it BEFORE Q1/Q2: its dW stores (store
-//       bound) overlap the dgrads' weight reads (read bound) on other SMs
+//       then the resident kernel for the rest (it depends on nothing of the pass)
 //   Q5  gate/up weight gradient (streaming, then resident): each work unit
 //       waits until every dGU tile of its group is in memory -- no barrier
 //   --- grid barrier
@@ -62,14 +60,10 @@ struct FusedBwdArgs {
     int *mt_base;                  // [G + 1] first M tile of each group (written in Q0)
 };
 
-// trace points: start, end of Q0, end of the dgrads (for every second CTA after its
-// down weight gradient), end of the down weight gradient (the others), end of the
-// gate/up weight gradient, end of the slot gradients, of the router partials + dx,
-// of the router-gradient reduction
+// trace points: start, end of Q0, end of the dgrads, of the down weight gradient,
+// of the gate/up weight gradient, of the slot gradients, of the router partials +
+// dx, of the router-gradient reduction
 constexpr int kFusedBwdTracePoints = 8;
-
-// every kDownWgradFirst-th CTA runs the down weight gradient before the dgrads (0: none)
-constexpr int kDownWgradFirst = 2;
 
 struct FusedBwdMaps {
     CUtensorMap d1B, d1Bs, d1O;              // down dgrad: W_down (MN-major), shared, dGU out
@@ -97,6 +91,7 @@ struct FusedBwdCfg {
     static constexpr int SMEM_BYTES = 1024 + REGION + 2 * ResDown::BAR_BYTES + 16;
     static_assert(SMEM_BYTES <= 232448, "shared memory");
     static_assert(ResDown::BAR_BYTES == ResGU::BAR_BYTES, "barrier blocks");
+    static_assert(drouter_stream_bytes(kFusedThreads, 256) <= REGION, "router-gradient stream");
     static_assert(DgradDown::THREADS <= kFusedThreads && WgradDown::THREADS <= kFusedThreads &&
                   DgradGU::THREADS <= kFusedThreads && WgradGU::THREADS <= kFusedThreads &&
                   ResDown::THREADS <= kFusedThreads && ResGU::THREADS <= kFusedThreads, "phase roles fit the launch");
@@ -150,23 +145,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.gs.epoch = (epoch + 1) & kEpochMask;
 
     // ---------------------------------------------------------------- Q1, Q2, Q3, Q5
-    // The down weight gradient depends on nothing of this pass: every kDownWgradFirst-th
-    // CTA runs it first, so its dW stores overlap the dgrads' weight reads on other SMs.
-    // The gate/up weight gradient waits per group for that group's dGU (readiness).
+    // No barrier between the four GEMMs: a CTA moves on when a GEMM's tile counter
+    // is exhausted, so the next GEMM starts on SMs that the previous one's tail
+    // leaves idle.  The gate/up weight gradient waits per group for that group's dGU.
     if (alive) {
-        const bool dw_first = kDownWgradFirst > 0 && blockIdx.x % kDownWgradFirst == kDownWgradFirst - 1;
-        if (dw_first) {
-            tc_fence_after();
-            gemm_phase<typename F::WgradDown>(smem, gbars + 2 * GB, aux, tmem_base, m.w2B, m.w2B, m.w2B, m.w2O,
-                                              m.w2O2, m.w2O, a.g2);
-            if constexpr (N256) {
-                if (a.g2_units > 0) {
-                    tc_fence_after();
-                    wgrad_resident_phase<typename F::ResDown>(smem, rbars, tmem_base, m.w2B, m.w2B, m.w2O, m.w2O2,
-                                                              a.g2r);
-                }
-            }
-        }
         tc_fence_after();
         gemm_phase<typename F::DgradDown>(smem, gbars, aux, tmem_base, m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O,
                                           a.g1);
@@ -174,16 +156,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         gemm_phase<typename F::DgradGU>(smem, gbars + GB, aux, tmem_base, m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O,
                                         a.g3);
         fused_bwd_stamp(a, 2);
-        if (!dw_first) {
-            tc_fence_after();
-            gemm_phase<typename F::WgradDown>(smem, gbars + 2 * GB, aux, tmem_base, m.w2B, m.w2B, m.w2B, m.w2O,
-                                              m.w2O2, m.w2O, a.g2);
-            if constexpr (N256) {
-                if (a.g2_units > 0) {
-                    tc_fence_after();
-                    wgrad_resident_phase<typename F::ResDown>(smem, rbars, tmem_base, m.w2B, m.w2B, m.w2O, m.w2O2,
-                                                              a.g2r);
-                }
+        tc_fence_after();
+        gemm_phase<typename F::WgradDown>(smem, gbars + 2 * GB, aux, tmem_base, m.w2B, m.w2B, m.w2B, m.w2O, m.w2O2,
+                                          m.w2O, a.g2);
+        if constexpr (N256) {
+            if (a.g2_units > 0) {
+                tc_fence_after();
+                wgrad_resident_phase<typename F::ResDown>(smem, rbars, tmem_base, m.w2B, m.w2B, m.w2O, m.w2O2, a.g2r);
             }
         }
         fused_bwd_stamp(a, 3);
@@ -210,20 +189,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
 
     // ---------------------------------------------------------------- Q5
+    // router-gradient partials, then the dx sum, both streamed through the
+    // region's shared memory (drouter_stream, dx_stream)
     if (alive) {
-        // router-gradient partials: five teams of two warps per CTA, one item each
-        const int n_items = a.chunk_start[a.E] * (a.H / 256);
-        const int hb = a.H / 256;
-        constexpr int teams = kFusedThreads / 64;
-        const int team = warp >> 1;
-        float(*s_acc)[256] = reinterpret_cast<float(*)[256]>(smem) + team * 8;
-        for (int item = blockIdx.x * teams + team; item < n_items; item += gridDim.x * teams)
-            drouter_partial_team(item / hb, (item % hb) * 256, warp & 1, threadIdx.x & 31, 1 + team, a.x, a.dl,
-                                 a.offsets, a.chunk_start, a.perm, a.partial, a.H, a.E, a.k, a.chunk_rows, s_acc);
-        __syncthreads();                       // the teams' scratch is free again
-        const long long n = static_cast<long long>(a.T) * (a.H / 8);
-        for (long long i = gtid; i < n; i += gstride)
-            dx_combine_elem<8>(i, a.dxs, a.dl, a.topk_idx, a.router_w, a.dx, a.H, a.k, a.S);
+        drouter_stream(a.x, a.dl, a.offsets, a.chunk_start, a.perm, a.partial, a.H, a.E, a.k, a.chunk_rows, smem);
+        __syncthreads();                       // the region is free again
+        dx_stream(a.dxs, a.dl, a.topk_idx, a.router_w, a.dx, a.T, a.H, a.k, a.S, smem, F::REGION);
     }
     fused_bwd_stamp(a, 6);
     alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);

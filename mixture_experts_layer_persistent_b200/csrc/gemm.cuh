@@ -420,12 +420,36 @@ __device__ __forceinline__ void signal_ready(int *ctr, int lane)
     __syncwarp();
 }
 
-// Producer lane: wait for every M tile of group g (bounded, as wait_ready).
-__device__ __forceinline__ bool wait_group_ready(const GemmArgs &a, int g, volatile int *abort, int *status)
+// Producer warp: wait for every M tile of group g (bounded, as wait_ready).  The
+// 32 lanes check 32 M tiles' counters at a time (one round trip for a group of up
+// to 4096 rows); the warp barrier and a fence then order every lane's acquire
+// before the loads lane 0 issues.  Callers check a group once per CTA: a CTA's
+// tiles (work units) of one group are claimed one after another.
+__device__ __forceinline__ bool wait_group_ready(const GemmArgs &a, int g, int lane, volatile int *abort,
+                                                 int *status)
 {
     const int m0 = a.mt_base[g], m1 = a.mt_base[g + 1];
-    for (int mt = m0; mt < m1; ++mt)
-        if (!wait_ready(a.ready + mt, a.ready_target, abort, status)) return false;
+    const uint64_t t0 = globaltimer();
+    for (int base = m0; base < m1; base += 32) {
+        const int mt = base + lane;
+        for (uint32_t i = 0;; ++i) {
+            const bool done = mt >= m1 || ld_acquire_gpu(a.ready + mt) >= a.ready_target;
+            if (__all_sync(0xffffffffu, done)) break;
+            if ((i & 63u) == 63u) {
+                const bool give_up = lane == 0 && (*abort || globaltimer() - t0 > kWaitLimitNs);
+                if (__any_sync(0xffffffffu, give_up)) {
+                    if (lane == 0) {
+                        *abort = 1;
+                        atomicOr(status, kStatusTimeout);
+                    }
+                    return false;
+                }
+            }
+        }
+    }
+    __syncwarp();
+    __threadfence();
+    fence_proxy_async_global();
     return true;
 }
 
@@ -521,6 +545,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
         int stage = 0;
         uint32_t phase = 0;
         int fills = 0;                   // stages whose loads this producer issued
+        int ready_g = -1;                // ragged K: last group found complete
         int tile = blockIdx.x;
         for (int it = 0;; ++it) {
             bool put = true;
@@ -528,8 +553,10 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                 if (args.ready_role == kReadyWaitGroup && tile < total) {
                     // the group's rows of the contiguous operand come from an earlier phase
                     const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
-                    if (lane == 0) put = wait_group_ready(args, t.g, abort_flag, status);
-                    put = __shfl_sync(0xffffffffu, put, 0);
+                    if (t.g != ready_g) {
+                        put = wait_group_ready(args, t.g, lane, abort_flag, status);
+                        ready_g = t.g;
+                    }
                     if (!put) tile = total;
                 }
             } else {

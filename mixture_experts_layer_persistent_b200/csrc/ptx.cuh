@@ -175,6 +175,12 @@ __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
 }
 
+// cp.async groups: close the copies issued since the last commit into a group;
+// wait until at most N of this thread's groups are still in flight.
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // Arrive on `bar` once all cp.async copies issued so far by this thread have
 // landed (the arrival is counted in the barrier's initial count).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar)

@@ -158,6 +158,7 @@ __device__ __forceinline__ void wgrad_resident_phase(uint8_t *smem, uint64_t *ba
         // ------------------------------------------------------------ TMA producer (contiguous operand)
         int stage = 0;
         uint32_t phase = 0, bphase = 0;
+        int ready_g = -1;                  // last group found complete
         int fills = 0;                   // ring stages whose loads this producer issued
         uint32_t bfill = 0;              // bit kb: parity of the next fill of resident block kb
         uint32_t bfilled = 0;            // bit kb: resident block kb filled by TMA at least once
@@ -181,10 +182,10 @@ __device__ __forceinline__ void wgrad_resident_phase(uint8_t *smem, uint64_t *ba
                     bfilled |= 1u << kb;
                 }
             } else {
-                if (args.ready_role == kReadyWaitGroup) {
+                if (args.ready_role == kReadyWaitGroup && w.g != ready_g) {
                     // the group's A rows come from an earlier phase of the launch
-                    if (lane == 0) ok = wait_group_ready(args, w.g, abort_flag, status);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    ok = wait_group_ready(args, w.g, lane, abort_flag, status);
+                    ready_g = w.g;
                     if (!ok) break;
                 }
                 // A = rows krow0.. of the contiguous [R, M] matrix, columns of M tile mt
