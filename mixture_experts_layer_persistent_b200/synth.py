@@ -55,16 +55,6 @@ WORKLOADS = {
                            seed=3),
     "dsv3_zipf": Workload("dsv3_zipf", T=16384, H=7168, E=256, k=8, I=2048, S=1, Is=2048,
                           score_fn=1, n_group=8, topk_group=4, zipf=1.2, seed=4),
-    # DeepSeek-V3 expert shape with 32 experts: small enough for kernel captures
-    # (about 6 GB on the device with gradients) while every operand exceeds L2
-    "dsv3_e32": Workload("dsv3_e32", T=1024, H=7168, E=32, k=8, I=2048, S=1, Is=2048,
-                         score_fn=1, n_group=8, topk_group=4, seed=5),
-    # the same with 128 rows per routed expert on average, as in dsv3
-    "dsv3_e32_r128": Workload("dsv3_e32_r128", T=512, H=7168, E=32, k=8, I=2048, S=1, Is=2048,
-                              score_fn=1, n_group=8, topk_group=4, seed=6),
-    # MXFP8 forward with 256 rows per routed expert on average, as in dsv3_mxfp8
-    "dsv3_mxfp8_e32": Workload("dsv3_mxfp8_e32", T=1024, H=7168, E=32, k=8, I=2048, S=1, Is=2048,
-                               score_fn=1, n_group=8, topk_group=4, mxfp8=True, backward=False, seed=7),
     # 16 routed experts of the DeepSeek-V3 shape, 128 rows each on average (as dsv3), for
     # per-kernel counter captures: about 3 GB on the device with gradients, every weight
     # tensor larger than L2
