@@ -42,9 +42,12 @@ class Cfg(ctypes.Structure):
                 ("act_kind", ctypes.c_int), ("w_kind", ctypes.c_int), ("r_kind", ctypes.c_int)]
 
 
+_INPUTS = ("x", "Wr", "bias", "lbias", "Wgu", "Wdn", "Wgu_s", "Wdn_s", "dy",
+           "Wgu_b", "Wdn_b", "Wgu_sb", "Wdn_sb")
+
+
 class Inputs(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in
-                ("x", "Wr", "bias", "lbias", "Wgu", "Wdn", "Wgu_s", "Wdn_s", "dy")]
+    _fields_ = [(n, ctypes.c_void_p) for n in _INPUTS]
 
 
 _lib = None
@@ -73,6 +76,7 @@ def lib():
         _lib.orc_mx_scale_exp.argtypes = [d]
         _lib.orc_mx_quantize.argtypes = [p, i64, i64, p, p]
         _lib.orc_mx_fakequant_bf16.argtypes = [p, i64, i64]
+        _lib.orc_mx_fakequant_cols_bf16.argtypes = [p, i64, i64, i64]
         cp = ctypes.POINTER(Cfg)
         ip = ctypes.POINTER(Inputs)
         _lib.orc_route.argtypes = [cp, p, p, p, p, p, i, p, p, p, p, p]
@@ -108,6 +112,9 @@ class Layer:
 
     x, dy, expert weights: uint16 bf16 bit patterns (or float64 for finite
     differences); router_w, e_bias, logit_bias: float32 (or float64).
+    MXFP8 backward: Wgu_b, Wdn_b (Wgu_sb, Wdn_sb) are the weight copies
+    fake-quantised along the data-gradient contraction axis
+    (mx_fakequant_cols_bf16), needed by bwd, drouter and the dw functions.
     """
 
     def __init__(self, T, H, E, k, I, S=0, Is=0, score_fn=0, n_group=1, topk_group=1,
@@ -126,7 +133,7 @@ class Layer:
         self.cfg.act_kind = _kind(x)
         self.cfg.w_kind = _kind(self.arrays.get("Wgu"))
         self.cfg.r_kind = _kind(self.arrays.get("Wr"))
-        for name in ("x", "Wr", "bias", "lbias", "Wgu", "Wdn", "Wgu_s", "Wdn_s", "dy"):
+        for name in _INPUTS:
             setattr(self.inp, name, _ptr(self.arrays.get(name)))
         return self
 
@@ -203,8 +210,9 @@ class Layer:
         G = np.zeros((n, c.k))
         idx = np.ascontiguousarray(idx, np.int32)
         w = np.ascontiguousarray(w, np.float64)
-        lib().orc_bwd_tokens(ctypes.byref(c), ctypes.byref(self.inp), _ptr(idx), _ptr(w),
-                             _ptr(tokens), n, _ptr(dx), _ptr(dl), _ptr(G))
+        rc = lib().orc_bwd_tokens(ctypes.byref(c), ctypes.byref(self.inp), _ptr(idx), _ptr(w),
+                                  _ptr(tokens), n, _ptr(dx), _ptr(dl), _ptr(G))
+        assert rc == 0, "MXFP8 backward needs the weight copies Wgu_b, Wdn_b (Wgu_sb, Wdn_sb)"
         return dx, dl, G
 
     def drouter(self, idx, w, experts):
@@ -222,10 +230,11 @@ class Layer:
         I = c.Is if shared else c.I
         dgu = np.zeros((2 * I, c.H))
         ddn = np.zeros((c.H, I))
-        lib().orc_dw_full(ctypes.byref(c), ctypes.byref(self.inp),
-                          _ptr(np.ascontiguousarray(idx, np.int32)),
-                          _ptr(np.ascontiguousarray(w, np.float64)), group, int(shared),
-                          _ptr(dgu), _ptr(ddn))
+        rc = lib().orc_dw_full(ctypes.byref(c), ctypes.byref(self.inp),
+                               _ptr(np.ascontiguousarray(idx, np.int32)),
+                               _ptr(np.ascontiguousarray(w, np.float64)), group, int(shared),
+                               _ptr(dgu), _ptr(ddn))
+        assert rc >= 0
         return dgu, ddn
 
     def dw_entries(self, idx, w, group, shared, which, rows, cols):
@@ -233,10 +242,11 @@ class Layer:
         rows = np.ascontiguousarray(rows, np.int32)
         cols = np.ascontiguousarray(cols, np.int32)
         out = np.zeros(len(rows))
-        lib().orc_dw_entries(ctypes.byref(c), ctypes.byref(self.inp),
-                             _ptr(np.ascontiguousarray(idx, np.int32)),
-                             _ptr(np.ascontiguousarray(w, np.float64)), group, int(shared), which,
-                             _ptr(rows), _ptr(cols), len(rows), _ptr(out))
+        rc = lib().orc_dw_entries(ctypes.byref(c), ctypes.byref(self.inp),
+                                  _ptr(np.ascontiguousarray(idx, np.int32)),
+                                  _ptr(np.ascontiguousarray(w, np.float64)), group, int(shared), which,
+                                  _ptr(rows), _ptr(cols), len(rows), _ptr(out))
+        assert rc >= 0
         return out
 
 
@@ -277,6 +287,15 @@ def mx_fakequant_bf16(bits: np.ndarray) -> None:
     K = bits.shape[-1]
     rows = bits.size // K
     assert lib().orc_mx_fakequant_bf16(_ptr(bits), rows, K) == 0
+
+
+def mx_fakequant_cols_bf16(bits: np.ndarray) -> None:
+    """In place: bf16 bits [..., R, C] -> MXFP8-dequantised values with blocks of 32
+    consecutive rows of each column (quantisation along R)."""
+    assert bits.dtype == np.uint16 and bits.flags.c_contiguous and bits.ndim >= 2
+    R, C = bits.shape[-2:]
+    batch = bits.size // (R * C)
+    assert lib().orc_mx_fakequant_cols_bf16(_ptr(bits), batch, R, C) == 0
 
 
 def num_threads() -> int:

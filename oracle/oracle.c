@@ -34,6 +34,18 @@
  * block rule below; weights are fake-quantised by the caller with
  * orc_mx_fakequant_bf16 before use.
  *
+ * MXFP8 backward (not claimed by the pages; the plain reading of "MXFP8
+ * training" applied to this layer): the two data-gradient products run on
+ * MXFP8 operands quantised along their own contraction axis -- dy along H for
+ * dy . W_down, and dGU along 2I (blocks of 32 inside the gate and the up half)
+ * for dGU . W_gate_up, with weight copies that the caller fake-quantises along
+ * that axis (orc_mx_fakequant_cols_bf16: W_down along H, W_gate_up along 2I).
+ * dGU is quantised from its unrounded value.  The slot gradient is read off the
+ * same product, G_j = <Q(dy) . W_down, Q(h_j)>, as the layer's fused epilogue
+ * does.  The weight gradients stay BF16 products: dW_gate_up from the stored
+ * bf16 dGU and the quantised x the forward used, dW_down from the bf16 dy and
+ * bf16(w Q(h)).
+ *
  * Pins.  Every function here is checked by tests that do not call it to
  * produce their own expected values: brute-force top-k, closed forms of the
  * weights, permutation invariants, a dense SwiGLU MLP via library matmuls,
@@ -205,6 +217,26 @@ int orc_mx_fakequant_bf16(uint16_t *data, int64_t rows, int64_t K)
     return 0;
 }
 
+/* Replace a bf16 tensor [batch, R, C] in place by its MXFP8-dequantised values
+ * with blocks of 32 consecutive rows of each column (quantisation along R, the
+ * axis a product with the transposed matrix contracts over). */
+int orc_mx_fakequant_cols_bf16(uint16_t *data, int64_t batch, int64_t R, int64_t C)
+{
+    if (R % 32) return -1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < batch; b++)
+        for (int64_t c = 0; c < C; c++) {
+            double v[32];
+            uint16_t *m = data + b * R * C + c;
+            for (int64_t r0 = 0; r0 < R; r0 += 32) {
+                for (int i = 0; i < 32; i++) v[i] = bf16_bits_to_d(m[(r0 + i) * C]);
+                mx_block(v, 32, NULL, NULL);
+                for (int i = 0; i < 32; i++) m[(r0 + i) * C] = orc_bf16_bits(v[i]);
+            }
+        }
+    return 0;
+}
+
 static inline double mirror(const orc_cfg *c, double v) { return c->pure ? v : orc_round_bf16(v); }
 
 /* ---------------------------------------------------------------- routing */
@@ -354,21 +386,26 @@ int orc_dispatch(const orc_cfg *c, const int32_t *idx, int32_t *counts, int32_t 
 
 typedef struct {
     const void *x, *Wr, *bias, *lbias, *Wgu, *Wdn, *Wgu_s, *Wdn_s, *dy;
+    /* MXFP8 backward: the weight copies quantised along the data-gradient
+     * contraction axis (same layouts as Wgu, Wdn, Wgu_s, Wdn_s) */
+    const void *Wgu_b, *Wdn_b, *Wgu_sb, *Wdn_sb;
 } orc_inputs;
 
 /* the weights of slot j of a token: routed expert idx[j] for j < k, shared
- * expert j-k otherwise */
-typedef struct { const void *Wgu; const void *Wdn; int64_t gu_off, dn_off; int I; } slot_w;
+ * expert j-k otherwise (Wgu_b, Wdn_b: the MXFP8 backward's copies) */
+typedef struct { const void *Wgu, *Wdn, *Wgu_b, *Wdn_b; int64_t gu_off, dn_off; int I; } slot_w;
 
 static slot_w slot_weights(const orc_cfg *c, const orc_inputs *in, int e_or_shared, int shared)
 {
     slot_w s;
     if (!shared) {
         s.Wgu = in->Wgu; s.Wdn = in->Wdn; s.I = c->I;
+        s.Wgu_b = in->Wgu_b; s.Wdn_b = in->Wdn_b;
         s.gu_off = (int64_t)e_or_shared * 2 * c->I * c->H;
         s.dn_off = (int64_t)e_or_shared * c->H * c->I;
     } else {
         s.Wgu = in->Wgu_s; s.Wdn = in->Wdn_s; s.I = c->Is;
+        s.Wgu_b = in->Wgu_sb; s.Wdn_b = in->Wdn_sb;
         s.gu_off = (int64_t)e_or_shared * 2 * c->Is * c->H;
         s.dn_off = (int64_t)e_or_shared * c->H * c->Is;
     }
@@ -512,15 +549,18 @@ static void dlogits_token(const orc_cfg *c, const double *prob, const int *idx, 
 }
 
 /* SwiGLU backward of one row: dh given, g/u as stored (mirrored to bf16).
- * dg = dh u sig(g) (1 + g (1 - sig(g))), du = dh silu(g); both stored bf16. */
+ * dg = dh u sig(g) (1 + g (1 - sig(g))), du = dh silu(g); both stored bf16.
+ * raw (or NULL): the same two halves before the bf16 mirror. */
 static void swiglu_bwd(const orc_cfg *c, const double *g, const double *u, const double *dh, int I,
-                       double *dgu)
+                       double *dgu, double *raw)
 {
     for (int i = 0; i < I; i++) {
         double gb = mirror(c, g[i]), ub = mirror(c, u[i]);
         double sg = 1.0 / (1.0 + exp(-gb));
-        dgu[i] = mirror(c, dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)));
-        dgu[I + i] = mirror(c, dh[i] * gb * sg);
+        double dg = dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)), du = dh[i] * gb * sg;
+        dgu[i] = mirror(c, dg);
+        dgu[I + i] = mirror(c, du);
+        if (raw) { raw[i] = dg; raw[I + i] = du; }
     }
 }
 
@@ -534,24 +574,99 @@ static void down_dgrad(const orc_cfg *c, const slot_w *s, const double *dO, doub
     }
 }
 
+/* MXFP8 backward: a = Q(dy) W_down with the copy quantised along H (dyq is the
+ * row already quantised per 1x32 block) */
+static void down_dgrad_mx(const orc_cfg *c, const slot_w *s, const double *dyq, double *a)
+{
+    for (int i = 0; i < s->I; i++) a[i] = 0.0;
+    for (int n = 0; n < c->H; n++) {
+        double d = dyq[n];
+        for (int i = 0; i < s->I; i++) a[i] += d * ld(s->Wdn_b, s->dn_off + (int64_t)n * s->I + i, c->w_kind);
+    }
+}
+
+/* dy row of token t: dyd as stored (bf16), dyq quantised per 1x32 block along H
+ * in MXFP8 mode (the operand of the MXFP8 down dgrad), else a copy */
+static void load_dy(const orc_cfg *c, const void *dy, int t, double *dyd, double *dyq)
+{
+    for (int q = 0; q < c->H; q++) dyd[q] = dyq[q] = ld(dy, (int64_t)t * c->H + q, c->act_kind);
+    if (c->mx)
+        for (int b = 0; b < c->H; b += 32) mx_block(dyq + b, 32, NULL, NULL);
+}
+
+/* MXFP8 backward inputs present (the weight copies of the data gradients) */
+static int mx_bwd_ready(const orc_cfg *c, const orc_inputs *in)
+{
+    if (!c->mx) return 1;
+    if (c->I % 32 || !in->Wgu_b || !in->Wdn_b) return 0;
+    if (c->S && (c->Is % 32 || !in->Wgu_sb || !in->Wdn_sb)) return 0;
+    return 1;
+}
+
+/* One slot's data gradients.  h: the slot's h as the forward stored it (for G);
+ * dyd/dyq: the token's dy row (as stored / quantised); wj: routing weight.
+ * Writes dgu [2I] (stored bf16 values), the per-slot dx row dxs [H] (fp32 on the
+ * layer: unrounded) and, when G is given, G = <dy, o_j> (BF16: o_j = h Wd^T;
+ * MXFP8: <Q(dy) Wd, Q(h)> from the quantised product, the fused epilogue's value). */
+static void slot_backward(const orc_cfg *c, const slot_w *s, const double *g, const double *u, const double *h,
+                          const double *dyd, const double *dyq, double wj, double *dh, double *dgu,
+                          double *raw, double *dxs, double *G)
+{
+    const int H = c->H, I = s->I;
+    if (!c->mx) {
+        if (G) {
+            double a = 0.0;
+            for (int n = 0; n < H; n++) {
+                double o = 0.0;
+                for (int i = 0; i < I; i++) o += h[i] * ld(s->Wdn, s->dn_off + (int64_t)n * I + i, c->w_kind);
+                a += dyd[n] * o;
+            }
+            *G = a;
+        }
+        for (int q = 0; q < H; q++) dxs[q] = wj * dyd[q];          /* dO, reused as scratch */
+        down_dgrad(c, s, dxs, dh);
+    } else {
+        down_dgrad_mx(c, s, dyq, dh);
+        if (G) {
+            double a = 0.0;
+            for (int i = 0; i < I; i++) a += dh[i] * h[i];
+            *G = a;
+        }
+        for (int i = 0; i < I; i++) dh[i] *= wj;
+    }
+    swiglu_bwd(c, g, u, dh, I, dgu, raw);
+    const void *Wg = c->mx ? s->Wgu_b : s->Wgu;
+    const double *op = dgu;
+    if (c->mx) {                                   /* Q(dGU) per 1x32 block of each half */
+        for (int b = 0; b < 2 * I; b += 32) mx_block(raw + b, 32, NULL, NULL);
+        op = raw;
+    }
+    for (int q = 0; q < H; q++) {
+        double a = 0.0;
+        for (int i = 0; i < 2 * I; i++) a += op[i] * ld(Wg, s->gu_off + (int64_t)i * H + q, c->w_kind);
+        dxs[q] = a;
+    }
+}
+
 /* per-token backward: dx [n, H], dlogit [n, k], G [n, k] (any may be NULL but dx) */
 int orc_bwd_tokens(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, const double *w,
                    const int32_t *tokens, int n, double *dx, double *dlogit, double *Gout)
 {
     const int H = c->H, k = c->k, kk = c->k + c->S, E = c->E;
     const int Im = c->I > c->Is ? c->I : c->Is;
+    if (!mx_bwd_ready(c, in)) return -1;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int ti = 0; ti < n; ti++) {
         int t = tokens[ti];
-        double *xd = (double *)malloc(sizeof(double) * (4 * H + 6 * Im + 2 * E + 2 * k));
-        double *dyd = xd + H, *acc = dyd + H, *dO = acc + H;
-        double *g = dO + H, *u = g + Im, *h = u + Im, *dh = h + Im, *dgu = dh + Im;  /* dgu: 2 Im */
-        double *lgt = dgu + 2 * Im, *prob = lgt + E, *G = prob + E, *dl = G + k;
-        double *o = (double *)malloc(sizeof(double) * H);
+        double *xd = (double *)malloc(sizeof(double) * (5 * H + 8 * Im + 2 * E + 2 * k));
+        double *dyd = xd + H, *dyq = dyd + H, *acc = dyq + H, *dxs = acc + H;
+        double *g = dxs + H, *u = g + Im, *h = u + Im, *dh = h + Im, *dgu = dh + Im, *raw = dgu + 2 * Im;
+        double *lgt = raw + 2 * Im, *prob = lgt + E, *G = prob + E, *dl = G + k;
         int id[256];
         double ww[256];
         load_x(c, in->x, t, xd);
-        for (int q = 0; q < H; q++) { dyd[q] = ld(in->dy, (int64_t)t * H + q, c->act_kind); acc[q] = 0.0; }
+        load_dy(c, in->dy, t, dyd, dyq);
+        for (int q = 0; q < H; q++) acc[q] = 0.0;
         route_token(c, in->x, in->Wr, in->bias, in->lbias, t, id, ww, lgt, prob);
         for (int j = 0; j < k; j++) {
             id[j] = idx[(int64_t)t * k + j];
@@ -562,21 +677,9 @@ int orc_bwd_tokens(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, c
             slot_w s = slot_weights(c, in, shared ? j - k : id[j], shared);
             double wj = shared ? 1.0 : ww[j];
             gate_up(c, &s, xd, g, u);
-            if (!shared) {
-                swiglu_h(c, g, u, s.I, h);
-                down(c, &s, h, o);
-                double a = 0.0;
-                for (int q = 0; q < H; q++) a += dyd[q] * o[q];
-                G[j] = a;
-            }
-            for (int q = 0; q < H; q++) dO[q] = wj * dyd[q];
-            down_dgrad(c, &s, dO, dh);
-            swiglu_bwd(c, g, u, dh, s.I, dgu);
-            for (int q = 0; q < H; q++) {
-                double a = 0.0;
-                for (int i = 0; i < 2 * s.I; i++) a += dgu[i] * ld(s.Wgu, s.gu_off + (int64_t)i * H + q, c->w_kind);
-                acc[q] += a;                      /* per-slot dx rows are stored in fp32 */
-            }
+            swiglu_h(c, g, u, s.I, h);
+            slot_backward(c, &s, g, u, h, dyd, dyq, wj, dh, dgu, raw, dxs, shared ? NULL : &G[j]);
+            for (int q = 0; q < H; q++) acc[q] += dxs[q];     /* per-slot dx rows are stored in fp32 */
         }
         dlogits_token(c, prob, id, ww, G, dl);
         for (int q = 0; q < H; q++) {
@@ -586,7 +689,6 @@ int orc_bwd_tokens(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, c
         }
         if (dlogit) for (int j = 0; j < k; j++) dlogit[(int64_t)ti * k + j] = dl[j];
         if (Gout) for (int j = 0; j < k; j++) Gout[(int64_t)ti * k + j] = G[j];
-        free(o);
         free(xd);
     }
     return 0;
@@ -639,12 +741,15 @@ static int group_rows(const orc_cfg *c, const int32_t *idx, const double *w, int
  *   which = 0: dW_gate_up[n, q] = sum_r dGU_r[n] x[tok_r, q]          (n < 2I)
  *   which = 1: dW_down[q, i]    = sum_r dy[tok_r, q] hw_r[i],  hw = bf16(w_r h_r)
  * Rows r ascending in token.  rows/cols: ne entry coordinates; out: ne values
- * (bf16-mirrored like the layer's outputs). */
+ * (bf16-mirrored like the layer's outputs).  MXFP8 mode: x and h as the forward
+ * quantised them, dGU from the MXFP8 down dgrad (Q(dy) with the copy of W_down
+ * quantised along H). */
 int orc_dw_entries(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, const double *w,
                    int grp, int shared, int which, const int32_t *rows, const int32_t *cols, int ne,
                    double *out)
 {
     const int H = c->H;
+    if (!mx_bwd_ready(c, in)) return -1;
     slot_w s = slot_weights(c, in, grp, shared);
     const int I = s.I;
     int32_t *tok = (int32_t *)malloc(sizeof(int32_t) * (c->T + 1));
@@ -655,25 +760,45 @@ int orc_dw_entries(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, c
     for (int q = 0; q < ne; q++) {
         int a = rows[q], b = cols[q];
         int i = which == 0 ? (a % I) : b;            /* the inter index involved */
+        int i0 = c->mx ? i / 32 * 32 : i, nb = c->mx ? 32 : 1;   /* MX: the whole block of i */
         double sum = 0.0;
-        double *xd = (double *)malloc(sizeof(double) * H);
+        double *xd = (double *)malloc(sizeof(double) * (3 * H + 64));
+        double *dyd = xd + H, *dyq = dyd + H, *hb = dyq + H;
         for (int r = 0; r < m; r++) {
             int t = tok[r];
             load_x(c, in->x, t, xd);
             double g = 0.0, u = 0.0;
-            for (int h = 0; h < H; h++) {
-                g += xd[h] * ld(s.Wgu, s.gu_off + (int64_t)i * H + h, c->w_kind);
-                u += xd[h] * ld(s.Wgu, s.gu_off + (int64_t)(I + i) * H + h, c->w_kind);
+            for (int v = 0; v < nb; v++) {
+                int iv = i0 + v;
+                double gv = 0.0, uv = 0.0;
+                for (int h = 0; h < H; h++) {
+                    gv += xd[h] * ld(s.Wgu, s.gu_off + (int64_t)iv * H + h, c->w_kind);
+                    uv += xd[h] * ld(s.Wgu, s.gu_off + (int64_t)(I + iv) * H + h, c->w_kind);
+                }
+                hb[v] = silu(gv) * uv;
+                if (iv == i) { g = gv; u = uv; }
             }
             if (which == 1) {
-                double hh = mirror(c, silu(g) * u);
+                double hh;
+                if (c->mx) {
+                    mx_block(hb, 32, NULL, NULL);
+                    hh = hb[i - i0];
+                } else {
+                    hh = mirror(c, hb[0]);
+                }
                 double hw = mirror(c, wr[r] * hh);
                 sum += ld(in->dy, (int64_t)t * H + a, c->act_kind) * hw;
             } else {
                 double dh = 0.0;
-                for (int n = 0; n < H; n++)
-                    dh += wr[r] * ld(in->dy, (int64_t)t * H + n, c->act_kind) *
-                          ld(s.Wdn, s.dn_off + (int64_t)n * I + i, c->w_kind);
+                if (c->mx) {
+                    load_dy(c, in->dy, t, dyd, dyq);
+                    for (int n = 0; n < H; n++) dh += dyq[n] * ld(s.Wdn_b, s.dn_off + (int64_t)n * I + i, c->w_kind);
+                    dh *= wr[r];
+                } else {
+                    for (int n = 0; n < H; n++)
+                        dh += wr[r] * ld(in->dy, (int64_t)t * H + n, c->act_kind) *
+                              ld(s.Wdn, s.dn_off + (int64_t)n * I + i, c->w_kind);
+                }
                 double gb = mirror(c, g), ub = mirror(c, u);
                 double sg = 1.0 / (1.0 + exp(-gb));
                 double d = a < I ? dh * ub * sg * (1.0 + gb * (1.0 - sg)) : dh * gb * sg;
@@ -693,6 +818,7 @@ int orc_dw_full(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, cons
                 int shared, double *dWgu, double *dWdn)
 {
     const int H = c->H;
+    if (!mx_bwd_ready(c, in)) return -1;
     slot_w s = slot_weights(c, in, grp, shared);
     const int I = s.I;
     int32_t *tok = (int32_t *)malloc(sizeof(int32_t) * (c->T + 1));
@@ -703,18 +829,22 @@ int orc_dw_full(const orc_cfg *c, const orc_inputs *in, const int32_t *idx, cons
     double *HW = (double *)malloc(sizeof(double) * ((int64_t)m * I + 1));
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < m; r++) {
-        double *g = (double *)malloc(sizeof(double) * (5 * I + H));
-        double *u = g + I, *h = u + I, *dh = h + I, *dO = dh + I;
+        double *g = (double *)malloc(sizeof(double) * (4 * I + 3 * H));
+        double *u = g + I, *h = u + I, *dh = h + I, *dyd = dh + I, *dyq = dyd + H, *dO = dyq + H;
         int t = tok[r];
         load_x(c, in->x, t, X + (int64_t)r * H);
         gate_up(c, &s, X + (int64_t)r * H, g, u);
-        for (int i = 0; i < I; i++) {
-            double hh = mirror(c, silu(g[i]) * u[i]);
-            HW[(int64_t)r * I + i] = mirror(c, wr[r] * hh);
+        swiglu_h(c, g, u, I, h);                  /* stored h: bf16, or MX blocks */
+        for (int i = 0; i < I; i++) HW[(int64_t)r * I + i] = mirror(c, wr[r] * h[i]);
+        load_dy(c, in->dy, t, dyd, dyq);
+        if (c->mx) {
+            down_dgrad_mx(c, &s, dyq, dh);
+            for (int i = 0; i < I; i++) dh[i] *= wr[r];
+        } else {
+            for (int q = 0; q < H; q++) dO[q] = wr[r] * dyd[q];
+            down_dgrad(c, &s, dO, dh);
         }
-        for (int q = 0; q < H; q++) dO[q] = wr[r] * ld(in->dy, (int64_t)t * H + q, c->act_kind);
-        down_dgrad(c, &s, dO, dh);
-        swiglu_bwd(c, g, u, dh, I, DGU + (int64_t)r * 2 * I);
+        swiglu_bwd(c, g, u, dh, I, DGU + (int64_t)r * 2 * I, NULL);
         free(g);
     }
 #pragma omp parallel for schedule(static)

@@ -86,10 +86,12 @@ MUTATIONS = [
      "dl[j] = rho / S * (G[j] - gbar) * s * (1.0 - s);", "dl[j] = rho / S * (G[j] - gbar) * s;",
      "test_gradients_match_finite_differences"),
     ("silu_derivative_term_dropped",
-     "dgu[i] = mirror(c, dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)));", "dgu[i] = mirror(c, dh[i] * ub * sg);",
+     "double dg = dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)), du = dh[i] * gb * sg;",
+     "double dg = dh[i] * ub * sg, du = dh[i] * gb * sg;",
      "test_gradients_match_finite_differences"),
     ("du_uses_g_not_silu",
-     "dgu[I + i] = mirror(c, dh[i] * gb * sg);", "dgu[I + i] = mirror(c, dh[i] * gb);",
+     "double dg = dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)), du = dh[i] * gb * sg;",
+     "double dg = dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)), du = dh[i] * gb;",
      "test_gradients_match_finite_differences"),
     ("dx_misses_router_path",
      "dx[(int64_t)ti * H + q] = mirror(c, acc[q] + r);", "dx[(int64_t)ti * H + q] = mirror(c, acc[q]);",
@@ -102,7 +104,7 @@ MUTATIONS = [
      "dh[i] += d * ld(s->Wdn, s->dn_off + (int64_t)i * c->H + n, c->w_kind);",
      "test_gradients_match_finite_differences"),
     ("dw_down_unweighted_h",
-     "HW[(int64_t)r * I + i] = mirror(c, wr[r] * hh);", "HW[(int64_t)r * I + i] = mirror(c, hh);",
+     "HW[(int64_t)r * I + i] = mirror(c, wr[r] * h[i]);", "HW[(int64_t)r * I + i] = mirror(c, h[i]);",
      "test_gradients_match_finite_differences"),
     # top-k margins (the gap margin rejection reads) and non-finite scores
     ("gap_on_unbiased_scores",
@@ -123,11 +125,13 @@ MUTATIONS = [
      "double gb = mirror(c, g[i]), ub = mirror(c, u[i]);", "double gb = g[i], ub = u[i];",
      "test_backward_mirrors_sit_at_stored_tensors"),
     ("dh_rounded_instead_of_dgu",
-     "dgu[i] = mirror(c, dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)));\n        dgu[I + i] = mirror(c, dh[i] * gb * sg);",
-     "dgu[i] = mirror(c, dh[i]) * ub * sg * (1.0 + gb * (1.0 - sg));\n        dgu[I + i] = mirror(c, dh[i]) * gb * sg;",
+     "double dg = dh[i] * ub * sg * (1.0 + gb * (1.0 - sg)), du = dh[i] * gb * sg;\n        dgu[i] = mirror(c, dg);\n"
+     "        dgu[I + i] = mirror(c, du);",
+     "double dg = mirror(c, dh[i]) * ub * sg * (1.0 + gb * (1.0 - sg)), du = mirror(c, dh[i]) * gb * sg;\n"
+     "        dgu[i] = dg;\n        dgu[I + i] = du;",
      "test_backward_mirrors_sit_at_stored_tensors"),
     ("wh_not_rounded",
-     "HW[(int64_t)r * I + i] = mirror(c, wr[r] * hh);", "HW[(int64_t)r * I + i] = wr[r] * hh;",
+     "HW[(int64_t)r * I + i] = mirror(c, wr[r] * h[i]);", "HW[(int64_t)r * I + i] = wr[r] * h[i];",
      "test_backward_mirrors_sit_at_stored_tensors"),
     ("dx_not_rounded",
      "dx[(int64_t)ti * H + q] = mirror(c, acc[q] + r);", "dx[(int64_t)ti * H + q] = acc[q] + r;",
@@ -136,8 +140,8 @@ MUTATIONS = [
      "dWgu[(int64_t)n * H + q] = mirror(c, a);", "dWgu[(int64_t)n * H + q] = a;",
      "test_backward_mirrors_sit_at_stored_tensors"),
     ("slot_dx_rows_rounded",
-     "acc[q] += a;                      /* per-slot dx rows are stored in fp32 */",
-     "acc[q] += mirror(c, a);",
+     "acc[q] += dxs[q];     /* per-slot dx rows are stored in fp32 */",
+     "acc[q] += mirror(c, dxs[q]);",
      "test_backward_mirrors_sit_at_stored_tensors"),
     # number formats
     ("bf16_truncates",
@@ -155,12 +159,39 @@ MUTATIONS = [
      "while (amax > ldexp(448.0, e)) e++;", "while (amax >= ldexp(448.0, e)) e++;",
      "test_mx_scale_golden"),
     ("mx_x_not_quantised",
-     "if (c->mx)\n        for (int b = 0; b < c->H; b += 32)", "if (0)\n        for (int b = 0; b < c->H; b += 32)",
+     "if (c->mx)\n        for (int b = 0; b < c->H; b += 32) mx_block(xd + b",
+     "if (0)\n        for (int b = 0; b < c->H; b += 32) mx_block(xd + b",
      "test_mxfp8_single_expert_matches_fakequant_mlp"),
     ("mx_h_not_quantised",
      "for (int b = 0; b < I; b += 32) mx_block(h + b, 32, NULL, NULL);",
      "for (int b = 0; b < 0; b += 32) mx_block(h + b, 32, NULL, NULL);",
      "test_mxfp8_single_expert_matches_fakequant_mlp"),
+    # MXFP8 backward (the data-gradient products on MXFP8 operands)
+    ("mx_dy_not_quantised",
+     "if (c->mx)\n        for (int b = 0; b < c->H; b += 32) mx_block(dyq + b",
+     "if (0)\n        for (int b = 0; b < c->H; b += 32) mx_block(dyq + b",
+     "test_mxfp8_backward_restated"),
+    ("mx_down_dgrad_reads_forward_copy",
+     "a[i] += d * ld(s->Wdn_b,", "a[i] += d * ld(s->Wdn,",
+     "test_mxfp8_backward_restated"),
+    ("mx_gate_up_dgrad_reads_forward_copy",
+     "const void *Wg = c->mx ? s->Wgu_b : s->Wgu;", "const void *Wg = s->Wgu;",
+     "test_mxfp8_backward_restated"),
+    ("mx_slot_grad_after_routing_weight",
+     "        down_dgrad_mx(c, s, dyq, dh);\n        if (G) {",
+     "        down_dgrad_mx(c, s, dyq, dh);\n        for (int i = 0; i < I; i++) dh[i] *= wj;\n        if (G) {",
+     "test_mxfp8_backward_restated"),
+    ("mx_dgu_not_quantised",
+     "for (int b = 0; b < 2 * I; b += 32) mx_block(raw + b, 32, NULL, NULL);",
+     "for (int b = 0; b < 0; b += 32) mx_block(raw + b, 32, NULL, NULL);",
+     "test_mxfp8_backward_restated"),
+    ("mx_dw_down_unquantised_h",
+     "swiglu_h(c, g, u, I, h);                  /* stored h: bf16, or MX blocks */",
+     "for (int i = 0; i < I; i++) h[i] = mirror(c, silu(g[i]) * u[i]);",
+     "test_mxfp8_backward_restated"),
+    ("mx_column_blocks_skipped",
+     "for (int64_t r0 = 0; r0 < R; r0 += 32) {", "for (int64_t r0 = 0; r0 < R; r0 += 64) {",
+     "test_mx_fakequant_cols_is_rows_of_transpose"),
 ]
 CONTROL = ("control", None, None, None)
 

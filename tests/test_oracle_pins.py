@@ -603,3 +603,123 @@ def test_backward_mirrors_sit_at_stored_tensors():
         HW = _rb(np.array([r[1] * r[2] for r in rs]).reshape(len(rs), -1))     # stored w*h
         np.testing.assert_allclose(dgu_full, _rb(DGU.T @ xd[toks]), rtol=1e-9, atol=1e-12)
         np.testing.assert_allclose(ddn_full, _rb(dyd[toks].T @ HW), rtol=1e-9, atol=1e-12)
+
+
+# ------------------------------------------------------------------ MXFP8 backward
+def _fq_rows(a):
+    """MXFP8 fake-quantisation of each row of `a` [..., K] in blocks of 32: scale
+    exponent by the golden rule (smallest e with amax <= 448 * 2^e), codes by
+    torch's e4m3 conversion of a / 2^e."""
+    a = np.asarray(a, np.float64)
+    out = np.empty_like(a)
+    flat, res = a.reshape(-1, a.shape[-1]), out.reshape(-1, a.shape[-1])
+    for r in range(flat.shape[0]):
+        for b in range(0, flat.shape[1], 32):
+            blk = flat[r, b:b + 32]
+            amax = np.abs(blk).max()
+            e = -127
+            if amax > 0:
+                e = math.frexp(amax)[1] - 10
+                while amax > 448.0 * 2.0 ** e:
+                    e += 1
+            q = torch.from_numpy((blk / 2.0 ** e).astype(np.float32)).to(torch.float8_e4m3fn)
+            res[r, b:b + 32] = q.float().numpy() * 2.0 ** e
+    return out
+
+
+def test_mx_fakequant_cols_is_rows_of_transpose():
+    rng = np.random.default_rng(96)
+    W = _rand_bf16(rng, (3, 64, 40), 0.3)
+    got = W.copy()
+    oracle.mx_fakequant_cols_bf16(got)
+    want = np.stack([_fq_rows(_bits_to_f64(W[b]).T).T for b in range(3)])
+    assert np.array_equal(_bits_to_f64(got), want)
+
+
+def test_mxfp8_backward_restated():
+    """MXFP8 backward: dx and the weight gradients equal a numpy restatement in
+    which only the two data-gradient products take MXFP8 operands -- dy quantised
+    along H times W_down quantised along H, and dGU (quantised from its unrounded
+    value, blocks of 32 inside each half) times W_gate_up quantised along 2I --
+    with the slot gradient read off the first product against the forward's
+    quantised h; the weight gradients are bf16 products of the stored dGU and the
+    quantised x, and of dy and bf16(w Q(h)).  Softmax scoring, one shared expert."""
+    rng = np.random.default_rng(97)
+    T, H, E, k, I, Is = 16, 64, 4, 2, 32, 32
+    x = _rand_bf16(rng, (T, H), 1.0)
+    dy = _rand_bf16(rng, (T, H), 1.0)
+    Wr = rng.standard_normal((E, H)).astype(np.float32) / 8
+    # rows of 2^0 .. 2^-19 magnitude: along a row an MX block holds values of one size, so it
+    # keeps 4 significant bits; down a column it spans 19 binades, and the smallest values
+    # fall below the e4m3 normal range of the block's scale -- the two copies differ there
+    def graded(shape):
+        a = rng.standard_normal(shape) * 0.1 * 2.0 ** -(np.arange(shape[1]) % 20)[None, :, None]
+        return _f32_to_bf16_bits_torch(a.astype(np.float32))
+    raw = {"Wgu": graded((E, 2 * I, H)), "Wdn": graded((E, H, I)), "Wgu_s": graded((1, 2 * Is, H)),
+           "Wdn_s": graded((1, H, Is))}
+    fwd, bwd = {}, {}
+    for n, a in raw.items():                  # forward copies along the last axis, backward along the other
+        fwd[n] = a.copy()
+        oracle.mx_fakequant_bf16(fwd[n])
+        bwd[n] = a.copy()
+        oracle.mx_fakequant_cols_bf16(bwd[n])
+        assert (fwd[n] != bwd[n]).mean() > 0.01
+    L = oracle.Layer(T, H, E, k, I, S=1, Is=Is, mx=True).set(
+        x=x, Wr=Wr, dy=dy, Wgu=fwd["Wgu"], Wdn=fwd["Wdn"], Wgu_s=fwd["Wgu_s"], Wdn_s=fwd["Wdn_s"],
+        Wgu_b=bwd["Wgu"], Wdn_b=bwd["Wdn"], Wgu_sb=bwd["Wgu_s"], Wdn_sb=bwd["Wdn_s"])
+    idx, w, _ = L.route()
+    dx, _, G = L.bwd(idx, w)
+    xq, dyd = _fq_rows(_bits_to_f64(x)), _bits_to_f64(dy)
+    dyq = _fq_rows(dyd)
+    Wr64 = Wr.astype(np.float64)
+
+    def mats(shared, e):
+        f = lambda n: _bits_to_f64(fwd[n + ("_s" if shared else "")][e])
+        b = lambda n: _bits_to_f64(bwd[n + ("_s" if shared else "")][e])
+        gu, dn, gub, dnb = f("Wgu"), f("Wdn"), b("Wgu"), b("Wdn")
+        n2 = len(gu) // 2
+        return gu[:n2], gu[n2:], dn, gub, dnb
+
+    def slot(t, shared, e, wj):
+        Wg, Wu, Wd, Wgub, Wdnb = mats(shared, e)
+        g, u = Wg @ xq[t], Wu @ xq[t]
+        hq = _fq_rows(g / (1 + np.exp(-g)) * u)                 # the forward's quantised h
+        a = Wdnb.T @ dyq[t]                                      # Q(dy) W_down (copy along H)
+        dh = wj * a
+        gb, ub = _rb(g), _rb(u)
+        sg = 1 / (1 + np.exp(-gb))
+        dgu_raw = np.concatenate([dh * ub * sg * (1 + gb * (1 - sg)), dh * gb * sg])
+        dxs = Wgub.T @ _fq_rows(dgu_raw)                          # Q(dGU) W_gate_up (copy along 2I)
+        return a @ hq, hq, _rb(dgu_raw), dxs
+
+    want_dx, want_G = np.zeros((T, H)), np.zeros((T, k))
+    rows = {g: [] for g in [(False, e) for e in range(E)] + [(True, 0)]}
+    for t in range(T):
+        acc = np.zeros(H)
+        for j in range(k + 1):
+            shared = j == k
+            e = 0 if shared else idx[t, j]
+            wj = 1.0 if shared else w[t, j]
+            Gj, hq, dgu, dxs = slot(t, shared, e, wj)
+            acc += dxs
+            if not shared:
+                want_G[t, j] = Gj
+            rows[(shared, e)].append((t, wj, hq, dgu))
+        dl = w[t] * (want_G[t] - (w[t] * want_G[t]).sum())
+        want_dx[t] = _rb(acc + dl @ Wr64[idx[t]])
+    np.testing.assert_allclose(G, want_G, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(dx, want_dx, rtol=1e-9, atol=1e-12)
+    for (shared, e), rs in rows.items():
+        dgu_full, ddn_full = L.dw_full(idx, w, e, shared)
+        toks = [r[0] for r in rs]
+        DGU = np.array([r[3] for r in rs]).reshape(len(rs), -1)
+        HW = _rb(np.array([r[1] * r[2] for r in rs]).reshape(len(rs), -1))
+        want_gu, want_dn = _rb(DGU.T @ xq[toks]), _rb(dyd[toks].T @ HW)
+        np.testing.assert_allclose(dgu_full, want_gu, rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(ddn_full, want_dn, rtol=1e-9, atol=1e-12)
+        r_, c_ = np.array([0, 5, 2 * (Is if shared else I) - 1]), np.array([3, H - 1, 17])
+        np.testing.assert_allclose(L.dw_entries(idx, w, e, shared, 0, r_, c_), want_gu[r_, c_], rtol=1e-9,
+                                   atol=1e-12)
+        r_, c_ = np.array([0, H - 1, 9]), np.array([0, 31, 20])
+        np.testing.assert_allclose(L.dw_entries(idx, w, e, shared, 1, r_, c_), want_dn[r_, c_], rtol=1e-9,
+                                   atol=1e-12)
