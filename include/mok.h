@@ -4,7 +4,8 @@
  * The layer is the one the pages centre on: a DeepSeek-V3-type MoE layer
  * ("Cursor åpner megakernelen som ga 41 prosent flere tokens i sekundet",
  * last paragraph), forward in BF16 and MXFP8 and backward in BF16
- * ("Megakernels are dead and back…", section "Números de MoK"), computed
+ * ("Megakernels are dead and back…", section "Números de MoK"; the MXFP8
+ * backward below is this library's extension, not claimed there), computed
  * deterministically with no CPU-GPU synchronisation inside the layer
  * ("Cursor veröffentlicht MoE-Megakernel Mixture-of-Kittens als Open Source",
  * section "Kommunikation im Kernel").  All experts live on one GPU.
@@ -55,7 +56,7 @@ extern "C" {
 #define MOK_SCORE_SIGMOID 1       /* sigmoid scores + selection bias, group-limited top-k */
 
 #define MOK_DTYPE_BF16 0          /* bf16 operands, fp32 accumulation */
-#define MOK_DTYPE_MXFP8 1         /* e4m3 operands with 1x32 ue8m0 block scales (forward only) */
+#define MOK_DTYPE_MXFP8 1         /* e4m3 operands with 1x32 ue8m0 block scales */
 
 typedef struct moe_cfg {
     int32_t T;            /* tokens in the batch, >= 1 */
@@ -83,6 +84,14 @@ typedef struct moe_cfg {
  * (contraction) axis, for the tensors [E*2I, H] and [E*H, I] (S in place of E
  * for the shared experts), in the packed weight-scale layout that
  * moe_quantize_mxfp8_weights writes.
+ * The MXFP8 backward also reads the weights quantised along the other axis,
+ * transposed, as moe_quantize_mxfp8_weights_t writes them:
+ *   wt_down    [E, I, H] e4m3: W_down[e]^T quantised along H; st_down its scales
+ *              (packed layout of the [E*I, H] tensor)
+ *   wt_gate_up [E, H, 2I] e4m3: W_gate_up[e]^T quantised along 2I; st_gate_up its
+ *              scales (packed layout of the [E*H, 2I] tensor)
+ *   wst_*, sst_* the same for the shared experts.
+ * They are ignored (and may be NULL) otherwise.
  */
 typedef struct moe_params {
     const float *router_w;      /* [E, H] fp32 */
@@ -96,6 +105,14 @@ typedef struct moe_params {
     const void *ws_down;
     const uint8_t *ss_gate_up;
     const uint8_t *ss_down;
+    const void *wt_gate_up;
+    const void *wt_down;
+    const uint8_t *st_gate_up;
+    const uint8_t *st_down;
+    const void *wst_gate_up;
+    const void *wst_down;
+    const uint8_t *sst_gate_up;
+    const uint8_t *sst_down;
 } moe_params;
 
 /* Routing record (device pointers; any may be NULL to skip that output). */
@@ -149,16 +166,28 @@ int moe_workspace_size(const moe_cfg *cfg, size_t *ctx_bytes, size_t *fwd_scratc
  * score (as -inf), so every token still gets top_k distinct experts in
  * [0, E) (ties to the lower index); such a token's weights and outputs are
  * NaN.  Other tokens are unaffected.
+ * MOK_DTYPE_MXFP8 with save_for_backward != 0 also keeps, for moe_bwd, the
+ * gate/up pre-activations, the dequantised h and w * h (bf16) and the
+ * dequantised x.
  */
 int moe_fwd(const moe_cfg *cfg, const void *x, const moe_params *params, void *y,
             const moe_routing *routing, void *ctx, size_t ctx_bytes, int save_for_backward,
             void *scratch, size_t scratch_bytes, void *stream);
 
 /*
- * Backward pass (MOK_DTYPE_BF16 only).  x and dy: [T, H] bf16 (device); ctx:
- * the buffer a moe_fwd call with save_for_backward != 0 filled for the same x
- * and params.  Computes dx, the expert weight gradients and the router weight
- * gradient (the selection bias gets none) with fixed reduction orders.
+ * Backward pass.  x and dy: [T, H] bf16 (device); ctx: the buffer a moe_fwd
+ * call with save_for_backward != 0 filled for the same x and params.  Computes
+ * dx, the expert weight gradients and the router weight gradient (the
+ * selection bias gets none) with fixed reduction orders.
+ * MOK_DTYPE_MXFP8: the two data-gradient GEMMs take MXFP8 operands quantised
+ * along their contraction axis -- dy (1x32 blocks along H) times wt_down, and
+ * dGU = d(gate, up) (1x32 blocks along 2I, quantised from fp32 in the down
+ * dgrad's epilogue) times wt_gate_up; the slot gradients come from the first
+ * product against the forward's quantised h; the weight gradients are BF16
+ * GEMMs (dW_gate_up from the bf16 dGU and the dequantised x, dW_down from dy
+ * and the saved w * h).  It needs the wt_* / st_* (and wst_* / sst_*) params
+ * and I a multiple of 256 (MOK_ERR_UNSUPPORTED otherwise), and runs as a
+ * sequence of kernels whatever the schedule (the one-launch backward is BF16).
  */
 int moe_bwd(const moe_cfg *cfg, const void *x, const void *dy, const moe_params *params,
             const void *ctx, size_t ctx_bytes, const moe_grads *grads, void *scratch,
@@ -207,6 +236,19 @@ int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *
  */
 int moe_quantize_mxfp8_weights(const void *src, int64_t rows, int64_t K, void *q, void *scales,
                                void *stream);
+
+/*
+ * Transposed weight quantisation for the MXFP8 backward: src [batch, R, C]
+ * bf16 (device) -> q [batch, C, R] e4m3 (row (b, c) of the [batch*C, R] matrix
+ * is column c of src[b]), quantised along R in blocks of 32 with the rule of
+ * moe_quantize_mxfp8, and scales in the packed weight-scale layout of that
+ * [batch*C, R] matrix (as moe_quantize_mxfp8_weights).  R and batch*C must be
+ * multiples of 128, C a multiple of 32 (MOK_ERR_INVALID otherwise).  W_down
+ * [E, H, I] gives wt_down (R = H, C = I); W_gate_up [E, 2I, H] gives
+ * wt_gate_up (R = 2I, C = H).
+ */
+int moe_quantize_mxfp8_weights_t(const void *src, int64_t batch, int64_t R, int64_t C, void *q,
+                                 void *scales, void *stream);
 
 /*
  * Phase tracing.  When events are set, every later moe_fwd (moe_bwd) records
@@ -266,11 +308,12 @@ int moe_fwd_static(const moe_cfg *cfg, const void *x, const moe_params *params, 
  * and until that buffer is next written.  R = T * (top_k + n_shared) sorted
  * rows: the routed rows expert-major (the order of moe_routing.perm), then
  * n_shared blocks of T rows (shared expert s, token t at row T*top_k + s*T + t).
- *   MOK_SAVED_H          [R, I] bf16 h = silu(g) u (BF16 layer)
+ *   MOK_SAVED_H          [R, I] bf16 h = silu(g) u (BF16 layer; MXFP8 with
+ *                        save_for_backward: the dequantised h)
  *   MOK_SAVED_HQ         [R, I] e4m3 codes of h (MXFP8 layer)
  *   MOK_SAVED_HS         [R, I/32] ue8m0 scale bytes of h, row-major (MXFP8 layer)
- *   MOK_SAVED_GU         [R, 2I] bf16 gate and up pre-activations (BF16, save_for_backward)
- *   MOK_SAVED_HW         [R, I] bf16 routing weight times h (BF16, save_for_backward)
+ *   MOK_SAVED_GU         [R, 2I] bf16 gate and up pre-activations (save_for_backward)
+ *   MOK_SAVED_HW         [R, I] bf16 routing weight times h (save_for_backward)
  *   MOK_SAVED_ROW_TOKEN  [R] int32 token of each sorted row
  *   MOK_SAVED_ROW_W      [R] fp32 routing weight of each sorted row (1 for shared rows)
  * Returns MOK_ERR_UNSUPPORTED when the configuration keeps no such tensor and

@@ -47,7 +47,8 @@ class moe_cfg(ctypes.Structure):
 class moe_params(ctypes.Structure):
     _fields_ = [(n, _vp) for n in ("router_w", "e_bias", "logit_bias", "w_gate_up", "w_down",
                                     "s_gate_up", "s_down", "ws_gate_up", "ws_down", "ss_gate_up",
-                                    "ss_down")]
+                                    "ss_down", "wt_gate_up", "wt_down", "st_gate_up", "st_down",
+                                    "wst_gate_up", "wst_down", "sst_gate_up", "sst_down")]
 
 
 class moe_routing(ctypes.Structure):
@@ -89,6 +90,8 @@ def lib():
                                    _vp, _sz, _vp]
         L.moe_quantize_mxfp8.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
         L.moe_quantize_mxfp8_weights.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
+        L.moe_quantize_mxfp8_weights_t.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _vp, _vp,
+                                                   _vp]
         L.moe_status.argtypes = [_vp, P(_i32)]
         L.moe_trace_events.argtypes = [P(_vp), ctypes.c_int, P(_vp), ctypes.c_int]
         L.moe_fwd_static.argtypes = [P(moe_cfg), _vp, P(moe_params), _vp, _vp]
@@ -103,7 +106,8 @@ def lib():
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
-                     "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_quantize_mxfp8_weights", "moe_status",
+                     "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_quantize_mxfp8_weights",
+                     "moe_quantize_mxfp8_weights_t", "moe_status",
                      "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal", "moe_saved_tensor",
                      "moe_set_schedule", "moe_get_schedule", "moe_trace_device"):
             getattr(L, name).restype = ctypes.c_int
@@ -190,6 +194,10 @@ def moe_quantize_mxfp8(src, rows, K, q, scales, stream):
 
 def moe_quantize_mxfp8_weights(src, rows, K, q, scales, stream):
     _check("moe_quantize_mxfp8_weights", lib().moe_quantize_mxfp8_weights(src, rows, K, q, scales, stream))
+
+
+def moe_quantize_mxfp8_weights_t(src, batch, R, C, q, scales, stream):
+    _check("moe_quantize_mxfp8_weights_t", lib().moe_quantize_mxfp8_weights_t(src, batch, R, C, q, scales, stream))
 
 
 def moe_status(stream) -> int:

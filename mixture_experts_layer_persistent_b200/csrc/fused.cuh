@@ -76,6 +76,7 @@ struct FusedFwdArgs {
     int T, H, E, k, S;
     const __nv_bfloat16 *x;        // MXFP8: quantised into xq, xs
     uint8_t *xq, *xs;
+    __nv_bfloat16 *xdq;            // MXFP8 training: the dequantised x (or null)
     // P1-P4
     GemmArgs gr, ga, gd;
     SelectArgs sa;
@@ -219,7 +220,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     for (long long i = gtid; i < static_cast<long long>(a.E) * a.H; i += gstride) router_split_elem(i, a.router_w, a.wr3, a.H);
     if constexpr (MX) {
         const long long nb = static_cast<long long>(a.T) * a.H / 32;
-        for (long long b = gtid; b < nb; b += gstride) quantize_block(b, a.x, a.xq, a.xs, a.H / 32, 0);
+        for (long long b = gtid; b < nb; b += gstride) quantize_block(b, a.x, a.xq, a.xs, a.H / 32, 0, a.xdq);
     }
     fused_stamp(a, 1);
     int nb = 0;                                      // barriers passed

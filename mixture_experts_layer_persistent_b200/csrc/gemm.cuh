@@ -67,7 +67,10 @@ struct GemmArgs {
     int sf_ld;                    // A scale bytes per row (K / 32)
     int sfb_row_tiles;            // 128-row blocks of the routed weight tensor
     int sfb_row_tiles_s;          // 128-row blocks of the shared weight tensor
-    uint8_t *out_scales;          // MXFP8 SwiGLU epilogue: scales of h [R, I/32]
+    uint8_t *out_scales;          // MXFP8 SwiGLU epilogue: scales of h [R, I/32]; MXFP8 SwiGLU-backward
+                                  // epilogue: scales of dGU [R, 2I/32]
+    uint8_t *out_q;               // MXFP8 SwiGLU-backward epilogue: e4m3 codes of dGU [R, 2I]
+    __nv_bfloat16 *out_hb;        // MXFP8 SwiGLU epilogue, training: the dequantised h [R, I] (with out2, out3)
     __nv_bfloat16 *out;           // main output
     __nv_bfloat16 *out_s;         // EPI_WGRAD: output of the shared groups
     __nv_bfloat16 *out2;          // EPI_SWIGLU: saved gate/up pre-activations [R, 2I] (or null)
@@ -148,8 +151,9 @@ struct GemmCfg {
     // standalone kernel: ring, then the phase's barrier block, group tables and TMEM slot
     static constexpr int SMEM_BYTES = 1024 + RING_BYTES + kGemmBarBytes + kGemmAuxBytes + 16;
     static constexpr uint32_t IDESC = idesc_bf16(BM, BN, A_MN, B_MN);
-    static_assert(!MX || (!A_MN && !B_MN && !RAGGED_K && BN == 256 && (EPI == EPI_SWIGLU || EPI == EPI_PUSH)),
-                  "MXFP8 serves the forward expert GEMMs");
+    static_assert(!MX || (!A_MN && !B_MN && !RAGGED_K && BN == 256 &&
+                          (EPI == EPI_SWIGLU || EPI == EPI_PUSH || EPI == EPI_DSWIGLU)),
+                  "MXFP8 serves the K-major expert GEMMs: the forward's and the data gradients'");
     static_assert(BN == 128 || BN == 256, "BN");
     static_assert(!RAGGED_K || (A_MN && B_MN), "weight gradients take both operands MN-major");
     static_assert(!RAGGED_K || (A_GATHER != B_GATHER), "one operand of a weight gradient is gathered");
@@ -354,6 +358,29 @@ __device__ __forceinline__ void store_row_direct(void *dst, const uint32_t *p)
     uint4 *d = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
     for (int c = 0; c < 8; ++c) d[c] = make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+}
+
+// 64 bytes (32 bf16) of this lane's own row with plain 16-byte stores
+__device__ __forceinline__ void store_row64(void *dst, const uint32_t *p)
+{
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) d[c] = make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+}
+
+// One 1x32 MXFP8 block of this lane's row: 32 e4m3 codes at q, the ue8m0 byte at sc
+__device__ __forceinline__ void mx_store_block(const float (&v)[32], uint8_t *q, uint8_t *sc)
+{
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int e = mx_exponent(amax);
+    uint32_t w[8];
+    mx_codes32(v, e, w);
+    uint4 *d = reinterpret_cast<uint4 *>(q);
+    d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    *sc = static_cast<uint8_t>(e + 127);
 }
 
 // 128 bytes of this lane's own row (null = zeros) straight into registers: the
@@ -894,6 +921,14 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         tmem_ld32(taddr + 32 * (blk + 1), gb[(blk + 1) & 1]);
                         tmem_ld32(taddr + 128 + 32 * (blk + 1), ub[(blk + 1) & 1]);
                     }
+                    if (args.out2 && valid) {
+                        // training: the gate and up pre-activations as bf16
+                        uint32_t pg[16], pu[16];
+                        pack_bf16<32>(g, pg);
+                        pack_bf16<32>(u, pu);
+                        store_row64(args.out2 + (size_t)r * 2 * I + n0 + 32 * blk, pg);
+                        store_row64(args.out2 + (size_t)r * 2 * I + I + n0 + 32 * blk, pu);
+                    }
                     float amax = 0.0f;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -912,6 +947,20 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         q[8 * blk + i] = word;
                     }
                     sc |= static_cast<uint32_t>(e + 127) << (8 * blk);
+                    if (args.out_hb && valid) {
+                        // training: the dequantised h (exact in bf16) and w times it, rounded
+                        const float w = args.row_w[r];
+                        uint32_t ph[16], pw[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const uint32_t word = q[8 * blk + (i >> 1)] >> (16 * (i & 1));
+                            const float h0 = mx_decode(word, e), h1 = mx_decode(word >> 8, e);
+                            ph[i] = pack_bf16x2(h0, h1);
+                            pw[i] = pack_bf16x2(w * h0, w * h1);
+                        }
+                        store_row64(args.out_hb + (size_t)r * I + n0 + 32 * blk, ph);
+                        store_row64(args.out3 + (size_t)r * I + n0 + 32 * blk, pw);
+                    }
                     if (blk < 3) tmem_ld_wait();
                     if (blk == 2) {
                         tc_fence_before();
@@ -965,19 +1014,35 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                     }
                 }
             } else if constexpr (C::EPI == EPI_PUSH && C::MX) {
-                // MXFP8 forward: bf16 rows pushed into their (token, slot) row
                 const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
-                __nv_bfloat16 *dst = args.out + (size_t)dst_row * args.ldo + t.nt * C::BN;
+                if (args.out_f32) {
+                    // MXFP8 gate/up dgrad: fp32 rows pushed into their (token, slot) row
+                    float *dst = args.out_f32 + (size_t)dst_row * args.ldo + t.nt * C::BN;
 #pragma unroll 1
-                for (int c = 0; c < C::BN; c += 64) {
-                    float v[64];
-                    uint32_t p[32];
-                    tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
-                    tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-                    tmem_ld_wait();
-                    pack_bf16<64>(v, p);
-                    if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
-                    else if (valid) store_row_direct(dst + c, p);
+                    for (int c = 0; c < C::BN; c += 32) {
+                        float v[32];
+                        uint32_t p[32];
+                        tmem_ld32(taddr + c, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
+                        if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
+                        else if (valid) store_row_direct(dst + c, p);
+                    }
+                } else {
+                    // MXFP8 forward: bf16 rows pushed into their (token, slot) row
+                    __nv_bfloat16 *dst = args.out + (size_t)dst_row * args.ldo + t.nt * C::BN;
+#pragma unroll 1
+                    for (int c = 0; c < C::BN; c += 64) {
+                        float v[64];
+                        uint32_t p[32];
+                        tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
+                        tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                        tmem_ld_wait();
+                        pack_bf16<64>(v, p);
+                        if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
+                        else if (valid) store_row_direct(dst + c, p);
+                    }
                 }
             } else if constexpr (C::EPI == EPI_PUSH) {
                 // fp32 rows pushed into their (token, slot) row of the slot buffer
@@ -1058,6 +1123,16 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         }
                         pack_bf16<32>(dg, dgp + 16 * half);
                         pack_bf16<32>(du, dup + 16 * half);
+                        if constexpr (C::MX) {
+                            // MXFP8 backward: dGU quantised per 1x32 block (from fp32) for the gate/up dgrad
+                            if (valid) {
+                                const int cg = n0 + c + 32 * half;
+                                mx_store_block(dg, args.out_q + (size_t)r * 2 * I + cg,
+                                               args.out_scales + (size_t)r * (2 * I / 32) + cg / 32);
+                                mx_store_block(du, args.out_q + (size_t)r * 2 * I + I + cg,
+                                               args.out_scales + (size_t)r * (2 * I / 32) + (I + cg) / 32);
+                            }
+                        }
                     }
                     if (full) {
                         store_block_tile(stg, dgp, lane, &tmO, n0 + c, row0);

@@ -190,6 +190,7 @@ struct State {
     __nv_bfloat16 *gu, *h, *hw;
     float *O;                       // per-(token, slot) rows: fp32 (BF16), bf16 (MXFP8 forward)
     uint8_t *xq, *xs, *hq, *hs;     // MXFP8 operands
+    __nv_bfloat16 *xdq;             // MXFP8 training: the dequantised x (weight-gradient operand)
     int *sched;                     // [kSchedCounters] forward GEMM tile counters
     int *ready;                     // [n_mtiles] per-M-tile readiness (persistent forward)
     int *zero;                      // sched, ready and hist: the counters the persistent forward zeroes
@@ -233,14 +234,18 @@ State carve_state(const moe_cfg &c, void *buf, bool training)
     st.gu = training ? cv.take<__nv_bfloat16>(s.R * 2 * s.I) : nullptr;
     st.hw = training ? cv.take<__nv_bfloat16>(s.R * s.I) : nullptr;
     if (mx) {
-        st.h = nullptr;
+        // training also keeps the dequantised h (the down dgrad's slot-gradient operand)
+        // and the dequantised x (the gate/up weight gradient's operand)
+        st.h = training ? cv.take<__nv_bfloat16>(s.R * s.I) : nullptr;
         st.hq = cv.take<uint8_t>(s.R * s.I);
         st.hs = cv.take<uint8_t>(s.R * s.I / 32);
         st.xq = cv.take<uint8_t>(s.T * s.H);
         st.xs = cv.take<uint8_t>(s.T * s.H / 32);
+        st.xdq = training ? cv.take<__nv_bfloat16>(s.T * s.H) : nullptr;
     } else {
         st.h = cv.take<__nv_bfloat16>(s.R * s.I);
         st.hq = st.hs = st.xq = st.xs = nullptr;
+        st.xdq = nullptr;
     }
     st.O = mx ? reinterpret_cast<float *>(cv.take<__nv_bfloat16>(s.T * s.kk * s.H)) : cv.take<float>(s.T * s.kk * s.H);
     st.bytes = align_up(cv.off, 256);
@@ -257,6 +262,8 @@ struct BwdScratch {
     int n_zero;
     unsigned long long *gs_flags; // grid-barrier tags, release tag, epoch
     int *mt_base;                 // [G + 1] first M tile of each group (persistent backward)
+    uint8_t *dyq, *dys;           // MXFP8: dy codes [T, H] and scales [T, H/32]
+    uint8_t *dguq, *dgus;         // MXFP8: dGU codes [R, 2I] and scales [R, 2I/32]
     size_t bytes;
 };
 
@@ -277,6 +284,12 @@ BwdScratch carve_bwd(const moe_cfg &c, void *buf)
     b.ready = b.zero + kSchedCounters;
     b.gs_flags = cv.take<unsigned long long>(kMaxFusedCtas + 2);
     b.mt_base = cv.take<int>(s.G + 1);
+    if (c.dtype == MOK_DTYPE_MXFP8) {
+        b.dyq = cv.take<uint8_t>(s.T * s.H);
+        b.dys = cv.take<uint8_t>(s.T * s.H / 32);
+        b.dguq = cv.take<uint8_t>(s.R * 2 * s.I);
+        b.dgus = cv.take<uint8_t>(s.R * 2 * s.I / 32);
+    }
     b.bytes = align_up(cv.off, 256);
     return b;
 }
@@ -457,6 +470,9 @@ int build_fwd_plan(const moe_cfg &c, const void *x, const moe_params &p, const S
         ga.num_kb = c.H / 128;
         ga.out = reinterpret_cast<__nv_bfloat16 *>(st.hq);
         ga.out_scales = st.hs;
+        ga.out2 = training ? st.gu : nullptr;       // training: g/u, the dequantised h, w * h
+        ga.out_hb = training ? st.h : nullptr;
+        ga.out3 = training ? st.hw : nullptr;
         ga.gather_src = reinterpret_cast<const __nv_bfloat16 *>(st.xq);
         ga.sfa_src = st.xs;
         ga.sfb_src = p.s_gate_up;
@@ -479,6 +495,7 @@ int build_fwd_plan(const moe_cfg &c, const void *x, const moe_params &p, const S
         gd.out = reinterpret_cast<__nv_bfloat16 *>(st.O);
         gd.out_f32 = nullptr;
         gd.out_scales = nullptr;
+        gd.out2 = gd.out3 = gd.out_hb = nullptr;
         gd.ldo = c.H;
         gd.gather_src = nullptr;
         gd.sfa_src = st.hs;
@@ -564,7 +581,8 @@ int forward_split(const moe_cfg &c, const void *x, const moe_params &p, void *y,
     if (mx) {
         const long long xb = s.T * s.H / 32;
         MOK_TRY(launch_k(quantize_mxfp8_kernel, dim3(blocks_for(xb, 256)), dim3(256), 0, stream, "quantize_mxfp8_kernel",
-                         static_cast<const __nv_bfloat16 *>(x), xb, st.xq, st.xs, static_cast<long long>(s.H / 32), 0ll));
+                         static_cast<const __nv_bfloat16 *>(x), xb, st.xq, st.xs, static_cast<long long>(s.H / 32), 0ll,
+                         st.xdq));
         MOK_TRY(launch_gemm<typename FusedCfg<true>::GateUp>(pl.m.gB, pl.m.gB, pl.m.gBs, pl.m.gO, pl.m.gO2, pl.m.gO3,
                                                             ga, dev.sms, stream));
         MOK_TRY(mark_fwd(3, stream));
@@ -614,6 +632,7 @@ int launch_fused(const moe_cfg &c, const void *x, const moe_params &p, void *y, 
     a.x = static_cast<const __nv_bfloat16 *>(x);
     a.xq = st.xq;
     a.xs = st.xs;
+    a.xdq = st.xdq;
     a.gr = pl.gr;
     a.ga = pl.ga;
     a.gd = pl.gd;
@@ -671,9 +690,19 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
 // ------------------------------------------------------------------ backward
 // Tensor maps and arguments of every step of the backward, shared by the split
 // schedule and the persistent one.
+// MXFP8 backward's data-gradient GEMMs: the down dgrad pulls dy's e4m3 rows by
+// token (as the MXFP8 gate/up forward pulls x) against W_down^T quantised along
+// H, with the SwiGLU-backward epilogue that also quantises dGU; the gate/up dgrad
+// reads those dGU codes (as the MXFP8 down forward reads h's) against
+// W_gate_up^T quantised along 2I and pushes fp32 rows
+using DgradDownMX = GemmCfg<256, false, false, true, false, false, EPI_DSWIGLU, true>;
+using DgradGUMX = GemmCfg<256, false, false, false, false, false, EPI_PUSH, true>;
+
 struct BwdPlan {
     FusedBwdMaps m;
     GemmArgs g1, g2, g3, g4;
+    bool mx;                    // MXFP8 data gradients
+    const void *dy;             // [T, H] bf16 (quantised first under MXFP8)
     int g2_grid, g4_grid;       // split launches of the streaming weight gradients
     int g2_units, g4_units;     // resident weight-gradient work units (0: none)
     bool n256;                  // I is a multiple of 256
@@ -684,6 +713,7 @@ int build_bwd_plan(const moe_cfg &c, const void *x, const void *dy, const moe_pa
 {
     const Shapes s = shapes(c);
     pl.n256 = c.I % 256 == 0;
+    pl.dy = dy;
     GemmArgs base{};
     base.num_groups = static_cast<int>(s.G);
     base.num_routed = c.E;
@@ -757,6 +787,40 @@ int build_bwd_plan(const moe_cfg &c, const void *x, const void *dy, const moe_pa
     g3.ldo = c.H;
     g3.ready_target = 4 * g1.n_tiles;     // four epilogue warps per down-dgrad tile, its N tiles per M tile
 
+    pl.mx = c.dtype == MOK_DTYPE_MXFP8;
+    if (pl.mx) {
+        // down dgrad on MXFP8 operands: dy codes (gathered by token) x W_down^T (K = H)
+        if (!make_tmap(&pl.m.d1B, p.wt_down, s.H, s.E * s.I, 128, 256, 1)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.d1Bs, s.S ? p.wst_down : p.wt_down, s.H, (s.S ? s.S : s.E) * s.I, 128, 256, 1))
+            return MOK_ERR_INVALID;
+        g1.num_kb = c.H / 128;
+        g1.b_rows_per_group = c.I;
+        g1.n_tiles = c.I / 256;
+        g1.gather_src = reinterpret_cast<const __nv_bfloat16 *>(bs.dyq);
+        g1.sfa_src = bs.dys;
+        g1.sf_ld = c.H / 32;
+        g1.sfb_src = p.st_down;
+        g1.sfb_src_s = s.S ? p.sst_down : p.st_down;
+        g1.sfb_row_tiles = static_cast<int>(s.E * s.I / 128);
+        g1.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : s.E) * s.I / 128);
+        g1.out_q = bs.dguq;
+        g1.out_scales = bs.dgus;
+        // gate/up dgrad on MXFP8 operands: dGU codes x W_gate_up^T (K = 2I)
+        if (!make_tmap(&pl.m.d3A, bs.dguq, 2 * s.I, s.R, 128, 128, 1)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.d3B, p.wt_gate_up, 2 * s.I, s.E * s.H, 128, 256, 1)) return MOK_ERR_INVALID;
+        if (!make_tmap(&pl.m.d3Bs, s.S ? p.wst_gate_up : p.wt_gate_up, 2 * s.I, (s.S ? s.S : s.E) * s.H, 128, 256, 1))
+            return MOK_ERR_INVALID;
+        g3.num_kb = 2 * c.I / 128;
+        g3.b_rows_per_group = c.H;
+        g3.gather_src = nullptr;
+        g3.sfa_src = bs.dgus;
+        g3.sf_ld = 2 * c.I / 32;
+        g3.sfb_src = p.st_gate_up;
+        g3.sfb_src_s = s.S ? p.sst_gate_up : p.st_gate_up;
+        g3.sfb_row_tiles = static_cast<int>(s.E * s.H / 128);
+        g3.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : s.E) * s.H / 128);
+    }
+
     // wgrad of gate/up: dW_gate_up[g] = sum_r dGU_r^T x[token r]
     if (!make_tmap(&pl.m.w4A, bs.dgu, 2 * s.I, s.R, 64, 64, 2)) return MOK_ERR_INVALID;
     if (!make_tmap(&pl.m.w4O, gr.dw_gate_up, s.H, s.E * 2 * s.I, 64, 32, 2)) return MOK_ERR_INVALID;
@@ -765,7 +829,7 @@ int build_bwd_plan(const moe_cfg &c, const void *x, const void *dy, const moe_pa
     GemmArgs &g4 = pl.g4;
     g4 = base;
     g4.sched = bs.sched + 3;
-    g4.gather_src = static_cast<const __nv_bfloat16 *>(x);
+    g4.gather_src = pl.mx ? st.xdq : static_cast<const __nv_bfloat16 *>(x);   // MXFP8: the x the forward used
     g4.m_tiles = 2 * c.I / 128;
     g4.n_tiles = c.H / 256;
     g4.out = static_cast<__nv_bfloat16 *>(gr.dw_gate_up);
@@ -794,7 +858,13 @@ int backward_split(const moe_cfg &c, const void *x, const moe_params &p, const S
     const FusedBwdMaps &m = pl.m;
 
     MOK_TRY(mark_bwd(0, stream));
-    if (pl.n256)
+    if (pl.mx) {
+        const long long nb = s.T * s.H / 32;
+        MOK_TRY(launch_k(quantize_mxfp8_kernel, dim3(blocks_for(nb, 256)), dim3(256), 0, stream, "quantize_mxfp8_kernel",
+                         static_cast<const __nv_bfloat16 *>(pl.dy), nb, bs.dyq, bs.dys,
+                         static_cast<long long>(s.H / 32), 0ll, static_cast<__nv_bfloat16 *>(nullptr)));
+        MOK_TRY(launch_gemm<DgradDownMX>(m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1, dev.sms, stream));
+    } else if (pl.n256)
         MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradDown>(m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1,
                                                                   dev.sms, stream));
     else
@@ -829,8 +899,11 @@ int backward_split(const moe_cfg &c, const void *x, const moe_params &p, const S
     }
 
     MOK_TRY(mark_bwd(5, stream));
-    MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradGU>(m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O, g3, dev.sms,
-                                                            stream));
+    if (pl.mx)
+        MOK_TRY(launch_gemm<DgradGUMX>(m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O, g3, dev.sms, stream));
+    else
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradGU>(m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O, g3,
+                                                                dev.sms, stream));
 
     MOK_TRY(mark_bwd(6, stream));
     MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::WgradGU>(m.w4A, m.w4A, m.w4A, m.w4O, m.w4O2, m.w4O, g4, pl.g4_grid,
@@ -925,7 +998,7 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     t_launches = 0;
     BwdPlan pl;
     MOK_TRY(build_bwd_plan(c, x, dy, p, st, gr, bs, dev, pl));
-    if (t_schedule == MOK_SCHEDULE_PERSISTENT) {
+    if (t_schedule == MOK_SCHEDULE_PERSISTENT && !pl.mx) {     // the one-launch backward is BF16
         t_pdl = false;
         return pl.n256 ? launch_fused_bwd<true>(c, x, p, st, gr, bs, dev, pl, stream)
                        : launch_fused_bwd<false>(c, x, p, st, gr, bs, dev, pl, stream);
@@ -970,7 +1043,6 @@ int moe_fwd(const moe_cfg *cfg, const void *x, const moe_params *params, void *y
     const DeviceInfo *dev = device_info();
     if (!dev) return MOK_ERR_DEVICE;
     const bool training = save_for_backward != 0;
-    if (training && cfg->dtype == MOK_DTYPE_MXFP8) return fail(MOK_ERR_UNSUPPORTED, "MXFP8 is forward-only (no saved state)");
     void *buf = training ? ctx : scratch;
     const size_t have = training ? ctx_bytes : scratch_bytes;
     const State need = carve_state(*cfg, nullptr, training);
@@ -985,7 +1057,16 @@ int moe_bwd(const moe_cfg *cfg, const void *x, const void *dy, const moe_params 
 {
     MOK_TRY(check_cfg(cfg));
     MOK_TRY(check_params(*cfg, params));
-    if (cfg->dtype != MOK_DTYPE_BF16) return MOK_ERR_UNSUPPORTED;
+    if (cfg->dtype == MOK_DTYPE_MXFP8) {
+        const moe_params &q = *params;
+        if (!q.wt_gate_up || !q.wt_down || !q.st_gate_up || !q.st_down ||
+            (cfg->n_shared > 0 && (!q.wst_gate_up || !q.wst_down || !q.sst_gate_up || !q.sst_down)))
+            return fail(MOK_ERR_INVALID, "moe_bwd (MXFP8): the transposed weight copies wt_* / st_* are missing");
+        const void *w[] = {q.wt_gate_up, q.wt_down, q.wst_gate_up, q.wst_down};
+        for (const void *v : w)
+            if (v && !aligned16(v)) return MOK_ERR_INVALID;
+        if (cfg->I % 256) return fail(MOK_ERR_UNSUPPORTED, "moe_bwd (MXFP8): I must be a multiple of 256");
+    }
     if (!x || !dy || !grads || !grads->dx || !grads->dw_gate_up || !grads->dw_down || !grads->drouter_w)
         return MOK_ERR_INVALID;
     if (cfg->n_shared > 0 && (!grads->dws_gate_up || !grads->dws_down)) return MOK_ERR_INVALID;
@@ -1068,7 +1149,7 @@ static int quantize(const void *src, int64_t rows, int64_t K, void *q, void *sca
     if (nb == 0) return MOK_OK;
     quantize_mxfp8_kernel<<<blocks_for(nb, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const __nv_bfloat16 *>(src), nb, static_cast<uint8_t *>(q), static_cast<uint8_t *>(scales), K / 32,
-        packed ? rows / 128 : 0);
+        packed ? rows / 128 : 0, static_cast<__nv_bfloat16 *>(nullptr));
     if (const cudaError_t e_ = cudaGetLastError(); e_ != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "quantize_mxfp8_kernel launch", e_);
     return MOK_OK;
@@ -1082,6 +1163,23 @@ int moe_quantize_mxfp8(const void *src, int64_t rows, int64_t K, void *q, void *
 int moe_quantize_mxfp8_weights(const void *src, int64_t rows, int64_t K, void *q, void *scales, void *stream)
 {
     return quantize(src, rows, K, q, scales, true, stream);
+}
+
+int moe_quantize_mxfp8_weights_t(const void *src, int64_t batch, int64_t R, int64_t C, void *q, void *scales,
+                                 void *stream)
+{
+    if (!src || !q || !scales || batch < 0 || R <= 0 || C <= 0) return MOK_ERR_INVALID;
+    if (R % 128 || C % 32 || (batch * C) % 128)
+        return fail(MOK_ERR_INVALID, "moe_quantize_mxfp8_weights_t: R and batch*C must be multiples of 128, C of 32");
+    if (!aligned16(src) || !aligned16(q)) return MOK_ERR_INVALID;
+    if (!device_info()) return MOK_ERR_DEVICE;
+    const long long n = batch * C * (R / 32);
+    if (n == 0) return MOK_OK;
+    quantize_mxfp8_t_kernel<<<blocks_for(n, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16 *>(src), batch, R, C, static_cast<uint8_t *>(q), static_cast<uint8_t *>(scales));
+    if (const cudaError_t e_ = cudaGetLastError(); e_ != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "quantize_mxfp8_t_kernel launch", e_);
+    return MOK_OK;
 }
 
 int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events, int n_bwd)
@@ -1150,7 +1248,6 @@ int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_
 {
     MOK_TRY(check_cfg(cfg));
     const bool training = save_for_backward != 0;
-    if (training && cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
     // carve over a stand-in base address: only the differences are used
     char *const base = reinterpret_cast<char *>(uintptr_t(1) << 40);
     const State st = carve_state(*cfg, base, training);

@@ -7,6 +7,7 @@
 // is e + 127 and every element is x * 2^-e rounded to nearest even e4m3 with
 // saturation.  With this rule no element saturates.
 #pragma once
+#include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include "ptx.cuh"
 
@@ -41,11 +42,35 @@ __device__ __forceinline__ long long packed_scale_offset(long long row, long lon
     return ((j >> 2) * row_tiles + (row >> 7)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (j & 3);
 }
 
+// e4m3 codes (4 per word, low byte first) of 32 values, scaled by 2^-e
+__device__ __forceinline__ void mx_codes32(const float (&v)[32], int e, uint32_t (&w)[8])
+{
+    const float s = exp2_neg(e);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(v[4 * i + j] * s, __NV_SATFINITE, __NV_E4M3);
+            word |= static_cast<uint32_t>(c) << (8 * j);
+        }
+        w[i] = word;
+    }
+}
+
+// value of e4m3 code byte c times 2^e (exact; representable in bf16)
+__device__ __forceinline__ float mx_decode(uint32_t c, int e)
+{
+    const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c & 0xFFu), __NV_E4M3);
+    return ldexpf(__half2float(__half(h)), e);
+}
+
 // Block b (32 elements) of src.  row_tiles = 0: scales [rows, K/32] row-major;
-// row_tiles = rows / 128: packed layout
+// row_tiles = rows / 128: packed layout.  deq (or null): the dequantised values
+// in bf16 (exact), for the MXFP8 backward's weight gradient
 __device__ __forceinline__ void quantize_block(long long b, const __nv_bfloat16 *__restrict__ src,
                                                uint8_t *__restrict__ q, uint8_t *__restrict__ scales, long long kb32,
-                                               long long row_tiles)
+                                               long long row_tiles, __nv_bfloat16 *__restrict__ deq = nullptr)
 {
     const uint4 *p = reinterpret_cast<const uint4 *>(src + b * 32);
     float v[32];
@@ -61,33 +86,62 @@ __device__ __forceinline__ void quantize_block(long long b, const __nv_bfloat16 
 #pragma unroll
     for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
     const int e = mx_exponent(amax);
-    const float s = exp2_neg(e);
     uint32_t w[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(v[4 * i + j] * s, __NV_SATFINITE, __NV_E4M3);
-            word |= static_cast<uint32_t>(c) << (8 * j);
-        }
-        w[i] = word;
-    }
+    mx_codes32(v, e, w);
     uint4 *dst = reinterpret_cast<uint4 *>(q + b * 32);
     dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
     dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     const long long at = row_tiles ? packed_scale_offset(b / kb32, b % kb32, row_tiles) : b;
     scales[at] = static_cast<uint8_t>(e + 127);
+    if (deq) {
+        uint32_t p[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            p[i] = pack_bf16x2(mx_decode(w[i >> 1] >> (16 * (i & 1)), e), mx_decode(w[i >> 1] >> (16 * (i & 1) + 8), e));
+        uint4 *d = reinterpret_cast<uint4 *>(deq + b * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+    }
 }
 
 __global__ void __launch_bounds__(256) quantize_mxfp8_kernel(const __nv_bfloat16 *__restrict__ src,
                                                              long long nblocks, uint8_t *__restrict__ q,
                                                              uint8_t *__restrict__ scales, long long kb32,
-                                                             long long row_tiles)
+                                                             long long row_tiles, __nv_bfloat16 *__restrict__ deq)
 {
     griddep_enter();
     const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (b < nblocks) quantize_block(b, src, q, scales, kb32, row_tiles);
+    if (b < nblocks) quantize_block(b, src, q, scales, kb32, row_tiles, deq);
+}
+
+// Transposed quantisation: thread = (matrix b, column c, 32-row block j) of src
+// [batch, R, C]; its 32 values down the column become row (b*C + c), K block j
+// of q [batch*C, R], scale packed for that matrix (row_tiles = batch*C/128).
+// Consecutive threads take consecutive columns, so each of the 32 row loads of
+// a warp is one 64-byte segment.
+__global__ void __launch_bounds__(256) quantize_mxfp8_t_kernel(const __nv_bfloat16 *__restrict__ src,
+                                                               long long batch, long long R, long long C,
+                                                               uint8_t *__restrict__ q, uint8_t *__restrict__ scales)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long kb32 = R / 32;
+    if (i >= batch * C * kb32) return;
+    const long long c = i % C, j = (i / C) % kb32, b = i / (C * kb32);
+    const __nv_bfloat16 *col = src + (b * R + j * 32) * C + c;
+    float v[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) v[r] = __bfloat162float(col[r * C]);
+    float amax = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 32; ++r) amax = fmaxf(amax, fabsf(v[r]));
+    const int e = mx_exponent(amax);
+    uint32_t w[8];
+    mx_codes32(v, e, w);
+    const long long row = b * C + c;
+    uint4 *dst = reinterpret_cast<uint4 *>(q + row * R + j * 32);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    scales[packed_scale_offset(row, j, batch * C / 128)] = static_cast<uint8_t>(e + 127);
 }
 
 }  // namespace mok

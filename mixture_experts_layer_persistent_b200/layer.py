@@ -33,7 +33,9 @@ class MoELayer:
     """One layer's parameters plus the buffers the C ABI needs.
 
     params: dict of device tensors (router_w, e_bias, logit_bias, w_gate_up,
-    w_down, ws_gate_up, ws_down and, for MXFP8, the s_* scale tensors).
+    w_down, ws_gate_up, ws_down and, for MXFP8, the s_* scale tensors; the MXFP8
+    backward also reads the transposed copies wt_*, st_*, wst_*, sst_* made by
+    quantize_mxfp8_weights_t).
     """
 
     def __init__(self, cfg: abi.moe_cfg, params: dict, training: bool = True, device=None):
@@ -52,7 +54,9 @@ class MoELayer:
             _ptr(p["router_w"]), _ptr(p.get("e_bias")), _ptr(p.get("logit_bias")),
             _ptr(p["w_gate_up"]), _ptr(p["w_down"]), _ptr(p.get("s_gate_up")), _ptr(p.get("s_down")),
             _ptr(p.get("ws_gate_up")), _ptr(p.get("ws_down")), _ptr(p.get("ss_gate_up")),
-            _ptr(p.get("ss_down")))
+            _ptr(p.get("ss_down")), _ptr(p.get("wt_gate_up")), _ptr(p.get("wt_down")),
+            _ptr(p.get("st_gate_up")), _ptr(p.get("st_down")), _ptr(p.get("wst_gate_up")),
+            _ptr(p.get("wst_down")), _ptr(p.get("sst_gate_up")), _ptr(p.get("sst_down")))
 
     def stream(self):
         return torch.cuda.current_stream(self.device).cuda_stream
@@ -142,4 +146,16 @@ def quantize_mxfp8_weights(src: torch.Tensor):
     s = torch.empty(rows * (K // 32), dtype=torch.uint8, device=src.device)
     abi.moe_quantize_mxfp8_weights(src.data_ptr(), rows, K, q.data_ptr(), s.data_ptr(),
                                    torch.cuda.current_stream(src.device).cuda_stream)
+    return q, s
+
+
+def quantize_mxfp8_weights_t(src: torch.Tensor):
+    """Expert weights bf16 [batch, R, C] -> the MXFP8 backward's copy: e4m3 codes
+    [batch, C, R] quantised along R and their scales (flat uint8, packed layout of
+    the [batch*C, R] matrix) via libmok."""
+    batch, R, C = src.shape
+    q = torch.empty((batch, C, R), dtype=torch.uint8, device=src.device)
+    s = torch.empty(batch * C * (R // 32), dtype=torch.uint8, device=src.device)
+    abi.moe_quantize_mxfp8_weights_t(src.data_ptr(), batch, R, C, q.data_ptr(), s.data_ptr(),
+                                     torch.cuda.current_stream(src.device).cuda_stream)
     return q, s

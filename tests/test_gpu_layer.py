@@ -161,3 +161,85 @@ def test_mxfp8_forward_matches_oracle(wl):
     y2 = layer.forward(case["x"])
     torch.cuda.synchronize()
     assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
+
+
+# ---------------------------------------------------------------- MXFP8 backward
+def _mx_train_params(params):
+    from mixture_experts_layer_persistent_b200 import quantize_mxfp8_weights_t
+    out = _mx_params(params)
+    for name, tname, sname in (("w_gate_up", "wt_gate_up", "st_gate_up"), ("w_down", "wt_down", "st_down"),
+                               ("ws_gate_up", "wst_gate_up", "sst_gate_up"), ("ws_down", "wst_down", "sst_down")):
+        if params.get(name) is None:
+            out[tname] = out[sname] = None
+            continue
+        out[tname], out[sname] = quantize_mxfp8_weights_t(params[name])
+    return out
+
+
+def _rel_rms(got, want):
+    got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
+    return float(np.sqrt(np.sum((got - want) ** 2) / max(np.sum(want ** 2), 1e-300)))
+
+
+MX_BWD_CASES = [
+    synth.scaled(MEDIUM_MX, name="medium_mx_bwd", backward=True, seed=24),
+    synth.scaled(MEDIUM_MX, name="medium_mx_bwd_softmax", T=333, score_fn=0, n_group=1, topk_group=1, S=2,
+                 Is=256, backward=True, seed=25),
+]
+
+
+@pytest.mark.parametrize("wl", MX_BWD_CASES, ids=lambda w: w.name)
+def test_mxfp8_backward_matches_oracle(wl):
+    """MXFP8 training step: the forward as above, then dx (pooled and per token), the
+    router weight gradient of the hottest, a median and the lightest routed expert,
+    and the weight gradients of the hottest and a median routed expert and of every
+    shared expert, each within 2e-2 relative RMS of the oracle's MXFP8 backward (the
+    data gradients on MXFP8 operands, the weight gradients BF16); reruns
+    bit-identical."""
+    import oracle
+    case = make_case(wl, device="cuda", gen_device="cpu", mx=True)
+    params = _mx_train_params(case["params"])
+    layer = MoELayer(cfg_for(wl), params, training=True, device=torch.device("cuda"))
+    routing = layer.new_routing()
+    y = layer.forward(case["x"], routing=routing)
+    grads = layer.backward(case["x"], case["dy"])
+    torch.cuda.synchronize()
+    assert layer.status() == 0
+    assert np.array_equal(routing["topk_idx"].cpu().numpy(), case["idx"])
+    L = case["L"]
+    for name in ("Wgu", "Wdn", "Wgu_s", "Wdn_s"):
+        if L.arrays.get(name) is not None:
+            a, b = L.arrays[name].copy(), L.arrays[name].copy()
+            oracle.mx_fakequant_bf16(a)
+            oracle.mx_fakequant_cols_bf16(b)
+            L.set(**{name: a, name.replace("_s", "") + ("_sb" if name.endswith("_s") else "_b"): b})
+    idx, w = case["idx"], case["w"]
+    yo = L.fwd(idx, w)
+    ey, _ = rel_rms_per_token(to_np(y), yo)
+    dxo, _, _ = L.bwd(idx, w)
+    edx, wdx = rel_rms_per_token(to_np(grads["dx"]), dxo)
+    counts = np.bincount(idx.ravel(), minlength=wl.E)
+    order = np.argsort(-counts, kind="stable")
+    experts = [int(order[0]), int(order[len(order) // 2]), int(order[np.nonzero(counts[order])[0][-1]])]
+    edr = _rel_rms(grads["drouter_w"].cpu().numpy()[experts], L.drouter(idx, w, experts))
+    edw = []
+    for grp, shared in [(experts[0], False), (experts[1], False)] + [(s_, True) for s_ in range(wl.S)]:
+        dgu, ddn = L.dw_full(idx, w, grp, shared)
+        gdgu = to_np(grads["dws_gate_up" if shared else "dw_gate_up"][grp])
+        gddn = to_np(grads["dws_down" if shared else "dw_down"][grp])
+        edw += [_rel_rms(gdgu, dgu), _rel_rms(gddn, ddn)]
+    print(f"{wl.name}: relative RMS y {ey:.3g}, dx {edx:.3g} (worst token {wdx:.3g}), dWr {edr:.3g}, "
+          f"dW {max(edw):.3g} (worst of {len(edw)})")
+    for e in (ey, edx, wdx, edr, max(edw)):
+        assert e <= 2e-2, (ey, edx, wdx, edr, edw)
+    # reruns of the training step are bit-identical
+    y2 = layer.forward(case["x"])
+    g2 = layer.backward(case["x"], case["dy"])
+    torch.cuda.synchronize()
+    assert torch.equal(y2.view(torch.int16), y.view(torch.int16))
+    for k, v in grads.items():
+        if v is None:
+            continue
+        a = g2[k].view(torch.int32) if v.dtype == torch.float32 else g2[k].view(torch.int16)
+        b = v.view(torch.int32) if v.dtype == torch.float32 else v.view(torch.int16)
+        assert torch.equal(a, b), k

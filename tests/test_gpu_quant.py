@@ -54,3 +54,26 @@ def test_weight_quantize_packs_the_same_scales(shape):
     at = packed_scale_offsets(np.arange(shape[0]), shape[1] // 32, shape[0])
     assert np.array_equal(np.sort(at.ravel()), np.arange(s.numel()))
     assert np.array_equal(s.cpu().numpy()[at], os_)
+
+
+@pytest.mark.parametrize("shape", [(2, 256, 192), (3, 512, 384)])
+def test_transposed_weight_quantize_matches_oracle(shape):
+    """moe_quantize_mxfp8_weights_t: codes [batch, C, R] and packed scales equal the
+    oracle's quantisation of each transposed matrix (rows of src[b]^T along R),
+    byte for byte, on rows of very different magnitudes (so the blocks down a
+    column hold values far apart)."""
+    from mixture_experts_layer_persistent_b200 import quantize_mxfp8_weights_t
+    from tests._support import packed_scale_offsets
+    batch, R, C = shape
+    g = torch.Generator().manual_seed(R + C)
+    x = torch.randn(shape, generator=g) * torch.exp2(torch.randint(-20, 20, (batch, R, 1), generator=g).float())
+    xb = x.to(torch.bfloat16)
+    q, s = quantize_mxfp8_weights_t(xb.cuda())
+    torch.cuda.synchronize()
+    bits = xb.view(torch.int16).numpy().view(np.uint16)
+    t_bits = np.ascontiguousarray(bits.transpose(0, 2, 1)).reshape(batch * C, R)
+    oq, os_ = oracle.mx_quantize(t_bits)
+    assert np.array_equal(q.cpu().numpy().reshape(batch * C, R), oq)
+    at = packed_scale_offsets(np.arange(batch * C), R // 32, batch * C)
+    assert np.array_equal(np.sort(at.ravel()), np.arange(s.numel()))
+    assert np.array_equal(s.cpu().numpy()[at], os_)
