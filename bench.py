@@ -681,15 +681,20 @@ def bf16_workload_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
 def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
     """Forward tokens/s of the MXFP8 layer (weights quantised once, outside the timed region)."""
     import torch
-    from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, moe_trace_events, quantize_mxfp8_weights, synth
+    from mixture_experts_layer_persistent_b200 import (MoELayer, abi, cfg_for, moe_trace_events, quantize_mxfp8_weights,
+                                                       quantize_mxfp8_weights_t, synth)
     p = synth.draw_params(wl, dev)
     params = {k: p[k] for k in ("router_w", "e_bias", "logit_bias")}
-    for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
-                        ("ws_down", "ss_down")):
+    for name, sname, tname, tsname in (("w_gate_up", "s_gate_up", "wt_gate_up", "st_gate_up"),
+                                       ("w_down", "s_down", "wt_down", "st_down"),
+                                       ("ws_gate_up", "ss_gate_up", "wst_gate_up", "sst_gate_up"),
+                                       ("ws_down", "ss_down", "wst_down", "sst_down")):
         if p.get(name) is None:
-            params[name] = params[sname] = None
+            params[name] = params[sname] = params[tname] = params[tsname] = None
         else:
+            # the forward's copy, and the backward's (transposed, quantised along the other axis)
             params[name], params[sname] = quantize_mxfp8_weights(p[name])
+            params[tname], params[tsname] = quantize_mxfp8_weights_t(p[name])
             p[name] = None
     del p
     torch.cuda.empty_cache()
@@ -728,7 +733,10 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
                   for j, n in enumerate(FWD_PHASES)}
     flops = 6 * wl.H * wl.I * wl.T * (wl.k + wl.S)
     gemm_ms = max(1e-9, phases["gate_up_gemm"] + phases["down_gemm"])
-    del layer, params, x, y
+    del layer
+    torch.cuda.empty_cache()
+    train = mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist)
+    del params, x, y
     torch.cuda.empty_cache()
     # the FP8 denominator: a library FP8 GEMM measured on this GPU in this run; the MXFP8
     # forward loop is short (K forwards of a few ms), so the burst figure is its peak
@@ -746,7 +754,66 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
             "expert_gemm_tc_peak_frac": flops / (gemm_ms / 1e3) / 1e12 / peak,
             "gate_up_tc_peak_frac": 4 * wl.H * wl.I * wl.T * (wl.k + wl.S) / (max(1e-9, phases["gate_up_gemm"]) / 1e3)
             / 1e12 / peak,
+            "device_status": status,
+            "training_step": mxfp8_train_roofline(train, wl, peak, pk["bf16"])}
+
+
+def mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist):
+    """One MXFP8 training step per iteration: the forward with saved state, then the
+    backward (MXFP8 data gradients, BF16 weight gradients), timed together with CUDA
+    events; the backward's steps with the split schedule's events."""
+    import torch
+    from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, moe_trace_events, synth
+    layer = MoELayer(cfg_for(wl), params, training=True, device=dev)
+    dy = synth.draw_dy(wl, dev)
+    grads = layer.new_grads()
+    for _ in range(warmup):
+        layer.forward(x, y)
+        layer.backward(x, dy, grads)
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    bev = [[mk() for _ in range(abi.MOK_BWD_PHASES + 1)] for _ in range(K)]
+    for e in [e for ev in bev for e in ev]:
+        e.record()
+    start, end = mk(), mk()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    start.record()
+    for i in range(K):
+        layer.forward(x, y)
+        moe_trace_events(None, [e.cuda_event for e in bev[i]])
+        layer.backward(x, dy, grads)
+    end.record()
+    torch.cuda.synchronize()
+    moe_trace_events(None, None)
+    status = layer.status()
+    t = torch.tensor([start.elapsed_time(end)], device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / K
+    # (down_dgrad_gemm includes the quantisation of dy)
+    phases = {n: round(statistics.mean(bev[i][j].elapsed_time(bev[i][j + 1]) for i in range(K)), 4)
+              for j, n in enumerate(BWD_PHASES)}
+    del layer, grads, dy
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "tokens_per_s": wl.T * world / (ms / 1e3), "bwd_phases_ms": phases,
             "device_status": status}
+
+
+def mxfp8_train_roofline(train, wl, fp8_peak_tf, bf16_peak_tf):
+    """The training step against its compute floor: the forward and the two data
+    gradients are MXFP8 products (12 H I FLOP per (token, slot) row), the two weight
+    gradients BF16 (6 H I); floor = each at its own measured peak."""
+    R = wl.T * (wl.k + wl.S)
+    mx_flop, bf_flop = 12.0 * wl.H * wl.I * R, 6.0 * wl.H * wl.I * R
+    floor_ms = (mx_flop / (fp8_peak_tf * 1e12) + bf_flop / (bf16_peak_tf * 1e12)) * 1e3
+    out = dict(train)
+    out.update({"workload": f"{wl.name}: MXFP8 training step (fwd + bwd)",
+                "tflops": (mx_flop + bf_flop) / (train["ms_per_step"] / 1e3) / 1e12,
+                "compute_floor_ms": floor_ms, "frac_of_compute_floor": floor_ms / train["ms_per_step"],
+                "floor_peaks": {"fp8_tflops": fp8_peak_tf, "bf16_tflops": bf16_peak_tf}})
+    return out
 
 
 def e2e_run(layer, wl, x, dy, grads, K, world, dist):
