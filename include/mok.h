@@ -186,8 +186,8 @@ int moe_fwd(const moe_cfg *cfg, const void *x, const moe_params *params, void *y
  * product against the forward's quantised h; the weight gradients are BF16
  * GEMMs (dW_gate_up from the bf16 dGU and the dequantised x, dW_down from dy
  * and the saved w * h).  It needs the wt_* / st_* (and wst_* / sst_*) params
- * and I a multiple of 256 (MOK_ERR_UNSUPPORTED otherwise), and runs as a
- * sequence of kernels whatever the schedule (the one-launch backward is BF16).
+ * and I a multiple of 256 (MOK_ERR_UNSUPPORTED otherwise).  Under the
+ * persistent schedule it is one launch, as the BF16 backward.
  */
 int moe_bwd(const moe_cfg *cfg, const void *x, const void *dy, const moe_params *params,
             const void *ctx, size_t ctx_bytes, const moe_grads *grads, void *scratch,

@@ -6,7 +6,8 @@
 // backward among the measured passes).  One cooperative launch, one CTA per SM,
 // 320 threads; phases, with the grid barriers of fused.cuh:
 //
-//   Q0  zero the launch's tile and readiness counters; the groups' first M tiles
+//   Q0  zero the launch's tile and readiness counters; the groups' first M tiles;
+//       MXFP8: quantise dy
 //   --- grid barrier
 //   Q1  down dgrad GEMM with the SwiGLU-backward epilogue (dGU, slot-gradient
 //       partials); each epilogue warp counts its finished tile on the M tile's
@@ -31,6 +32,7 @@
 // only after the last asynchronous arrival on its barriers (the producer waits
 // for the MMA's release of its last stages; see gemm_phase).
 #pragma once
+#include <type_traits>
 #include "fused.cuh"
 #include "wgrad.cuh"
 
@@ -58,6 +60,9 @@ struct FusedBwdArgs {
     unsigned long long *trace;     // null, or [kFusedBwdTracePoints][gridDim.x] globaltimer stamps
     const int *offsets_all;        // [G + 1] row ranges of all groups (routed, then shared)
     int *mt_base;                  // [G + 1] first M tile of each group (written in Q0)
+    // MXFP8 backward: dy quantised in Q0 (1x32 blocks along H) for the down dgrad
+    const __nv_bfloat16 *dy;
+    uint8_t *dyq, *dys;
 };
 
 // trace points: start, end of Q0, end of the dgrads, of the down weight gradient,
@@ -72,12 +77,21 @@ struct FusedBwdMaps {
     CUtensorMap w4A, w4O, w4O2;              // gate/up wgrad: dGU, dW_gate_up, dWs_gate_up
 };
 
-template <bool N256>
+// MXFP8 backward's data-gradient GEMMs: the down dgrad pulls dy's e4m3 rows by
+// token (as the MXFP8 gate/up forward pulls x) against W_down^T quantised along
+// H, with the SwiGLU-backward epilogue that also quantises dGU; the gate/up dgrad
+// reads those dGU codes (as the MXFP8 down forward reads h's) against
+// W_gate_up^T quantised along 2I and pushes fp32 rows
+using DgradDownMX = GemmCfg<256, false, false, true, false, false, EPI_DSWIGLU, true>;
+using DgradGUMX = GemmCfg<256, false, false, false, false, false, EPI_PUSH, true>;
+
+template <bool N256, bool MX = false>
 struct FusedBwdCfg {
+    static_assert(!MX || N256, "the MXFP8 backward takes N = 256 tiles");
     static constexpr int BN = N256 ? 256 : 128;
-    using DgradDown = GemmCfg<BN, false, true, true, false, false, EPI_DSWIGLU>;
+    using DgradDown = std::conditional_t<MX, DgradDownMX, GemmCfg<BN, false, true, true, false, false, EPI_DSWIGLU>>;
     using WgradDown = GemmCfg<BN, true, true, true, false, true, EPI_WGRAD>;
-    using DgradGU = GemmCfg<256, false, true, false, false, false, EPI_PUSH>;
+    using DgradGU = std::conditional_t<MX, DgradGUMX, GemmCfg<256, false, true, false, false, false, EPI_PUSH>>;
     using WgradGU = GemmCfg<256, true, true, false, true, true, EPI_WGRAD>;
     using ResDown = WgradResCfg<true>;
     using ResGU = WgradResCfg<false>;
@@ -102,11 +116,11 @@ __device__ __forceinline__ void fused_bwd_stamp(const FusedBwdArgs &a, int point
     if (a.trace && threadIdx.x == 0) a.trace[static_cast<size_t>(point) * gridDim.x + blockIdx.x] = globaltimer();
 }
 
-template <bool N256>
+template <bool N256, bool MX>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     moe_bwd_fused_kernel(const __grid_constant__ FusedBwdMaps m, const __grid_constant__ FusedBwdArgs a)
 {
-    using F = FusedBwdCfg<N256>;
+    using F = FusedBwdCfg<N256, MX>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *gbars = reinterpret_cast<uint64_t *>(smem + F::GEMM_RING);          // 4 GEMM barrier blocks
@@ -131,6 +145,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     // ---------------------------------------------------------------- Q0
     for (long long i = gtid; i < a.n_zero; i += gstride) a.zero[i] = 0;
+    if constexpr (MX) {
+        const long long nb = static_cast<long long>(a.T) * (a.H / 32);
+        for (long long b = gtid; b < nb; b += gstride) quantize_block(b, a.dy, a.dyq, a.dys, a.H / 32, 0);
+    }
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         // first M tile of every group in the down dgrad's tiling (readiness counters)
         int acc = 0;

@@ -690,14 +690,6 @@ int forward(const moe_cfg &c, const void *x, const moe_params &p, void *y, const
 // ------------------------------------------------------------------ backward
 // Tensor maps and arguments of every step of the backward, shared by the split
 // schedule and the persistent one.
-// MXFP8 backward's data-gradient GEMMs: the down dgrad pulls dy's e4m3 rows by
-// token (as the MXFP8 gate/up forward pulls x) against W_down^T quantised along
-// H, with the SwiGLU-backward epilogue that also quantises dGU; the gate/up dgrad
-// reads those dGU codes (as the MXFP8 down forward reads h's) against
-// W_gate_up^T quantised along 2I and pushes fp32 rows
-using DgradDownMX = GemmCfg<256, false, false, true, false, false, EPI_DSWIGLU, true>;
-using DgradGUMX = GemmCfg<256, false, false, false, false, false, EPI_PUSH, true>;
-
 struct BwdPlan {
     FusedBwdMaps m;
     GemmArgs g1, g2, g3, g4;
@@ -920,11 +912,11 @@ int backward_split(const moe_cfg &c, const void *x, const moe_params &p, const S
 }
 
 // Persistent schedule: the whole backward as one cooperative launch (fused_bwd.cuh).
-template <bool N256>
+template <bool N256, bool MX>
 int launch_fused_bwd(const moe_cfg &c, const void *x, const moe_params &p, const State &st, const moe_grads &gr,
                      const BwdScratch &bs, const DeviceInfo &dev, const BwdPlan &pl, cudaStream_t stream)
 {
-    using F = FusedBwdCfg<N256>;
+    using F = FusedBwdCfg<N256, MX>;
     if (dev.sms > kMaxFusedCtas) return fail(MOK_ERR_UNSUPPORTED, "more SMs than the grid barrier holds");
     const Shapes s = shapes(c);
     FusedBwdArgs a{};
@@ -968,10 +960,13 @@ int launch_fused_bwd(const moe_cfg &c, const void *x, const moe_params &p, const
     a.routed_scale = c.routed_scale;
     a.dxs = bs.dxs;
     a.dx = static_cast<__nv_bfloat16 *>(gr.dx);
+    a.dy = static_cast<const __nv_bfloat16 *>(pl.dy);
+    a.dyq = bs.dyq;
+    a.dys = bs.dys;
     a.trace = (t_dev_trace_bwd && t_dev_trace_bwd_bytes >= sizeof(unsigned long long) * kFusedBwdTracePoints * dev.sms)
                   ? t_dev_trace_bwd : nullptr;
 
-    cudaError_t e = cudaFuncSetAttribute(moe_bwd_fused_kernel<N256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(moe_bwd_fused_kernel<N256, MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          F::SMEM_BYTES);
     if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(moe_bwd_fused_kernel)", e);
     cudaLaunchConfig_t lc = {};
@@ -985,7 +980,7 @@ int launch_fused_bwd(const moe_cfg &c, const void *x, const moe_params &p, const
     lc.attrs = attr;
     lc.numAttrs = 1;
     MOK_TRY(mark_bwd(0, stream));
-    e = cudaLaunchKernelEx(&lc, moe_bwd_fused_kernel<N256>, pl.m, a);
+    e = cudaLaunchKernelEx(&lc, moe_bwd_fused_kernel<N256, MX>, pl.m, a);
     if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaLaunchKernelEx(moe_bwd_fused_kernel, cooperative)", e);
     ++t_launches;
     for (int i = 1; i <= MOK_BWD_PHASES; ++i) MOK_TRY(mark_bwd(i, stream));
@@ -998,10 +993,11 @@ int backward(const moe_cfg &c, const void *x, const void *dy, const moe_params &
     t_launches = 0;
     BwdPlan pl;
     MOK_TRY(build_bwd_plan(c, x, dy, p, st, gr, bs, dev, pl));
-    if (t_schedule == MOK_SCHEDULE_PERSISTENT && !pl.mx) {     // the one-launch backward is BF16
+    if (t_schedule == MOK_SCHEDULE_PERSISTENT) {
         t_pdl = false;
-        return pl.n256 ? launch_fused_bwd<true>(c, x, p, st, gr, bs, dev, pl, stream)
-                       : launch_fused_bwd<false>(c, x, p, st, gr, bs, dev, pl, stream);
+        if (pl.mx) return launch_fused_bwd<true, true>(c, x, p, st, gr, bs, dev, pl, stream);
+        return pl.n256 ? launch_fused_bwd<true, false>(c, x, p, st, gr, bs, dev, pl, stream)
+                       : launch_fused_bwd<false, false>(c, x, p, st, gr, bs, dev, pl, stream);
     }
     return backward_split(c, x, p, st, gr, bs, dev, pl, stream);
 }

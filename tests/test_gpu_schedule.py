@@ -15,7 +15,8 @@ import numpy as np
 import pytest
 import torch
 
-from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, quantize_mxfp8_weights, synth
+from mixture_experts_layer_persistent_b200 import (MoELayer, abi, cfg_for, quantize_mxfp8_weights,
+                                                   quantize_mxfp8_weights_t, synth)
 from tests._support import assert_close, make_case, to_np
 
 pytestmark = pytest.mark.gpu
@@ -35,6 +36,9 @@ MX_CASES = [
                    mxfp8=True, backward=False, seed=45),
     synth.Workload("sched_mx_i384", T=411, H=768, E=12, k=3, I=384, S=2, Is=384, score_fn=1, n_group=4,
                    topk_group=2, mxfp8=True, backward=False, seed=46),
+    # the MXFP8 training step: the persistent backward is one launch here too
+    synth.Workload("sched_mx_train", T=700, H=512, E=16, k=4, I=256, S=1, Is=256, score_fn=0, mxfp8=True,
+                   seed=47),
 ]
 
 
@@ -47,6 +51,10 @@ def _params(wl, dev):
     for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
                         ("ws_down", "ss_down")):
         out[name], out[sname] = quantize_mxfp8_weights(params[name]) if params.get(name) is not None else (None, None)
+        if wl.backward:
+            t = "wt" + name[1:] if name.startswith("w_") else "wst" + name[2:]
+            ts = "st" + name[1:] if name.startswith("w_") else "sst" + name[2:]
+            out[t], out[ts] = quantize_mxfp8_weights_t(params[name]) if params.get(name) is not None else (None, None)
     return out
 
 
@@ -71,7 +79,7 @@ def _saved(layer, mx):
     names = ([abi.MOK_SAVED_HQ, abi.MOK_SAVED_HS] if mx else [abi.MOK_SAVED_H]) + [abi.MOK_SAVED_ROW_TOKEN,
                                                                                     abi.MOK_SAVED_ROW_W]
     if layer.training:
-        names += [abi.MOK_SAVED_GU, abi.MOK_SAVED_HW]
+        names += [abi.MOK_SAVED_GU, abi.MOK_SAVED_HW] + ([abi.MOK_SAVED_H] if mx else [])
     return {n: layer.saved(n).clone() for n in names}
 
 
@@ -80,7 +88,7 @@ def test_persistent_forward_equals_split_forward(wl):
     dev = torch.device("cuda")
     params = _params(wl, dev)
     x = synth.draw_x(wl, "cpu").to(dev)
-    training = wl.backward and not wl.mxfp8
+    training = wl.backward
     layer = MoELayer(cfg_for(wl), params, training=training, device=dev)
     y_s, r_s, n_s = _forward(layer, x, abi.MOK_SCHEDULE_SPLIT)
     saved_s = _saved(layer, wl.mxfp8)
