@@ -735,7 +735,7 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
     gemm_ms = max(1e-9, phases["gate_up_gemm"] + phases["down_gemm"])
     del layer
     torch.cuda.empty_cache()
-    train = mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist)
+    train = mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist, do_ab)
     del params, x, y
     torch.cuda.empty_cache()
     # the FP8 denominator: a library FP8 GEMM measured on this GPU in this run; the MXFP8
@@ -758,10 +758,11 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
             "training_step": mxfp8_train_roofline(train, wl, peak, pk["bf16"])}
 
 
-def mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist):
+def mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist, do_ab=True):
     """One MXFP8 training step per iteration: the forward with saved state, then the
     backward (MXFP8 data gradients, BF16 weight gradients), timed together with CUDA
-    events; the backward's steps with the split schedule's events."""
+    events under the default schedule; then the backward alone in the interleaved
+    schedule A/B (per-step times from the split schedule's events)."""
     import torch
     from mixture_experts_layer_persistent_b200 import MoELayer, abi, cfg_for, moe_trace_events, synth
     layer = MoELayer(cfg_for(wl), params, training=True, device=dev)
@@ -772,9 +773,6 @@ def mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist):
         layer.backward(x, dy, grads)
     torch.cuda.synchronize()
     mk = lambda: torch.cuda.Event(enable_timing=True)
-    bev = [[mk() for _ in range(abi.MOK_BWD_PHASES + 1)] for _ in range(K)]
-    for e in [e for ev in bev for e in ev]:
-        e.record()
     start, end = mk(), mk()
     torch.cuda.synchronize()
     if world > 1:
@@ -782,23 +780,21 @@ def mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist):
     start.record()
     for i in range(K):
         layer.forward(x, y)
-        moe_trace_events(None, [e.cuda_event for e in bev[i]])
         layer.backward(x, dy, grads)
     end.record()
     torch.cuda.synchronize()
-    moe_trace_events(None, None)
     status = layer.status()
     t = torch.tensor([start.elapsed_time(end)], device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item()) / K
-    # (down_dgrad_gemm includes the quantisation of dy)
-    phases = {n: round(statistics.mean(bev[i][j].elapsed_time(bev[i][j + 1]) for i in range(K)), 4)
-              for j, n in enumerate(BWD_PHASES)}
+    launches = abi.moe_launch_count()
+    # the backward alone, per schedule (down_dgrad_gemm includes the quantisation of dy)
+    ab = backward_ab(layer, x, dy, grads, K) if do_ab else None
     del layer, grads, dy
     torch.cuda.empty_cache()
-    return {"ms_per_step": ms, "tokens_per_s": wl.T * world / (ms / 1e3), "bwd_phases_ms": phases,
-            "device_status": status}
+    return {"ms_per_step": ms, "tokens_per_s": wl.T * world / (ms / 1e3), "bwd_launches": launches,
+            "backward_schedule_ab": ab, "device_status": status}
 
 
 def mxfp8_train_roofline(train, wl, fp8_peak_tf, bf16_peak_tf):
