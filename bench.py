@@ -681,10 +681,11 @@ def bf16_workload_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
 def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
     """Forward tokens/s of the MXFP8 layer (weights quantised once, outside the timed region)."""
     import torch
-    from mixture_experts_layer_persistent_b200 import (MoELayer, abi, cfg_for, moe_trace_events, quantize_mxfp8_weights,
-                                                       quantize_mxfp8_weights_t, synth)
+    from mixture_experts_layer_persistent_b200 import (MoELayer, abi, cfg_for, moe_trace_events,
+                                                       quantize_mxfp8_weights_both, synth)
     p = synth.draw_params(wl, dev)
     params = {k: p[k] for k in ("router_w", "e_bias", "logit_bias")}
+    master = {}                 # the bf16 weights the training step requantises
     for name, sname, tname, tsname in (("w_gate_up", "s_gate_up", "wt_gate_up", "st_gate_up"),
                                        ("w_down", "s_down", "wt_down", "st_down"),
                                        ("ws_gate_up", "ss_gate_up", "wst_gate_up", "sst_gate_up"),
@@ -693,9 +694,8 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
             params[name] = params[sname] = params[tname] = params[tsname] = None
         else:
             # the forward's copy, and the backward's (transposed, quantised along the other axis)
-            params[name], params[sname] = quantize_mxfp8_weights(p[name])
-            params[tname], params[tsname] = quantize_mxfp8_weights_t(p[name])
-            p[name] = None
+            params[name], params[sname], params[tname], params[tsname] = quantize_mxfp8_weights_both(p[name])
+            master[name] = (p[name], (params[name], params[sname], params[tname], params[tsname]))
     del p
     torch.cuda.empty_cache()
     x = synth.draw_x(wl, dev)
@@ -735,8 +735,8 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
     gemm_ms = max(1e-9, phases["gate_up_gemm"] + phases["down_gemm"])
     del layer
     torch.cuda.empty_cache()
-    train = mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist, do_ab)
-    del params, x, y
+    train = mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist, do_ab, master)
+    del params, x, y, master
     torch.cuda.empty_cache()
     # the FP8 denominator: a library FP8 GEMM measured on this GPU in this run; the MXFP8
     # forward loop is short (K forwards of a few ms), so the burst figure is its peak
@@ -758,7 +758,7 @@ def mxfp8_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
             "training_step": mxfp8_train_roofline(train, wl, peak, pk["bf16"])}
 
 
-def mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist, do_ab=True):
+def mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist, do_ab=True, master=None):
     """One MXFP8 training step per iteration: the forward with saved state, then the
     backward (MXFP8 data gradients, BF16 weight gradients), timed together with CUDA
     events under the default schedule; then the backward alone in the interleaved
@@ -789,12 +789,36 @@ def mxfp8_train(wl, params, x, y, dev, K, warmup, world, dist, do_ab=True):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     ms = float(t.item()) / K
     launches = abi.moe_launch_count()
+    # the requantisation after an optimizer step: both MXFP8 copies of every expert
+    # weight tensor from its bf16 master, in place (one read of each master)
+    from mixture_experts_layer_persistent_b200 import quantize_mxfp8_weights_both
+    requant_ms = None
+    if master:
+        def requant():
+            for w, out in master.values():
+                quantize_mxfp8_weights_both(w, out)
+        requant()
+        torch.cuda.synchronize()
+        s0, s1 = mk(), mk()
+        s0.record()
+        for _ in range(K):
+            requant()
+        s1.record()
+        torch.cuda.synchronize()
+        requant_ms = s0.elapsed_time(s1) / K
     # the backward alone, per schedule (down_dgrad_gemm includes the quantisation of dy)
     ab = backward_ab(layer, x, dy, grads, K) if do_ab else None
     del layer, grads, dy
     torch.cuda.empty_cache()
-    return {"ms_per_step": ms, "tokens_per_s": wl.T * world / (ms / 1e3), "bwd_launches": launches,
-            "backward_schedule_ab": ab, "device_status": status}
+    wbytes = sum(w.numel() * 2 for w, _ in master.values()) if master else 0
+    out = {"ms_per_step": ms, "tokens_per_s": wl.T * world / (ms / 1e3), "bwd_launches": launches,
+           "backward_schedule_ab": ab, "device_status": status}
+    if requant_ms is not None:
+        # bytes: the bf16 masters read once, both e4m3 copies and their scales written
+        nb = wbytes + wbytes + wbytes // 32
+        out.update({"requant_ms": requant_ms, "requant_gbs": nb / (requant_ms / 1e3) / 1e9,
+                    "tokens_per_s_with_requant": wl.T * world / ((ms + requant_ms) / 1e3)})
+    return out
 
 
 def mxfp8_train_roofline(train, wl, fp8_peak_tf, bf16_peak_tf):

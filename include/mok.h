@@ -251,6 +251,17 @@ int moe_quantize_mxfp8_weights_t(const void *src, int64_t batch, int64_t R, int6
                                  void *scales, void *stream);
 
 /*
+ * Both MXFP8 copies of a weight tensor from one read of it, for the
+ * requantisation after each optimizer step of MXFP8 training: src [batch, R, C]
+ * bf16 (device) -> q [batch, R, C] and scales exactly as
+ * moe_quantize_mxfp8_weights(src, batch*R, C, ...) writes them, and qt
+ * [batch, C, R] and scales_t exactly as moe_quantize_mxfp8_weights_t writes
+ * them.  R must be a multiple of 128 and C of 256 (MOK_ERR_INVALID otherwise).
+ */
+int moe_quantize_mxfp8_weights_both(const void *src, int64_t batch, int64_t R, int64_t C, void *q,
+                                    void *scales, void *qt, void *scales_t, void *stream);
+
+/*
  * Phase tracing.  When events are set, every later moe_fwd (moe_bwd) records
  * fwd_events[i] (bwd_events[i]) on its stream just before launching phase i
  * and the last event after its final launch, so that elapsed times between

@@ -92,6 +92,8 @@ def lib():
         L.moe_quantize_mxfp8_weights.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
         L.moe_quantize_mxfp8_weights_t.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _vp, _vp,
                                                    _vp]
+        L.moe_quantize_mxfp8_weights_both.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _vp, _vp,
+                                                      _vp, _vp, _vp]
         L.moe_status.argtypes = [_vp, P(_i32)]
         L.moe_trace_events.argtypes = [P(_vp), ctypes.c_int, P(_vp), ctypes.c_int]
         L.moe_fwd_static.argtypes = [P(moe_cfg), _vp, P(moe_params), _vp, _vp]
@@ -107,7 +109,7 @@ def lib():
         L.moe_last_error.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
                      "moe_fwd_host", "moe_bwd_host", "moe_quantize_mxfp8", "moe_quantize_mxfp8_weights",
-                     "moe_quantize_mxfp8_weights_t", "moe_status",
+                     "moe_quantize_mxfp8_weights_t", "moe_quantize_mxfp8_weights_both", "moe_status",
                      "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal", "moe_saved_tensor",
                      "moe_set_schedule", "moe_get_schedule", "moe_trace_device"):
             getattr(L, name).restype = ctypes.c_int
@@ -194,6 +196,11 @@ def moe_quantize_mxfp8(src, rows, K, q, scales, stream):
 
 def moe_quantize_mxfp8_weights(src, rows, K, q, scales, stream):
     _check("moe_quantize_mxfp8_weights", lib().moe_quantize_mxfp8_weights(src, rows, K, q, scales, stream))
+
+
+def moe_quantize_mxfp8_weights_both(src, batch, R, C, q, scales, qt, scales_t, stream):
+    _check("moe_quantize_mxfp8_weights_both",
+           lib().moe_quantize_mxfp8_weights_both(src, batch, R, C, q, scales, qt, scales_t, stream))
 
 
 def moe_quantize_mxfp8_weights_t(src, batch, R, C, q, scales, stream):

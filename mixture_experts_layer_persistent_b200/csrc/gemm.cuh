@@ -936,16 +936,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         amax = fmaxf(amax, fabsf(g[i]));
                     }
                     const int e = mx_exponent(amax);
-                    const float sf = exp2_neg(e);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        uint32_t word = 0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            word |= static_cast<uint32_t>(__nv_cvt_float_to_fp8(g[4 * i + j] * sf, __NV_SATFINITE, __NV_E4M3))
-                                    << (8 * j);
-                        q[8 * blk + i] = word;
-                    }
+                    mx_codes32(g, e, q + 8 * blk);
                     sc |= static_cast<uint32_t>(e + 127) << (8 * blk);
                     if (args.out_hb && valid) {
                         // training: the dequantised h (exact in bf16) and w times it, rounded

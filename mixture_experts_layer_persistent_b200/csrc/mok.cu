@@ -1178,6 +1178,24 @@ int moe_quantize_mxfp8_weights_t(const void *src, int64_t batch, int64_t R, int6
     return MOK_OK;
 }
 
+int moe_quantize_mxfp8_weights_both(const void *src, int64_t batch, int64_t R, int64_t C, void *q, void *scales,
+                                    void *qt, void *scales_t, void *stream)
+{
+    if (!src || !q || !scales || !qt || !scales_t || batch < 0 || R <= 0 || C <= 0) return MOK_ERR_INVALID;
+    if (R % 128 || C % 256)
+        return fail(MOK_ERR_INVALID, "moe_quantize_mxfp8_weights_both: R must be a multiple of 128, C of 256");
+    if (!aligned16(src) || !aligned16(q) || !aligned16(qt)) return MOK_ERR_INVALID;
+    if (!device_info()) return MOK_ERR_DEVICE;
+    const long long n = batch * (R / 32) * (C / kQuantBothCols);
+    if (n == 0) return MOK_OK;
+    quantize_mxfp8_both_kernel<<<static_cast<unsigned>(n), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16 *>(src), batch, R, C, static_cast<uint8_t *>(q), static_cast<uint8_t *>(scales),
+        static_cast<uint8_t *>(qt), static_cast<uint8_t *>(scales_t));
+    if (const cudaError_t e_ = cudaGetLastError(); e_ != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "quantize_mxfp8_both_kernel launch", e_);
+    return MOK_OK;
+}
+
 int moe_trace_events(void *const *fwd_events, int n_fwd, void *const *bwd_events, int n_bwd)
 {
     if (n_fwd < 0 || n_bwd < 0) return MOK_ERR_INVALID;

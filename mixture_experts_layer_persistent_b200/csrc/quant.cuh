@@ -42,19 +42,18 @@ __device__ __forceinline__ long long packed_scale_offset(long long row, long lon
     return ((j >> 2) * row_tiles + (row >> 7)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (j & 3);
 }
 
-// e4m3 codes (4 per word, low byte first) of 32 values, scaled by 2^-e
-__device__ __forceinline__ void mx_codes32(const float (&v)[32], int e, uint32_t (&w)[8])
+// e4m3 codes (4 per word, low byte first) of 32 values, scaled by 2^-e; two
+// values per conversion (the pair's first value in the low byte)
+__device__ __forceinline__ void mx_codes32(const float *v, int e, uint32_t *w)
 {
     const float s = exp2_neg(e);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const __nv_fp8_storage_t c = __nv_cvt_float_to_fp8(v[4 * i + j] * s, __NV_SATFINITE, __NV_E4M3);
-            word |= static_cast<uint32_t>(c) << (8 * j);
-        }
-        w[i] = word;
+        const __nv_fp8x2_storage_t lo =
+            __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i] * s, v[4 * i + 1] * s), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t hi =
+            __nv_cvt_float2_to_fp8x2(make_float2(v[4 * i + 2] * s, v[4 * i + 3] * s), __NV_SATFINITE, __NV_E4M3);
+        w[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
     }
 }
 
@@ -142,6 +141,75 @@ __global__ void __launch_bounds__(256) quantize_mxfp8_t_kernel(const __nv_bfloat
     dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
     dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     scales[packed_scale_offset(row, j, batch * C / 128)] = static_cast<uint8_t>(e + 127);
+}
+
+
+// Both MXFP8 copies of a weight tensor src [batch, R, C] from one read of it: the
+// forward's (q [batch, R, C] along C, scales packed for [batch*R, C]) and the
+// backward's (qt [batch, C, R] along R, scales packed for [batch*C, R]).  CTA =
+// a 32 x 256 tile (32 rows of R, 256 columns of C) staged in shared memory;
+// thread t then quantises row block (t % 32, t / 32) of the tile for q and column
+// t for qt (a warp reads 32 rows, or 32 columns, so shared memory sees no bank
+// conflict), with the arithmetic of quantize_block and quantize_mxfp8_t_kernel.
+constexpr int kQuantBothCols = 256;
+__global__ void __launch_bounds__(256) quantize_mxfp8_both_kernel(const __nv_bfloat16 *__restrict__ src,
+                                                                  long long batch, long long R, long long C,
+                                                                  uint8_t *__restrict__ q, uint8_t *__restrict__ s,
+                                                                  uint8_t *__restrict__ qt,
+                                                                  uint8_t *__restrict__ st)
+{
+    // bf16 tile; a row is 264 elements (132 words): the 32 rows of a warp's 16-byte
+    // row reads fall on 8 distinct groups of 4 banks (4 wavefronts, the minimum)
+    __shared__ __align__(16) __nv_bfloat16 tile[32][kQuantBothCols + 8];
+    const long long ct = C / kQuantBothCols, rt = R / 32;
+    const long long b = blockIdx.x / (ct * rt);
+    const long long r0 = (blockIdx.x / ct) % rt * 32, c0 = blockIdx.x % ct * kQuantBothCols;
+    const int t = threadIdx.x;
+    // stage: 32 rows x 256 columns, 16-byte loads (a warp reads one 512-byte row piece)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int idx = i * 256 + t, row = idx >> 5, c8 = (idx & 31) * 8;
+        *reinterpret_cast<uint4 *>(&tile[row][c8]) =
+            *reinterpret_cast<const uint4 *>(src + ((b * R + r0 + row) * C + c0 + c8));
+    }
+    __syncthreads();
+    float v[32];
+    uint32_t w[8];
+    {   // the forward's copy: 32 consecutive columns of one row
+        const int row = t & 31, blk = t >> 5;
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(&tile[row][blk * 32 + 8 * i]);
+            v[8 * i + 0] = bf16_lo(u.x); v[8 * i + 1] = bf16_hi(u.x); v[8 * i + 2] = bf16_lo(u.y);
+            v[8 * i + 3] = bf16_hi(u.y); v[8 * i + 4] = bf16_lo(u.z); v[8 * i + 5] = bf16_hi(u.z);
+            v[8 * i + 6] = bf16_lo(u.w); v[8 * i + 7] = bf16_hi(u.w);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        const int e = mx_exponent(amax);
+        mx_codes32(v, e, w);
+        const long long grow = b * R + r0 + row, gcol = c0 + blk * 32;
+        uint4 *dst = reinterpret_cast<uint4 *>(q + grow * C + gcol);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        s[packed_scale_offset(grow, gcol / 32, batch * R / 128)] = static_cast<uint8_t>(e + 127);
+    }
+    {   // the backward's copy: column t, 32 consecutive rows
+        float amax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            v[i] = __bfloat162float(tile[i][t]);
+            amax = fmaxf(amax, fabsf(v[i]));
+        }
+        const int e = mx_exponent(amax);
+        mx_codes32(v, e, w);
+        const long long grow = b * C + c0 + t;
+        uint4 *dst = reinterpret_cast<uint4 *>(qt + grow * R + r0);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        st[packed_scale_offset(grow, r0 / 32, batch * C / 128)] = static_cast<uint8_t>(e + 127);
+    }
 }
 
 }  // namespace mok

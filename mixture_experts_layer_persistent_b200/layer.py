@@ -159,3 +159,19 @@ def quantize_mxfp8_weights_t(src: torch.Tensor):
     abi.moe_quantize_mxfp8_weights_t(src.data_ptr(), batch, R, C, q.data_ptr(), s.data_ptr(),
                                      torch.cuda.current_stream(src.device).cuda_stream)
     return q, s
+
+
+def quantize_mxfp8_weights_both(src: torch.Tensor, out=None):
+    """Expert weights bf16 [batch, R, C] -> both MXFP8 copies from one read: (q, s) as
+    quantize_mxfp8_weights and (qt, st) as quantize_mxfp8_weights_t, via libmok.
+    out: optional (q, s, qt, st) tensors to write into (requantisation in place)."""
+    batch, R, C = src.shape
+    if out is None:
+        out = (torch.empty((batch, R, C), dtype=torch.uint8, device=src.device),
+               torch.empty(batch * R * (C // 32), dtype=torch.uint8, device=src.device),
+               torch.empty((batch, C, R), dtype=torch.uint8, device=src.device),
+               torch.empty(batch * C * (R // 32), dtype=torch.uint8, device=src.device))
+    q, s, qt, st = out
+    abi.moe_quantize_mxfp8_weights_both(src.data_ptr(), batch, R, C, q.data_ptr(), s.data_ptr(), qt.data_ptr(),
+                                        st.data_ptr(), torch.cuda.current_stream(src.device).cuda_stream)
+    return out

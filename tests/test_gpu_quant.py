@@ -77,3 +77,24 @@ def test_transposed_weight_quantize_matches_oracle(shape):
     at = packed_scale_offsets(np.arange(batch * C), R // 32, batch * C)
     assert np.array_equal(np.sort(at.ravel()), np.arange(s.numel()))
     assert np.array_equal(s.cpu().numpy()[at], os_)
+
+
+@pytest.mark.parametrize("shape", [(2, 256, 512), (3, 384, 768)])
+def test_both_copies_in_one_pass(shape):
+    """moe_quantize_mxfp8_weights_both: byte for byte the outputs of
+    moe_quantize_mxfp8_weights and moe_quantize_mxfp8_weights_t, and in place."""
+    from mixture_experts_layer_persistent_b200 import (quantize_mxfp8_weights, quantize_mxfp8_weights_both,
+                                                       quantize_mxfp8_weights_t)
+    g = torch.Generator().manual_seed(shape[2])
+    x = torch.randn(shape, generator=g) * torch.exp2(torch.randint(-20, 20, (shape[0], shape[1], 1), generator=g).float())
+    xb = x.to(torch.bfloat16).cuda()
+    q, s, qt, st = quantize_mxfp8_weights_both(xb)
+    q1, s1 = quantize_mxfp8_weights(xb)
+    qt1, st1 = quantize_mxfp8_weights_t(xb)
+    out = tuple(torch.full_like(t, 0x5A) for t in (q, s, qt, st))
+    quantize_mxfp8_weights_both(xb, out)
+    torch.cuda.synchronize()
+    for a, b in ((q, q1), (s, s1), (qt, qt1), (st, st1)):
+        assert torch.equal(a.view(-1), b.view(-1))
+    for a, b in zip(out, (q, s, qt, st)):
+        assert torch.equal(a, b)
