@@ -55,3 +55,29 @@ def test_calls_fail_loudly_without_a_device():
     p = abi.moe_params()
     with pytest.raises(abi.MokError):
         abi.moe_fwd(c, 16, p, 16, None, None, 0, 0, 16, 1 << 30, None)
+
+
+def test_mxfp8_backward_argument_checks():
+    """moe_bwd with MOK_DTYPE_MXFP8 refuses, before touching any device, a call
+    without the transposed weight copies (MOK_ERR_INVALID) and an I that is not a
+    multiple of 256 (MOK_ERR_UNSUPPORTED).  The pointers are never dereferenced."""
+    fake = 1 << 20                                    # aligned, never read
+    g = abi.moe_grads(fake, fake, fake, fake, None, None)
+
+    def params(with_t):
+        p = abi.moe_params(router_w=fake, w_gate_up=fake, w_down=fake, s_gate_up=fake, s_down=fake)
+        if with_t:
+            p.wt_gate_up = p.wt_down = p.st_gate_up = p.st_down = fake
+        return p
+
+    c = make_cfg(64, 256, 8, 256, 2, dtype=abi.MOK_DTYPE_MXFP8)
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_bwd(c, fake, fake, params(False), fake, 1 << 30, g, fake, 1 << 30, None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
+    c = make_cfg(64, 256, 8, 384, 2, dtype=abi.MOK_DTYPE_MXFP8)
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_bwd(c, fake, fake, params(True), fake, 1 << 30, g, fake, 1 << 30, None)
+    assert ei.value.code == abi.MOK_ERR_UNSUPPORTED
+    with pytest.raises(abi.MokError) as ei:      # the one-pass quantiser's shape rule
+        abi.moe_quantize_mxfp8_weights_both(fake, 2, 256, 384, fake, fake, fake, fake, None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
