@@ -228,7 +228,11 @@ __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const i
     return t;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+// silu(g) = g sigmoid(g) with the hardware exponential and reciprocal (CUDA's
+// __expf and __fdividef intrinsics: a few ulp of fp32, far inside the layer's
+// tolerances); for g < -88, __expf(-g) is inf and the quotient 0
+__device__ __forceinline__ float sigmoid_f(float g) { return __fdividef(1.0f, 1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return g * sigmoid_f(g); }
 
 template <int N>
 __device__ __forceinline__ void pack_bf16(const float *v, uint32_t *p)
@@ -1108,7 +1112,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                             const float ui = (i & 1) ? bf16_hi(uw) : bf16_lo(uw);
                             gsum = fmaf(v[i], (i & 1) ? bf16_hi(hw) : bf16_lo(hw), gsum);
                             const float dh = w * v[i];
-                            const float sg = 1.0f / (1.0f + expf(-gi));
+                            const float sg = sigmoid_f(gi);
                             dg[i] = dh * ui * sg * (1.0f + gi * (1.0f - sg));
                             du[i] = dh * gi * sg;
                         }
