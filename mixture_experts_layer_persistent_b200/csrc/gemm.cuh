@@ -129,6 +129,9 @@ struct GemmCfg {
     // streamers, the MXFP8 gate/up GEMM among them (one block per warp and
     // tile), keep four.
     static constexpr bool MX_SWIGLU = MX && EPI == EPI_SWIGLU;
+    // single-accumulator (MXFP8) epilogues hand the accumulator back to the MMA warp
+    // as soon as its last columns are in registers, before their conversion and stores
+    static constexpr bool EARLY_RELEASE = MX;
     static constexpr bool HEAVY_EPI = BN == 256 && ((MX && !MX_SWIGLU) || RAGGED_K);
     static constexpr int STAGES = HEAVY_EPI ? 3 : (BN == 256 ? 4 : (RAGGED_K ? 6 : 5));
     static constexpr int EPI_BUFS = (HEAVY_EPI || (!RAGGED_K && BN != 256)) ? 2 : 1;
@@ -1019,6 +1022,10 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         uint32_t p[32];
                         tmem_ld32(taddr + c, v);
                         tmem_ld_wait();
+                        if (c == C::BN - 32) {
+                            tc_fence_before();
+                            mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
+                        }
 #pragma unroll
                         for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
                         if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
@@ -1034,6 +1041,10 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
                         tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
                         tmem_ld_wait();
+                        if (c == C::BN - 64) {
+                            tc_fence_before();
+                            mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
+                        }
                         pack_bf16<64>(v, p);
                         if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
                         else if (valid) store_row_direct(dst + c, p);
@@ -1104,6 +1115,12 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         float v[32], dg[32], du[32];
                         tmem_ld32(taddr + c + 32 * half, v);
                         tmem_ld_wait();
+                        if constexpr (C::EARLY_RELEASE) {
+                            if (c == C::BN - 64 && half == 1) {
+                                tc_fence_before();
+                                mbar_arrive(&acce[acc]);     // every column of the accumulator is in registers
+                            }
+                        }
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
                             const uint32_t gw = gp[16 * half + (i >> 1)], uw = up[16 * half + (i >> 1)];
@@ -1152,7 +1169,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                     else if (valid) store_row_direct(args.out_f32 + ((size_t)t.nt * args.rows_total + r) * 256 + c, p);
                 }
             }
-            if constexpr (!C::MX_SWIGLU) {
+            if constexpr (!C::EARLY_RELEASE) {
                 tc_fence_before();
                 mbar_arrive(&acce[acc]);
             }
