@@ -212,6 +212,24 @@ int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host,
                  const moe_grads *grads, void *scratch, size_t scratch_bytes, void *stream);
 
 /*
+ * One training step through host buffers: the forward (state saved in ctx) and
+ * the backward.  x_host, dy_host: [T, H] bf16 (host) in; y_host, dx_host:
+ * [T, H] bf16 (host) out; the weight and router gradients go to `grads` on the
+ * device (grads->dx is ignored).  The transfers overlap the passes: dy is
+ * uploaded on a second stream of the library's while the forward runs, and y
+ * is downloaded on it while the backward runs, so with pinned host buffers
+ * only the upload of x and the download of dx add to the step.  The results
+ * equal those of moe_fwd_host + moe_bwd_host byte for byte.  scratch: device
+ * memory of at least moe_host_scratch_size(cfg, 2, ...) bytes (backward = 2
+ * asks for this call's size).  The call waits for both streams before it
+ * returns.  The second stream (one per host thread and device) is created on
+ * first use and kept.
+ */
+int moe_step_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, const moe_params *params,
+                  void *y_host, void *dx_host, void *ctx, size_t ctx_bytes, const moe_grads *grads,
+                  void *scratch, size_t scratch_bytes, void *stream);
+
+/*
  * MXFP8 quantisation along the last axis: src [rows, K] bf16 (device) ->
  * q [rows, K] e4m3 codes and scales [rows, K/32] ue8m0 (device).  Per block of
  * 32 consecutive elements the exponent e is the smallest integer with

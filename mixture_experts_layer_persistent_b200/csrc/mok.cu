@@ -1085,7 +1085,7 @@ int moe_host_scratch_size(const moe_cfg *cfg, int backward, size_t *bytes)
     MOK_TRY(check_cfg(cfg));
     const size_t io = align_up(static_cast<size_t>(cfg->T) * cfg->H * 2, 256);
     size_t inner = backward ? carve_bwd(*cfg, nullptr).bytes : carve_state(*cfg, nullptr, false).bytes;
-    if (bytes) *bytes = (backward ? 3 : 2) * io + inner;
+    if (bytes) *bytes = (backward == 2 ? 4 : backward ? 3 : 2) * io + inner;
     return MOK_OK;
 }
 
@@ -1133,6 +1133,96 @@ int moe_bwd_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, co
     if (const cudaError_t e_ = cudaStreamSynchronize(st); e_ != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaStreamSynchronize", e_);
     return MOK_OK;
+}
+
+namespace {
+// The second stream and the events of moe_step_host, per host thread and device.
+struct StepStreams {
+    int device = -1;
+    cudaStream_t side = nullptr;
+    cudaEvent_t start = nullptr, dy_in = nullptr, y_ready = nullptr, y_out = nullptr;
+};
+thread_local StepStreams t_step;
+
+int step_streams(StepStreams *&ss)
+{
+    int dev = 0;
+    if (const cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return fail(MOK_ERR_DEVICE, "cudaGetDevice", e);
+    ss = &t_step;
+    if (ss->device == dev) return MOK_OK;
+    if (ss->side) {                 // another device: release the old handles first
+        cudaStreamDestroy(ss->side);
+        cudaEventDestroy(ss->start);
+        cudaEventDestroy(ss->dy_in);
+        cudaEventDestroy(ss->y_ready);
+        cudaEventDestroy(ss->y_out);
+        *ss = StepStreams{};
+    }
+    if (const cudaError_t e = cudaStreamCreateWithFlags(&ss->side, cudaStreamNonBlocking); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaStreamCreateWithFlags", e);
+    cudaEvent_t *evs[] = {&ss->start, &ss->dy_in, &ss->y_ready, &ss->y_out};
+    for (cudaEvent_t *ev : evs)
+        if (const cudaError_t e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming); e != cudaSuccess)
+            return fail(MOK_ERR_LAUNCH, "cudaEventCreateWithFlags", e);
+    ss->device = dev;
+    return MOK_OK;
+}
+}  // namespace
+
+int moe_step_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, const moe_params *params,
+                  void *y_host, void *dx_host, void *ctx, size_t ctx_bytes, const moe_grads *grads, void *scratch,
+                  size_t scratch_bytes, void *stream)
+{
+    MOK_TRY(check_cfg(cfg));
+    if (!x_host || !dy_host || !y_host || !dx_host || !scratch || !grads) return MOK_ERR_INVALID;
+    size_t need = 0;
+    moe_host_scratch_size(cfg, 2, &need);
+    if (scratch_bytes < need) return MOK_ERR_WORKSPACE;
+    if (!device_info()) return MOK_ERR_DEVICE;
+    StepStreams *ss = nullptr;
+    MOK_TRY(step_streams(ss));
+    const size_t io = align_up(static_cast<size_t>(cfg->T) * cfg->H * 2, 256);
+    const size_t nb = static_cast<size_t>(cfg->T) * cfg->H * 2;
+    char *s = static_cast<char *>(scratch);
+    char *x = s, *y = s + io, *dy = s + 2 * io, *dx = s + 3 * io, *inner = s + 4 * io;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    int rc = MOK_OK;
+#define STEP_CUDA(call, what)                                      \
+    if ((e = (call)) != cudaSuccess) {                             \
+        rc = fail(MOK_ERR_LAUNCH, what, e);                        \
+        goto done;                                                 \
+    }
+    // the side stream starts after everything already enqueued on `stream` (which may
+    // still read this scratch buffer)
+    STEP_CUDA(cudaEventRecord(ss->start, st), "cudaEventRecord");
+    STEP_CUDA(cudaStreamWaitEvent(ss->side, ss->start, 0), "cudaStreamWaitEvent");
+    STEP_CUDA(cudaMemcpyAsync(dy, dy_host, nb, cudaMemcpyHostToDevice, ss->side), "cudaMemcpyAsync(dy)");
+    STEP_CUDA(cudaEventRecord(ss->dy_in, ss->side), "cudaEventRecord");
+    STEP_CUDA(cudaMemcpyAsync(x, x_host, nb, cudaMemcpyHostToDevice, st), "cudaMemcpyAsync(x)");
+    if ((rc = moe_fwd(cfg, x, params, y, nullptr, ctx, ctx_bytes, 1, nullptr, 0, stream)) != MOK_OK) goto done;
+    // y leaves on the side stream while the backward runs
+    STEP_CUDA(cudaEventRecord(ss->y_ready, st), "cudaEventRecord");
+    STEP_CUDA(cudaStreamWaitEvent(ss->side, ss->y_ready, 0), "cudaStreamWaitEvent");
+    STEP_CUDA(cudaMemcpyAsync(y_host, y, nb, cudaMemcpyDeviceToHost, ss->side), "cudaMemcpyAsync(y)");
+    STEP_CUDA(cudaEventRecord(ss->y_out, ss->side), "cudaEventRecord");
+    STEP_CUDA(cudaStreamWaitEvent(st, ss->dy_in, 0), "cudaStreamWaitEvent");
+    {
+        moe_grads g = *grads;
+        g.dx = dx;
+        if ((rc = moe_bwd(cfg, x, dy, params, ctx, ctx_bytes, &g, inner, scratch_bytes - 4 * io, stream)) != MOK_OK)
+            goto done;
+    }
+    STEP_CUDA(cudaMemcpyAsync(dx_host, dx, nb, cudaMemcpyDeviceToHost, st), "cudaMemcpyAsync(dx)");
+    STEP_CUDA(cudaStreamWaitEvent(st, ss->y_out, 0), "cudaStreamWaitEvent");
+#undef STEP_CUDA
+done:
+    // both streams drain before the call returns, on success and on failure
+    if (const cudaError_t e2 = cudaStreamSynchronize(ss->side); e2 != cudaSuccess && rc == MOK_OK)
+        rc = fail(MOK_ERR_LAUNCH, "cudaStreamSynchronize(side)", e2);
+    if (const cudaError_t e2 = cudaStreamSynchronize(st); e2 != cudaSuccess && rc == MOK_OK)
+        rc = fail(MOK_ERR_LAUNCH, "cudaStreamSynchronize", e2);
+    return rc;
 }
 
 static int quantize(const void *src, int64_t rows, int64_t K, void *q, void *scales, bool packed, void *stream)

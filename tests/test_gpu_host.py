@@ -49,3 +49,36 @@ def test_host_entry_points_match_device_api(reuse_x):
     for k in ("dw_gate_up", "dw_down", "dws_gate_up", "dws_down"):
         assert torch.equal(grads[k].view(torch.int16), g_ref[k].view(torch.int16)), k
     assert torch.equal(grads["drouter_w"].view(torch.int32), g_ref["drouter_w"].view(torch.int32))
+
+
+def test_step_host_matches_device_api():
+    """moe_step_host (forward + backward through host buffers, transfers overlapping
+    the passes on a second stream) against the device calls, byte for byte, twice in
+    a row (the second step reuses the scratch buffer the first one left)."""
+    case = make_case(WL, device="cuda", gen_device="cpu")
+    dev = torch.device("cuda")
+    layer = MoELayer(cfg_for(WL), case["params"], training=True, device=dev)
+    y_ref = layer.forward(case["x"]).clone()
+    g_ref = {k: (v.clone() if v is not None else None) for k, v in layer.backward(case["x"], case["dy"]).items()}
+    torch.cuda.synchronize()
+    c = layer.cfg
+    hx = case["x"].cpu().pin_memory()
+    hdy = case["dy"].cpu().pin_memory()
+    n = abi.moe_host_scratch_size(c, 2)
+    scratch = torch.empty(n, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        hy = torch.empty_like(hx).pin_memory()
+        hdx = torch.empty_like(hx).pin_memory()
+        grads = layer.new_grads()
+        g = abi.moe_grads(None, grads["dw_gate_up"].data_ptr(), grads["dw_down"].data_ptr(),
+                          grads["drouter_w"].data_ptr(),
+                          grads["dws_gate_up"].data_ptr() if grads["dws_gate_up"] is not None else None,
+                          grads["dws_down"].data_ptr() if grads["dws_down"] is not None else None)
+        abi.moe_step_host(c, hx.data_ptr(), hdy.data_ptr(), layer.cparams, hy.data_ptr(), hdx.data_ptr(),
+                          layer.ctx.data_ptr(), layer.ctx_bytes, g, scratch.data_ptr(), n, layer.stream())
+        assert layer.status() == 0
+        assert torch.equal(hy.view(torch.int16), y_ref.cpu().view(torch.int16))
+        assert torch.equal(hdx.view(torch.int16), g_ref["dx"].cpu().view(torch.int16))
+        for k in ("dw_gate_up", "dw_down", "dws_gate_up", "dws_down"):
+            assert torch.equal(grads[k].view(torch.int16), g_ref[k].view(torch.int16)), k
+        assert torch.equal(grads["drouter_w"].view(torch.int32), g_ref["drouter_w"].view(torch.int32))
