@@ -29,7 +29,8 @@
 //       dependency idea of "Megakernels are dead and back…", the case against
 //       megakernels: tile-level triggers instead of a kernel boundary).
 //   --- grid barrier
-//   P5  fixed-order combine of the slot rows
+//   P5  fixed-order combine of the slot rows, streamed through shared memory
+//       (combine.cuh: combine_stream)
 //
 // The phases run the same device code as the separate kernels of the split
 // schedule, so both schedules give byte-identical results.

@@ -1,4 +1,5 @@
-// fused_bwd.cuh -- the whole BF16 backward pass as ONE persistent launch.
+// fused_bwd.cuh -- the whole backward pass as ONE persistent launch (BF16, or
+// with the two data-gradient GEMMs on MXFP8 operands).
 //
 // The counterpart of the persistent forward (fused.cuh) for the backward of
 // the layer ("Cursor åpner megakernelen som ga 41 prosent flere tokens i
@@ -16,14 +17,16 @@
 //       every down-dgrad tile of those rows is in memory -- no barrier
 //   Q3  down weight gradient: streaming kernel for groups of more than 256 rows,
 //       then the resident kernel for the rest (it depends on nothing of the pass)
-//   Q5  gate/up weight gradient (streaming, then resident): each work unit
-//       waits until every dGU tile of its group is in memory -- no barrier
+//       gate/up weight gradient (streaming, then resident): each CTA checks,
+//       once per group, that every dGU tile of the group is in memory -- no
+//       barrier
 //   --- grid barrier
 //   Q4  slot gradients and routing-logit gradients (one thread per token)
 //   --- grid barrier
-//   Q6  router-gradient partial sums and the dx sum
+//   Q5  router-gradient partial sums and the dx sum, streamed through shared
+//       memory (combine.cuh: drouter_stream, dx_stream)
 //   --- grid barrier
-//   Q7  router-gradient reduction
+//   Q6  router-gradient reduction
 //
 // Every phase runs the device code of the split schedule's kernels, so the two
 // schedules give byte-identical gradients.  The resident weight-gradient phases
@@ -162,7 +165,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     bool alive = grid_sync(a.gs, epoch, nb++, true, a.status, s_flag);
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.gs.epoch = (epoch + 1) & kEpochMask;
 
-    // ---------------------------------------------------------------- Q1, Q2, Q3, Q5
+    // ---------------------------------------------------------------- Q1, Q2, Q3 (both dgrads, both weight gradients)
     // No barrier between the four GEMMs: a CTA moves on when a GEMM's tile counter
     // is exhausted, so the next GEMM starts on SMs that the previous one's tail
     // leaves idle.  The gate/up weight gradient waits per group for that group's dGU.
