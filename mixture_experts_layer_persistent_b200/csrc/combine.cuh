@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *__restrict
 
 
 // ---- the same sums in the persistent kernels --------------------------------
-// A persistent CTA has 10 warps per SM, far too few to hide HBM latency with the
+// A persistent CTA has 8 warps per SM, far too few to hide HBM latency with the
 // one-thread-per-element code above (the split kernels rely on 64 resident warps
 // per SM).  Here every thread streams its own 16-byte pieces through a private
 // ring of shared-memory slots with cp.async, NS units deep, so the loads of the

@@ -6,8 +6,8 @@
 // veröffentlicht MoE-Megakernel Mixture-of-Kittens als Open Source",
 // introduction), so that nothing between the layer's steps waits on the CPU
 // ("Kommunikation im Kernel").  On one B200 the steps become phases of one
-// cooperative launch, one CTA per SM, 320 threads (the GEMM roles: TMA
-// producer, MMA issuer, four epilogue warps, four pull warps):
+// cooperative launch, one CTA per SM, 256 threads (the GEMM roles: TMA
+// producer, MMA issuer, four epilogue warps, two pull warps):
 //
 //   P0  zero the launch's counters; split the router weights into three bf16
 //       terms; MXFP8: quantise x
@@ -52,7 +52,7 @@
 
 namespace mok {
 
-constexpr int kFusedThreads = 320;
+constexpr int kFusedThreads = 64 + 32 * (4 + kPullWarps);   // the GEMM roles: 8 warps
 constexpr int kMaxFusedCtas = 1024;
 // Above any phase's own bounded waits (a CTA stops waiting after its first
 // 2 s timeout in a phase, and P4 holds two phases).

@@ -5,7 +5,7 @@
 // the layer ("Cursor åpner megakernelen som ga 41 prosent flere tokens i
 // sekundet": one deterministic kernel for the MoE layer's training step, BF16
 // backward among the measured passes).  One cooperative launch, one CTA per SM,
-// 320 threads; phases, with the grid barriers of fused.cuh:
+// 256 threads; phases, with the grid barriers of fused.cuh:
 //
 //   Q0  zero the launch's tile and readiness counters; the groups' first M tiles;
 //       MXFP8: quantise dy

@@ -9,7 +9,7 @@
 //   router (one group of all tokens, split over K): partial logits of x . [Wr_hi|Wr_mid|Wr_lo]^T
 //
 // Operand rows that belong to a token are pulled by index straight from the
-// token matrix into the shared-memory ring by four pull warps issuing 16-byte
+// token matrix into the shared-memory ring by two pull warps issuing 16-byte
 // cp.async copies (the pull-at-dispatch idea of "Cursor åpner
 // megakernelen…", paragraph on pulling versus pushing tokens, re-derived for
 // one GPU: the expert tile fetches its rows instead of a separate scatter
@@ -38,6 +38,11 @@ constexpr int BM = 128;        // UMMA M (cta_group::1, all 128 TMEM lanes)
 constexpr int BK = 64;         // one 128-byte swizzle row of bf16
 constexpr int kMaxGroups = 264;
 constexpr int kPanelM = 8;     // ragged-M raster panel height (M tiles)
+// cp.async pull warps of a kernel with a gathered operand (or MXFP8 activation
+// scales): two, so that with the TMA producer, the MMA issuer and the four
+// epilogue warps a CTA is 8 warps, two per SM sub-partition, and a thread may
+// hold up to 255 registers (10 warps put three on two sub-partitions: 168)
+constexpr int kPullWarps = 2;
 
 enum Epi : int { EPI_SWIGLU = 0, EPI_PUSH = 1, EPI_DSWIGLU = 2, EPI_WGRAD = 3, EPI_ROUTER = 4 };
 
@@ -136,7 +141,7 @@ struct GemmCfg {
     static constexpr int STAGES = HEAVY_EPI ? 3 : (BN == 256 ? 4 : (RAGGED_K ? 6 : 5));
     static constexpr int EPI_BUFS = (HEAVY_EPI || (!RAGGED_K && BN != 256)) ? 2 : 1;
     static constexpr int EPI_WARPS = 4;
-    static constexpr int PULL_WARPS = (A_GATHER || B_GATHER || MX) ? 4 : 0;   // cp.async warps
+    static constexpr int PULL_WARPS = (A_GATHER || B_GATHER || MX) ? kPullWarps : 0;   // cp.async warps
     static constexpr int PULL_WARP0 = 2 + EPI_WARPS;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + PULL_WARPS);
     static constexpr int GATHER_BYTES = A_GATHER ? A_BYTES : (B_GATHER ? B_BYTES : 0);
@@ -701,9 +706,11 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
         // matrix with 16-byte cp.async into the 128-byte-swizzled layout the MMA
         // descriptors expect (16-byte chunk c of row r lands at chunk c ^ (r & 7)).
         if constexpr (C::PULL_WARPS > 0) {
+            constexpr int NP = 32 * C::PULL_WARPS;      // pull threads
+            constexpr int RS = NP / 8;                  // a thread's rows are RS apart
             const int p = threadIdx.x - 32 * C::PULL_WARP0;
             const int c16 = p & 7;
-            const int r0 = p >> 3;                      // 0..15
+            const int r0 = p >> 3;                      // 0 .. RS-1
             const uint8_t *src = reinterpret_cast<const uint8_t *>(args.gather_src);
             const size_t ld = static_cast<size_t>(args.gather_ld) * C::ESIZE;   // bytes per token row
             int stage = 0;
@@ -713,38 +720,45 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                 if (tile >= total) break;
                 const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
                 if constexpr (!C::RAGGED_K) {
-                    // K-major A: the tile's 128 rows, this thread's rows r0 + 16 i
-                    int tok[8];
+                    // K-major A: the tile's 128 rows, this thread's rows r0 + RS i
+                    int tok[BM / RS];
                     if constexpr (C::A_GATHER) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const int r = r0 + 16 * i;
+                        for (int i = 0; i < BM / RS; ++i) {
+                            const int r = r0 + RS * i;
                             tok[i] = r < t.rows ? __ldg(args.row_token + t.m0 + r) : 0;
                         }
                     }
-                    // MXFP8 scales of A: row p (its token row when A is gathered); the weight
-                    // scales come with B from the producer
-                    const uint8_t *sfa = nullptr;
+                    // MXFP8 scales of A: rows p + NP q (their token rows when A is gathered);
+                    // the weight scales come with B from the producer
+                    const uint8_t *sfa[BM / NP];
                     if constexpr (C::MX) {
-                        const int ar = p < t.rows ? (C::A_GATHER ? __ldg(args.row_token + t.m0 + p) : t.m0 + p)
-                                                  : (C::A_GATHER ? 0 : t.m0);
-                        sfa = args.sfa_src + (size_t)ar * args.sf_ld;
+#pragma unroll
+                        for (int q = 0; q < BM / NP; ++q) {
+                            const int m = p + NP * q;
+                            const int ar = m < t.rows ? (C::A_GATHER ? __ldg(args.row_token + t.m0 + m) : t.m0 + m)
+                                                      : (C::A_GATHER ? 0 : t.m0);
+                            sfa[q] = args.sfa_src + (size_t)ar * args.sf_ld;
+                        }
                     }
                     for (int kb = 0; kb < t.nkb; ++kb) {
                         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status)) goto pull_done;
                         if constexpr (C::A_GATHER) {
                             uint8_t *dst = tiles + stage * C::STAGE_BYTES;
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                const int r = r0 + 16 * i;
+                            for (int i = 0; i < BM / RS; ++i) {
+                                const int r = r0 + RS * i;
                                 cp_async16(dst + r * 128 + ((c16 ^ (r & 7)) << 4), src + tok[i] * ld + kb * 128 + c16 * 16);
                             }
                         }
                         if constexpr (C::MX) {
                             // SF atom layout: the 4 scales of row m at byte 16 (m % 32) + 4 (m / 32) of its 128-row block
                             uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
-                            const int at = 16 * (p & 31) + 4 * (p >> 5);
-                            cp_async4(sf + at, sfa + kb * 4);
+#pragma unroll
+                            for (int q = 0; q < BM / NP; ++q) {
+                                const int m = p + NP * q;
+                                cp_async4(sf + 16 * (m & 31) + 4 * (m >> 5), sfa[q] + kb * 4);
+                            }
                         }
                         cp_async_arrive_noinc(&full_bar[stage]);
                         if (++stage == C::STAGES) {
@@ -753,17 +767,18 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         }
                     }
                 } else {
-                    // MN-major operand: 64 gathered K rows per block, this thread's rows r0 + 16 i
+                    // MN-major operand: 64 gathered K rows per block, this thread's rows r0 + RS i
                     constexpr int CH = (C::A_GATHER ? BM : C::BN) / 64;
+                    constexpr int NR = BK / RS;                 // rows per thread and K block
                     constexpr int OFF = C::A_GATHER ? 0 : C::A_BYTES;
                     const int mn0 = C::A_GATHER ? t.m0 : t.nt * C::BN;
                     const int end = t.krow0 + t.krows;
                     // token rows of K blocks kb, kb+1, kb+2: fetched three blocks ahead so
                     // that the index loads never stall the copies
-                    int tk0[4], tk1[4], tk2[4];
+                    int tk0[NR], tk1[NR], tk2[NR];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int kr = t.krow0 + r0 + 16 * i;
+                    for (int i = 0; i < NR; ++i) {
+                        const int kr = t.krow0 + r0 + RS * i;
                         tk0[i] = kr < end ? __ldg(args.row_token + kr) : 0;
                         tk1[i] = kr + BK < end ? __ldg(args.row_token + kr + BK) : 0;
                         tk2[i] = kr + 2 * BK < end ? __ldg(args.row_token + kr + 2 * BK) : 0;
@@ -772,8 +787,8 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status)) goto pull_done;
                         uint8_t *dst = tiles + stage * C::STAGE_BYTES + OFF;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int r = r0 + 16 * i;
+                        for (int i = 0; i < NR; ++i) {
+                            const int r = r0 + RS * i;
                             const uint8_t *row = src + tk0[i] * ld + mn0 * C::ESIZE + c16 * 16;
 #pragma unroll
                             for (int j = 0; j < CH; ++j)
@@ -781,8 +796,8 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         }
                         cp_async_arrive_noinc(&full_bar[stage]);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int kr = t.krow0 + (kb + 3) * BK + r0 + 16 * i;
+                        for (int i = 0; i < NR; ++i) {
+                            const int kr = t.krow0 + (kb + 3) * BK + r0 + RS * i;
                             tk0[i] = tk1[i];
                             tk1[i] = tk2[i];
                             tk2[i] = kr < end ? __ldg(args.row_token + kr) : 0;

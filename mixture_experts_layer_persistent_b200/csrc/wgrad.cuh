@@ -46,7 +46,7 @@ struct WgradResCfg {
     static constexpr int STAGES = 4;
     static constexpr int EPI_WARPS = 4;                      // 4 or 8 (two per TMEM lane quarter)
     static constexpr int EPI_BUFS = 2;
-    static constexpr int PULL_WARPS = 4;
+    static constexpr int PULL_WARPS = kPullWarps;
     static constexpr int PULL_WARP0 = 2 + EPI_WARPS;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + PULL_WARPS);
     static constexpr int TMEM_COLS = 2 * BN;                 // two accumulators
@@ -233,9 +233,11 @@ __device__ __forceinline__ void wgrad_resident_phase(uint8_t *smem, uint64_t *ba
         }
     } else if (warp >= C::PULL_WARP0) {
         // ------------------------------------------------------------ pull warps (gathered operand)
-        // Thread p copies 16-byte column c16 of rows r0 + 16 i (i < 4) of every
+        // Thread p copies 16-byte column c16 of rows r0 + RS i (i < NR) of every
         // 64-row K block; a row's token index is the same for every M tile of
         // the unit, so the indices are read once per unit.
+        constexpr int RS = 32 * C::PULL_WARPS / 8;     // a thread's rows are RS apart
+        constexpr int NR = BK / RS;                    // rows per thread and K block
         const int p = threadIdx.x - 32 * C::PULL_WARP0;
         const int c16 = p & 7;
         const int r0 = p >> 3;
@@ -249,12 +251,12 @@ __device__ __forceinline__ void wgrad_resident_phase(uint8_t *smem, uint64_t *ba
         for (int u = blockIdx.x; u < total && ok; u += gridDim.x) {
             const WUnit w = decode_unit(u, args, nbig, m_chunks);
             if (w.nkb == 0) continue;
-            int tok[C::KB_MAX][4];
+            int tok[C::KB_MAX][NR];
 #pragma unroll
             for (int kb = 0; kb < C::KB_MAX; ++kb)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int kr = kb * BK + r0 + 16 * i;
+                for (int i = 0; i < NR; ++i) {
+                    const int kr = kb * BK + r0 + RS * i;
                     tok[kb][i] = kr < w.krows ? __ldg(args.row_token + w.krow0 + kr) : -1;
                 }
             if constexpr (C::B_GATHER) {
@@ -267,8 +269,8 @@ __device__ __forceinline__ void wgrad_resident_phase(uint8_t *smem, uint64_t *ba
                     if (kb >= w.nkb) break;
                     uint8_t *dst = sB + kb * C::B_KB_BYTES;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int r = r0 + 16 * i;
+                    for (int i = 0; i < NR; ++i) {
+                        const int r = r0 + RS * i;
                         uint8_t *d = dst + r * 128 + ((c16 ^ (r & 7)) << 4);
                         if (tok[kb][i] >= 0) {
                             const uint8_t *row = src + tok[kb][i] * ld + (w.nt * C::BN) * 2 + c16 * 16;
@@ -292,8 +294,8 @@ __device__ __forceinline__ void wgrad_resident_phase(uint8_t *smem, uint64_t *ba
                         if (!ok) break;
                         uint8_t *dst = sA + stage * C::A_BYTES;
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int r = r0 + 16 * i;
+                        for (int i = 0; i < NR; ++i) {
+                            const int r = r0 + RS * i;
                             uint8_t *d = dst + r * 128 + ((c16 ^ (r & 7)) << 4);
                             if (tok[kb][i] >= 0) {
                                 const uint8_t *row = src + tok[kb][i] * ld + (mt * BM) * 2 + c16 * 16;
