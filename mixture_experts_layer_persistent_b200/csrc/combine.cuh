@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(const float *__restrict
 // A persistent CTA has 8 warps per SM, far too few to hide HBM latency with the
 // one-thread-per-element code above (the split kernels rely on 64 resident warps
 // per SM).  Here every thread streams its own 16-byte pieces through a private
-// ring of shared-memory slots with cp.async, NS units deep, so the loads of the
+// ring of shared-memory slots with cp.async, NS units deep (up to 6), so the loads of the
 // next NS-1 units are in flight while a unit is summed.  A thread reads back only
 // the bytes it copied itself, so no barrier is needed between copy and use.  The
 // arithmetic per output column is that of combine_elem / dx_combine_elem /
@@ -273,11 +273,11 @@ __device__ __forceinline__ uint8_t *stream_slot(uint8_t *ring, int s, int R, int
     return ring + ((static_cast<size_t>(s) * R + j) * blockDim.x + threadIdx.x) * 16;
 }
 
-// stages that fit: units of R rows of 16 bytes per thread, at most 4
+// stages that fit: units of R rows of 16 bytes per thread, at most 6
 __device__ __forceinline__ int stream_stages(int R, int ring_bytes)
 {
     const int ns = ring_bytes / (R * 16 * static_cast<int>(blockDim.x));
-    return ns < 1 ? 1 : (ns > 4 ? 4 : ns);
+    return ns < 1 ? 1 : (ns > 6 ? 6 : ns);
 }
 
 template <int EPU>
@@ -357,7 +357,9 @@ __device__ __forceinline__ void combine_stream(const Slot *__restrict__ O, const
     case 1: combine_stream_ns<Slot, 1>(O, topk_w, y, T, H, k, S, ring); break;
     case 2: combine_stream_ns<Slot, 2>(O, topk_w, y, T, H, k, S, ring); break;
     case 3: combine_stream_ns<Slot, 3>(O, topk_w, y, T, H, k, S, ring); break;
-    default: combine_stream_ns<Slot, 4>(O, topk_w, y, T, H, k, S, ring); break;
+    case 4: combine_stream_ns<Slot, 4>(O, topk_w, y, T, H, k, S, ring); break;
+    case 5: combine_stream_ns<Slot, 5>(O, topk_w, y, T, H, k, S, ring); break;
+    default: combine_stream_ns<Slot, 6>(O, topk_w, y, T, H, k, S, ring); break;
     }
 }
 
@@ -436,20 +438,22 @@ __device__ __forceinline__ void dx_stream(const float *__restrict__ dXs, const f
     case 1: dx_stream_ns<1>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
     case 2: dx_stream_ns<2>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
     case 3: dx_stream_ns<3>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
-    default: dx_stream_ns<4>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
+    case 4: dx_stream_ns<4>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
+    case 5: dx_stream_ns<5>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
+    default: dx_stream_ns<6>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
     }
 }
 
 // Router-gradient partial sums: warp = item (row chunk, 256 columns), lane = 8
 // columns.  The item's rows run in units of 8 (one row per residue r0 + w mod 8),
-// four units deep; a warp-private table in shared memory holds each row's token
+// kDrouterStages units deep; a warp-private table in shared memory holds each row's token
 // and dl, loaded once per item.  Sums per residue in ascending row order, then
 // over the residues in order of w, as drouter_partial_kernel.
-//   smem: the ring (4 stages x 8 rows x 16 bytes per thread), then the warps'
+//   smem: the ring (kDrouterStages stages x 8 rows x 16 bytes per thread), then the warps'
 //   row tables (kDrouterMaxRows x 8 bytes per warp), then chunk_start and offsets
 //   ((E + 1) ints each).  Needs drouter_stream_bytes(E) bytes.
 constexpr int kDrouterMaxRows = 256;             // rows per chunk at most
-constexpr int kDrouterStages = 4;
+constexpr int kDrouterStages = 6;
 __host__ __device__ constexpr int drouter_stream_bytes(int threads, int E)
 {
     return kDrouterStages * 8 * 16 * threads + threads / 32 * kDrouterMaxRows * 8 + 2 * (E + 1) * 4;
