@@ -413,8 +413,10 @@ int moe_launch_count(int *count);
  * Fault-injection hook for testing the bounded waits.  While enabled (non-zero),
  * every BF16 forward launched by this host thread makes CTA 0 of the gate/up
  * GEMM and CTA 0 of the down GEMM skip the signal that hands their first
- * accumulator to the epilogue; each epilogue's wait then runs out after about
- * 2 s, the kernel records MOK_STATUS_TIMEOUT and returns (no trap, no fault).
+ * accumulator to the epilogue, and every backward does the same in its down
+ * dgrad GEMM; each epilogue's wait then runs out after about 2 s (and, in a
+ * persistent pass, so do the readiness waits of the tiles that need the missing
+ * one), the kernel records MOK_STATUS_TIMEOUT and returns (no trap, no fault).
  * Results of such a call are meaningless.  Off by default.
  */
 int moe_test_drop_signal(int enable);

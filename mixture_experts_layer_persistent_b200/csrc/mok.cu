@@ -735,6 +735,7 @@ int build_bwd_plan(const moe_cfg &c, const void *x, const void *dy, const moe_pa
     g1.gpart = bs.gpart;
     g1.out = bs.dgu;
     g1.n_tiles = pl.n256 ? c.I / 256 : c.I / 128;   // N = 256 halves the gathered dy rows per weight byte
+    g1.test_drop_signal = t_drop_signal;
 
     // wgrad of down: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
     if (!make_tmap(&pl.m.w2O, gr.dw_down, s.I, s.E * s.H, 64, 32, 2)) return MOK_ERR_INVALID;
