@@ -209,7 +209,7 @@ def backward_algorithmic(wl, counts):
 
 
 BWD_STAMP_PHASES = ["q0_zero", "dgrads", "down_wgrad_after_dgrads", "gate_up_wgrad_after_down_wgrad", "slot_grad",
-                    "router_partial_dx", "router_reduce"]
+                    "router_partial", "dx_sum", "router_reduce"]
 
 
 STAMP_PHASES = ["p0_zero_split_quant", "router_gemm", "select", "dispatch", "gate_up_gemm", "down_after_gate_up",
@@ -222,13 +222,14 @@ def stamp_phases(bufs, sms, names=None):
     release) to the last CTA's end of its own; the down GEMM overlaps the gate/up
     tail, so its span counts only the part after the last gate/up tile."""
     import numpy as np
-    acc = np.zeros(len(names or STAMP_PHASES))
+    names = names or STAMP_PHASES
+    acc = np.zeros(len(names))
     for b in bufs:
-        t = b.view(-1, sms).cpu().numpy().astype(np.float64)
+        t = b.view(-1, sms).cpu().numpy().astype(np.float64)[: len(names) + 1]
         ends = t.max(axis=1)
         acc[0] += ends[1] - t[0].min()
         acc[1:] += np.diff(ends[1:])
-    return {n: round(float(v) / len(bufs) / 1e6, 4) for n, v in zip(names or STAMP_PHASES, acc)}
+    return {n: round(float(v) / len(bufs) / 1e6, 4) for n, v in zip(names, acc)}
 
 
 def _ab(layer, run, K, legs, trace_split, stamp_names):

@@ -393,12 +393,12 @@ int moe_get_schedule(int *schedule);
  * and CTA b, the globaltimer value (ns) at buf[p * SMs + b].  Forward points:
  * p = 0 start, then the end of the zeroing / router-split / quantisation
  * phase, the router GEMM, the top-k, the dispatch, the gate/up GEMM, the down
- * GEMM and the combine.  Backward points: p = 0 start, then the end of the
- * zeroing, of the two dgrads, of the down weight gradient, of the gate/up
- * weight gradient, of the slot gradients, of the router partial sums + dx, and
- * of the router-gradient reduction.  NULL stops the stamps.
+ * GEMM and the combine; p = 8 repeats the end.  Backward points: p = 0 start,
+ * then the end of the zeroing, of the two dgrads, of the down weight gradient,
+ * of the gate/up weight gradient, of the slot gradients, of the router partial
+ * sums, of dx, and of the router-gradient reduction.  NULL stops the stamps.
  */
-#define MOK_TRACE_POINTS 8
+#define MOK_TRACE_POINTS 9
 int moe_trace_device(void *buf, size_t bytes, void *bwd_buf, size_t bwd_bytes);
 
 /*

@@ -32,7 +32,7 @@ MOK_STATIC_SCRATCH_BYTES = 32 << 20
 MOK_SCHEDULE_PERSISTENT = 0
 MOK_SCHEDULE_SPLIT = 1
 MOK_SCHEDULE_SPLIT_PDL = 2
-MOK_TRACE_POINTS = 8
+MOK_TRACE_POINTS = 9
 MOK_SAVED_H, MOK_SAVED_HQ, MOK_SAVED_HS, MOK_SAVED_GU, MOK_SAVED_HW, MOK_SAVED_ROW_TOKEN, MOK_SAVED_ROW_W = range(7)
 
 _i32, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t

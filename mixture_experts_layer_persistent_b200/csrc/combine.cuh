@@ -192,6 +192,53 @@ __device__ __forceinline__ void drouter_reduce_elem(long long i, const float *__
     dWr[i] = s;
 }
 
+// The same reduction in the persistent kernel: four columns per thread and four
+// independent column groups in flight (one dependent load at a time per thread
+// cannot hide the latency with 8 warps per SM); each element still sums its
+// chunks in ascending order from 0 (same bits).
+__device__ __forceinline__ void drouter_reduce_stream(const float *__restrict__ partial,
+                                                      const int *__restrict__ chunk_start, float *__restrict__ dWr,
+                                                      int H, int E)
+{
+    constexpr int U = 4;
+    const long long nq = static_cast<long long>(E) * H / 4;
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long q0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; q0 < nq; q0 += U * stride) {
+        int c0[U], c1[U];
+        long long i4[U];
+        float4 acc[U];
+        int nmax = 0;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const long long q = q0 + u * stride;
+            i4[u] = q * 4;
+            c0[u] = c1[u] = 0;
+            if (q < nq) {
+                const int e = static_cast<int>(i4[u] / H);
+                c0[u] = chunk_start[e];
+                c1[u] = chunk_start[e + 1];
+            }
+            acc[u] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            nmax = max(nmax, c1[u] - c0[u]);
+        }
+        for (int j = 0; j < nmax; ++j) {
+            float4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (c0[u] + j < c1[u])
+                    v[u] = *reinterpret_cast<const float4 *>(partial + static_cast<size_t>(c0[u] + j) * H + i4[u] % H);
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (c0[u] + j < c1[u]) {
+                    acc[u].x += v[u].x; acc[u].y += v[u].y; acc[u].z += v[u].z; acc[u].w += v[u].w;
+                }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (q0 + u * stride < nq) *reinterpret_cast<float4 *>(dWr + i4[u]) = acc[u];
+    }
+}
+
 __global__ void __launch_bounds__(256) drouter_reduce_kernel(const float *__restrict__ partial,
                                                              const int *__restrict__ chunk_start,
                                                              float *__restrict__ dWr, int H, int E)

@@ -89,8 +89,9 @@ struct FusedFwdArgs {
     unsigned long long *trace;     // null, or [kFusedTracePoints][gridDim.x] globaltimer stamps
 };
 
-// trace points: start, then the end of P0, P1, P2, P3, gate/up, down, P5
-constexpr int kFusedTracePoints = 8;
+// trace points: start, then the end of P0, P1, P2, P3, gate/up, down, P5; the
+// ninth repeats the end (the backward has one point more)
+constexpr int kFusedTracePoints = 9;
 
 struct FusedMaps {
     CUtensorMap rA, rB, rO;                  // router GEMM
@@ -184,7 +185,7 @@ struct FusedCfg {
     static_assert(Router::THREADS <= kFusedThreads && GateUp::THREADS <= kFusedThreads &&
                   Down::THREADS <= kFusedThreads, "phase roles fit the launch");
     // routing phases use the ring's memory: select rows, dispatch masks and tables
-    static_assert(kFusedThreads / 32 * 256 * 4 <= RING && (256 * 32 + 512) * 4 <= RING, "routing scratch");
+    static_assert(kFusedThreads / 32 * 256 * 4 <= RING && (256 * kMaskWords + 512) * 4 <= RING, "routing scratch");
 };
 
 template <bool MX>
@@ -245,8 +246,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
 
     // ---------------------------------------------------------------- P3
     if (alive) {
-        uint32_t(*s_mask)[32] = reinterpret_cast<uint32_t(*)[32]>(smem);
-        int *s_base = reinterpret_cast<int *>(smem) + 256 * 32;
+        uint32_t(*s_mask)[kMaskWords] = reinterpret_cast<uint32_t(*)[kMaskWords]>(smem);
+        int *s_base = reinterpret_cast<int *>(smem) + 256 * kMaskWords;
         int *s_cnt = s_base + 256;
         for (int c = blockIdx.x; c < a.n_chunks; c += gridDim.x)
             dispatch_scan_place_chunk(a.da, c, a.n_chunks, c == 0, s_mask, s_base, s_cnt);
@@ -279,6 +280,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
                                   F::RING);
     }
     fused_stamp(a, 7);
+    fused_stamp(a, 8);
 
     tc_fence_before();
     __syncthreads();

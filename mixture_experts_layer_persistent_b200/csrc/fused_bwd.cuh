@@ -69,9 +69,9 @@ struct FusedBwdArgs {
 };
 
 // trace points: start, end of Q0, end of the dgrads, of the down weight gradient,
-// of the gate/up weight gradient, of the slot gradients, of the router partials +
-// dx, of the router-gradient reduction
-constexpr int kFusedBwdTracePoints = 8;
+// of the gate/up weight gradient, of the slot gradients, of the router partials,
+// of dx, of the router-gradient reduction
+constexpr int kFusedBwdTracePoints = 9;
 
 struct FusedBwdMaps {
     CUtensorMap d1B, d1Bs, d1O;              // down dgrad: W_down (MN-major), shared, dGU out
@@ -212,20 +212,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     // ---------------------------------------------------------------- Q5
     // router-gradient partials, then the dx sum, both streamed through the
     // region's shared memory (drouter_stream, dx_stream)
-    if (alive) {
-        drouter_stream(a.x, a.dl, a.offsets, a.chunk_start, a.perm, a.partial, a.H, a.E, a.k, a.chunk_rows, smem);
-        __syncthreads();                       // the region is free again
-        dx_stream(a.dxs, a.dl, a.topk_idx, a.router_w, a.dx, a.T, a.H, a.k, a.S, smem, F::REGION);
-    }
+    if (alive) drouter_stream(a.x, a.dl, a.offsets, a.chunk_start, a.perm, a.partial, a.H, a.E, a.k, a.chunk_rows, smem);
     fused_bwd_stamp(a, 6);
+    __syncthreads();                           // the region is free again
+    if (alive) dx_stream(a.dxs, a.dl, a.topk_idx, a.router_w, a.dx, a.T, a.H, a.k, a.S, smem, F::REGION);
+    fused_bwd_stamp(a, 7);
     alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
 
     // ---------------------------------------------------------------- Q6
-    if (alive) {
-        const long long n = static_cast<long long>(a.E) * a.H;
-        for (long long i = gtid; i < n; i += gstride) drouter_reduce_elem(i, a.partial, a.chunk_start, a.drouter_w, a.H);
-    }
-    fused_bwd_stamp(a, 7);
+    if (alive) drouter_reduce_stream(a.partial, a.chunk_start, a.drouter_w, a.H, a.E);
+    fused_bwd_stamp(a, 8);
 
     tc_fence_before();
     __syncthreads();

@@ -616,72 +616,144 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
             const bool routed = t.g < args.num_routed;
             const CUtensorMap *mB = routed ? &tmB : &tmB_s;
             const int gl = routed ? t.g : t.g - args.num_routed;
-            const int claim_kb = t.nkb > kClaimAhead ? t.nkb - kClaimAhead : 0;
-            int next = 0;
-            if (t.nkb == 0 && lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(args.sched, 1);
-            for (int kb = 0; kb < t.nkb; ++kb) {
-                if (kb == claim_kb && lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(args.sched, 1);
+            if constexpr (C::RAGGED_K) {
+                // weight gradients (MN-major operands, two and four boxes per K block, a
+                // few K blocks per tile): the lanes issue the boxes in parallel after
+                // lane 0's wait, which measured faster here than lane 0 alone
+                const int claim_kb = t.nkb > kClaimAhead ? t.nkb - kClaimAhead : 0;
+                int next = 0;
+                if (t.nkb == 0 && lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(args.sched, 1);
+                for (int kb = 0; kb < t.nkb; ++kb) {
+                    if (kb == claim_kb && lane == 0) next = static_cast<int>(gridDim.x) + atomicAdd(args.sched, 1);
+                    bool ok = true;
+                    if (lane == 0) {
+                        ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status);
+                        if (ok) mbar_arrive_expect_tx(&full_bar[stage], C::TMA_BYTES);
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) goto producer_done;
+                    uint8_t *sA = tiles + stage * C::STAGE_BYTES;
+                    uint8_t *sB = sA + C::A_BYTES;
+                    uint64_t *fb = &full_bar[stage];
+                    const int kg = C::EPI == EPI_ROUTER ? t.nt * args.num_kb + kb : kb;   // global K block
+                    constexpr int KE = C::KB_ELEMS;
+                    // ---- A (gathered A rows come from the pull warps)
+                    if constexpr (!C::A_GATHER && !C::A_MN) {
+                        if (lane == 0) {
+                            const int kc = C::EPI == EPI_ROUTER ? (kg * BK) % args.a_k_mod : kb * KE;
+                            tma_load_2d(sA, &tmA, fb, kc, t.m0);
+                        }
+                    } else if constexpr (!C::A_GATHER && C::A_MN) {
+                        if (lane < BM / 64) tma_load_2d(sA + lane * 8192, &tmA, fb, t.m0 + lane * 64, t.krow0 + kb * BK);
+                    }
+                    // ---- B
+                    if constexpr (!C::B_MN) {
+                        if (lane == 0) {
+                            if constexpr (C::EPI == EPI_SWIGLU) {
+                                const int row = gl * args.b_rows_per_group + t.nt * 128;
+                                tma_load_2d(sB, mB, fb, kb * KE, row);
+                                tma_load_2d(sB + 128 * 128, mB, fb, kb * KE, row + args.b_half);
+                            } else if constexpr (C::EPI == EPI_ROUTER) {
+                                tma_load_2d(sB, mB, fb, kg * BK, 0);
+                            } else {
+                                tma_load_2d(sB, mB, fb, kb * KE, gl * args.b_rows_per_group + t.nt * C::BN);
+                            }
+                        }
+                    } else if constexpr (!C::B_GATHER && !C::RAGGED_K) {
+                        if (lane < C::BN / 64)
+                            tma_load_2d(sB + lane * 8192, mB, fb, t.nt * C::BN + lane * 64,
+                                        gl * args.b_rows_per_group + kb * BK);
+                    } else if constexpr (!C::B_GATHER && C::RAGGED_K) {
+                        if (lane < C::BN / 64)
+                            tma_load_2d(sB + lane * 8192, &tmB, fb, t.nt * C::BN + lane * 64, t.krow0 + kb * BK);
+                    }
+                    if constexpr (C::MX) {
+                        // the weight scales of this K block: one packed 512-byte tile per 128 B rows
+                        if (lane == 0) {
+                            const uint8_t *sb = routed ? args.sfb_src : args.sfb_src_s;
+                            const long long rt = routed ? args.sfb_row_tiles : args.sfb_row_tiles_s;
+                            const int r0 = gl * args.b_rows_per_group + (C::EPI == EPI_SWIGLU ? t.nt * 128 : t.nt * C::BN);
+                            const int r1 = C::EPI == EPI_SWIGLU ? r0 + args.b_half : r0 + 128;
+                            uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
+                            bulk_load(sf + 512, sb + (static_cast<long long>(kb) * rt + (r0 >> 7)) * 512, 512, fb);
+                            bulk_load(sf + 1024, sb + (static_cast<long long>(kb) * rt + (r1 >> 7)) * 512, 512, fb);
+                        }
+                    }
+                    ++fills;
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                tile = __shfl_sync(0xffffffffu, next, 0);
+            } else {
+                // lane 0 alone runs the tile's K loop
+                const int claim_kb = t.nkb > kClaimAhead ? t.nkb - kClaimAhead : 0;
+                int next = 0;
                 bool ok = true;
                 if (lane == 0) {
-                    ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status);
-                    if (ok) mbar_arrive_expect_tx(&full_bar[stage], C::TMA_BYTES);
+                    // the tile's K loop by lane 0 alone (no warp-wide step per K block)
+                    if (t.nkb == 0) next = static_cast<int>(gridDim.x) + atomicAdd(args.sched, 1);
+                    for (int kb = 0; kb < t.nkb; ++kb) {
+                        if (kb == claim_kb) next = static_cast<int>(gridDim.x) + atomicAdd(args.sched, 1);
+                        ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status);
+                        if (!ok) break;
+                        mbar_arrive_expect_tx(&full_bar[stage], C::TMA_BYTES);
+                        uint8_t *sA = tiles + stage * C::STAGE_BYTES;
+                        uint8_t *sB = sA + C::A_BYTES;
+                        uint64_t *fb = &full_bar[stage];
+                        const int kg = C::EPI == EPI_ROUTER ? t.nt * args.num_kb + kb : kb;   // global K block
+                        constexpr int KE = C::KB_ELEMS;
+                        // ---- A (gathered A rows come from the pull warps)
+                        if constexpr (!C::A_GATHER && !C::A_MN) {
+                            const int kc = C::EPI == EPI_ROUTER ? (kg * BK) % args.a_k_mod : kb * KE;
+                            tma_load_2d(sA, &tmA, fb, kc, t.m0);
+                        } else if constexpr (!C::A_GATHER && C::A_MN) {
+#pragma unroll
+                            for (int c = 0; c < BM / 64; ++c)
+                                tma_load_2d(sA + c * 8192, &tmA, fb, t.m0 + c * 64, t.krow0 + kb * BK);
+                        }
+                        // ---- B
+                        if constexpr (!C::B_MN) {
+                            if constexpr (C::EPI == EPI_SWIGLU) {
+                                const int row = gl * args.b_rows_per_group + t.nt * 128;
+                                tma_load_2d(sB, mB, fb, kb * KE, row);
+                                tma_load_2d(sB + 128 * 128, mB, fb, kb * KE, row + args.b_half);
+                            } else if constexpr (C::EPI == EPI_ROUTER) {
+                                tma_load_2d(sB, mB, fb, kg * BK, 0);
+                            } else {
+                                tma_load_2d(sB, mB, fb, kb * KE, gl * args.b_rows_per_group + t.nt * C::BN);
+                            }
+                        } else if constexpr (!C::B_GATHER && !C::RAGGED_K) {
+#pragma unroll
+                            for (int c = 0; c < C::BN / 64; ++c)
+                                tma_load_2d(sB + c * 8192, mB, fb, t.nt * C::BN + c * 64, gl * args.b_rows_per_group + kb * BK);
+                        } else if constexpr (!C::B_GATHER && C::RAGGED_K) {
+#pragma unroll
+                            for (int c = 0; c < C::BN / 64; ++c)
+                                tma_load_2d(sB + c * 8192, &tmB, fb, t.nt * C::BN + c * 64, t.krow0 + kb * BK);
+                        }
+                        if constexpr (C::MX) {
+                            // the weight scales of this K block: one packed 512-byte tile per 128 B rows
+                            const uint8_t *sb = routed ? args.sfb_src : args.sfb_src_s;
+                            const long long rt = routed ? args.sfb_row_tiles : args.sfb_row_tiles_s;
+                            const int r0 = gl * args.b_rows_per_group + (C::EPI == EPI_SWIGLU ? t.nt * 128 : t.nt * C::BN);
+                            const int r1 = C::EPI == EPI_SWIGLU ? r0 + args.b_half : r0 + 128;
+                            uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
+                            bulk_load(sf + 512, sb + (static_cast<long long>(kb) * rt + (r0 >> 7)) * 512, 512, fb);
+                            bulk_load(sf + 1024, sb + (static_cast<long long>(kb) * rt + (r1 >> 7)) * 512, 512, fb);
+                        }
+                        ++fills;
+                        if (++stage == C::STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) goto producer_done;
-                uint8_t *sA = tiles + stage * C::STAGE_BYTES;
-                uint8_t *sB = sA + C::A_BYTES;
-                uint64_t *fb = &full_bar[stage];
-                const int kg = C::EPI == EPI_ROUTER ? t.nt * args.num_kb + kb : kb;   // global K block
-                constexpr int KE = C::KB_ELEMS;
-                // ---- A (gathered A rows come from the pull warps)
-                if constexpr (!C::A_GATHER && !C::A_MN) {
-                    if (lane == 0) {
-                        const int kc = C::EPI == EPI_ROUTER ? (kg * BK) % args.a_k_mod : kb * KE;
-                        tma_load_2d(sA, &tmA, fb, kc, t.m0);
-                    }
-                } else if constexpr (!C::A_GATHER && C::A_MN) {
-                    if (lane < BM / 64) tma_load_2d(sA + lane * 8192, &tmA, fb, t.m0 + lane * 64, t.krow0 + kb * BK);
-                }
-                // ---- B
-                if constexpr (!C::B_MN) {
-                    if (lane == 0) {
-                        if constexpr (C::EPI == EPI_SWIGLU) {
-                            const int row = gl * args.b_rows_per_group + t.nt * 128;
-                            tma_load_2d(sB, mB, fb, kb * KE, row);
-                            tma_load_2d(sB + 128 * 128, mB, fb, kb * KE, row + args.b_half);
-                        } else if constexpr (C::EPI == EPI_ROUTER) {
-                            tma_load_2d(sB, mB, fb, kg * BK, 0);
-                        } else {
-                            tma_load_2d(sB, mB, fb, kb * KE, gl * args.b_rows_per_group + t.nt * C::BN);
-                        }
-                    }
-                } else if constexpr (!C::B_GATHER && !C::RAGGED_K) {
-                    if (lane < C::BN / 64)
-                        tma_load_2d(sB + lane * 8192, mB, fb, t.nt * C::BN + lane * 64,
-                                    gl * args.b_rows_per_group + kb * BK);
-                } else if constexpr (!C::B_GATHER && C::RAGGED_K) {
-                    if (lane < C::BN / 64)
-                        tma_load_2d(sB + lane * 8192, &tmB, fb, t.nt * C::BN + lane * 64, t.krow0 + kb * BK);
-                }
-                if constexpr (C::MX) {
-                    // the weight scales of this K block: one packed 512-byte tile per 128 B rows
-                    if (lane == 0) {
-                        const uint8_t *sb = routed ? args.sfb_src : args.sfb_src_s;
-                        const long long rt = routed ? args.sfb_row_tiles : args.sfb_row_tiles_s;
-                        const int r0 = gl * args.b_rows_per_group + (C::EPI == EPI_SWIGLU ? t.nt * 128 : t.nt * C::BN);
-                        const int r1 = C::EPI == EPI_SWIGLU ? r0 + args.b_half : r0 + 128;
-                        uint8_t *sf = sf_tiles + stage * C::SF_BYTES;
-                        bulk_load(sf + 512, sb + (static_cast<long long>(kb) * rt + (r0 >> 7)) * 512, 512, fb);
-                        bulk_load(sf + 1024, sb + (static_cast<long long>(kb) * rt + (r1 >> 7)) * 512, 512, fb);
-                    }
-                }
-                ++fills;
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                tile = __shfl_sync(0xffffffffu, next, 0);
             }
-            tile = __shfl_sync(0xffffffffu, next, 0);
         }
     producer_done:
         if (lane == 0) {
@@ -814,6 +886,12 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
+        // Lane 0 alone runs a tile's K loop: the tensor core queues about one MMA
+        // beyond the one it executes, so every cycle the issuer spends between two
+        // K blocks (a warp shuffle and barrier per block cost about a fifth of the
+        // MMA rate) is tensor-core idle time; the warp joins once per tile.  The
+        // weight gradients keep the warp in the loop (their last K block's tail rows
+        // are zeroed by the 32 lanes).
         int stage = 0, acc = 0;
         uint32_t phase = 0, acc_phase = 0;
         for (int it = 0;; ++it) {
@@ -826,35 +904,80 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
             if (!ok) break;
             tc_fence_after();
             const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
-            for (int kb = 0; kb < t.nkb; ++kb) {
-                if (lane == 0) ok = mbar_wait(&full_bar[stage], phase, abort_flag, status);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                uint8_t *sA = tiles + stage * C::STAGE_BYTES;
-                uint8_t *sB = sA + C::A_BYTES;
-                if constexpr (C::RAGGED_K) {
-                    const int valid = t.krows - kb * BK;
-                    if (valid < BK) {
-                        // rows past the group's end: zero them in the contiguous operand
-                        // (the gathered operand holds finite rows there)
-                        uint8_t *base = C::A_GATHER ? sB : sA;
-                        const int chunks = C::A_GATHER ? C::BN / 64 : BM / 64;
-                        const int n16 = (BK - valid) * 8;
-                        for (int c = 0; c < chunks; ++c) {
-                            uint4 *p = reinterpret_cast<uint4 *>(base + c * 8192 + valid * 128);
-                            for (int i = lane; i < n16; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
+            if constexpr (C::RAGGED_K) {
+                // weight gradients (a few K blocks per tile, the last one ragged): the
+                // warp walks the K loop together, which measured faster here
+                for (int kb = 0; kb < t.nkb; ++kb) {
+                    if (lane == 0) ok = mbar_wait(&full_bar[stage], phase, abort_flag, status);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    uint8_t *sA = tiles + stage * C::STAGE_BYTES;
+                    uint8_t *sB = sA + C::A_BYTES;
+                    if constexpr (C::RAGGED_K) {
+                        const int valid = t.krows - kb * BK;
+                        if (valid < BK) {
+                            // rows past the group's end: zero them in the contiguous operand
+                            // (the gathered operand holds finite rows there)
+                            uint8_t *base = C::A_GATHER ? sB : sA;
+                            const int chunks = C::A_GATHER ? C::BN / 64 : BM / 64;
+                            const int n16 = (BK - valid) * 8;
+                            for (int c = 0; c < chunks; ++c) {
+                                uint4 *p = reinterpret_cast<uint4 *>(base + c * 8192 + valid * 128);
+                                for (int i = lane; i < n16; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
+                            }
+                            fence_proxy_async_smem();
+                            __syncwarp();
                         }
-                        fence_proxy_async_smem();
-                        __syncwarp();
+                    }
+                    tc_fence_after();
+                    if (lane == 0) {
+                        if constexpr (C::PULL_WARPS > 0) fence_proxy_async_smem();   // cp.async data -> tensor core
+                        const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+                        if constexpr (C::MX) {
+                            // scales of this K block into TMEM (issued before, so ordered with, the MMAs)
+                            const uint32_t sf0 = smem_u32(sf_tiles + stage * C::SF_BYTES);
+                            const uint32_t tsfa = tmem_base + C::SF_TMEM_COL, tsfb = tsfa + 4;
+                            tmem_cp_32x128b_x4(tsfa, smem_desc_plain(sf0));
+#pragma unroll
+                            for (int b = 0; b < C::BN / 128; ++b) tmem_cp_32x128b_x4(tsfb + 4 * b, smem_desc_plain(sf0 + 512 + 512 * b));
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const uint64_t ad = smem_desc_sw128(a0 + k * 32, 16, 1024);
+                                const uint64_t bd = smem_desc_sw128(b0 + k * 32, 16, 1024);
+                                const uint32_t j = static_cast<uint32_t>(k);
+                                umma_mxf8(d_tmem, ad, bd, idesc_mxf8(BM, C::BN, j), tsfa | (j << 30), tsfb | (j << 30),
+                                          (kb | k) != 0 ? 1u : 0u);
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < BK / 16; ++k) {
+                                const uint64_t ad = C::A_MN ? smem_desc_sw128(a0 + k * 2048, 8192, 1024)
+                                                            : smem_desc_sw128(a0 + k * 32, 16, 1024);
+                                const uint64_t bd = C::B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024)
+                                                            : smem_desc_sw128(b0 + k * 32, 16, 1024);
+                                umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                            }
+                        }
+                        umma_commit(&empty_bar[stage]);
+                    }
+                    __syncwarp();
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
                     }
                 }
-                tc_fence_after();
-                if (lane == 0) {
+                if (!ok) break;
+            } else {
+                // issue K block kb from stage st (lane 0); every lane advances stage / phase
+                // itself, so the warp needs no broadcast of them
+                auto issue_kb = [&](int kb, int st) {
+                    uint8_t *sA = tiles + st * C::STAGE_BYTES;
+                    uint8_t *sB = sA + C::A_BYTES;
                     if constexpr (C::PULL_WARPS > 0) fence_proxy_async_smem();   // cp.async data -> tensor core
                     const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
                     if constexpr (C::MX) {
                         // scales of this K block into TMEM (issued before, so ordered with, the MMAs)
-                        const uint32_t sf0 = smem_u32(sf_tiles + stage * C::SF_BYTES);
+                        const uint32_t sf0 = smem_u32(sf_tiles + st * C::SF_BYTES);
                         const uint32_t tsfa = tmem_base + C::SF_TMEM_COL, tsfb = tsfa + 4;
                         tmem_cp_32x128b_x4(tsfa, smem_desc_plain(sf0));
 #pragma unroll
@@ -877,15 +1000,30 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                             umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | k) != 0 ? 1u : 0u);
                         }
                     }
-                    umma_commit(&empty_bar[stage]);
+                    umma_commit(&empty_bar[st]);
+                };
+                if (lane == 0) {
+                    int st = stage;
+                    uint32_t ph = phase;
+                    for (int kb = 0; kb < t.nkb; ++kb) {
+                        ok = mbar_wait(&full_bar[st], ph, abort_flag, status);
+                        if (!ok) break;
+                        tc_fence_after();
+                        issue_kb(kb, st);
+                        if (++st == C::STAGES) {
+                            st = 0;
+                            ph ^= 1u;
+                        }
+                    }
                 }
-                __syncwarp();
-                if (++stage == C::STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                for (int kb = 0; kb < t.nkb; ++kb)
+                    if (++stage == C::STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
             }
-            if (!ok) break;
             if (lane == 0 && !(args.test_drop_signal && blockIdx.x == 0 && tile == 0)) {
                 if (t.nkb > 0) umma_commit(&accf[acc]);
                 else mbar_arrive(&accf[acc]);

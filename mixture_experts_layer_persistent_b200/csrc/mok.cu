@@ -160,7 +160,7 @@ int router_splits(long long T, long long H)
     const long long m_tiles = (T + BM - 1) / BM;
     const long long kb = 3 * H / BK;
     long long target = 148 / m_tiles;
-    if (target > 8) target = 8;
+    if (target > kMaxRouterSplits) target = kMaxRouterSplits;
     int best = 1;
     for (int d = 1; d <= target; ++d)
         if (kb % d == 0) best = d;
@@ -571,9 +571,11 @@ int forward_split(const moe_cfg &c, const void *x, const moe_params &p, void *y,
     MOK_TRY(launch_k(router_select_kernel, dim3(blocks_for(s.T, 8)), dim3(256), 0, stream, "router_select_kernel", pl.sa));
 
     MOK_TRY(mark_fwd(1, stream));
-    MOK_TRY(launch_k(dispatch_count_kernel, dim3(pl.n_chunks), dim3(1024), 0, stream, "dispatch_count_kernel", pl.da));
+    MOK_TRY(launch_k(dispatch_count_kernel, dim3(pl.n_chunks), dim3(kDispatchChunk), 0, stream, "dispatch_count_kernel",
+                     pl.da));
     MOK_TRY(launch_k(dispatch_scan_kernel, dim3(1), dim3(256), 0, stream, "dispatch_scan_kernel", pl.da, pl.n_chunks));
-    MOK_TRY(launch_k(dispatch_place_kernel, dim3(pl.n_chunks), dim3(1024), 0, stream, "dispatch_place_kernel", pl.da));
+    MOK_TRY(launch_k(dispatch_place_kernel, dim3(pl.n_chunks), dim3(kDispatchChunk), 0, stream, "dispatch_place_kernel",
+                     pl.da));
 
     MOK_TRY(mark_fwd(2, stream));
     GemmArgs ga = pl.ga, gd = pl.gd;

@@ -63,7 +63,11 @@ struct SelectArgs {
                                 // before: the selection also counts each (token, slot) there
 };
 
-constexpr int kDispatchChunk = 1024;   // tokens per dispatch chunk
+// tokens per dispatch chunk: enough chunks that the placement spreads over many
+// CTAs, few enough mask words per expert (kDispatchChunk / 32) for the rank scan
+constexpr int kDispatchChunk = 256;
+constexpr int kMaxRouterSplits = 8;     // K splits of the router GEMM at most
+constexpr int kMaskWords = kDispatchChunk / 32;
 
 // one (value, index) candidate; larger value wins, then lower index
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib)
@@ -96,6 +100,19 @@ __device__ __forceinline__ void select_token(const SelectArgs &a, int t, int lan
 {
     const int E = a.E;
     const int npl = (E + 31) / 32;
+    // every partial and bias of the token is loaded before the first sum (one
+    // round trip instead of one per split and expert); the sums keep split order
+    float part[kMaxRouterSplits][8], lb[8], eb[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        const bool on = i < npl && e < E;
+#pragma unroll
+        for (int s = 0; s < kMaxRouterSplits; ++s)
+            part[s][i] = on && s < a.n_split ? a.partial[((size_t)s * a.T + t) * 256 + e] : 0.0f;
+        lb[i] = on && a.logit_bias ? a.logit_bias[e] : 0.0f;
+        eb[i] = on && a.e_bias ? a.e_bias[e] : 0.0f;
+    }
     float lgv[8], sel[8], sc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -105,15 +122,17 @@ __device__ __forceinline__ void select_token(const SelectArgs &a, int t, int lan
         sc[i] = 0.0f;
         if (i < npl && e < E) {
             float lg = 0.0f;
-            for (int s = 0; s < a.n_split; ++s) lg += a.partial[((size_t)s * a.T + t) * 256 + e];
-            if (a.logit_bias) lg += a.logit_bias[e];
+#pragma unroll
+            for (int s = 0; s < kMaxRouterSplits; ++s)
+                if (s < a.n_split) lg += part[s][i];
+            if (a.logit_bias) lg += lb[i];
             lgv[i] = lg;
             if (a.score_fn == 0) {
                 sel[i] = rank_score(lg);
             } else {
                 const float sg = 1.0f / (1.0f + expf(-lg));
                 sc[i] = sg;
-                sel[i] = rank_score(sg + (a.e_bias ? a.e_bias[e] : 0.0f));
+                sel[i] = rank_score(sg + (a.e_bias ? eb[i] : 0.0f));
             }
         }
     }
@@ -154,8 +173,9 @@ __device__ __forceinline__ void select_token(const SelectArgs &a, int t, int lan
     }
     // top-k by repeated warp argmax over the experts not yet taken; k <= E, so
     // every round finds a candidate and bi is always an expert index below E
-    int my_idx[16];
-    float my_val[16];
+    // lane j < k keeps the j-th selected expert and its value (k <= 16)
+    int my_idx = 0;
+    float my_val = 0.0f;
     unsigned taken = 0;      // bit i: expert lane + 32 i already selected
     for (int j = 0; j < a.k; ++j) {
         float bv = -INFINITY;
@@ -169,7 +189,6 @@ __device__ __forceinline__ void select_token(const SelectArgs &a, int t, int lan
             }
         }
         warp_argmax(bv, bi);
-        my_idx[j] = bi;
         float wv = 0.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i)
@@ -177,24 +196,31 @@ __device__ __forceinline__ void select_token(const SelectArgs &a, int t, int lan
                 taken |= 1u << i;                                     // the owner retires the winner
                 wv = a.score_fn == 0 ? lgv[i] : sc[i];               // logit (softmax) or sigmoid score
             }
-        my_val[j] = __shfl_sync(0xffffffffu, wv, bi & 31);
+        const float val = __shfl_sync(0xffffffffu, wv, bi & 31);
+        if (lane == j) {
+            my_idx = bi;
+            my_val = val;
+        }
     }
-    if (lane == 0) {
-        float wsum = 0.0f;
-        float p[16];
-        if (a.score_fn == 0) {
-            const float m = my_val[0];
-            for (int j = 0; j < a.k; ++j) { p[j] = expf(my_val[j] - m); wsum += p[j]; }
-        } else {
-            for (int j = 0; j < a.k; ++j) { p[j] = my_val[j]; wsum += p[j]; }
-        }
-        for (int j = 0; j < a.k; ++j) {
-            const float q = p[j] / wsum;
-            a.topk_idx[(size_t)t * a.k + j] = my_idx[j];
-            a.topk_w[(size_t)t * a.k + j] = a.routed_scale * q;
-            a.topk_p[(size_t)t * a.k + j] = a.score_fn == 0 ? q : my_val[j];
-            if (a.hist) atomicAdd(&a.hist[(size_t)(t / kDispatchChunk) * E + my_idx[j]], 1);
-        }
+    // renormalised weights: softmax over the selected logits (shifted by the
+    // first, the largest) or the selected sigmoid scores; the sum runs in
+    // selection order
+    float p = 0.0f;
+    if (a.score_fn == 0) {
+        const float m = __shfl_sync(0xffffffffu, my_val, 0);
+        if (lane < a.k) p = expf(my_val - m);
+    } else if (lane < a.k) {
+        p = my_val;
+    }
+    float wsum = 0.0f;
+    for (int j = 0; j < a.k; ++j) wsum += __shfl_sync(0xffffffffu, p, j);
+    if (lane < a.k) {
+        const float q = p / wsum;
+        const size_t o = (size_t)t * a.k + lane;
+        a.topk_idx[o] = my_idx;
+        a.topk_w[o] = a.routed_scale * q;
+        a.topk_p[o] = a.score_fn == 0 ? q : my_val;
+        if (a.hist) atomicAdd(&a.hist[(size_t)(t / kDispatchChunk) * E + my_idx], 1);
     }
 }
 
@@ -248,13 +274,13 @@ __global__ void __launch_bounds__(1024) dispatch_count_kernel(const DispatchArgs
     griddep_enter();
     __shared__ int s_cnt[256];
     const int c = blockIdx.x, tid = threadIdx.x;
-    for (int e = tid; e < a.E; e += 1024) s_cnt[e] = 0;
+    for (int e = tid; e < a.E; e += blockDim.x) s_cnt[e] = 0;
     __syncthreads();
     const int t = c * kDispatchChunk + tid;
     if (t < a.T)
         for (int j = 0; j < a.k; ++j) atomicAdd(&s_cnt[checked_expert(a.topk_idx[(size_t)t * a.k + j], a.E, a.status)], 1);
     __syncthreads();
-    for (int e = tid; e < a.E; e += 1024) a.hist[(size_t)c * a.E + e] = s_cnt[e];
+    for (int e = tid; e < a.E; e += blockDim.x) a.hist[(size_t)c * a.E + e] = s_cnt[e];
 }
 
 // One block: counts, exclusive offsets, each chunk's first row per expert (in
@@ -266,8 +292,10 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
     __shared__ int s_off[257];
     const int e = threadIdx.x, E = a.E, T = a.T;
     int total = 0;
-    if (e < E)
+    if (e < E) {
+#pragma unroll 8
         for (int c = 0; c < n_chunks; ++c) total += a.hist[(size_t)c * E + e];
+    }
     s_cnt[e] = e < E ? total : 0;
     __syncthreads();
     if (e == 0) {
@@ -311,15 +339,16 @@ __global__ void __launch_bounds__(256) dispatch_scan_kernel(const DispatchArgs a
 // and the placement; CTA `writer` also writes counts, offsets, the
 // router-gradient chunk starts and the group order.  The placement is the one
 // of dispatch_place_kernel below, with the token of a thread strided by the
-// block size.  s_mask: [256][32] words, s_base / s_cnt: 256 ints each.
+// block size.  s_mask: [256][kMaskWords] words, s_base / s_cnt: 256 ints each.
 __device__ __forceinline__ void dispatch_scan_place_chunk(const DispatchArgs &a, int c, int n_chunks, bool writer,
-                                                          uint32_t (*s_mask)[32], int *s_base, int *s_cnt)
+                                                          uint32_t (*s_mask)[kMaskWords], int *s_base, int *s_cnt)
 {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int E = a.E, k = a.k, kk = a.k + a.S, T = a.T;
-    for (int q = tid; q < E * 32; q += nthr) (&s_mask[0][0])[q] = 0u;
+    for (int q = tid; q < E * kMaskWords; q += nthr) (&s_mask[0][0])[q] = 0u;
     if (tid < E) {
         int total = 0, before = 0;
+#pragma unroll 8
         for (int cc = 0; cc < n_chunks; ++cc) {
             const int h = a.hist[(size_t)cc * E + tid];
             if (cc < c) before += h;
@@ -395,10 +424,10 @@ __device__ __forceinline__ void dispatch_scan_place_chunk(const DispatchArgs &a,
 __global__ void __launch_bounds__(1024) dispatch_place_kernel(const DispatchArgs a)
 {
     griddep_enter();
-    __shared__ uint32_t s_mask[256][32];
+    __shared__ uint32_t s_mask[256][kMaskWords];
     const int c = blockIdx.x, tid = threadIdx.x;
     const int E = a.E, k = a.k, kk = a.k + a.S, T = a.T;
-    for (int q = tid; q < E * 32; q += 1024) (&s_mask[0][0])[q] = 0u;
+    for (int q = tid; q < E * kMaskWords; q += blockDim.x) (&s_mask[0][0])[q] = 0u;
     __syncthreads();
     const int t = c * kDispatchChunk + tid;
     const int word = tid >> 5, bit = tid & 31;
