@@ -175,7 +175,10 @@ __device__ __forceinline__ void fused_stamp(const FusedFwdArgs &a, int point)
 template <bool MX>
 struct FusedCfg {
     using Router = GemmCfg<256, false, false, false, false, false, EPI_ROUTER>;
-    using GateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU, MX>;
+    // BF16 gate/up: 256-row pair tiles (MXFP8 keeps 128-row tiles: its block scales take
+    // TMEM columns); the down GEMM's push epilogue is heavy, so it keeps double-buffered
+    // 128-row tiles
+    using GateUp = GemmCfg<256, false, false, true, false, false, EPI_SWIGLU, MX, !MX>;
     using Down = GemmCfg<256, false, false, false, false, false, EPI_PUSH, MX>;
     static constexpr int cmax(int a, int b) { return a > b ? a : b; }
     static constexpr int RING = cmax(Router::RING_BYTES, cmax(GateUp::RING_BYTES, Down::RING_BYTES));

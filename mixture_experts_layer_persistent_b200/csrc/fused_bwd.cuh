@@ -92,8 +92,11 @@ template <bool N256, bool MX = false>
 struct FusedBwdCfg {
     static_assert(!MX || N256, "the MXFP8 backward takes N = 256 tiles");
     static constexpr int BN = N256 ? 256 : 128;
-    using DgradDown = std::conditional_t<MX, DgradDownMX, GemmCfg<BN, false, true, true, false, false, EPI_DSWIGLU>>;
+    // BF16 data gradients on 256-row pair tiles (at N = 256)
+    using DgradDown =
+        std::conditional_t<MX, DgradDownMX, GemmCfg<BN, false, true, true, false, false, EPI_DSWIGLU, false, N256>>;
     using WgradDown = GemmCfg<BN, true, true, true, false, true, EPI_WGRAD>;
+    // (the push epilogue's fp32 rows are heavy: its GEMM keeps double-buffered 128-row tiles)
     using DgradGU = std::conditional_t<MX, DgradGUMX, GemmCfg<256, false, true, false, false, false, EPI_PUSH>>;
     using WgradGU = GemmCfg<256, true, true, false, true, true, EPI_WGRAD>;
     using ResDown = WgradResCfg<true>;
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
         for (long long b = gtid; b < nb; b += gstride) quantize_block(b, a.dy, a.dyq, a.dys, a.H / 32, 0);
     }
     if (blockIdx.x == 0 && threadIdx.x == 0) {
-        // first M tile of every group in the down dgrad's tiling (readiness counters)
+        // first 128-row M tile of every group (the readiness counters' index)
         int acc = 0;
         for (int g = 0; g <= a.g1.num_groups; ++g) {
             a.mt_base[g] = acc;

@@ -95,15 +95,16 @@ struct GemmArgs {
     int m_per_unit;               // resident weight-gradient kernel: M tiles per work unit
     int *sched;                   // tile counter of this launch, zero before it (one per launch)
     // Per-M-tile readiness between two ragged-M GEMMs of one persistent launch (the
-    // gate/up GEMM produces the rows the down GEMM reads).  Counter of the M tile
-    // (g, mt) = ready[tstart(g) / n_tiles + mt], zero before the producing phase.
+    // gate/up GEMM produces the rows the down GEMM reads).  One counter per 128-row M
+    // tile whatever either GEMM's tile height: counter of the M tile (g, mt) =
+    // ready[(128-row M tiles of the groups before g) + mt], zero before the producing phase.
     int *ready;                   // null: no readiness tracking
     int ready_role;               // kReadySignal: each epilogue warp adds 1 per tile once its stores
                                   // are complete; kReadyWait: the producer waits for ready_target
                                   // before it hands a tile to the other roles
     int ready_target;
-    const int *mt_base;           // kReadyWaitGroup: [G + 1] first M tile of each group in the producing
-                                  // GEMM's tiling (the group's counters are mt_base[g] .. mt_base[g+1]-1)
+    const int *mt_base;           // kReadyWaitGroup: [G + 1] first 128-row M tile of each group (the
+                                  // group's counters are mt_base[g] .. mt_base[g+1]-1)
 };
 
 // kReadyWaitGroup: a weight-gradient phase waits, before it loads a group's rows,
@@ -111,9 +112,17 @@ struct GemmArgs {
 constexpr int kReadyNone = 0, kReadySignal = 1, kReadyWait = 2, kReadyWaitGroup = 3;
 
 template <int BN_, bool A_MN_, bool B_MN_, bool A_GATHER_, bool B_GATHER_, bool RAGGED_K_, int EPI_,
-          bool MX_ = false>
+          bool MX_ = false, bool PAIR_ = false>
 struct GemmCfg {
     static constexpr int BN = BN_;
+    // Pair tiles: 256 rows of a group per tile, as two 128-row halves with their own
+    // accumulator (TMEM columns 0.. and BN..) that share each weight stage.  An
+    // expert of 129-256 rows then streams its weight strip once, in one CTA, whose
+    // tensor core has time to spare while it waits for HBM, instead of a second
+    // CTA running a whole K loop for a few rows.  The two accumulators take all of
+    // TMEM, so a tile's epilogue is not overlapped with the next tile's MMAs.
+    static constexpr bool PAIR = PAIR_;
+    static constexpr int TM = PAIR ? 2 * BM : BM;                // rows per tile
     static constexpr bool A_MN = A_MN_, B_MN = B_MN_, A_GATHER = A_GATHER_, B_GATHER = B_GATHER_;
     static constexpr bool RAGGED_K = RAGGED_K_;
     static constexpr int EPI = EPI_;
@@ -122,7 +131,8 @@ struct GemmCfg {
     static constexpr int KB_ELEMS = 128 / ESIZE;                 // K elements per 128-byte block row
     static constexpr int A_BYTES = BM * 128;
     static constexpr int B_BYTES = BN * 128;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int A_STAGE = (PAIR ? 2 : 1) * A_BYTES;     // A halves, then B, in a stage
+    static constexpr int STAGE_BYTES = A_STAGE + B_BYTES;
     static constexpr int SF_BYTES = MX ? 512 + BN * 4 : 0;       // SFA (128 rows) + SFB (BN rows), 4 bytes each
     // Tuning (measured at the DeepSeek-V3 shape): the weight-streaming kernels
     // want a deep operand ring; BN = 128 and MXFP8 trade a stage for a second
@@ -138,16 +148,16 @@ struct GemmCfg {
     // as soon as its last columns are in registers, before their conversion and stores
     static constexpr bool EARLY_RELEASE = MX;
     static constexpr bool HEAVY_EPI = BN == 256 && ((MX && !MX_SWIGLU) || RAGGED_K);
-    static constexpr int STAGES = HEAVY_EPI ? 3 : (BN == 256 ? 4 : (RAGGED_K ? 6 : 5));
+    static constexpr int STAGES = (HEAVY_EPI || PAIR) ? 3 : (BN == 256 ? 4 : (RAGGED_K ? 6 : 5));
     static constexpr int EPI_BUFS = (HEAVY_EPI || (!RAGGED_K && BN != 256)) ? 2 : 1;
     static constexpr int EPI_WARPS = 4;
     static constexpr int PULL_WARPS = (A_GATHER || B_GATHER || MX) ? kPullWarps : 0;   // cp.async warps
     static constexpr int PULL_WARP0 = 2 + EPI_WARPS;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + PULL_WARPS);
-    static constexpr int GATHER_BYTES = A_GATHER ? A_BYTES : (B_GATHER ? B_BYTES : 0);
+    static constexpr int GATHER_BYTES = A_GATHER ? A_STAGE : (B_GATHER ? B_BYTES : 0);
     // MXFP8: the weight scales of a K block (two 512-byte tiles) come with B
     static constexpr int TMA_BYTES = STAGE_BYTES - GATHER_BYTES + (MX ? 1024 : 0);
-    static constexpr int ACC_BUFS = MX ? 1 : 2;                  // MXFP8 needs TMEM columns for the scales
+    static constexpr int ACC_BUFS = (MX || PAIR) ? 1 : 2;        // MXFP8 needs TMEM columns for the scales
     static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
     static constexpr int SF_TMEM_COL = 256;                      // SFA at 256..259, SFB at 260..
     static constexpr int EPI_STAGE_BYTES = EPI_WARPS * EPI_BUFS * 4096;   // 32 x 128-byte blocks per epilogue warp
@@ -163,6 +173,7 @@ struct GemmCfg {
                           (EPI == EPI_SWIGLU || EPI == EPI_PUSH || EPI == EPI_DSWIGLU)),
                   "MXFP8 serves the K-major expert GEMMs: the forward's and the data gradients'");
     static_assert(BN == 128 || BN == 256, "BN");
+    static_assert(!PAIR || (!MX && !RAGGED_K && !A_MN && BN == 256), "pair tiles: BF16 with a K-major A");
     static_assert(!RAGGED_K || (A_MN && B_MN), "weight gradients take both operands MN-major");
     static_assert(!RAGGED_K || (A_GATHER != B_GATHER), "one operand of a weight gradient is gathered");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -221,14 +232,14 @@ __device__ __forceinline__ Tile decode_tile(int tile, const GemmArgs &a, const i
         // the same time share one weight strip (read from HBM once) while the
         // panel's activation rows stay in L2.
         const int local = tile - s_tstart[lo];
-        const int mtiles = (s_off[lo + 1] - s_off[lo] + BM - 1) / BM;
+        const int mtiles = (s_off[lo + 1] - s_off[lo] + C::TM - 1) / C::TM;
         const int per_panel = kPanelM * a.n_tiles;
         const int pnl = local / per_panel, rem = local - pnl * per_panel;
         const int ps = min(kPanelM, mtiles - pnl * kPanelM);
         t.nt = rem / ps;
         const int mt = pnl * kPanelM + (rem - t.nt * ps);
-        t.m0 = s_off[lo] + mt * BM;
-        t.rows = min(BM, s_off[lo + 1] - t.m0);
+        t.m0 = s_off[lo] + mt * C::TM;
+        t.rows = min(C::TM, s_off[lo + 1] - t.m0);
         t.krow0 = 0;
         t.krows = 0;
         t.nkb = a.num_kb;
@@ -531,20 +542,34 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
         }
         __syncwarp();
         if constexpr (!C::RAGGED_K) {
-            // tile prefix over groups: ceil(rows / BM) * n_tiles tiles each (warp scan)
-            int carry = 0;
+            // tile prefix over groups: ceil(rows / TM) * n_tiles tiles each, and the first
+            // 128-row M tile of each group, which indexes the readiness counters whatever
+            // the tile height (warp scans; the second goes where ragged-K GEMMs keep the
+            // group order)
+            int carry = 0, mcarry = 0;
             for (int base = 0; base < G; base += 32) {
                 const int g = base + lane;
-                int v = 0;
-                if (g < G) v = ((s_off[g + 1] - s_off[g] + BM - 1) / BM) * args.n_tiles;
-                int incl = v;
+                int v = 0, mv = 0;
+                if (g < G) {
+                    v = ((s_off[g + 1] - s_off[g] + C::TM - 1) / C::TM) * args.n_tiles;
+                    mv = (s_off[g + 1] - s_off[g] + BM - 1) / BM;
+                }
+                int incl = v, mincl = mv;
 #pragma unroll
                 for (int d = 1; d < 32; d <<= 1) {
                     const int o = __shfl_up_sync(0xffffffffu, incl, d);
-                    if (lane >= d) incl += o;
+                    const int mo = __shfl_up_sync(0xffffffffu, mincl, d);
+                    if (lane >= d) {
+                        incl += o;
+                        mincl += mo;
+                    }
                 }
-                if (g < G) s_tstart[g] = carry + incl - v;
+                if (g < G) {
+                    s_tstart[g] = carry + incl - v;
+                    s_gorder[g] = mcarry + mincl - mv;
+                }
                 carry += __shfl_sync(0xffffffffu, incl, 31);
+                mcarry += __shfl_sync(0xffffffffu, mincl, 31);
             }
             if (lane == 0) s_tstart[G] = carry;
         }
@@ -602,8 +627,14 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                 if (args.ready_role == kReadyWait && tile < total) {
                     // the rows this tile reads are produced by an earlier phase of the launch
                     const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
-                    const int mt = s_tstart[t.g] / args.n_tiles + (t.m0 - s_off[t.g]) / BM;
-                    if (lane == 0) put = wait_ready(args.ready + mt, args.ready_target, abort_flag, status);
+                    // (s_gorder holds each group's first 128-row M tile here; a pair tile
+                    // needs both of its M tiles)
+                    const int mt = s_gorder[t.g] + (t.m0 - s_off[t.g]) / BM;
+                    if (lane == 0) {
+                        put = wait_ready(args.ready + mt, args.ready_target, abort_flag, status);
+                        if (C::PAIR && put && t.rows > BM)
+                            put = wait_ready(args.ready + mt + 1, args.ready_target, abort_flag, status);
+                    }
                     put = __shfl_sync(0xffffffffu, put, 0);
                     if (!put) tile = total;          // publish "no more work" to the other roles
                 }
@@ -633,7 +664,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) goto producer_done;
                     uint8_t *sA = tiles + stage * C::STAGE_BYTES;
-                    uint8_t *sB = sA + C::A_BYTES;
+                    uint8_t *sB = sA + C::A_STAGE;
                     uint64_t *fb = &full_bar[stage];
                     const int kg = C::EPI == EPI_ROUTER ? t.nt * args.num_kb + kb : kb;   // global K block
                     constexpr int KE = C::KB_ELEMS;
@@ -688,6 +719,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                 tile = __shfl_sync(0xffffffffu, next, 0);
             } else {
                 // lane 0 alone runs the tile's K loop
+                const bool pair2 = C::PAIR && t.rows > BM;           // a pair tile's second half holds rows
                 const int claim_kb = t.nkb > kClaimAhead ? t.nkb - kClaimAhead : 0;
                 int next = 0;
                 bool ok = true;
@@ -698,9 +730,11 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         if (kb == claim_kb) next = static_cast<int>(gridDim.x) + atomicAdd(args.sched, 1);
                         ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag, status);
                         if (!ok) break;
-                        mbar_arrive_expect_tx(&full_bar[stage], C::TMA_BYTES);
+                        // a pair tile whose second half holds no rows loads only the first A half
+                        mbar_arrive_expect_tx(&full_bar[stage],
+                                              C::TMA_BYTES - (C::PAIR && !C::A_GATHER && !pair2 ? C::A_BYTES : 0));
                         uint8_t *sA = tiles + stage * C::STAGE_BYTES;
-                        uint8_t *sB = sA + C::A_BYTES;
+                        uint8_t *sB = sA + C::A_STAGE;
                         uint64_t *fb = &full_bar[stage];
                         const int kg = C::EPI == EPI_ROUTER ? t.nt * args.num_kb + kb : kb;   // global K block
                         constexpr int KE = C::KB_ELEMS;
@@ -708,6 +742,9 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         if constexpr (!C::A_GATHER && !C::A_MN) {
                             const int kc = C::EPI == EPI_ROUTER ? (kg * BK) % args.a_k_mod : kb * KE;
                             tma_load_2d(sA, &tmA, fb, kc, t.m0);
+                            if constexpr (C::PAIR) {
+                                if (pair2) tma_load_2d(sA + C::A_BYTES, &tmA, fb, kc, t.m0 + BM);
+                            }
                         } else if constexpr (!C::A_GATHER && C::A_MN) {
 #pragma unroll
                             for (int c = 0; c < BM / 64; ++c)
@@ -792,11 +829,13 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                 if (tile >= total) break;
                 const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
                 if constexpr (!C::RAGGED_K) {
-                    // K-major A: the tile's 128 rows, this thread's rows r0 + RS i
-                    int tok[BM / RS];
+                    // K-major A: the tile's TM rows, this thread's rows r0 + RS i (a pair
+                    // tile's second half only when it holds rows: the MMA skips it otherwise)
+                    int tok[C::TM / RS];
+                    const int copy_rows = C::PAIR && t.rows > BM ? C::TM : BM;
                     if constexpr (C::A_GATHER) {
 #pragma unroll
-                        for (int i = 0; i < BM / RS; ++i) {
+                        for (int i = 0; i < C::TM / RS; ++i) {
                             const int r = r0 + RS * i;
                             tok[i] = r < t.rows ? __ldg(args.row_token + t.m0 + r) : 0;
                         }
@@ -818,9 +857,10 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         if constexpr (C::A_GATHER) {
                             uint8_t *dst = tiles + stage * C::STAGE_BYTES;
 #pragma unroll
-                            for (int i = 0; i < BM / RS; ++i) {
+                            for (int i = 0; i < C::TM / RS; ++i) {
                                 const int r = r0 + RS * i;
-                                cp_async16(dst + r * 128 + ((c16 ^ (r & 7)) << 4), src + tok[i] * ld + kb * 128 + c16 * 16);
+                                if (C::TM == BM || r < copy_rows)
+                                    cp_async16(dst + r * 128 + ((c16 ^ (r & 7)) << 4), src + tok[i] * ld + kb * 128 + c16 * 16);
                             }
                         }
                         if constexpr (C::MX) {
@@ -842,7 +882,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                     // MN-major operand: 64 gathered K rows per block, this thread's rows r0 + RS i
                     constexpr int CH = (C::A_GATHER ? BM : C::BN) / 64;
                     constexpr int NR = BK / RS;                 // rows per thread and K block
-                    constexpr int OFF = C::A_GATHER ? 0 : C::A_BYTES;
+                    constexpr int OFF = C::A_GATHER ? 0 : C::A_STAGE;
                     const int mn0 = C::A_GATHER ? t.m0 : t.nt * C::BN;
                     const int end = t.krow0 + t.krows;
                     // token rows of K blocks kb, kb+1, kb+2: fetched three blocks ahead so
@@ -912,7 +952,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     uint8_t *sA = tiles + stage * C::STAGE_BYTES;
-                    uint8_t *sB = sA + C::A_BYTES;
+                    uint8_t *sB = sA + C::A_STAGE;
                     if constexpr (C::RAGGED_K) {
                         const int valid = t.krows - kb * BK;
                         if (valid < BK) {
@@ -970,9 +1010,10 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
             } else {
                 // issue K block kb from stage st (lane 0); every lane advances stage / phase
                 // itself, so the warp needs no broadcast of them
+                const bool pair2 = C::PAIR && t.rows > BM;          // a pair tile's second half holds rows
                 auto issue_kb = [&](int kb, int st) {
                     uint8_t *sA = tiles + st * C::STAGE_BYTES;
-                    uint8_t *sB = sA + C::A_BYTES;
+                    uint8_t *sB = sA + C::A_STAGE;
                     if constexpr (C::PULL_WARPS > 0) fence_proxy_async_smem();   // cp.async data -> tensor core
                     const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
                     if constexpr (C::MX) {
@@ -998,6 +1039,19 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                             const uint64_t bd = C::B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024)
                                                         : smem_desc_sw128(b0 + k * 32, 16, 1024);
                             umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | k) != 0 ? 1u : 0u);
+                        }
+                        if constexpr (C::PAIR) {
+                            if (pair2) {
+                                // the second half's rows against the same weight block
+                                const uint32_t a1 = a0 + C::A_BYTES;
+#pragma unroll
+                                for (int k = 0; k < BK / 16; ++k) {
+                                    const uint64_t bd = C::B_MN ? smem_desc_sw128(b0 + k * 2048, 8192, 1024)
+                                                                : smem_desc_sw128(b0 + k * 32, 16, 1024);
+                                    umma_bf16(d_tmem + C::BN, smem_desc_sw128(a1 + k * 32, 16, 1024), bd, C::IDESC,
+                                              (kb | k) != 0 ? 1u : 0u);
+                                }
+                            }
                         }
                     }
                     umma_commit(&empty_bar[st]);
@@ -1053,121 +1107,168 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
         for (int it = 0;; ++it) {
             const int tile = sched_take(sch, it, total, lane, abort_flag, status);
             if (tile >= total) break;
-            const Tile t = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
+            const Tile tt = decode_tile<C>(tile, args, s_off, s_tstart, s_gorder, G);
             if (!mbar_wait(&accf[acc], acc_phase, abort_flag, status)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem_base + static_cast<uint32_t>(acc * C::BN) + (static_cast<uint32_t>(eq * 32) << 16);
-            const bool valid = row < t.rows;
-            const bool full = eq * 32 + 31 < t.rows;        // all 32 rows of this warp's block valid
-            const int row0 = t.m0 + eq * 32;                // first row of the block (ragged-M)
-            if constexpr (C::EPI == EPI_SWIGLU && C::MX) {
-                // h = silu(g) u quantised per 32 columns: e4m3 codes [R, I] and ue8m0 scales [R, I/32]
-                const int r = t.m0 + row;
-                const int I = args.inter;
-                const int n0 = t.nt * 128;
-                uint32_t q[32];
-                uint32_t sc = 0;
-                // the single accumulator is handed back to the MMA warp as soon as its
-                // last columns are in registers: the loads of block b + 1 overlap the
-                // math of block b
-                float gb[2][32], ub[2][32];
-                tmem_ld32(taddr, gb[0]);
-                tmem_ld32(taddr + 128, ub[0]);
-                tmem_ld_wait();
-#pragma unroll
-                for (int blk = 0; blk < 4; ++blk) {
-                    float *g = gb[blk & 1], *u = ub[blk & 1];
-                    if (blk < 3) {
-                        tmem_ld32(taddr + 32 * (blk + 1), gb[(blk + 1) & 1]);
-                        tmem_ld32(taddr + 128 + 32 * (blk + 1), ub[(blk + 1) & 1]);
-                    }
-                    if (args.out2 && valid) {
-                        // training: the gate and up pre-activations as bf16
-                        uint32_t pg[16], pu[16];
-                        pack_bf16<32>(g, pg);
-                        pack_bf16<32>(u, pu);
-                        store_row64(args.out2 + (size_t)r * 2 * I + n0 + 32 * blk, pg);
-                        store_row64(args.out2 + (size_t)r * 2 * I + I + n0 + 32 * blk, pu);
-                    }
-                    float amax = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        g[i] = silu_f(g[i]) * u[i];
-                        amax = fmaxf(amax, fabsf(g[i]));
-                    }
-                    const int e = mx_exponent(amax);
-                    mx_codes32(g, e, q + 8 * blk);
-                    sc |= static_cast<uint32_t>(e + 127) << (8 * blk);
-                    if (args.out_hb && valid) {
-                        // training: the dequantised h (exact in bf16) and w times it, rounded
-                        const float w = args.row_w[r];
-                        uint32_t ph[16], pw[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const uint32_t word = q[8 * blk + (i >> 1)] >> (16 * (i & 1));
-                            const float h0 = mx_decode(word, e), h1 = mx_decode(word >> 8, e);
-                            ph[i] = pack_bf16x2(h0, h1);
-                            pw[i] = pack_bf16x2(w * h0, w * h1);
-                        }
-                        store_row64(args.out_hb + (size_t)r * I + n0 + 32 * blk, ph);
-                        store_row64(args.out3 + (size_t)r * I + n0 + 32 * blk, pw);
-                    }
-                    if (blk < 3) tmem_ld_wait();
-                    if (blk == 2) {
-                        tc_fence_before();
-                        mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
-                    }
+            // a pair tile's halves one after the other (accumulator columns 0.. and BN..)
+            for (int hh = 0; hh < (C::PAIR ? 2 : 1); ++hh) {
+                Tile t = tt;
+                if constexpr (C::PAIR) {
+                    t.m0 = tt.m0 + hh * BM;
+                    t.rows = min(BM, tt.rows - hh * BM);
+                    if (t.rows <= 0) break;
                 }
-                uint8_t *qout = reinterpret_cast<uint8_t *>(args.out);
-                if (full) store_block_tile(stg, q, lane, &tmO, n0, row0);
-                else if (valid) store_row_direct(qout + (size_t)r * I + n0, q);
-                if (valid) *reinterpret_cast<uint32_t *>(args.out_scales + (size_t)r * (I / 32) + t.nt * 4) = sc;
-            } else if constexpr (C::EPI == EPI_SWIGLU) {
-                const int r = t.m0 + row;
-                const int I = args.inter;
-                const int n0 = t.nt * 128;
-                const float w = (valid && args.out3) ? args.row_w[r] : 0.0f;
+                const uint32_t taddr = tmem_base + static_cast<uint32_t>((C::PAIR ? hh : acc) * C::BN) +
+                                       (static_cast<uint32_t>(eq * 32) << 16);
+                const bool valid = row < t.rows;
+                const bool full = eq * 32 + 31 < t.rows;        // all 32 rows of this warp's block valid
+                const int row0 = t.m0 + eq * 32;                // first row of the block (ragged-M)
+                if constexpr (C::EPI == EPI_SWIGLU && C::MX) {
+                    // h = silu(g) u quantised per 32 columns: e4m3 codes [R, I] and ue8m0 scales [R, I/32]
+                    const int r = t.m0 + row;
+                    const int I = args.inter;
+                    const int n0 = t.nt * 128;
+                    uint32_t q[32];
+                    uint32_t sc = 0;
+                    // the single accumulator is handed back to the MMA warp as soon as its
+                    // last columns are in registers: the loads of block b + 1 overlap the
+                    // math of block b
+                    float gb[2][32], ub[2][32];
+                    tmem_ld32(taddr, gb[0]);
+                    tmem_ld32(taddr + 128, ub[0]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int blk = 0; blk < 4; ++blk) {
+                        float *g = gb[blk & 1], *u = ub[blk & 1];
+                        if (blk < 3) {
+                            tmem_ld32(taddr + 32 * (blk + 1), gb[(blk + 1) & 1]);
+                            tmem_ld32(taddr + 128 + 32 * (blk + 1), ub[(blk + 1) & 1]);
+                        }
+                        if (args.out2 && valid) {
+                            // training: the gate and up pre-activations as bf16
+                            uint32_t pg[16], pu[16];
+                            pack_bf16<32>(g, pg);
+                            pack_bf16<32>(u, pu);
+                            store_row64(args.out2 + (size_t)r * 2 * I + n0 + 32 * blk, pg);
+                            store_row64(args.out2 + (size_t)r * 2 * I + I + n0 + 32 * blk, pu);
+                        }
+                        float amax = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            g[i] = silu_f(g[i]) * u[i];
+                            amax = fmaxf(amax, fabsf(g[i]));
+                        }
+                        const int e = mx_exponent(amax);
+                        mx_codes32(g, e, q + 8 * blk);
+                        sc |= static_cast<uint32_t>(e + 127) << (8 * blk);
+                        if (args.out_hb && valid) {
+                            // training: the dequantised h (exact in bf16) and w times it, rounded
+                            const float w = args.row_w[r];
+                            uint32_t ph[16], pw[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                const uint32_t word = q[8 * blk + (i >> 1)] >> (16 * (i & 1));
+                                const float h0 = mx_decode(word, e), h1 = mx_decode(word >> 8, e);
+                                ph[i] = pack_bf16x2(h0, h1);
+                                pw[i] = pack_bf16x2(w * h0, w * h1);
+                            }
+                            store_row64(args.out_hb + (size_t)r * I + n0 + 32 * blk, ph);
+                            store_row64(args.out3 + (size_t)r * I + n0 + 32 * blk, pw);
+                        }
+                        if (blk < 3) tmem_ld_wait();
+                        if (blk == 2) {
+                            tc_fence_before();
+                            mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
+                        }
+                    }
+                    uint8_t *qout = reinterpret_cast<uint8_t *>(args.out);
+                    if (full) store_block_tile(stg, q, lane, &tmO, n0, row0);
+                    else if (valid) store_row_direct(qout + (size_t)r * I + n0, q);
+                    if (valid) *reinterpret_cast<uint32_t *>(args.out_scales + (size_t)r * (I / 32) + t.nt * 4) = sc;
+                } else if constexpr (C::EPI == EPI_SWIGLU) {
+                    const int r = t.m0 + row;
+                    const int I = args.inter;
+                    const int n0 = t.nt * 128;
+                    const float w = (valid && args.out3) ? args.row_w[r] : 0.0f;
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 64) {
-                    uint32_t hp[32], wp[32];
+                    for (int c = 0; c < 128; c += 64) {
+                        uint32_t hp[32], wp[32];
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float g[32], u[32];
-                        tmem_ld32(taddr + c + 32 * half, g);
-                        tmem_ld32(taddr + 128 + c + 32 * half, u);
-                        tmem_ld_wait();
+                        for (int half = 0; half < 2; ++half) {
+                            float g[32], u[32];
+                            tmem_ld32(taddr + c + 32 * half, g);
+                            tmem_ld32(taddr + 128 + c + 32 * half, u);
+                            tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
-                        pack_bf16<32>(g, hp + 16 * half);
+                            for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];
+                            pack_bf16<32>(g, hp + 16 * half);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) g[i] = w * bf16_round(g[i]);
-                        pack_bf16<32>(g, wp + 16 * half);
+                            for (int i = 0; i < 32; ++i) g[i] = w * bf16_round(g[i]);
+                            pack_bf16<32>(g, wp + 16 * half);
+                        }
+                        if (full) store_block_tile(stg, hp, lane, &tmO, n0 + c, row0);
+                        else if (valid) store_row_direct(args.out + (size_t)r * I + n0 + c, hp);
+                        if (args.out3) {
+                            if (full) store_block_tile(stg, wp, lane, &tmO3, n0 + c, row0);
+                            else if (valid) store_row_direct(args.out3 + (size_t)r * I + n0 + c, wp);
+                        }
+                        if (args.out2) {
+#pragma unroll
+                            for (int part = 0; part < 2; ++part) {       // gate, then up pre-activations
+                                float v[64];
+                                uint32_t p[32];
+                                tmem_ld32(taddr + 128 * part + c, *reinterpret_cast<float(*)[32]>(v));
+                                tmem_ld32(taddr + 128 * part + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                                tmem_ld_wait();
+                                pack_bf16<64>(v, p);
+                                const int col = part * I + n0 + c;
+                                if (full) store_block_tile(stg, p, lane, &tmO2, col, row0);
+                                else if (valid) store_row_direct(args.out2 + (size_t)r * 2 * I + col, p);
+                            }
+                        }
                     }
-                    if (full) store_block_tile(stg, hp, lane, &tmO, n0 + c, row0);
-                    else if (valid) store_row_direct(args.out + (size_t)r * I + n0 + c, hp);
-                    if (args.out3) {
-                        if (full) store_block_tile(stg, wp, lane, &tmO3, n0 + c, row0);
-                        else if (valid) store_row_direct(args.out3 + (size_t)r * I + n0 + c, wp);
-                    }
-                    if (args.out2) {
+                } else if constexpr (C::EPI == EPI_PUSH && C::MX) {
+                    const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
+                    if (args.out_f32) {
+                        // MXFP8 gate/up dgrad: fp32 rows pushed into their (token, slot) row
+                        float *dst = args.out_f32 + (size_t)dst_row * args.ldo + t.nt * C::BN;
+#pragma unroll 1
+                        for (int c = 0; c < C::BN; c += 32) {
+                            float v[32];
+                            uint32_t p[32];
+                            tmem_ld32(taddr + c, v);
+                            tmem_ld_wait();
+                            if (c == C::BN - 32) {
+                                tc_fence_before();
+                                mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
+                            }
 #pragma unroll
-                        for (int part = 0; part < 2; ++part) {       // gate, then up pre-activations
+                            for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
+                            if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
+                            else if (valid) store_row_direct(dst + c, p);
+                        }
+                    } else {
+                        // MXFP8 forward: bf16 rows pushed into their (token, slot) row
+                        __nv_bfloat16 *dst = args.out + (size_t)dst_row * args.ldo + t.nt * C::BN;
+#pragma unroll 1
+                        for (int c = 0; c < C::BN; c += 64) {
                             float v[64];
                             uint32_t p[32];
-                            tmem_ld32(taddr + 128 * part + c, *reinterpret_cast<float(*)[32]>(v));
-                            tmem_ld32(taddr + 128 * part + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                            tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
+                            tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
                             tmem_ld_wait();
+                            if (c == C::BN - 64) {
+                                tc_fence_before();
+                                mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
+                            }
                             pack_bf16<64>(v, p);
-                            const int col = part * I + n0 + c;
-                            if (full) store_block_tile(stg, p, lane, &tmO2, col, row0);
-                            else if (valid) store_row_direct(args.out2 + (size_t)r * 2 * I + col, p);
+                            if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
+                            else if (valid) store_row_direct(dst + c, p);
                         }
                     }
-                }
-            } else if constexpr (C::EPI == EPI_PUSH && C::MX) {
-                const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
-                if (args.out_f32) {
-                    // MXFP8 gate/up dgrad: fp32 rows pushed into their (token, slot) row
+                } else if constexpr (C::EPI == EPI_PUSH) {
+                    // fp32 rows pushed into their (token, slot) row of the slot buffer
+                    const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
                     float *dst = args.out_f32 + (size_t)dst_row * args.ldo + t.nt * C::BN;
 #pragma unroll 1
                     for (int c = 0; c < C::BN; c += 32) {
@@ -1175,151 +1276,114 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         uint32_t p[32];
                         tmem_ld32(taddr + c, v);
                         tmem_ld_wait();
-                        if (c == C::BN - 32) {
-                            tc_fence_before();
-                            mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
-                        }
 #pragma unroll
                         for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
                         if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
                         else if (valid) store_row_direct(dst + c, p);
                     }
-                } else {
-                    // MXFP8 forward: bf16 rows pushed into their (token, slot) row
-                    __nv_bfloat16 *dst = args.out + (size_t)dst_row * args.ldo + t.nt * C::BN;
+                } else if constexpr (C::EPI == EPI_WGRAD) {
+                    const bool routed = t.g < args.num_routed;
+                    const int gl = routed ? t.g : t.g - args.num_routed;
+                    const int grow0 = gl * args.m_tiles * BM + t.m0 + eq * 32;   // row in the [groups * M, N] view
+                    constexpr int COLS = C::BN * 4 / C::EPI_WARPS;               // columns of this warp
+                    const int c0 = (ew >> 2) * COLS;
+                    float v[64];
+                    if (t.nkb > 0) {
+                        tmem_ld32(taddr + c0, *reinterpret_cast<float(*)[32]>(v));
+                        tmem_ld32(taddr + c0 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                        tmem_ld_wait();
+                    }
+#pragma unroll 1
+                    for (int c = c0; c < c0 + COLS; c += 64) {
+                        uint32_t p[32];
+                        if (t.nkb > 0) {
+                            pack_bf16<64>(v, p);
+                            if (c + 64 < c0 + COLS) {          // next block's TMEM load overlaps this block's store
+                                tmem_ld32(taddr + c + 64, *reinterpret_cast<float(*)[32]>(v));
+                                tmem_ld32(taddr + c + 96, *reinterpret_cast<float(*)[32]>(v + 32));
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) p[i] = 0u;
+                        }
+                        store_block_tile(stg, p, lane, routed ? &tmO : &tmO2, t.nt * C::BN + c, grow0);
+                        if (t.nkb > 0 && c + 64 < c0 + COLS) tmem_ld_wait();
+                    }
+                } else if constexpr (C::EPI == EPI_DSWIGLU) {
+                    const int r = t.m0 + row;
+                    const int I = args.inter;
+                    const int n0 = t.nt * C::BN;
+                    const float w = valid ? args.row_w[r] : 0.0f;
+                    const __nv_bfloat16 *gsrc = valid ? args.aux + (size_t)r * 2 * I + n0 : nullptr;
+                    // slot gradient of a routed row: G = <dy, o> = <dy W_down, h>, summed here over
+                    // this tile's columns (v before the routing weight) against the saved h
+                    const bool routed_row = valid && t.g < args.num_routed;
+                    const __nv_bfloat16 *hsrc = routed_row ? args.aux_h + (size_t)r * I + n0 : nullptr;
+                    float gsum = 0.0f;
 #pragma unroll 1
                     for (int c = 0; c < C::BN; c += 64) {
-                        float v[64];
+                        uint32_t gp[32], up[32], dgp[32], dup[32], hp[32];
+                        load_row_direct(gp, gsrc ? gsrc + c : nullptr);
+                        load_row_direct(up, gsrc ? gsrc + I + c : nullptr);
+                        load_row_direct(hp, hsrc ? hsrc + c : nullptr);
+#pragma unroll
+                        for (int half = 0; half < 2; ++half) {
+                            float v[32], dg[32], du[32];
+                            tmem_ld32(taddr + c + 32 * half, v);
+                            tmem_ld_wait();
+                            if constexpr (C::EARLY_RELEASE) {
+                                if (c == C::BN - 64 && half == 1) {
+                                    tc_fence_before();
+                                    mbar_arrive(&acce[acc]);     // every column of the accumulator is in registers
+                                }
+                            }
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) {
+                                const uint32_t gw = gp[16 * half + (i >> 1)], uw = up[16 * half + (i >> 1)];
+                                const uint32_t hw = hp[16 * half + (i >> 1)];
+                                const float gi = (i & 1) ? bf16_hi(gw) : bf16_lo(gw);
+                                const float ui = (i & 1) ? bf16_hi(uw) : bf16_lo(uw);
+                                gsum = fmaf(v[i], (i & 1) ? bf16_hi(hw) : bf16_lo(hw), gsum);
+                                const float dh = w * v[i];
+                                const float sg = sigmoid_f(gi);
+                                dg[i] = dh * ui * sg * (1.0f + gi * (1.0f - sg));
+                                du[i] = dh * gi * sg;
+                            }
+                            pack_bf16<32>(dg, dgp + 16 * half);
+                            pack_bf16<32>(du, dup + 16 * half);
+                            if constexpr (C::MX) {
+                                // MXFP8 backward: dGU quantised per 1x32 block (from fp32) for the gate/up dgrad
+                                if (valid) {
+                                    const int cg = n0 + c + 32 * half;
+                                    mx_store_block(dg, args.out_q + (size_t)r * 2 * I + cg,
+                                                   args.out_scales + (size_t)r * (2 * I / 32) + cg / 32);
+                                    mx_store_block(du, args.out_q + (size_t)r * 2 * I + I + cg,
+                                                   args.out_scales + (size_t)r * (2 * I / 32) + (I + cg) / 32);
+                                }
+                            }
+                        }
+                        if (full) {
+                            store_block_tile(stg, dgp, lane, &tmO, n0 + c, row0);
+                            store_block_tile(stg, dup, lane, &tmO, I + n0 + c, row0);
+                        } else if (valid) {
+                            store_row_direct(args.out + (size_t)r * 2 * I + n0 + c, dgp);
+                            store_row_direct(args.out + (size_t)r * 2 * I + I + n0 + c, dup);
+                        }
+                    }
+                    if (routed_row) args.gpart[(size_t)r * args.n_tiles + t.nt] = gsum;
+                } else {   // EPI_ROUTER: fp32 partial logits of this K split
+                    const int r = t.m0 + row;
+#pragma unroll 1
+                    for (int c = 0; c < 256; c += 32) {
+                        float v[32];
                         uint32_t p[32];
-                        tmem_ld32(taddr + c, *reinterpret_cast<float(*)[32]>(v));
-                        tmem_ld32(taddr + c + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+                        tmem_ld32(taddr + c, v);
                         tmem_ld_wait();
-                        if (c == C::BN - 64) {
-                            tc_fence_before();
-                            mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
-                        }
-                        pack_bf16<64>(v, p);
-                        if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
-                        else if (valid) store_row_direct(dst + c, p);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
+                        if (full) store_block_tile(stg, p, lane, &tmO, c, t.nt * args.rows_total + row0);
+                        else if (valid) store_row_direct(args.out_f32 + ((size_t)t.nt * args.rows_total + r) * 256 + c, p);
                     }
-                }
-            } else if constexpr (C::EPI == EPI_PUSH) {
-                // fp32 rows pushed into their (token, slot) row of the slot buffer
-                const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
-                float *dst = args.out_f32 + (size_t)dst_row * args.ldo + t.nt * C::BN;
-#pragma unroll 1
-                for (int c = 0; c < C::BN; c += 32) {
-                    float v[32];
-                    uint32_t p[32];
-                    tmem_ld32(taddr + c, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
-                    if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
-                    else if (valid) store_row_direct(dst + c, p);
-                }
-            } else if constexpr (C::EPI == EPI_WGRAD) {
-                const bool routed = t.g < args.num_routed;
-                const int gl = routed ? t.g : t.g - args.num_routed;
-                const int grow0 = gl * args.m_tiles * BM + t.m0 + eq * 32;   // row in the [groups * M, N] view
-                constexpr int COLS = C::BN * 4 / C::EPI_WARPS;               // columns of this warp
-                const int c0 = (ew >> 2) * COLS;
-                float v[64];
-                if (t.nkb > 0) {
-                    tmem_ld32(taddr + c0, *reinterpret_cast<float(*)[32]>(v));
-                    tmem_ld32(taddr + c0 + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-                    tmem_ld_wait();
-                }
-#pragma unroll 1
-                for (int c = c0; c < c0 + COLS; c += 64) {
-                    uint32_t p[32];
-                    if (t.nkb > 0) {
-                        pack_bf16<64>(v, p);
-                        if (c + 64 < c0 + COLS) {          // next block's TMEM load overlaps this block's store
-                            tmem_ld32(taddr + c + 64, *reinterpret_cast<float(*)[32]>(v));
-                            tmem_ld32(taddr + c + 96, *reinterpret_cast<float(*)[32]>(v + 32));
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) p[i] = 0u;
-                    }
-                    store_block_tile(stg, p, lane, routed ? &tmO : &tmO2, t.nt * C::BN + c, grow0);
-                    if (t.nkb > 0 && c + 64 < c0 + COLS) tmem_ld_wait();
-                }
-            } else if constexpr (C::EPI == EPI_DSWIGLU) {
-                const int r = t.m0 + row;
-                const int I = args.inter;
-                const int n0 = t.nt * C::BN;
-                const float w = valid ? args.row_w[r] : 0.0f;
-                const __nv_bfloat16 *gsrc = valid ? args.aux + (size_t)r * 2 * I + n0 : nullptr;
-                // slot gradient of a routed row: G = <dy, o> = <dy W_down, h>, summed here over
-                // this tile's columns (v before the routing weight) against the saved h
-                const bool routed_row = valid && t.g < args.num_routed;
-                const __nv_bfloat16 *hsrc = routed_row ? args.aux_h + (size_t)r * I + n0 : nullptr;
-                float gsum = 0.0f;
-#pragma unroll 1
-                for (int c = 0; c < C::BN; c += 64) {
-                    uint32_t gp[32], up[32], dgp[32], dup[32], hp[32];
-                    load_row_direct(gp, gsrc ? gsrc + c : nullptr);
-                    load_row_direct(up, gsrc ? gsrc + I + c : nullptr);
-                    load_row_direct(hp, hsrc ? hsrc + c : nullptr);
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float v[32], dg[32], du[32];
-                        tmem_ld32(taddr + c + 32 * half, v);
-                        tmem_ld_wait();
-                        if constexpr (C::EARLY_RELEASE) {
-                            if (c == C::BN - 64 && half == 1) {
-                                tc_fence_before();
-                                mbar_arrive(&acce[acc]);     // every column of the accumulator is in registers
-                            }
-                        }
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const uint32_t gw = gp[16 * half + (i >> 1)], uw = up[16 * half + (i >> 1)];
-                            const uint32_t hw = hp[16 * half + (i >> 1)];
-                            const float gi = (i & 1) ? bf16_hi(gw) : bf16_lo(gw);
-                            const float ui = (i & 1) ? bf16_hi(uw) : bf16_lo(uw);
-                            gsum = fmaf(v[i], (i & 1) ? bf16_hi(hw) : bf16_lo(hw), gsum);
-                            const float dh = w * v[i];
-                            const float sg = sigmoid_f(gi);
-                            dg[i] = dh * ui * sg * (1.0f + gi * (1.0f - sg));
-                            du[i] = dh * gi * sg;
-                        }
-                        pack_bf16<32>(dg, dgp + 16 * half);
-                        pack_bf16<32>(du, dup + 16 * half);
-                        if constexpr (C::MX) {
-                            // MXFP8 backward: dGU quantised per 1x32 block (from fp32) for the gate/up dgrad
-                            if (valid) {
-                                const int cg = n0 + c + 32 * half;
-                                mx_store_block(dg, args.out_q + (size_t)r * 2 * I + cg,
-                                               args.out_scales + (size_t)r * (2 * I / 32) + cg / 32);
-                                mx_store_block(du, args.out_q + (size_t)r * 2 * I + I + cg,
-                                               args.out_scales + (size_t)r * (2 * I / 32) + (I + cg) / 32);
-                            }
-                        }
-                    }
-                    if (full) {
-                        store_block_tile(stg, dgp, lane, &tmO, n0 + c, row0);
-                        store_block_tile(stg, dup, lane, &tmO, I + n0 + c, row0);
-                    } else if (valid) {
-                        store_row_direct(args.out + (size_t)r * 2 * I + n0 + c, dgp);
-                        store_row_direct(args.out + (size_t)r * 2 * I + I + n0 + c, dup);
-                    }
-                }
-                if (routed_row) args.gpart[(size_t)r * args.n_tiles + t.nt] = gsum;
-            } else {   // EPI_ROUTER: fp32 partial logits of this K split
-                const int r = t.m0 + row;
-#pragma unroll 1
-                for (int c = 0; c < 256; c += 32) {
-                    float v[32];
-                    uint32_t p[32];
-                    tmem_ld32(taddr + c, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
-                    if (full) store_block_tile(stg, p, lane, &tmO, c, t.nt * args.rows_total + row0);
-                    else if (valid) store_row_direct(args.out_f32 + ((size_t)t.nt * args.rows_total + r) * 256 + c, p);
                 }
             }
             if constexpr (!C::EARLY_RELEASE) {
@@ -1327,8 +1391,13 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                 mbar_arrive(&acce[acc]);
             }
             if constexpr (!C::RAGGED_K) {
-                if (args.ready_role == kReadySignal)
-                    signal_ready(args.ready + s_tstart[t.g] / args.n_tiles + (t.m0 - s_off[t.g]) / BM, lane);
+                // one counter per 128-row M tile (s_gorder holds each group's first one);
+                // a pair tile signals both of its M tiles once both halves are stored
+                if (args.ready_role == kReadySignal) {
+                    const int mt = s_gorder[tt.g] + (tt.m0 - s_off[tt.g]) / BM;
+                    signal_ready(args.ready + mt, lane);
+                    if (C::PAIR && tt.rows > BM) signal_ready(args.ready + mt + 1, lane);
+                }
             }
             if (++acc == C::ACC_BUFS) {
                 acc = 0;
