@@ -32,7 +32,7 @@
 
 namespace mok {
 
-constexpr int kResidentRows = 256;
+constexpr int kResidentRows = 192;
 
 template <bool A_GATHER_>
 struct WgradResCfg {
@@ -45,7 +45,7 @@ struct WgradResCfg {
     static constexpr int B_BYTES = KB_MAX * B_KB_BYTES;
     static constexpr int STAGES = 4;
     static constexpr int EPI_WARPS = 4;                      // 4 or 8 (two per TMEM lane quarter)
-    static constexpr int EPI_BUFS = 2;
+    static constexpr int EPI_BUFS = 4;
     static constexpr int PULL_WARPS = kPullWarps;
     static constexpr int PULL_WARP0 = 2 + EPI_WARPS;
     static constexpr int THREADS = 64 + 32 * (EPI_WARPS + PULL_WARPS);
