@@ -61,7 +61,7 @@ WORKLOADS = {
     "dsv3_e16_r128": Workload("dsv3_e16_r128", T=256, H=7168, E=16, k=8, I=2048, S=1, Is=2048,
                               score_fn=1, n_group=8, topk_group=4, seed=8),
     # the same with 512 rows per expert (the mean load of the skewed workload): every group
-    # exceeds 256 rows, so the streaming weight-gradient kernel does all the work
+    # exceeds the resident kernel's 192 rows, so the streaming weight-gradient kernel does all the work
     "dsv3_e16_r512": Workload("dsv3_e16_r512", T=1024, H=7168, E=16, k=8, I=2048, S=1, Is=2048,
                               score_fn=1, n_group=8, topk_group=4, seed=10),
     # the MXFP8 forward of the same shape with 256 rows per routed expert (as dsv3_mxfp8)

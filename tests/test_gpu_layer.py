@@ -19,10 +19,11 @@ MEDIUM_SIGMOID = synth.Workload("medium_sigmoid", T=700, H=512, E=16, k=4, I=256
                                 score_fn=1, n_group=4, topk_group=2, seed=11)
 MEDIUM_SOFTMAX = synth.Workload("medium_softmax", T=333, H=768, E=12, k=3, I=384, S=2, Is=384,
                                 seed=12)
-# skewed routing: groups on both sides of the 256-row split between the resident and the
-# streaming weight-gradient kernels (one of exactly 256 rows), and empty groups
+# skewed routing: groups on both sides of the 192-row split between the resident and the
+# streaming weight-gradient kernels (one of exactly 192 rows), and an empty group
+RESIDENT_ROWS = 192
 MEDIUM_ZIPF = synth.Workload("medium_zipf", T=900, H=512, E=16, k=4, I=256, S=1, Is=256, score_fn=1,
-                             n_group=4, topk_group=2, zipf=1.5, seed=13)
+                             n_group=4, topk_group=2, zipf=1.5, seed=142)
 MEDIUM_ZIPF_SPARSE = synth.scaled(MEDIUM_ZIPF, name="medium_zipf_sparse", zipf=3.5)
 CASES = [synth.WORKLOADS["tiny"], MEDIUM_SIGMOID, MEDIUM_SOFTMAX, MEDIUM_ZIPF, MEDIUM_ZIPF_SPARSE]
 
@@ -74,7 +75,7 @@ def test_backward_matches_oracle(ran):
     assert_close(to_np(grads["drouter_w"]), dwr, "drouter_w")
     counts = np.bincount(idx.ravel(), minlength=wl.E)
     experts = {0, wl.E - 1, int(np.argmax(counts)), int(np.argmin(counts))}
-    small, large = np.flatnonzero(counts <= 256), np.flatnonzero(counts > 256)
+    small, large = np.flatnonzero(counts <= RESIDENT_ROWS), np.flatnonzero(counts > RESIDENT_ROWS)
     if small.size:
         experts.add(int(small[np.argmax(counts[small])]))     # largest group of the resident kernel
     if large.size:
