@@ -230,6 +230,34 @@ int moe_step_host(const moe_cfg *cfg, const void *x_host, const void *dy_host, c
                   void *scratch, size_t scratch_bytes, void *stream);
 
 /*
+ * Pipelined training steps through host buffers: the same step as moe_step_host
+ * (same results, byte for byte), enqueued without waiting, so that consecutive
+ * calls on one stream overlap every transfer with the passes.  Each call:
+ *   - takes x from the device x slot of this call when the previous call
+ *     uploaded x_host there (its x_next_host), else uploads it first;
+ *   - uploads dy on the library's upload stream (once the previous step's
+ *     backward has read the device copy) while the forward runs;
+ *   - downloads y on the library's download stream while the backward runs, and
+ *     uploads x_next_host (NULL: none) into the other x slot meanwhile;
+ *   - downloads dx (two device dx slots) while the next step runs.
+ * Arguments as moe_step_host; scratch: at least moe_host_scratch_size(cfg, 3, ...)
+ * bytes (two x slots, y, dy, two dx slots, the backward's workspace), the same
+ * buffer for every call of a sequence (another buffer starts a new sequence).
+ * The host buffers x_host, x_next_host, dy_host must stay unchanged, and
+ * y_host, dx_host must not be read, until moe_step_host_sync returns; the
+ * weight and router gradients in `grads` (device) are overwritten by every
+ * call, in stream order.  On an error every stream of the sequence is drained
+ * before the call returns.  The two streams (per host thread and device) are
+ * created on first use and kept.
+ */
+int moe_step_host_async(const moe_cfg *cfg, const void *x_host, const void *x_next_host, const void *dy_host,
+                        const moe_params *params, void *y_host, void *dx_host, void *ctx, size_t ctx_bytes,
+                        const moe_grads *grads, void *scratch, size_t scratch_bytes, void *stream);
+/* Waits until every step enqueued by moe_step_host_async on this host thread, and
+ * `stream`, have completed (all of their transfers included). */
+int moe_step_host_sync(void *stream);
+
+/*
  * MXFP8 quantisation along the last axis: src [rows, K] bf16 (device) ->
  * q [rows, K] e4m3 codes and scales [rows, K/32] ue8m0 (device).  Per block of
  * 32 consecutive elements the exponent e is the smallest integer with

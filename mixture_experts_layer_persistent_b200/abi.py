@@ -90,6 +90,9 @@ def lib():
                                    _vp, _sz, _vp]
         L.moe_step_host.argtypes = [P(moe_cfg), _vp, _vp, P(moe_params), _vp, _vp, _vp, _sz, P(moe_grads), _vp,
                                     _sz, _vp]
+        L.moe_step_host_async.argtypes = [P(moe_cfg), _vp, _vp, _vp, P(moe_params), _vp, _vp, _vp, _sz,
+                                          P(moe_grads), _vp, _sz, _vp]
+        L.moe_step_host_sync.argtypes = [_vp]
         L.moe_quantize_mxfp8.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
         L.moe_quantize_mxfp8_weights.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, _vp, _vp, _vp]
         L.moe_quantize_mxfp8_weights_t.argtypes = [_vp, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, _vp, _vp,
@@ -110,7 +113,8 @@ def lib():
         L.moe_last_error.argtypes = []
         L.moe_last_error.restype = ctypes.c_char_p
         for name in ("moe_workspace_size", "moe_fwd", "moe_bwd", "moe_host_scratch_size",
-                     "moe_fwd_host", "moe_bwd_host", "moe_step_host", "moe_quantize_mxfp8", "moe_quantize_mxfp8_weights",
+                     "moe_fwd_host", "moe_bwd_host", "moe_step_host", "moe_step_host_async", "moe_step_host_sync",
+                     "moe_quantize_mxfp8", "moe_quantize_mxfp8_weights",
                      "moe_quantize_mxfp8_weights_t", "moe_quantize_mxfp8_weights_both", "moe_status",
                      "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal", "moe_saved_tensor",
                      "moe_set_schedule", "moe_get_schedule", "moe_trace_device"):
@@ -158,7 +162,7 @@ def moe_saved_tensor(cfg: moe_cfg, save_for_backward: bool, which: int):
 
 
 def moe_host_scratch_size(cfg: moe_cfg, backward) -> int:
-    """backward: False (moe_fwd_host), True (moe_bwd_host) or 2 (moe_step_host)."""
+    """backward: False (moe_fwd_host), True (moe_bwd_host), 2 (moe_step_host) or 3 (moe_step_host_async)."""
     n = _sz()
     _check("moe_host_scratch_size", lib().moe_host_scratch_size(ctypes.byref(cfg), int(backward),
                                                                 ctypes.byref(n)))
@@ -198,6 +202,17 @@ def moe_step_host(cfg, x_host, dy_host, params, y_host, dx_host, ctx, ctx_bytes,
     _check("moe_step_host", lib().moe_step_host(ctypes.byref(cfg), x_host, dy_host, ctypes.byref(params), y_host,
                                                 dx_host, ctx, ctx_bytes, ctypes.byref(grads), scratch, scratch_bytes,
                                                 stream))
+
+
+def moe_step_host_async(cfg, x_host, x_next_host, dy_host, params, y_host, dx_host, ctx, ctx_bytes, grads, scratch,
+                        scratch_bytes, stream):
+    _check("moe_step_host_async", lib().moe_step_host_async(ctypes.byref(cfg), x_host, x_next_host, dy_host,
+                                                            ctypes.byref(params), y_host, dx_host, ctx, ctx_bytes,
+                                                            ctypes.byref(grads), scratch, scratch_bytes, stream))
+
+
+def moe_step_host_sync(stream):
+    _check("moe_step_host_sync", lib().moe_step_host_sync(stream))
 
 
 def moe_quantize_mxfp8(src, rows, K, q, scales, stream):

@@ -1088,7 +1088,7 @@ int moe_host_scratch_size(const moe_cfg *cfg, int backward, size_t *bytes)
     MOK_TRY(check_cfg(cfg));
     const size_t io = align_up(static_cast<size_t>(cfg->T) * cfg->H * 2, 256);
     size_t inner = backward ? carve_bwd(*cfg, nullptr).bytes : carve_state(*cfg, nullptr, false).bytes;
-    if (bytes) *bytes = (backward == 2 ? 4 : backward ? 3 : 2) * io + inner;
+    if (bytes) *bytes = (backward == 3 ? 6 : backward == 2 ? 4 : backward ? 3 : 2) * io + inner;
     return MOK_OK;
 }
 
@@ -1146,6 +1146,49 @@ struct StepStreams {
     cudaEvent_t start = nullptr, dy_in = nullptr, y_ready = nullptr, y_out = nullptr;
 };
 thread_local StepStreams t_step;
+
+// Pipelined host steps (moe_step_host_async): an upload and a download stream per
+// host thread and device, the events that order them with the caller's stream,
+// and which host x each of the two device x slots holds.
+struct PipeStreams {
+    int device = -1;
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t fwd_done = nullptr, bwd_done = nullptr, dy_in = nullptr, y_out = nullptr;
+    cudaEvent_t x_ready[2] = {nullptr, nullptr}, dx_out[2] = {nullptr, nullptr};
+    const void *scratch = nullptr;      // the scratch buffer of the calls in flight
+    const void *slot_x[2] = {nullptr, nullptr};   // host x uploaded (or on its way) into each slot
+    unsigned long long calls = 0;
+};
+thread_local PipeStreams t_pipe;
+
+int pipe_streams(PipeStreams *&ps)
+{
+    int dev = 0;
+    if (const cudaError_t e = cudaGetDevice(&dev); e != cudaSuccess) return fail(MOK_ERR_DEVICE, "cudaGetDevice", e);
+    ps = &t_pipe;
+    if (ps->device == dev) return MOK_OK;
+    if (ps->up) {                   // another device: release the old handles first
+        cudaStreamSynchronize(ps->up);
+        cudaStreamSynchronize(ps->down);
+        cudaStreamDestroy(ps->up);
+        cudaStreamDestroy(ps->down);
+        cudaEvent_t evs[] = {ps->fwd_done, ps->bwd_done, ps->dy_in, ps->y_out, ps->x_ready[0], ps->x_ready[1],
+                             ps->dx_out[0], ps->dx_out[1]};
+        for (cudaEvent_t ev : evs) cudaEventDestroy(ev);
+        *ps = PipeStreams{};
+    }
+    if (const cudaError_t e = cudaStreamCreateWithFlags(&ps->up, cudaStreamNonBlocking); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaStreamCreateWithFlags", e);
+    if (const cudaError_t e = cudaStreamCreateWithFlags(&ps->down, cudaStreamNonBlocking); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaStreamCreateWithFlags", e);
+    cudaEvent_t *evs[] = {&ps->fwd_done, &ps->bwd_done, &ps->dy_in, &ps->y_out, &ps->x_ready[0], &ps->x_ready[1],
+                          &ps->dx_out[0], &ps->dx_out[1]};
+    for (cudaEvent_t *ev : evs)
+        if (const cudaError_t e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming); e != cudaSuccess)
+            return fail(MOK_ERR_LAUNCH, "cudaEventCreateWithFlags", e);
+    ps->device = dev;
+    return MOK_OK;
+}
 
 int step_streams(StepStreams *&ss)
 {
@@ -1225,6 +1268,104 @@ done:
         rc = fail(MOK_ERR_LAUNCH, "cudaStreamSynchronize(side)", e2);
     if (const cudaError_t e2 = cudaStreamSynchronize(st); e2 != cudaSuccess && rc == MOK_OK)
         rc = fail(MOK_ERR_LAUNCH, "cudaStreamSynchronize", e2);
+    return rc;
+}
+
+int moe_step_host_async(const moe_cfg *cfg, const void *x_host, const void *x_next_host, const void *dy_host,
+                        const moe_params *params, void *y_host, void *dx_host, void *ctx, size_t ctx_bytes,
+                        const moe_grads *grads, void *scratch, size_t scratch_bytes, void *stream)
+{
+    MOK_TRY(check_cfg(cfg));
+    if (!x_host || !dy_host || !y_host || !dx_host || !scratch || !grads) return MOK_ERR_INVALID;
+    size_t need = 0;
+    moe_host_scratch_size(cfg, 3, &need);
+    if (scratch_bytes < need) return MOK_ERR_WORKSPACE;
+    if (!device_info()) return MOK_ERR_DEVICE;
+    PipeStreams *ps = nullptr;
+    MOK_TRY(pipe_streams(ps));
+    if (ps->scratch != scratch) {       // a new sequence: nothing of this buffer is prefetched
+        ps->scratch = scratch;
+        ps->slot_x[0] = ps->slot_x[1] = nullptr;
+        ps->calls = 0;
+    }
+    const int p = static_cast<int>(ps->calls & 1u);
+    const size_t io = align_up(static_cast<size_t>(cfg->T) * cfg->H * 2, 256);
+    const size_t nb = static_cast<size_t>(cfg->T) * cfg->H * 2;
+    char *s = static_cast<char *>(scratch);
+    char *xs[2] = {s, s + io}, *y = s + 2 * io, *dy = s + 3 * io, *dxs[2] = {s + 4 * io, s + 5 * io};
+    char *inner = s + 6 * io;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    int rc = MOK_OK;
+#define PIPE_CUDA(call, what)                                      \
+    if ((e = (call)) != cudaSuccess) {                             \
+        rc = fail(MOK_ERR_LAUNCH, what, e);                        \
+        goto fail_sync;                                            \
+    }
+    // x of this step in slot p: prefetched by the previous call, or uploaded now (after
+    // any prefetch still landing in that slot)
+    PIPE_CUDA(cudaStreamWaitEvent(st, ps->x_ready[p], 0), "cudaStreamWaitEvent");
+    if (ps->slot_x[p] != x_host) {
+        PIPE_CUDA(cudaMemcpyAsync(xs[p], x_host, nb, cudaMemcpyHostToDevice, st), "cudaMemcpyAsync(x)");
+        ps->slot_x[p] = x_host;
+    }
+    // dy on the upload stream once the previous step's backward has read the buffer
+    PIPE_CUDA(cudaStreamWaitEvent(ps->up, ps->bwd_done, 0), "cudaStreamWaitEvent");
+    PIPE_CUDA(cudaMemcpyAsync(dy, dy_host, nb, cudaMemcpyHostToDevice, ps->up), "cudaMemcpyAsync(dy)");
+    PIPE_CUDA(cudaEventRecord(ps->dy_in, ps->up), "cudaEventRecord");
+    // the forward writes y once the previous step's y has left
+    PIPE_CUDA(cudaStreamWaitEvent(st, ps->y_out, 0), "cudaStreamWaitEvent");
+    if ((rc = moe_fwd(cfg, xs[p], params, y, nullptr, ctx, ctx_bytes, 1, nullptr, 0, stream)) != MOK_OK)
+        goto fail_sync;
+    PIPE_CUDA(cudaEventRecord(ps->fwd_done, st), "cudaEventRecord");
+    PIPE_CUDA(cudaStreamWaitEvent(ps->down, ps->fwd_done, 0), "cudaStreamWaitEvent");
+    PIPE_CUDA(cudaMemcpyAsync(y_host, y, nb, cudaMemcpyDeviceToHost, ps->down), "cudaMemcpyAsync(y)");
+    PIPE_CUDA(cudaEventRecord(ps->y_out, ps->down), "cudaEventRecord");
+    // the next step's x into the other slot while this step's backward runs (its last
+    // reader, the previous step, is done: the upload stream waited for it above)
+    if (x_next_host) {
+        PIPE_CUDA(cudaMemcpyAsync(xs[1 - p], x_next_host, nb, cudaMemcpyHostToDevice, ps->up),
+                  "cudaMemcpyAsync(next x)");
+        PIPE_CUDA(cudaEventRecord(ps->x_ready[1 - p], ps->up), "cudaEventRecord");
+        ps->slot_x[1 - p] = x_next_host;
+    } else {
+        ps->slot_x[1 - p] = nullptr;
+    }
+    // the backward writes dx into slot p once the download of two steps ago has read it
+    PIPE_CUDA(cudaStreamWaitEvent(st, ps->dy_in, 0), "cudaStreamWaitEvent");
+    PIPE_CUDA(cudaStreamWaitEvent(st, ps->dx_out[p], 0), "cudaStreamWaitEvent");
+    {
+        moe_grads g = *grads;
+        g.dx = dxs[p];
+        if ((rc = moe_bwd(cfg, xs[p], dy, params, ctx, ctx_bytes, &g, inner, scratch_bytes - 6 * io, stream)) !=
+            MOK_OK)
+            goto fail_sync;
+    }
+    PIPE_CUDA(cudaEventRecord(ps->bwd_done, st), "cudaEventRecord");
+    PIPE_CUDA(cudaStreamWaitEvent(ps->down, ps->bwd_done, 0), "cudaStreamWaitEvent");
+    PIPE_CUDA(cudaMemcpyAsync(dx_host, dxs[p], nb, cudaMemcpyDeviceToHost, ps->down), "cudaMemcpyAsync(dx)");
+    PIPE_CUDA(cudaEventRecord(ps->dx_out[p], ps->down), "cudaEventRecord");
+#undef PIPE_CUDA
+    ++ps->calls;
+    return MOK_OK;
+fail_sync:
+    // a failed step leaves nothing in flight: every stream of the sequence drains
+    cudaStreamSynchronize(ps->up);
+    cudaStreamSynchronize(ps->down);
+    cudaStreamSynchronize(st);
+    ps->scratch = nullptr;
+    return rc;
+}
+
+int moe_step_host_sync(void *stream)
+{
+    PipeStreams *ps = nullptr;
+    MOK_TRY(pipe_streams(ps));
+    int rc = MOK_OK;
+    cudaStream_t ss[] = {ps->up, ps->down, static_cast<cudaStream_t>(stream)};
+    for (cudaStream_t s2 : ss)
+        if (const cudaError_t e = cudaStreamSynchronize(s2); e != cudaSuccess && rc == MOK_OK)
+            rc = fail(MOK_ERR_LAUNCH, "cudaStreamSynchronize", e);
     return rc;
 }
 

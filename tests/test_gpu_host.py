@@ -82,3 +82,49 @@ def test_step_host_matches_device_api():
         for k in ("dw_gate_up", "dw_down", "dws_gate_up", "dws_down"):
             assert torch.equal(grads[k].view(torch.int16), g_ref[k].view(torch.int16)), k
         assert torch.equal(grads["drouter_w"].view(torch.int32), g_ref["drouter_w"].view(torch.int32))
+
+
+def test_step_host_async_pipeline_matches_device_api():
+    """moe_step_host_async over three steps with different inputs (each call prefetching
+    the next step's x; y and dx of a step leaving while the next one runs): every
+    step's y and dx, and the last step's weight and router gradients, equal those of
+    the device calls byte for byte.  A second sequence on the same scratch, without
+    prefetch, gives the same bytes again."""
+    case = make_case(WL, device="cuda", gen_device="cpu")
+    dev = torch.device("cuda")
+    layer = MoELayer(cfg_for(WL), case["params"], training=True, device=dev)
+    xs = [torch.roll(case["x"], 7 * i, 0).contiguous() for i in range(3)]
+    dys = [torch.roll(case["dy"], 5 * i, 0).contiguous() for i in range(3)]
+    refs = []
+    for x, dy in zip(xs, dys):
+        y = layer.forward(x).clone()
+        g = {k: (v.clone() if v is not None else None) for k, v in layer.backward(x, dy).items()}
+        refs.append((y, g))
+    torch.cuda.synchronize()
+    c = layer.cfg
+    hxs = [x.cpu().pin_memory() for x in xs]
+    hdys = [dy.cpu().pin_memory() for dy in dys]
+    n = abi.moe_host_scratch_size(c, 3)
+    scratch = torch.empty(n, dtype=torch.uint8, device=dev)
+    grads = layer.new_grads()
+    g = abi.moe_grads(None, grads["dw_gate_up"].data_ptr(), grads["dw_down"].data_ptr(),
+                      grads["drouter_w"].data_ptr(),
+                      grads["dws_gate_up"].data_ptr() if grads["dws_gate_up"] is not None else None,
+                      grads["dws_down"].data_ptr() if grads["dws_down"] is not None else None)
+    for prefetch in (True, False):
+        hys = [torch.empty_like(hxs[0]).pin_memory() for _ in range(3)]
+        hdxs = [torch.empty_like(hxs[0]).pin_memory() for _ in range(3)]
+        for i in range(3):
+            nxt = hxs[i + 1].data_ptr() if prefetch and i + 1 < 3 else None
+            abi.moe_step_host_async(c, hxs[i].data_ptr(), nxt, hdys[i].data_ptr(), layer.cparams, hys[i].data_ptr(),
+                                    hdxs[i].data_ptr(), layer.ctx.data_ptr(), layer.ctx_bytes, g, scratch.data_ptr(),
+                                    n, layer.stream())
+        abi.moe_step_host_sync(layer.stream())
+        assert layer.status() == 0
+        for i, (y_ref, g_ref) in enumerate(refs):
+            assert torch.equal(hys[i].view(torch.int16), y_ref.cpu().view(torch.int16)), (prefetch, i)
+            assert torch.equal(hdxs[i].view(torch.int16), g_ref["dx"].cpu().view(torch.int16)), (prefetch, i)
+        g_last = refs[-1][1]
+        for k in ("dw_gate_up", "dw_down", "dws_gate_up", "dws_down"):
+            assert torch.equal(grads[k].view(torch.int16), g_last[k].view(torch.int16)), (prefetch, k)
+        assert torch.equal(grads["drouter_w"].view(torch.int32), g_last["drouter_w"].view(torch.int32))
