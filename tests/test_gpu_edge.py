@@ -2,7 +2,10 @@
 
 One token; every expert selected (top_k = E); a single routed expert (a dense
 SwiGLU MLP plus a shared expert); the largest top_k (16); sigmoid scoring without
-a group limit and with a routing scale other than 1; the minimum H and I.  Each
+a group limit and with a routing scale other than 1; the minimum H and I; groups
+of exactly 128, 129, 256 and 257 rows (one routed and one shared expert, every
+token in both: the edges of the 128-row tiles and of the 256-row pair tiles,
+whose second half is then full, absent, or a single row).  Each
 runs the forward and the backward; routing is bit-exact, floats within
 |gpu - oracle| <= 1e-2 + 1e-2 |oracle|.
 """
@@ -23,7 +26,8 @@ EDGE = [
     synth.Workload("sigmoid_scaled", T=96, H=512, E=16, k=4, I=256, score_fn=1, routed_scale=2.5, seed=55),
     synth.Workload("groups_scaled", T=80, H=256, E=16, k=3, I=128, S=1, Is=128, score_fn=1, n_group=4,
                    topk_group=2, routed_scale=0.5, seed=56),
-]
+] + [synth.Workload(f"rows_{t}", T=t, H=256, E=1, k=1, I=256, S=1, Is=256, seed=57 + i)
+     for i, t in enumerate((128, 129, 256, 257))]
 
 
 @pytest.mark.parametrize("wl", EDGE, ids=lambda w: w.name)
