@@ -476,11 +476,102 @@ __device__ __forceinline__ void dx_stream_ns(const float *__restrict__ dXs, cons
     cp_async_wait<0>();
 }
 
+// The same sum for k <= 8 (the DeepSeek-V3 layer): only the k + S dX rows (HBM)
+// go through the ring, twice as deep; the token's k router-weight rows (L2-resident)
+// come into registers with plain loads one unit ahead.
+template <int NS>
+__device__ __forceinline__ void dx_stream_k8_ns(const float *__restrict__ dXs, const float *__restrict__ dl,
+                                                const int *__restrict__ topk_idx, const float *__restrict__ router_w,
+                                                __nv_bfloat16 *__restrict__ dx, int T, int H, int k, int S,
+                                                uint8_t *ring)
+{
+    constexpr int KM = 8;
+    const int lane = threadIdx.x & 31;
+    const int nw = gridDim.x * (blockDim.x >> 5);
+    const int kk = k + S, units = H / 128;
+    int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    float dn = 0.0f;
+    int en = 0;
+    if (t < T && lane < k) {
+        dn = dl[static_cast<size_t>(t) * k + lane];
+        en = topk_idx[static_cast<size_t>(t) * k + lane];
+    }
+    for (; t < T; t += nw) {
+        const float dc = dn;
+        const int ec = en;
+        if (t + nw < T && lane < k) {
+            dn = dl[static_cast<size_t>(t + nw) * k + lane];
+            en = topk_idx[static_cast<size_t>(t + nw) * k + lane];
+        }
+        const float *rows = dXs + static_cast<size_t>(t) * kk * H + lane * 4;
+        const float *wrow[KM];
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+            wrow[j] = router_w + static_cast<size_t>(__shfl_sync(0xffffffffu, ec, j < k ? j : 0)) * H + lane * 4;
+        float4 wn[KM];
+#pragma unroll
+        for (int j = 0; j < KM; ++j) wn[j] = j < k ? __ldg(reinterpret_cast<const float4 *>(wrow[j])) : float4{};
+        auto issue = [&](int u) {
+            for (int j = 0; j < kk; ++j)
+                cp_async16(stream_slot(ring, u % NS, kk, j), rows + static_cast<size_t>(j) * H + u * 128);
+        };
+#pragma unroll
+        for (int u = 0; u < NS - 1; ++u) {
+            if (u < units) issue(u);
+            cp_async_commit();
+        }
+        for (int u = 0; u < units; ++u) {
+            if (u + NS - 1 < units) issue(u + NS - 1);
+            cp_async_commit();
+            float4 wc[KM];
+#pragma unroll
+            for (int j = 0; j < KM; ++j) wc[j] = wn[j];
+            if (u + 1 < units) {
+#pragma unroll
+                for (int j = 0; j < KM; ++j)
+                    if (j < k) wn[j] = __ldg(reinterpret_cast<const float4 *>(wrow[j] + (u + 1) * 128));
+            }
+            cp_async_wait<NS - 1>();
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, r[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            for (int j = 0; j < kk; ++j) {
+                float v[4];
+                slot_values<4>(stream_slot(ring, u % NS, kk, j), v);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[q] += v[q];
+            }
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                if (j < k) {
+                    const float d = __shfl_sync(0xffffffffu, dc, j);
+                    r[0] = fmaf(d, wc[j].x, r[0]);
+                    r[1] = fmaf(d, wc[j].y, r[1]);
+                    r[2] = fmaf(d, wc[j].z, r[2]);
+                    r[3] = fmaf(d, wc[j].w, r[3]);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[q] += r[q];
+            store_bf16<4>(dx + static_cast<size_t>(t) * H + u * 128 + lane * 4, acc);
+        }
+    }
+    cp_async_wait<0>();
+}
+
 __device__ __forceinline__ void dx_stream(const float *__restrict__ dXs, const float *__restrict__ dl,
                                           const int *__restrict__ topk_idx, const float *__restrict__ router_w,
                                           __nv_bfloat16 *__restrict__ dx, int T, int H, int k, int S, uint8_t *ring,
                                           int ring_bytes)
 {
+    if (k <= 8) {
+        switch (stream_stages(k + S, ring_bytes)) {
+        case 1: dx_stream_k8_ns<1>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); return;
+        case 2: dx_stream_k8_ns<2>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); return;
+        case 3: dx_stream_k8_ns<3>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); return;
+        case 4: dx_stream_k8_ns<4>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); return;
+        case 5: dx_stream_k8_ns<5>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); return;
+        default: dx_stream_k8_ns<6>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); return;
+        }
+    }
     switch (stream_stages(2 * k + S, ring_bytes)) {
     case 1: dx_stream_ns<1>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
     case 2: dx_stream_ns<2>(dXs, dl, topk_idx, router_w, dx, T, H, k, S, ring); break;
