@@ -81,3 +81,25 @@ def test_mxfp8_backward_argument_checks():
     with pytest.raises(abi.MokError) as ei:      # the one-pass quantiser's shape rule
         abi.moe_quantize_mxfp8_weights_both(fake, 2, 256, 384, fake, fake, fake, fake, None)
     assert ei.value.code == abi.MOK_ERR_INVALID
+
+
+def test_pipelined_host_step_argument_checks():
+    """moe_step_host_async refuses missing host buffers (MOK_ERR_INVALID) and a scratch
+    buffer smaller than moe_host_scratch_size(cfg, 3) (MOK_ERR_WORKSPACE) before it
+    touches a device; the pipelined scratch holds two x and two dx slots more than
+    moe_step_host's.  The pointers are never dereferenced."""
+    c = make_cfg(64, 256, 8, 128, 2)
+    io = 64 * 256 * 2
+    n2, n3 = abi.moe_host_scratch_size(c, 2), abi.moe_host_scratch_size(c, 3)
+    assert n3 - n2 == 2 * ((io + 255) // 256 * 256)
+    p, g = abi.moe_params(), abi.moe_grads()
+    args = dict(x_host=16, x_next_host=None, dy_host=16, y_host=16, dx_host=16)
+    for missing in ("x_host", "dy_host", "y_host", "dx_host"):
+        a = dict(args, **{missing: None})
+        with pytest.raises(abi.MokError) as ei:
+            abi.moe_step_host_async(c, a["x_host"], a["x_next_host"], a["dy_host"], p, a["y_host"], a["dx_host"], 16, 0,
+                                    g, 16, n3, None)
+        assert ei.value.code == abi.MOK_ERR_INVALID, missing
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_step_host_async(c, 16, None, 16, p, 16, 16, 16, 0, g, 16, n3 - 1, None)
+    assert ei.value.code == abi.MOK_ERR_WORKSPACE
