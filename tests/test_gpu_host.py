@@ -128,3 +128,48 @@ def test_step_host_async_pipeline_matches_device_api():
         for k in ("dw_gate_up", "dw_down", "dws_gate_up", "dws_down"):
             assert torch.equal(grads[k].view(torch.int16), g_last[k].view(torch.int16)), (prefetch, k)
         assert torch.equal(grads["drouter_w"].view(torch.int32), g_last["drouter_w"].view(torch.int32))
+
+
+def test_step_host_async_mxfp8_matches_device_api():
+    """The pipelined host steps drive the MXFP8 training step too (MXFP8 forward and data
+    gradients, BF16 weight gradients): two steps with different inputs, each step's y and
+    dx and the last step's gradients byte for byte against the device calls."""
+    from tests.test_gpu_layer import MX_BWD_CASES, _mx_train_params
+    wl = MX_BWD_CASES[0]
+    case = make_case(wl, device="cuda", gen_device="cpu", mx=True)
+    dev = torch.device("cuda")
+    layer = MoELayer(cfg_for(wl), _mx_train_params(case["params"]), training=True, device=dev)
+    xs = [case["x"], torch.roll(case["x"], 11, 0).contiguous()]
+    dys = [case["dy"], torch.roll(case["dy"], 3, 0).contiguous()]
+    refs = []
+    for x, dy in zip(xs, dys):
+        y = layer.forward(x).clone()
+        g = {k: (v.clone() if v is not None else None) for k, v in layer.backward(x, dy).items()}
+        refs.append((y, g))
+    torch.cuda.synchronize()
+    c = layer.cfg
+    hxs = [x.cpu().pin_memory() for x in xs]
+    hdys = [dy.cpu().pin_memory() for dy in dys]
+    hys = [torch.empty_like(hxs[0]).pin_memory() for _ in range(2)]
+    hdxs = [torch.empty_like(hxs[0]).pin_memory() for _ in range(2)]
+    n = abi.moe_host_scratch_size(c, 3)
+    scratch = torch.empty(n, dtype=torch.uint8, device=dev)
+    grads = layer.new_grads()
+    g = abi.moe_grads(None, grads["dw_gate_up"].data_ptr(), grads["dw_down"].data_ptr(),
+                      grads["drouter_w"].data_ptr(),
+                      grads["dws_gate_up"].data_ptr() if grads["dws_gate_up"] is not None else None,
+                      grads["dws_down"].data_ptr() if grads["dws_down"] is not None else None)
+    for i in range(2):
+        nxt = hxs[1].data_ptr() if i == 0 else None
+        abi.moe_step_host_async(c, hxs[i].data_ptr(), nxt, hdys[i].data_ptr(), layer.cparams, hys[i].data_ptr(),
+                                hdxs[i].data_ptr(), layer.ctx.data_ptr(), layer.ctx_bytes, g, scratch.data_ptr(), n,
+                                layer.stream())
+    abi.moe_step_host_sync(layer.stream())
+    assert layer.status() == 0
+    for i, (y_ref, g_ref) in enumerate(refs):
+        assert torch.equal(hys[i].view(torch.int16), y_ref.cpu().view(torch.int16)), i
+        assert torch.equal(hdxs[i].view(torch.int16), g_ref["dx"].cpu().view(torch.int16)), i
+    for k in ("dw_gate_up", "dw_down", "dws_gate_up", "dws_down"):
+        if refs[-1][1][k] is not None:
+            assert torch.equal(grads[k].view(torch.int16), refs[-1][1][k].view(torch.int16)), k
+    assert torch.equal(grads["drouter_w"].view(torch.int32), refs[-1][1]["drouter_w"].view(torch.int32))
