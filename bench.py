@@ -52,6 +52,8 @@ def parse():
                     help="BF16 workloads also measured, comma-separated ('none' to skip)")
     ap.add_argument("--mx-workload", default="dsv3_mxfp8",
                     help="MXFP8 forward workload measured after the main one ('none' to skip)")
+    ap.add_argument("--ep-world", type=int, default=8,
+                    help="ranks of the expert-parallel forward emulated on one GPU (0 to skip)")
     return ap.parse_args()
 
 
@@ -567,6 +569,13 @@ def main():
         mx = mxfp8_run(synth.scaled(mwl, seed=mwl.seed + 1000 * rank), dev, K, args.warmup, world, dist, pk,
                        not args.no_ab)
 
+    # ---------------- expert-parallel forward, its ranks emulated on this GPU
+    ep = None
+    if args.ep_world > 0:
+        ep = ep_emulated_run(synth.scaled(wl, name=wl.name + "_ep", T=wl.T // args.ep_world,
+                                          seed=wl.seed + 1000 * rank + 7), args.ep_world, dev, K, args.warmup)
+        torch.cuda.empty_cache()
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -603,6 +612,7 @@ def main():
             "phase_roofline": phase_roofline,
             "mxfp8": mx,
             "bf16_workloads": extra,
+            "ep_emulated": ep,
             "e2e": e2e, "cpu_baseline": cpu,
         }
         print(json.dumps(line))
@@ -676,6 +686,57 @@ def bf16_workload_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
                     "bwd_tc_peak_frac_of_measured_sustained":
                         2 * fwd_flops / (bwd_ms / 1e3) / 1e12 / pk["bf16_sustained"]})
     del layer, params, grads
+    return out
+
+
+def ep_emulated_run(wl, W, dev, K, warmup):
+    """The expert-parallel forward with its W ranks (wl.T tokens each) run on this GPU in
+    stream order, against the one-GPU forward of the same W * wl.T tokens.  Both do the
+    same expert arithmetic; the difference is what the rank split adds on one device (the
+    owners' row layouts, the pull copy of every received row, per-rank launches and
+    tails).  No NVLink is crossed: this is the data path, not a multi-GPU measurement."""
+    import torch
+    from mixture_experts_layer_persistent_b200 import EPWorld, MoELayer, cfg_for, split_params, synth
+    params = synth.draw_params(wl, dev)
+    xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(W)]
+    ep = EPWorld(cfg_for(wl), W, [split_params(params, W, r, wl.E) for r in range(W)], device=dev)
+    ys = [torch.empty_like(x) for x in xs]
+    whole = synth.scaled(wl, T=wl.T * W)
+    one = MoELayer(cfg_for(whole), params, training=False, device=dev)
+    xw = torch.cat(xs)
+    yw = torch.empty_like(xw)
+    routing = one.new_routing()
+    one.forward(xw, yw, routing=routing)
+    counts = routing["counts"].cpu().numpy()
+    recv = counts.reshape(W, wl.E // W).sum(axis=1)        # rows each rank's experts receive
+    for _ in range(warmup):
+        ep.forward(xs, ys)
+        one.forward(xw, yw)
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    t_ep, t_one = [], []
+    for _ in range(K):                                  # interleaved legs
+        a, b = mk(), mk()
+        a.record(); ep.forward(xs, ys); b.record()
+        c, d = mk(), mk()
+        c.record(); one.forward(xw, yw); d.record()
+        t_ep.append((a, b)); t_one.append((c, d))
+    torch.cuda.synchronize()
+    ms_ep = statistics.mean(a.elapsed_time(b) for a, b in t_ep)
+    ms_one = statistics.mean(c.elapsed_time(d) for c, d in t_one)
+    status = one.status()
+    out = {"workload": f"{wl.name}: the forward of {W} ranks x {wl.T} tokens, E={wl.E} experts "
+                       f"({wl.E // W} per rank), top-{wl.k}, H={wl.H}, I={wl.I}, {wl.S} shared, all ranks on one GPU",
+           "world": W, "tokens_per_rank": wl.T,
+           "ms": ms_ep, "tokens_per_s": W * wl.T / (ms_ep / 1e3),
+           "one_gpu_ms": ms_one, "one_gpu_tokens_per_s": W * wl.T / (ms_one / 1e3),
+           "ep_over_one_gpu_time": ms_ep / ms_one,
+           "received_rows_per_rank": [int(v) for v in recv],
+           "received_rows_max_over_mean": float(recv.max() / max(1e-9, recv.mean())),
+           "pull_bytes": int((recv.sum() + W * wl.T) * wl.H * 2),
+           "device_status": status, "launches_per_forward": W * (6 + 5 + 1),
+           "note": "ranks emulated in stream order on one device; no link crossed"}
+    del ep, one, params, xs, ys, xw, yw
     return out
 
 

@@ -33,6 +33,8 @@ MOK_SCHEDULE_PERSISTENT = 0
 MOK_SCHEDULE_SPLIT = 1
 MOK_SCHEDULE_SPLIT_PDL = 2
 MOK_TRACE_POINTS = 9
+MOK_EP_MAX_RANKS = 8
+MOK_EP_IPC_HANDLE_BYTES = 64
 MOK_SAVED_H, MOK_SAVED_HQ, MOK_SAVED_HS, MOK_SAVED_GU, MOK_SAVED_HW, MOK_SAVED_ROW_TOKEN, MOK_SAVED_ROW_W = range(7)
 
 _i32, _f32, _vp, _sz = ctypes.c_int32, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
@@ -108,6 +110,13 @@ def lib():
         L.moe_set_schedule.argtypes = [ctypes.c_int]
         L.moe_get_schedule.argtypes = [P(_i32)]
         L.moe_trace_device.argtypes = [_vp, _sz, _vp, _sz]
+        L.moe_ep_size.argtypes = [P(moe_cfg), _i32, P(_sz), P(_sz)]
+        L.moe_ep_route.argtypes = [P(moe_cfg), _i32, _i32, _vp, P(moe_params), _vp, _sz, _vp]
+        L.moe_ep_experts.argtypes = [P(moe_cfg), _i32, _i32, P(_vp), P(_vp), P(moe_params), _vp, _sz, _vp]
+        L.moe_ep_combine.argtypes = [P(moe_cfg), _i32, _i32, _vp, _vp, _vp]
+        L.moe_ep_ipc_handle.argtypes = [_vp, _vp, P(_sz)]
+        L.moe_ep_ipc_open.argtypes = [_vp, _sz, P(_vp)]
+        L.moe_ep_ipc_close.argtypes = [_vp, _sz]
         L.moe_strerror.argtypes = [ctypes.c_int]
         L.moe_strerror.restype = ctypes.c_char_p
         L.moe_last_error.argtypes = []
@@ -117,7 +126,9 @@ def lib():
                      "moe_quantize_mxfp8", "moe_quantize_mxfp8_weights",
                      "moe_quantize_mxfp8_weights_t", "moe_quantize_mxfp8_weights_both", "moe_status",
                      "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal", "moe_saved_tensor",
-                     "moe_set_schedule", "moe_get_schedule", "moe_trace_device"):
+                     "moe_set_schedule", "moe_get_schedule", "moe_trace_device", "moe_ep_size", "moe_ep_route",
+                     "moe_ep_experts", "moe_ep_combine", "moe_ep_ipc_handle", "moe_ep_ipc_open",
+                     "moe_ep_ipc_close"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -261,3 +272,46 @@ def moe_launch_count() -> int:
 def moe_test_drop_signal(enable: bool):
     """Fault injection for the bounded waits (see include/mok.h)."""
     _check("moe_test_drop_signal", lib().moe_test_drop_signal(int(enable)))
+
+
+def moe_ep_size(cfg: moe_cfg, world: int):
+    """(state_bytes, scratch_bytes) of one rank of an expert-parallel forward."""
+    a, b = _sz(), _sz()
+    _check("moe_ep_size", lib().moe_ep_size(ctypes.byref(cfg), int(world), ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
+
+
+def moe_ep_route(cfg, world, rank, x, params, state, state_bytes, stream):
+    _check("moe_ep_route", lib().moe_ep_route(ctypes.byref(cfg), int(world), int(rank), x, ctypes.byref(params),
+                                              state, state_bytes, stream))
+
+
+def moe_ep_experts(cfg, world, rank, x_ranks, state_ranks, params, scratch, scratch_bytes, stream):
+    xs = (_vp * len(x_ranks))(*x_ranks)
+    ss = (_vp * len(state_ranks))(*state_ranks)
+    _check("moe_ep_experts", lib().moe_ep_experts(ctypes.byref(cfg), int(world), int(rank), xs, ss,
+                                                  ctypes.byref(params), scratch, scratch_bytes, stream))
+
+
+def moe_ep_combine(cfg, world, rank, state, y, stream):
+    _check("moe_ep_combine", lib().moe_ep_combine(ctypes.byref(cfg), int(world), int(rank), state, y, stream))
+
+
+def moe_ep_ipc_handle(dev_ptr):
+    """(handle bytes, offset) of the device allocation holding dev_ptr."""
+    h = ctypes.create_string_buffer(MOK_EP_IPC_HANDLE_BYTES)
+    off = _sz()
+    _check("moe_ep_ipc_handle", lib().moe_ep_ipc_handle(dev_ptr, h, ctypes.byref(off)))
+    return h.raw, off.value
+
+
+def moe_ep_ipc_open(handle: bytes, offset: int) -> int:
+    if len(handle) != MOK_EP_IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle is %d bytes" % MOK_EP_IPC_HANDLE_BYTES)
+    p = _vp()
+    _check("moe_ep_ipc_open", lib().moe_ep_ipc_open(handle, offset, ctypes.byref(p)))
+    return p.value
+
+
+def moe_ep_ipc_close(dev_ptr: int, offset: int) -> None:
+    _check("moe_ep_ipc_close", lib().moe_ep_ipc_close(dev_ptr, offset))

@@ -1,0 +1,187 @@
+// ep.cuh -- expert parallelism: the rank-crossing steps of the forward.
+//
+// "Cursor åpner megakernelen…" (the pull-versus-push paragraph) and
+// "Megakernels are dead and back…" ("Números de MoK"): the GPU that owns an
+// expert pulls the token rows routed to it from the GPU that holds them, and
+// pushes each expert output row back to that GPU, where the fixed-order k-sum
+// runs.  Here rank r owns the routed experts [r E_loc, (r+1) E_loc) and every
+// rank routes its own T tokens over all E experts (route.cuh, unchanged).
+//
+// The owner's sorted rows: for each of its experts j (ascending), the rows of
+// every source rank s (ascending), each source's rows in its own dispatch
+// order (token ascending), then the shared experts' rows of the owner's own
+// tokens.  Every output row depends only on its own input row and the expert's
+// weights, so the order changes no value: each rank's y equals the one-GPU
+// layer's on its tokens, byte for byte.
+//
+// Peer buffers are addressed through plain pointers valid on this device (the
+// owner's own buffers, another allocation on the same device, or another GPU's
+// memory mapped into this process); loads and stores are ordinary global ones
+// (no TMA, no multicast).  The calls of one phase must be complete on every
+// rank before any rank starts the next phase; the caller orders them.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "mok.h"
+
+namespace mok {
+
+constexpr int kEpMaxRanks = MOK_EP_MAX_RANKS;
+// Row codes that cross ranks: (rank << kEpRankShift) | row on that rank
+constexpr int kEpRankShift = 24;
+constexpr int kEpRowMask = (1 << kEpRankShift) - 1;
+
+// Every rank's routing record and slot rows, as this device addresses them.
+struct EpView {
+    const int *counts[kEpMaxRanks];     // [E] tokens of rank s per expert
+    const int *offsets[kEpMaxRanks];    // [E + S + 1] rank s's sorted-row ranges
+    const int *perm[kEpMaxRanks];       // [T k] rank s's sorted row -> t k + slot
+    const float *topk_w[kEpMaxRanks];   // [T k] rank s's routing weights
+    const __nv_bfloat16 *x[kEpMaxRanks];   // [T, H] rank s's tokens
+    float *O[kEpMaxRanks];              // [T, k + S, H] rank s's fp32 slot rows
+};
+
+struct EpArgs {
+    int world, rank;
+    int T, H, k, kk, S, E_loc;
+    int rr_cap;            // routed rows this rank can receive: world T min(k, E_loc)
+    int *seg;              // [E_loc world + 1] first sorted row of each (expert, source) segment; seg[n] = routed rows
+    int *offsets;          // [E_loc + S + 1] the owner's group ranges (routed experts, then shared)
+    int *row_token;        // [rows] row of x_recv each sorted row reads
+    int *row_src;          // [rows] (source rank << 24) | token
+    int *row_slot;         // [rows] (source rank << 24) | slot row t (k + S) + slot in that rank's O
+    float *row_w;          // [rows] routing weight (1 for shared rows)
+    float **push;          // [kEpMaxRanks] slot rows of every rank, for the push epilogue
+    __nv_bfloat16 *x_recv; // [T + rr_cap, H] the owner's own tokens, then every received row
+    int *status;
+};
+
+// One block of 256 threads: segment sizes from every source's counts, their
+// exclusive scan (ascending (expert, source)), the owner's group ranges and
+// the push table.  E_loc * world = E <= 256 segments, one per thread.
+__global__ void __launch_bounds__(256) ep_layout_kernel(EpView v, EpArgs a)
+{
+    __shared__ int s_scan[256];
+    __shared__ int s_total;
+    const int n = a.E_loc * a.world;
+    const int i = threadIdx.x;
+    int c = 0;
+    if (i < n) {
+        const int j = i / a.world, s = i - j * a.world;
+        c = v.counts[s][a.rank * a.E_loc + j];
+        if (c < 0 || c > a.T) c = -1;       // impossible count: reject the whole layout below
+    }
+    s_scan[i] = c;
+    __syncthreads();
+    // inclusive Hillis-Steele scan
+    for (int d = 1; d < 256; d <<= 1) {
+        const int add = i >= d ? s_scan[i - d] : 0;
+        __syncthreads();
+        s_scan[i] += add;
+        __syncthreads();
+    }
+    if (i == 0) s_total = s_scan[n - 1];
+    __shared__ int s_bad;
+    if (i == 0) s_bad = 0;
+    __syncthreads();
+    if (c < 0) atomicOr(&s_bad, 1);
+    __syncthreads();
+    // Bound every index the later steps use: a layout larger than the receive
+    // buffers (impossible for counts written by the dispatch) becomes empty.
+    const bool ok = !s_bad && s_total <= a.rr_cap;
+    if (!ok && i == 0) atomicOr(a.status, MOK_STATUS_BAD_INDEX);
+    const int total = ok ? s_total : 0;
+    const int excl = ok ? s_scan[i] - c : 0;
+    if (i < n) a.seg[i] = excl;
+    if (i == 0) a.seg[n] = total;
+    if (i < n && i % a.world == 0) a.offsets[i / a.world] = excl;
+    if (i <= a.S) a.offsets[a.E_loc + i] = total + i * a.T;
+    if (i < a.world) a.push[i] = v.O[i];
+}
+
+// Sorted rows of the owner.  Blocks [0, n): segment b = (expert j, source s)
+// copies source s's rows of expert e = rank E_loc + j; blocks after those:
+// the shared experts' rows of the owner's own tokens, 256 tokens per block.
+__global__ void __launch_bounds__(256) ep_rows_kernel(EpView v, EpArgs a)
+{
+    const int n = a.E_loc * a.world;
+    const int b = blockIdx.x;
+    if (b < n) {
+        const int j = b / a.world, s = b - j * a.world;
+        const int e = a.rank * a.E_loc + j;
+        const int base = a.seg[b];
+        const int cnt = a.seg[b + 1] - base;
+        const int src0 = v.offsets[s][e];
+        const int tk = a.T * a.k;
+        // a range outside the source's rows (impossible for a record the dispatch wrote)
+        // leaves every row of the segment in bounds: token 0, slot 0, weight 0
+        const bool range_ok = src0 >= 0 && src0 + cnt <= tk;
+        if (!range_ok && threadIdx.x == 0 && cnt > 0) atomicOr(a.status, MOK_STATUS_BAD_INDEX);
+        for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+            int q = range_ok ? v.perm[s][src0 + i] : 0;  // t k + slot on rank s
+            if (q < 0 || q >= tk) {
+                atomicOr(a.status, MOK_STATUS_BAD_INDEX);
+                q = 0;
+            }
+            const int t = q / a.k, slot = q - t * a.k;
+            const int r = base + i;
+            a.row_token[r] = a.T + r;
+            a.row_src[r] = (s << kEpRankShift) | t;
+            a.row_slot[r] = (s << kEpRankShift) | (t * a.kk + slot);
+            a.row_w[r] = range_ok ? v.topk_w[s][q] : 0.0f;
+        }
+    } else {
+        const int nb = (a.T + 255) / 256;
+        const int sb = b - n;
+        const int s2 = sb / nb;
+        const int t = (sb - s2 * nb) * 256 + threadIdx.x;
+        if (s2 < a.S && t < a.T) {
+            const int r = a.seg[n] + s2 * a.T + t;
+            a.row_token[r] = t;
+            a.row_src[r] = (a.rank << kEpRankShift) | t;
+            a.row_slot[r] = (a.rank << kEpRankShift) | (t * a.kk + a.k + s2);
+            a.row_w[r] = 1.0f;
+        }
+    }
+}
+
+// Pull at dispatch: x_recv[t] = own x[t] for t < T, x_recv[T + r] = x of the
+// row's source rank at its token.  One warp per row, 16-byte loads, four in
+// flight per lane; every remote row crosses the link once.
+__global__ void __launch_bounds__(256) ep_pull_kernel(EpView v, EpArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int n_warps = (gridDim.x * blockDim.x) >> 5;
+    const int rows = a.T + a.seg[a.E_loc * a.world];
+    const int vec = a.H / 8;                           // 16-byte vectors per row (H % 256 == 0)
+    for (int r = warp; r < rows; r += n_warps) {
+        const __nv_bfloat16 *src;
+        if (r < a.T) {
+            src = v.x[a.rank] + (size_t)r * a.H;
+        } else {
+            const int code = a.row_src[r - a.T];
+            const int s = code >> kEpRankShift, t = code & kEpRowMask;
+            if (s < 0 || s >= a.world || t >= a.T) {    // never written so by ep_rows_kernel
+                if (lane == 0) atomicOr(a.status, MOK_STATUS_BAD_INDEX);
+                continue;
+            }
+            src = v.x[s] + (size_t)t * a.H;
+        }
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+        uint4 *d4 = reinterpret_cast<uint4 *>(a.x_recv + (size_t)r * a.H);
+        for (int c = lane; c < vec; c += 128) {        // vec is a multiple of 32
+            uint4 q[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (c + 32 * u < vec) q[u] = s4[c + 32 * u];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (c + 32 * u < vec) d4[c + 32 * u] = q[u];
+        }
+    }
+}
+
+}  // namespace mok

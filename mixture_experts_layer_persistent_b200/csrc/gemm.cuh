@@ -81,6 +81,8 @@ struct GemmArgs {
     __nv_bfloat16 *out2;          // EPI_SWIGLU: saved gate/up pre-activations [R, 2I] (or null)
     __nv_bfloat16 *out3;          // EPI_SWIGLU: w * h [R, I] (or null)
     float *out_f32;               // EPI_ROUTER: partial logits [n_tiles, rows, 256]; EPI_PUSH: fp32 slot rows
+    float *const *push_dst;       // BF16 EPI_PUSH across ranks (expert parallelism): slot rows of every rank;
+                                  // row_slot is then (rank << 24) | slot row, every row a plain store (null: off)
     const __nv_bfloat16 *aux;     // EPI_DSWIGLU: saved gate/up pre-activations [R, 2I]
     const __nv_bfloat16 *aux_h;   // EPI_DSWIGLU: saved h [R, I] (the down GEMM's A operand)
     float *gpart;                 // EPI_DSWIGLU: <dy W_down, h> of each routed row over each N tile [R_routed, n_tiles]
@@ -1267,9 +1269,16 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         }
                     }
                 } else if constexpr (C::EPI == EPI_PUSH) {
-                    // fp32 rows pushed into their (token, slot) row of the slot buffer
-                    const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
-                    float *dst = args.out_f32 + (size_t)dst_row * args.ldo + t.nt * C::BN;
+                    // fp32 rows pushed into their (token, slot) row of the slot buffer; across
+                    // ranks into the slot buffer of the token's rank, with plain stores
+                    int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
+                    float *obase = args.out_f32;
+                    const bool tma = full && !args.push_dst;
+                    if (args.push_dst) {
+                        obase = args.push_dst[dst_row >> 24];
+                        dst_row &= (1 << 24) - 1;
+                    }
+                    float *dst = obase + (size_t)dst_row * args.ldo + t.nt * C::BN;
 #pragma unroll 1
                     for (int c = 0; c < C::BN; c += 32) {
                         float v[32];
@@ -1278,7 +1287,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                         tmem_ld_wait();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
-                        if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
+                        if (tma) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
                         else if (valid) store_row_direct(dst + c, p);
                     }
                 } else if constexpr (C::EPI == EPI_WGRAD) {

@@ -7,10 +7,12 @@
 
 #include <cudaTypedefs.h>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
 #include "combine.cuh"
+#include "ep.cuh"
 #include "fused.cuh"
 #include "fused_bwd.cuh"
 #include "gemm.cuh"
@@ -399,11 +401,12 @@ struct FwdPlan {
     int n_chunks;
 };
 
-int build_fwd_plan(const moe_cfg &c, const void *x, const moe_params &p, const State &st, const DeviceInfo &dev,
-                   bool training, FwdPlan &pl)
+// Router logits, top-k and dispatch of the forward (every schedule, and the
+// routing phase of expert parallelism).
+int build_route_plan(const moe_cfg &c, const void *x, const moe_params &p, const State &st, const DeviceInfo &dev,
+                     FwdPlan &pl)
 {
     const Shapes s = shapes(c);
-    const bool mx = c.dtype == MOK_DTYPE_MXFP8;
     // router logits on the tensor cores: x . [Wr_hi | Wr_mid | Wr_lo]^T, split over K
     if (!make_tmap(&pl.m.rA, x, s.H, s.T, BK, 128, 2)) return fail(MOK_ERR_INVALID, "tensor map (x)");
     if (!make_tmap(&pl.m.rB, st.wr3, 3 * s.H, s.E, BK, 256, 2)) return fail(MOK_ERR_INVALID, "tensor map (router)");
@@ -441,6 +444,15 @@ int build_fwd_plan(const moe_cfg &c, const void *x, const moe_params &p, const S
     da.hist = st.hist;
     da.status = dev.status;
     pl.n_chunks = static_cast<int>((s.T + kDispatchChunk - 1) / kDispatchChunk);
+    return MOK_OK;
+}
+
+int build_fwd_plan(const moe_cfg &c, const void *x, const moe_params &p, const State &st, const DeviceInfo &dev,
+                   bool training, FwdPlan &pl)
+{
+    const Shapes s = shapes(c);
+    const bool mx = c.dtype == MOK_DTYPE_MXFP8;
+    MOK_TRY(build_route_plan(c, x, p, st, dev, pl));
 
     GemmArgs &ga = pl.ga;
     GemmArgs &gd = pl.gd;
@@ -555,6 +567,28 @@ int copy_routing(const moe_routing *routing, const State &st, const Shapes &s, c
     return MOK_OK;
 }
 
+// Router split, router GEMM and top-k (the split schedule's first launches).
+int launch_router(const moe_cfg &c, const moe_params &p, const State &st, const DeviceInfo &dev, const FwdPlan &pl,
+                  cudaStream_t stream)
+{
+    const Shapes s = shapes(c);
+    MOK_TRY(launch_k(router_split_kernel, dim3(blocks_for(s.E * s.H, 256)), dim3(256), 0, stream, "router_split_kernel",
+                     p.router_w, st.wr3, c.E, c.H, st.all_rows, c.T));
+    MOK_TRY(launch_gemm<typename FusedCfg<false>::Router>(pl.m.rA, pl.m.rB, pl.m.rB, pl.m.rO, pl.m.rO, pl.m.rO, pl.gr,
+                                                         dev.sms, stream));
+    return launch_k(router_select_kernel, dim3(blocks_for(s.T, 8)), dim3(256), 0, stream, "router_select_kernel", pl.sa);
+}
+
+// Counts, scan and placement of the sorted rows.
+int launch_dispatch(const FwdPlan &pl, cudaStream_t stream)
+{
+    MOK_TRY(launch_k(dispatch_count_kernel, dim3(pl.n_chunks), dim3(kDispatchChunk), 0, stream, "dispatch_count_kernel",
+                     pl.da));
+    MOK_TRY(launch_k(dispatch_scan_kernel, dim3(1), dim3(256), 0, stream, "dispatch_scan_kernel", pl.da, pl.n_chunks));
+    return launch_k(dispatch_place_kernel, dim3(pl.n_chunks), dim3(kDispatchChunk), 0, stream, "dispatch_place_kernel",
+                    pl.da);
+}
+
 // Split schedule: one launch per step, in stream order.
 int forward_split(const moe_cfg &c, const void *x, const moe_params &p, void *y, const State &st,
                   const DeviceInfo &dev, const FwdPlan &pl, cudaStream_t stream)
@@ -564,18 +598,9 @@ int forward_split(const moe_cfg &c, const void *x, const moe_params &p, void *y,
     if (const cudaError_t e = cudaMemsetAsync(st.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
     MOK_TRY(mark_fwd(0, stream));
-    MOK_TRY(launch_k(router_split_kernel, dim3(blocks_for(s.E * s.H, 256)), dim3(256), 0, stream, "router_split_kernel",
-                     p.router_w, st.wr3, c.E, c.H, st.all_rows, c.T));
-    MOK_TRY(launch_gemm<typename FusedCfg<false>::Router>(pl.m.rA, pl.m.rB, pl.m.rB, pl.m.rO, pl.m.rO, pl.m.rO, pl.gr,
-                                                         dev.sms, stream));
-    MOK_TRY(launch_k(router_select_kernel, dim3(blocks_for(s.T, 8)), dim3(256), 0, stream, "router_select_kernel", pl.sa));
-
+    MOK_TRY(launch_router(c, p, st, dev, pl, stream));
     MOK_TRY(mark_fwd(1, stream));
-    MOK_TRY(launch_k(dispatch_count_kernel, dim3(pl.n_chunks), dim3(kDispatchChunk), 0, stream, "dispatch_count_kernel",
-                     pl.da));
-    MOK_TRY(launch_k(dispatch_scan_kernel, dim3(1), dim3(256), 0, stream, "dispatch_scan_kernel", pl.da, pl.n_chunks));
-    MOK_TRY(launch_k(dispatch_place_kernel, dim3(pl.n_chunks), dim3(kDispatchChunk), 0, stream, "dispatch_place_kernel",
-                     pl.da));
+    MOK_TRY(launch_dispatch(pl, stream));
 
     MOK_TRY(mark_fwd(2, stream));
     GemmArgs ga = pl.ga, gd = pl.gd;
@@ -1016,6 +1041,144 @@ int check_params(const moe_cfg &c, const moe_params *p)
         if (q && !aligned16(q)) return MOK_ERR_INVALID;
     return MOK_OK;
 }
+
+// ------------------------------------------------------------------ expert parallelism
+// Scratch of one rank's expert phase: its sorted rows, the token rows it
+// pulled and the h of those rows, sized for the largest share it can receive
+// (every token of every rank choosing min(k, E_loc) of its experts).
+struct EpScratch {
+    int *seg, *offsets, *row_token, *row_src, *row_slot;
+    float *row_w;
+    float **push;
+    int *sched;
+    __nv_bfloat16 *x_recv, *h;
+    long long rr_cap, rows_cap;
+    size_t bytes;
+};
+
+EpScratch carve_ep(const moe_cfg &c, int world, void *buf)
+{
+    const Shapes s = shapes(c);
+    const long long el = s.E / world;
+    EpScratch e{};
+    e.rr_cap = static_cast<long long>(world) * s.T * std::min<long long>(s.k, el);
+    e.rows_cap = e.rr_cap + s.S * s.T;
+    Carver cv(buf);
+    e.seg = cv.take<int>(s.E + 1);
+    e.offsets = cv.take<int>(el + s.S + 1);
+    e.row_token = cv.take<int>(e.rows_cap);
+    e.row_src = cv.take<int>(e.rows_cap);
+    e.row_slot = cv.take<int>(e.rows_cap);
+    e.row_w = cv.take<float>(e.rows_cap);
+    e.push = cv.take<float *>(kEpMaxRanks);
+    e.sched = cv.take<int>(kSchedCounters);
+    e.x_recv = cv.take<__nv_bfloat16>((s.T + e.rr_cap) * s.H);
+    e.h = cv.take<__nv_bfloat16>(e.rows_cap * s.I);
+    e.bytes = align_up(cv.off, 256);
+    return e;
+}
+
+int check_ep(const moe_cfg *c, int world, int rank)
+{
+    MOK_TRY(check_cfg(c));
+    if (world < 1 || world > kEpMaxRanks || rank < 0 || rank >= world || c->E % world) return MOK_ERR_INVALID;
+    if (c->dtype != MOK_DTYPE_BF16) return MOK_ERR_UNSUPPORTED;
+    if (static_cast<long long>(c->T) * (c->top_k + c->n_shared) >= (1ll << kEpRankShift)) return MOK_ERR_INVALID;
+    const long long rows = static_cast<long long>(world) * c->T * std::min(c->top_k, c->E / world) +
+                           static_cast<long long>(c->n_shared + 1) * c->T;
+    if (rows >= (1ll << 31)) return MOK_ERR_INVALID;
+    return MOK_OK;
+}
+
+int ep_route(const moe_cfg &c, const void *x, const moe_params &p, const State &st, const DeviceInfo &dev,
+             cudaStream_t stream)
+{
+    t_launches = 0;
+    t_pdl = false;
+    FwdPlan pl;
+    MOK_TRY(build_route_plan(c, x, p, st, dev, pl));
+    if (const cudaError_t e = cudaMemsetAsync(st.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
+    MOK_TRY(launch_router(c, p, st, dev, pl, stream));
+    return launch_dispatch(pl, stream);
+}
+
+int ep_experts(const moe_cfg &c, int world, int rank, const void *const *xr, void *const *sr, const moe_params &p,
+               const EpScratch &es, const DeviceInfo &dev, cudaStream_t stream)
+{
+    t_launches = 0;
+    t_pdl = false;
+    const Shapes s = shapes(c);
+    const int el = c.E / world;
+    EpView v{};
+    for (int r = 0; r < world; ++r) {
+        const State q = carve_state(c, sr[r], false);
+        v.counts[r] = q.counts;
+        v.offsets[r] = q.offsets;
+        v.perm[r] = q.perm;
+        v.topk_w[r] = q.topk_w;
+        v.x[r] = static_cast<const __nv_bfloat16 *>(xr[r]);
+        v.O[r] = q.O;
+    }
+    EpArgs a{};
+    a.world = world; a.rank = rank;
+    a.T = c.T; a.H = c.H; a.k = c.top_k; a.kk = static_cast<int>(s.kk); a.S = c.n_shared; a.E_loc = el;
+    a.rr_cap = static_cast<int>(es.rr_cap);
+    a.seg = es.seg; a.offsets = es.offsets;
+    a.row_token = es.row_token; a.row_src = es.row_src; a.row_slot = es.row_slot; a.row_w = es.row_w;
+    a.push = es.push; a.x_recv = es.x_recv; a.status = dev.status;
+
+    // tensor maps: the rank's experts, the shared experts, h, and its own slot rows
+    // (the push epilogue stores through es.push instead; the map only has to exist)
+    const State own = carve_state(c, sr[rank], false);
+    CUtensorMap gB, gBs, gO, dA, dB, dBs, dO;
+    if (!make_tmap(&gB, p.w_gate_up, s.H, el * 2 * s.I, BK, 128, 2) ||
+        !make_tmap(&gBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : el) * 2 * s.I, BK, 128, 2) ||
+        !make_tmap(&gO, es.h, s.I, es.rows_cap, 64, 32, 2) ||
+        !make_tmap(&dA, es.h, s.I, es.rows_cap, BK, 128, 2) ||
+        !make_tmap(&dB, p.w_down, s.I, el * s.H, BK, 256, 2) ||
+        !make_tmap(&dBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : el) * s.H, BK, 256, 2) ||
+        !make_tmap(&dO, own.O, s.H, s.T * s.kk, 32, 1, 4))
+        return fail(MOK_ERR_INVALID, "tensor map (expert-parallel GEMMs)");
+    GemmArgs ga{};
+    ga.sched = es.sched + 0;
+    ga.num_groups = el + c.n_shared;
+    ga.num_routed = el;
+    ga.offsets = es.offsets;
+    ga.row_token = es.row_token;
+    ga.row_slot = es.row_slot;
+    ga.row_w = es.row_w;
+    ga.n_tiles = c.I / 128;
+    ga.num_kb = c.H / BK;
+    ga.b_rows_per_group = 2 * c.I;
+    ga.b_half = c.I;
+    ga.inter = c.I;
+    ga.gather_src = es.x_recv;
+    ga.gather_ld = c.H;
+    ga.out = es.h;
+    ga.status = dev.status;
+    GemmArgs gd = ga;
+    gd.sched = es.sched + 1;
+    gd.n_tiles = c.H / 256;
+    gd.num_kb = c.I / BK;
+    gd.b_rows_per_group = c.H;
+    gd.b_half = 0;
+    gd.out = nullptr;
+    gd.out_f32 = own.O;
+    gd.push_dst = es.push;
+    gd.ldo = c.H;
+
+    if (const cudaError_t e = cudaMemsetAsync(es.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
+    MOK_TRY(launch_k(ep_layout_kernel, dim3(1), dim3(256), 0, stream, "ep_layout_kernel", v, a));
+    MOK_TRY(launch_k(ep_rows_kernel, dim3(static_cast<unsigned>(c.E + c.n_shared * blocks_for(c.T, 256))), dim3(256), 0,
+                     stream, "ep_rows_kernel", v, a));
+    MOK_TRY(launch_k(ep_pull_kernel, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", v, a));
+    MOK_TRY(launch_gemm<typename FusedCfg<false>::GateUp>(gB, gB, gBs, gO, gO, gO, ga, dev.sms, stream));
+    return launch_gemm<typename FusedCfg<false>::Down>(dA, dB, dBs, dO, dO, dO, gd, dev.sms, stream);
+}
+
+PFN_cuMemGetAddressRange_v3020 g_addr_range = nullptr;
 
 }  // namespace
 }  // namespace mok
@@ -1515,6 +1678,119 @@ int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_
     if (!p) return MOK_ERR_UNSUPPORTED;
     if (offset) *offset = static_cast<size_t>(static_cast<const char *>(p) - base);
     if (bytes) *bytes = n;
+    return MOK_OK;
+}
+
+int moe_ep_size(const moe_cfg *cfg, int32_t world, size_t *state_bytes, size_t *scratch_bytes)
+{
+    MOK_TRY(check_ep(cfg, world, 0));
+    if (state_bytes) *state_bytes = carve_state(*cfg, nullptr, false).bytes;
+    if (scratch_bytes) *scratch_bytes = carve_ep(*cfg, world, nullptr).bytes;
+    return MOK_OK;
+}
+
+int moe_ep_route(const moe_cfg *cfg, int32_t world, int32_t rank, const void *x, const moe_params *params,
+                 void *state, size_t state_bytes, void *stream)
+{
+    MOK_TRY(check_ep(cfg, world, rank));
+    if (!params || !params->router_w || !aligned16(params->router_w)) return MOK_ERR_INVALID;
+    if (!x || !aligned16(x) || !state || !aligned16(state)) return MOK_ERR_INVALID;
+    if (state_bytes < carve_state(*cfg, nullptr, false).bytes) return MOK_ERR_WORKSPACE;
+    const DeviceInfo *dev = device_info();
+    if (!dev) return MOK_ERR_DEVICE;
+    return ep_route(*cfg, x, *params, carve_state(*cfg, state, false), *dev, static_cast<cudaStream_t>(stream));
+}
+
+int moe_ep_experts(const moe_cfg *cfg, int32_t world, int32_t rank, const void *const *x_ranks,
+                   void *const *state_ranks, const moe_params *params, void *scratch, size_t scratch_bytes,
+                   void *stream)
+{
+    MOK_TRY(check_ep(cfg, world, rank));
+    if (!params || !params->w_gate_up || !params->w_down || !x_ranks || !state_ranks) return MOK_ERR_INVALID;
+    if (cfg->n_shared > 0 && (!params->ws_gate_up || !params->ws_down)) return MOK_ERR_INVALID;
+    const void *w[] = {params->w_gate_up, params->w_down, params->ws_gate_up, params->ws_down};
+    for (const void *q : w)
+        if (q && !aligned16(q)) return MOK_ERR_INVALID;
+    for (int r = 0; r < world; ++r)
+        if (!x_ranks[r] || !state_ranks[r] || !aligned16(x_ranks[r]) || !aligned16(state_ranks[r]))
+            return MOK_ERR_INVALID;
+    if (!scratch || !aligned16(scratch)) return MOK_ERR_INVALID;
+    const EpScratch need = carve_ep(*cfg, world, nullptr);
+    if (scratch_bytes < need.bytes) return MOK_ERR_WORKSPACE;
+    const DeviceInfo *dev = device_info();
+    if (!dev) return MOK_ERR_DEVICE;
+    return ep_experts(*cfg, world, rank, x_ranks, state_ranks, *params, carve_ep(*cfg, world, scratch), *dev,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int moe_ep_combine(const moe_cfg *cfg, int32_t world, int32_t rank, const void *state, void *y, void *stream)
+{
+    MOK_TRY(check_ep(cfg, world, rank));
+    if (!state || !aligned16(state) || !y || !aligned16(y)) return MOK_ERR_INVALID;
+    const DeviceInfo *dev = device_info();
+    if (!dev) return MOK_ERR_DEVICE;
+    t_launches = 0;
+    t_pdl = false;
+    const State st = carve_state(*cfg, const_cast<void *>(state), false);
+    const Shapes s = shapes(*cfg);
+    return launch_k(combine_kernel<float>, dim3(blocks_for(s.T * s.H / 8, 256)), dim3(256), 0,
+                    static_cast<cudaStream_t>(stream), "combine_kernel", static_cast<const float *>(st.O),
+                    static_cast<const float *>(st.topk_w), static_cast<__nv_bfloat16 *>(y), cfg->T, cfg->H,
+                    cfg->top_k, cfg->n_shared);
+}
+
+static int ep_alloc_base(const void *dev_ptr, char **base)
+{
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!g_addr_range) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+                q == cudaDriverEntryPointSuccess)
+                g_addr_range = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fn);
+        }
+    }
+    if (!g_addr_range) return fail(MOK_ERR_DEVICE, "cuMemGetAddressRange not available");
+    CUdeviceptr b = 0;
+    size_t n = 0;
+    if (g_addr_range(&b, &n, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+        return fail(MOK_ERR_INVALID, "cuMemGetAddressRange: not a device allocation");
+    *base = reinterpret_cast<char *>(b);
+    return MOK_OK;
+}
+
+int moe_ep_ipc_handle(const void *dev_ptr, void *handle, size_t *offset)
+{
+    if (!dev_ptr || !handle || !offset) return MOK_ERR_INVALID;
+    static_assert(sizeof(cudaIpcMemHandle_t) == MOK_EP_IPC_HANDLE_BYTES, "IPC handle size");
+    char *base = nullptr;
+    MOK_TRY(ep_alloc_base(dev_ptr, &base));
+    cudaIpcMemHandle_t h;
+    if (const cudaError_t e = cudaIpcGetMemHandle(&h, base); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaIpcGetMemHandle", e);
+    std::memcpy(handle, &h, sizeof(h));
+    *offset = static_cast<size_t>(static_cast<const char *>(dev_ptr) - base);
+    return MOK_OK;
+}
+
+int moe_ep_ipc_open(const void *handle, size_t offset, void **dev_ptr)
+{
+    if (!handle || !dev_ptr) return MOK_ERR_INVALID;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    void *base = nullptr;
+    if (const cudaError_t e = cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaIpcOpenMemHandle", e);
+    *dev_ptr = static_cast<char *>(base) + offset;
+    return MOK_OK;
+}
+
+int moe_ep_ipc_close(void *dev_ptr, size_t offset)
+{
+    if (!dev_ptr) return MOK_ERR_INVALID;
+    if (const cudaError_t e = cudaIpcCloseMemHandle(static_cast<char *>(dev_ptr) - offset); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaIpcCloseMemHandle", e);
     return MOK_OK;
 }
 

@@ -29,6 +29,17 @@ def cfg_for(wl, dtype=None) -> abi.moe_cfg:
                     wl.topk_group, wl.routed_scale, dtype)
 
 
+def make_params(p: dict) -> abi.moe_params:
+    """C parameter record of a dict of device tensors (missing keys: NULL)."""
+    return abi.moe_params(
+        _ptr(p.get("router_w")), _ptr(p.get("e_bias")), _ptr(p.get("logit_bias")),
+        _ptr(p.get("w_gate_up")), _ptr(p.get("w_down")), _ptr(p.get("s_gate_up")), _ptr(p.get("s_down")),
+        _ptr(p.get("ws_gate_up")), _ptr(p.get("ws_down")), _ptr(p.get("ss_gate_up")),
+        _ptr(p.get("ss_down")), _ptr(p.get("wt_gate_up")), _ptr(p.get("wt_down")),
+        _ptr(p.get("st_gate_up")), _ptr(p.get("st_down")), _ptr(p.get("wst_gate_up")),
+        _ptr(p.get("wst_down")), _ptr(p.get("sst_gate_up")), _ptr(p.get("sst_down")))
+
+
 class MoELayer:
     """One layer's parameters plus the buffers the C ABI needs.
 
@@ -49,14 +60,7 @@ class MoELayer:
                                    device=self.device)
         self.bwd_scratch = torch.empty(self.bwd_bytes if training else 0, dtype=torch.uint8,
                                        device=self.device)
-        p = params
-        self.cparams = abi.moe_params(
-            _ptr(p["router_w"]), _ptr(p.get("e_bias")), _ptr(p.get("logit_bias")),
-            _ptr(p["w_gate_up"]), _ptr(p["w_down"]), _ptr(p.get("s_gate_up")), _ptr(p.get("s_down")),
-            _ptr(p.get("ws_gate_up")), _ptr(p.get("ws_down")), _ptr(p.get("ss_gate_up")),
-            _ptr(p.get("ss_down")), _ptr(p.get("wt_gate_up")), _ptr(p.get("wt_down")),
-            _ptr(p.get("st_gate_up")), _ptr(p.get("st_down")), _ptr(p.get("wst_gate_up")),
-            _ptr(p.get("wst_down")), _ptr(p.get("sst_gate_up")), _ptr(p.get("sst_down")))
+        self.cparams = make_params(params)
 
     def stream(self):
         return torch.cuda.current_stream(self.device).cuda_stream

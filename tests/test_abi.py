@@ -103,3 +103,57 @@ def test_pipelined_host_step_argument_checks():
     with pytest.raises(abi.MokError) as ei:
         abi.moe_step_host_async(c, 16, None, 16, p, 16, 16, 16, 0, g, 16, n3 - 1, None)
     assert ei.value.code == abi.MOK_ERR_WORKSPACE
+
+
+def test_expert_parallel_sizes_and_argument_checks():
+    """moe_ep_size gives the per-rank state (the forward scratch: routing record and
+    slot rows) and a receive scratch sized for the largest share a rank can get
+    (world T min(k, E/world) routed rows plus the shared rows); the EP calls refuse
+    bad ranks, an E that world does not divide, MXFP8, row codes past 24 bits, NULL
+    or short buffers -- all before touching a device (no pointer is dereferenced)."""
+    T, H, E, I, k, W = 512, 7168, 256, 2048, 8, 8
+    c = make_cfg(T, H, E, I, k, 1, I, 1, 8, 4)
+    state, scratch = abi.moe_ep_size(c, W)
+    assert state == abi.moe_workspace_size(c)[1]
+    rr = W * T * min(k, E // W)
+    rows = rr + T
+    assert scratch >= (T + rr) * H * 2 + rows * I * 2 + rows * 16
+    # E/world < k: a token puts at most E/world of its k slots on one rank
+    c2 = make_cfg(200, 256, 8, 128, 2)
+    _, s8 = abi.moe_ep_size(c2, 8)
+    _, s1 = abi.moe_ep_size(c2, 1)
+    assert s8 >= (200 + 8 * 200 * 1) * 256 * 2 and s1 >= (200 + 200 * 2) * 256 * 2
+    for world, cfg, code in ((0, c, abi.MOK_ERR_INVALID), (9, c, abi.MOK_ERR_INVALID),
+                             (3, make_cfg(64, 256, 8, 128, 2), abi.MOK_ERR_INVALID),
+                             (2, make_cfg(64, 256, 8, 128, 2, dtype=abi.MOK_DTYPE_MXFP8), abi.MOK_ERR_UNSUPPORTED),
+                             (2, make_cfg(1 << 21, 256, 8, 128, 8), abi.MOK_ERR_INVALID)):
+        with pytest.raises(abi.MokError) as ei:
+            abi.moe_ep_size(cfg, world)
+        assert ei.value.code == code, (world, code)
+    small = make_cfg(64, 256, 8, 128, 2)
+    st, sc = abi.moe_ep_size(small, 2)
+    p = abi.moe_params(router_w=16, w_gate_up=16, w_down=16)
+    for rank in (-1, 2):
+        with pytest.raises(abi.MokError) as ei:
+            abi.moe_ep_route(small, 2, rank, 16, p, 16, st, None)
+        assert ei.value.code == abi.MOK_ERR_INVALID
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_route(small, 2, 0, 16, p, 16, st - 1, None)
+    assert ei.value.code == abi.MOK_ERR_WORKSPACE
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_route(small, 2, 0, None, p, 16, st, None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_experts(small, 2, 0, [16, 16], [16, 16], p, 16, sc - 1, None)
+    assert ei.value.code == abi.MOK_ERR_WORKSPACE
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_experts(small, 2, 0, [16, None], [16, 16], p, 16, sc, None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_combine(small, 2, 0, 16, None, None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_ipc_handle(None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
+    with pytest.raises(ValueError):
+        abi.moe_ep_ipc_open(b"short", 0)
