@@ -461,61 +461,90 @@ const char *moe_strerror(int code);
  * thread's next failing call. */
 const char *moe_last_error(void);
 
-/* ---- expert parallelism (forward) ------------------------------------------
+/* ---- expert parallelism ------------------------------------------------------
  * "Cursor åpner megakernelen…" (the pull-versus-push paragraph) and
  * "Megakernels are dead and back…" ("Números de MoK"): experts are spread over
  * `world` ranks (one GPU each); the rank that owns an expert pulls the token
  * rows routed to it from the ranks that hold them and pushes every expert
- * output row back to its token's rank, where the fixed-order k-sum runs.
+ * output row back to its token's rank, where the fixed-order k-sum runs.  The
+ * backward mirrors it: the owner pulls dy rows the same way and pushes the dX
+ * rows and the slot-gradient partials of each routed row back to its token's
+ * rank; the weight gradients of an expert are computed whole on its owner.
  *
  * cfg describes the whole layer: E counts every routed expert and must be a
  * multiple of world (1 <= world <= MOK_EP_MAX_RANKS); T is the tokens of ONE
  * rank.  Rank r holds its own T tokens and owns the routed experts
- * [r E/world, (r+1) E/world); the shared experts run on every rank for its own
- * tokens.  BF16 only (MOK_ERR_UNSUPPORTED for MXFP8); T (top_k + n_shared)
- * must stay below 2^24.
+ * [r E/world, (r+1) E/world); the router and the shared experts run on every
+ * rank for its own tokens.  BF16 only (MOK_ERR_UNSUPPORTED for MXFP8); T
+ * (top_k + n_shared) must stay below 2^24.
  *
- * Buffers (caller-allocated device memory, 16-byte aligned):
+ * Buffers (caller-allocated device memory, 16-byte aligned), from moe_ep_size:
  *   state    per rank, state_bytes: the rank's routing record and its fp32 slot
  *            rows.  Other ranks read the routing record and write slot rows.
- *   scratch  per rank, scratch_bytes: the rows the rank receives (x rows and
- *            the expert rows' h), sized for the largest possible share,
- *            world T min(top_k, E/world) routed rows.
+ *   scratch  per rank, scratch_bytes: the rows the rank receives (x rows, h and,
+ *            when training, g/u, w h, the pulled dy rows and dGU), sized for the
+ *            largest possible share, world T min(top_k, E/world) routed rows.
+ *            A training forward's scratch is read by that rank's backward.
+ *   bwd      per rank, bwd_bytes (backward only): the dX slot rows and
+ *            slot-gradient partials other ranks write, and the rank's dl and
+ *            router-gradient partial sums.
  *
- * A forward step is three calls on every rank; every rank's call of one phase
- * must be complete before any rank starts the next phase.  On one device (ranks
- * emulated by separate buffer sets) that is the calls in this order on one
- * stream; on several GPUs, a device-side barrier between the phases (for
- * example a one-element NCCL all-reduce on the same stream, which ends on
- * every rank only after every rank's earlier kernels):
+ * A step is a sequence of phases; every rank's call of one phase must be
+ * complete before any rank starts the next.  On one device (ranks emulated by
+ * separate buffer sets) that is the calls in this order on one stream; on
+ * several GPUs, a device-side barrier between the phases (for example a
+ * one-element NCCL all-reduce on the same stream, which ends on every rank only
+ * after every rank's earlier kernels).  Forward:
  *   moe_ep_route    router logits, top-k and dispatch of the rank's tokens into
  *                   its state (params: router_w, e_bias, logit_bias).
  *   moe_ep_experts  the owner's sorted rows from every rank's routing record,
  *                   the pull of those token rows into its scratch (one plain
  *                   16-byte-load copy; every remote row crosses the link once),
- *                   the gate/up GEMM with SwiGLU, and the down GEMM whose
- *                   epilogue stores each fp32 output row into the slot row of
- *                   the token's rank through that rank's state pointer.
- *                   x_ranks[s] and state_ranks[s] (s < world) are rank s's x and
- *                   state as this device addresses them (its own buffers, or
- *                   peer mappings: moe_ep_ipc_*); params: w_gate_up [E/world,
- *                   2I, H] and w_down [E/world, H, I] of the rank's experts,
- *                   ws_* of the shared experts.
+ *                   the gate/up GEMM with SwiGLU (training: also g/u and w h),
+ *                   and the down GEMM whose epilogue stores each fp32 output row
+ *                   into the slot row of the token's rank through that rank's
+ *                   state pointer.  x_ranks[s] and state_ranks[s] (s < world) are
+ *                   rank s's x and state as this device addresses them (its own
+ *                   buffers, or peer mappings: moe_ep_ipc_*); params: w_gate_up
+ *                   [E/world, 2I, H] and w_down [E/world, H, I] of the rank's
+ *                   experts, ws_* of the shared experts.
  *   moe_ep_combine  y = the fixed-order sum of the rank's slot rows.
- * Each rank's y equals moe_fwd of its T tokens with all E experts, byte for
- * byte.  A routing record that would overflow the receive buffers (impossible
- * for one written by moe_ep_route) records MOK_STATUS_BAD_INDEX and is treated
- * as empty.  The same buffers must not be used by two steps at once.
+ * Backward (after a forward with training != 0 on the same buffers):
+ *   moe_ep_bwd_experts  the owner pulls the dy rows of its rows from dy_ranks[s],
+ *                   runs the down dgrad (SwiGLU backward) and pushes each routed
+ *                   row's slot-gradient partials into bwd_ranks[s], runs the
+ *                   gate/up dgrad whose epilogue stores each fp32 dX row into the
+ *                   dX slot row of the token's rank, and the weight gradients:
+ *                   grads->dw_gate_up [E/world, 2I, H] and dw_down [E/world, H, I]
+ *                   of its experts (over every rank's rows), dws_* the shared
+ *                   experts' gradient over this rank's tokens.
+ *   moe_ep_bwd_combine  slot gradients, grads->drouter_w (over this rank's
+ *                   tokens) and grads->dx of the rank's tokens.
+ * Each rank's y and dx equal moe_fwd / moe_bwd of its T tokens with all E
+ * experts, byte for byte, and so do its drouter_w and dws_* (the router and the
+ * shared experts are replicated: their full gradients are the sums over ranks,
+ * as for data-parallel replicas).  An owner's dw_* equal moe_bwd's rows of its
+ * experts on the concatenation of every rank's tokens when that batch routes its
+ * tokens the same way.  A routing record that would overflow the receive
+ * buffers (impossible for one written by moe_ep_route) records
+ * MOK_STATUS_BAD_INDEX and is treated as empty.  The same buffers must not be
+ * used by two steps at once.
  */
 #define MOK_EP_MAX_RANKS 8
 #define MOK_EP_IPC_HANDLE_BYTES 64
-int moe_ep_size(const moe_cfg *cfg, int32_t world, size_t *state_bytes, size_t *scratch_bytes);
+int moe_ep_size(const moe_cfg *cfg, int32_t world, int32_t training, size_t *state_bytes, size_t *scratch_bytes,
+                size_t *bwd_bytes);
 int moe_ep_route(const moe_cfg *cfg, int32_t world, int32_t rank, const void *x, const moe_params *params,
                  void *state, size_t state_bytes, void *stream);
-int moe_ep_experts(const moe_cfg *cfg, int32_t world, int32_t rank, const void *const *x_ranks,
+int moe_ep_experts(const moe_cfg *cfg, int32_t world, int32_t rank, int32_t training, const void *const *x_ranks,
                    void *const *state_ranks, const moe_params *params, void *scratch, size_t scratch_bytes,
                    void *stream);
 int moe_ep_combine(const moe_cfg *cfg, int32_t world, int32_t rank, const void *state, void *y, void *stream);
+int moe_ep_bwd_experts(const moe_cfg *cfg, int32_t world, int32_t rank, const void *const *dy_ranks,
+                       void *const *bwd_ranks, const moe_params *params, const moe_grads *grads, void *scratch,
+                       size_t scratch_bytes, void *stream);
+int moe_ep_bwd_combine(const moe_cfg *cfg, int32_t world, int32_t rank, const void *x, const moe_params *params,
+                       const void *state, void *bwd, size_t bwd_bytes, const moe_grads *grads, void *stream);
 
 /* Peer mappings for moe_ep_experts across processes on one node.
  * moe_ep_ipc_handle writes into `handle` (MOK_EP_IPC_HANDLE_BYTES bytes) the

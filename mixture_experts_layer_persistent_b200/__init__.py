@@ -10,7 +10,7 @@ from .abi import (MOK_DTYPE_BF16, MOK_DTYPE_MXFP8, MOK_SCORE_SIGMOID, MOK_SCORE_
                   moe_host_scratch_size, moe_params, moe_quantize_mxfp8, moe_quantize_mxfp8_weights,
                   moe_quantize_mxfp8_weights_both, moe_quantize_mxfp8_weights_t, moe_routing, moe_status, moe_strerror, moe_trace_events,
                   moe_workspace_size)
-from .ep import EPRank, EPWorld, exchange_pointers, split_params
+from .ep import EPRank, EPWorld, exchange_pointers, new_rank_grads, split_params
 from .layer import (MoELayer, cfg_for, make_cfg, quantize_mxfp8, quantize_mxfp8_weights,
                     quantize_mxfp8_weights_both, quantize_mxfp8_weights_t)
 
@@ -21,5 +21,5 @@ __all__ = [
     "moe_quantize_mxfp8_weights_both", "moe_quantize_mxfp8_weights_t", "moe_routing", "moe_status", "moe_strerror", "moe_trace_events",
     "moe_workspace_size", "MoELayer", "cfg_for", "make_cfg", "quantize_mxfp8", "quantize_mxfp8_weights",
     "quantize_mxfp8_weights_both", "quantize_mxfp8_weights_t", "EPRank", "EPWorld", "exchange_pointers",
-    "split_params",
+    "new_rank_grads", "split_params",
 ]

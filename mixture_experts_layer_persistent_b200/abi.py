@@ -110,10 +110,14 @@ def lib():
         L.moe_set_schedule.argtypes = [ctypes.c_int]
         L.moe_get_schedule.argtypes = [P(_i32)]
         L.moe_trace_device.argtypes = [_vp, _sz, _vp, _sz]
-        L.moe_ep_size.argtypes = [P(moe_cfg), _i32, P(_sz), P(_sz)]
+        L.moe_ep_size.argtypes = [P(moe_cfg), _i32, _i32, P(_sz), P(_sz), P(_sz)]
         L.moe_ep_route.argtypes = [P(moe_cfg), _i32, _i32, _vp, P(moe_params), _vp, _sz, _vp]
-        L.moe_ep_experts.argtypes = [P(moe_cfg), _i32, _i32, P(_vp), P(_vp), P(moe_params), _vp, _sz, _vp]
+        L.moe_ep_experts.argtypes = [P(moe_cfg), _i32, _i32, _i32, P(_vp), P(_vp), P(moe_params), _vp, _sz, _vp]
         L.moe_ep_combine.argtypes = [P(moe_cfg), _i32, _i32, _vp, _vp, _vp]
+        L.moe_ep_bwd_experts.argtypes = [P(moe_cfg), _i32, _i32, P(_vp), P(_vp), P(moe_params), P(moe_grads), _vp,
+                                         _sz, _vp]
+        L.moe_ep_bwd_combine.argtypes = [P(moe_cfg), _i32, _i32, _vp, P(moe_params), _vp, _vp, _sz, P(moe_grads),
+                                         _vp]
         L.moe_ep_ipc_handle.argtypes = [_vp, _vp, P(_sz)]
         L.moe_ep_ipc_open.argtypes = [_vp, _sz, P(_vp)]
         L.moe_ep_ipc_close.argtypes = [_vp, _sz]
@@ -127,7 +131,8 @@ def lib():
                      "moe_quantize_mxfp8_weights_t", "moe_quantize_mxfp8_weights_both", "moe_status",
                      "moe_trace_events", "moe_fwd_static", "moe_test_drop_signal", "moe_saved_tensor",
                      "moe_set_schedule", "moe_get_schedule", "moe_trace_device", "moe_ep_size", "moe_ep_route",
-                     "moe_ep_experts", "moe_ep_combine", "moe_ep_ipc_handle", "moe_ep_ipc_open",
+                     "moe_ep_experts", "moe_ep_combine", "moe_ep_bwd_experts", "moe_ep_bwd_combine",
+                     "moe_ep_ipc_handle", "moe_ep_ipc_open",
                      "moe_ep_ipc_close"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -274,11 +279,12 @@ def moe_test_drop_signal(enable: bool):
     _check("moe_test_drop_signal", lib().moe_test_drop_signal(int(enable)))
 
 
-def moe_ep_size(cfg: moe_cfg, world: int):
-    """(state_bytes, scratch_bytes) of one rank of an expert-parallel forward."""
-    a, b = _sz(), _sz()
-    _check("moe_ep_size", lib().moe_ep_size(ctypes.byref(cfg), int(world), ctypes.byref(a), ctypes.byref(b)))
-    return a.value, b.value
+def moe_ep_size(cfg: moe_cfg, world: int, training: bool = False):
+    """(state_bytes, scratch_bytes, bwd_bytes) of one rank of an expert-parallel layer."""
+    a, b, c = _sz(), _sz(), _sz()
+    _check("moe_ep_size", lib().moe_ep_size(ctypes.byref(cfg), int(world), int(training), ctypes.byref(a),
+                                            ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
 
 
 def moe_ep_route(cfg, world, rank, x, params, state, state_bytes, stream):
@@ -286,11 +292,25 @@ def moe_ep_route(cfg, world, rank, x, params, state, state_bytes, stream):
                                               state, state_bytes, stream))
 
 
-def moe_ep_experts(cfg, world, rank, x_ranks, state_ranks, params, scratch, scratch_bytes, stream):
+def moe_ep_experts(cfg, world, rank, training, x_ranks, state_ranks, params, scratch, scratch_bytes, stream):
     xs = (_vp * len(x_ranks))(*x_ranks)
     ss = (_vp * len(state_ranks))(*state_ranks)
-    _check("moe_ep_experts", lib().moe_ep_experts(ctypes.byref(cfg), int(world), int(rank), xs, ss,
+    _check("moe_ep_experts", lib().moe_ep_experts(ctypes.byref(cfg), int(world), int(rank), int(training), xs, ss,
                                                   ctypes.byref(params), scratch, scratch_bytes, stream))
+
+
+def moe_ep_bwd_experts(cfg, world, rank, dy_ranks, bwd_ranks, params, grads, scratch, scratch_bytes, stream):
+    ds = (_vp * len(dy_ranks))(*dy_ranks)
+    bs = (_vp * len(bwd_ranks))(*bwd_ranks)
+    _check("moe_ep_bwd_experts", lib().moe_ep_bwd_experts(ctypes.byref(cfg), int(world), int(rank), ds, bs,
+                                                          ctypes.byref(params), ctypes.byref(grads), scratch,
+                                                          scratch_bytes, stream))
+
+
+def moe_ep_bwd_combine(cfg, world, rank, x, params, state, bwd, bwd_bytes, grads, stream):
+    _check("moe_ep_bwd_combine", lib().moe_ep_bwd_combine(ctypes.byref(cfg), int(world), int(rank), x,
+                                                          ctypes.byref(params), state, bwd, bwd_bytes,
+                                                          ctypes.byref(grads), stream))
 
 
 def moe_ep_combine(cfg, world, rank, state, y, stream):

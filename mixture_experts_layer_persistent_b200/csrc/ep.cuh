@@ -32,6 +32,7 @@ constexpr int kEpMaxRanks = MOK_EP_MAX_RANKS;
 // Row codes that cross ranks: (rank << kEpRankShift) | row on that rank
 constexpr int kEpRankShift = 24;
 constexpr int kEpRowMask = (1 << kEpRankShift) - 1;
+constexpr int kEpMaxGroups = 256 + 4;   // routed experts of one rank + shared experts
 
 // Every rank's routing record and slot rows, as this device addresses them.
 struct EpView {
@@ -52,7 +53,9 @@ struct EpArgs {
     int *row_token;        // [rows] row of x_recv each sorted row reads
     int *row_src;          // [rows] (source rank << 24) | token
     int *row_slot;         // [rows] (source rank << 24) | slot row t (k + S) + slot in that rank's O
+    int *row_gdst;         // [routed rows] (source rank << 24) | the row's position in the source's sorted rows
     float *row_w;          // [rows] routing weight (1 for shared rows)
+    int *gorder;           // [E_loc + S] the owner's groups by rows descending, index ascending
     float **push;          // [kEpMaxRanks] slot rows of every rank, for the push epilogue
     __nv_bfloat16 *x_recv; // [T + rr_cap, H] the owner's own tokens, then every received row
     int *status;
@@ -99,6 +102,20 @@ __global__ void __launch_bounds__(256) ep_layout_kernel(EpView v, EpArgs a)
     if (i < n && i % a.world == 0) a.offsets[i / a.world] = excl;
     if (i <= a.S) a.offsets[a.E_loc + i] = total + i * a.T;
     if (i < a.world) a.push[i] = v.O[i];
+    // longest-first group order of the weight gradients (ties: lower index first)
+    __shared__ int s_rows[kEpMaxGroups];
+    const int G = a.E_loc + a.S;
+    for (int g = i; g < G; g += blockDim.x) {
+        int rows = a.T;                                      // a shared group: the owner's T tokens
+        if (g < a.E_loc) rows = ok ? s_scan[(g + 1) * a.world - 1] - (g ? s_scan[g * a.world - 1] : 0) : 0;
+        s_rows[g] = rows;
+    }
+    __syncthreads();
+    for (int g = i; g < G; g += blockDim.x) {
+        int rank = 0;
+        for (int h = 0; h < G; ++h) rank += s_rows[h] > s_rows[g] || (s_rows[h] == s_rows[g] && h < g);
+        a.gorder[rank] = g;
+    }
 }
 
 // Sorted rows of the owner.  Blocks [0, n): segment b = (expert j, source s)
@@ -130,6 +147,7 @@ __global__ void __launch_bounds__(256) ep_rows_kernel(EpView v, EpArgs a)
             a.row_token[r] = a.T + r;
             a.row_src[r] = (s << kEpRankShift) | t;
             a.row_slot[r] = (s << kEpRankShift) | (t * a.kk + slot);
+            a.row_gdst[r] = (s << kEpRankShift) | (range_ok ? src0 + i : 0);
             a.row_w[r] = range_ok ? v.topk_w[s][q] : 0.0f;
         }
     } else {
@@ -181,6 +199,36 @@ __global__ void __launch_bounds__(256) ep_pull_kernel(EpView v, EpArgs a)
             for (int u = 0; u < 4; ++u)
                 if (c + 32 * u < vec) d4[c + 32 * u] = q[u];
         }
+    }
+}
+
+// Per-rank pointer table in device memory (the push epilogues read it).
+struct EpTable {
+    float *p[kEpMaxRanks];
+};
+__global__ void ep_table_kernel(EpTable t, float **dst, int n)
+{
+    if (threadIdx.x < n) dst[threadIdx.x] = t.p[threadIdx.x];
+}
+
+// Backward: the slot-gradient partials <dy W_down, h> of every routed row the
+// owner computed (nt floats per row, its down dgrad's N tiles) go to the row's
+// source rank, at the row's position in the source's sorted rows, where the
+// slot gradients are formed.  One thread per (row, tile).
+__global__ void __launch_bounds__(256) ep_push_gpart_kernel(const float *gpart, const int *row_gdst, const int *seg,
+                                                            int n_seg, int nt, float **gdst, int world, int tk,
+                                                            int *status)
+{
+    const long long n = static_cast<long long>(seg[n_seg]) * nt;
+    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += static_cast<long long>(gridDim.x) * 256) {
+        const int r = static_cast<int>(i / nt), j = static_cast<int>(i - static_cast<long long>(r) * nt);
+        const int code = row_gdst[r];
+        const int s = code >> kEpRankShift, q = code & kEpRowMask;
+        if (s < 0 || s >= world || q >= tk) {       // never written so by ep_rows_kernel
+            atomicOr(status, MOK_STATUS_BAD_INDEX);
+            continue;
+        }
+        gdst[s][static_cast<size_t>(q) * nt + j] = gpart[i];
     }
 }
 

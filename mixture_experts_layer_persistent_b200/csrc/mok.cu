@@ -1047,16 +1047,21 @@ int check_params(const moe_cfg &c, const moe_params *p)
 // pulled and the h of those rows, sized for the largest share it can receive
 // (every token of every rank choosing min(k, E_loc) of its experts).
 struct EpScratch {
-    int *seg, *offsets, *row_token, *row_src, *row_slot;
+    int *seg, *offsets, *gorder, *row_token, *row_src, *row_slot, *row_gdst;
     float *row_w;
-    float **push;
+    float **push;                   // [kEpMaxRanks] every rank's fp32 slot rows (forward push)
+    float **push_dx;                // [kEpMaxRanks] every rank's fp32 dX slot rows (backward push)
+    float **push_g;                 // [kEpMaxRanks] every rank's slot-gradient partials
     int *sched;
     __nv_bfloat16 *x_recv, *h;
+    __nv_bfloat16 *gu, *hw;         // training: saved g/u and w h of the owner's rows
+    __nv_bfloat16 *dy_recv, *dgu;   // training: pulled dy rows, dGU
+    float *gpart;                   // training: slot-gradient partials of the owner's routed rows
     long long rr_cap, rows_cap;
     size_t bytes;
 };
 
-EpScratch carve_ep(const moe_cfg &c, int world, void *buf)
+EpScratch carve_ep(const moe_cfg &c, int world, bool training, void *buf)
 {
     const Shapes s = shapes(c);
     const long long el = s.E / world;
@@ -1066,16 +1071,48 @@ EpScratch carve_ep(const moe_cfg &c, int world, void *buf)
     Carver cv(buf);
     e.seg = cv.take<int>(s.E + 1);
     e.offsets = cv.take<int>(el + s.S + 1);
+    e.gorder = cv.take<int>(el + s.S);
     e.row_token = cv.take<int>(e.rows_cap);
     e.row_src = cv.take<int>(e.rows_cap);
     e.row_slot = cv.take<int>(e.rows_cap);
+    e.row_gdst = cv.take<int>(e.rr_cap);
     e.row_w = cv.take<float>(e.rows_cap);
     e.push = cv.take<float *>(kEpMaxRanks);
+    e.push_dx = cv.take<float *>(kEpMaxRanks);
+    e.push_g = cv.take<float *>(kEpMaxRanks);
     e.sched = cv.take<int>(kSchedCounters);
     e.x_recv = cv.take<__nv_bfloat16>((s.T + e.rr_cap) * s.H);
     e.h = cv.take<__nv_bfloat16>(e.rows_cap * s.I);
+    if (training) {
+        e.gu = cv.take<__nv_bfloat16>(e.rows_cap * 2 * s.I);
+        e.hw = cv.take<__nv_bfloat16>(e.rows_cap * s.I);
+        e.dy_recv = cv.take<__nv_bfloat16>((s.T + e.rr_cap) * s.H);
+        e.dgu = cv.take<__nv_bfloat16>(e.rows_cap * 2 * s.I);
+        e.gpart = cv.take<float>(e.rr_cap * (s.I / 128));
+    }
     e.bytes = align_up(cv.off, 256);
     return e;
+}
+
+// A rank's buffer of the backward's token side: what the owners push to it (the
+// dX slot rows and the slot-gradient partials of its routed rows) and what it
+// computes from them.
+struct EpSrcBwd {
+    float *dl, *gpart, *partial, *dxs;
+    size_t bytes;
+};
+
+EpSrcBwd carve_ep_src_bwd(const moe_cfg &c, void *buf)
+{
+    const Shapes s = shapes(c);
+    Carver cv(buf);
+    EpSrcBwd b{};
+    b.dl = cv.take<float>(s.TK);
+    b.gpart = cv.take<float>(s.TK * (s.I / 128));
+    b.partial = cv.take<float>(s.max_chunks * s.H);
+    b.dxs = cv.take<float>(s.T * s.kk * s.H);
+    b.bytes = align_up(cv.off, 256);
+    return b;
 }
 
 int check_ep(const moe_cfg *c, int world, int rank)
@@ -1103,8 +1140,8 @@ int ep_route(const moe_cfg &c, const void *x, const moe_params &p, const State &
     return launch_dispatch(pl, stream);
 }
 
-int ep_experts(const moe_cfg &c, int world, int rank, const void *const *xr, void *const *sr, const moe_params &p,
-               const EpScratch &es, const DeviceInfo &dev, cudaStream_t stream)
+int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void *const *xr, void *const *sr,
+               const moe_params &p, const EpScratch &es, const DeviceInfo &dev, cudaStream_t stream)
 {
     t_launches = 0;
     t_pdl = false;
@@ -1126,15 +1163,18 @@ int ep_experts(const moe_cfg &c, int world, int rank, const void *const *xr, voi
     a.rr_cap = static_cast<int>(es.rr_cap);
     a.seg = es.seg; a.offsets = es.offsets;
     a.row_token = es.row_token; a.row_src = es.row_src; a.row_slot = es.row_slot; a.row_w = es.row_w;
+    a.row_gdst = es.row_gdst; a.gorder = es.gorder;
     a.push = es.push; a.x_recv = es.x_recv; a.status = dev.status;
 
     // tensor maps: the rank's experts, the shared experts, h, and its own slot rows
     // (the push epilogue stores through es.push instead; the map only has to exist)
     const State own = carve_state(c, sr[rank], false);
-    CUtensorMap gB, gBs, gO, dA, dB, dBs, dO;
+    CUtensorMap gB, gBs, gO, gO2, gO3, dA, dB, dBs, dO;
     if (!make_tmap(&gB, p.w_gate_up, s.H, el * 2 * s.I, BK, 128, 2) ||
         !make_tmap(&gBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : el) * 2 * s.I, BK, 128, 2) ||
         !make_tmap(&gO, es.h, s.I, es.rows_cap, 64, 32, 2) ||
+        !make_tmap(&gO2, training ? es.gu : es.h, training ? 2 * s.I : s.I, es.rows_cap, 64, 32, 2) ||
+        !make_tmap(&gO3, training ? es.hw : es.h, s.I, es.rows_cap, 64, 32, 2) ||
         !make_tmap(&dA, es.h, s.I, es.rows_cap, BK, 128, 2) ||
         !make_tmap(&dB, p.w_down, s.I, el * s.H, BK, 256, 2) ||
         !make_tmap(&dBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : el) * s.H, BK, 256, 2) ||
@@ -1156,6 +1196,8 @@ int ep_experts(const moe_cfg &c, int world, int rank, const void *const *xr, voi
     ga.gather_src = es.x_recv;
     ga.gather_ld = c.H;
     ga.out = es.h;
+    ga.out2 = training ? es.gu : nullptr;       // training: g/u and w h for the backward
+    ga.out3 = training ? es.hw : nullptr;
     ga.status = dev.status;
     GemmArgs gd = ga;
     gd.sched = es.sched + 1;
@@ -1164,6 +1206,7 @@ int ep_experts(const moe_cfg &c, int world, int rank, const void *const *xr, voi
     gd.b_rows_per_group = c.H;
     gd.b_half = 0;
     gd.out = nullptr;
+    gd.out2 = gd.out3 = nullptr;
     gd.out_f32 = own.O;
     gd.push_dst = es.push;
     gd.ldo = c.H;
@@ -1174,8 +1217,183 @@ int ep_experts(const moe_cfg &c, int world, int rank, const void *const *xr, voi
     MOK_TRY(launch_k(ep_rows_kernel, dim3(static_cast<unsigned>(c.E + c.n_shared * blocks_for(c.T, 256))), dim3(256), 0,
                      stream, "ep_rows_kernel", v, a));
     MOK_TRY(launch_k(ep_pull_kernel, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", v, a));
-    MOK_TRY(launch_gemm<typename FusedCfg<false>::GateUp>(gB, gB, gBs, gO, gO, gO, ga, dev.sms, stream));
+    MOK_TRY(launch_gemm<typename FusedCfg<false>::GateUp>(gB, gB, gBs, gO, gO2, gO3, ga, dev.sms, stream));
     return launch_gemm<typename FusedCfg<false>::Down>(dA, dB, dBs, dO, dO, dO, gd, dev.sms, stream);
+}
+
+// Backward, owner side: pull dy rows, down dgrad (SwiGLU backward, slot-gradient
+// partials pushed to the rows' ranks), gate/up dgrad (dX rows pushed into the
+// dX slot rows of the tokens' ranks), both weight gradients of the owner's experts
+// (and this rank's share of the shared experts'), from the rows the forward kept.
+int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr, void *const *br,
+                   const moe_params &p, const moe_grads &gr, const EpScratch &es, const DeviceInfo &dev,
+                   cudaStream_t stream)
+{
+    t_launches = 0;
+    t_pdl = false;
+    const Shapes s = shapes(c);
+    const int el = c.E / world;
+    const long long G = el + s.S;
+    const bool n256 = c.I % 256 == 0;
+    EpView v{};
+    EpTable tdx{}, tg{};
+    for (int r = 0; r < world; ++r) {
+        v.x[r] = static_cast<const __nv_bfloat16 *>(dyr[r]);
+        const EpSrcBwd q = carve_ep_src_bwd(c, br[r]);
+        tdx.p[r] = q.dxs;
+        tg.p[r] = q.gpart;
+    }
+    const EpSrcBwd own = carve_ep_src_bwd(c, br[rank]);
+    EpArgs a{};
+    a.world = world; a.rank = rank;
+    a.T = c.T; a.H = c.H; a.k = c.top_k; a.kk = static_cast<int>(s.kk); a.S = c.n_shared; a.E_loc = el;
+    a.rr_cap = static_cast<int>(es.rr_cap);
+    a.seg = es.seg; a.row_src = es.row_src;
+    a.x_recv = es.dy_recv; a.status = dev.status;
+
+    GemmArgs base{};
+    base.num_groups = static_cast<int>(G);
+    base.num_routed = el;
+    base.offsets = es.offsets;
+    base.gorder = es.gorder;
+    base.row_token = es.row_token;
+    base.row_slot = es.row_slot;
+    base.row_w = es.row_w;
+    base.inter = c.I;
+    base.gather_src = es.dy_recv;
+    base.gather_ld = c.H;
+    base.status = dev.status;
+
+    FusedBwdMaps m;
+    // down dgrad: dh = w (dy W_down), SwiGLU backward -> dGU, slot-gradient partials
+    if (!make_tmap(&m.d1B, p.w_down, s.I, el * s.H, 64, 64, 2) ||
+        !make_tmap(&m.d1Bs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : el) * s.H, 64, 64, 2) ||
+        !make_tmap(&m.d1O, es.dgu, 2 * s.I, es.rows_cap, 64, 32, 2))
+        return fail(MOK_ERR_INVALID, "tensor map (expert-parallel down dgrad)");
+    GemmArgs g1 = base;
+    g1.sched = es.sched + 2;
+    g1.num_kb = c.H / BK;
+    g1.b_rows_per_group = c.H;
+    g1.aux = es.gu;
+    g1.aux_h = es.h;
+    g1.gpart = es.gpart;
+    g1.out = es.dgu;
+    g1.n_tiles = n256 ? c.I / 256 : c.I / 128;
+
+    // down wgrad: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
+    if (!make_tmap(&m.w2O, gr.dw_down, s.I, el * s.H, 64, 32, 2) ||
+        !make_tmap(&m.w2O2, s.S ? gr.dws_down : gr.dw_down, s.I, (s.S ? s.S : el) * s.H, 64, 32, 2) ||
+        !make_tmap(&m.w2B, es.hw, s.I, es.rows_cap, 64, 64, 2))
+        return fail(MOK_ERR_INVALID, "tensor map (expert-parallel down wgrad)");
+    GemmArgs g2 = base;
+    g2.sched = es.sched + 3;
+    g2.m_tiles = c.H / 128;
+    g2.out = static_cast<__nv_bfloat16 *>(gr.dw_down);
+    g2.out_s = static_cast<__nv_bfloat16 *>(gr.dws_down);
+    g2.ldo = c.I;
+    g2.group_out_elems = s.H * s.I;
+    int g2_units = 0;
+    if (n256) {
+        g2.n_tiles = c.I / 256;
+        g2.k_split = kResidentRows;
+        g2.m_per_unit = resident_m_per_unit(g2.m_tiles);
+        g2_units = static_cast<int>(G * g2.n_tiles * ((g2.m_tiles + g2.m_per_unit - 1) / g2.m_per_unit));
+    } else {
+        g2.n_tiles = c.I / 128;
+    }
+    const long long t2 = G * g2.m_tiles * g2.n_tiles;
+    const int g2_grid = static_cast<int>(t2 < dev.sms ? t2 : dev.sms);
+
+    // gate/up dgrad: dX rows = dGU W_gate_up, pushed into the tokens' ranks
+    if (!make_tmap(&m.d3A, es.dgu, 2 * s.I, es.rows_cap, BK, 128, 2) ||
+        !make_tmap(&m.d3B, p.w_gate_up, s.H, el * 2 * s.I, 64, 64, 2) ||
+        !make_tmap(&m.d3Bs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : el) * 2 * s.I, 64, 64, 2) ||
+        !make_tmap(&m.d3O, own.dxs, s.H, s.T * s.kk, 32, 1, 4))
+        return fail(MOK_ERR_INVALID, "tensor map (expert-parallel gate/up dgrad)");
+    GemmArgs g3 = base;
+    g3.sched = es.sched + 4;
+    g3.n_tiles = c.H / 256;
+    g3.num_kb = 2 * c.I / BK;
+    g3.b_rows_per_group = 2 * c.I;
+    g3.out_f32 = own.dxs;
+    g3.push_dst = es.push_dx;
+    g3.ldo = c.H;
+
+    // gate/up wgrad: dW_gate_up[g] = sum_r dGU_r^T x[token r] (the pulled x rows)
+    if (!make_tmap(&m.w4A, es.dgu, 2 * s.I, es.rows_cap, 64, 64, 2) ||
+        !make_tmap(&m.w4O, gr.dw_gate_up, s.H, el * 2 * s.I, 64, 32, 2) ||
+        !make_tmap(&m.w4O2, s.S ? gr.dws_gate_up : gr.dw_gate_up, s.H, (s.S ? s.S : el) * 2 * s.I, 64, 32, 2))
+        return fail(MOK_ERR_INVALID, "tensor map (expert-parallel gate/up wgrad)");
+    GemmArgs g4 = base;
+    g4.sched = es.sched + 5;
+    g4.gather_src = es.x_recv;
+    g4.m_tiles = 2 * c.I / 128;
+    g4.n_tiles = c.H / 256;
+    g4.out = static_cast<__nv_bfloat16 *>(gr.dw_gate_up);
+    g4.out_s = static_cast<__nv_bfloat16 *>(gr.dws_gate_up);
+    g4.ldo = c.H;
+    g4.group_out_elems = 2 * s.I * s.H;
+    g4.k_split = kResidentRows;
+    g4.m_per_unit = resident_m_per_unit(g4.m_tiles);
+    const long long t4 = G * g4.m_tiles * g4.n_tiles;
+    const int g4_grid = static_cast<int>(t4 < dev.sms ? t4 : dev.sms);
+    const int g4_units = static_cast<int>(G * g4.n_tiles * ((g4.m_tiles + g4.m_per_unit - 1) / g4.m_per_unit));
+
+    if (const cudaError_t e = cudaMemsetAsync(es.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
+    MOK_TRY(launch_k(ep_table_kernel, dim3(1), dim3(32), 0, stream, "ep_table_kernel", tdx, es.push_dx, world));
+    MOK_TRY(launch_k(ep_table_kernel, dim3(1), dim3(32), 0, stream, "ep_table_kernel", tg, es.push_g, world));
+    MOK_TRY(launch_k(ep_pull_kernel, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", v, a));
+    if (n256)
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradDown>(m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1,
+                                                                  dev.sms, stream));
+    else
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<false>::DgradDown>(m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1,
+                                                                   dev.sms, stream));
+    MOK_TRY(launch_k(ep_push_gpart_kernel, dim3(dev.sms), dim3(256), 0, stream, "ep_push_gpart_kernel",
+                     static_cast<const float *>(es.gpart), static_cast<const int *>(es.row_gdst),
+                     static_cast<const int *>(es.seg), c.E, g1.n_tiles, es.push_g, world, c.T * c.top_k, dev.status));
+    if (n256) {
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::WgradDown>(m.w2B, m.w2B, m.w2B, m.w2O, m.w2O2, m.w2O, g2,
+                                                                  g2_grid, stream));
+        MOK_TRY(launch_wgrad_resident<WgradResCfg<true>>(m.w2B, m.w2B, m.w2O, m.w2O2, g2,
+                                                         g2_units < dev.sms ? g2_units : dev.sms, stream));
+    } else {
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<false>::WgradDown>(m.w2B, m.w2B, m.w2B, m.w2O, m.w2O2, m.w2O, g2,
+                                                                   g2_grid, stream));
+    }
+    MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradGU>(m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O, g3, dev.sms,
+                                                            stream));
+    MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::WgradGU>(m.w4A, m.w4A, m.w4A, m.w4O, m.w4O2, m.w4O, g4, g4_grid,
+                                                            stream));
+    return launch_wgrad_resident<WgradResCfg<false>>(m.w4A, m.w4A, m.w4O, m.w4O2, g4,
+                                                     g4_units < dev.sms ? g4_units : dev.sms, stream);
+}
+
+// Backward, token side: slot gradients from the partials the owners pushed, the
+// router gradient of this rank's tokens, dx from the dX slot rows they pushed.
+int ep_bwd_combine(const moe_cfg &c, const void *x, const moe_params &p, const State &st, const EpSrcBwd &b,
+                   const moe_grads &gr, const DeviceInfo &dev, cudaStream_t stream)
+{
+    t_launches = 0;
+    t_pdl = false;
+    const Shapes s = shapes(c);
+    const int n_parts = c.I % 256 == 0 ? c.I / 256 : c.I / 128;
+    MOK_TRY(launch_k(slot_grad_kernel, dim3(blocks_for(s.T, 256)), dim3(256), 0, stream, "slot_grad_kernel",
+                     static_cast<const float *>(b.gpart), n_parts, static_cast<const int *>(st.inv_perm),
+                     static_cast<const float *>(st.topk_w), static_cast<const float *>(st.topk_p), b.dl, c.T,
+                     c.top_k, c.score_fn, c.routed_scale));
+    MOK_TRY(launch_k(drouter_partial_kernel, dim3(static_cast<unsigned>(s.max_chunks), c.H / 256), dim3(256), 0, stream,
+                     "drouter_partial_kernel", static_cast<const __nv_bfloat16 *>(x), static_cast<const float *>(b.dl),
+                     static_cast<const int *>(st.offsets), static_cast<const int *>(st.chunk_start),
+                     static_cast<const int *>(st.perm), b.partial, c.H, c.E, c.top_k, kChunkRows));
+    MOK_TRY(launch_k(drouter_reduce_kernel, dim3(blocks_for(s.E * s.H, 256)), dim3(256), 0, stream,
+                     "drouter_reduce_kernel", static_cast<const float *>(b.partial),
+                     static_cast<const int *>(st.chunk_start), gr.drouter_w, c.H, c.E));
+    return launch_k(dx_combine_kernel, dim3(blocks_for(s.T * s.H / 8, 256)), dim3(256), 0, stream,
+                    "dx_combine_kernel", static_cast<const float *>(b.dxs), static_cast<const float *>(b.dl),
+                    static_cast<const int *>(st.topk_idx), p.router_w, static_cast<__nv_bfloat16 *>(gr.dx), c.T, c.H,
+                    c.top_k, c.n_shared);
 }
 
 PFN_cuMemGetAddressRange_v3020 g_addr_range = nullptr;
@@ -1681,11 +1899,13 @@ int moe_saved_tensor(const moe_cfg *cfg, int save_for_backward, int which, size_
     return MOK_OK;
 }
 
-int moe_ep_size(const moe_cfg *cfg, int32_t world, size_t *state_bytes, size_t *scratch_bytes)
+int moe_ep_size(const moe_cfg *cfg, int32_t world, int32_t training, size_t *state_bytes, size_t *scratch_bytes,
+                size_t *bwd_bytes)
 {
     MOK_TRY(check_ep(cfg, world, 0));
     if (state_bytes) *state_bytes = carve_state(*cfg, nullptr, false).bytes;
-    if (scratch_bytes) *scratch_bytes = carve_ep(*cfg, world, nullptr).bytes;
+    if (scratch_bytes) *scratch_bytes = carve_ep(*cfg, world, training != 0, nullptr).bytes;
+    if (bwd_bytes) *bwd_bytes = carve_ep_src_bwd(*cfg, nullptr).bytes;
     return MOK_OK;
 }
 
@@ -1701,7 +1921,7 @@ int moe_ep_route(const moe_cfg *cfg, int32_t world, int32_t rank, const void *x,
     return ep_route(*cfg, x, *params, carve_state(*cfg, state, false), *dev, static_cast<cudaStream_t>(stream));
 }
 
-int moe_ep_experts(const moe_cfg *cfg, int32_t world, int32_t rank, const void *const *x_ranks,
+int moe_ep_experts(const moe_cfg *cfg, int32_t world, int32_t rank, int32_t training, const void *const *x_ranks,
                    void *const *state_ranks, const moe_params *params, void *scratch, size_t scratch_bytes,
                    void *stream)
 {
@@ -1715,12 +1935,51 @@ int moe_ep_experts(const moe_cfg *cfg, int32_t world, int32_t rank, const void *
         if (!x_ranks[r] || !state_ranks[r] || !aligned16(x_ranks[r]) || !aligned16(state_ranks[r]))
             return MOK_ERR_INVALID;
     if (!scratch || !aligned16(scratch)) return MOK_ERR_INVALID;
-    const EpScratch need = carve_ep(*cfg, world, nullptr);
+    const EpScratch need = carve_ep(*cfg, world, training != 0, nullptr);
     if (scratch_bytes < need.bytes) return MOK_ERR_WORKSPACE;
     const DeviceInfo *dev = device_info();
     if (!dev) return MOK_ERR_DEVICE;
-    return ep_experts(*cfg, world, rank, x_ranks, state_ranks, *params, carve_ep(*cfg, world, scratch), *dev,
-                      static_cast<cudaStream_t>(stream));
+    return ep_experts(*cfg, world, rank, training != 0, x_ranks, state_ranks, *params,
+                      carve_ep(*cfg, world, training != 0, scratch), *dev, static_cast<cudaStream_t>(stream));
+}
+
+int moe_ep_bwd_experts(const moe_cfg *cfg, int32_t world, int32_t rank, const void *const *dy_ranks,
+                       void *const *bwd_ranks, const moe_params *params, const moe_grads *grads, void *scratch,
+                       size_t scratch_bytes, void *stream)
+{
+    MOK_TRY(check_ep(cfg, world, rank));
+    if (!params || !params->w_gate_up || !params->w_down || !dy_ranks || !bwd_ranks || !grads) return MOK_ERR_INVALID;
+    if (cfg->n_shared > 0 && (!params->ws_gate_up || !params->ws_down || !grads->dws_gate_up || !grads->dws_down))
+        return MOK_ERR_INVALID;
+    const void *w[] = {params->w_gate_up, params->w_down, params->ws_gate_up, params->ws_down, grads->dw_gate_up,
+                       grads->dw_down, grads->dws_gate_up, grads->dws_down};
+    for (const void *q : w)
+        if (q && !aligned16(q)) return MOK_ERR_INVALID;
+    if (!grads->dw_gate_up || !grads->dw_down) return MOK_ERR_INVALID;
+    for (int r = 0; r < world; ++r)
+        if (!dy_ranks[r] || !bwd_ranks[r] || !aligned16(dy_ranks[r]) || !aligned16(bwd_ranks[r]))
+            return MOK_ERR_INVALID;
+    if (!scratch || !aligned16(scratch)) return MOK_ERR_INVALID;
+    if (scratch_bytes < carve_ep(*cfg, world, true, nullptr).bytes) return MOK_ERR_WORKSPACE;
+    const DeviceInfo *dev = device_info();
+    if (!dev) return MOK_ERR_DEVICE;
+    return ep_bwd_experts(*cfg, world, rank, dy_ranks, bwd_ranks, *params, *grads, carve_ep(*cfg, world, true, scratch),
+                          *dev, static_cast<cudaStream_t>(stream));
+}
+
+int moe_ep_bwd_combine(const moe_cfg *cfg, int32_t world, int32_t rank, const void *x, const moe_params *params,
+                       const void *state, void *bwd, size_t bwd_bytes, const moe_grads *grads, void *stream)
+{
+    MOK_TRY(check_ep(cfg, world, rank));
+    if (!params || !params->router_w || !aligned16(params->router_w) || !grads || !grads->dx || !grads->drouter_w)
+        return MOK_ERR_INVALID;
+    if (!aligned16(grads->dx) || !aligned16(grads->drouter_w)) return MOK_ERR_INVALID;
+    if (!x || !aligned16(x) || !state || !aligned16(state) || !bwd || !aligned16(bwd)) return MOK_ERR_INVALID;
+    if (bwd_bytes < carve_ep_src_bwd(*cfg, nullptr).bytes) return MOK_ERR_WORKSPACE;
+    const DeviceInfo *dev = device_info();
+    if (!dev) return MOK_ERR_DEVICE;
+    return ep_bwd_combine(*cfg, x, *params, carve_state(*cfg, const_cast<void *>(state), false),
+                          carve_ep_src_bwd(*cfg, bwd), *grads, *dev, static_cast<cudaStream_t>(stream));
 }
 
 int moe_ep_combine(const moe_cfg *cfg, int32_t world, int32_t rank, const void *state, void *y, void *stream)

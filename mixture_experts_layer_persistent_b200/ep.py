@@ -1,5 +1,5 @@
-"""Expert parallelism around the C ABI: buffers, peer pointers and the order of
-the phases.  All arithmetic runs in libmok's kernels (moe_ep_* in
+"""Expert parallelism around the C ABI (forward and backward): buffers, peer
+pointers and the order of the phases.  All arithmetic runs in libmok's kernels (moe_ep_* in
 include/mok.h).
 
 "Cursor åpner megakernelen…" (the pull-versus-push paragraph): the rank that
@@ -38,19 +38,42 @@ def split_params(params: dict, world: int, rank: int, E: int) -> dict:
     return out
 
 
-class EPWorld:
-    """All `world` ranks of an expert-parallel forward on the current device."""
+def _grads(g: dict):
+    return abi.moe_grads(*(None if g.get(n) is None else g[n].data_ptr() for n in
+                           ("dx", "dw_gate_up", "dw_down", "drouter_w", "dws_gate_up", "dws_down")))
 
-    def __init__(self, cfg: abi.moe_cfg, world: int, rank_params: list, device=None):
+
+def new_rank_grads(cfg: abi.moe_cfg, world: int, device) -> dict:
+    """Gradient tensors of one rank: dx and the router / shared-expert gradients of
+    its tokens, dw_* of its own experts."""
+    c, el = cfg, cfg.E // world
+    g = {"dx": torch.empty((c.T, c.H), dtype=torch.bfloat16, device=device),
+         "dw_gate_up": torch.empty((el, 2 * c.I, c.H), dtype=torch.bfloat16, device=device),
+         "dw_down": torch.empty((el, c.H, c.I), dtype=torch.bfloat16, device=device),
+         "drouter_w": torch.empty((c.E, c.H), dtype=torch.float32, device=device),
+         "dws_gate_up": None, "dws_down": None}
+    if c.n_shared:
+        g["dws_gate_up"] = torch.empty((c.n_shared, 2 * c.I, c.H), dtype=torch.bfloat16, device=device)
+        g["dws_down"] = torch.empty((c.n_shared, c.H, c.I), dtype=torch.bfloat16, device=device)
+    return g
+
+
+class EPWorld:
+    """All `world` ranks of an expert-parallel layer on the current device."""
+
+    def __init__(self, cfg: abi.moe_cfg, world: int, rank_params: list, training: bool = False, device=None):
         if len(rank_params) != world:
             raise ValueError("one parameter dict per rank")
-        self.cfg, self.world = cfg, world
+        self.cfg, self.world, self.training = cfg, world, training
         self.device = torch.device(device or "cuda")
-        self.state_bytes, self.scratch_bytes = abi.moe_ep_size(cfg, world)
-        self.states = [torch.empty(self.state_bytes, dtype=torch.uint8, device=self.device) for _ in range(world)]
-        self.scratch = [torch.empty(self.scratch_bytes, dtype=torch.uint8, device=self.device) for _ in range(world)]
+        self.state_bytes, self.scratch_bytes, self.bwd_bytes = abi.moe_ep_size(cfg, world, training)
+        mk = lambda n: torch.empty(n, dtype=torch.uint8, device=self.device)
+        self.states = [mk(self.state_bytes) for _ in range(world)]
+        self.scratch = [mk(self.scratch_bytes) for _ in range(world)]
+        self.bwd = [mk(self.bwd_bytes) for _ in range(world)] if training else None
         self.params = rank_params            # keeps the tensors alive
         self.cparams = [make_params(p) for p in rank_params]
+        self.xs = None
 
     def forward(self, xs: list, ys: list = None) -> list:
         c, W = self.cfg, self.world
@@ -64,10 +87,31 @@ class EPWorld:
         for r in range(W):
             abi.moe_ep_route(c, W, r, xp[r], self.cparams[r], sp[r], self.state_bytes, st)
         for r in range(W):
-            abi.moe_ep_experts(c, W, r, xp, sp, self.cparams[r], self.scratch[r].data_ptr(), self.scratch_bytes, st)
+            abi.moe_ep_experts(c, W, r, self.training, xp, sp, self.cparams[r], self.scratch[r].data_ptr(),
+                               self.scratch_bytes, st)
         for r in range(W):
             abi.moe_ep_combine(c, W, r, sp[r], ys[r].data_ptr(), st)
+        self.xs = xs
         return ys
+
+    def backward(self, dys: list, grads: list = None) -> list:
+        """Per-rank gradients after a training forward of the same xs (new_rank_grads)."""
+        c, W = self.cfg, self.world
+        if not self.training or self.xs is None:
+            raise RuntimeError("backward needs a training forward first")
+        if grads is None:
+            grads = [new_rank_grads(c, W, self.device) for _ in range(W)]
+        st = torch.cuda.current_stream(self.device).cuda_stream
+        dp = [d.data_ptr() for d in dys]
+        bp = [b.data_ptr() for b in self.bwd]
+        cg = [_grads(g) for g in grads]
+        for r in range(W):
+            abi.moe_ep_bwd_experts(c, W, r, dp, bp, self.cparams[r], cg[r], self.scratch[r].data_ptr(),
+                                   self.scratch_bytes, st)
+        for r in range(W):
+            abi.moe_ep_bwd_combine(c, W, r, self.xs[r].data_ptr(), self.cparams[r], self.states[r].data_ptr(),
+                                   bp[r], self.bwd_bytes, cg[r], st)
+        return grads
 
 
 def exchange_pointers(local_ptr: int, group=None, export=None, open_=None, opened=None):
@@ -102,30 +146,38 @@ def exchange_pointers(local_ptr: int, group=None, export=None, open_=None, opene
 
 
 class EPRank:
-    """This process's rank of an expert-parallel forward (one GPU per process).
+    """This process's rank of an expert-parallel layer (one GPU per process).
 
-    x goes into ``self.x`` (peers read it); ``forward`` runs route, barrier,
-    experts, barrier, combine on the current stream.
+    x goes into ``self.x`` and dy into ``self.dy`` (peers read both);
+    ``forward`` runs route, barrier, experts, barrier, combine on the current
+    stream, ``backward`` barrier, experts, barrier, combine.
     """
 
-    def __init__(self, cfg: abi.moe_cfg, params: dict, group=None, device=None):
+    def __init__(self, cfg: abi.moe_cfg, params: dict, training: bool = False, group=None, device=None):
         import torch.distributed as dist
         self.dist = dist
         self.group = group
         self.cfg = cfg
+        self.training = training
         self.world = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
         self.device = torch.device(device or "cuda")
-        self.state_bytes, self.scratch_bytes = abi.moe_ep_size(cfg, self.world)
-        self.state = torch.empty(self.state_bytes, dtype=torch.uint8, device=self.device)
-        self.scratch = torch.empty(self.scratch_bytes, dtype=torch.uint8, device=self.device)
+        self.state_bytes, self.scratch_bytes, self.bwd_bytes = abi.moe_ep_size(cfg, self.world, training)
+        mk = lambda n: torch.empty(n, dtype=torch.uint8, device=self.device)
+        self.state = mk(self.state_bytes)
+        self.scratch = mk(self.scratch_bytes)
+        self.bwd = mk(self.bwd_bytes) if training else None
         self.x = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=self.device)
+        self.dy = torch.empty((cfg.T, cfg.H), dtype=torch.bfloat16, device=self.device) if training else None
         self.params = params
         self.cparams = make_params(params)
         self._flag = torch.zeros(1, dtype=torch.int32, device=self.device)
         torch.cuda.synchronize(self.device)          # buffers exist before peers map them
         self.x_ptrs, self._opened = exchange_pointers(self.x.data_ptr(), group)
         self.state_ptrs, self._opened = exchange_pointers(self.state.data_ptr(), group, opened=self._opened)
+        if training:
+            self.dy_ptrs, self._opened = exchange_pointers(self.dy.data_ptr(), group, opened=self._opened)
+            self.bwd_ptrs, self._opened = exchange_pointers(self.bwd.data_ptr(), group, opened=self._opened)
 
     def _barrier(self):
         self.dist.all_reduce(self._flag, group=self.group)
@@ -137,11 +189,24 @@ class EPRank:
         st = torch.cuda.current_stream(self.device).cuda_stream
         abi.moe_ep_route(c, W, r, self.x.data_ptr(), self.cparams, self.state.data_ptr(), self.state_bytes, st)
         self._barrier()
-        abi.moe_ep_experts(c, W, r, self.x_ptrs, self.state_ptrs, self.cparams, self.scratch.data_ptr(),
-                           self.scratch_bytes, st)
+        abi.moe_ep_experts(c, W, r, self.training, self.x_ptrs, self.state_ptrs, self.cparams,
+                           self.scratch.data_ptr(), self.scratch_bytes, st)
         self._barrier()
         abi.moe_ep_combine(c, W, r, self.state.data_ptr(), y.data_ptr(), st)
         return y
+
+    def backward(self, grads: dict = None) -> dict:
+        c, W, r = self.cfg, self.world, self.rank
+        grads = grads or new_rank_grads(c, W, self.device)
+        cg = _grads(grads)
+        st = torch.cuda.current_stream(self.device).cuda_stream
+        self._barrier()                              # every rank's dy is in place
+        abi.moe_ep_bwd_experts(c, W, r, self.dy_ptrs, self.bwd_ptrs, self.cparams, cg, self.scratch.data_ptr(),
+                               self.scratch_bytes, st)
+        self._barrier()
+        abi.moe_ep_bwd_combine(c, W, r, self.x.data_ptr(), self.cparams, self.state.data_ptr(),
+                               self.bwd.data_ptr(), self.bwd_bytes, cg, st)
+        return grads
 
     def close(self):
         torch.cuda.synchronize(self.device)

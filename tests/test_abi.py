@@ -113,15 +113,20 @@ def test_expert_parallel_sizes_and_argument_checks():
     or short buffers -- all before touching a device (no pointer is dereferenced)."""
     T, H, E, I, k, W = 512, 7168, 256, 2048, 8, 8
     c = make_cfg(T, H, E, I, k, 1, I, 1, 8, 4)
-    state, scratch = abi.moe_ep_size(c, W)
+    state, scratch, bwd = abi.moe_ep_size(c, W)
+    _, scratch_t, _ = abi.moe_ep_size(c, W, True)
     assert state == abi.moe_workspace_size(c)[1]
     rr = W * T * min(k, E // W)
     rows = rr + T
     assert scratch >= (T + rr) * H * 2 + rows * I * 2 + rows * 16
+    # training adds g/u, w h, the pulled dy rows, dGU and the slot-gradient partials
+    assert scratch_t >= scratch + rows * (2 * I + I + 2 * I) * 2 + (T + rr) * H * 2 + rr * (I // 128) * 4
+    # the token side of the backward: dX slot rows and the slot-gradient partials others push
+    assert bwd >= T * 9 * H * 4 + T * k * (I // 128) * 4
     # E/world < k: a token puts at most E/world of its k slots on one rank
     c2 = make_cfg(200, 256, 8, 128, 2)
-    _, s8 = abi.moe_ep_size(c2, 8)
-    _, s1 = abi.moe_ep_size(c2, 1)
+    _, s8, _ = abi.moe_ep_size(c2, 8)
+    _, s1, _ = abi.moe_ep_size(c2, 1)
     assert s8 >= (200 + 8 * 200 * 1) * 256 * 2 and s1 >= (200 + 200 * 2) * 256 * 2
     for world, cfg, code in ((0, c, abi.MOK_ERR_INVALID), (9, c, abi.MOK_ERR_INVALID),
                              (3, make_cfg(64, 256, 8, 128, 2), abi.MOK_ERR_INVALID),
@@ -131,7 +136,8 @@ def test_expert_parallel_sizes_and_argument_checks():
             abi.moe_ep_size(cfg, world)
         assert ei.value.code == code, (world, code)
     small = make_cfg(64, 256, 8, 128, 2)
-    st, sc = abi.moe_ep_size(small, 2)
+    st, sc, bb = abi.moe_ep_size(small, 2)
+    _, sct, _ = abi.moe_ep_size(small, 2, True)
     p = abi.moe_params(router_w=16, w_gate_up=16, w_down=16)
     for rank in (-1, 2):
         with pytest.raises(abi.MokError) as ei:
@@ -144,10 +150,26 @@ def test_expert_parallel_sizes_and_argument_checks():
         abi.moe_ep_route(small, 2, 0, None, p, 16, st, None)
     assert ei.value.code == abi.MOK_ERR_INVALID
     with pytest.raises(abi.MokError) as ei:
-        abi.moe_ep_experts(small, 2, 0, [16, 16], [16, 16], p, 16, sc - 1, None)
+        abi.moe_ep_experts(small, 2, 0, 0, [16, 16], [16, 16], p, 16, sc - 1, None)
     assert ei.value.code == abi.MOK_ERR_WORKSPACE
     with pytest.raises(abi.MokError) as ei:
-        abi.moe_ep_experts(small, 2, 0, [16, None], [16, 16], p, 16, sc, None)
+        abi.moe_ep_experts(small, 2, 0, 0, [16, None], [16, 16], p, 16, sc, None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
+    with pytest.raises(abi.MokError) as ei:      # a training forward needs the larger scratch
+        abi.moe_ep_experts(small, 2, 0, 1, [16, 16], [16, 16], p, 16, sct - 1, None)
+    assert ei.value.code == abi.MOK_ERR_WORKSPACE
+    g = abi.moe_grads(dx=16, dw_gate_up=16, dw_down=16, drouter_w=16)
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_bwd_experts(small, 2, 0, [16, 16], [16, 16], p, g, 16, sct - 1, None)
+    assert ei.value.code == abi.MOK_ERR_WORKSPACE
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_bwd_experts(small, 2, 1, [16, None], [16, 16], p, g, 16, sct, None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_bwd_combine(small, 2, 0, 16, p, 16, 16, bb - 1, g, None)
+    assert ei.value.code == abi.MOK_ERR_WORKSPACE
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_bwd_combine(small, 2, 0, 16, p, 16, 16, bb, abi.moe_grads(dx=16), None)
     assert ei.value.code == abi.MOK_ERR_INVALID
     with pytest.raises(abi.MokError) as ei:
         abi.moe_ep_combine(small, 2, 0, 16, None, None)

@@ -1,4 +1,4 @@
-"""Expert parallelism: each rank's y against the one-GPU layer on its tokens.
+"""Expert parallelism: each rank's y and gradients against the one-GPU layer.
 
 The ranks run on one device with one buffer set each (EPWorld), the phases in
 stream order.  Rank r owns the routed experts [r E/world, (r+1) E/world); its
@@ -9,6 +9,14 @@ and the k-sum runs in slot order on the token's rank, so each rank's y must
 equal moe_fwd of the same tokens with all E experts byte for byte, whatever
 share of the rows each rank receives.  Rank 0's y is also checked against the
 oracle at the layer tolerance.
+
+Backward: the owner pulls dy rows like x rows and pushes dX rows and the
+slot-gradient partials back to the tokens' ranks, so each rank's dx, router
+gradient and shared-expert gradient equal moe_bwd on its tokens byte for byte;
+an owner's expert weight gradients (summed over every rank's rows, in rank then
+token order) equal moe_bwd's on the concatenated batch, byte for byte when that
+batch routes its tokens the same way (the same router K split), else at the
+layer tolerance.
 """
 import numpy as np
 import pytest
@@ -48,6 +56,22 @@ def _rank_inputs(wl, world, dev, margins=True):
         bits.append(xb)
         xs.append(bits_to_bf16(xb, dev))
     return params, xs, bits
+
+
+def _margin_xs(wl, params, world, dev):
+    """One x per rank with top-k margins >= 1e-3, routed by the oracle from the router
+    parameters alone (no expert weight leaves the device)."""
+    f32 = lambda t: None if t is None else t.detach().float().cpu().numpy()
+    xs = []
+    for r in range(world):
+        wr = synth.scaled(wl, seed=wl.seed * 100 + r)
+        L = oracle.Layer(wl.T, wl.H, wl.E, wl.k, wl.I, S=wl.S, Is=wl.Is, score_fn=wl.score_fn, n_group=wl.n_group,
+                         topk_group=wl.topk_group, routed_scale=wl.routed_scale)
+        L.set(x=synth.bf16_bits(synth.draw_x(wr, dev)), Wr=f32(params["router_w"]), bias=f32(params.get("e_bias")),
+              lbias=f32(params.get("logit_bias")))
+        xb, _, _, _ = oracle.margin_reject(L, lambda a, wr=wr: synth.bf16_bits(synth.draw_x(wr, dev, attempt=a)))
+        xs.append(bits_to_bf16(xb, dev))
+    return xs
 
 
 def _same(a, b):
@@ -99,3 +123,104 @@ def test_dsv3_expert_shape_over_eight_ranks():
             assert _same(ys[r], y_ref), f"{wl.name} rank {r}: y differs from moe_fwd"
         del ep, layer, params, xs, ys
         torch.cuda.empty_cache()
+
+
+def _rank_dys(wl, world, dev):
+    return [synth.draw_dy(synth.scaled(wl, seed=wl.seed * 100 + 50 + r), dev) for r in range(world)]
+
+
+@pytest.mark.parametrize("world,wl", CASES, ids=[f"{w.name}-w{n}" for n, w in CASES])
+def test_backward_matches_the_one_gpu_layer(world, wl):
+    dev = torch.device("cuda")
+    params, xs, bits = _rank_inputs(wl, world, dev)
+    dys = _rank_dys(wl, world, dev)
+    cfg = cfg_for(wl)
+    el = wl.E // world
+    ep = EPWorld(cfg, world, [split_params(params, world, r, wl.E) for r in range(world)], training=True)
+    ys = ep.forward(xs)
+    grads = ep.backward(dys)
+    torch.cuda.synchronize()
+    assert abi.moe_status(torch.cuda.current_stream().cuda_stream) == 0
+    # per rank: y, dx, the router gradient and the shared experts' gradient of its tokens
+    layer = MoELayer(cfg, params, training=True)
+    for r in range(world):
+        y_ref = layer.forward(xs[r]).clone()
+        g_ref = layer.backward(xs[r], dys[r])
+        torch.cuda.synchronize()
+        assert _same(ys[r], y_ref), f"rank {r}: y"
+        for n in ("dx", "drouter_w", "dws_gate_up", "dws_down"):
+            if g_ref.get(n) is not None:
+                assert _same(grads[r][n], g_ref[n]), f"rank {r}: {n}"
+    assert layer.status() == 0
+    # the owners' expert gradients against the one-GPU layer on every rank's tokens
+    whole = synth.scaled(wl, T=wl.T * world)
+    big = MoELayer(cfg_for(whole), params, training=True)
+    routing = big.new_routing()
+    big.forward(torch.cat(xs), routing=routing)
+    g_all = big.backward(torch.cat(xs), torch.cat(dys))
+    torch.cuda.synchronize()
+    assert big.status() == 0
+    same_routing = True
+    for r in range(world):                 # does the concatenated batch route each token as its rank did?
+        rr = layer.new_routing()
+        layer.forward(xs[r], routing=rr)
+        sl = slice(r * wl.T, (r + 1) * wl.T)
+        same_routing &= _same(rr["topk_idx"], routing["topk_idx"][sl]) and _same(rr["topk_w"], routing["topk_w"][sl])
+    assert same_routing, "these cases keep the router's K split, so the routing must agree"
+    for r in range(world):
+        for n in ("dw_gate_up", "dw_down"):
+            assert _same(grads[r][n], g_all[n][r * el:(r + 1) * el]), f"owner {r}: {n}"
+    # rank 0's dx against the oracle
+    L = oracle_layer(wl, params, bits[0], synth.bf16_bits(dys[0]))
+    idx, w, _ = L.route()
+    dxo, _, _ = L.bwd(idx, w)
+    assert_close(to_np(grads[0]["dx"]), dxo, f"{wl.name} rank 0 dx vs oracle")
+
+
+def test_backward_dsv3_expert_shape_over_eight_ranks():
+    """The DeepSeek-V3 shape over 8 ranks of 256 tokens (32 experts per rank, about
+    64 rows per expert): per-rank y, dx, router and shared-expert gradients byte-equal
+    to moe_bwd of the rank's tokens; each owner's expert weight gradients byte-equal
+    to moe_bwd's on all 2048 tokens.  At 256 and 2048 tokens the router splits its
+    contraction the same way (8 K splits), so that batch routes every token as its
+    rank did (checked); top-k margins of 1e-3 as everywhere."""
+    dev = torch.device("cuda")
+    world = 8
+    wl = synth.scaled(synth.WORKLOADS["dsv3"], name="ep_dsv3_bwd", T=256, seed=58)
+    el = wl.E // world
+    params = synth.draw_params(wl, dev)
+    xs = _margin_xs(wl, params, world, dev)
+    dys = _rank_dys(wl, world, dev)
+    cfg = cfg_for(wl)
+    ep = EPWorld(cfg, world, [split_params(params, world, r, wl.E) for r in range(world)], training=True)
+    ys = ep.forward(xs)
+    grads = ep.backward(dys)
+    torch.cuda.synchronize()
+    assert abi.moe_status(torch.cuda.current_stream().cuda_stream) == 0
+    layer = MoELayer(cfg, params, training=True)
+    routings = []
+    for r in range(world):
+        rr = layer.new_routing()
+        y_ref = layer.forward(xs[r], routing=rr)
+        g_ref = layer.backward(xs[r], dys[r])
+        torch.cuda.synchronize()
+        assert _same(ys[r], y_ref), f"rank {r}: y"
+        for n in ("dx", "drouter_w", "dws_gate_up", "dws_down"):
+            assert _same(grads[r][n], g_ref[n]), f"rank {r}: {n}"
+        routings.append(rr)
+        del g_ref
+    del layer
+    torch.cuda.empty_cache()
+    big = MoELayer(cfg_for(synth.scaled(wl, T=wl.T * world)), params, training=True)
+    routing = big.new_routing()
+    big.forward(torch.cat(xs), routing=routing)
+    g_all = big.backward(torch.cat(xs), torch.cat(dys))
+    torch.cuda.synchronize()
+    assert big.status() == 0
+    for r in range(world):
+        sl = slice(r * wl.T, (r + 1) * wl.T)
+        assert _same(routings[r]["topk_idx"], routing["topk_idx"][sl]), f"rank {r}: selection"
+        assert _same(routings[r]["topk_w"], routing["topk_w"][sl]), f"rank {r}: routing weights"
+    for r in range(world):
+        for n in ("dw_gate_up", "dw_down"):
+            assert _same(grads[r][n], g_all[n][r * el:(r + 1) * el]), f"owner {r}: {n}"
