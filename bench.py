@@ -690,20 +690,25 @@ def bf16_workload_run(wl, dev, K, warmup, world, dist, pk, do_ab=True):
 
 
 def ep_emulated_run(wl, W, dev, K, warmup):
-    """The expert-parallel forward with its W ranks (wl.T tokens each) run on this GPU in
-    stream order, against the one-GPU forward of the same W * wl.T tokens.  Both do the
-    same expert arithmetic; the difference is what the rank split adds on one device (the
-    owners' row layouts, the pull copy of every received row, per-rank launches and
-    tails).  No NVLink is crossed: this is the data path, not a multi-GPU measurement."""
+    """The expert-parallel layer with its W ranks (wl.T tokens each) run on this GPU in
+    stream order, against the one-GPU layer on the same W * wl.T tokens: forward, and
+    forward + backward.  Both do the same expert arithmetic; the difference is what the
+    rank split adds on one device (the owners' row layouts, the pull copies of the
+    received x and dy rows, per-rank launches and tails).  No NVLink is crossed: this is
+    the data path, not a multi-GPU measurement."""
     import torch
-    from mixture_experts_layer_persistent_b200 import EPWorld, MoELayer, cfg_for, split_params, synth
+    from mixture_experts_layer_persistent_b200 import EPWorld, MoELayer, cfg_for, new_rank_grads, split_params, synth
     params = synth.draw_params(wl, dev)
     xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(W)]
-    ep = EPWorld(cfg_for(wl), W, [split_params(params, W, r, wl.E) for r in range(W)], device=dev)
+    dys = [synth.draw_dy(synth.scaled(wl, seed=wl.seed * 100 + 50 + r), dev) for r in range(W)]
+    cfg = cfg_for(wl)
+    ep = EPWorld(cfg, W, [split_params(params, W, r, wl.E) for r in range(W)], training=True, device=dev)
     ys = [torch.empty_like(x) for x in xs]
+    eg = [new_rank_grads(cfg, W, dev) for _ in range(W)]
     whole = synth.scaled(wl, T=wl.T * W)
-    one = MoELayer(cfg_for(whole), params, training=False, device=dev)
-    xw = torch.cat(xs)
+    one = MoELayer(cfg_for(whole), params, training=True, device=dev)
+    og = one.new_grads()
+    xw, dyw = torch.cat(xs), torch.cat(dys)
     yw = torch.empty_like(xw)
     routing = one.new_routing()
     one.forward(xw, yw, routing=routing)
@@ -711,32 +716,38 @@ def ep_emulated_run(wl, W, dev, K, warmup):
     recv = counts.reshape(W, wl.E // W).sum(axis=1)        # rows each rank's experts receive
     for _ in range(warmup):
         ep.forward(xs, ys)
+        ep.backward(dys, eg)
         one.forward(xw, yw)
+        one.backward(xw, dyw, og)
     torch.cuda.synchronize()
     mk = lambda: torch.cuda.Event(enable_timing=True)
-    t_ep, t_one = [], []
+    legs = {"ep": [], "one": []}
     for _ in range(K):                                  # interleaved legs
-        a, b = mk(), mk()
-        a.record(); ep.forward(xs, ys); b.record()
-        c, d = mk(), mk()
-        c.record(); one.forward(xw, yw); d.record()
-        t_ep.append((a, b)); t_one.append((c, d))
+        ev = [mk() for _ in range(3)]
+        ev[0].record(); ep.forward(xs, ys); ev[1].record(); ep.backward(dys, eg); ev[2].record()
+        legs["ep"].append(ev)
+        ev = [mk() for _ in range(3)]
+        ev[0].record(); one.forward(xw, yw); ev[1].record(); one.backward(xw, dyw, og); ev[2].record()
+        legs["one"].append(ev)
     torch.cuda.synchronize()
-    ms_ep = statistics.mean(a.elapsed_time(b) for a, b in t_ep)
-    ms_one = statistics.mean(c.elapsed_time(d) for c, d in t_one)
+    fwd = {k: statistics.mean(e[0].elapsed_time(e[1]) for e in v) for k, v in legs.items()}
+    step = {k: statistics.mean(e[0].elapsed_time(e[2]) for e in v) for k, v in legs.items()}
     status = one.status()
-    out = {"workload": f"{wl.name}: the forward of {W} ranks x {wl.T} tokens, E={wl.E} experts "
-                       f"({wl.E // W} per rank), top-{wl.k}, H={wl.H}, I={wl.I}, {wl.S} shared, all ranks on one GPU",
+    n = W * wl.T
+    out = {"workload": f"{wl.name}: {W} ranks x {wl.T} tokens, E={wl.E} experts ({wl.E // W} per rank), "
+                       f"top-{wl.k}, H={wl.H}, I={wl.I}, {wl.S} shared, BF16, all ranks on one GPU",
            "world": W, "tokens_per_rank": wl.T,
-           "ms": ms_ep, "tokens_per_s": W * wl.T / (ms_ep / 1e3),
-           "one_gpu_ms": ms_one, "one_gpu_tokens_per_s": W * wl.T / (ms_one / 1e3),
-           "ep_over_one_gpu_time": ms_ep / ms_one,
+           "fwd_ms": fwd["ep"], "fwd_tokens_per_s": n / (fwd["ep"] / 1e3),
+           "step_ms": step["ep"], "step_tokens_per_s": n / (step["ep"] / 1e3),
+           "one_gpu_fwd_ms": fwd["one"], "one_gpu_step_ms": step["one"],
+           "ep_over_one_gpu_fwd_time": fwd["ep"] / fwd["one"],
+           "ep_over_one_gpu_step_time": step["ep"] / step["one"],
            "received_rows_per_rank": [int(v) for v in recv],
            "received_rows_max_over_mean": float(recv.max() / max(1e-9, recv.mean())),
-           "pull_bytes": int((recv.sum() + W * wl.T) * wl.H * 2),
-           "device_status": status, "launches_per_forward": W * (6 + 5 + 1),
+           "pull_bytes_per_step": int(2 * (recv.sum() + W * wl.T) * wl.H * 2),
+           "device_status": status,
            "note": "ranks emulated in stream order on one device; no link crossed"}
-    del ep, one, params, xs, ys, xw, yw
+    del ep, one, params, xs, ys, dys, eg, og, xw, yw, dyw
     return out
 
 
