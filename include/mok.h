@@ -475,8 +475,13 @@ const char *moe_last_error(void);
  * multiple of world (1 <= world <= MOK_EP_MAX_RANKS); T is the tokens of ONE
  * rank.  Rank r holds its own T tokens and owns the routed experts
  * [r E/world, (r+1) E/world); the router and the shared experts run on every
- * rank for its own tokens.  BF16 only (MOK_ERR_UNSUPPORTED for MXFP8); T
- * (top_k + n_shared) must stay below 2^24.
+ * rank for its own tokens.  BF16 forward and backward; MXFP8 forward without
+ * saved state (MOK_ERR_UNSUPPORTED for an MXFP8 training forward or backward:
+ * each rank then quantises its x in moe_ep_route, the owners pull its e4m3 rows
+ * and scales, and the slot rows are bf16; the rank's w_* are e4m3 codes with
+ * s_* scales packed for its own [E/world * 2I, H] and [E/world * H, I] tensors,
+ * as moe_quantize_mxfp8_weights writes them for that slice).  T (top_k +
+ * n_shared) must stay below 2^24.
  *
  * Buffers (caller-allocated device memory, 16-byte aligned), from moe_ep_size:
  *   state    per rank, state_bytes: the rank's routing record and its fp32 slot

@@ -40,7 +40,6 @@ struct EpView {
     const int *offsets[kEpMaxRanks];    // [E + S + 1] rank s's sorted-row ranges
     const int *perm[kEpMaxRanks];       // [T k] rank s's sorted row -> t k + slot
     const float *topk_w[kEpMaxRanks];   // [T k] rank s's routing weights
-    const __nv_bfloat16 *x[kEpMaxRanks];   // [T, H] rank s's tokens
     float *O[kEpMaxRanks];              // [T, k + S, H] rank s's fp32 slot rows
 };
 
@@ -57,7 +56,6 @@ struct EpArgs {
     float *row_w;          // [rows] routing weight (1 for shared rows)
     int *gorder;           // [E_loc + S] the owner's groups by rows descending, index ascending
     float **push;          // [kEpMaxRanks] slot rows of every rank, for the push epilogue
-    __nv_bfloat16 *x_recv; // [T + rr_cap, H] the owner's own tokens, then every received row
     int *status;
 };
 
@@ -165,20 +163,33 @@ __global__ void __launch_bounds__(256) ep_rows_kernel(EpView v, EpArgs a)
     }
 }
 
-// Pull at dispatch: x_recv[t] = own x[t] for t < T, x_recv[T + r] = x of the
-// row's source rank at its token.  One warp per row, 16-byte loads, four in
-// flight per lane; every remote row crosses the link once.
-__global__ void __launch_bounds__(256) ep_pull_kernel(EpView v, EpArgs a)
+// Pull at dispatch: dst row t = the owner's own row t for t < T, dst row T + r =
+// row r's token row on its source rank (x, dy, or x's MXFP8 codes or scales).
+// One warp per row, V-sized loads (16 or 8 bytes), four in flight per lane;
+// every remote row crosses the link once.
+struct EpPull {
+    const uint8_t *src[kEpMaxRanks];   // every rank's token rows, row_bytes each
+    uint8_t *dst;                      // [T + routed rows, row_bytes]
+    long long row_bytes;               // a multiple of sizeof(V)
+    int T, world, rank;
+    const int *seg;                    // routed rows = seg[n_seg]
+    int n_seg;
+    const int *row_src;                // (source rank << 24) | token of each routed row
+    int *status;
+};
+
+template <typename V>
+__global__ void __launch_bounds__(256) ep_pull_kernel(EpPull a)
 {
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int n_warps = (gridDim.x * blockDim.x) >> 5;
-    const int rows = a.T + a.seg[a.E_loc * a.world];
-    const int vec = a.H / 8;                           // 16-byte vectors per row (H % 256 == 0)
+    const int rows = a.T + a.seg[a.n_seg];
+    const int vec = static_cast<int>(a.row_bytes / static_cast<long long>(sizeof(V)));
     for (int r = warp; r < rows; r += n_warps) {
-        const __nv_bfloat16 *src;
+        const uint8_t *src;
         if (r < a.T) {
-            src = v.x[a.rank] + (size_t)r * a.H;
+            src = a.src[a.rank] + r * a.row_bytes;
         } else {
             const int code = a.row_src[r - a.T];
             const int s = code >> kEpRankShift, t = code & kEpRowMask;
@@ -186,18 +197,18 @@ __global__ void __launch_bounds__(256) ep_pull_kernel(EpView v, EpArgs a)
                 if (lane == 0) atomicOr(a.status, MOK_STATUS_BAD_INDEX);
                 continue;
             }
-            src = v.x[s] + (size_t)t * a.H;
+            src = a.src[s] + t * a.row_bytes;
         }
-        const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
-        uint4 *d4 = reinterpret_cast<uint4 *>(a.x_recv + (size_t)r * a.H);
-        for (int c = lane; c < vec; c += 128) {        // vec is a multiple of 32
-            uint4 q[4];
+        const V *sv = reinterpret_cast<const V *>(src);
+        V *dv = reinterpret_cast<V *>(a.dst + r * a.row_bytes);
+        for (int c = lane; c < vec; c += 128) {
+            V q[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                if (c + 32 * u < vec) q[u] = s4[c + 32 * u];
+                if (c + 32 * u < vec) q[u] = sv[c + 32 * u];
 #pragma unroll
             for (int u = 0; u < 4; ++u)
-                if (c + 32 * u < vec) d4[c + 32 * u] = q[u];
+                if (c + 32 * u < vec) dv[c + 32 * u] = q[u];
         }
     }
 }

@@ -81,8 +81,9 @@ struct GemmArgs {
     __nv_bfloat16 *out2;          // EPI_SWIGLU: saved gate/up pre-activations [R, 2I] (or null)
     __nv_bfloat16 *out3;          // EPI_SWIGLU: w * h [R, I] (or null)
     float *out_f32;               // EPI_ROUTER: partial logits [n_tiles, rows, 256]; EPI_PUSH: fp32 slot rows
-    float *const *push_dst;       // BF16 EPI_PUSH across ranks (expert parallelism): slot rows of every rank;
-                                  // row_slot is then (rank << 24) | slot row, every row a plain store (null: off)
+    float *const *push_dst;       // EPI_PUSH across ranks (expert parallelism): slot rows of every rank (fp32, or
+                                  // bf16 in the MXFP8 forward); row_slot is then (rank << 24) | slot row, every
+                                  // row a plain store (null: off)
     const __nv_bfloat16 *aux;     // EPI_DSWIGLU: saved gate/up pre-activations [R, 2I]
     const __nv_bfloat16 *aux_h;   // EPI_DSWIGLU: saved h [R, I] (the down GEMM's A operand)
     float *gpart;                 // EPI_DSWIGLU: <dy W_down, h> of each routed row over each N tile [R_routed, n_tiles]
@@ -1250,8 +1251,16 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                             else if (valid) store_row_direct(dst + c, p);
                         }
                     } else {
-                        // MXFP8 forward: bf16 rows pushed into their (token, slot) row
-                        __nv_bfloat16 *dst = args.out + (size_t)dst_row * args.ldo + t.nt * C::BN;
+                        // MXFP8 forward: bf16 rows pushed into their (token, slot) row; across
+                        // ranks into the slot rows of the token's rank, with plain stores
+                        __nv_bfloat16 *obase = args.out;
+                        int prow = dst_row;
+                        if (args.push_dst) {
+                            obase = reinterpret_cast<__nv_bfloat16 *>(args.push_dst[dst_row >> 24]);
+                            prow = dst_row & ((1 << 24) - 1);
+                        }
+                        const bool tma = full && !args.push_dst;
+                        __nv_bfloat16 *dst = obase + (size_t)prow * args.ldo + t.nt * C::BN;
 #pragma unroll 1
                         for (int c = 0; c < C::BN; c += 64) {
                             float v[64];
@@ -1264,7 +1273,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                                 mbar_arrive(&acce[acc]);         // every column of the accumulator is in registers
                             }
                             pack_bf16<64>(v, p);
-                            if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
+                            if (tma) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
                             else if (valid) store_row_direct(dst + c, p);
                         }
                     }

@@ -1057,6 +1057,8 @@ struct EpScratch {
     __nv_bfloat16 *gu, *hw;         // training: saved g/u and w h of the owner's rows
     __nv_bfloat16 *dy_recv, *dgu;   // training: pulled dy rows, dGU
     float *gpart;                   // training: slot-gradient partials of the owner's routed rows
+    uint8_t *xq_recv, *xs_recv;     // MXFP8: pulled e4m3 x rows and their scales
+    uint8_t *hq, *hs;               // MXFP8: h codes and scales
     long long rr_cap, rows_cap;
     size_t bytes;
 };
@@ -1081,6 +1083,14 @@ EpScratch carve_ep(const moe_cfg &c, int world, bool training, void *buf)
     e.push_dx = cv.take<float *>(kEpMaxRanks);
     e.push_g = cv.take<float *>(kEpMaxRanks);
     e.sched = cv.take<int>(kSchedCounters);
+    if (c.dtype == MOK_DTYPE_MXFP8) {               // (inference only)
+        e.xq_recv = cv.take<uint8_t>((s.T + e.rr_cap) * s.H);
+        e.xs_recv = cv.take<uint8_t>((s.T + e.rr_cap) * s.H / 32);
+        e.hq = cv.take<uint8_t>(e.rows_cap * s.I);
+        e.hs = cv.take<uint8_t>(e.rows_cap * s.I / 32);
+        e.bytes = align_up(cv.off, 256);
+        return e;
+    }
     e.x_recv = cv.take<__nv_bfloat16>((s.T + e.rr_cap) * s.H);
     e.h = cv.take<__nv_bfloat16>(e.rows_cap * s.I);
     if (training) {
@@ -1115,11 +1125,30 @@ EpSrcBwd carve_ep_src_bwd(const moe_cfg &c, void *buf)
     return b;
 }
 
+// Pull every rank's rows of `row_bytes` bytes (src[s]: rank s's [T, row_bytes]
+// matrix) into dst: the owner's own T rows, then each received row.
+int launch_pull(const void *const *src, int world, int rank, void *dst, long long row_bytes, const EpScratch &es,
+                const moe_cfg &c, const DeviceInfo &dev, cudaStream_t stream)
+{
+    EpPull a{};
+    for (int r = 0; r < world; ++r) a.src[r] = static_cast<const uint8_t *>(src[r]);
+    a.dst = static_cast<uint8_t *>(dst);
+    a.row_bytes = row_bytes;
+    a.T = c.T; a.world = world; a.rank = rank;
+    a.seg = es.seg; a.n_seg = c.E;
+    a.row_src = es.row_src;
+    a.status = dev.status;
+    if (row_bytes % 16 == 0)
+        return launch_k(ep_pull_kernel<uint4>, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", a);
+    if (row_bytes % 8 == 0)
+        return launch_k(ep_pull_kernel<uint2>, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", a);
+    return fail(MOK_ERR_INVALID, "expert-parallel pull: rows of a multiple of 8 bytes");
+}
+
 int check_ep(const moe_cfg *c, int world, int rank)
 {
     MOK_TRY(check_cfg(c));
     if (world < 1 || world > kEpMaxRanks || rank < 0 || rank >= world || c->E % world) return MOK_ERR_INVALID;
-    if (c->dtype != MOK_DTYPE_BF16) return MOK_ERR_UNSUPPORTED;
     if (static_cast<long long>(c->T) * (c->top_k + c->n_shared) >= (1ll << kEpRankShift)) return MOK_ERR_INVALID;
     const long long rows = static_cast<long long>(world) * c->T * std::min(c->top_k, c->E / world) +
                            static_cast<long long>(c->n_shared + 1) * c->T;
@@ -1137,7 +1166,133 @@ int ep_route(const moe_cfg &c, const void *x, const moe_params &p, const State &
     if (const cudaError_t e = cudaMemsetAsync(st.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
     MOK_TRY(launch_router(c, p, st, dev, pl, stream));
-    return launch_dispatch(pl, stream);
+    MOK_TRY(launch_dispatch(pl, stream));
+    if (c.dtype != MOK_DTYPE_MXFP8) return MOK_OK;
+    // MXFP8: the rank's x codes and scales, which the owners pull
+    const long long xb = static_cast<long long>(c.T) * c.H / 32;
+    return launch_k(quantize_mxfp8_kernel, dim3(blocks_for(xb, 256)), dim3(256), 0, stream, "quantize_mxfp8_kernel",
+                    static_cast<const __nv_bfloat16 *>(x), xb, st.xq, st.xs, static_cast<long long>(c.H / 32), 0ll,
+                    static_cast<__nv_bfloat16 *>(nullptr));
+}
+
+// Tensor maps and arguments of an owner's two expert GEMMs.
+struct EpGemms {
+    CUtensorMap gB, gBs, gO, gO2, gO3, dA, dB, dBs, dO;
+    GemmArgs ga, gd;
+};
+
+// MXFP8 (inference): gate/up on the pulled x codes with the SwiGLU epilogue
+// requantising h, down with the push epilogue storing bf16 rows into the slot
+// rows of the tokens' ranks.
+int ep_plan_mx(const moe_cfg &c, int el, const moe_params &p, const State &own, const EpScratch &es,
+               const DeviceInfo &dev, EpGemms &q)
+{
+    const Shapes s = shapes(c);
+    if (!make_tmap(&q.gB, p.w_gate_up, s.H, el * 2 * s.I, 128, 128, 1) ||
+        !make_tmap(&q.gBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : el) * 2 * s.I, 128, 128, 1) ||
+        !make_tmap(&q.gO, es.hq, s.I, es.rows_cap, 128, 32, 1) ||
+        !make_tmap(&q.dA, es.hq, s.I, es.rows_cap, 128, 128, 1) ||
+        !make_tmap(&q.dB, p.w_down, s.I, el * s.H, 128, 256, 1) ||
+        !make_tmap(&q.dBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : el) * s.H, 128, 256, 1) ||
+        !make_tmap(&q.dO, own.O, s.H, s.T * s.kk, 64, 1, 2))
+        return fail(MOK_ERR_INVALID, "tensor map (expert-parallel MXFP8 GEMMs)");
+    q.gO2 = q.gO3 = q.gO;
+    GemmArgs &ga = q.ga;
+    ga = GemmArgs{};
+    ga.sched = es.sched + 0;
+    ga.num_groups = el + c.n_shared;
+    ga.num_routed = el;
+    ga.offsets = es.offsets;
+    ga.row_token = es.row_token;
+    ga.row_slot = es.row_slot;
+    ga.row_w = es.row_w;
+    ga.n_tiles = c.I / 128;
+    ga.num_kb = c.H / 128;
+    ga.b_rows_per_group = 2 * c.I;
+    ga.b_half = c.I;
+    ga.inter = c.I;
+    ga.gather_src = reinterpret_cast<const __nv_bfloat16 *>(es.xq_recv);
+    ga.gather_ld = c.H;
+    ga.out = reinterpret_cast<__nv_bfloat16 *>(es.hq);
+    ga.out_scales = es.hs;
+    ga.sfa_src = es.xs_recv;
+    ga.sfb_src = p.s_gate_up;
+    ga.sfb_src_s = s.S ? p.ss_gate_up : p.s_gate_up;
+    ga.sf_ld = c.H / 32;
+    ga.sfb_row_tiles = static_cast<int>(el * 2 * s.I / 128);
+    ga.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : el) * 2 * s.I / 128);
+    ga.status = dev.status;
+    GemmArgs &gd = q.gd;
+    gd = ga;
+    gd.sched = es.sched + 1;
+    gd.n_tiles = c.H / 256;
+    gd.num_kb = c.I / 128;
+    gd.b_rows_per_group = c.H;
+    gd.b_half = 0;
+    gd.out = reinterpret_cast<__nv_bfloat16 *>(own.O);
+    gd.out_scales = nullptr;
+    gd.ldo = c.H;
+    gd.gather_src = nullptr;
+    gd.push_dst = es.push;
+    gd.sfa_src = es.hs;
+    gd.sfb_src = p.s_down;
+    gd.sfb_src_s = s.S ? p.ss_down : p.s_down;
+    gd.sf_ld = c.I / 32;
+    gd.sfb_row_tiles = static_cast<int>(el * s.H / 128);
+    gd.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : el) * s.H / 128);
+    return MOK_OK;
+}
+
+// BF16: gate/up on the pulled x rows with the SwiGLU epilogue (training: also g/u
+// and w h), down with the push epilogue storing fp32 rows into the slot rows of
+// the tokens' ranks (the map over the owner's own slot rows only has to exist).
+int ep_plan_bf16(const moe_cfg &c, int el, bool training, const moe_params &p, const State &own,
+                 const EpScratch &es, const DeviceInfo &dev, EpGemms &q)
+{
+    const Shapes s = shapes(c);
+    if (!make_tmap(&q.gB, p.w_gate_up, s.H, el * 2 * s.I, BK, 128, 2) ||
+        !make_tmap(&q.gBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : el) * 2 * s.I, BK, 128, 2) ||
+        !make_tmap(&q.gO, es.h, s.I, es.rows_cap, 64, 32, 2) ||
+        !make_tmap(&q.gO2, training ? es.gu : es.h, training ? 2 * s.I : s.I, es.rows_cap, 64, 32, 2) ||
+        !make_tmap(&q.gO3, training ? es.hw : es.h, s.I, es.rows_cap, 64, 32, 2) ||
+        !make_tmap(&q.dA, es.h, s.I, es.rows_cap, BK, 128, 2) ||
+        !make_tmap(&q.dB, p.w_down, s.I, el * s.H, BK, 256, 2) ||
+        !make_tmap(&q.dBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : el) * s.H, BK, 256, 2) ||
+        !make_tmap(&q.dO, own.O, s.H, s.T * s.kk, 32, 1, 4))
+        return fail(MOK_ERR_INVALID, "tensor map (expert-parallel GEMMs)");
+    GemmArgs &ga = q.ga;
+    ga = GemmArgs{};
+    ga.sched = es.sched + 0;
+    ga.num_groups = el + c.n_shared;
+    ga.num_routed = el;
+    ga.offsets = es.offsets;
+    ga.row_token = es.row_token;
+    ga.row_slot = es.row_slot;
+    ga.row_w = es.row_w;
+    ga.n_tiles = c.I / 128;
+    ga.num_kb = c.H / BK;
+    ga.b_rows_per_group = 2 * c.I;
+    ga.b_half = c.I;
+    ga.inter = c.I;
+    ga.gather_src = es.x_recv;
+    ga.gather_ld = c.H;
+    ga.out = es.h;
+    ga.out2 = training ? es.gu : nullptr;
+    ga.out3 = training ? es.hw : nullptr;
+    ga.status = dev.status;
+    GemmArgs &gd = q.gd;
+    gd = ga;
+    gd.sched = es.sched + 1;
+    gd.n_tiles = c.H / 256;
+    gd.num_kb = c.I / BK;
+    gd.b_rows_per_group = c.H;
+    gd.b_half = 0;
+    gd.out = nullptr;
+    gd.out2 = gd.out3 = nullptr;
+    gd.out_f32 = own.O;
+    gd.push_dst = es.push;
+    gd.ldo = c.H;
+    return MOK_OK;
 }
 
 int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void *const *xr, void *const *sr,
@@ -1154,7 +1309,6 @@ int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void 
         v.offsets[r] = q.offsets;
         v.perm[r] = q.perm;
         v.topk_w[r] = q.topk_w;
-        v.x[r] = static_cast<const __nv_bfloat16 *>(xr[r]);
         v.O[r] = q.O;
     }
     EpArgs a{};
@@ -1164,61 +1318,35 @@ int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void 
     a.seg = es.seg; a.offsets = es.offsets;
     a.row_token = es.row_token; a.row_src = es.row_src; a.row_slot = es.row_slot; a.row_w = es.row_w;
     a.row_gdst = es.row_gdst; a.gorder = es.gorder;
-    a.push = es.push; a.x_recv = es.x_recv; a.status = dev.status;
+    a.push = es.push; a.status = dev.status;
 
-    // tensor maps: the rank's experts, the shared experts, h, and its own slot rows
-    // (the push epilogue stores through es.push instead; the map only has to exist)
+    const bool mx = c.dtype == MOK_DTYPE_MXFP8;
     const State own = carve_state(c, sr[rank], false);
-    CUtensorMap gB, gBs, gO, gO2, gO3, dA, dB, dBs, dO;
-    if (!make_tmap(&gB, p.w_gate_up, s.H, el * 2 * s.I, BK, 128, 2) ||
-        !make_tmap(&gBs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : el) * 2 * s.I, BK, 128, 2) ||
-        !make_tmap(&gO, es.h, s.I, es.rows_cap, 64, 32, 2) ||
-        !make_tmap(&gO2, training ? es.gu : es.h, training ? 2 * s.I : s.I, es.rows_cap, 64, 32, 2) ||
-        !make_tmap(&gO3, training ? es.hw : es.h, s.I, es.rows_cap, 64, 32, 2) ||
-        !make_tmap(&dA, es.h, s.I, es.rows_cap, BK, 128, 2) ||
-        !make_tmap(&dB, p.w_down, s.I, el * s.H, BK, 256, 2) ||
-        !make_tmap(&dBs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : el) * s.H, BK, 256, 2) ||
-        !make_tmap(&dO, own.O, s.H, s.T * s.kk, 32, 1, 4))
-        return fail(MOK_ERR_INVALID, "tensor map (expert-parallel GEMMs)");
-    GemmArgs ga{};
-    ga.sched = es.sched + 0;
-    ga.num_groups = el + c.n_shared;
-    ga.num_routed = el;
-    ga.offsets = es.offsets;
-    ga.row_token = es.row_token;
-    ga.row_slot = es.row_slot;
-    ga.row_w = es.row_w;
-    ga.n_tiles = c.I / 128;
-    ga.num_kb = c.H / BK;
-    ga.b_rows_per_group = 2 * c.I;
-    ga.b_half = c.I;
-    ga.inter = c.I;
-    ga.gather_src = es.x_recv;
-    ga.gather_ld = c.H;
-    ga.out = es.h;
-    ga.out2 = training ? es.gu : nullptr;       // training: g/u and w h for the backward
-    ga.out3 = training ? es.hw : nullptr;
-    ga.status = dev.status;
-    GemmArgs gd = ga;
-    gd.sched = es.sched + 1;
-    gd.n_tiles = c.H / 256;
-    gd.num_kb = c.I / BK;
-    gd.b_rows_per_group = c.H;
-    gd.b_half = 0;
-    gd.out = nullptr;
-    gd.out2 = gd.out3 = nullptr;
-    gd.out_f32 = own.O;
-    gd.push_dst = es.push;
-    gd.ldo = c.H;
+    EpGemms q;
+    MOK_TRY(mx ? ep_plan_mx(c, el, p, own, es, dev, q) : ep_plan_bf16(c, el, training, p, own, es, dev, q));
 
     if (const cudaError_t e = cudaMemsetAsync(es.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
     MOK_TRY(launch_k(ep_layout_kernel, dim3(1), dim3(256), 0, stream, "ep_layout_kernel", v, a));
     MOK_TRY(launch_k(ep_rows_kernel, dim3(static_cast<unsigned>(c.E + c.n_shared * blocks_for(c.T, 256))), dim3(256), 0,
                      stream, "ep_rows_kernel", v, a));
-    MOK_TRY(launch_k(ep_pull_kernel, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", v, a));
-    MOK_TRY(launch_gemm<typename FusedCfg<false>::GateUp>(gB, gB, gBs, gO, gO2, gO3, ga, dev.sms, stream));
-    return launch_gemm<typename FusedCfg<false>::Down>(dA, dB, dBs, dO, dO, dO, gd, dev.sms, stream);
+    if (mx) {
+        // pull the x codes and scales each rank quantised in its routing phase
+        const void *xq[kEpMaxRanks], *xs[kEpMaxRanks];
+        for (int r = 0; r < world; ++r) {
+            const State st_r = carve_state(c, sr[r], false);
+            xq[r] = st_r.xq;
+            xs[r] = st_r.xs;
+        }
+        MOK_TRY(launch_pull(xq, world, rank, es.xq_recv, c.H, es, c, dev, stream));
+        MOK_TRY(launch_pull(xs, world, rank, es.xs_recv, c.H / 32, es, c, dev, stream));
+        MOK_TRY(launch_gemm<typename FusedCfg<true>::GateUp>(q.gB, q.gB, q.gBs, q.gO, q.gO2, q.gO3, q.ga, dev.sms,
+                                                            stream));
+        return launch_gemm<typename FusedCfg<true>::Down>(q.dA, q.dB, q.dBs, q.dO, q.dO, q.dO, q.gd, dev.sms, stream);
+    }
+    MOK_TRY(launch_pull(xr, world, rank, es.x_recv, 2ll * c.H, es, c, dev, stream));
+    MOK_TRY(launch_gemm<typename FusedCfg<false>::GateUp>(q.gB, q.gB, q.gBs, q.gO, q.gO2, q.gO3, q.ga, dev.sms, stream));
+    return launch_gemm<typename FusedCfg<false>::Down>(q.dA, q.dB, q.dBs, q.dO, q.dO, q.dO, q.gd, dev.sms, stream);
 }
 
 // Backward, owner side: pull dy rows, down dgrad (SwiGLU backward, slot-gradient
@@ -1235,21 +1363,13 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
     const int el = c.E / world;
     const long long G = el + s.S;
     const bool n256 = c.I % 256 == 0;
-    EpView v{};
     EpTable tdx{}, tg{};
     for (int r = 0; r < world; ++r) {
-        v.x[r] = static_cast<const __nv_bfloat16 *>(dyr[r]);
         const EpSrcBwd q = carve_ep_src_bwd(c, br[r]);
         tdx.p[r] = q.dxs;
         tg.p[r] = q.gpart;
     }
     const EpSrcBwd own = carve_ep_src_bwd(c, br[rank]);
-    EpArgs a{};
-    a.world = world; a.rank = rank;
-    a.T = c.T; a.H = c.H; a.k = c.top_k; a.kk = static_cast<int>(s.kk); a.S = c.n_shared; a.E_loc = el;
-    a.rr_cap = static_cast<int>(es.rr_cap);
-    a.seg = es.seg; a.row_src = es.row_src;
-    a.x_recv = es.dy_recv; a.status = dev.status;
 
     GemmArgs base{};
     base.num_groups = static_cast<int>(G);
@@ -1343,7 +1463,7 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
     MOK_TRY(launch_k(ep_table_kernel, dim3(1), dim3(32), 0, stream, "ep_table_kernel", tdx, es.push_dx, world));
     MOK_TRY(launch_k(ep_table_kernel, dim3(1), dim3(32), 0, stream, "ep_table_kernel", tg, es.push_g, world));
-    MOK_TRY(launch_k(ep_pull_kernel, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", v, a));
+    MOK_TRY(launch_pull(dyr, world, rank, es.dy_recv, 2ll * c.H, es, c, dev, stream));
     if (n256)
         MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradDown>(m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1,
                                                                   dev.sms, stream));
@@ -1903,6 +2023,7 @@ int moe_ep_size(const moe_cfg *cfg, int32_t world, int32_t training, size_t *sta
                 size_t *bwd_bytes)
 {
     MOK_TRY(check_ep(cfg, world, 0));
+    if (training && cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
     if (state_bytes) *state_bytes = carve_state(*cfg, nullptr, false).bytes;
     if (scratch_bytes) *scratch_bytes = carve_ep(*cfg, world, training != 0, nullptr).bytes;
     if (bwd_bytes) *bwd_bytes = carve_ep_src_bwd(*cfg, nullptr).bytes;
@@ -1926,8 +2047,12 @@ int moe_ep_experts(const moe_cfg *cfg, int32_t world, int32_t rank, int32_t trai
                    void *stream)
 {
     MOK_TRY(check_ep(cfg, world, rank));
+    if (training && cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
     if (!params || !params->w_gate_up || !params->w_down || !x_ranks || !state_ranks) return MOK_ERR_INVALID;
     if (cfg->n_shared > 0 && (!params->ws_gate_up || !params->ws_down)) return MOK_ERR_INVALID;
+    if (cfg->dtype == MOK_DTYPE_MXFP8 &&
+        (!params->s_gate_up || !params->s_down || (cfg->n_shared > 0 && (!params->ss_gate_up || !params->ss_down))))
+        return MOK_ERR_INVALID;
     const void *w[] = {params->w_gate_up, params->w_down, params->ws_gate_up, params->ws_down};
     for (const void *q : w)
         if (q && !aligned16(q)) return MOK_ERR_INVALID;
@@ -1948,6 +2073,7 @@ int moe_ep_bwd_experts(const moe_cfg *cfg, int32_t world, int32_t rank, const vo
                        size_t scratch_bytes, void *stream)
 {
     MOK_TRY(check_ep(cfg, world, rank));
+    if (cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
     if (!params || !params->w_gate_up || !params->w_down || !dy_ranks || !bwd_ranks || !grads) return MOK_ERR_INVALID;
     if (cfg->n_shared > 0 && (!params->ws_gate_up || !params->ws_down || !grads->dws_gate_up || !grads->dws_down))
         return MOK_ERR_INVALID;
@@ -1971,6 +2097,7 @@ int moe_ep_bwd_combine(const moe_cfg *cfg, int32_t world, int32_t rank, const vo
                        const void *state, void *bwd, size_t bwd_bytes, const moe_grads *grads, void *stream)
 {
     MOK_TRY(check_ep(cfg, world, rank));
+    if (cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
     if (!params || !params->router_w || !aligned16(params->router_w) || !grads || !grads->dx || !grads->drouter_w)
         return MOK_ERR_INVALID;
     if (!aligned16(grads->dx) || !aligned16(grads->drouter_w)) return MOK_ERR_INVALID;
@@ -1992,6 +2119,11 @@ int moe_ep_combine(const moe_cfg *cfg, int32_t world, int32_t rank, const void *
     t_pdl = false;
     const State st = carve_state(*cfg, const_cast<void *>(state), false);
     const Shapes s = shapes(*cfg);
+    if (cfg->dtype == MOK_DTYPE_MXFP8)       // the MXFP8 forward's slot rows are bf16
+        return launch_k(combine_kernel<__nv_bfloat16>, dim3(blocks_for(s.T * s.H / 8, 256)), dim3(256), 0,
+                        static_cast<cudaStream_t>(stream), "combine_kernel",
+                        reinterpret_cast<const __nv_bfloat16 *>(st.O), static_cast<const float *>(st.topk_w),
+                        static_cast<__nv_bfloat16 *>(y), cfg->T, cfg->H, cfg->top_k, cfg->n_shared);
     return launch_k(combine_kernel<float>, dim3(blocks_for(s.T * s.H / 8, 256)), dim3(256), 0,
                     static_cast<cudaStream_t>(stream), "combine_kernel", static_cast<const float *>(st.O),
                     static_cast<const float *>(st.topk_w), static_cast<__nv_bfloat16 *>(y), cfg->T, cfg->H,

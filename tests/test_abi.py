@@ -130,11 +130,24 @@ def test_expert_parallel_sizes_and_argument_checks():
     assert s8 >= (200 + 8 * 200 * 1) * 256 * 2 and s1 >= (200 + 200 * 2) * 256 * 2
     for world, cfg, code in ((0, c, abi.MOK_ERR_INVALID), (9, c, abi.MOK_ERR_INVALID),
                              (3, make_cfg(64, 256, 8, 128, 2), abi.MOK_ERR_INVALID),
-                             (2, make_cfg(64, 256, 8, 128, 2, dtype=abi.MOK_DTYPE_MXFP8), abi.MOK_ERR_UNSUPPORTED),
                              (2, make_cfg(1 << 21, 256, 8, 128, 8), abi.MOK_ERR_INVALID)):
         with pytest.raises(abi.MokError) as ei:
             abi.moe_ep_size(cfg, world)
         assert ei.value.code == code, (world, code)
+    # MXFP8: the forward without saved state only
+    mxc = make_cfg(64, 256, 8, 128, 2, dtype=abi.MOK_DTYPE_MXFP8)
+    mst, msc, _ = abi.moe_ep_size(mxc, 2)
+    assert msc >= (64 + 2 * 64 * 2) * (256 + 8) + (2 * 64 * 2) * (128 + 4)
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_size(mxc, 2, True)
+    assert ei.value.code == abi.MOK_ERR_UNSUPPORTED
+    pm = abi.moe_params(router_w=16, w_gate_up=16, w_down=16)      # MXFP8 without weight scales
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_experts(mxc, 2, 0, 0, [16, 16], [16, 16], pm, 16, msc, None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_experts(mxc, 2, 0, 1, [16, 16], [16, 16], pm, 16, msc, None)
+    assert ei.value.code == abi.MOK_ERR_UNSUPPORTED
     small = make_cfg(64, 256, 8, 128, 2)
     st, sc, bb = abi.moe_ep_size(small, 2)
     _, sct, _ = abi.moe_ep_size(small, 2, True)

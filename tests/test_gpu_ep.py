@@ -23,7 +23,8 @@ import pytest
 import torch
 
 import oracle
-from mixture_experts_layer_persistent_b200 import EPWorld, MoELayer, abi, cfg_for, split_params, synth
+from mixture_experts_layer_persistent_b200 import (EPWorld, MoELayer, abi, cfg_for, quantize_mxfp8_weights,
+                                                   split_params, synth)
 from tests._support import assert_close, bits_to_bf16, oracle_layer, to_np
 
 pytestmark = pytest.mark.gpu
@@ -224,3 +225,74 @@ def test_backward_dsv3_expert_shape_over_eight_ranks():
     for r in range(world):
         for n in ("dw_gate_up", "dw_down"):
             assert _same(grads[r][n], g_all[n][r * el:(r + 1) * el]), f"owner {r}: {n}"
+
+
+def _mx_params(params, world, E):
+    """MXFP8 weights of the whole layer (for moe_fwd) and of each rank's experts (each
+    rank quantises its own slice: the same codes, scales packed for the slice)."""
+    full = {k: params[k] for k in ("router_w", "e_bias", "logit_bias")}
+    for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
+                        ("ws_down", "ss_down")):
+        full[name], full[sname] = (quantize_mxfp8_weights(params[name]) if params.get(name) is not None
+                                   else (None, None))
+    el = E // world
+    ranks = []
+    for r in range(world):
+        p = dict(full)
+        for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down")):
+            p[name], p[sname] = quantize_mxfp8_weights(params[name][r * el:(r + 1) * el].contiguous())
+        ranks.append(p)
+    return full, ranks
+
+
+MX_CASES = [
+    (4, synth.Workload("ep_mx", T=300, H=512, E=16, k=4, I=256, S=1, Is=256, score_fn=1, n_group=4, topk_group=2,
+                       mxfp8=True, backward=False, seed=61)),
+    (3, synth.Workload("ep_mx_i384", T=211, H=768, E=12, k=3, I=384, S=2, Is=384, mxfp8=True, backward=False,
+                       seed=62)),
+    (8, synth.Workload("ep_mx_one_expert_per_rank", T=150, H=256, E=8, k=2, I=128, mxfp8=True, backward=False,
+                       seed=63)),
+]
+
+
+@pytest.mark.parametrize("world,wl", MX_CASES, ids=[f"{w.name}-w{n}" for n, w in MX_CASES])
+def test_mxfp8_forward_matches_the_one_gpu_layer(world, wl):
+    """MXFP8: each rank quantises its x in the routing phase and the owners pull the
+    e4m3 rows and their scales; each rank's y equals the one-GPU MXFP8 forward's on its
+    tokens byte for byte."""
+    dev = torch.device("cuda")
+    params = synth.draw_params(wl, dev)
+    xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(world)]
+    full, ranks = _mx_params(params, world, wl.E)
+    cfg = cfg_for(wl)
+    ep = EPWorld(cfg, world, ranks)
+    ys = ep.forward(xs)
+    torch.cuda.synchronize()
+    assert abi.moe_status(torch.cuda.current_stream().cuda_stream) == 0
+    layer = MoELayer(cfg, full, training=False)
+    for r in range(world):
+        y_ref = layer.forward(xs[r]).clone()
+        torch.cuda.synchronize()
+        assert _same(ys[r], y_ref), f"rank {r}: y differs from the MXFP8 moe_fwd"
+    assert layer.status() == 0
+
+
+def test_mxfp8_dsv3_expert_shape_over_eight_ranks():
+    dev = torch.device("cuda")
+    world = 8
+    wl = synth.scaled(synth.WORKLOADS["dsv3_mxfp8"], name="ep_mx_dsv3", T=1024, seed=64)
+    params = synth.draw_params(wl, dev)
+    xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(world)]
+    full, ranks = _mx_params(params, world, wl.E)
+    del params
+    torch.cuda.empty_cache()
+    cfg = cfg_for(wl)
+    ep = EPWorld(cfg, world, ranks)
+    ys = ep.forward(xs)
+    torch.cuda.synchronize()
+    assert abi.moe_status(torch.cuda.current_stream().cuda_stream) == 0
+    layer = MoELayer(cfg, full, training=False)
+    for r in range(world):
+        y_ref = layer.forward(xs[r])
+        torch.cuda.synchronize()
+        assert _same(ys[r], y_ref), f"rank {r}: y differs from the MXFP8 moe_fwd"
