@@ -713,7 +713,9 @@ def ep_emulated_run(wl, W, dev, K, warmup):
     routing = one.new_routing()
     one.forward(xw, yw, routing=routing)
     counts = routing["counts"].cpu().numpy()
-    recv = counts.reshape(W, wl.E // W).sum(axis=1)        # rows each rank's experts receive
+    recv = counts.reshape(W, wl.E // W).sum(axis=1)        # expert rows each rank's experts receive
+    owner = routing["topk_idx"].long() // (wl.E // W)      # owning rank of every (token, slot)
+    pairs = int(torch.zeros(W * wl.T, W, device=owner.device).scatter_(1, owner, 1.0).sum().item())
     for _ in range(warmup):
         ep.forward(xs, ys)
         ep.backward(dys, eg)
@@ -744,7 +746,8 @@ def ep_emulated_run(wl, W, dev, K, warmup):
            "ep_over_one_gpu_step_time": step["ep"] / step["one"],
            "received_rows_per_rank": [int(v) for v in recv],
            "received_rows_max_over_mean": float(recv.max() / max(1e-9, recv.mean())),
-           "pull_bytes_per_step": int(2 * (recv.sum() + W * wl.T) * wl.H * 2),
+           "pulled_rows_per_token": pairs / (W * wl.T),
+           "pull_bytes_per_step": int(2 * (pairs + W * wl.T) * wl.H * 2),
            "device_status": status,
            "note": "ranks emulated in stream order on one device; no link crossed"}
     del ep, one, params, xs, ys, dys, eg, og, xw, yw, dyw

@@ -486,9 +486,11 @@ const char *moe_last_error(void);
  * Buffers (caller-allocated device memory, 16-byte aligned), from moe_ep_size:
  *   state    per rank, state_bytes: the rank's routing record and its fp32 slot
  *            rows.  Other ranks read the routing record and write slot rows.
- *   scratch  per rank, scratch_bytes: the rows the rank receives (x rows, h and,
- *            when training, g/u, w h, the pulled dy rows and dGU), sized for the
- *            largest possible share, world T min(top_k, E/world) routed rows.
+ *   scratch  per rank, scratch_bytes: the rows the rank receives, sized for the
+ *            largest possible share: the pulled token rows (x, and when training
+ *            dy), one per (rank, token) with an expert here, at most world T; the
+ *            expert rows (h and, when training, g/u, w h and dGU), one per
+ *            (token, slot) routed here, at most world T min(top_k, E/world).
  *            A training forward's scratch is read by that rank's backward.
  *   bwd      per rank, bwd_bytes (backward only): the dX slot rows and
  *            slot-gradient partials other ranks write, and the rank's dl and
@@ -504,7 +506,8 @@ const char *moe_last_error(void);
  *                   its state (params: router_w, e_bias, logit_bias).
  *   moe_ep_experts  the owner's sorted rows from every rank's routing record,
  *                   the pull of those token rows into its scratch (one plain
- *                   16-byte-load copy; every remote row crosses the link once),
+ *                   16-byte-load copy; a token crosses the link once per owner,
+ *                   whatever number of its experts that owner holds),
  *                   the gate/up GEMM with SwiGLU (training: also g/u and w h),
  *                   and the down GEMM whose epilogue stores each fp32 output row
  *                   into the slot row of the token's rank through that rank's

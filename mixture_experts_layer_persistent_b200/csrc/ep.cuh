@@ -40,6 +40,7 @@ struct EpView {
     const int *offsets[kEpMaxRanks];    // [E + S + 1] rank s's sorted-row ranges
     const int *perm[kEpMaxRanks];       // [T k] rank s's sorted row -> t k + slot
     const float *topk_w[kEpMaxRanks];   // [T k] rank s's routing weights
+    const int *topk_idx[kEpMaxRanks];   // [T k] rank s's selected experts
     float *O[kEpMaxRanks];              // [T, k + S, H] rank s's fp32 slot rows
 };
 
@@ -50,7 +51,9 @@ struct EpArgs {
     int *seg;              // [E_loc world + 1] first sorted row of each (expert, source) segment; seg[n] = routed rows
     int *offsets;          // [E_loc + S + 1] the owner's group ranges (routed experts, then shared)
     int *row_token;        // [rows] row of x_recv each sorted row reads
-    int *row_src;          // [rows] (source rank << 24) | token
+    int *recv_idx;         // [world T] received row of (source rank, token), -1 if none
+    int *uniq_src;         // [world T] (source rank << 24) | token of each received row
+    int *n_recv;           // received rows (distinct (source rank, token) pairs)
     int *row_slot;         // [rows] (source rank << 24) | slot row t (k + S) + slot in that rank's O
     int *row_gdst;         // [routed rows] (source rank << 24) | the row's position in the source's sorted rows
     float *row_w;          // [rows] routing weight (1 for shared rows)
@@ -116,6 +119,48 @@ __global__ void __launch_bounds__(256) ep_layout_kernel(EpView v, EpArgs a)
     }
 }
 
+// The token rows the owner receives: every (source rank, token) pair with at
+// least one selected expert on the owner, once, in (rank, token) order -- a token
+// with several of its experts on one owner crosses the link once.  One block of
+// 1024 threads, each a run of consecutive pairs: count, block scan, write.
+__global__ void __launch_bounds__(1024) ep_unique_kernel(EpView v, EpArgs a)
+{
+    __shared__ int s_scan[1024];
+    const int n = a.world * a.T;
+    const int per = (n + 1023) / 1024;
+    const int i0 = threadIdx.x * per, i1 = min(n, i0 + per);
+    const int e0 = a.rank * a.E_loc, e1 = e0 + a.E_loc;
+    auto wanted = [&](int i) {
+        const int s = i / a.T, t = i - s * a.T;
+        const int *idx = v.topk_idx[s] + (size_t)t * a.k;
+        bool w = false;
+        for (int j = 0; j < a.k; ++j) w |= idx[j] >= e0 && idx[j] < e1;
+        return w;
+    };
+    int cnt = 0;
+    for (int i = i0; i < i1; ++i) cnt += wanted(i);
+    s_scan[threadIdx.x] = cnt;
+    __syncthreads();
+    for (int d = 1; d < 1024; d <<= 1) {
+        const int add = threadIdx.x >= d ? s_scan[threadIdx.x - d] : 0;
+        __syncthreads();
+        s_scan[threadIdx.x] += add;
+        __syncthreads();
+    }
+    int u = s_scan[threadIdx.x] - cnt;
+    for (int i = i0; i < i1; ++i) {
+        if (wanted(i)) {
+            const int s = i / a.T;
+            a.recv_idx[i] = u;
+            a.uniq_src[u] = (s << kEpRankShift) | (i - s * a.T);
+            ++u;
+        } else {
+            a.recv_idx[i] = -1;
+        }
+    }
+    if (threadIdx.x == 1023) *a.n_recv = s_scan[1023];
+}
+
 // Sorted rows of the owner.  Blocks [0, n): segment b = (expert j, source s)
 // copies source s's rows of expert e = rank E_loc + j; blocks after those:
 // the shared experts' rows of the owner's own tokens, 256 tokens per block.
@@ -142,8 +187,12 @@ __global__ void __launch_bounds__(256) ep_rows_kernel(EpView v, EpArgs a)
             }
             const int t = q / a.k, slot = q - t * a.k;
             const int r = base + i;
-            a.row_token[r] = a.T + r;
-            a.row_src[r] = (s << kEpRankShift) | t;
+            int u = a.recv_idx[s * a.T + t];
+            if (u < 0) {                                 // a row the selection does not list
+                atomicOr(a.status, MOK_STATUS_BAD_INDEX);
+                u = 0;
+            }
+            a.row_token[r] = a.T + u;
             a.row_slot[r] = (s << kEpRankShift) | (t * a.kk + slot);
             a.row_gdst[r] = (s << kEpRankShift) | (range_ok ? src0 + i : 0);
             a.row_w[r] = range_ok ? v.topk_w[s][q] : 0.0f;
@@ -156,25 +205,23 @@ __global__ void __launch_bounds__(256) ep_rows_kernel(EpView v, EpArgs a)
         if (s2 < a.S && t < a.T) {
             const int r = a.seg[n] + s2 * a.T + t;
             a.row_token[r] = t;
-            a.row_src[r] = (a.rank << kEpRankShift) | t;
             a.row_slot[r] = (a.rank << kEpRankShift) | (t * a.kk + a.k + s2);
             a.row_w[r] = 1.0f;
         }
     }
 }
 
-// Pull at dispatch: dst row t = the owner's own row t for t < T, dst row T + r =
-// row r's token row on its source rank (x, dy, or x's MXFP8 codes or scales).
+// Pull at dispatch: dst row t = the owner's own row t for t < T, dst row T + u =
+// the u-th received (source rank, token) row (x, dy, or x's MXFP8 codes or scales).
 // One warp per row, V-sized loads (16 or 8 bytes), four in flight per lane;
 // every remote row crosses the link once.
 struct EpPull {
     const uint8_t *src[kEpMaxRanks];   // every rank's token rows, row_bytes each
-    uint8_t *dst;                      // [T + routed rows, row_bytes]
+    uint8_t *dst;                      // [T + received rows, row_bytes]
     long long row_bytes;               // a multiple of sizeof(V)
     int T, world, rank;
-    const int *seg;                    // routed rows = seg[n_seg]
-    int n_seg;
-    const int *row_src;                // (source rank << 24) | token of each routed row
+    const int *n_recv;                 // received rows
+    const int *row_src;                // (source rank << 24) | token of each received row
     int *status;
 };
 
@@ -184,7 +231,7 @@ __global__ void __launch_bounds__(256) ep_pull_kernel(EpPull a)
     const int lane = threadIdx.x & 31;
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int n_warps = (gridDim.x * blockDim.x) >> 5;
-    const int rows = a.T + a.seg[a.n_seg];
+    const int rows = a.T + min(*a.n_recv, a.world * a.T);
     const int vec = static_cast<int>(a.row_bytes / static_cast<long long>(sizeof(V)));
     for (int r = warp; r < rows; r += n_warps) {
         const uint8_t *src;

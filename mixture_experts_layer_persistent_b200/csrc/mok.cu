@@ -1047,7 +1047,8 @@ int check_params(const moe_cfg &c, const moe_params *p)
 // pulled and the h of those rows, sized for the largest share it can receive
 // (every token of every rank choosing min(k, E_loc) of its experts).
 struct EpScratch {
-    int *seg, *offsets, *gorder, *row_token, *row_src, *row_slot, *row_gdst;
+    int *seg, *offsets, *gorder, *row_token, *row_slot, *row_gdst;
+    int *recv_idx, *uniq_src, *n_recv;   // the distinct (source rank, token) rows received
     float *row_w;
     float **push;                   // [kEpMaxRanks] every rank's fp32 slot rows (forward push)
     float **push_dx;                // [kEpMaxRanks] every rank's fp32 dX slot rows (backward push)
@@ -1060,6 +1061,7 @@ struct EpScratch {
     uint8_t *xq_recv, *xs_recv;     // MXFP8: pulled e4m3 x rows and their scales
     uint8_t *hq, *hs;               // MXFP8: h codes and scales
     long long rr_cap, rows_cap;
+    long long n_pull;               // received token rows at most: world T
     size_t bytes;
 };
 
@@ -1070,12 +1072,15 @@ EpScratch carve_ep(const moe_cfg &c, int world, bool training, void *buf)
     EpScratch e{};
     e.rr_cap = static_cast<long long>(world) * s.T * std::min<long long>(s.k, el);
     e.rows_cap = e.rr_cap + s.S * s.T;
+    e.n_pull = static_cast<long long>(world) * s.T;
     Carver cv(buf);
     e.seg = cv.take<int>(s.E + 1);
     e.offsets = cv.take<int>(el + s.S + 1);
     e.gorder = cv.take<int>(el + s.S);
     e.row_token = cv.take<int>(e.rows_cap);
-    e.row_src = cv.take<int>(e.rows_cap);
+    e.recv_idx = cv.take<int>(static_cast<long long>(world) * s.T);
+    e.uniq_src = cv.take<int>(static_cast<long long>(world) * s.T);
+    e.n_recv = cv.take<int>(1);
     e.row_slot = cv.take<int>(e.rows_cap);
     e.row_gdst = cv.take<int>(e.rr_cap);
     e.row_w = cv.take<float>(e.rows_cap);
@@ -1084,19 +1089,19 @@ EpScratch carve_ep(const moe_cfg &c, int world, bool training, void *buf)
     e.push_g = cv.take<float *>(kEpMaxRanks);
     e.sched = cv.take<int>(kSchedCounters);
     if (c.dtype == MOK_DTYPE_MXFP8) {               // (inference only)
-        e.xq_recv = cv.take<uint8_t>((s.T + e.rr_cap) * s.H);
-        e.xs_recv = cv.take<uint8_t>((s.T + e.rr_cap) * s.H / 32);
+        e.xq_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H);
+        e.xs_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H / 32);
         e.hq = cv.take<uint8_t>(e.rows_cap * s.I);
         e.hs = cv.take<uint8_t>(e.rows_cap * s.I / 32);
         e.bytes = align_up(cv.off, 256);
         return e;
     }
-    e.x_recv = cv.take<__nv_bfloat16>((s.T + e.rr_cap) * s.H);
+    e.x_recv = cv.take<__nv_bfloat16>((s.T + e.n_pull) * s.H);
     e.h = cv.take<__nv_bfloat16>(e.rows_cap * s.I);
     if (training) {
         e.gu = cv.take<__nv_bfloat16>(e.rows_cap * 2 * s.I);
         e.hw = cv.take<__nv_bfloat16>(e.rows_cap * s.I);
-        e.dy_recv = cv.take<__nv_bfloat16>((s.T + e.rr_cap) * s.H);
+        e.dy_recv = cv.take<__nv_bfloat16>((s.T + e.n_pull) * s.H);
         e.dgu = cv.take<__nv_bfloat16>(e.rows_cap * 2 * s.I);
         e.gpart = cv.take<float>(e.rr_cap * (s.I / 128));
     }
@@ -1135,8 +1140,8 @@ int launch_pull(const void *const *src, int world, int rank, void *dst, long lon
     a.dst = static_cast<uint8_t *>(dst);
     a.row_bytes = row_bytes;
     a.T = c.T; a.world = world; a.rank = rank;
-    a.seg = es.seg; a.n_seg = c.E;
-    a.row_src = es.row_src;
+    a.n_recv = es.n_recv;
+    a.row_src = es.uniq_src;
     a.status = dev.status;
     if (row_bytes % 16 == 0)
         return launch_k(ep_pull_kernel<uint4>, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", a);
@@ -1309,6 +1314,7 @@ int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void 
         v.offsets[r] = q.offsets;
         v.perm[r] = q.perm;
         v.topk_w[r] = q.topk_w;
+        v.topk_idx[r] = q.topk_idx;
         v.O[r] = q.O;
     }
     EpArgs a{};
@@ -1316,7 +1322,8 @@ int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void 
     a.T = c.T; a.H = c.H; a.k = c.top_k; a.kk = static_cast<int>(s.kk); a.S = c.n_shared; a.E_loc = el;
     a.rr_cap = static_cast<int>(es.rr_cap);
     a.seg = es.seg; a.offsets = es.offsets;
-    a.row_token = es.row_token; a.row_src = es.row_src; a.row_slot = es.row_slot; a.row_w = es.row_w;
+    a.row_token = es.row_token; a.row_slot = es.row_slot; a.row_w = es.row_w;
+    a.recv_idx = es.recv_idx; a.uniq_src = es.uniq_src; a.n_recv = es.n_recv;
     a.row_gdst = es.row_gdst; a.gorder = es.gorder;
     a.push = es.push; a.status = dev.status;
 
@@ -1328,6 +1335,7 @@ int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void 
     if (const cudaError_t e = cudaMemsetAsync(es.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
     MOK_TRY(launch_k(ep_layout_kernel, dim3(1), dim3(256), 0, stream, "ep_layout_kernel", v, a));
+    MOK_TRY(launch_k(ep_unique_kernel, dim3(1), dim3(1024), 0, stream, "ep_unique_kernel", v, a));
     MOK_TRY(launch_k(ep_rows_kernel, dim3(static_cast<unsigned>(c.E + c.n_shared * blocks_for(c.T, 256))), dim3(256), 0,
                      stream, "ep_rows_kernel", v, a));
     if (mx) {

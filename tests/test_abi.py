@@ -108,7 +108,8 @@ def test_pipelined_host_step_argument_checks():
 def test_expert_parallel_sizes_and_argument_checks():
     """moe_ep_size gives the per-rank state (the forward scratch: routing record and
     slot rows) and a receive scratch sized for the largest share a rank can get
-    (world T min(k, E/world) routed rows plus the shared rows); the EP calls refuse
+    (world T min(k, E/world) expert rows plus the shared rows, world T pulled token
+    rows); the EP calls refuse
     bad ranks, an E that world does not divide, MXFP8, row codes past 24 bits, NULL
     or short buffers -- all before touching a device (no pointer is dereferenced)."""
     T, H, E, I, k, W = 512, 7168, 256, 2048, 8, 8
@@ -116,18 +117,19 @@ def test_expert_parallel_sizes_and_argument_checks():
     state, scratch, bwd = abi.moe_ep_size(c, W)
     _, scratch_t, _ = abi.moe_ep_size(c, W, True)
     assert state == abi.moe_workspace_size(c)[1]
-    rr = W * T * min(k, E // W)
+    rr = W * T * min(k, E // W)          # expert rows: one per (token, slot) routed here
     rows = rr + T
-    assert scratch >= (T + rr) * H * 2 + rows * I * 2 + rows * 16
+    pulled = T + W * T                    # token rows: the own ones, then one per (rank, token) routed here
+    assert scratch >= pulled * H * 2 + rows * I * 2 + rows * 12
     # training adds g/u, w h, the pulled dy rows, dGU and the slot-gradient partials
-    assert scratch_t >= scratch + rows * (2 * I + I + 2 * I) * 2 + (T + rr) * H * 2 + rr * (I // 128) * 4
+    assert scratch_t >= scratch + rows * (2 * I + I + 2 * I) * 2 + pulled * H * 2 + rr * (I // 128) * 4
     # the token side of the backward: dX slot rows and the slot-gradient partials others push
     assert bwd >= T * 9 * H * 4 + T * k * (I // 128) * 4
     # E/world < k: a token puts at most E/world of its k slots on one rank
     c2 = make_cfg(200, 256, 8, 128, 2)
     _, s8, _ = abi.moe_ep_size(c2, 8)
     _, s1, _ = abi.moe_ep_size(c2, 1)
-    assert s8 >= (200 + 8 * 200 * 1) * 256 * 2 and s1 >= (200 + 200 * 2) * 256 * 2
+    assert s8 >= (200 + 8 * 200) * 256 * 2 + 8 * 200 * 128 * 2 and s1 >= (200 + 200) * 256 * 2 + 400 * 128 * 2
     for world, cfg, code in ((0, c, abi.MOK_ERR_INVALID), (9, c, abi.MOK_ERR_INVALID),
                              (3, make_cfg(64, 256, 8, 128, 2), abi.MOK_ERR_INVALID),
                              (2, make_cfg(1 << 21, 256, 8, 128, 8), abi.MOK_ERR_INVALID)):
@@ -137,7 +139,7 @@ def test_expert_parallel_sizes_and_argument_checks():
     # MXFP8: the forward without saved state only
     mxc = make_cfg(64, 256, 8, 128, 2, dtype=abi.MOK_DTYPE_MXFP8)
     mst, msc, _ = abi.moe_ep_size(mxc, 2)
-    assert msc >= (64 + 2 * 64 * 2) * (256 + 8) + (2 * 64 * 2) * (128 + 4)
+    assert msc >= (64 + 2 * 64) * (256 + 8) + (2 * 64 * 2) * (128 + 4)
     with pytest.raises(abi.MokError) as ei:
         abi.moe_ep_size(mxc, 2, True)
     assert ei.value.code == abi.MOK_ERR_UNSUPPORTED
