@@ -53,7 +53,9 @@ def parse():
     ap.add_argument("--mx-workload", default="dsv3_mxfp8",
                     help="MXFP8 forward workload measured after the main one ('none' to skip)")
     ap.add_argument("--ep-world", type=int, default=8,
-                    help="ranks of the expert-parallel forward emulated on one GPU (0 to skip)")
+                    help="ranks of the expert-parallel layer emulated on one GPU (0 to skip)")
+    ap.add_argument("--ep-only", action="store_true",
+                    help="run only the emulated expert-parallel measurement (profiling runs)")
     return ap.parse_args()
 
 
@@ -421,6 +423,15 @@ def main():
     abi.moe_set_schedule(sched)
     wl = synth.WORKLOADS[args.workload]
     wl = synth.scaled(wl, seed=wl.seed + 1000 * rank)
+    if args.ep_only:
+        W = max(1, args.ep_world)
+        ep = ep_emulated_run(synth.scaled(wl, name=wl.name + "_ep", T=wl.T // W, seed=wl.seed + 7), W, dev,
+                             args.steps, args.warmup)
+        if rank == 0:
+            print(json.dumps({"ep_emulated": ep}))
+        if world > 1:
+            dist.destroy_process_group()
+        return
     params = synth.draw_params(wl, dev)
     x = synth.draw_x(wl, dev)
     dy = synth.draw_dy(wl, dev)
