@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(256) ep_layout_kernel(EpView v, EpArgs a)
 // 1024 threads, each a run of consecutive pairs: count, block scan, write.
 __global__ void __launch_bounds__(1024) ep_unique_kernel(EpView v, EpArgs a)
 {
-    __shared__ int s_scan[1024];
+    __shared__ int s_warp[32];
     const int n = a.world * a.T;
     const int per = (n + 1023) / 1024;
     const int i0 = threadIdx.x * per, i1 = min(n, i0 + per);
@@ -134,22 +134,46 @@ __global__ void __launch_bounds__(1024) ep_unique_kernel(EpView v, EpArgs a)
         const int s = i / a.T, t = i - s * a.T;
         const int *idx = v.topk_idx[s] + (size_t)t * a.k;
         bool w = false;
-        for (int j = 0; j < a.k; ++j) w |= idx[j] >= e0 && idx[j] < e1;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)             // k <= 16: every load issued before the compares
+            if (j < a.k) {
+                const int e = idx[j];
+                w |= e >= e0 && e < e1;
+            }
         return w;
     };
+    // first pass: flags of this thread's run (kept in a mask while the run is at most 32 long)
+    unsigned mask = 0;
     int cnt = 0;
-    for (int i = i0; i < i1; ++i) cnt += wanted(i);
-    s_scan[threadIdx.x] = cnt;
-    __syncthreads();
-    for (int d = 1; d < 1024; d <<= 1) {
-        const int add = threadIdx.x >= d ? s_scan[threadIdx.x - d] : 0;
-        __syncthreads();
-        s_scan[threadIdx.x] += add;
-        __syncthreads();
-    }
-    int u = s_scan[threadIdx.x] - cnt;
     for (int i = i0; i < i1; ++i) {
-        if (wanted(i)) {
+        const bool w = wanted(i);
+        if (w && i - i0 < 32) mask |= 1u << (i - i0);
+        cnt += w;
+    }
+    // block-wide exclusive scan of the counts: within warps, then over the 32 warp sums
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int inc = cnt;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, inc, d);
+        if (lane >= d) inc += o;
+    }
+    if (lane == 31) s_warp[wid] = inc;
+    __syncthreads();
+    if (wid == 0) {
+        int ws = s_warp[lane];
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, ws, d);
+            if (lane >= d) ws += o;
+        }
+        s_warp[lane] = ws;                           // inclusive over warps
+    }
+    __syncthreads();
+    int u = (wid ? s_warp[wid - 1] : 0) + inc - cnt;
+    for (int i = i0; i < i1; ++i) {
+        const bool w = i - i0 < 32 ? (mask >> (i - i0)) & 1u : wanted(i);
+        if (w) {
             const int s = i / a.T;
             a.recv_idx[i] = u;
             a.uniq_src[u] = (s << kEpRankShift) | (i - s * a.T);
@@ -158,7 +182,7 @@ __global__ void __launch_bounds__(1024) ep_unique_kernel(EpView v, EpArgs a)
             a.recv_idx[i] = -1;
         }
     }
-    if (threadIdx.x == 1023) *a.n_recv = s_scan[1023];
+    if (threadIdx.x == 1023) *a.n_recv = s_warp[31];
 }
 
 // Sorted rows of the owner.  Blocks [0, n): segment b = (expert j, source s)
