@@ -586,6 +586,12 @@ def main():
         ep = ep_emulated_run(synth.scaled(wl, name=wl.name + "_ep", T=wl.T // args.ep_world,
                                           seed=wl.seed + 1000 * rank + 7), args.ep_world, dev, K, args.warmup)
         torch.cuda.empty_cache()
+        if args.mx_workload and args.mx_workload != "none":
+            mwl = synth.WORKLOADS[args.mx_workload]
+            ep["mxfp8_forward"] = ep_emulated_mx_run(
+                synth.scaled(mwl, name=mwl.name + "_ep", T=mwl.T // args.ep_world, seed=mwl.seed + 1000 * rank + 7),
+                args.ep_world, dev, K, args.warmup)
+            torch.cuda.empty_cache()
 
     if rank == 0:
         line = {
@@ -762,6 +768,55 @@ def ep_emulated_run(wl, W, dev, K, warmup):
            "device_status": status,
            "note": "ranks emulated in stream order on one device; no link crossed"}
     del ep, one, params, xs, ys, dys, eg, og, xw, yw, dyw
+    return out
+
+
+def ep_emulated_mx_run(wl, W, dev, K, warmup):
+    """The MXFP8 expert-parallel forward (inference) with its W ranks (wl.T tokens each)
+    on this GPU in stream order, against the one-GPU MXFP8 forward of the same tokens.
+    Each rank quantises its own experts' weights and its own x; owners pull e4m3 rows
+    and scales.  No link is crossed: the data path, not a multi-GPU measurement."""
+    import torch
+    from mixture_experts_layer_persistent_b200 import EPWorld, MoELayer, cfg_for, quantize_mxfp8_weights, synth
+    params = synth.draw_params(wl, dev)
+    full = {k: params[k] for k in ("router_w", "e_bias", "logit_bias")}
+    for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
+                        ("ws_down", "ss_down")):
+        full[name], full[sname] = quantize_mxfp8_weights(params[name]) if params.get(name) is not None else (None, None)
+    el = wl.E // W
+    ranks = []
+    for r in range(W):
+        p = dict(full)
+        for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down")):
+            p[name], p[sname] = quantize_mxfp8_weights(params[name][r * el:(r + 1) * el].contiguous())
+        ranks.append(p)
+    del params
+    xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(W)]
+    ep = EPWorld(cfg_for(wl), W, ranks, device=dev)
+    ys = [torch.empty_like(x) for x in xs]
+    one = MoELayer(cfg_for(synth.scaled(wl, T=wl.T * W)), full, training=False, device=dev)
+    xw = torch.cat(xs)
+    yw = torch.empty_like(xw)
+    for _ in range(warmup):
+        ep.forward(xs, ys)
+        one.forward(xw, yw)
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)
+    t_ep, t_one = [], []
+    for _ in range(K):
+        a, b, c, d = mk(), mk(), mk(), mk()
+        a.record(); ep.forward(xs, ys); b.record()
+        c.record(); one.forward(xw, yw); d.record()
+        t_ep.append((a, b)); t_one.append((c, d))
+    torch.cuda.synchronize()
+    ms_ep = statistics.mean(a.elapsed_time(b) for a, b in t_ep)
+    ms_one = statistics.mean(c.elapsed_time(d) for c, d in t_one)
+    out = {"workload": f"{wl.name}: MXFP8 forward of {W} ranks x {wl.T} tokens, E={wl.E} experts "
+                       f"({el} per rank), top-{wl.k}, H={wl.H}, I={wl.I}, {wl.S} shared, all ranks on one GPU",
+           "world": W, "tokens_per_rank": wl.T, "fwd_ms": ms_ep, "fwd_tokens_per_s": W * wl.T / (ms_ep / 1e3),
+           "one_gpu_fwd_ms": ms_one, "ep_over_one_gpu_fwd_time": ms_ep / ms_one, "device_status": one.status(),
+           "note": "ranks emulated in stream order on one device; no link crossed"}
+    del ep, one, full, ranks, xs, ys, xw, yw
     return out
 
 
