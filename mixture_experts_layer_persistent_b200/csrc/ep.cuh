@@ -65,10 +65,12 @@ struct EpArgs {
 // One block of 256 threads: segment sizes from every source's counts, their
 // exclusive scan (ascending (expert, source)), the owner's group ranges and
 // the push table.  E_loc * world = E <= 256 segments, one per thread.
-__global__ void __launch_bounds__(256) ep_layout_kernel(EpView v, EpArgs a)
+// s_scan: 256 + 2 + kEpMaxGroups ints of shared memory.
+__device__ __forceinline__ void ep_layout_block(const EpView &v, const EpArgs &a, int *s_scan)
 {
-    __shared__ int s_scan[256];
-    __shared__ int s_total;
+    int &s_total = s_scan[256];
+    int &s_bad = s_scan[257];
+    int *s_rows = s_scan + 258;
     const int n = a.E_loc * a.world;
     const int i = threadIdx.x;
     int c = 0;
@@ -87,7 +89,6 @@ __global__ void __launch_bounds__(256) ep_layout_kernel(EpView v, EpArgs a)
         __syncthreads();
     }
     if (i == 0) s_total = s_scan[n - 1];
-    __shared__ int s_bad;
     if (i == 0) s_bad = 0;
     __syncthreads();
     if (c < 0) atomicOr(&s_bad, 1);
@@ -104,7 +105,6 @@ __global__ void __launch_bounds__(256) ep_layout_kernel(EpView v, EpArgs a)
     if (i <= a.S) a.offsets[a.E_loc + i] = total + i * a.T;
     if (i < a.world) a.push[i] = v.O[i];
     // longest-first group order of the weight gradients (ties: lower index first)
-    __shared__ int s_rows[kEpMaxGroups];
     const int G = a.E_loc + a.S;
     for (int g = i; g < G; g += blockDim.x) {
         int rows = a.T;                                      // a shared group: the owner's T tokens
@@ -119,15 +119,22 @@ __global__ void __launch_bounds__(256) ep_layout_kernel(EpView v, EpArgs a)
     }
 }
 
+__global__ void __launch_bounds__(256) ep_layout_kernel(EpView v, EpArgs a)
+{
+    __shared__ int s_scan[256 + 2 + kEpMaxGroups];
+    ep_layout_block(v, a, s_scan);
+}
+
 // The token rows the owner receives: every (source rank, token) pair with at
 // least one selected expert on the owner, once, in (rank, token) order -- a token
-// with several of its experts on one owner crosses the link once.  One block of
-// 1024 threads, each a run of consecutive pairs: count, block scan, write.
-__global__ void __launch_bounds__(1024) ep_unique_kernel(EpView v, EpArgs a)
+// with several of its experts on one owner crosses the link once.  One block,
+// each thread a run of consecutive pairs: count, block scan, write.
+// Any block size that is a multiple of 32, up to 1024; s_warp: 32 ints of shared memory.
+__device__ __forceinline__ void ep_unique_block(const EpView &v, const EpArgs &a, int *s_warp)
 {
-    __shared__ int s_warp[32];
+    const int nt = blockDim.x, nw = nt >> 5;
     const int n = a.world * a.T;
-    const int per = (n + 1023) / 1024;
+    const int per = (n + nt - 1) / nt;
     const int i0 = threadIdx.x * per, i1 = min(n, i0 + per);
     const int e0 = a.rank * a.E_loc, e1 = e0 + a.E_loc;
     auto wanted = [&](int i) {
@@ -161,13 +168,13 @@ __global__ void __launch_bounds__(1024) ep_unique_kernel(EpView v, EpArgs a)
     if (lane == 31) s_warp[wid] = inc;
     __syncthreads();
     if (wid == 0) {
-        int ws = s_warp[lane];
+        int ws = lane < nw ? s_warp[lane] : 0;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const int o = __shfl_up_sync(0xffffffffu, ws, d);
             if (lane >= d) ws += o;
         }
-        s_warp[lane] = ws;                           // inclusive over warps
+        if (lane < nw) s_warp[lane] = ws;            // inclusive over warps
     }
     __syncthreads();
     int u = (wid ? s_warp[wid - 1] : 0) + inc - cnt;
@@ -182,16 +189,21 @@ __global__ void __launch_bounds__(1024) ep_unique_kernel(EpView v, EpArgs a)
             a.recv_idx[i] = -1;
         }
     }
-    if (threadIdx.x == 1023) *a.n_recv = s_warp[31];
+    if (threadIdx.x == nt - 1) *a.n_recv = s_warp[nw - 1];
+}
+
+__global__ void __launch_bounds__(1024) ep_unique_kernel(EpView v, EpArgs a)
+{
+    __shared__ int s_warp[32];
+    ep_unique_block(v, a, s_warp);
 }
 
 // Sorted rows of the owner.  Blocks [0, n): segment b = (expert j, source s)
 // copies source s's rows of expert e = rank E_loc + j; blocks after those:
 // the shared experts' rows of the owner's own tokens, 256 tokens per block.
-__global__ void __launch_bounds__(256) ep_rows_kernel(EpView v, EpArgs a)
+__device__ __forceinline__ void ep_rows_block(const EpView &v, const EpArgs &a, int b)
 {
     const int n = a.E_loc * a.world;
-    const int b = blockIdx.x;
     if (b < n) {
         const int j = b / a.world, s = b - j * a.world;
         const int e = a.rank * a.E_loc + j;
@@ -235,6 +247,11 @@ __global__ void __launch_bounds__(256) ep_rows_kernel(EpView v, EpArgs a)
     }
 }
 
+// blocks: E_loc world segments, then S ceil(T / 256) blocks of shared rows
+__device__ __forceinline__ int ep_row_blocks(const EpArgs &a) { return a.E_loc * a.world + a.S * ((a.T + 255) / 256); }
+
+__global__ void __launch_bounds__(256) ep_rows_kernel(EpView v, EpArgs a) { ep_rows_block(v, a, blockIdx.x); }
+
 // Pull at dispatch: dst row t = the owner's own row t for t < T, dst row T + u =
 // the u-th received (source rank, token) row (x, dy, or x's MXFP8 codes or scales).
 // One warp per row, V-sized loads (16 or 8 bytes), four in flight per lane;
@@ -250,11 +267,8 @@ struct EpPull {
 };
 
 template <typename V>
-__global__ void __launch_bounds__(256) ep_pull_kernel(EpPull a)
+__device__ __forceinline__ void ep_pull_rows(const EpPull &a, int warp, int n_warps, int lane)
 {
-    const int lane = threadIdx.x & 31;
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int n_warps = (gridDim.x * blockDim.x) >> 5;
     const int rows = a.T + min(*a.n_recv, a.world * a.T);
     const int vec = static_cast<int>(a.row_bytes / static_cast<long long>(sizeof(V)));
     for (int r = warp; r < rows; r += n_warps) {
@@ -282,6 +296,12 @@ __global__ void __launch_bounds__(256) ep_pull_kernel(EpPull a)
                 if (c + 32 * u < vec) dv[c + 32 * u] = q[u];
         }
     }
+}
+
+template <typename V>
+__global__ void __launch_bounds__(256) ep_pull_kernel(EpPull a)
+{
+    ep_pull_rows<V>(a, (blockIdx.x * blockDim.x + threadIdx.x) >> 5, (gridDim.x * blockDim.x) >> 5, threadIdx.x & 31);
 }
 
 // Per-rank pointer table in device memory (the push epilogues read it).

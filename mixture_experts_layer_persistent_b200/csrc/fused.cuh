@@ -35,11 +35,11 @@
 // The phases run the same device code as the separate kernels of the split
 // schedule, so both schedules give byte-identical results.
 //
-// Grid barrier.  Arrival tags carry a launch epoch kept in the pass's buffer:
-// every CTA reads the epoch once at the start, CTA 0 advances it right after
-// the first barrier (when every CTA has read it), so a stale tag of an earlier
-// launch (or of a CUDA-graph replay) never matches, and nothing has to be zeroed
-// before the launch.  Each CTA publishes its tag; CTA 0 waits (bounded) for
+// Grid barrier.  Arrival tags carry a marker byte and a launch epoch kept in the
+// pass's buffer: every CTA reads the epoch once at the start, CTA 0 advances it
+// right after the first barrier (when every CTA has read it), so a stale tag of
+// an earlier launch (or of a CUDA-graph replay) never matches, leftover memory
+// lacks the marker, and nothing has to be zeroed before the launch.  Each CTA publishes its tag; CTA 0 waits (bounded) for
 // every tag and then publishes the release tag, which every CTA waits for
 // (bounded).  A CTA whose barrier wait runs out records MOK_STATUS_TIMEOUT and
 // skips the rest of the work (still arriving at the later barriers), so a
@@ -57,7 +57,13 @@ constexpr int kMaxFusedCtas = 1024;
 // Above any phase's own bounded waits (a CTA stops waiting after its first
 // 2 s timeout in a phase, and P4 holds two phases).
 constexpr uint64_t kGridSyncLimitNs = 10000000000ull;
-constexpr unsigned long long kEpochMask = (1ull << 56) - 1;
+// Tag of barrier b of a launch: marker byte | 48-bit epoch | b + 1.  The marker
+// keeps leftover memory from reading as a tag: the words of a buffer's first use
+// hold whatever was there (all-ones, from an int array of -1s, would otherwise
+// read as every barrier reached), and a word matches only with the marker byte,
+// the launch's epoch and a barrier index at least b + 1.
+constexpr unsigned long long kEpochMask = (1ull << 48) - 1;
+constexpr unsigned long long kTagMarker = 0xA5ull;
 
 struct GridSync {
     unsigned long long *flags;     // [gridDim.x] arrival tag of each CTA
@@ -111,10 +117,15 @@ __device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned 
     return v;
 }
 
-// tag of barrier b: reached when the epoch matches and the barrier index is b or later
+__device__ __forceinline__ unsigned long long barrier_tag(unsigned long long epoch, int b)
+{
+    return (kTagMarker << 56) | (epoch << 8) | static_cast<unsigned long long>(b + 1);
+}
+
+// reached when the marker and the epoch match and the barrier index is b or later
 __device__ __forceinline__ bool tag_reached(unsigned long long v, unsigned long long epoch, int b)
 {
-    return (v >> 8) == epoch && static_cast<int>(v & 0xFFu) >= b + 1;
+    return (v >> 56) == kTagMarker && ((v >> 8) & kEpochMask) == epoch && static_cast<int>(v & 0xFFu) >= b + 1;
 }
 
 // Barrier b of the launch.  Returns whether this CTA is still alive.
@@ -122,7 +133,7 @@ __device__ __forceinline__ bool grid_sync(const GridSync &gs, unsigned long long
                                           int *status, volatile int *s_flag)
 {
     __syncthreads();                                 // the CTA's work of the phase is issued and done
-    const unsigned long long tag = (epoch << 8) | static_cast<unsigned long long>(b + 1);
+    const unsigned long long tag = barrier_tag(epoch, b);
     const int lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         __threadfence();

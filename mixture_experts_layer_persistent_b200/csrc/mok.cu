@@ -13,6 +13,7 @@
 
 #include "combine.cuh"
 #include "ep.cuh"
+#include "ep_fused.cuh"
 #include "fused.cuh"
 #include "fused_bwd.cuh"
 #include "gemm.cuh"
@@ -1053,7 +1054,11 @@ struct EpScratch {
     float **push;                   // [kEpMaxRanks] every rank's fp32 slot rows (forward push)
     float **push_dx;                // [kEpMaxRanks] every rank's fp32 dX slot rows (backward push)
     float **push_g;                 // [kEpMaxRanks] every rank's slot-gradient partials
-    int *sched;
+    int *sched;                     // [kSchedCounters] tile counters
+    int *ready;                     // [n_mtiles] per-M-tile readiness (persistent experts phase)
+    int *zero;                      // sched and ready: the counters the persistent phase zeroes
+    int n_zero;
+    unsigned long long *gs_flags;   // grid-barrier tags, release tag, epoch
     __nv_bfloat16 *x_recv, *h;
     __nv_bfloat16 *gu, *hw;         // training: saved g/u and w h of the owner's rows
     __nv_bfloat16 *dy_recv, *dgu;   // training: pulled dy rows, dGU
@@ -1087,7 +1092,12 @@ EpScratch carve_ep(const moe_cfg &c, int world, bool training, void *buf)
     e.push = cv.take<float *>(kEpMaxRanks);
     e.push_dx = cv.take<float *>(kEpMaxRanks);
     e.push_g = cv.take<float *>(kEpMaxRanks);
-    e.sched = cv.take<int>(kSchedCounters);
+    const int n_mtiles = static_cast<int>(e.rows_cap / BM + el + s.S + 1);
+    e.n_zero = kSchedCounters + n_mtiles;
+    e.zero = cv.take<int>(e.n_zero);
+    e.sched = e.zero;
+    e.ready = e.zero + kSchedCounters;
+    e.gs_flags = cv.take<unsigned long long>(kMaxFusedCtas + 2);
     if (c.dtype == MOK_DTYPE_MXFP8) {               // (inference only)
         e.xq_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H);
         e.xs_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H / 32);
@@ -1128,26 +1138,6 @@ EpSrcBwd carve_ep_src_bwd(const moe_cfg &c, void *buf)
     b.dxs = cv.take<float>(s.T * s.kk * s.H);
     b.bytes = align_up(cv.off, 256);
     return b;
-}
-
-// Pull every rank's rows of `row_bytes` bytes (src[s]: rank s's [T, row_bytes]
-// matrix) into dst: the owner's own T rows, then each received row.
-int launch_pull(const void *const *src, int world, int rank, void *dst, long long row_bytes, const EpScratch &es,
-                const moe_cfg &c, const DeviceInfo &dev, cudaStream_t stream)
-{
-    EpPull a{};
-    for (int r = 0; r < world; ++r) a.src[r] = static_cast<const uint8_t *>(src[r]);
-    a.dst = static_cast<uint8_t *>(dst);
-    a.row_bytes = row_bytes;
-    a.T = c.T; a.world = world; a.rank = rank;
-    a.n_recv = es.n_recv;
-    a.row_src = es.uniq_src;
-    a.status = dev.status;
-    if (row_bytes % 16 == 0)
-        return launch_k(ep_pull_kernel<uint4>, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", a);
-    if (row_bytes % 8 == 0)
-        return launch_k(ep_pull_kernel<uint2>, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", a);
-    return fail(MOK_ERR_INVALID, "expert-parallel pull: rows of a multiple of 8 bytes");
 }
 
 int check_ep(const moe_cfg *c, int world, int rank)
@@ -1300,6 +1290,93 @@ int ep_plan_bf16(const moe_cfg &c, int el, bool training, const moe_params &p, c
     return MOK_OK;
 }
 
+// Fill one pull of rows of `row_bytes` bytes from every rank's src matrix (src[s]:
+// rank s's [T, row_bytes] rows) into dst: the owner's own T rows, then each
+// received row.
+int make_pull(EpPull &a, int &unit16, const void *const *src, int world, int rank, void *dst, long long row_bytes,
+              const EpScratch &es, const moe_cfg &c, const DeviceInfo &dev);
+
+int launch_pull(const void *const *src, int world, int rank, void *dst, long long row_bytes, const EpScratch &es,
+                const moe_cfg &c, const DeviceInfo &dev, cudaStream_t stream)
+{
+    EpPull a;
+    int unit16 = 0;
+    MOK_TRY(make_pull(a, unit16, src, world, rank, dst, row_bytes, es, c, dev));
+    return unit16 ? launch_k(ep_pull_kernel<uint4>, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", a)
+                  : launch_k(ep_pull_kernel<uint2>, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_pull_kernel", a);
+}
+
+int make_pull(EpPull &a, int &unit16, const void *const *src, int world, int rank, void *dst, long long row_bytes,
+              const EpScratch &es, const moe_cfg &c, const DeviceInfo &dev)
+{
+    a = EpPull{};
+    for (int r = 0; r < world; ++r) a.src[r] = static_cast<const uint8_t *>(src[r]);
+    a.dst = static_cast<uint8_t *>(dst);
+    a.row_bytes = row_bytes;
+    a.T = c.T; a.world = world; a.rank = rank;
+    a.n_recv = es.n_recv;
+    a.row_src = es.uniq_src;
+    a.status = dev.status;
+    if (row_bytes % 8) return fail(MOK_ERR_INVALID, "expert-parallel pull: rows of a multiple of 8 bytes");
+    unit16 = row_bytes % 16 == 0;
+    return MOK_OK;
+}
+
+// The persistent experts phase: one cooperative launch (ep_fused.cuh).  src0/src1:
+// the ranks' x rows (BF16), or their x codes and x scales (MXFP8).
+template <bool MX>
+int launch_ep_fused(const moe_cfg &c, int world, int rank, const void *const *src0, const void *const *src1,
+                    const EpView &v, const EpArgs &ea, const EpScratch &es, const EpGemms &q, const DeviceInfo &dev,
+                    cudaStream_t stream)
+{
+    using F = FusedCfg<MX>;
+    if (dev.sms > kMaxFusedCtas) return fail(MOK_ERR_UNSUPPORTED, "more SMs than the grid barrier holds");
+    EpFusedArgs a{};
+    a.gs.flags = es.gs_flags;
+    a.gs.go = es.gs_flags + kMaxFusedCtas;
+    a.gs.epoch = es.gs_flags + kMaxFusedCtas + 1;
+    a.status = dev.status;
+    a.zero = es.zero;
+    a.n_zero = es.n_zero;
+    a.v = v;
+    a.ea = ea;
+    if (MX) {
+        a.n_pull = 2;
+        MOK_TRY(make_pull(a.pull[0], a.pull16[0], src0, world, rank, es.xq_recv, c.H, es, c, dev));
+        MOK_TRY(make_pull(a.pull[1], a.pull16[1], src1, world, rank, es.xs_recv, c.H / 32, es, c, dev));
+    } else {
+        a.n_pull = 1;
+        MOK_TRY(make_pull(a.pull[0], a.pull16[0], src0, world, rank, es.x_recv, 2ll * c.H, es, c, dev));
+    }
+    a.ga = q.ga;
+    a.gd = q.gd;
+    a.ga.ready = a.gd.ready = es.ready;
+    a.ga.ready_role = kReadySignal;
+    a.gd.ready_role = kReadyWait;
+    a.gd.ready_target = 4 * (c.I / 128);    // four epilogue warps per gate/up tile, I/128 tiles per M tile
+    FusedMaps m{};
+    m.gB = q.gB; m.gBs = q.gBs; m.gO = q.gO; m.gO2 = q.gO2; m.gO3 = q.gO3;
+    m.dA = q.dA; m.dB = q.dB; m.dBs = q.dBs; m.dO = q.dO;
+    m.rA = m.rB = m.rO = q.gB;                // unused by this kernel
+    cudaError_t e = cudaFuncSetAttribute(moe_ep_experts_fused_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         F::SMEM_BYTES);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(moe_ep_experts_fused_kernel)", e);
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(static_cast<unsigned>(dev.sms));
+    lc.blockDim = dim3(kFusedThreads);
+    lc.dynamicSmemBytes = F::SMEM_BYTES;
+    lc.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&lc, moe_ep_experts_fused_kernel<MX>, m, a);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaLaunchKernelEx(moe_ep_experts_fused_kernel, cooperative)", e);
+    ++t_launches;
+    return MOK_OK;
+}
+
 int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void *const *xr, void *const *sr,
                const moe_params &p, const EpScratch &es, const DeviceInfo &dev, cudaStream_t stream)
 {
@@ -1331,6 +1408,17 @@ int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void 
     const State own = carve_state(c, sr[rank], false);
     EpGemms q;
     MOK_TRY(mx ? ep_plan_mx(c, el, p, own, es, dev, q) : ep_plan_bf16(c, el, training, p, own, es, dev, q));
+    if (t_schedule == MOK_SCHEDULE_PERSISTENT) {
+        const void *xq[kEpMaxRanks] = {}, *xs[kEpMaxRanks] = {};
+        if (mx)
+            for (int r = 0; r < world; ++r) {
+                const State st_r = carve_state(c, sr[r], false);
+                xq[r] = st_r.xq;
+                xs[r] = st_r.xs;
+            }
+        return mx ? launch_ep_fused<true>(c, world, rank, xq, xs, v, a, es, q, dev, stream)
+                  : launch_ep_fused<false>(c, world, rank, xr, nullptr, v, a, es, q, dev, stream);
+    }
 
     if (const cudaError_t e = cudaMemsetAsync(es.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);

@@ -296,3 +296,78 @@ def test_mxfp8_dsv3_expert_shape_over_eight_ranks():
         y_ref = layer.forward(xs[r])
         torch.cuda.synchronize()
         assert _same(ys[r], y_ref), f"rank {r}: y differs from the MXFP8 moe_fwd"
+
+
+@pytest.mark.parametrize("mx", [False, True], ids=["bf16_train", "mxfp8"])
+def test_persistent_and_split_experts_phase_agree(mx):
+    """The owner's experts phase as one persistent launch (the default) and as the
+    split launches: y (and, for BF16, every gradient of the backward that reads the
+    forward's saved rows) byte for byte, and one launch for the persistent phase."""
+    dev = torch.device("cuda")
+    world = 4
+    wl = synth.Workload("ep_sched", T=300, H=512, E=16, k=4, I=256, S=1, Is=256, score_fn=1, n_group=4,
+                        topk_group=2, mxfp8=mx, backward=not mx, seed=65)
+    params = synth.draw_params(wl, dev)
+    xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(world)]
+    if mx:
+        _, rank_params = _mx_params(params, world, wl.E)
+    else:
+        rank_params = [split_params(params, world, r, wl.E) for r in range(world)]
+    dys = _rank_dys(wl, world, dev)
+    out = {}
+    for sched in (abi.MOK_SCHEDULE_PERSISTENT, abi.MOK_SCHEDULE_SPLIT):
+        abi.moe_set_schedule(sched)
+        try:
+            ep = EPWorld(cfg_for(wl), world, rank_params, training=not mx)
+            ys = ep.forward(xs)
+            n = None
+            if sched == abi.MOK_SCHEDULE_PERSISTENT:
+                abi.moe_ep_experts(cfg_for(wl), world, world - 1, not mx, [x.data_ptr() for x in xs],
+                                   [s.data_ptr() for s in ep.states], ep.cparams[world - 1],
+                                   ep.scratch[world - 1].data_ptr(), ep.scratch_bytes,
+                                   torch.cuda.current_stream().cuda_stream)
+                n = abi.moe_launch_count()
+            grads = None if mx else ep.backward(dys)
+            torch.cuda.synchronize()
+        finally:
+            abi.moe_set_schedule(abi.MOK_SCHEDULE_PERSISTENT)
+        assert abi.moe_status(torch.cuda.current_stream().cuda_stream) == 0
+        out[sched] = ([y.clone() for y in ys], grads, n)
+    (yp, gp, n), (ys_, gs, _) = out[abi.MOK_SCHEDULE_PERSISTENT], out[abi.MOK_SCHEDULE_SPLIT]
+    assert n == 1, "the persistent experts phase is one launch"
+    for r in range(world):
+        assert _same(yp[r], ys_[r]), f"rank {r}: y"
+        if not mx:
+            for k in gp[r]:
+                if gp[r][k] is not None:
+                    assert _same(gp[r][k], gs[r][k]), f"rank {r}: {k}"
+
+
+def test_experts_phase_on_buffers_of_ones():
+    """The persistent experts phase on state and scratch buffers filled with 0xFF bytes
+    (what an int array of -1s leaves behind) before their first use: the grid
+    barriers must not read leftover words as arrivals, so the result equals the one
+    on zeroed buffers byte for byte and no status bit is set."""
+    dev = torch.device("cuda")
+    world = 4
+    wl = synth.Workload("ep_ones", T=300, H=512, E=16, k=4, I=256, S=1, Is=256, score_fn=1, n_group=4,
+                        topk_group=2, seed=66)
+    params = synth.draw_params(wl, dev)
+    xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(world)]
+    dys = _rank_dys(wl, world, dev)
+    rank_params = [split_params(params, world, r, wl.E) for r in range(world)]
+    res = []
+    for fill in (0x00, 0xFF):
+        ep = EPWorld(cfg_for(wl), world, rank_params, training=True)
+        for t in ep.states + ep.scratch + ep.bwd:
+            t.fill_(fill)
+        ys = ep.forward(xs)
+        g = ep.backward(dys)
+        torch.cuda.synchronize()
+        assert abi.moe_status(torch.cuda.current_stream().cuda_stream) == 0, f"fill {fill:#x}"
+        res.append(([y.clone() for y in ys], g))
+    for r in range(world):
+        assert _same(res[0][0][r], res[1][0][r]), f"rank {r}: y"
+        for k in res[0][1][r]:
+            if res[0][1][r][k] is not None:
+                assert _same(res[0][1][r][k], res[1][1][r][k]), f"rank {r}: {k}"

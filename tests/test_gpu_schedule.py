@@ -177,3 +177,29 @@ def test_device_phase_stamps():
         # the phases behind the first grid barrier end after every CTA finished the first phase
         assert (t[2:].min(axis=1) >= t[1].max()).all()
     assert buf.view(abi.MOK_TRACE_POINTS, sms).max() <= bbuf.view(abi.MOK_TRACE_POINTS, sms).min()
+
+
+@pytest.mark.parametrize("wl", [CASES[1], MX_CASES[2]], ids=lambda w: w.name)
+def test_persistent_passes_on_buffers_of_ones(wl):
+    """The persistent forward and backward on ctx and scratch buffers filled with 0xFF
+    bytes before their first use (leftover memory of an int array of -1s): the grid
+    barriers must not read those words as arrivals, so every output equals the one
+    on zeroed buffers byte for byte, with no status bit set."""
+    dev = torch.device("cuda")
+    params = _params(wl, dev)
+    x = synth.draw_x(wl, dev)
+    dy = synth.draw_dy(wl, dev) if wl.backward else None
+    res = []
+    for fill in (0x00, 0xFF):
+        layer = MoELayer(cfg_for(wl), params, training=wl.backward, device=dev)
+        for t in (layer.ctx, layer.scratch, layer.bwd_scratch):
+            t.fill_(fill)
+        y = layer.forward(x).clone()
+        g = layer.backward(x, dy) if wl.backward else {}
+        torch.cuda.synchronize()
+        assert layer.status() == 0, f"fill {fill:#x}"
+        res.append((y, g))
+    assert _same(res[0][0], res[1][0]), "y"
+    for k, v in res[0][1].items():
+        if v is not None:
+            assert _same(v, res[1][1][k]), k
