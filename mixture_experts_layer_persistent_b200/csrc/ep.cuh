@@ -317,12 +317,12 @@ __global__ void ep_table_kernel(EpTable t, float **dst, int n)
 // owner computed (nt floats per row, its down dgrad's N tiles) go to the row's
 // source rank, at the row's position in the source's sorted rows, where the
 // slot gradients are formed.  One thread per (row, tile).
-__global__ void __launch_bounds__(256) ep_push_gpart_kernel(const float *gpart, const int *row_gdst, const int *seg,
-                                                            int n_seg, int nt, float **gdst, int world, int tk,
-                                                            int *status)
+__device__ __forceinline__ void ep_push_gpart(const float *gpart, const int *row_gdst, const int *seg, int n_seg,
+                                              int nt, float *const *gdst, int world, int tk, int *status,
+                                              long long first, long long stride)
 {
     const long long n = static_cast<long long>(seg[n_seg]) * nt;
-    for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n; i += static_cast<long long>(gridDim.x) * 256) {
+    for (long long i = first; i < n; i += stride) {
         const int r = static_cast<int>(i / nt), j = static_cast<int>(i - static_cast<long long>(r) * nt);
         const int code = row_gdst[r];
         const int s = code >> kEpRankShift, q = code & kEpRowMask;
@@ -332,6 +332,14 @@ __global__ void __launch_bounds__(256) ep_push_gpart_kernel(const float *gpart, 
         }
         gdst[s][static_cast<size_t>(q) * nt + j] = gpart[i];
     }
+}
+
+__global__ void __launch_bounds__(256) ep_push_gpart_kernel(const float *gpart, const int *row_gdst, const int *seg,
+                                                            int n_seg, int nt, float **gdst, int world, int tk,
+                                                            int *status)
+{
+    ep_push_gpart(gpart, row_gdst, seg, n_seg, nt, gdst, world, tk, status, blockIdx.x * 256ll + threadIdx.x,
+                  static_cast<long long>(gridDim.x) * 256);
 }
 
 }  // namespace mok

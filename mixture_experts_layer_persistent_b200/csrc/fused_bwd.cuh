@@ -122,6 +122,47 @@ __device__ __forceinline__ void fused_bwd_stamp(const FusedBwdArgs &a, int point
     if (a.trace && threadIdx.x == 0) a.trace[static_cast<size_t>(point) * gridDim.x + blockIdx.x] = globaltimer();
 }
 
+// Q1-Q3 of a persistent backward: both dgrads and both weight gradients.  No
+// barrier between the four GEMMs: a CTA moves on when a GEMM's tile counter is
+// exhausted, so the next GEMM starts on SMs that the previous one's tail leaves
+// idle.  The gate/up dgrad waits per M tile and the gate/up weight gradient per
+// group for the down dgrad's dGU rows.  trace: stamps 2 and 3 (or null).
+template <class F, bool N256>
+__device__ __forceinline__ void bwd_expert_gemms(uint8_t *smem, uint64_t *gbars, int *aux, uint64_t *rbars,
+                                                 uint32_t tmem_base, const FusedBwdMaps &m, const GemmArgs &g1,
+                                                 const GemmArgs &g2, const GemmArgs &g2r, const GemmArgs &g3,
+                                                 const GemmArgs &g4, const GemmArgs &g4r, int g2_units, int g4_units,
+                                                 unsigned long long *trace)
+{
+    constexpr int GB = kGemmBarBytes / 8;           // uint64 per GEMM barrier block
+    constexpr int RB = F::ResDown::BAR_BYTES / 8;
+    auto stamp = [&](int point) {
+        if (trace && threadIdx.x == 0) trace[static_cast<size_t>(point) * gridDim.x + blockIdx.x] = globaltimer();
+    };
+    tc_fence_after();
+    gemm_phase<typename F::DgradDown>(smem, gbars, aux, tmem_base, m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1);
+    tc_fence_after();
+    gemm_phase<typename F::DgradGU>(smem, gbars + GB, aux, tmem_base, m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O, g3);
+    stamp(2);
+    tc_fence_after();
+    gemm_phase<typename F::WgradDown>(smem, gbars + 2 * GB, aux, tmem_base, m.w2B, m.w2B, m.w2B, m.w2O, m.w2O2, m.w2O,
+                                      g2);
+    if constexpr (N256) {
+        if (g2_units > 0) {
+            tc_fence_after();
+            wgrad_resident_phase<typename F::ResDown>(smem, rbars, tmem_base, m.w2B, m.w2B, m.w2O, m.w2O2, g2r);
+        }
+    }
+    stamp(3);
+    tc_fence_after();
+    gemm_phase<typename F::WgradGU>(smem, gbars + 3 * GB, aux, tmem_base, m.w4A, m.w4A, m.w4A, m.w4O, m.w4O2, m.w4O,
+                                    g4);
+    if (g4_units > 0) {
+        tc_fence_after();
+        wgrad_resident_phase<typename F::ResGU>(smem, rbars + RB, tmem_base, m.w4A, m.w4A, m.w4O, m.w4O2, g4r);
+    }
+}
+
 template <bool N256, bool MX>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     moe_bwd_fused_kernel(const __grid_constant__ FusedBwdMaps m, const __grid_constant__ FusedBwdArgs a)
@@ -137,8 +178,6 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     const int warp = threadIdx.x >> 5;
     const long long gtid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
     const long long gstride = static_cast<long long>(gridDim.x) * blockDim.x;
-    constexpr int GB = kGemmBarBytes / 8;           // uint64 per GEMM barrier block
-    constexpr int RB = F::ResDown::BAR_BYTES / 8;
 
     if (threadIdx.x == 0) reinterpret_cast<volatile unsigned long long *>(tmem_slot + 2)[0] = *a.gs.epoch & kEpochMask;
     if (warp == 1) tmem_alloc(tmem_slot, 512);
@@ -169,34 +208,9 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.gs.epoch = (epoch + 1) & kEpochMask;
 
     // ---------------------------------------------------------------- Q1, Q2, Q3 (both dgrads, both weight gradients)
-    // No barrier between the four GEMMs: a CTA moves on when a GEMM's tile counter
-    // is exhausted, so the next GEMM starts on SMs that the previous one's tail
-    // leaves idle.  The gate/up weight gradient waits per group for that group's dGU.
     if (alive) {
-        tc_fence_after();
-        gemm_phase<typename F::DgradDown>(smem, gbars, aux, tmem_base, m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O,
-                                          a.g1);
-        tc_fence_after();
-        gemm_phase<typename F::DgradGU>(smem, gbars + GB, aux, tmem_base, m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O,
-                                        a.g3);
-        fused_bwd_stamp(a, 2);
-        tc_fence_after();
-        gemm_phase<typename F::WgradDown>(smem, gbars + 2 * GB, aux, tmem_base, m.w2B, m.w2B, m.w2B, m.w2O, m.w2O2,
-                                          m.w2O, a.g2);
-        if constexpr (N256) {
-            if (a.g2_units > 0) {
-                tc_fence_after();
-                wgrad_resident_phase<typename F::ResDown>(smem, rbars, tmem_base, m.w2B, m.w2B, m.w2O, m.w2O2, a.g2r);
-            }
-        }
-        fused_bwd_stamp(a, 3);
-        tc_fence_after();
-        gemm_phase<typename F::WgradGU>(smem, gbars + 3 * GB, aux, tmem_base, m.w4A, m.w4A, m.w4A, m.w4O, m.w4O2,
-                                        m.w4O, a.g4);
-        if (a.g4_units > 0) {
-            tc_fence_after();
-            wgrad_resident_phase<typename F::ResGU>(smem, rbars + RB, tmem_base, m.w4A, m.w4A, m.w4O, m.w4O2, a.g4r);
-        }
+        bwd_expert_gemms<F, N256>(smem, gbars, aux, rbars, tmem_base, m, a.g1, a.g2, a.g2r, a.g3, a.g4, a.g4r,
+                                  a.g2_units, a.g4_units, a.trace);
     } else {
         fused_bwd_stamp(a, 2);
         fused_bwd_stamp(a, 3);

@@ -1059,6 +1059,7 @@ struct EpScratch {
     int *zero;                      // sched and ready: the counters the persistent phase zeroes
     int n_zero;
     unsigned long long *gs_flags;   // grid-barrier tags, release tag, epoch
+    int *mt_base;                   // [G + 1] first 128-row M tile of each group (persistent backward phase)
     __nv_bfloat16 *x_recv, *h;
     __nv_bfloat16 *gu, *hw;         // training: saved g/u and w h of the owner's rows
     __nv_bfloat16 *dy_recv, *dgu;   // training: pulled dy rows, dGU
@@ -1098,6 +1099,7 @@ EpScratch carve_ep(const moe_cfg &c, int world, bool training, void *buf)
     e.sched = e.zero;
     e.ready = e.zero + kSchedCounters;
     e.gs_flags = cv.take<unsigned long long>(kMaxFusedCtas + 2);
+    e.mt_base = cv.take<int>(el + s.S + 1);
     if (c.dtype == MOK_DTYPE_MXFP8) {               // (inference only)
         e.xq_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H);
         e.xs_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H / 32);
@@ -1445,6 +1447,71 @@ int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void 
     return launch_gemm<typename FusedCfg<false>::Down>(q.dA, q.dB, q.dBs, q.dO, q.dO, q.dO, q.gd, dev.sms, stream);
 }
 
+// The persistent backward experts phase: one cooperative launch (ep_fused.cuh).
+template <bool N256>
+int launch_ep_bwd_fused(const moe_cfg &c, int world, int rank, const void *const *dyr, const EpTable &tdx,
+                        const EpTable &tg, const EpScratch &es, const FusedBwdMaps &m, const GemmArgs &g1,
+                        const GemmArgs &g2, const GemmArgs &g3, const GemmArgs &g4, int g2_units, int g4_units,
+                        const DeviceInfo &dev, cudaStream_t stream)
+{
+    using F = FusedBwdCfg<N256, false>;
+    if (dev.sms > kMaxFusedCtas) return fail(MOK_ERR_UNSUPPORTED, "more SMs than the grid barrier holds");
+    EpBwdFusedArgs a{};
+    a.gs.flags = es.gs_flags;
+    a.gs.go = es.gs_flags + kMaxFusedCtas;
+    a.gs.epoch = es.gs_flags + kMaxFusedCtas + 1;
+    a.status = dev.status;
+    a.zero = es.zero;
+    a.n_zero = es.n_zero;
+    MOK_TRY(make_pull(a.pull, a.pull16, dyr, world, rank, es.dy_recv, 2ll * c.H, es, c, dev));
+    a.tdx = tdx;
+    a.tg = tg;
+    a.push_dx = es.push_dx;
+    a.push_g = es.push_g;
+    a.world = world;
+    a.g1 = g1;
+    a.g1.ready = es.ready;
+    a.g1.ready_role = kReadySignal;
+    a.g2 = a.g2r = g2;
+    a.g3 = g3;
+    a.g3.ready = es.ready;
+    a.g3.ready_role = kReadyWait;
+    a.g3.ready_target = 4 * g1.n_tiles;     // four epilogue warps per down-dgrad tile, its N tiles per M tile
+    a.g4 = a.g4r = g4;
+    a.g4.ready = a.g4r.ready = es.ready;
+    a.g4.ready_role = a.g4r.ready_role = kReadyWaitGroup;
+    a.g4.ready_target = a.g4r.ready_target = 4 * g1.n_tiles;
+    a.g4.mt_base = a.g4r.mt_base = es.mt_base;
+    a.g2_units = g2_units;
+    a.g4_units = g4_units;
+    a.offsets_all = es.offsets;
+    a.mt_base = es.mt_base;
+    a.gpart = es.gpart;
+    a.row_gdst = es.row_gdst;
+    a.seg = es.seg;
+    a.n_seg = c.E;
+    a.nt = g1.n_tiles;
+    a.tk = c.T * c.top_k;
+    cudaError_t e = cudaFuncSetAttribute(moe_ep_bwd_experts_fused_kernel<N256>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM_BYTES);
+    if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(moe_ep_bwd_experts_fused_kernel)", e);
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(static_cast<unsigned>(dev.sms));
+    lc.blockDim = dim3(kFusedThreads);
+    lc.dynamicSmemBytes = F::SMEM_BYTES;
+    lc.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&lc, moe_ep_bwd_experts_fused_kernel<N256>, m, a);
+    if (e != cudaSuccess)
+        return fail(MOK_ERR_LAUNCH, "cudaLaunchKernelEx(moe_ep_bwd_experts_fused_kernel, cooperative)", e);
+    ++t_launches;
+    return MOK_OK;
+}
+
 // Backward, owner side: pull dy rows, down dgrad (SwiGLU backward, slot-gradient
 // partials pushed to the rows' ranks), gate/up dgrad (dX rows pushed into the
 // dX slot rows of the tokens' ranks), both weight gradients of the owner's experts
@@ -1555,6 +1622,11 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
     const int g4_grid = static_cast<int>(t4 < dev.sms ? t4 : dev.sms);
     const int g4_units = static_cast<int>(G * g4.n_tiles * ((g4.m_tiles + g4.m_per_unit - 1) / g4.m_per_unit));
 
+    if (t_schedule == MOK_SCHEDULE_PERSISTENT)
+        return n256 ? launch_ep_bwd_fused<true>(c, world, rank, dyr, tdx, tg, es, m, g1, g2, g3, g4, g2_units, g4_units,
+                                                dev, stream)
+                    : launch_ep_bwd_fused<false>(c, world, rank, dyr, tdx, tg, es, m, g1, g2, g3, g4, g2_units, g4_units,
+                                                 dev, stream);
     if (const cudaError_t e = cudaMemsetAsync(es.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
     MOK_TRY(launch_k(ep_table_kernel, dim3(1), dim3(32), 0, stream, "ep_table_kernel", tdx, es.push_dx, world));
