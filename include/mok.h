@@ -475,13 +475,17 @@ const char *moe_last_error(void);
  * multiple of world (1 <= world <= MOK_EP_MAX_RANKS); T is the tokens of ONE
  * rank.  Rank r holds its own T tokens and owns the routed experts
  * [r E/world, (r+1) E/world); the router and the shared experts run on every
- * rank for its own tokens.  BF16 forward and backward; MXFP8 forward without
- * saved state (MOK_ERR_UNSUPPORTED for an MXFP8 training forward or backward:
- * each rank then quantises its x in moe_ep_route, the owners pull its e4m3 rows
- * and scales, and the slot rows are bf16; the rank's w_* are e4m3 codes with
- * s_* scales packed for its own [E/world * 2I, H] and [E/world * H, I] tensors,
- * as moe_quantize_mxfp8_weights writes them for that slice).  T (top_k +
- * n_shared) must stay below 2^24.
+ * rank for its own tokens.  BF16 and MXFP8, forward and backward (an MXFP8
+ * training forward or backward needs I to be a multiple of 256,
+ * MOK_ERR_UNSUPPORTED otherwise).  MXFP8: each rank quantises its x in
+ * moe_ep_route and the owners pull its e4m3 rows and scales (the forward's slot
+ * rows are bf16); in the backward the owner pulls the bf16 dy rows and
+ * quantises them itself (1x32 blocks along H depend on the row alone) and
+ * decodes the pulled x codes for the gate/up weight gradient; the rank's w_*
+ * are e4m3 codes with s_* scales packed for its own [E/world * 2I, H] and
+ * [E/world * H, I] tensors (moe_quantize_mxfp8_weights of that slice) and, for
+ * the backward, wt_* / st_* the transposed copies of the slice
+ * (moe_quantize_mxfp8_weights_t).  T (top_k + n_shared) must stay below 2^24.
  *
  * Buffers (caller-allocated device memory, 16-byte aligned), from moe_ep_size:
  *   state    per rank, state_bytes: the rank's routing record and its fp32 slot

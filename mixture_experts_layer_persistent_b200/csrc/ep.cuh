@@ -25,6 +25,7 @@
 #include <cstdint>
 
 #include "mok.h"
+#include "quant.cuh"
 
 namespace mok {
 
@@ -302,6 +303,47 @@ template <typename V>
 __global__ void __launch_bounds__(256) ep_pull_kernel(EpPull a)
 {
     ep_pull_rows<V>(a, (blockIdx.x * blockDim.x + threadIdx.x) >> 5, (gridDim.x * blockDim.x) >> 5, threadIdx.x & 31);
+}
+
+// MXFP8 training, owner side, over its own and received rows (T + *n_recv, H
+// wide): quantise the pulled bf16 dy rows into e4m3 codes and row-major ue8m0
+// scales (the MXFP8 down dgrad's operand; a row's 1x32 blocks depend on that row
+// alone, so they equal the token's rank's own quantisation), and decode the
+// pulled x codes into bf16 (the gate/up weight gradient's operand, exactly the
+// values the forward used).  One 32-element block per thread and step.
+struct EpMxPrep {
+    const __nv_bfloat16 *dy;       // [rows, H] pulled dy rows
+    uint8_t *dyq, *dys;            // [rows, H], [rows, H / 32]
+    const uint8_t *xq, *xs;        // [rows, H], [rows, H / 32] pulled x codes and scales
+    __nv_bfloat16 *xdq;            // [rows, H] decoded x
+    const int *n_recv;
+    int T, world, H;
+};
+
+__device__ __forceinline__ void ep_mx_prepare(const EpMxPrep &a, long long first, long long stride)
+{
+    const long long kb32 = a.H / 32;
+    const long long nb = (a.T + min(*a.n_recv, a.world * a.T)) * kb32;
+    for (long long b = first; b < nb; b += stride) {
+        quantize_block(b, a.dy, a.dyq, a.dys, kb32, 0);
+        const int e = static_cast<int>(a.xs[b]) - 127;
+        const uint4 *q = reinterpret_cast<const uint4 *>(a.xq + b * 32);
+        uint32_t w[8];
+        const uint4 q0 = q[0], q1 = q[1];
+        w[0] = q0.x; w[1] = q0.y; w[2] = q0.z; w[3] = q0.w; w[4] = q1.x; w[5] = q1.y; w[6] = q1.z; w[7] = q1.w;
+        uint32_t p[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            p[i] = pack_bf16x2(mx_decode(w[i >> 1] >> (16 * (i & 1)), e), mx_decode(w[i >> 1] >> (16 * (i & 1) + 8), e));
+        uint4 *d = reinterpret_cast<uint4 *>(a.xdq + b * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) d[i] = make_uint4(p[4 * i], p[4 * i + 1], p[4 * i + 2], p[4 * i + 3]);
+    }
+}
+
+__global__ void __launch_bounds__(256) ep_mx_prepare_kernel(EpMxPrep a)
+{
+    ep_mx_prepare(a, blockIdx.x * 256ll + threadIdx.x, static_cast<long long>(gridDim.x) * 256);
 }
 
 // Per-rank pointer table in device memory (the push epilogues read it).

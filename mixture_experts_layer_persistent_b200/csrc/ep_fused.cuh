@@ -104,11 +104,14 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     }
 }
 
-// The owner's backward experts phase as one persistent launch (BF16):
+// The owner's backward experts phase as one persistent launch:
 //
 //   B0  zero the launch's counters; the per-rank dX and slot-gradient tables; the
 //       first 128-row M tile of every group; the pull of the dy rows (all warps)
 //   --- grid barrier
+//   B0b MXFP8 only: the pulled dy rows quantised, the pulled x codes decoded
+//       (ep_mx_prepare)
+//   --- grid barrier (MXFP8 only)
 //   B1  down dgrad, gate/up dgrad (its push epilogue stores each dX row into the
 //       dX slot rows of the token's rank), both weight gradients: the persistent
 //       backward's GEMM phases (bwd_expert_gemms), with their per-tile readiness
@@ -131,13 +134,14 @@ struct EpBwdFusedArgs {
     const float *gpart;            // the owner's slot-gradient partials, [routed rows, nt]
     const int *row_gdst, *seg;
     int n_seg, nt, tk;
+    EpMxPrep prep;                 // MXFP8: dy quantised and x decoded after the pull (B0b)
 };
 
-template <bool N256>
+template <bool N256, bool MX>
 __global__ void __launch_bounds__(kFusedThreads, 1)
     moe_ep_bwd_experts_fused_kernel(const __grid_constant__ FusedBwdMaps m, const __grid_constant__ EpBwdFusedArgs a)
 {
-    using F = FusedBwdCfg<N256, false>;
+    using F = FusedBwdCfg<N256, MX>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *gbars = reinterpret_cast<uint64_t *>(smem + F::GEMM_RING);
@@ -175,6 +179,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1)
     int nb = 0;
     bool alive = grid_sync(a.gs, epoch, nb++, true, a.status, s_flag);
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.gs.epoch = (epoch + 1) & kEpochMask;   // every CTA has read it
+
+    // ---------------------------------------------------------------- B0b (MXFP8)
+    if constexpr (MX) {
+        if (alive) ep_mx_prepare(a.prep, gtid, gstride);
+        alive = grid_sync(a.gs, epoch, nb++, alive, a.status, s_flag);
+    }
 
     // ---------------------------------------------------------------- B1
     if (alive)

@@ -1233,8 +1233,16 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                 } else if constexpr (C::EPI == EPI_PUSH && C::MX) {
                     const int dst_row = valid ? args.row_slot[t.m0 + row] : 0;
                     if (args.out_f32) {
-                        // MXFP8 gate/up dgrad: fp32 rows pushed into their (token, slot) row
-                        float *dst = args.out_f32 + (size_t)dst_row * args.ldo + t.nt * C::BN;
+                        // MXFP8 gate/up dgrad: fp32 rows pushed into their (token, slot) row; across
+                        // ranks into the dX slot rows of the token's rank, with plain stores
+                        float *fbase = args.out_f32;
+                        int frow = dst_row;
+                        if (args.push_dst) {
+                            fbase = args.push_dst[dst_row >> 24];
+                            frow = dst_row & ((1 << 24) - 1);
+                        }
+                        const bool ftma = full && !args.push_dst;
+                        float *dst = fbase + (size_t)frow * args.ldo + t.nt * C::BN;
 #pragma unroll 1
                         for (int c = 0; c < C::BN; c += 32) {
                             float v[32];
@@ -1247,7 +1255,7 @@ __device__ __forceinline__ void gemm_phase(uint8_t *smem, uint64_t *bar_block, i
                             }
 #pragma unroll
                             for (int i = 0; i < 32; ++i) p[i] = __float_as_uint(v[i]);
-                            if (full) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
+                            if (ftma) store_block_scatter(stg, p, lane, &tmO, t.nt * C::BN + c, dst_row);
                             else if (valid) store_row_direct(dst + c, p);
                         }
                     } else {

@@ -1066,6 +1066,8 @@ struct EpScratch {
     float *gpart;                   // training: slot-gradient partials of the owner's routed rows
     uint8_t *xq_recv, *xs_recv;     // MXFP8: pulled e4m3 x rows and their scales
     uint8_t *hq, *hs;               // MXFP8: h codes and scales
+    uint8_t *dyq_recv, *dys_recv;   // MXFP8 training: the pulled dy rows quantised
+    uint8_t *dguq, *dgus;           // MXFP8 training: dGU codes and scales
     long long rr_cap, rows_cap;
     long long n_pull;               // received token rows at most: world T
     size_t bytes;
@@ -1100,11 +1102,26 @@ EpScratch carve_ep(const moe_cfg &c, int world, bool training, void *buf)
     e.ready = e.zero + kSchedCounters;
     e.gs_flags = cv.take<unsigned long long>(kMaxFusedCtas + 2);
     e.mt_base = cv.take<int>(el + s.S + 1);
-    if (c.dtype == MOK_DTYPE_MXFP8) {               // (inference only)
+    if (c.dtype == MOK_DTYPE_MXFP8) {
         e.xq_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H);
         e.xs_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H / 32);
         e.hq = cv.take<uint8_t>(e.rows_cap * s.I);
         e.hs = cv.take<uint8_t>(e.rows_cap * s.I / 32);
+        if (training) {
+            // forward: g/u, the dequantised h, w Q(h); backward: the decoded x rows, the
+            // pulled dy rows and their quantisation, dGU in bf16 and MXFP8, the partials
+            e.gu = cv.take<__nv_bfloat16>(e.rows_cap * 2 * s.I);
+            e.h = cv.take<__nv_bfloat16>(e.rows_cap * s.I);
+            e.hw = cv.take<__nv_bfloat16>(e.rows_cap * s.I);
+            e.x_recv = cv.take<__nv_bfloat16>((s.T + e.n_pull) * s.H);
+            e.dy_recv = cv.take<__nv_bfloat16>((s.T + e.n_pull) * s.H);
+            e.dyq_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H);
+            e.dys_recv = cv.take<uint8_t>((s.T + e.n_pull) * s.H / 32);
+            e.dgu = cv.take<__nv_bfloat16>(e.rows_cap * 2 * s.I);
+            e.dguq = cv.take<uint8_t>(e.rows_cap * 2 * s.I);
+            e.dgus = cv.take<uint8_t>(e.rows_cap * 2 * s.I / 32);
+            e.gpart = cv.take<float>(e.rr_cap * (s.I / 128));
+        }
         e.bytes = align_up(cv.off, 256);
         return e;
     }
@@ -1181,7 +1198,7 @@ struct EpGemms {
 // MXFP8 (inference): gate/up on the pulled x codes with the SwiGLU epilogue
 // requantising h, down with the push epilogue storing bf16 rows into the slot
 // rows of the tokens' ranks.
-int ep_plan_mx(const moe_cfg &c, int el, const moe_params &p, const State &own, const EpScratch &es,
+int ep_plan_mx(const moe_cfg &c, int el, bool training, const moe_params &p, const State &own, const EpScratch &es,
                const DeviceInfo &dev, EpGemms &q)
 {
     const Shapes s = shapes(c);
@@ -1212,6 +1229,9 @@ int ep_plan_mx(const moe_cfg &c, int el, const moe_params &p, const State &own, 
     ga.gather_ld = c.H;
     ga.out = reinterpret_cast<__nv_bfloat16 *>(es.hq);
     ga.out_scales = es.hs;
+    ga.out2 = training ? es.gu : nullptr;       // training: g/u, the dequantised h, w Q(h)
+    ga.out_hb = training ? es.h : nullptr;
+    ga.out3 = training ? es.hw : nullptr;
     ga.sfa_src = es.xs_recv;
     ga.sfb_src = p.s_gate_up;
     ga.sfb_src_s = s.S ? p.ss_gate_up : p.s_gate_up;
@@ -1228,6 +1248,7 @@ int ep_plan_mx(const moe_cfg &c, int el, const moe_params &p, const State &own, 
     gd.b_half = 0;
     gd.out = reinterpret_cast<__nv_bfloat16 *>(own.O);
     gd.out_scales = nullptr;
+    gd.out2 = gd.out3 = gd.out_hb = nullptr;
     gd.ldo = c.H;
     gd.gather_src = nullptr;
     gd.push_dst = es.push;
@@ -1409,7 +1430,7 @@ int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void 
     const bool mx = c.dtype == MOK_DTYPE_MXFP8;
     const State own = carve_state(c, sr[rank], false);
     EpGemms q;
-    MOK_TRY(mx ? ep_plan_mx(c, el, p, own, es, dev, q) : ep_plan_bf16(c, el, training, p, own, es, dev, q));
+    MOK_TRY(mx ? ep_plan_mx(c, el, training, p, own, es, dev, q) : ep_plan_bf16(c, el, training, p, own, es, dev, q));
     if (t_schedule == MOK_SCHEDULE_PERSISTENT) {
         const void *xq[kEpMaxRanks] = {}, *xs[kEpMaxRanks] = {};
         if (mx)
@@ -1448,13 +1469,13 @@ int ep_experts(const moe_cfg &c, int world, int rank, bool training, const void 
 }
 
 // The persistent backward experts phase: one cooperative launch (ep_fused.cuh).
-template <bool N256>
+template <bool N256, bool MX>
 int launch_ep_bwd_fused(const moe_cfg &c, int world, int rank, const void *const *dyr, const EpTable &tdx,
                         const EpTable &tg, const EpScratch &es, const FusedBwdMaps &m, const GemmArgs &g1,
                         const GemmArgs &g2, const GemmArgs &g3, const GemmArgs &g4, int g2_units, int g4_units,
-                        const DeviceInfo &dev, cudaStream_t stream)
+                        const EpMxPrep &prep, const DeviceInfo &dev, cudaStream_t stream)
 {
-    using F = FusedBwdCfg<N256, false>;
+    using F = FusedBwdCfg<N256, MX>;
     if (dev.sms > kMaxFusedCtas) return fail(MOK_ERR_UNSUPPORTED, "more SMs than the grid barrier holds");
     EpBwdFusedArgs a{};
     a.gs.flags = es.gs_flags;
@@ -1492,7 +1513,8 @@ int launch_ep_bwd_fused(const moe_cfg &c, int world, int rank, const void *const
     a.n_seg = c.E;
     a.nt = g1.n_tiles;
     a.tk = c.T * c.top_k;
-    cudaError_t e = cudaFuncSetAttribute(moe_ep_bwd_experts_fused_kernel<N256>,
+    a.prep = prep;
+    cudaError_t e = cudaFuncSetAttribute(moe_ep_bwd_experts_fused_kernel<N256, MX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, F::SMEM_BYTES);
     if (e != cudaSuccess) return fail(MOK_ERR_LAUNCH, "cudaFuncSetAttribute(moe_ep_bwd_experts_fused_kernel)", e);
     cudaLaunchConfig_t lc = {};
@@ -1505,7 +1527,7 @@ int launch_ep_bwd_fused(const moe_cfg &c, int world, int rank, const void *const
     attr[0].val.cooperative = 1;
     lc.attrs = attr;
     lc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&lc, moe_ep_bwd_experts_fused_kernel<N256>, m, a);
+    e = cudaLaunchKernelEx(&lc, moe_ep_bwd_experts_fused_kernel<N256, MX>, m, a);
     if (e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaLaunchKernelEx(moe_ep_bwd_experts_fused_kernel, cooperative)", e);
     ++t_launches;
@@ -1526,6 +1548,7 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
     const int el = c.E / world;
     const long long G = el + s.S;
     const bool n256 = c.I % 256 == 0;
+    const bool mx = c.dtype == MOK_DTYPE_MXFP8;
     EpTable tdx{}, tg{};
     for (int r = 0; r < world; ++r) {
         const EpSrcBwd q = carve_ep_src_bwd(c, br[r]);
@@ -1549,8 +1572,11 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
 
     FusedBwdMaps m;
     // down dgrad: dh = w (dy W_down), SwiGLU backward -> dGU, slot-gradient partials
-    if (!make_tmap(&m.d1B, p.w_down, s.I, el * s.H, 64, 64, 2) ||
-        !make_tmap(&m.d1Bs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : el) * s.H, 64, 64, 2) ||
+    // (MXFP8: on the quantised dy rows against W_down^T quantised along H)
+    if (!(mx ? make_tmap(&m.d1B, p.wt_down, s.H, el * s.I, 128, 256, 1) &&
+                   make_tmap(&m.d1Bs, s.S ? p.wst_down : p.wt_down, s.H, (s.S ? s.S : el) * s.I, 128, 256, 1)
+             : make_tmap(&m.d1B, p.w_down, s.I, el * s.H, 64, 64, 2) &&
+                   make_tmap(&m.d1Bs, s.S ? p.ws_down : p.w_down, s.I, (s.S ? s.S : el) * s.H, 64, 64, 2)) ||
         !make_tmap(&m.d1O, es.dgu, 2 * s.I, es.rows_cap, 64, 32, 2))
         return fail(MOK_ERR_INVALID, "tensor map (expert-parallel down dgrad)");
     GemmArgs g1 = base;
@@ -1562,6 +1588,19 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
     g1.gpart = es.gpart;
     g1.out = es.dgu;
     g1.n_tiles = n256 ? c.I / 256 : c.I / 128;
+    if (mx) {
+        g1.num_kb = c.H / 128;
+        g1.b_rows_per_group = c.I;
+        g1.gather_src = reinterpret_cast<const __nv_bfloat16 *>(es.dyq_recv);
+        g1.sfa_src = es.dys_recv;
+        g1.sf_ld = c.H / 32;
+        g1.sfb_src = p.st_down;
+        g1.sfb_src_s = s.S ? p.sst_down : p.st_down;
+        g1.sfb_row_tiles = static_cast<int>(el * s.I / 128);
+        g1.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : el) * s.I / 128);
+        g1.out_q = es.dguq;
+        g1.out_scales = es.dgus;
+    }
 
     // down wgrad: dW_down[g] = sum_r dy[token r]^T (w_r h_r)
     if (!make_tmap(&m.w2O, gr.dw_down, s.I, el * s.H, 64, 32, 2) ||
@@ -1588,9 +1627,12 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
     const int g2_grid = static_cast<int>(t2 < dev.sms ? t2 : dev.sms);
 
     // gate/up dgrad: dX rows = dGU W_gate_up, pushed into the tokens' ranks
-    if (!make_tmap(&m.d3A, es.dgu, 2 * s.I, es.rows_cap, BK, 128, 2) ||
-        !make_tmap(&m.d3B, p.w_gate_up, s.H, el * 2 * s.I, 64, 64, 2) ||
-        !make_tmap(&m.d3Bs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : el) * 2 * s.I, 64, 64, 2) ||
+    if (!(mx ? make_tmap(&m.d3A, es.dguq, 2 * s.I, es.rows_cap, 128, 128, 1) &&
+                   make_tmap(&m.d3B, p.wt_gate_up, 2 * s.I, el * s.H, 128, 256, 1) &&
+                   make_tmap(&m.d3Bs, s.S ? p.wst_gate_up : p.wt_gate_up, 2 * s.I, (s.S ? s.S : el) * s.H, 128, 256, 1)
+             : make_tmap(&m.d3A, es.dgu, 2 * s.I, es.rows_cap, BK, 128, 2) &&
+                   make_tmap(&m.d3B, p.w_gate_up, s.H, el * 2 * s.I, 64, 64, 2) &&
+                   make_tmap(&m.d3Bs, s.S ? p.ws_gate_up : p.w_gate_up, s.H, (s.S ? s.S : el) * 2 * s.I, 64, 64, 2)) ||
         !make_tmap(&m.d3O, own.dxs, s.H, s.T * s.kk, 32, 1, 4))
         return fail(MOK_ERR_INVALID, "tensor map (expert-parallel gate/up dgrad)");
     GemmArgs g3 = base;
@@ -1601,6 +1643,17 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
     g3.out_f32 = own.dxs;
     g3.push_dst = es.push_dx;
     g3.ldo = c.H;
+    if (mx) {
+        g3.num_kb = 2 * c.I / 128;
+        g3.b_rows_per_group = c.H;
+        g3.gather_src = nullptr;
+        g3.sfa_src = es.dgus;
+        g3.sf_ld = 2 * c.I / 32;
+        g3.sfb_src = p.st_gate_up;
+        g3.sfb_src_s = s.S ? p.sst_gate_up : p.st_gate_up;
+        g3.sfb_row_tiles = static_cast<int>(el * s.H / 128);
+        g3.sfb_row_tiles_s = static_cast<int>((s.S ? s.S : el) * s.H / 128);
+    }
 
     // gate/up wgrad: dW_gate_up[g] = sum_r dGU_r^T x[token r] (the pulled x rows)
     if (!make_tmap(&m.w4A, es.dgu, 2 * s.I, es.rows_cap, 64, 64, 2) ||
@@ -1622,17 +1675,33 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
     const int g4_grid = static_cast<int>(t4 < dev.sms ? t4 : dev.sms);
     const int g4_units = static_cast<int>(G * g4.n_tiles * ((g4.m_tiles + g4.m_per_unit - 1) / g4.m_per_unit));
 
-    if (t_schedule == MOK_SCHEDULE_PERSISTENT)
-        return n256 ? launch_ep_bwd_fused<true>(c, world, rank, dyr, tdx, tg, es, m, g1, g2, g3, g4, g2_units, g4_units,
-                                                dev, stream)
-                    : launch_ep_bwd_fused<false>(c, world, rank, dyr, tdx, tg, es, m, g1, g2, g3, g4, g2_units, g4_units,
-                                                 dev, stream);
+    EpMxPrep prep{};                         // MXFP8: quantise the pulled dy rows, decode the x codes
+    prep.dy = es.dy_recv;
+    prep.dyq = es.dyq_recv;
+    prep.dys = es.dys_recv;
+    prep.xq = es.xq_recv;
+    prep.xs = es.xs_recv;
+    prep.xdq = es.x_recv;
+    prep.n_recv = es.n_recv;
+    prep.T = c.T; prep.world = world; prep.H = c.H;
+    if (t_schedule == MOK_SCHEDULE_PERSISTENT) {
+        if (mx)
+            return launch_ep_bwd_fused<true, true>(c, world, rank, dyr, tdx, tg, es, m, g1, g2, g3, g4, g2_units,
+                                                   g4_units, prep, dev, stream);
+        return n256 ? launch_ep_bwd_fused<true, false>(c, world, rank, dyr, tdx, tg, es, m, g1, g2, g3, g4, g2_units,
+                                                       g4_units, prep, dev, stream)
+                    : launch_ep_bwd_fused<false, false>(c, world, rank, dyr, tdx, tg, es, m, g1, g2, g3, g4, g2_units,
+                                                        g4_units, prep, dev, stream);
+    }
     if (const cudaError_t e = cudaMemsetAsync(es.sched, 0, kSchedCounters * sizeof(int), stream); e != cudaSuccess)
         return fail(MOK_ERR_LAUNCH, "cudaMemsetAsync(tile counters)", e);
     MOK_TRY(launch_k(ep_table_kernel, dim3(1), dim3(32), 0, stream, "ep_table_kernel", tdx, es.push_dx, world));
     MOK_TRY(launch_k(ep_table_kernel, dim3(1), dim3(32), 0, stream, "ep_table_kernel", tg, es.push_g, world));
     MOK_TRY(launch_pull(dyr, world, rank, es.dy_recv, 2ll * c.H, es, c, dev, stream));
-    if (n256)
+    if (mx) {
+        MOK_TRY(launch_k(ep_mx_prepare_kernel, dim3(dev.sms * 8), dim3(256), 0, stream, "ep_mx_prepare_kernel", prep));
+        MOK_TRY(launch_gemm<DgradDownMX>(m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1, dev.sms, stream));
+    } else if (n256)
         MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradDown>(m.d1B, m.d1B, m.d1Bs, m.d1O, m.d1O, m.d1O, g1,
                                                                   dev.sms, stream));
     else
@@ -1650,8 +1719,11 @@ int ep_bwd_experts(const moe_cfg &c, int world, int rank, const void *const *dyr
         MOK_TRY(launch_gemm<typename FusedBwdCfg<false>::WgradDown>(m.w2B, m.w2B, m.w2B, m.w2O, m.w2O2, m.w2O, g2,
                                                                    g2_grid, stream));
     }
-    MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradGU>(m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O, g3, dev.sms,
-                                                            stream));
+    if (mx)
+        MOK_TRY(launch_gemm<DgradGUMX>(m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O, g3, dev.sms, stream));
+    else
+        MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::DgradGU>(m.d3A, m.d3B, m.d3Bs, m.d3O, m.d3O, m.d3O, g3,
+                                                                dev.sms, stream));
     MOK_TRY(launch_gemm<typename FusedBwdCfg<true>::WgradGU>(m.w4A, m.w4A, m.w4A, m.w4O, m.w4O2, m.w4O, g4, g4_grid,
                                                             stream));
     return launch_wgrad_resident<WgradResCfg<false>>(m.w4A, m.w4A, m.w4O, m.w4O2, g4,
@@ -2191,7 +2263,7 @@ int moe_ep_size(const moe_cfg *cfg, int32_t world, int32_t training, size_t *sta
                 size_t *bwd_bytes)
 {
     MOK_TRY(check_ep(cfg, world, 0));
-    if (training && cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
+    if (training && cfg->dtype == MOK_DTYPE_MXFP8 && cfg->I % 256) return MOK_ERR_UNSUPPORTED;
     if (state_bytes) *state_bytes = carve_state(*cfg, nullptr, false).bytes;
     if (scratch_bytes) *scratch_bytes = carve_ep(*cfg, world, training != 0, nullptr).bytes;
     if (bwd_bytes) *bwd_bytes = carve_ep_src_bwd(*cfg, nullptr).bytes;
@@ -2215,7 +2287,7 @@ int moe_ep_experts(const moe_cfg *cfg, int32_t world, int32_t rank, int32_t trai
                    void *stream)
 {
     MOK_TRY(check_ep(cfg, world, rank));
-    if (training && cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
+    if (training && cfg->dtype == MOK_DTYPE_MXFP8 && cfg->I % 256) return MOK_ERR_UNSUPPORTED;
     if (!params || !params->w_gate_up || !params->w_down || !x_ranks || !state_ranks) return MOK_ERR_INVALID;
     if (cfg->n_shared > 0 && (!params->ws_gate_up || !params->ws_down)) return MOK_ERR_INVALID;
     if (cfg->dtype == MOK_DTYPE_MXFP8 &&
@@ -2241,8 +2313,15 @@ int moe_ep_bwd_experts(const moe_cfg *cfg, int32_t world, int32_t rank, const vo
                        size_t scratch_bytes, void *stream)
 {
     MOK_TRY(check_ep(cfg, world, rank));
-    if (cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
+    if (cfg->dtype == MOK_DTYPE_MXFP8 && cfg->I % 256) return MOK_ERR_UNSUPPORTED;
     if (!params || !params->w_gate_up || !params->w_down || !dy_ranks || !bwd_ranks || !grads) return MOK_ERR_INVALID;
+    if (cfg->dtype == MOK_DTYPE_MXFP8) {
+        // the transposed weight copies of the data gradients (moe_quantize_mxfp8_weights_t of the rank's slice)
+        const moe_params &q = *params;
+        if (!q.wt_gate_up || !q.wt_down || !q.st_gate_up || !q.st_down ||
+            (cfg->n_shared > 0 && (!q.wst_gate_up || !q.wst_down || !q.sst_gate_up || !q.sst_down)))
+            return MOK_ERR_INVALID;
+    }
     if (cfg->n_shared > 0 && (!params->ws_gate_up || !params->ws_down || !grads->dws_gate_up || !grads->dws_down))
         return MOK_ERR_INVALID;
     const void *w[] = {params->w_gate_up, params->w_down, params->ws_gate_up, params->ws_down, grads->dw_gate_up,
@@ -2265,7 +2344,6 @@ int moe_ep_bwd_combine(const moe_cfg *cfg, int32_t world, int32_t rank, const vo
                        const void *state, void *bwd, size_t bwd_bytes, const moe_grads *grads, void *stream)
 {
     MOK_TRY(check_ep(cfg, world, rank));
-    if (cfg->dtype == MOK_DTYPE_MXFP8) return MOK_ERR_UNSUPPORTED;
     if (!params || !params->router_w || !aligned16(params->router_w) || !grads || !grads->dx || !grads->drouter_w)
         return MOK_ERR_INVALID;
     if (!aligned16(grads->dx) || !aligned16(grads->drouter_w)) return MOK_ERR_INVALID;

@@ -140,9 +140,11 @@ def test_expert_parallel_sizes_and_argument_checks():
     mxc = make_cfg(64, 256, 8, 128, 2, dtype=abi.MOK_DTYPE_MXFP8)
     mst, msc, _ = abi.moe_ep_size(mxc, 2)
     assert msc >= (64 + 2 * 64) * (256 + 8) + (2 * 64 * 2) * (128 + 4)
-    with pytest.raises(abi.MokError) as ei:
+    with pytest.raises(abi.MokError) as ei:      # MXFP8 training needs I % 256 == 0
         abi.moe_ep_size(mxc, 2, True)
     assert ei.value.code == abi.MOK_ERR_UNSUPPORTED
+    mxt = make_cfg(64, 256, 8, 256, 2, dtype=abi.MOK_DTYPE_MXFP8)
+    _, msct, mbb = abi.moe_ep_size(mxt, 2, True)
     pm = abi.moe_params(router_w=16, w_gate_up=16, w_down=16)      # MXFP8 without weight scales
     with pytest.raises(abi.MokError) as ei:
         abi.moe_ep_experts(mxc, 2, 0, 0, [16, 16], [16, 16], pm, 16, msc, None)
@@ -150,6 +152,11 @@ def test_expert_parallel_sizes_and_argument_checks():
     with pytest.raises(abi.MokError) as ei:
         abi.moe_ep_experts(mxc, 2, 0, 1, [16, 16], [16, 16], pm, 16, msc, None)
     assert ei.value.code == abi.MOK_ERR_UNSUPPORTED
+    pms = abi.moe_params(router_w=16, w_gate_up=16, w_down=16, s_gate_up=16, s_down=16)   # no transposed copies
+    with pytest.raises(abi.MokError) as ei:
+        abi.moe_ep_bwd_experts(mxt, 2, 0, [16, 16], [16, 16], pms, abi.moe_grads(dx=16, dw_gate_up=16, dw_down=16,
+                                                                                 drouter_w=16), 16, msct, None)
+    assert ei.value.code == abi.MOK_ERR_INVALID
     small = make_cfg(64, 256, 8, 128, 2)
     st, sc, bb = abi.moe_ep_size(small, 2)
     _, sct, _ = abi.moe_ep_size(small, 2, True)

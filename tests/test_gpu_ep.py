@@ -24,7 +24,7 @@ import torch
 
 import oracle
 from mixture_experts_layer_persistent_b200 import (EPWorld, MoELayer, abi, cfg_for, quantize_mxfp8_weights,
-                                                   split_params, synth)
+                                                   quantize_mxfp8_weights_t, split_params, synth)
 from tests._support import assert_close, bits_to_bf16, oracle_layer, to_np
 
 pytestmark = pytest.mark.gpu
@@ -298,19 +298,85 @@ def test_mxfp8_dsv3_expert_shape_over_eight_ranks():
         assert _same(ys[r], y_ref), f"rank {r}: y differs from the MXFP8 moe_fwd"
 
 
-@pytest.mark.parametrize("mx", [False, True], ids=["bf16_train", "mxfp8"])
-def test_persistent_and_split_experts_phase_agree(mx):
-    """The owner's experts phase as one persistent launch (the default) and as the
-    split launches: y (and, for BF16, every gradient of the backward that reads the
-    forward's saved rows) byte for byte, and one launch for the persistent phase."""
+def _mx_train_params(params, world, E):
+    """_mx_params plus the transposed copies the MXFP8 backward reads, for the whole
+    layer and for each rank's slice."""
+    full, ranks = _mx_params(params, world, E)
+    el = E // world
+    for name in ("w_gate_up", "w_down", "ws_gate_up", "ws_down"):
+        t = "wt" + name[1:] if name.startswith("w_") else "wst" + name[2:]
+        ts = "st" + name[1:] if name.startswith("w_") else "sst" + name[2:]
+        if params.get(name) is None:
+            continue
+        full[t], full[ts] = quantize_mxfp8_weights_t(params[name])
+        for r in range(world):
+            if name.startswith("ws"):
+                ranks[r][t], ranks[r][ts] = full[t], full[ts]
+            else:
+                ranks[r][t], ranks[r][ts] = quantize_mxfp8_weights_t(params[name][r * el:(r + 1) * el].contiguous())
+    return full, ranks
+
+
+def test_mxfp8_training_matches_the_one_gpu_layer():
+    """The MXFP8 training step over 4 ranks: every rank's y, dx, router and
+    shared-expert gradients byte-equal to the one-GPU MXFP8 layer's (forward with saved
+    state + MXFP8 backward) on its tokens; every owner's expert weight gradients
+    byte-equal to the one-GPU layer's on the concatenated batch (same router K split,
+    so the same routing, checked)."""
+    dev = torch.device("cuda")
+    world = 4
+    wl = synth.Workload("ep_mx_train", T=300, H=512, E=16, k=4, I=256, S=1, Is=256, score_fn=1, n_group=4,
+                        topk_group=2, mxfp8=True, seed=67)
+    el = wl.E // world
+    params = synth.draw_params(wl, dev)
+    xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(world)]
+    dys = _rank_dys(wl, world, dev)
+    full, ranks = _mx_train_params(params, world, wl.E)
+    cfg = cfg_for(wl)
+    ep = EPWorld(cfg, world, ranks, training=True)
+    ys = ep.forward(xs)
+    grads = ep.backward(dys)
+    torch.cuda.synchronize()
+    assert abi.moe_status(torch.cuda.current_stream().cuda_stream) == 0
+    layer = MoELayer(cfg, full, training=True)
+    for r in range(world):
+        y_ref = layer.forward(xs[r]).clone()
+        g_ref = layer.backward(xs[r], dys[r])
+        torch.cuda.synchronize()
+        assert _same(ys[r], y_ref), f"rank {r}: y"
+        for n in ("dx", "drouter_w", "dws_gate_up", "dws_down"):
+            assert _same(grads[r][n], g_ref[n]), f"rank {r}: {n}"
+    big = MoELayer(cfg_for(synth.scaled(wl, T=wl.T * world)), full, training=True)
+    routing = big.new_routing()
+    big.forward(torch.cat(xs), routing=routing)
+    g_all = big.backward(torch.cat(xs), torch.cat(dys))
+    torch.cuda.synchronize()
+    assert big.status() == 0
+    for r in range(world):
+        rr = layer.new_routing()
+        layer.forward(xs[r], routing=rr)
+        sl = slice(r * wl.T, (r + 1) * wl.T)
+        assert _same(rr["topk_idx"], routing["topk_idx"][sl]) and _same(rr["topk_w"], routing["topk_w"][sl])
+    for r in range(world):
+        for n in ("dw_gate_up", "dw_down"):
+            assert _same(grads[r][n], g_all[n][r * el:(r + 1) * el]), f"owner {r}: {n}"
+
+
+@pytest.mark.parametrize("mx,train", [(False, True), (True, False), (True, True)],
+                         ids=["bf16_train", "mxfp8", "mxfp8_train"])
+def test_persistent_and_split_experts_phase_agree(mx, train):
+    """The owner's experts phases as one persistent launch each (the default) and as
+    the split launches: y and, when training, every gradient of the backward that
+    reads the forward's saved rows, byte for byte; one launch for the persistent
+    forward experts phase."""
     dev = torch.device("cuda")
     world = 4
     wl = synth.Workload("ep_sched", T=300, H=512, E=16, k=4, I=256, S=1, Is=256, score_fn=1, n_group=4,
-                        topk_group=2, mxfp8=mx, backward=not mx, seed=65)
+                        topk_group=2, mxfp8=mx, backward=train, seed=65)
     params = synth.draw_params(wl, dev)
     xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(world)]
     if mx:
-        _, rank_params = _mx_params(params, world, wl.E)
+        _, rank_params = (_mx_train_params if train else _mx_params)(params, world, wl.E)
     else:
         rank_params = [split_params(params, world, r, wl.E) for r in range(world)]
     dys = _rank_dys(wl, world, dev)
@@ -318,16 +384,16 @@ def test_persistent_and_split_experts_phase_agree(mx):
     for sched in (abi.MOK_SCHEDULE_PERSISTENT, abi.MOK_SCHEDULE_SPLIT):
         abi.moe_set_schedule(sched)
         try:
-            ep = EPWorld(cfg_for(wl), world, rank_params, training=not mx)
+            ep = EPWorld(cfg_for(wl), world, rank_params, training=train)
             ys = ep.forward(xs)
             n = None
             if sched == abi.MOK_SCHEDULE_PERSISTENT:
-                abi.moe_ep_experts(cfg_for(wl), world, world - 1, not mx, [x.data_ptr() for x in xs],
+                abi.moe_ep_experts(cfg_for(wl), world, world - 1, train, [x.data_ptr() for x in xs],
                                    [s.data_ptr() for s in ep.states], ep.cparams[world - 1],
                                    ep.scratch[world - 1].data_ptr(), ep.scratch_bytes,
                                    torch.cuda.current_stream().cuda_stream)
                 n = abi.moe_launch_count()
-            grads = None if mx else ep.backward(dys)
+            grads = ep.backward(dys) if train else None
             torch.cuda.synchronize()
         finally:
             abi.moe_set_schedule(abi.MOK_SCHEDULE_PERSISTENT)
@@ -337,7 +403,7 @@ def test_persistent_and_split_experts_phase_agree(mx):
     assert n == 1, "the persistent experts phase is one launch"
     for r in range(world):
         assert _same(yp[r], ys_[r]), f"rank {r}: y"
-        if not mx:
+        if train:
             for k in gp[r]:
                 if gp[r][k] is not None:
                     assert _same(gp[r][k], gs[r][k]), f"rank {r}: {k}"
