@@ -427,6 +427,11 @@ def main():
         W = max(1, args.ep_world)
         ep = ep_emulated_run(synth.scaled(wl, name=wl.name + "_ep", T=wl.T // W, seed=wl.seed + 7), W, dev,
                              args.steps, args.warmup)
+        if args.mx_workload and args.mx_workload != "none":
+            torch.cuda.empty_cache()
+            mwl = synth.WORKLOADS[args.mx_workload]
+            ep["mxfp8"] = ep_emulated_mx_run(synth.scaled(mwl, name=mwl.name + "_ep", T=mwl.T // W,
+                                                          seed=mwl.seed + 7), W, dev, args.steps, args.warmup)
         if rank == 0:
             print(json.dumps({"ep_emulated": ep}))
         if world > 1:
@@ -588,7 +593,7 @@ def main():
         torch.cuda.empty_cache()
         if args.mx_workload and args.mx_workload != "none":
             mwl = synth.WORKLOADS[args.mx_workload]
-            ep["mxfp8_forward"] = ep_emulated_mx_run(
+            ep["mxfp8"] = ep_emulated_mx_run(
                 synth.scaled(mwl, name=mwl.name + "_ep", T=mwl.T // args.ep_world, seed=mwl.seed + 1000 * rank + 7),
                 args.ep_world, dev, K, args.warmup)
             torch.cuda.empty_cache()
@@ -772,51 +777,79 @@ def ep_emulated_run(wl, W, dev, K, warmup):
 
 
 def ep_emulated_mx_run(wl, W, dev, K, warmup):
-    """The MXFP8 expert-parallel forward (inference) with its W ranks (wl.T tokens each)
-    on this GPU in stream order, against the one-GPU MXFP8 forward of the same tokens.
-    Each rank quantises its own experts' weights and its own x; owners pull e4m3 rows
-    and scales.  No link is crossed: the data path, not a multi-GPU measurement."""
+    """The MXFP8 expert-parallel layer with its W ranks (wl.T tokens each) on this GPU in
+    stream order, against the one-GPU MXFP8 layer on the same tokens: the forward
+    (inference), and the training step (forward with saved state + MXFP8 backward).
+    Each rank quantises its own experts' weights (both copies) and its own x; owners
+    pull e4m3 rows and scales of x and the bf16 dy rows.  No link is crossed: the data
+    path, not a multi-GPU measurement."""
     import torch
-    from mixture_experts_layer_persistent_b200 import EPWorld, MoELayer, cfg_for, quantize_mxfp8_weights, synth
+    from mixture_experts_layer_persistent_b200 import (EPWorld, MoELayer, cfg_for, new_rank_grads,
+                                                       quantize_mxfp8_weights, quantize_mxfp8_weights_t, synth)
     params = synth.draw_params(wl, dev)
     full = {k: params[k] for k in ("router_w", "e_bias", "logit_bias")}
     for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down"), ("ws_gate_up", "ss_gate_up"),
                         ("ws_down", "ss_down")):
         full[name], full[sname] = quantize_mxfp8_weights(params[name]) if params.get(name) is not None else (None, None)
+    for name in ("w_gate_up", "w_down", "ws_gate_up", "ws_down"):
+        t = "wt" + name[1:] if name.startswith("w_") else "wst" + name[2:]
+        ts = "st" + name[1:] if name.startswith("w_") else "sst" + name[2:]
+        if params.get(name) is not None:
+            full[t], full[ts] = quantize_mxfp8_weights_t(params[name])
     el = wl.E // W
     ranks = []
     for r in range(W):
         p = dict(full)
-        for name, sname in (("w_gate_up", "s_gate_up"), ("w_down", "s_down")):
-            p[name], p[sname] = quantize_mxfp8_weights(params[name][r * el:(r + 1) * el].contiguous())
+        for name, sname, t, ts in (("w_gate_up", "s_gate_up", "wt_gate_up", "st_gate_up"),
+                                   ("w_down", "s_down", "wt_down", "st_down")):
+            sl = params[name][r * el:(r + 1) * el].contiguous()
+            p[name], p[sname] = quantize_mxfp8_weights(sl)
+            p[t], p[ts] = quantize_mxfp8_weights_t(sl)
         ranks.append(p)
     del params
     xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(W)]
-    ep = EPWorld(cfg_for(wl), W, ranks, device=dev)
+    dys = [synth.draw_dy(synth.scaled(wl, seed=wl.seed * 100 + 50 + r), dev) for r in range(W)]
+    cfg = cfg_for(wl)
+    ep = EPWorld(cfg, W, ranks, device=dev)
+    ept = EPWorld(cfg, W, ranks, training=True, device=dev)
     ys = [torch.empty_like(x) for x in xs]
-    one = MoELayer(cfg_for(synth.scaled(wl, T=wl.T * W)), full, training=False, device=dev)
-    xw = torch.cat(xs)
+    eg = [new_rank_grads(cfg, W, dev) for _ in range(W)]
+    whole = synth.scaled(wl, T=wl.T * W)
+    one = MoELayer(cfg_for(whole), full, training=False, device=dev)
+    onet = MoELayer(cfg_for(whole), full, training=True, device=dev)
+    og = onet.new_grads()
+    xw, dyw = torch.cat(xs), torch.cat(dys)
     yw = torch.empty_like(xw)
     for _ in range(warmup):
         ep.forward(xs, ys)
         one.forward(xw, yw)
+        ept.forward(xs, ys)
+        ept.backward(dys, eg)
+        onet.forward(xw, yw)
+        onet.backward(xw, dyw, og)
     torch.cuda.synchronize()
     mk = lambda: torch.cuda.Event(enable_timing=True)
-    t_ep, t_one = [], []
+    legs = {"ep": [], "one": [], "ep_train": [], "one_train": []}
     for _ in range(K):
-        a, b, c, d = mk(), mk(), mk(), mk()
-        a.record(); ep.forward(xs, ys); b.record()
-        c.record(); one.forward(xw, yw); d.record()
-        t_ep.append((a, b)); t_one.append((c, d))
+        for key, run in (("ep", lambda: ep.forward(xs, ys)), ("one", lambda: one.forward(xw, yw)),
+                         ("ep_train", lambda: (ept.forward(xs, ys), ept.backward(dys, eg))),
+                         ("one_train", lambda: (onet.forward(xw, yw), onet.backward(xw, dyw, og)))):
+            a, b = mk(), mk()
+            a.record(); run(); b.record()
+            legs[key].append((a, b))
     torch.cuda.synchronize()
-    ms_ep = statistics.mean(a.elapsed_time(b) for a, b in t_ep)
-    ms_one = statistics.mean(c.elapsed_time(d) for c, d in t_one)
-    out = {"workload": f"{wl.name}: MXFP8 forward of {W} ranks x {wl.T} tokens, E={wl.E} experts "
+    ms = {k: statistics.mean(a.elapsed_time(b) for a, b in v) for k, v in legs.items()}
+    n = W * wl.T
+    out = {"workload": f"{wl.name}: MXFP8 layer of {W} ranks x {wl.T} tokens, E={wl.E} experts "
                        f"({el} per rank), top-{wl.k}, H={wl.H}, I={wl.I}, {wl.S} shared, all ranks on one GPU",
-           "world": W, "tokens_per_rank": wl.T, "fwd_ms": ms_ep, "fwd_tokens_per_s": W * wl.T / (ms_ep / 1e3),
-           "one_gpu_fwd_ms": ms_one, "ep_over_one_gpu_fwd_time": ms_ep / ms_one, "device_status": one.status(),
+           "world": W, "tokens_per_rank": wl.T, "fwd_ms": ms["ep"], "fwd_tokens_per_s": n / (ms["ep"] / 1e3),
+           "one_gpu_fwd_ms": ms["one"], "ep_over_one_gpu_fwd_time": ms["ep"] / ms["one"],
+           "training_step_ms": ms["ep_train"], "training_step_tokens_per_s": n / (ms["ep_train"] / 1e3),
+           "one_gpu_training_step_ms": ms["one_train"],
+           "ep_over_one_gpu_training_step_time": ms["ep_train"] / ms["one_train"],
+           "device_status": onet.status(),
            "note": "ranks emulated in stream order on one device; no link crossed"}
-    del ep, one, full, ranks, xs, ys, xw, yw
+    del ep, ept, one, onet, full, ranks, xs, ys, xw, yw, dys, dyw, eg, og
     return out
 
 
