@@ -437,3 +437,35 @@ def test_experts_phase_on_buffers_of_ones():
         for k in res[0][1][r]:
             if res[0][1][r][k] is not None:
                 assert _same(res[0][1][r][k], res[1][1][r][k]), f"rank {r}: {k}"
+
+
+def test_owner_with_no_routed_rows():
+    """A logit term that rules out the experts of rank 1 (4..7): rank 1 receives no
+    routed row, its experts phase runs only its shared expert on its own 77 tokens
+    (a ragged count), and its experts' weight gradients are zero.  Every rank's y, dx,
+    router and shared-expert gradients equal the one-GPU layer's byte for byte, in
+    BF16 training."""
+    dev = torch.device("cuda")
+    world = 2
+    wl = synth.Workload("ep_empty_owner", T=77, H=256, E=8, k=2, I=128, S=1, Is=128, seed=68)
+    params = synth.draw_params(wl, dev)
+    params["logit_bias"] = torch.tensor([0.0] * 4 + [-100.0] * 4, device=dev)
+    xs = [synth.draw_x(synth.scaled(wl, seed=wl.seed * 100 + r), dev) for r in range(world)]
+    dys = _rank_dys(wl, world, dev)
+    cfg = cfg_for(wl)
+    ep = EPWorld(cfg, world, [split_params(params, world, r, wl.E) for r in range(world)], training=True)
+    ys = ep.forward(xs)
+    grads = ep.backward(dys)
+    torch.cuda.synchronize()
+    assert abi.moe_status(torch.cuda.current_stream().cuda_stream) == 0
+    layer = MoELayer(cfg, params, training=True)
+    for r in range(world):
+        routing = layer.new_routing()
+        y_ref = layer.forward(xs[r], routing=routing).clone()
+        g_ref = layer.backward(xs[r], dys[r])
+        torch.cuda.synchronize()
+        assert int(routing["counts"][4:].sum()) == 0, "the logit term keeps experts 4..7 empty"
+        assert _same(ys[r], y_ref), f"rank {r}: y"
+        for n in ("dx", "drouter_w", "dws_gate_up", "dws_down"):
+            assert _same(grads[r][n], g_ref[n]), f"rank {r}: {n}"
+    assert not grads[1]["dw_gate_up"].any() and not grads[1]["dw_down"].any(), "empty experts: zero weight gradients"
