@@ -28,7 +28,7 @@ CASES = [
     synth.Workload("sched_softmax_i384", T=333, H=768, E=12, k=3, I=384, S=2, Is=384, seed=42),
     synth.Workload("sched_zipf", T=900, H=512, E=16, k=4, I=256, S=1, Is=256, score_fn=1, n_group=4, topk_group=2,
                    zipf=3.5, seed=43),
-    # more than one dispatch chunk of 1024 tokens, one token per expert or none
+    # ten dispatch chunks of 256 tokens (the last one ragged), one token per expert or none
     synth.Workload("sched_chunks", T=2500, H=256, E=64, k=2, I=128, score_fn=0, seed=44),
 ]
 MX_CASES = [
